@@ -1,0 +1,512 @@
+"""Benchmark of the fused all-reduce + residual-add + RMSNorm (+FP8) epilogue.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl far|reference]
+
+One step = one call of the whole epilogue (W-partial reduce, residual add and
+new-residual write, mean square, normalise with gamma, FP8 quantisation) over
+one batch of synthetic rows.  The headline workload is the prefill one: W=4
+partials of 8192 x 8192 bf16 (1% outlier rows x50), residual N(0,2),
+eps=1e-5, static per-tensor FP8 with scale 0.05, the new residual and the FP8
+codes written (norm_out not requested).
+
+The metric is achieved HBM GB/s of algorithmic bytes (W*T*H*2 partials +
+T*H*2 residual in + H*2 gamma + T*H*2 residual out + T*H FP8 codes [+ 4T
+scales] [+ T*H*2 norm_out]) and its fraction of the measured HBM peak;
+tokens/s is reported beside it.  Inputs (640 MiB read per step) are larger
+than the 126 MB L2, so nothing stays cached between steps.
+
+Under torchrun (N > 1) every rank runs its own batch of rows (the rows are
+independent: weak scaling, no collective on the data path); the time is the
+max over ranks and `value` counts every rank's bytes.  `--impl reference`
+times the CPU fp64 oracle on a bounded sample of the same workload (rank 0).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+from reduce_residual_add_b200.inputs import WORKLOADS, Workload, as_u16, make_inputs  # noqa: E402
+
+HEADLINE = "c4_prefill_fp8_static"
+METRIC = "achieved HBM GB/s (% of B200 peak) and tokens/s of fused reduce+add+RMSNorm(+FP8)"
+FALLBACK_HBM_GBS = 6650.0
+
+
+def algorithmic_bytes(wl: Workload, rows: int, with_norm: bool) -> int:
+    T, H, W = rows, wl.H, wl.W
+    b = W * T * H * 2 + H * 2
+    if wl.has_residual:
+        b += T * H * 2          # residual in
+    b += T * H * 2              # new residual out
+    if with_norm:
+        b += T * H * 2
+    if wl.pattern in (1, 2):
+        b += T * H             # e4m3 codes
+    if wl.pattern == 2:
+        b += 4 * T             # per-token scales
+    return b
+
+
+def hbm_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region (NVML: read-only queries)
+# ---------------------------------------------------------------------------
+
+REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+           0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+           0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+           0x100: "display_clock_setting"}
+
+
+class ClockSampler(threading.Thread):
+    def __init__(self, device: int, period_s: float = 0.01):
+        super().__init__(daemon=True)
+        self.period = period_s
+        self.samples = []
+        self.reasons = 0
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self.ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            idx = device
+            try:
+                idx = torch.cuda._get_nvml_device_index(device)
+            except Exception:
+                vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+                if vis:
+                    idx = int(vis.split(",")[device])
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(idx)
+            self.nv = pynvml
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.ok = False
+
+    def run(self):
+        if not self.ok:
+            return
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                try:
+                    r = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                except AttributeError:
+                    r = nv.nvmlDeviceGetCurrentClocksThrottleReasons(self.h)
+                self.reasons |= int(r) & ~0x1
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def stop(self) -> dict:
+        self._stop.set()
+        if self.is_alive():
+            self.join(timeout=2)
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": [n for b, n in REASONS.items() if self.reasons & b],
+                "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------------------
+# distributed plumbing
+# ---------------------------------------------------------------------------
+
+def dist_setup(n_gpus: int):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------------------
+# the oracle on host cores (CPU baseline and reference arm)
+# ---------------------------------------------------------------------------
+
+def oracle_rate(wl: Workload, inp: dict, rows: int, with_norm: bool):
+    """Run the fp64 oracle on the first `rows` rows; return (seconds, bytes)."""
+    import oracle
+    ps = [as_u16(p[:rows]) for p in inp["partials"]]
+    res = None if inp["residual"] is None else as_u16(inp["residual"][:rows])
+    gam = as_u16(inp["gamma"])
+    t0 = time.perf_counter()
+    oracle.fused(ps, res, gam, wl.dtype, wl.eps, wl.weight_bias, wl.pattern,
+                 scale_in=wl.static_scale, want_norm=with_norm)
+    dt = time.perf_counter() - t0
+    return dt, algorithmic_bytes(wl, rows, with_norm)
+
+
+def cpu_baseline(wl: Workload, inp: dict, with_norm: bool, budget_s: float = 15.0) -> dict:
+    t1, _ = oracle_rate(wl, inp, 64, with_norm)
+    rows = int(min(wl.T, max(64, budget_s / max(t1 / 64, 1e-9))))
+    dt, b = oracle_rate(wl, inp, rows, with_norm)
+    return {"value": round(b / dt / 1e9, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "sample": "first %d of %d rows of %s, single-threaded C fp64 oracle, %.1f s"
+                      % (rows, wl.T, wl.name, dt),
+            "tokens_per_s": round(rows / dt, 2)}
+
+
+# ---------------------------------------------------------------------------
+# the CUDA path
+# ---------------------------------------------------------------------------
+
+class Case:
+    """Device buffers of one workload and a closure that launches one step."""
+
+    def __init__(self, ctx, wl: Workload, inp: dict, device, with_norm: bool, stream):
+        from reduce_residual_add_b200 import far
+        self.far = far
+        self.ctx, self.wl, self.with_norm, self.stream = ctx, wl, with_norm, stream
+        T, H = wl.T, wl.H
+        self.ps = [p.to(device) for p in inp["partials"]]
+        self.res = None if inp["residual"] is None else inp["residual"].to(device)
+        self.gam = inp["gamma"].to(device)
+        dt = wl.torch_dtype
+        self.rout = torch.empty(T, H, dtype=dt, device=device)
+        self.nout = torch.empty(T, H, dtype=dt, device=device) if (with_norm or wl.pattern == 0) else None
+        self.qout = torch.empty(T, H, dtype=torch.uint8, device=device) if wl.pattern else None
+        self.sout = torch.empty(T, dtype=torch.float32, device=device) if wl.pattern == 2 else None
+        self.sin = (torch.tensor([wl.static_scale], dtype=torch.float32, device=device)
+                    if wl.pattern == 1 else None)
+        self.bytes = algorithmic_bytes(wl, T, self.nout is not None)
+
+    def step(self):
+        self.far.far_fused(self.ctx, self.ps, self.res, self.gam, self.wl.eps,
+                           self.wl.weight_bias, self.wl.pattern, residual_out=self.rout,
+                           norm_out=self.nout, quant_out=self.qout, scale_in=self.sin,
+                           scale_out=self.sout, stream=self.stream)
+
+    def time_steps(self, k: int, warmup: int, per_launch: bool = True):
+        """(total seconds for k back-to-back steps, mean per-launch seconds)."""
+        s = self.stream
+        for _ in range(warmup):
+            self.step()
+        torch.cuda.synchronize()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(k)] if per_launch else None
+        first, last = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        first.record(s)
+        for i in range(k):
+            if per_launch:
+                ev[i][0].record(s)
+            self.step()
+            if per_launch:
+                ev[i][1].record(s)
+        last.record(s)
+        torch.cuda.synchronize()
+        total = first.elapsed_time(last) / 1e3
+        mean = (sum(a.elapsed_time(b) for a, b in ev) / k / 1e3) if per_launch else total / k
+        return total, mean
+
+
+def graph_time(case: Case, launches: int, reps: int = 5) -> float:
+    """Mean seconds per launch inside a CUDA graph of `launches` calls."""
+    s = case.stream
+    g = torch.cuda.CUDAGraph()
+    case.step()
+    torch.cuda.synchronize()
+    with torch.cuda.graph(g, stream=s):
+        for _ in range(launches):
+            case.step()
+    g.replay()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(s)
+    for _ in range(reps):
+        g.replay()
+    b.record(s)
+    torch.cuda.synchronize()
+    t = a.elapsed_time(b) / 1e3 / (reps * launches)
+    del g
+    return t
+
+
+def e2e_time(case: Case, inp: dict, steps: int):
+    """Through the public API from pinned host memory: every step copies the
+    inputs host->device, runs the call, and copies the outputs back."""
+    s = case.stream
+    h_ps = [p.pin_memory() for p in inp["partials"]]
+    h_res = None if inp["residual"] is None else inp["residual"].pin_memory()
+    h_gam = inp["gamma"].pin_memory()
+    h_rout = torch.empty(case.rout.shape, dtype=case.rout.dtype).pin_memory()
+    h_q = torch.empty(case.qout.shape, dtype=torch.uint8).pin_memory() if case.qout is not None else None
+    h_s = torch.empty(case.sout.shape, dtype=torch.float32).pin_memory() if case.sout is not None else None
+    h_n = torch.empty(case.nout.shape, dtype=case.nout.dtype).pin_memory() if case.nout is not None else None
+    h2d = sum(p.numel() * 2 for p in h_ps) + (h_res.numel() * 2 if h_res is not None else 0) + h_gam.numel() * 2
+    d2h = h_rout.numel() * 2 + (h_q.numel() if h_q is not None else 0) + \
+        (h_s.numel() * 4 if h_s is not None else 0) + (h_n.numel() * 2 if h_n is not None else 0)
+
+    def one():
+        with torch.cuda.stream(s):
+            for d, h in zip(case.ps, h_ps):
+                d.copy_(h, non_blocking=True)
+            if h_res is not None:
+                case.res.copy_(h_res, non_blocking=True)
+            case.gam.copy_(h_gam, non_blocking=True)
+            case.step()
+            h_rout.copy_(case.rout, non_blocking=True)
+            if h_q is not None:
+                h_q.copy_(case.qout, non_blocking=True)
+            if h_s is not None:
+                h_s.copy_(case.sout, non_blocking=True)
+            if h_n is not None:
+                h_n.copy_(case.nout, non_blocking=True)
+
+    one()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(s)
+    for _ in range(steps):
+        one()
+    b.record(s)
+    torch.cuda.synchronize()
+    return a.elapsed_time(b) / 1e3 / steps, h2d, d2h
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for f in ("far_kernels.cu", "far_internal.h"):
+        with open(os.path.join(ROOT, "reduce_residual_add_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+def profiled_traffic(workload: str):
+    """Per-launch DRAM bytes of the kernel from the committed ncu summary,
+    or None when the kernel source changed since it was captured."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        e = d[workload]
+        if e.get("source_sha256") != kernel_source_hash():
+            return None
+        return int(e["traffic_bytes_per_launch"])
+    except Exception:
+        return None
+
+
+def run_far(args, world, rank, local):
+    from reduce_residual_add_b200 import build as fbuild
+    from reduce_residual_add_b200 import far
+    fbuild.build()
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    wl = WORKLOADS[args.workload]
+    # each rank owns an independent batch of rows (seed offset by rank)
+    inp = make_inputs(wl.with_(seed=wl.seed + 1000 * rank))
+    stream = torch.cuda.Stream(device=device)
+    ctx = far.FarContext(local)
+    case = Case(ctx, wl, inp, device, args.with_norm, stream)
+    launch = far.far_describe_launch(ctx, wl.T, wl.H, wl.torch_dtype)
+
+    case.time_steps(0, args.warmup, per_launch=False)
+    barrier(world)
+    torch.cuda.synchronize()
+    sampler = ClockSampler(local)
+    sampler.start()
+    total, mean_launch = case.time_steps(args.steps, 0, per_launch=True)
+    clocks = sampler.stop()
+    barrier(world)
+    total_max = max_over_ranks(total, world)
+    bytes_all = sum_over_ranks(float(case.bytes) * args.steps, world)
+    rows_all = sum_over_ranks(float(wl.T) * args.steps, world)
+
+    value = bytes_all / total_max / 1e9
+    peak, peak_kind = hbm_peak()
+    achieved = case.bytes / mean_launch / 1e9
+    e2e_s, h2d, d2h = e2e_time(case, inp, args.e2e_steps)
+    e2e_s = max_over_ranks(e2e_s, world)
+
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(total_max / args.steps * 1e3, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": wl.dtype,
+        "data": "synthetic",
+        "config": {"workload": wl.name, "W": wl.W, "T": wl.T, "H": wl.H, "dtype": wl.dtype,
+                   "pattern": ["ar_residual_rmsnorm", "fp8_static", "fp8_per_token"][wl.pattern],
+                   "norm_out": case.nout is not None, "eps": wl.eps,
+                   "weight_bias": wl.weight_bias, "static_scale": wl.static_scale,
+                   "bytes_per_step": case.bytes, "rows_per_rank": wl.T,
+                   "l2": "inputs larger than L2 (%d MiB read per step vs 126 MB L2); no flush"
+                         % ((wl.W + 1) * wl.T * wl.H * 2 // 2 ** 20),
+                   "launch": launch, "parallelism": "rows sharded across %d rank(s), no collective" % world},
+        "tokens_per_s": round(rows_all / total_max, 1),
+        "pct_of_peak": round(100 * value / world / peak, 2),
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak,
+                     "unit": "GB/s", "frac": round(achieved / peak, 4),
+                     "peak_source": "%s (MEASURED_PEAKS.json hbm_gbs)" % peak_kind
+                                    if peak_kind == "measured" else "fallback 6.65 TB/s",
+                     "traffic": profiled_traffic(wl.name),
+                     "kernel": "far_prefill_kernel" if launch["regime"] == 2 else "far_decode_kernel",
+                     "mean_launch_us": round(mean_launch * 1e6, 3)},
+        "e2e": {"value": round(case.bytes / e2e_s / 1e9, 3), "unit": "GB/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "steps": args.e2e_steps, "ms_per_step": round(e2e_s * 1e3, 3)},
+        "gpu_launches": args.steps,
+        "clocks": clocks,
+    }
+
+    if world == 1 and not args.no_extras:
+        line["other_workloads"] = extras(ctx, device, stream)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(wl, inp, case.nout is not None)
+    ctx.close()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def extras(ctx, device, stream) -> dict:
+    """The other synthetic workloads, one short measurement each."""
+    from reduce_residual_add_b200 import far
+    out = {}
+    peak, _ = hbm_peak()
+    for name in ("c5_gemma_fp8_token_bf16", "c5_gemma_fp8_token_fp16", "c3_3d"):
+        wl = WORKLOADS[name]
+        inp = make_inputs(wl)
+        case = Case(ctx, wl, inp, device, False, stream)
+        total, mean = case.time_steps(200, 20, per_launch=True)
+        out[name] = {"GB/s": round(case.bytes / mean / 1e9, 1),
+                     "frac": round(case.bytes / mean / 1e9 / peak, 4),
+                     "us_per_call": round(mean * 1e6, 2), "tokens_per_s": round(wl.T / mean, 1),
+                     "bytes": case.bytes}
+        if name == "c3_3d":
+            out[name]["graph_us_per_call"] = round(graph_time(case, 50) * 1e6, 3)
+        del case
+    for T in (1, 8, 32, 80):
+        wl = WORKLOADS["c2_decode_T%d" % T]
+        inp = make_inputs(wl)
+        case = Case(ctx, wl, inp, device, False, stream)
+        row = {}
+        for reg, nm in ((far.FAR_REGIME_AUTO, "auto"), (far.FAR_REGIME_PREFILL, "prefill_kernel")):
+            far.far_set_regime(ctx, reg)
+            total, mean = case.time_steps(500, 50, per_launch=False)
+            row[nm] = {"stream_us_per_call": round(mean * 1e6, 3),
+                       "graph_us_per_call": round(graph_time(case, 100) * 1e6, 3)}
+        far.far_set_regime(ctx, far.FAR_REGIME_AUTO)
+        row["tokens_per_s_graph"] = round(T / (row["auto"]["graph_us_per_call"] * 1e-6), 1)
+        row["bytes"] = case.bytes
+        out[wl.name] = row
+        del case
+    return out
+
+
+def run_reference(args, world, rank):
+    """The CPU oracle, timed on this host's cores, on the same workload."""
+    if rank != 0:
+        return
+    wl = WORKLOADS[args.workload]
+    inp = make_inputs(wl)
+    with_norm = args.with_norm
+    t1, _ = oracle_rate(wl, inp, 16, with_norm)
+    per_row = t1 / 16
+    budget = 90.0
+    rows = max(1, min(wl.T, int(budget / (args.steps + args.warmup) / per_row)))
+    for _ in range(args.warmup):
+        oracle_rate(wl, inp, rows, with_norm)
+    tot_t, tot_b = 0.0, 0
+    for _ in range(args.steps):
+        dt, b = oracle_rate(wl, inp, rows, with_norm)
+        tot_t += dt
+        tot_b += b
+    value = tot_b / tot_t / 1e9
+    sample = "first %d of %d rows of %s per step, single-threaded C fp64 oracle" % (rows, wl.T, wl.name)
+    line = {"impl": "reference", "metric": METRIC, "value": round(value, 5), "unit": "GB/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(tot_t / args.steps * 1e3, 4), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": wl.name, "W": wl.W, "T": wl.T, "H": wl.H, "dtype": wl.dtype},
+            "tokens_per_s": round(rows * args.steps / tot_t, 3),
+            "cpu_baseline": {"value": round(value, 5), "unit": "GB/s", "cores": 1,
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": round(value, 5), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0},
+            "gpu_launches": 0}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["far", "reference"], default="far")
+    ap.add_argument("--workload", default=HEADLINE, choices=sorted(WORKLOADS))
+    ap.add_argument("--with-norm", action="store_true", help="also write norm_out")
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--no-extras", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    if args.impl == "reference":
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        rank = int(os.environ.get("RANK", "0"))
+        run_reference(args, world, rank)
+        return
+    world, rank, local = dist_setup(args.gpus)
+    try:
+        run_far(args, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

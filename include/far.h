@@ -1,0 +1,203 @@
+/*
+ * far.h -- C ABI of libfar.so: the fused "all-reduce + residual-add +
+ * RMSNorm (+FP8-e4m3)" epilogue of a row-parallel linear layer, on one
+ * B200 (sm_100a).
+ *
+ * What one call computes, for every row t of a (T, H) problem (row-major,
+ * contiguous, row stride H):
+ *
+ *   y[t,h]  = sum_{r<W} partials[r][t,h] + residual[t,h]          (fp32)
+ *   rinv[t] = 1 / sqrt( (1/H) sum_h y[t,h]^2 + eps )
+ *   o[t,h]  = y[t,h] * rinv[t] * (gamma[h] + weight_bias)
+ *
+ *   residual_out[t,h] = round_to_dtype(y[t,h])
+ *   norm_out[t,h]     = round_to_dtype(o[t,h])
+ *   static FP8:    quant_out[t,h] = e4m3_satfinite(o[t,h] / scale_in[0])
+ *   per-token FP8: scale_out[t] = max_h |o[t,h]| / 448,
+ *                  quant_out[t,h] = e4m3_satfinite(o[t,h] / scale_out[t])
+ *
+ * Sources (web pages, by title and section):
+ *  - vllm.models.common.ops.fused_allreduce_rms_norm, docstring of
+ *    fused_allreduce_rms_norm: the partials are the ranks' outputs of a
+ *    row-parallel linear run without its reduction; the result is
+ *    (normed_output, new_residual) = norm(all_reduce(hidden_states), residual);
+ *    the fused call passes fp32_acc=True, weight_bias=0.0 for standard
+ *    RMSNorm (1.0 for Gemma), and with one rank the op is the plain
+ *    norm(hidden_states, residual).
+ *  - PR #45307 report, call_trtllm_fused_allreduce_norm: norm_out,
+ *    quant_out, scale_out and scale_factor (here scale_in) are optional
+ *    outputs/inputs of one call; 3-D [batch, tokens, hidden] inputs are
+ *    flattened to (tokens, hidden) before the call.
+ *  - vllm.compilation.fusion, FusedAddRMSNormStaticQuantPattern and
+ *    FusedAddRMSNormDynamicQuantPattern: static per-tensor and dynamic
+ *    per-token symmetric FP8 after the fused add + RMSNorm; the dynamic one
+ *    returns one fp32 scale per token.
+ *  - vllm.compilation.sequence_parallelism, SequenceParallelismPass
+ *    docstring: AllReduce -> RMSNorm rewritten as ReduceScatter -> local
+ *    RMSNorm -> AllGather; far_fused_rows() is the local step on a block of
+ *    rows, writing at the rows' own offsets (the gather is the layout).
+ *  - vllm.distributed.device_communicators.aiter_custom_all_reduce,
+ *    use_1stage_fused_ar_rms: rows made of 16-byte packs and a token cap of
+ *    80 for the one-kernel path.  Here: H must be a multiple of 8 (16-byte
+ *    packs of 2-byte elements), and rows <= decode_max_rows (default 80) take
+ *    the cluster-per-row decode kernel.
+ *
+ * Ownership: the caller owns every buffer.  The library allocates and frees
+ * nothing per call and never synchronises the stream; a call only enqueues
+ * one kernel on `stream` and returns.  Results are ready when the stream
+ * reaches that point.  The W partials live in the same GPU's memory (the
+ * tensor-parallel ranks' outputs gathered on one device); they are read only.
+ *
+ * Errors: every argument is checked on the host before anything is
+ * enqueued.  A bad argument returns an error code and enqueues nothing;
+ * nothing is ever skipped silently.  A launch failure returns FAR_ERR_CUDA
+ * and far_last_error() gives the CUDA message (per thread).
+ */
+#ifndef FAR_H_
+#define FAR_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define FAR_VERSION 1
+#define FAR_MAX_W 16      /* most partial buffers per call            */
+#define FAR_MAX_H 16384   /* longest row (elements) the kernels hold  */
+#define FAR_E4M3_MAX 448.0f
+
+typedef enum {
+    FAR_OK = 0,
+    FAR_ERR_INVALID_ARG = 1, /* NULL where a buffer is required, W/T/rows out of range, overlap */
+    FAR_ERR_UNSUPPORTED = 2, /* H not a multiple of 8 or above FAR_MAX_H; device not sm_100 */
+    FAR_ERR_ALIGNMENT = 3,   /* a tensor pointer not 16-byte aligned (scales: 4-byte) */
+    FAR_ERR_CUDA = 4,        /* a CUDA runtime call or the launch failed */
+    FAR_ERR_TIMEOUT = 5,     /* reserved for bounded device-side waits */
+    FAR_ERR_INTERNAL = 6
+} far_status;
+
+typedef enum { FAR_BF16 = 0, FAR_FP16 = 1 } far_dtype;
+
+typedef enum {
+    /* writes residual_out (when there is one) and norm_out (required) */
+    FAR_AR_RESIDUAL_RMSNORM = 0,
+    /* + quant_out, reading the fp32 scalar scale_in[0]; norm_out optional */
+    FAR_AR_RESIDUAL_RMSNORM_FP8_STATIC = 1,
+    /* + quant_out and scale_out[T] (one fp32 scale per row); norm_out optional */
+    FAR_AR_RESIDUAL_RMSNORM_FP8_TOKEN = 2
+} far_pattern;
+
+typedef enum {
+    FAR_REGIME_AUTO = 0,    /* decode when rows <= decode_max_rows, else prefill */
+    FAR_REGIME_DECODE = 1,  /* one thread-block cluster per row            */
+    FAR_REGIME_PREFILL = 2  /* one CTA per row (or several rows per CTA)  */
+} far_regime;
+
+/* Opaque per-device context: caches the SM count, the compute capability
+ * and the tuning knobs (read once from the environment in far_create:
+ * FAR_DECODE_MAX_ROWS, FAR_FORCE_REGIME=decode|prefill, FAR_DECODE_CLUSTER,
+ * FAR_PREFILL_THREADS). */
+typedef struct far_ctx far_ctx;
+
+/* How one call would be launched (see far_describe_launch). */
+typedef struct {
+    int regime;           /* FAR_REGIME_DECODE or FAR_REGIME_PREFILL */
+    int ctas_per_row;     /* cluster size for decode, 1 for prefill */
+    int rows_per_cta;     /* prefill: rows handled by one CTA        */
+    int threads_per_cta;
+    int packs_per_thread; /* 16-byte packs of one row held by one thread */
+    int64_t grid_ctas;    /* CTAs of the launch                       */
+} far_launch_info;
+
+/* Create a context for CUDA device `device` (its ordinal).  Fails with
+ * FAR_ERR_UNSUPPORTED on a device other than compute capability 10.0 and
+ * with FAR_ERR_CUDA when the device cannot be queried. */
+far_status far_create(far_ctx **ctx, int device);
+
+/* Destroy a context (NULL is accepted).  Waits for nothing. */
+far_status far_destroy(far_ctx *ctx);
+
+/*
+ * The fused epilogue on all T rows.
+ *
+ *  partials      host array of W device pointers (1 <= W <= FAR_MAX_W), each
+ *                to a (T, H) tensor of `dtype`; read only.
+ *  residual      (T, H) `dtype`, or NULL for no residual input (the
+ *                sequence-parallel "First" pattern: y is the reduced sum).
+ *  residual_out  (T, H) `dtype` receiving round(y).  NULL with a residual
+ *                means in place: round(y) overwrites `residual`.  NULL with
+ *                no residual means no residual output.  It may equal
+ *                `residual`; it may overlap no other buffer.
+ *  gamma         (H,) `dtype`, the RMSNorm weight.
+ *  T, H          rows (tokens) and hidden size: T >= 0, 8 <= H <= FAR_MAX_H,
+ *                H % 8 == 0.  T == 0 is a valid no-op (buffer pointers are
+ *                then not checked: nothing is read or written).
+ *  eps           added to the mean square inside the root; finite, >= 0.
+ *  weight_bias   added to gamma in fp32 (0 standard, 1 Gemma-style); finite.
+ *  norm_out      (T, H) `dtype`; required by FAR_AR_RESIDUAL_RMSNORM,
+ *                optional (NULL) for the FP8 patterns.
+ *  quant_out     (T, H) uint8 e4m3fn codes; required by the FP8 patterns.
+ *  scale_in      device pointer to one fp32 (static FP8 only).
+ *  scale_out     device array of T fp32 (per-token FP8 only).
+ *  stream        a cudaStream_t (NULL: the legacy default stream).
+ *
+ * Tensor pointers must be 16-byte aligned, scale pointers 4-byte aligned.
+ */
+far_status far_fused(far_ctx *ctx,
+                     const void *const *partials, int W,
+                     const void *residual, void *residual_out,
+                     const void *gamma, int64_t T, int64_t H, far_dtype dtype,
+                     float eps, float weight_bias, far_pattern pattern,
+                     void *norm_out, void *quant_out,
+                     const float *scale_in, float *scale_out, void *stream);
+
+/*
+ * The same on rows [row_begin, row_end) of a T-row problem: the local-norm
+ * step of ReduceScatter -> RMSNorm -> AllGather.  All pointers address the
+ * full T-row tensors; rows outside the range are neither read nor written
+ * (scale_out included).  0 <= row_begin <= row_end <= T, else
+ * FAR_ERR_INVALID_ARG; an empty range is a no-op.  Disjoint row ranges
+ * together give exactly (bit for bit) the far_fused result.
+ */
+far_status far_fused_rows(far_ctx *ctx, int64_t row_begin, int64_t row_end,
+                          const void *const *partials, int W,
+                          const void *residual, void *residual_out,
+                          const void *gamma, int64_t T, int64_t H, far_dtype dtype,
+                          float eps, float weight_bias, far_pattern pattern,
+                          void *norm_out, void *quant_out,
+                          const float *scale_in, float *scale_out, void *stream);
+
+/* Host-only: the status far_fused_rows would return for these arguments
+ * before launching (it touches no GPU and needs no context). */
+far_status far_validate(int64_t row_begin, int64_t row_end,
+                        const void *const *partials, int W,
+                        const void *residual, const void *residual_out,
+                        const void *gamma, int64_t T, int64_t H, far_dtype dtype,
+                        float eps, float weight_bias, far_pattern pattern,
+                        const void *norm_out, const void *quant_out,
+                        const float *scale_in, const float *scale_out);
+
+/* Override the regime choice and the decode row threshold of a context
+ * (decode_max_rows < 0 keeps the current threshold). */
+far_status far_set_regime(far_ctx *ctx, far_regime regime, int decode_max_rows);
+
+/* Fill `info` with the launch geometry a call on `rows` rows would use. */
+far_status far_describe_launch(const far_ctx *ctx, int64_t rows, int64_t H,
+                               far_dtype dtype, far_launch_info *info);
+
+/* Static text for a status code. */
+const char *far_status_string(far_status s);
+
+/* The CUDA error text of the calling thread's last FAR_ERR_CUDA ("" if none). */
+const char *far_last_error(void);
+
+/* FAR_VERSION of the built library. */
+int far_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FAR_H_ */

@@ -1,0 +1,351 @@
+// far_abi.cu -- the C ABI declared in include/far.h: context, host-side
+// argument checks, the choice between the decode and prefill launch shapes,
+// and the launch.  No allocation, no synchronisation.
+#include <cmath>
+#include <cstdint>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <new>
+
+#include <cuda_runtime.h>
+
+#include "far.h"
+#include "far_internal.h"
+
+struct far_ctx {
+  int device;
+  int sm_count;
+  int cc_major;
+  int cc_minor;
+  int decode_max_rows;  // rows <= this take the decode (cluster) kernel
+  int force_regime;     // FAR_REGIME_*
+  int decode_cluster;   // preferred CTAs per row in decode
+  int prefill_threads;  // target threads per row in prefill
+};
+
+namespace {
+
+thread_local char g_last_error[256] = "";
+
+far_status cuda_fail(cudaError_t e, const char* what) {
+  std::snprintf(g_last_error, sizeof(g_last_error), "%s: %s (%s)", what,
+                cudaGetErrorString(e), cudaGetErrorName(e));
+  return FAR_ERR_CUDA;
+}
+
+int env_int(const char* name, int dflt) {
+  const char* s = std::getenv(name);
+  if (s == nullptr || *s == '\0') return dflt;
+  char* end = nullptr;
+  long v = std::strtol(s, &end, 10);
+  return (end != s) ? static_cast<int>(v) : dflt;
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+struct Range {
+  uintptr_t lo, hi;  // [lo, hi)
+};
+
+bool overlap(Range a, Range b) { return a.lo < b.hi && b.lo < a.hi; }
+
+Range span(const void* p, int64_t bytes) {
+  const uintptr_t lo = reinterpret_cast<uintptr_t>(p);
+  return Range{lo, lo + static_cast<uintptr_t>(bytes)};
+}
+
+int pow2_floor(int x) {
+  int p = 1;
+  while (p * 2 <= x) p *= 2;
+  return p;
+}
+
+int pow2_ceil(int x) {
+  int p = 1;
+  while (p < x) p *= 2;
+  return p;
+}
+
+// Prefill geometry: the fewest packs per thread (1, 2, 4 or 8) that keep a
+// row within `target` threads; rows of at most 32 packs share a CTA.
+void plan_prefill(int packs, int target, far::Launch* l) {
+  l->regime = FAR_REGIME_PREFILL;
+  l->cluster = 1;
+  if (packs <= 32) {
+    l->vpt = 1;
+    l->tpr = pow2_ceil(packs);
+    l->rows_per_cta = far::kMaxThreads / l->tpr;
+  } else {
+    int vpt = 1;
+    while (vpt < 8 && (packs + vpt - 1) / vpt > target) vpt *= 2;
+    l->vpt = vpt;
+    l->tpr = (((packs + vpt - 1) / vpt) + 31) / 32 * 32;
+    l->rows_per_cta = 1;
+  }
+  l->threads = l->tpr * l->rows_per_cta;
+}
+
+// Decode geometry: `cluster` CTAs per row (a power of two, at most 16, and
+// at most packs/32 so that each CTA has a warp of work, but large enough for
+// the slice to fit 256 threads at up to 8 packs each), each CTA's slice held
+// at 1, 2, 4 or 8 packs per thread.
+void plan_decode(int packs, int cluster_pref, far::Launch* l) {
+  l->regime = FAR_REGIME_DECODE;
+  int cl = pow2_floor(cluster_pref < 1 ? 1 : (cluster_pref > 16 ? 16 : cluster_pref));
+  while (cl > 1 && packs / cl < 32) cl /= 2;
+  while (cl < 16 && (packs + cl - 1) / cl > 8 * far::kMaxThreads) cl *= 2;
+  l->cluster = cl;
+  const int chunk = (packs + cl - 1) / cl;
+  int vpt = 1;
+  while (vpt < 8 && (chunk + vpt - 1) / vpt > far::kMaxThreads) vpt *= 2;
+  l->vpt = vpt;
+  l->tpr = (((chunk + vpt - 1) / vpt) + 31) / 32 * 32;
+  l->threads = l->tpr;
+  l->rows_per_cta = 1;
+}
+
+far::Launch plan(const far_ctx* ctx, int64_t rows, int64_t H) {
+  const int packs = static_cast<int>(H / far::kPackElems);
+  far::Launch l{};
+  bool decode;
+  if (ctx->force_regime == FAR_REGIME_DECODE)
+    decode = true;
+  else if (ctx->force_regime == FAR_REGIME_PREFILL)
+    decode = false;
+  else
+    decode = rows <= ctx->decode_max_rows && packs >= 64;
+  if (decode) {
+    plan_decode(packs, ctx->decode_cluster, &l);
+    l.grid = rows * l.cluster;
+  } else {
+    plan_prefill(packs, ctx->prefill_threads, &l);
+    l.grid = (rows + l.rows_per_cta - 1) / l.rows_per_cta;
+  }
+  return l;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* far_status_string(far_status s) {
+  switch (s) {
+    case FAR_OK: return "FAR_OK";
+    case FAR_ERR_INVALID_ARG: return "FAR_ERR_INVALID_ARG";
+    case FAR_ERR_UNSUPPORTED: return "FAR_ERR_UNSUPPORTED";
+    case FAR_ERR_ALIGNMENT: return "FAR_ERR_ALIGNMENT";
+    case FAR_ERR_CUDA: return "FAR_ERR_CUDA";
+    case FAR_ERR_TIMEOUT: return "FAR_ERR_TIMEOUT";
+    case FAR_ERR_INTERNAL: return "FAR_ERR_INTERNAL";
+  }
+  return "FAR_ERR_UNKNOWN";
+}
+
+const char* far_last_error(void) { return g_last_error; }
+
+int far_version(void) { return FAR_VERSION; }
+
+far_status far_create(far_ctx** ctx, int device) {
+  if (ctx == nullptr) return FAR_ERR_INVALID_ARG;
+  *ctx = nullptr;
+  int n = 0;
+  cudaError_t e = cudaGetDeviceCount(&n);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDeviceCount");
+  if (device < 0 || device >= n) return FAR_ERR_INVALID_ARG;
+  far_ctx c{};
+  c.device = device;
+  if ((e = cudaDeviceGetAttribute(&c.sm_count, cudaDevAttrMultiProcessorCount, device)) != cudaSuccess ||
+      (e = cudaDeviceGetAttribute(&c.cc_major, cudaDevAttrComputeCapabilityMajor, device)) != cudaSuccess ||
+      (e = cudaDeviceGetAttribute(&c.cc_minor, cudaDevAttrComputeCapabilityMinor, device)) != cudaSuccess)
+    return cuda_fail(e, "cudaDeviceGetAttribute");
+  if (c.cc_major != 10 || c.cc_minor != 0) {
+    std::snprintf(g_last_error, sizeof(g_last_error),
+                  "device %d has compute capability %d.%d; this library is built for sm_100a only",
+                  device, c.cc_major, c.cc_minor);
+    return FAR_ERR_UNSUPPORTED;
+  }
+  c.decode_max_rows = env_int("FAR_DECODE_MAX_ROWS", 80);
+  c.decode_cluster = env_int("FAR_DECODE_CLUSTER", 8);
+  c.prefill_threads = env_int("FAR_PREFILL_THREADS", 256);
+  if (c.prefill_threads < 32) c.prefill_threads = 32;
+  if (c.prefill_threads > far::kMaxThreads) c.prefill_threads = far::kMaxThreads;
+  c.force_regime = FAR_REGIME_AUTO;
+  if (const char* f = std::getenv("FAR_FORCE_REGIME")) {
+    if (std::strcmp(f, "decode") == 0) c.force_regime = FAR_REGIME_DECODE;
+    if (std::strcmp(f, "prefill") == 0) c.force_regime = FAR_REGIME_PREFILL;
+  }
+
+  int prev = -1;
+  if ((e = cudaGetDevice(&prev)) != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (prev != device && (e = cudaSetDevice(device)) != cudaSuccess) return cuda_fail(e, "cudaSetDevice");
+  e = far::configure_kernels();
+  if (prev != device) cudaSetDevice(prev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
+
+  far_ctx* out = new (std::nothrow) far_ctx(c);
+  if (out == nullptr) return FAR_ERR_INTERNAL;
+  *ctx = out;
+  return FAR_OK;
+}
+
+far_status far_destroy(far_ctx* ctx) {
+  delete ctx;
+  return FAR_OK;
+}
+
+far_status far_set_regime(far_ctx* ctx, far_regime regime, int decode_max_rows) {
+  if (ctx == nullptr) return FAR_ERR_INVALID_ARG;
+  if (regime != FAR_REGIME_AUTO && regime != FAR_REGIME_DECODE && regime != FAR_REGIME_PREFILL)
+    return FAR_ERR_INVALID_ARG;
+  ctx->force_regime = regime;
+  if (decode_max_rows >= 0) ctx->decode_max_rows = decode_max_rows;
+  return FAR_OK;
+}
+
+far_status far_describe_launch(const far_ctx* ctx, int64_t rows, int64_t H, far_dtype dtype,
+                               far_launch_info* info) {
+  if (ctx == nullptr || info == nullptr || rows < 0) return FAR_ERR_INVALID_ARG;
+  if (dtype != FAR_BF16 && dtype != FAR_FP16) return FAR_ERR_INVALID_ARG;
+  if (H <= 0 || H % far::kPackElems != 0 || H > far::kMaxH) return FAR_ERR_UNSUPPORTED;
+  const far::Launch l = plan(ctx, rows, H);
+  info->regime = l.regime;
+  info->ctas_per_row = l.cluster;
+  info->rows_per_cta = l.rows_per_cta;
+  info->threads_per_cta = l.threads;
+  info->packs_per_thread = l.vpt;
+  info->grid_ctas = l.grid;
+  return FAR_OK;
+}
+
+far_status far_validate(int64_t row_begin, int64_t row_end, const void* const* partials, int W,
+                        const void* residual, const void* residual_out, const void* gamma,
+                        int64_t T, int64_t H, far_dtype dtype, float eps, float weight_bias,
+                        far_pattern pattern, const void* norm_out, const void* quant_out,
+                        const float* scale_in, const float* scale_out) {
+  if (W < 1 || W > FAR_MAX_W || partials == nullptr) return FAR_ERR_INVALID_ARG;
+  if (T < 0 || H <= 0) return FAR_ERR_INVALID_ARG;
+  if (dtype != FAR_BF16 && dtype != FAR_FP16) return FAR_ERR_INVALID_ARG;
+  if (pattern != FAR_AR_RESIDUAL_RMSNORM && pattern != FAR_AR_RESIDUAL_RMSNORM_FP8_STATIC &&
+      pattern != FAR_AR_RESIDUAL_RMSNORM_FP8_TOKEN)
+    return FAR_ERR_INVALID_ARG;
+  if (H % far::kPackElems != 0 || H > FAR_MAX_H) return FAR_ERR_UNSUPPORTED;
+  if (row_begin < 0 || row_end < row_begin || row_end > T) return FAR_ERR_INVALID_ARG;
+  if (T > INT64_MAX / (H * 2)) return FAR_ERR_INVALID_ARG;
+  if (!std::isfinite(eps) || eps < 0.f || !std::isfinite(weight_bias)) return FAR_ERR_INVALID_ARG;
+  if (T == 0) return FAR_OK;  // nothing is read or written: buffers are not checked
+  if (gamma == nullptr) return FAR_ERR_INVALID_ARG;
+  for (int r = 0; r < W; ++r)
+    if (partials[r] == nullptr) return FAR_ERR_INVALID_ARG;
+  if (pattern == FAR_AR_RESIDUAL_RMSNORM && norm_out == nullptr) return FAR_ERR_INVALID_ARG;
+  if (pattern == FAR_AR_RESIDUAL_RMSNORM_FP8_STATIC && (quant_out == nullptr || scale_in == nullptr))
+    return FAR_ERR_INVALID_ARG;
+  if (pattern == FAR_AR_RESIDUAL_RMSNORM_FP8_TOKEN && (quant_out == nullptr || scale_out == nullptr))
+    return FAR_ERR_INVALID_ARG;
+
+  // 16-byte packs everywhere; fp32 scales need 4 bytes.
+  for (int r = 0; r < W; ++r)
+    if (!aligned(partials[r], 16)) return FAR_ERR_ALIGNMENT;
+  const void* tens[] = {residual, residual_out, gamma, norm_out, quant_out};
+  for (const void* p : tens)
+    if (p != nullptr && !aligned(p, 16)) return FAR_ERR_ALIGNMENT;
+  if (scale_in != nullptr && !aligned(scale_in, 4)) return FAR_ERR_ALIGNMENT;
+  if (scale_out != nullptr && !aligned(scale_out, 4)) return FAR_ERR_ALIGNMENT;
+
+  // Outputs overlap no input and no other output.  The one exception is the
+  // new residual written exactly over the residual (in place).
+  {
+    const int64_t tb = T * H * 2;
+    const void* res_w = (residual_out != nullptr) ? residual_out : residual;  // may be null
+    Range outs[4];
+    int no = 0;
+    if (res_w != nullptr) outs[no++] = span(res_w, tb);  // outs[0] when present
+    if (norm_out != nullptr) outs[no++] = span(norm_out, tb);
+    if (pattern != FAR_AR_RESIDUAL_RMSNORM) outs[no++] = span(quant_out, T * H);
+    if (pattern == FAR_AR_RESIDUAL_RMSNORM_FP8_TOKEN) outs[no++] = span(scale_out, T * 4);
+    Range ins[FAR_MAX_W + 3];
+    int ni = 0;
+    for (int r = 0; r < W; ++r) ins[ni++] = span(partials[r], tb);
+    const int res_in = (residual != nullptr) ? ni : -1;
+    if (residual != nullptr) ins[ni++] = span(residual, tb);
+    ins[ni++] = span(gamma, H * 2);
+    if (pattern == FAR_AR_RESIDUAL_RMSNORM_FP8_STATIC) ins[ni++] = span(scale_in, 4);
+    for (int i = 0; i < no; ++i) {
+      for (int j = 0; j < ni; ++j) {
+        if (!overlap(outs[i], ins[j])) continue;
+        const bool in_place = (i == 0 && res_w != nullptr && j == res_in && res_w == residual);
+        if (!in_place) return FAR_ERR_INVALID_ARG;
+      }
+      for (int j = i + 1; j < no; ++j)
+        if (overlap(outs[i], outs[j])) return FAR_ERR_INVALID_ARG;
+    }
+  }
+  return FAR_OK;
+}
+
+far_status far_fused_rows(far_ctx* ctx, int64_t row_begin, int64_t row_end,
+                          const void* const* partials, int W, const void* residual,
+                          void* residual_out, const void* gamma, int64_t T, int64_t H,
+                          far_dtype dtype, float eps, float weight_bias, far_pattern pattern,
+                          void* norm_out, void* quant_out, const float* scale_in, float* scale_out,
+                          void* stream) {
+  if (ctx == nullptr) return FAR_ERR_INVALID_ARG;
+  far_status st = far_validate(row_begin, row_end, partials, W, residual, residual_out, gamma, T, H,
+                               dtype, eps, weight_bias, pattern, norm_out, quant_out, scale_in,
+                               scale_out);
+  if (st != FAR_OK) return st;
+  if (row_end == row_begin) return FAR_OK;
+
+  far::Params p{};
+  for (int r = 0; r < W; ++r) p.partials[r] = partials[r];
+  p.residual = residual;
+  p.residual_out = (residual_out == nullptr) ? const_cast<void*>(residual) : residual_out;
+  p.gamma = gamma;
+  p.norm_out = norm_out;
+  p.quant_out = (pattern == FAR_AR_RESIDUAL_RMSNORM) ? nullptr : static_cast<uint8_t*>(quant_out);
+  p.scale_in = scale_in;
+  p.scale_out = scale_out;
+  p.W = W;
+  p.H = static_cast<int>(H);
+  p.packs = static_cast<int>(H / far::kPackElems);
+  p.pattern = static_cast<int>(pattern);
+  p.eps = eps;
+  p.weight_bias = weight_bias;
+
+  int prev = -1;
+  cudaError_t e = cudaGetDevice(&prev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (prev != ctx->device && (e = cudaSetDevice(ctx->device)) != cudaSuccess)
+    return cuda_fail(e, "cudaSetDevice");
+
+  // grid.y (decode) and grid.x (prefill) bound the rows of one launch
+  const int64_t rows = row_end - row_begin;
+  const far::Launch whole = plan(ctx, rows, H);
+  const int64_t max_rows = whole.regime == FAR_REGIME_DECODE
+                               ? 65535
+                               : static_cast<int64_t>(0x7fffffff) * whole.rows_per_cta;
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  for (int64_t b = row_begin; b < row_end && e == cudaSuccess; b += max_rows) {
+    const int64_t n = (row_end - b < max_rows) ? (row_end - b) : max_rows;
+    far::Launch l = whole;
+    l.grid = (whole.regime == FAR_REGIME_DECODE) ? n * l.cluster
+                                                 : (n + l.rows_per_cta - 1) / l.rows_per_cta;
+    p.row_begin = b;
+    p.row_end = b + n;
+    e = (l.regime == FAR_REGIME_DECODE) ? far::launch_decode(p, dtype, l, s)
+                                        : far::launch_prefill(p, dtype, l, s);
+  }
+  if (prev != ctx->device) cudaSetDevice(prev);
+  if (e != cudaSuccess) return cuda_fail(e, "kernel launch");
+  return FAR_OK;
+}
+
+far_status far_fused(far_ctx* ctx, const void* const* partials, int W, const void* residual,
+                     void* residual_out, const void* gamma, int64_t T, int64_t H, far_dtype dtype,
+                     float eps, float weight_bias, far_pattern pattern, void* norm_out,
+                     void* quant_out, const float* scale_in, float* scale_out, void* stream) {
+  return far_fused_rows(ctx, 0, T, partials, W, residual, residual_out, gamma, T, H, dtype, eps,
+                        weight_bias, pattern, norm_out, quant_out, scale_in, scale_out, stream);
+}
+
+}  // extern "C"

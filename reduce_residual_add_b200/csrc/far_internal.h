@@ -1,0 +1,59 @@
+// far_internal.h -- declarations shared by the ABI layer (far_abi.cu) and the
+// kernels (far_kernels.cu).  Not installed; the public interface is far.h.
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace far {
+
+constexpr int kMaxW = 16;        // partial buffers per call
+constexpr int kMaxH = 16384;     // longest row held in registers
+constexpr int kPackElems = 8;    // 2-byte elements per 16-byte pack
+constexpr int kMaxThreads = 256; // threads per CTA, both regimes
+
+enum Dtype : int { kBf16 = 0, kFp16 = 1 };
+enum Pattern : int { kNormOnly = 0, kFp8Static = 1, kFp8Token = 2 };
+
+// Everything one launch needs, passed by value in the kernel's parameter
+// space (about 200 bytes).
+struct Params {
+  const void* partials[kMaxW];  // W read-only (T, H) tensors
+  const void* residual;         // (T, H) or null
+  void* residual_out;           // (T, H) or null (may equal residual)
+  const void* gamma;            // (H,)
+  void* norm_out;               // (T, H) or null
+  uint8_t* quant_out;           // (T, H) e4m3 codes or null
+  const float* scale_in;        // static FP8 scale (1 float) or null
+  float* scale_out;             // per-row FP8 scales (T floats) or null
+  int64_t row_begin;            // rows [row_begin, row_end) of the T-row tensors
+  int64_t row_end;
+  int W;
+  int H;
+  int packs;                    // H / 8
+  int pattern;
+  float eps;
+  float weight_bias;
+};
+
+// Geometry of one launch, chosen on the host.
+struct Launch {
+  int regime;           // 1 decode (cluster per row), 2 prefill
+  int cluster;          // CTAs per row (decode)
+  int vpt;              // 16-byte packs per thread
+  int tpr;              // threads per row (prefill) / per CTA (decode)
+  int rows_per_cta;     // prefill
+  int threads;          // threads per CTA
+  int64_t grid;         // CTAs
+};
+
+// Enqueue one kernel on `stream`.  Returns the launch error (cudaSuccess if
+// the launch was accepted).
+cudaError_t launch_prefill(const Params& p, int dtype, const Launch& l, cudaStream_t stream);
+cudaError_t launch_decode(const Params& p, int dtype, const Launch& l, cudaStream_t stream);
+
+// One-time per-device set-up of kernel attributes (non-portable cluster
+// sizes).  Call with the device current.
+cudaError_t configure_kernels();
+
+}  // namespace far

@@ -1,0 +1,431 @@
+// far_kernels.cu -- sm_100a kernels of the fused "all-reduce + residual-add +
+// RMSNorm (+FP8-e4m3)" epilogue.
+//
+// Per row t (fused_allreduce_rms_norm docstring on the
+// vllm.models.common.ops.fused_allreduce_rms_norm page: the result is
+// norm(all_reduce(h), residual) with fp32 accumulation):
+//   y = sum_r p_r + residual          -> residual_out = round(y)
+//   rinv = 1/sqrt(mean(y^2) + eps)
+//   o = y * rinv * (gamma + weight_bias) -> norm_out = round(o)
+//   static FP8 (FusedAddRMSNormStaticQuantPattern): q = e4m3(o / scale)
+//   per-token FP8 (FusedAddRMSNormDynamicQuantPattern):
+//       scale_t = max|o| / 448, q = e4m3(o / scale_t)
+//
+// The work is HBM-bound (about 8 flops per (W+3)*2 bytes): no tensor cores.
+// A whole row stays in registers between its reduction and its scaling, so
+// every byte crosses HBM once.  Two launch shapes share one row routine:
+//  - prefill: one CTA per row (or 256/tpr rows per CTA when a row has at
+//    most 32 packs), 16-byte vector loads, warp-shuffle + shared-memory
+//    reductions;
+//  - decode: one thread-block cluster per row, each CTA a slice of the
+//    hidden dimension, the row's sum of squares (and amax) combined through
+//    distributed shared memory, so that a handful of rows still spreads
+//    over many SMs.
+#include <cooperative_groups.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
+#include <cuda_runtime.h>
+
+#include "far_internal.h"
+
+namespace cg = cooperative_groups;
+
+namespace far {
+namespace {
+
+// ---------------------------------------------------------------------------
+// 16-byte packs of eight 2-byte elements
+// ---------------------------------------------------------------------------
+
+struct Bf16T {
+  // bf16 is the upper half of an fp32: widening is a shift
+  static __device__ __forceinline__ void unpack(const uint4& v, float (&f)[8]) {
+    f[0] = __uint_as_float(v.x << 16);
+    f[1] = __uint_as_float(v.x & 0xffff0000u);
+    f[2] = __uint_as_float(v.y << 16);
+    f[3] = __uint_as_float(v.y & 0xffff0000u);
+    f[4] = __uint_as_float(v.z << 16);
+    f[5] = __uint_as_float(v.z & 0xffff0000u);
+    f[6] = __uint_as_float(v.w << 16);
+    f[7] = __uint_as_float(v.w & 0xffff0000u);
+  }
+  static __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
+    __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);  // round to nearest even
+    return *reinterpret_cast<uint32_t*>(&h);
+  }
+};
+
+struct Fp16T {
+  static __device__ __forceinline__ void unpack(const uint4& v, float (&f)[8]) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      __half2 h = *reinterpret_cast<const __half2*>(&w[i]);
+      float2 x = __half22float2(h);
+      f[2 * i] = x.x;
+      f[2 * i + 1] = x.y;
+    }
+  }
+  static __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
+    __half2 h = __floats2half2_rn(lo, hi);  // round to nearest even
+    return *reinterpret_cast<uint32_t*>(&h);
+  }
+};
+
+template <class DT>
+__device__ __forceinline__ uint4 pack8(const float (&f)[8]) {
+  return make_uint4(DT::pack2(f[0], f[1]), DT::pack2(f[2], f[3]),
+                    DT::pack2(f[4], f[5]), DT::pack2(f[6], f[7]));
+}
+
+// Four e4m3fn codes (round to nearest even, saturating to +-448), first
+// value in the lowest byte.
+__device__ __forceinline__ uint32_t e4m3x4(float a, float b, float c, float d) {
+  const uint32_t lo = __nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3);
+  const uint32_t hi = __nv_cvt_float2_to_fp8x2(make_float2(c, d), __NV_SATFINITE, __NV_E4M3);
+  return lo | (hi << 16);
+}
+
+// ---------------------------------------------------------------------------
+// memory access
+// ---------------------------------------------------------------------------
+
+// Partials: read once and never written during the kernel -> non-coherent
+// path, no L1 allocation.
+__device__ __forceinline__ uint4 ld_once(const uint4* p) {
+  uint4 r;
+  asm volatile("ld.global.nc.L1::no_allocate.L2::256B.v4.u32 {%0,%1,%2,%3}, [%4];"
+      : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+      : "l"(p));
+  return r;
+}
+
+// Residual: may be overwritten in place by the same thread afterwards, so
+// it takes the coherent path (still without L1 allocation).
+__device__ __forceinline__ uint4 ld_once_coherent(const uint4* p) {
+  uint4 r;
+  asm volatile("ld.global.L1::no_allocate.L2::256B.v4.u32 {%0,%1,%2,%3}, [%4];"
+      : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+      : "l"(p));
+  return r;
+}
+
+// ---------------------------------------------------------------------------
+// reductions over one row (all results identical in every thread of the row)
+// ---------------------------------------------------------------------------
+
+// Butterfly over `width` lanes: lane i and lane i^m add the same two values,
+// so every lane ends with the bit-identical total.
+__device__ __forceinline__ float group_sum(float v, int width) {
+  for (int m = width >> 1; m > 0; m >>= 1) v += __shfl_xor_sync(0xffffffffu, v, m, width);
+  return v;
+}
+__device__ __forceinline__ float group_max(float v, int width) {
+  for (int m = width >> 1; m > 0; m >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, m, width));
+  return v;
+}
+
+// A row inside one warp: blockDim.x lanes (a power of two <= 32) per row.
+struct SubwarpRed {
+  int width;
+  __device__ float sum(float v) const { return group_sum(v, width); }
+  __device__ float max(float v) const { return group_max(v, width); }
+  __device__ bool leader() const { return threadIdx.x == 0; }
+};
+
+// A row over the whole CTA (blockDim.x a multiple of 32, blockDim.y == 1).
+// Each warp reduces, lane 0 parks the warp total in shared memory, and after
+// one barrier every warp reduces the same <= 32 totals in the same order.
+struct BlockRed {
+  float* s_sum;  // [32]
+  float* s_max;  // [32]
+  __device__ float reduce(float v, float* slot, bool is_max) const {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    v = is_max ? group_max(v, 32) : group_sum(v, 32);
+    if (lane == 0) slot[warp] = v;
+    __syncthreads();
+    float t = lane < nw ? slot[lane] : 0.f;
+    return is_max ? group_max(t, 32) : group_sum(t, 32);
+  }
+  __device__ float sum(float v) const { return reduce(v, s_sum, false); }
+  __device__ float max(float v) const { return reduce(v, s_max, true); }
+  __device__ bool leader() const { return threadIdx.x == 0; }
+};
+
+// A row over a thread-block cluster: CTA totals meet in distributed shared
+// memory.  Every CTA reads all ranks' totals in rank order, so every CTA
+// holds the same bits.  Each quantity has its own slot, so no slot is
+// rewritten while a peer may still read it; the kernel ends with one more
+// cluster barrier before any CTA (and its shared memory) goes away.
+struct ClusterRed {
+  BlockRed blk;
+  float* s_cta;  // [2]: 0 = sum of squares, 1 = amax
+  __device__ float across(float t, int slot, bool is_max) const {
+    cg::cluster_group cl = cg::this_cluster();
+    if (threadIdx.x == 0) s_cta[slot] = t;
+    cl.sync();
+    const int lane = threadIdx.x & 31;
+    const int n = static_cast<int>(cl.num_blocks());
+    float u = 0.f;
+    if (lane < n) u = *cl.map_shared_rank(s_cta + slot, lane);
+    return is_max ? group_max(u, 32) : group_sum(u, 32);
+  }
+  __device__ float sum(float v) const { return across(blk.sum(v), 0, false); }
+  __device__ float max(float v) const { return across(blk.max(v), 1, true); }
+  __device__ bool leader() const {
+    return threadIdx.x == 0 && cg::this_cluster().block_rank() == 0;
+  }
+};
+
+// ---------------------------------------------------------------------------
+// one row (or one slice of it): packs j = j0 + k*jstride, k < VPT, j < jend
+// ---------------------------------------------------------------------------
+
+template <class DT, int VPT, class Red>
+__device__ __forceinline__ void fused_row(const Params& p, int64_t row, bool row_ok,
+                                          int j0, int jstride, int jend, const Red& red) {
+  const int64_t rbase = row * static_cast<int64_t>(p.packs);  // first pack of the row
+  float y[VPT][8];
+  bool ok[VPT];
+#pragma unroll
+  for (int k = 0; k < VPT; ++k) {
+    ok[k] = row_ok && (j0 + k * jstride) < jend;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) y[k][i] = 0.f;
+  }
+
+  // a1: sum the W partials in fp32, four buffers' loads in flight per step.
+  for (int r0 = 0; r0 < p.W; r0 += 4) {
+    uint4 v[4][VPT];
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+#pragma unroll
+      for (int k = 0; k < VPT; ++k) {
+        v[c][k] = make_uint4(0u, 0u, 0u, 0u);
+        if (r0 + c < p.W && ok[k])
+          v[c][k] = ld_once(static_cast<const uint4*>(p.partials[r0 + c]) + rbase + j0 + k * jstride);
+      }
+    }
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+#pragma unroll
+      for (int k = 0; k < VPT; ++k) {
+        float f[8];
+        DT::unpack(v[c][k], f);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) y[k][i] += f[i];
+      }
+    }
+  }
+
+  // a2: add the residual and write the new residual.
+  if (p.residual != nullptr) {
+    uint4 v[VPT];
+#pragma unroll
+    for (int k = 0; k < VPT; ++k) {
+      v[k] = make_uint4(0u, 0u, 0u, 0u);
+      if (ok[k]) v[k] = ld_once_coherent(static_cast<const uint4*>(p.residual) + rbase + j0 + k * jstride);
+    }
+#pragma unroll
+    for (int k = 0; k < VPT; ++k) {
+      float f[8];
+      DT::unpack(v[k], f);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) y[k][i] += f[i];
+    }
+  }
+  if (p.residual_out != nullptr) {
+#pragma unroll
+    for (int k = 0; k < VPT; ++k)
+      if (ok[k]) static_cast<uint4*>(p.residual_out)[rbase + j0 + k * jstride] = pack8<DT>(y[k]);
+  }
+
+  // a3: mean of squares; pairwise inside the thread, butterflies above it.
+  float sq[VPT];
+#pragma unroll
+  for (int k = 0; k < VPT; ++k) {
+    const float a = y[k][0] * y[k][0] + y[k][1] * y[k][1];
+    const float b = y[k][2] * y[k][2] + y[k][3] * y[k][3];
+    const float c = y[k][4] * y[k][4] + y[k][5] * y[k][5];
+    const float d = y[k][6] * y[k][6] + y[k][7] * y[k][7];
+    sq[k] = (a + b) + (c + d);
+  }
+#pragma unroll
+  for (int w = 1; w < VPT; w <<= 1)
+#pragma unroll
+    for (int k = 0; k + w < VPT; k += 2 * w) sq[k] += sq[k + w];
+  const float ss = red.sum(sq[0]);
+  const float ms = __fdiv_rn(ss, static_cast<float>(p.H));
+  const float rinv = __frsqrt_rn(ms + p.eps);
+
+  // a4: o = y * rinv * (gamma + weight_bias); a5: FP8 codes.
+  const bool fp8_static = p.pattern == kFp8Static;
+  const bool fp8_token = p.pattern == kFp8Token;
+  const float s_static = fp8_static ? __ldg(p.scale_in) : 1.f;
+  float amax = 0.f;
+#pragma unroll
+  for (int k = 0; k < VPT; ++k) {
+    if (!ok[k]) continue;
+    const int64_t pk = rbase + j0 + k * jstride;
+    float g[8];
+    DT::unpack(__ldg(static_cast<const uint4*>(p.gamma) + j0 + k * jstride), g);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) y[k][i] = (y[k][i] * rinv) * (g[i] + p.weight_bias);
+    if (p.norm_out != nullptr) static_cast<uint4*>(p.norm_out)[pk] = pack8<DT>(y[k]);
+    if (fp8_static) {
+      float q[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) q[i] = __fdiv_rn(y[k][i], s_static);
+      reinterpret_cast<uint2*>(p.quant_out)[pk] =
+          make_uint2(e4m3x4(q[0], q[1], q[2], q[3]), e4m3x4(q[4], q[5], q[6], q[7]));
+    }
+    if (fp8_token) {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(y[k][i]));
+    }
+  }
+
+  if (fp8_token) {
+    const float rowmax = red.max(amax);
+    const float scale = __fdiv_rn(rowmax, 448.f);
+    if (row_ok && red.leader()) p.scale_out[row] = scale;
+#pragma unroll
+    for (int k = 0; k < VPT; ++k) {
+      if (!ok[k]) continue;
+      const int64_t pk = rbase + j0 + k * jstride;
+      uint2 codes = make_uint2(0u, 0u);
+      if (scale != 0.f) {
+        float q[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) q[i] = __fdiv_rn(y[k][i], scale);
+        codes = make_uint2(e4m3x4(q[0], q[1], q[2], q[3]), e4m3x4(q[4], q[5], q[6], q[7]));
+      }
+      reinterpret_cast<uint2*>(p.quant_out)[pk] = codes;
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// kernels
+// ---------------------------------------------------------------------------
+
+// Prefill: blockDim = (tpr, rows_per_cta).  SUB: a row lives inside one warp
+// (tpr <= 32, power of two); otherwise one row per CTA.
+template <class DT, int VPT, bool SUB>
+__global__ void __launch_bounds__(kMaxThreads, (VPT >= 8 ? 1 : 2))
+far_prefill_kernel(const Params p) {
+  const int64_t row = p.row_begin + static_cast<int64_t>(blockIdx.x) * blockDim.y + threadIdx.y;
+  const bool row_ok = row < p.row_end;
+  if constexpr (SUB) {
+    const SubwarpRed red{static_cast<int>(blockDim.x)};
+    fused_row<DT, VPT>(p, row, row_ok, threadIdx.x, blockDim.x, p.packs, red);
+  } else {
+    __shared__ float s_sum[32], s_max[32];
+    const BlockRed red{s_sum, s_max};
+    fused_row<DT, VPT>(p, row, row_ok, threadIdx.x, blockDim.x, p.packs, red);
+  }
+}
+
+// Decode: grid = (cluster, rows), one cluster per row; CTA `rank` of the
+// cluster takes packs [rank*chunk, min(packs, (rank+1)*chunk)).
+template <class DT, int VPT>
+__global__ void __launch_bounds__(kMaxThreads, (VPT >= 8 ? 1 : 2))
+far_decode_kernel(const Params p) {
+  __shared__ float s_sum[32], s_max[32], s_cta[2];
+  cg::cluster_group cl = cg::this_cluster();
+  const int rank = static_cast<int>(cl.block_rank());
+  const int ncta = static_cast<int>(cl.num_blocks());
+  const int64_t row = p.row_begin + blockIdx.y;
+  const int chunk = (p.packs + ncta - 1) / ncta;
+  const int jbeg = rank * chunk;
+  const int jend = min(p.packs, jbeg + chunk);
+  const ClusterRed red{BlockRed{s_sum, s_max}, s_cta};
+  fused_row<DT, VPT>(p, row, row < p.row_end, jbeg + static_cast<int>(threadIdx.x),
+                     blockDim.x, jend, red);
+  cl.sync();  // keep this CTA's shared memory alive until every peer has read it
+}
+
+template <class DT, int VPT, bool SUB>
+cudaError_t launch_prefill_t(const Params& p, const Launch& l, cudaStream_t s) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(l.grid), 1, 1);
+  cfg.blockDim = dim3(static_cast<unsigned>(l.tpr), static_cast<unsigned>(l.rows_per_cta), 1);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = s;
+  cfg.attrs = nullptr;
+  cfg.numAttrs = 0;
+  return cudaLaunchKernelEx(&cfg, far_prefill_kernel<DT, VPT, SUB>, p);
+}
+
+template <class DT, int VPT>
+cudaError_t launch_decode_t(const Params& p, const Launch& l, cudaStream_t s) {
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = static_cast<unsigned>(l.cluster);
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(l.cluster), static_cast<unsigned>(l.grid / l.cluster), 1);
+  cfg.blockDim = dim3(static_cast<unsigned>(l.threads), 1, 1);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, far_decode_kernel<DT, VPT>, p);
+}
+
+template <class DT>
+cudaError_t launch_prefill_dt(const Params& p, const Launch& l, cudaStream_t s) {
+  if (l.tpr <= 32 && l.rows_per_cta > 1) return launch_prefill_t<DT, 1, true>(p, l, s);
+  switch (l.vpt) {
+    case 1: return launch_prefill_t<DT, 1, false>(p, l, s);
+    case 2: return launch_prefill_t<DT, 2, false>(p, l, s);
+    case 4: return launch_prefill_t<DT, 4, false>(p, l, s);
+    case 8: return launch_prefill_t<DT, 8, false>(p, l, s);
+    default: return cudaErrorInvalidConfiguration;
+  }
+}
+
+template <class DT>
+cudaError_t launch_decode_dt(const Params& p, const Launch& l, cudaStream_t s) {
+  switch (l.vpt) {
+    case 1: return launch_decode_t<DT, 1>(p, l, s);
+    case 2: return launch_decode_t<DT, 2>(p, l, s);
+    case 4: return launch_decode_t<DT, 4>(p, l, s);
+    case 8: return launch_decode_t<DT, 8>(p, l, s);
+    default: return cudaErrorInvalidConfiguration;
+  }
+}
+
+template <class DT>
+cudaError_t allow_large_clusters() {
+  cudaError_t e = cudaSuccess;
+  const auto set = [&](auto kern) {
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+  };
+  set(far_decode_kernel<DT, 1>);
+  set(far_decode_kernel<DT, 2>);
+  set(far_decode_kernel<DT, 4>);
+  set(far_decode_kernel<DT, 8>);
+  return e;
+}
+
+}  // namespace
+
+cudaError_t launch_prefill(const Params& p, int dtype, const Launch& l, cudaStream_t s) {
+  return dtype == kBf16 ? launch_prefill_dt<Bf16T>(p, l, s) : launch_prefill_dt<Fp16T>(p, l, s);
+}
+
+cudaError_t launch_decode(const Params& p, int dtype, const Launch& l, cudaStream_t s) {
+  return dtype == kBf16 ? launch_decode_dt<Bf16T>(p, l, s) : launch_decode_dt<Fp16T>(p, l, s);
+}
+
+cudaError_t configure_kernels() {
+  cudaError_t e = allow_large_clusters<Bf16T>();
+  if (e == cudaSuccess) e = allow_large_clusters<Fp16T>();
+  return e;
+}
+
+}  // namespace far

@@ -1,0 +1,156 @@
+"""Helpers of the GPU parity tests: run the CUDA path through the binding and
+compare it with the oracle under the stated tolerances.
+
+Tolerances:
+* bf16 / fp16 outputs: at most 1 ulp from the oracle's correctly rounded
+  value (distance on the format's ordered grid, subnormals included; the sign
+  of a zero is not compared);
+* e4m3 codes: at most 1 step on the ordered code grid; a code the oracle
+  saturates (+-448) must be saturated on the GPU too; NaN codes must agree;
+* per-token scales: relative error at most 1e-6 (exact when 0).
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import oracle
+from reduce_residual_add_b200 import far
+from reduce_residual_add_b200.inputs import as_u16
+
+SCALE_RTOL = 1e-6
+
+
+def _ordered(bits: np.ndarray, width: int) -> np.ndarray:
+    b = bits.astype(np.int64)
+    sign = 1 << (width - 1)
+    mag = b & (sign - 1)
+    return np.where(b & sign, -mag, mag)
+
+
+def _is_nan16(bits: np.ndarray, dtype: str) -> np.ndarray:
+    b = bits.astype(np.int64) & 0x7FFF
+    if dtype == "bf16":
+        return b > 0x7F80
+    return b > 0x7C00
+
+
+def ulp16(a: np.ndarray, b: np.ndarray, dtype: str) -> np.ndarray:
+    d = np.abs(_ordered(a, 16) - _ordered(b, 16))
+    na, nb = _is_nan16(a, dtype), _is_nan16(b, dtype)
+    d = np.where(na & nb, 0, d)
+    return np.where(na ^ nb, 1 << 20, d)
+
+
+def code_steps(a: np.ndarray, b: np.ndarray) -> np.ndarray:
+    d = np.abs(_ordered(a, 8) - _ordered(b, 8))
+    na, nb = (a & 0x7F) == 0x7F, (b & 0x7F) == 0x7F
+    d = np.where(na & nb, 0, d)
+    return np.where(na ^ nb, 1 << 20, d)
+
+
+def to_gpu(inp: dict, device="cuda") -> dict:
+    g = {"partials": [p.to(device) for p in inp["partials"]],
+         "residual": None if inp["residual"] is None else inp["residual"].to(device),
+         "gamma": inp["gamma"].to(device)}
+    return g
+
+
+def run_gpu(ctx, g: dict, eps: float, wb: float, pattern: int, scale_in=None, rows=None,
+            want_norm: bool = True, want_residual_out: bool = True, in_place: bool = False,
+            stream=None, guard: int = 0) -> dict:
+    """One call of the CUDA path; returns numpy arrays of the outputs (full T).
+
+    ``guard`` > 0 surrounds every output with that many canary bytes (0xA5)
+    and checks afterwards that none of them changed."""
+    ps = g["partials"]
+    T, H = ps[0].reshape(-1, g["gamma"].numel()).shape
+    dt = ps[0].dtype
+    dev = ps[0].device
+    canaries = []
+
+    def alloc(n_elems, dtype_):
+        es = torch.empty((), dtype=dtype_).element_size()
+        gb = (guard + 15) // 16 * 16
+        raw = torch.full((gb * 2 + n_elems * es,), 0xA5, dtype=torch.uint8, device=dev)
+        view = raw[gb:gb + n_elems * es].view(dtype_)
+        if guard:
+            canaries.append((raw, gb, n_elems * es))
+        else:
+            view.zero_()
+        return view
+
+    res = g["residual"]
+    rout = None
+    if res is not None and in_place:
+        res = res.clone()
+    elif want_residual_out:
+        rout = alloc(T * H, dt).view(T, H)
+    nout = alloc(T * H, dt).view(T, H) if want_norm else None
+    qout = alloc(T * H, torch.uint8).view(T, H) if pattern != 0 else None
+    sout = alloc(T, torch.float32) if pattern == 2 else None
+    sin = torch.tensor([scale_in], dtype=torch.float32, device=dev) if pattern == 1 else None
+    kw = dict(residual_out=rout, norm_out=nout, quant_out=qout, scale_in=sin, scale_out=sout,
+              stream=stream)
+    if rows is None:
+        far.far_fused(ctx, ps, res, g["gamma"], eps, wb, pattern, **kw)
+    else:
+        far.far_fused_rows(ctx, rows[0], rows[1], ps, res, g["gamma"], eps, wb, pattern, **kw)
+    torch.cuda.synchronize()
+    for raw, gb, n in canaries:
+        head, tail = raw[:gb], raw[gb + n:]
+        assert bool((head == 0xA5).all()) and bool((tail == 0xA5).all()), "write outside an output"
+    out = {}
+    if in_place and res is not None:
+        out["residual_out"] = as_u16(res.cpu().reshape(T, H))
+    elif rout is not None:
+        out["residual_out"] = as_u16(rout.cpu())
+    else:
+        out["residual_out"] = None
+    out["norm_out"] = None if nout is None else as_u16(nout.cpu())
+    out["quant_out"] = None if qout is None else qout.cpu().numpy()
+    out["scale_out"] = None if sout is None else sout.cpu().numpy()
+    return out
+
+
+def run_oracle(inp: dict, dtype: str, eps, wb, pattern, scale_in=None, rows=None, want_norm=True,
+               want_residual_out=True, row_list=None) -> dict:
+    ps = [as_u16(p) for p in inp["partials"]]
+    res = None if inp["residual"] is None else as_u16(inp["residual"])
+    gam = as_u16(inp["gamma"])
+    if row_list is None:
+        return oracle.fused(ps, res, gam, dtype, eps, wb, pattern, scale_in=scale_in, rows=rows,
+                            want_norm=want_norm, want_residual_out=want_residual_out)
+    out = None
+    for t in row_list:
+        out = oracle.fused(ps, res, gam, dtype, eps, wb, pattern, scale_in=scale_in,
+                           rows=(int(t), int(t) + 1), want_norm=want_norm,
+                           want_residual_out=want_residual_out, out=out)
+    return out
+
+
+def compare(gpu: dict, ref: dict, dtype: str, rows=None) -> dict:
+    """Assert the tolerances on the selected rows; return match statistics."""
+    sel = slice(None) if rows is None else rows
+    stats = {}
+    for key in ("residual_out", "norm_out"):
+        if ref.get(key) is None:
+            continue
+        assert gpu[key] is not None, key
+        d = ulp16(gpu[key][sel], ref[key][sel], dtype)
+        stats[key] = (int(d.max()) if d.size else 0, float((d == 0).mean()) if d.size else 1.0)
+        assert d.size == 0 or d.max() <= 1, (key, int(d.max()), np.argwhere(d > 1)[:5].tolist())
+    if ref.get("quant_out") is not None:
+        a, b = gpu["quant_out"][sel], ref["quant_out"][sel]
+        d = code_steps(a, b)
+        stats["quant_out"] = (int(d.max()) if d.size else 0, float((d == 0).mean()) if d.size else 1.0)
+        assert d.size == 0 or d.max() <= 1, ("quant_out", int(d.max()), np.argwhere(d > 1)[:5].tolist())
+        sat = (b & 0x7F) == 0x7E
+        assert np.array_equal(a[sat], b[sat]), "saturated codes differ"
+    if ref.get("scale_out") is not None:
+        a = gpu["scale_out"][sel].astype(np.float64)
+        b = ref["scale_out"][sel].astype(np.float64)
+        rel = np.where(b == 0, np.abs(a), np.abs(a - b) / np.where(b == 0, 1, np.abs(b)))
+        stats["scale_out"] = (float(rel.max()) if rel.size else 0.0, float((a == b).mean()) if a.size else 1.0)
+        assert rel.size == 0 or rel.max() <= SCALE_RTOL, ("scale_out", float(rel.max()))
+    return stats

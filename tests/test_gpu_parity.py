@@ -1,0 +1,279 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle.
+
+Small and ragged shapes are compared element by element; the full-size
+workloads (the W=4 8192x8192 static-FP8 prefill and the W=8 4096x7168
+per-token-FP8 Gemma workload, the shapes and launch configuration the bench
+times) on sampled rows the oracle computes one by one, every outlier row
+included.  Tolerances are in gpu_util.
+"""
+from __future__ import annotations
+
+import json
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from gpu_util import compare, run_gpu, run_oracle, to_gpu
+from reduce_residual_add_b200 import far
+from reduce_residual_add_b200.inputs import WORKLOADS, make_inputs, random_inputs
+
+pytestmark = pytest.mark.gpu
+
+LOG = os.environ.get("FAR_PARITY_LOG")
+
+
+def log(name, stats):
+    if LOG:
+        with open(LOG, "a") as f:
+            f.write(json.dumps({"case": name, **{k: v for k, v in stats.items()}}) + "\n")
+
+
+@pytest.fixture(scope="module")
+def ctx():
+    c = far.FarContext(0)
+    yield c
+    c.close()
+
+
+@pytest.fixture
+def regime(ctx):
+    """Set a regime for one test and restore automatic choice afterwards."""
+    def set_(r):
+        far.far_set_regime(ctx, r)
+    yield set_
+    far.far_set_regime(ctx, far.FAR_REGIME_AUTO)
+
+
+# (W, T, H, dtype, pattern, has_residual, weight_bias)
+SMALL = [
+    (2, 8, 64, "bf16", 0, True, 0.0),       # the small workload's shape
+    (1, 5, 8, "bf16", 0, True, 0.0),        # one pack per row
+    (3, 37, 256, "fp16", 1, True, 0.0),     # 32 packs: rows inside a warp
+    (4, 33, 264, "bf16", 2, True, 1.0),     # 33 packs: a ragged second warp
+    (5, 17, 1000, "bf16", 1, False, 0.0),   # ragged H, no residual
+    (8, 40, 4096, "bf16", 0, True, 0.0),
+    (16, 9, 2048, "fp16", 2, True, 0.0),    # the largest W
+    (2, 130, 7168, "bf16", 2, True, 1.0),
+    (4, 70, 8192, "bf16", 1, True, 0.0),
+    (3, 11, 8200, "fp16", 0, True, 0.0),    # 1025 packs: 8 per thread, ragged
+    (2, 6, 16384, "bf16", 2, True, 0.0),    # the largest H
+    (1, 64, 512, "bf16", 2, True, 0.0),     # one rank: plain add + RMSNorm
+    (7, 3, 6144, "fp16", 1, True, 1.0),
+]
+
+
+@pytest.mark.parametrize("reg", [far.FAR_REGIME_AUTO, far.FAR_REGIME_DECODE, far.FAR_REGIME_PREFILL])
+@pytest.mark.parametrize("case", SMALL, ids=lambda c: "W%d_T%d_H%d_%s_p%d_res%d_wb%g" % c)
+def test_small_shapes(ctx, regime, case, reg):
+    W, T, H, dt, pattern, has_res, wb = case
+    regime(reg)
+    inp = random_inputs(W, T, H, dtype=dt, seed=W * 1000 + T * 7 + H, has_residual=has_res)
+    eps, scale = 1e-6, 0.05
+    got = run_gpu(ctx, to_gpu(inp), eps, wb, pattern, scale_in=scale, guard=4096)
+    ref = run_oracle(inp, dt, eps, wb, pattern, scale_in=scale)
+    log("small %s reg%d" % (case, reg), compare(got, ref, dt))
+
+
+def test_small_workload_matches_golden_fixture(ctx):
+    import sys
+    sys.path.insert(0, os.path.join(os.path.dirname(__file__), "golden"))
+    from make_golden import read_fixture
+    fx = read_fixture(os.path.join(os.path.dirname(__file__), "golden", "c1_small_oracle.txt"))
+    wl = WORKLOADS["c1_small"]
+    inp = make_inputs(wl)
+    got = run_gpu(ctx, to_gpu(inp), wl.eps, wl.weight_bias, wl.pattern)
+    ref = {"residual_out": np.array(fx["residual_out"], np.uint16),
+           "norm_out": np.array(fx["norm_out"], np.uint16)}
+    log("c1 golden", compare(got, ref, "bf16"))
+
+
+@pytest.mark.parametrize("T", [1, 8, 32, 80])
+@pytest.mark.parametrize("reg", [far.FAR_REGIME_AUTO, far.FAR_REGIME_PREFILL])
+def test_decode_workload(ctx, regime, T, reg):
+    wl = WORKLOADS["c2_decode_T%d" % T]
+    regime(reg)
+    if reg == far.FAR_REGIME_AUTO:
+        assert far.far_describe_launch(ctx, T, wl.H)["regime"] == far.FAR_REGIME_DECODE
+    inp = make_inputs(wl)
+    got = run_gpu(ctx, to_gpu(inp), wl.eps, wl.weight_bias, wl.pattern, guard=256)
+    ref = run_oracle(inp, wl.dtype, wl.eps, wl.weight_bias, wl.pattern)
+    log("c2 T%d reg%d" % (T, reg), compare(got, ref, wl.dtype))
+
+
+def test_3d_input_and_row_slices(ctx):
+    """[4, 256, 2048] tensors go in as they are (the binding takes the 2-D
+    view); two 512-row slices equal the full call bit for bit."""
+    wl = WORKLOADS["c3_3d"]
+    inp = make_inputs(wl)
+    g = to_gpu(inp)
+    g3 = {"partials": [p.view(4, 256, 2048) for p in g["partials"]],
+          "residual": g["residual"].view(4, 256, 2048), "gamma": g["gamma"]}
+    full = run_gpu(ctx, g3, wl.eps, 0.0, 0)
+    ref = run_oracle(inp, "bf16", wl.eps, 0.0, 0)
+    log("c3 full", compare(full, ref, "bf16"))
+    for pattern in (0, 1, 2):
+        whole = run_gpu(ctx, g, wl.eps, 0.0, pattern, scale_in=0.05)
+        ps = g["partials"]
+        T, H = 1024, 2048
+        rout = torch.zeros(T, H, dtype=torch.bfloat16, device="cuda")
+        nout = torch.zeros_like(rout)
+        qout = torch.zeros(T, H, dtype=torch.uint8, device="cuda") if pattern else None
+        sout = torch.zeros(T, dtype=torch.float32, device="cuda") if pattern == 2 else None
+        sin = torch.tensor([0.05], device="cuda") if pattern == 1 else None
+        for b, e in ((0, 512), (512, 1024)):
+            far.far_fused_rows(ctx, b, e, ps, g["residual"], g["gamma"], wl.eps, 0.0, pattern,
+                               residual_out=rout, norm_out=nout, quant_out=qout, scale_in=sin,
+                               scale_out=sout)
+        torch.cuda.synchronize()
+        from reduce_residual_add_b200.inputs import as_u16
+        assert np.array_equal(as_u16(rout.cpu()), whole["residual_out"])
+        assert np.array_equal(as_u16(nout.cpu()), whole["norm_out"])
+        if pattern:
+            assert np.array_equal(qout.cpu().numpy(), whole["quant_out"])
+        if pattern == 2:
+            assert np.array_equal(sout.cpu().numpy(), whole["scale_out"])
+
+
+def test_row_slices_leave_other_rows_alone(ctx):
+    inp = random_inputs(3, 100, 1024, seed=5)
+    g = to_gpu(inp)
+    got = run_gpu(ctx, g, 1e-6, 0.0, 2, rows=(17, 61))
+    ref = run_oracle(inp, "bf16", 1e-6, 0.0, 2, rows=(17, 61))
+    log("rows 17..61", compare(got, ref, "bf16"))
+    # untouched rows keep the zeros run_gpu put there
+    for key in ("residual_out", "norm_out", "quant_out"):
+        assert not got[key][:17].any() and not got[key][61:].any()
+    assert not got["scale_out"][:17].any() and not got["scale_out"][61:].any()
+
+
+def _sample_rows(T, outliers, n, seed):
+    g = np.random.default_rng(seed)
+    rows = set(g.choice(T, size=n, replace=False).tolist())
+    rows |= {0, 1, T - 2, T - 1}
+    rows |= set(int(r) for r in outliers)
+    return np.array(sorted(rows))
+
+
+@pytest.mark.parametrize("with_norm", [False, True])
+def test_prefill_static_fp8_full_size(ctx, with_norm):
+    wl = WORKLOADS["c4_prefill_fp8_static"]
+    inp = make_inputs(wl)
+    g = to_gpu(inp)
+    got = run_gpu(ctx, g, wl.eps, wl.weight_bias, wl.pattern, scale_in=wl.static_scale,
+                  want_norm=with_norm)
+    rows = _sample_rows(wl.T, inp["outlier_rows"].tolist(), 160, 3)
+    ref = run_oracle(inp, wl.dtype, wl.eps, wl.weight_bias, wl.pattern,
+                     scale_in=wl.static_scale, want_norm=with_norm, row_list=rows)
+    log("c4 norm=%s" % with_norm, compare(got, ref, wl.dtype, rows=rows))
+
+
+@pytest.mark.parametrize("dt", ["bf16", "fp16"])
+def test_gemma_token_fp8_full_size(ctx, dt):
+    wl = WORKLOADS["c5_gemma_fp8_token_%s" % dt]
+    inp = make_inputs(wl)
+    got = run_gpu(ctx, to_gpu(inp), wl.eps, wl.weight_bias, wl.pattern)
+    rows = _sample_rows(wl.T, [], 160, 4)
+    ref = run_oracle(inp, dt, wl.eps, wl.weight_bias, wl.pattern, row_list=rows)
+    log("c5 %s" % dt, compare(got, ref, dt, rows=rows))
+    # properties at every row: one code at +-448 per row, scale > 0
+    q = got["quant_out"]
+    assert np.all(np.any((q & 0x7F) == 0x7E, axis=1))
+    assert np.all(got["scale_out"] > 0)
+
+
+def test_deterministic(ctx):
+    inp = random_inputs(4, 300, 7168, seed=9)
+    g = to_gpu(inp)
+    a = run_gpu(ctx, g, 1e-6, 1.0, 2)
+    b = run_gpu(ctx, g, 1e-6, 1.0, 2)
+    for k in ("residual_out", "norm_out", "quant_out", "scale_out"):
+        assert np.array_equal(a[k], b[k]), k
+
+
+def test_in_place_residual_and_side_stream(ctx):
+    inp = random_inputs(2, 50, 2048, seed=10)
+    s = torch.cuda.Stream()
+    got = run_gpu(ctx, to_gpu(inp), 1e-6, 0.0, 1, scale_in=0.1, in_place=True, stream=s)
+    ref = run_oracle(inp, "bf16", 1e-6, 0.0, 1, scale_in=0.1)
+    log("in place", compare(got, ref, "bf16"))
+
+
+def test_first_pattern_without_residual(ctx, regime):
+    for reg in (far.FAR_REGIME_DECODE, far.FAR_REGIME_PREFILL):
+        regime(reg)
+        inp = random_inputs(4, 12, 4096, seed=11, has_residual=False)
+        got = run_gpu(ctx, to_gpu(inp), 1e-6, 0.0, 2)
+        ref = run_oracle(inp, "bf16", 1e-6, 0.0, 2)
+        compare(got, ref, "bf16")
+        # norm only: no residual in, no residual out
+        got = run_gpu(ctx, to_gpu(inp), 1e-6, 0.0, 0, want_residual_out=False)
+        ref = run_oracle(inp, "bf16", 1e-6, 0.0, 0, want_residual_out=False)
+        compare(got, ref, "bf16")
+
+
+def test_zero_rows_saturation_and_nonfinite(ctx):
+    inp = random_inputs(2, 6, 1024, seed=12)
+    inp["partials"][0][1].zero_()
+    inp["partials"][1][1].zero_()
+    inp["residual"][1].zero_()                        # row 1 is all zero
+    inp["partials"][0][3, 5] = float("inf")           # row 3: inf -> NaN row
+    inp["partials"][1][4, 7] = float("nan")           # row 4: NaN row
+    for pattern, scale in ((0, None), (1, 2.0 ** -12), (2, None)):
+        got = run_gpu(ctx, to_gpu(inp), 1e-6, 0.0, pattern, scale_in=scale)
+        ref = run_oracle(inp, "bf16", 1e-6, 0.0, pattern, scale_in=scale)
+        keep = [0, 1, 2, 5] if pattern == 2 else None   # NaN rows: amax rules differ only in NaN
+        compare(got, ref, "bf16", rows=keep)
+        if pattern == 1:
+            assert np.all(got["quant_out"][0][(ref["quant_out"][0] & 0x7F) == 0x7E] & 0x7F == 0x7E)
+        if pattern == 2:
+            assert got["scale_out"][1] == 0 and not got["quant_out"][1].any()
+
+
+def test_empty_problem_and_slice_are_noops(ctx):
+    inp = random_inputs(2, 4, 64, seed=13)
+    g = to_gpu(inp)
+    rout = torch.full((4, 64), 7, dtype=torch.bfloat16, device="cuda")
+    nout = torch.full_like(rout, 7)
+    far.far_fused_rows(ctx, 2, 2, g["partials"], g["residual"], g["gamma"], 1e-6, 0.0, 0,
+                       residual_out=rout, norm_out=nout)
+    e = [torch.empty(0, 64, dtype=torch.bfloat16, device="cuda")] * 2
+    far.far_fused(ctx, e, e[0], g["gamma"], 1e-6, 0.0, 0, residual_out=e[0].clone(),
+                  norm_out=e[0].clone())
+    torch.cuda.synchronize()
+    assert bool((rout == 7).all()) and bool((nout == 7).all())
+
+
+def test_errors_are_reported_not_skipped(ctx):
+    inp = random_inputs(2, 4, 64, seed=14)
+    g = to_gpu(inp)
+    out = torch.empty(4, 64, dtype=torch.bfloat16, device="cuda")
+    bad = torch.empty(4 * 64 + 8, dtype=torch.bfloat16, device="cuda")[1:1 + 4 * 64].view(4, 64)
+    with pytest.raises(far.FarError) as e:
+        far.far_fused(ctx, g["partials"], g["residual"], g["gamma"], 1e-6, 0.0, 0,
+                      residual_out=out, norm_out=bad)
+    assert e.value.status == far.FAR_ERR_ALIGNMENT
+    with pytest.raises(far.FarError) as e:
+        far.far_fused(ctx, g["partials"], g["residual"], g["gamma"], 1e-6, 0.0, 0, residual_out=out)
+    assert e.value.status == far.FAR_ERR_INVALID_ARG
+    with pytest.raises(far.FarError) as e:
+        far.far_fused(ctx, g["partials"], g["residual"], g["gamma"], 1e-6, 0.0, 0,
+                      residual_out=out, norm_out=g["partials"][0])
+    assert e.value.status == far.FAR_ERR_INVALID_ARG
+    p12 = [torch.zeros(2, 12, dtype=torch.bfloat16, device="cuda")]
+    with pytest.raises(far.FarError) as e:
+        far.far_fused(ctx, p12, None, torch.ones(12, dtype=torch.bfloat16, device="cuda"), 1e-6,
+                      0.0, 0, norm_out=torch.empty(2, 12, dtype=torch.bfloat16, device="cuda"))
+    assert e.value.status == far.FAR_ERR_UNSUPPORTED
+
+
+def test_launch_plan(ctx):
+    d = far.far_describe_launch(ctx, 80, 4096)
+    assert d["regime"] == far.FAR_REGIME_DECODE and d["ctas_per_row"] >= 2
+    p = far.far_describe_launch(ctx, 81, 4096)
+    assert p["regime"] == far.FAR_REGIME_PREFILL
+    c4 = far.far_describe_launch(ctx, 8192, 8192)
+    assert c4["threads_per_cta"] * c4["packs_per_thread"] * 8 >= 8192
+    tiny = far.far_describe_launch(ctx, 8, 64)
+    assert tiny["regime"] == far.FAR_REGIME_PREFILL and tiny["rows_per_cta"] > 1
