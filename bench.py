@@ -86,7 +86,7 @@ class ClockSampler(threading.Thread):
         self.samples = []
         self.reasons = 0
         self.max_mhz = None
-        self._stop = threading.Event()
+        self._halt = threading.Event()
         self.ok = False
         try:
             import pynvml
@@ -109,7 +109,7 @@ class ClockSampler(threading.Thread):
         if not self.ok:
             return
         nv = self.nv
-        while not self._stop.is_set():
+        while not self._halt.is_set():
             try:
                 self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
                 try:
@@ -122,7 +122,7 @@ class ClockSampler(threading.Thread):
             time.sleep(self.period)
 
     def stop(self) -> dict:
-        self._stop.set()
+        self._halt.set()
         if self.is_alive():
             self.join(timeout=2)
         if not self.ok or not self.samples:
@@ -155,20 +155,22 @@ def barrier(world: int):
         dist.barrier()
 
 
-def max_over_ranks(x: float, world: int) -> float:
+def max_over_ranks(x: float, world: int, device="cuda") -> float:
+    """The largest value over ranks (the slowest rank's time)."""
     if world == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
 
 
-def sum_over_ranks(x: float, world: int) -> float:
+def sum_over_ranks(x: float, world: int, device="cuda") -> float:
+    """The total over ranks (bytes and rows of every rank)."""
     if world == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.SUM)
     return float(t.item())
 
@@ -236,6 +238,8 @@ class Case:
         for _ in range(warmup):
             self.step()
         torch.cuda.synchronize()
+        if k == 0:
+            return 0.0, 0.0
         ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
               for _ in range(k)] if per_launch else None
         first, last = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -262,13 +266,15 @@ def graph_time(case: Case, launches: int, reps: int = 5) -> float:
     with torch.cuda.graph(g, stream=s):
         for _ in range(launches):
             case.step()
-    g.replay()
+    with torch.cuda.stream(s):          # replay() launches on the current stream
+        g.replay()
     torch.cuda.synchronize()
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a.record(s)
-    for _ in range(reps):
-        g.replay()
-    b.record(s)
+    with torch.cuda.stream(s):
+        a.record(s)
+        for _ in range(reps):
+            g.replay()
+        b.record(s)
     torch.cuda.synchronize()
     t = a.elapsed_time(b) / 1e3 / (reps * launches)
     del g
@@ -347,6 +353,8 @@ def run_far(args, world, rank, local):
     device = torch.device("cuda", local)
     torch.cuda.set_device(device)
     wl = WORKLOADS[args.workload]
+    if args.rows:
+        wl = wl.with_(T=args.rows, outlier_frac=wl.outlier_frac)
     # each rank owns an independent batch of rows (seed offset by rank)
     inp = make_inputs(wl.with_(seed=wl.seed + 1000 * rank))
     stream = torch.cuda.Stream(device=device)
@@ -488,6 +496,8 @@ def main():
     ap.add_argument("--impl", choices=["far", "reference"], default="far")
     ap.add_argument("--workload", default=HEADLINE, choices=sorted(WORKLOADS))
     ap.add_argument("--with-norm", action="store_true", help="also write norm_out")
+    ap.add_argument("--rows", type=int, default=0,
+                    help="override the workload's row count (smaller cases for profiling)")
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--no-extras", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")

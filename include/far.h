@@ -98,7 +98,10 @@ typedef enum {
 /* Opaque per-device context: caches the SM count, the compute capability
  * and the tuning knobs (read once from the environment in far_create:
  * FAR_DECODE_MAX_ROWS, FAR_FORCE_REGIME=decode|prefill, FAR_DECODE_CLUSTER,
- * FAR_PREFILL_THREADS). */
+ * FAR_PREFILL_THREADS, FAR_PREFILL_KERNEL=1 ring | 0 direct,
+ * FAR_RING_CTAS_PER_SM=1..4 (default 2), FAR_RING_THREADS: consumer threads
+ * per ring CTA, at most 512 (default 256), FAR_RING_SLOTS: row-segment slots
+ * per ring CTA (2..32; default: about 72 KiB of segments, as many as fit)). */
 typedef struct far_ctx far_ctx;
 
 /* How one call would be launched (see far_describe_launch). */
@@ -109,6 +112,8 @@ typedef struct {
     int threads_per_cta;
     int packs_per_thread; /* 16-byte packs of one row held by one thread */
     int64_t grid_ctas;    /* CTAs of the launch                       */
+    int kernel;           /* prefill: 1 = TMA bulk-copy ring, 0 = direct loads */
+    int ring_slots;       /* ring: shared-memory slots of one row segment */
 } far_launch_info;
 
 /* Create a context for CUDA device `device` (its ordinal).  Fails with
@@ -186,6 +191,14 @@ far_status far_set_regime(far_ctx *ctx, far_regime regime, int decode_max_rows);
 /* Fill `info` with the launch geometry a call on `rows` rows would use. */
 far_status far_describe_launch(const far_ctx *ctx, int64_t rows, int64_t H,
                                far_dtype dtype, far_launch_info *info);
+
+/* Wait for `stream`, then read and clear the device-side error word of
+ * ctx's device.  FAR_ERR_TIMEOUT: a bounded wait inside a kernel launched
+ * since the last far_check gave up (after 2 s), and the outputs of those
+ * calls are not valid; the kernel still ended and the CUDA context stays
+ * usable.  FAR_OK otherwise.  Synchronises `stream`; not for use during
+ * stream capture. */
+far_status far_check(far_ctx *ctx, void *stream);
 
 /* Static text for a status code. */
 const char *far_status_string(far_status s);

@@ -6,6 +6,7 @@
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
+#include <mutex>
 #include <new>
 
 #include <cuda_runtime.h>
@@ -22,6 +23,14 @@ struct far_ctx {
   int force_regime;     // FAR_REGIME_*
   int decode_cluster;   // preferred CTAs per row in decode
   int prefill_threads;  // target threads per row in prefill
+  int prefill_kernel;   // 1 = TMA bulk-copy ring (default), 0 = direct loads
+  int ring_ctas_per_sm; // persistent ring CTAs per SM wanted (1..4)
+  int ring_threads;     // target consumer threads of a ring CTA
+  int ring_slots_max;   // at most this many ring slots
+  // ring CTAs per SM the occupancy calculator allows, per (dtype, packs):
+  // 0 = not asked yet, -1 = cannot run
+  std::mutex occ_mu;
+  int ring_occ[2][far::kMaxH / far::kPackElems + 1];
 };
 
 namespace {
@@ -105,7 +114,56 @@ void plan_decode(int packs, int cluster_pref, far::Launch* l) {
   l->rows_per_cta = 1;
 }
 
-far::Launch plan(const far_ctx* ctx, int64_t rows, int64_t H) {
+// Ring geometry: consumers = the fewest packs per thread (1, 2, 4, 8) that
+// keep within ring_threads, plus one producer warp; as many row-segment
+// slots (at most 32) as fit in a 1/ring_ctas_per_sm share of the SM's
+// 228 KiB of shared memory (less the 1 KiB the system keeps per CTA); a
+// persistent grid of sm_count x (the CTAs per SM the occupancy calculator
+// confirms, at most ring_ctas_per_sm), fewer for fewer rows.  Returns false
+// (the direct kernel runs) when fewer than two slots fit or the
+// configuration cannot be resident.
+bool plan_ring(const far_ctx* ctx, int packs, int64_t rows, int dtype, far::Launch* l) {
+  if (packs <= 32) return false;
+  int vpt = 1;
+  while (vpt < 8 && (packs + vpt - 1) / vpt > ctx->ring_threads) vpt *= 2;
+  const int tpr = (((packs + vpt - 1) / vpt) + 31) / 32 * 32;
+  if (tpr > far::kRingMaxConsumers) return false;
+  const int seg = packs * 16;
+  const int n_req = ctx->ring_ctas_per_sm;
+  int per_cta = 228 * 1024 / n_req - 1024;
+  if (per_cta > far::kRingSmemMax) per_cta = far::kRingSmemMax;
+  // header, gamma (one segment's worth of bytes), slots: about 72 KiB of
+  // segments in flight per CTA measured best (4 slots at H=8192, 5 at 7168)
+  int nslot = ctx->ring_slots_max > 0 ? ctx->ring_slots_max : 72 * 1024 / seg;
+  if (nslot > 32) nslot = 32;
+  while (nslot >= 2 && far::ring_header_bytes(nslot) + (nslot + 1) * seg > per_cta) --nslot;
+  if (nslot < 2) return false;
+  const int smem = far::ring_header_bytes(nslot) + (nslot + 1) * seg;
+  int occ;
+  {
+    std::lock_guard<std::mutex> lock(const_cast<far_ctx*>(ctx)->occ_mu);
+    int& cached = const_cast<far_ctx*>(ctx)->ring_occ[dtype][packs];
+    if (cached == 0) {
+      const int n = far::ring_occupancy(dtype, vpt, tpr + 32, smem);
+      cached = n > 0 ? n : -1;
+    }
+    occ = cached;
+  }
+  if (occ < 1) return false;
+  if (occ > n_req) occ = n_req;
+  l->kernel = 1;
+  l->vpt = vpt;
+  l->tpr = tpr;
+  l->rows_per_cta = 1;
+  l->nslot = nslot;
+  l->smem_bytes = smem;
+  l->threads = tpr + 32;
+  const int64_t ctas = static_cast<int64_t>(ctx->sm_count) * occ;
+  l->grid = rows < ctas ? rows : ctas;
+  return true;
+}
+
+far::Launch plan(const far_ctx* ctx, int64_t rows, int64_t H, int dtype) {
   const int packs = static_cast<int>(H / far::kPackElems);
   far::Launch l{};
   bool decode;
@@ -121,6 +179,7 @@ far::Launch plan(const far_ctx* ctx, int64_t rows, int64_t H) {
   } else {
     plan_prefill(packs, ctx->prefill_threads, &l);
     l.grid = (rows + l.rows_per_cta - 1) / l.rows_per_cta;
+    if (ctx->prefill_kernel == 1) plan_ring(ctx, packs, rows, dtype, &l);
   }
   return l;
 }
@@ -153,16 +212,19 @@ far_status far_create(far_ctx** ctx, int device) {
   cudaError_t e = cudaGetDeviceCount(&n);
   if (e != cudaSuccess) return cuda_fail(e, "cudaGetDeviceCount");
   if (device < 0 || device >= n) return FAR_ERR_INVALID_ARG;
-  far_ctx c{};
+  far_ctx* out = new (std::nothrow) far_ctx();
+  if (out == nullptr) return FAR_ERR_INTERNAL;
+  far_ctx& c = *out;
   c.device = device;
   if ((e = cudaDeviceGetAttribute(&c.sm_count, cudaDevAttrMultiProcessorCount, device)) != cudaSuccess ||
       (e = cudaDeviceGetAttribute(&c.cc_major, cudaDevAttrComputeCapabilityMajor, device)) != cudaSuccess ||
       (e = cudaDeviceGetAttribute(&c.cc_minor, cudaDevAttrComputeCapabilityMinor, device)) != cudaSuccess)
-    return cuda_fail(e, "cudaDeviceGetAttribute");
+    { delete out; return cuda_fail(e, "cudaDeviceGetAttribute"); }
   if (c.cc_major != 10 || c.cc_minor != 0) {
     std::snprintf(g_last_error, sizeof(g_last_error),
                   "device %d has compute capability %d.%d; this library is built for sm_100a only",
                   device, c.cc_major, c.cc_minor);
+    delete out;
     return FAR_ERR_UNSUPPORTED;
   }
   c.decode_max_rows = env_int("FAR_DECODE_MAX_ROWS", 80);
@@ -170,6 +232,16 @@ far_status far_create(far_ctx** ctx, int device) {
   c.prefill_threads = env_int("FAR_PREFILL_THREADS", 256);
   if (c.prefill_threads < 32) c.prefill_threads = 32;
   if (c.prefill_threads > far::kMaxThreads) c.prefill_threads = far::kMaxThreads;
+  c.prefill_kernel = env_int("FAR_PREFILL_KERNEL", 1) != 0 ? 1 : 0;
+  c.ring_ctas_per_sm = env_int("FAR_RING_CTAS_PER_SM", 2);
+  if (c.ring_ctas_per_sm < 1) c.ring_ctas_per_sm = 1;
+  if (c.ring_ctas_per_sm > 4) c.ring_ctas_per_sm = 4;
+  c.ring_threads = env_int("FAR_RING_THREADS", 256);
+  c.ring_slots_max = env_int("FAR_RING_SLOTS", 0);  // 0: by the 72 KiB rule
+  if (c.ring_slots_max < 0) c.ring_slots_max = 0;
+  if (c.ring_slots_max > 32) c.ring_slots_max = 32;
+  if (c.ring_threads < 32) c.ring_threads = 32;
+  if (c.ring_threads > far::kRingMaxConsumers) c.ring_threads = far::kRingMaxConsumers;
   c.force_regime = FAR_REGIME_AUTO;
   if (const char* f = std::getenv("FAR_FORCE_REGIME")) {
     if (std::strcmp(f, "decode") == 0) c.force_regime = FAR_REGIME_DECODE;
@@ -177,14 +249,14 @@ far_status far_create(far_ctx** ctx, int device) {
   }
 
   int prev = -1;
-  if ((e = cudaGetDevice(&prev)) != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
-  if (prev != device && (e = cudaSetDevice(device)) != cudaSuccess) return cuda_fail(e, "cudaSetDevice");
+  if ((e = cudaGetDevice(&prev)) != cudaSuccess) { delete out; return cuda_fail(e, "cudaGetDevice"); }
+  if (prev != device && (e = cudaSetDevice(device)) != cudaSuccess) {
+    delete out;
+    return cuda_fail(e, "cudaSetDevice");
+  }
   e = far::configure_kernels();
   if (prev != device) cudaSetDevice(prev);
-  if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
-
-  far_ctx* out = new (std::nothrow) far_ctx(c);
-  if (out == nullptr) return FAR_ERR_INTERNAL;
+  if (e != cudaSuccess) { delete out; return cuda_fail(e, "cudaFuncSetAttribute"); }
   *ctx = out;
   return FAR_OK;
 }
@@ -208,13 +280,43 @@ far_status far_describe_launch(const far_ctx* ctx, int64_t rows, int64_t H, far_
   if (ctx == nullptr || info == nullptr || rows < 0) return FAR_ERR_INVALID_ARG;
   if (dtype != FAR_BF16 && dtype != FAR_FP16) return FAR_ERR_INVALID_ARG;
   if (H <= 0 || H % far::kPackElems != 0 || H > far::kMaxH) return FAR_ERR_UNSUPPORTED;
-  const far::Launch l = plan(ctx, rows, H);
+  int prev = -1;
+  cudaError_t e = cudaGetDevice(&prev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (prev != ctx->device && (e = cudaSetDevice(ctx->device)) != cudaSuccess)
+    return cuda_fail(e, "cudaSetDevice");
+  const far::Launch l = plan(ctx, rows, H, dtype);
+  if (prev != ctx->device) cudaSetDevice(prev);
   info->regime = l.regime;
   info->ctas_per_row = l.cluster;
   info->rows_per_cta = l.rows_per_cta;
   info->threads_per_cta = l.threads;
   info->packs_per_thread = l.vpt;
   info->grid_ctas = l.grid;
+  info->kernel = l.kernel;
+  info->ring_slots = l.nslot;
+  return FAR_OK;
+}
+
+far_status far_check(far_ctx* ctx, void* stream) {
+  if (ctx == nullptr) return FAR_ERR_INVALID_ARG;
+  int prev = -1;
+  cudaError_t e = cudaGetDevice(&prev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (prev != ctx->device && (e = cudaSetDevice(ctx->device)) != cudaSuccess)
+    return cuda_fail(e, "cudaSetDevice");
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  unsigned word = 0;
+  e = far::read_error_word(&word, s);
+  if (e == cudaSuccess && word != 0) e = far::clear_error_word(s);
+  if (prev != ctx->device) cudaSetDevice(prev);
+  if (e != cudaSuccess) return cuda_fail(e, "far_check");
+  if (word != 0) {
+    std::snprintf(g_last_error, sizeof(g_last_error),
+                  "a bounded wait inside a kernel gave up (flags 0x%x); outputs of the "
+                  "calls since the last far_check are not valid", word);
+    return FAR_ERR_TIMEOUT;
+  }
   return FAR_OK;
 }
 
@@ -320,7 +422,7 @@ far_status far_fused_rows(far_ctx* ctx, int64_t row_begin, int64_t row_end,
 
   // grid.y (decode) and grid.x (prefill) bound the rows of one launch
   const int64_t rows = row_end - row_begin;
-  const far::Launch whole = plan(ctx, rows, H);
+  const far::Launch whole = plan(ctx, rows, H, dtype);
   const int64_t max_rows = whole.regime == FAR_REGIME_DECODE
                                ? 65535
                                : static_cast<int64_t>(0x7fffffff) * whole.rows_per_cta;
@@ -328,12 +430,20 @@ far_status far_fused_rows(far_ctx* ctx, int64_t row_begin, int64_t row_end,
   for (int64_t b = row_begin; b < row_end && e == cudaSuccess; b += max_rows) {
     const int64_t n = (row_end - b < max_rows) ? (row_end - b) : max_rows;
     far::Launch l = whole;
-    l.grid = (whole.regime == FAR_REGIME_DECODE) ? n * l.cluster
-                                                 : (n + l.rows_per_cta - 1) / l.rows_per_cta;
+    if (whole.regime == FAR_REGIME_DECODE)
+      l.grid = n * l.cluster;
+    else if (whole.kernel == 1)
+      l.grid = (n < whole.grid) ? n : whole.grid;
+    else
+      l.grid = (n + l.rows_per_cta - 1) / l.rows_per_cta;
     p.row_begin = b;
     p.row_end = b + n;
-    e = (l.regime == FAR_REGIME_DECODE) ? far::launch_decode(p, dtype, l, s)
-                                        : far::launch_prefill(p, dtype, l, s);
+    if (l.regime == FAR_REGIME_DECODE)
+      e = far::launch_decode(p, dtype, l, s);
+    else if (l.kernel == 1)
+      e = far::launch_ring(p, dtype, l, s);
+    else
+      e = far::launch_prefill(p, dtype, l, s);
   }
   if (prev != ctx->device) cudaSetDevice(prev);
   if (e != cudaSuccess) return cuda_fail(e, "kernel launch");

@@ -10,7 +10,9 @@ namespace far {
 constexpr int kMaxW = 16;        // partial buffers per call
 constexpr int kMaxH = 16384;     // longest row held in registers
 constexpr int kPackElems = 8;    // 2-byte elements per 16-byte pack
-constexpr int kMaxThreads = 256; // threads per CTA, both regimes
+constexpr int kMaxThreads = 256; // threads per row (CTA) in every kernel
+constexpr int kRingSmemMax = 227 * 1024;  // dynamic shared memory of one ring CTA
+constexpr int kRingMaxConsumers = 512;    // consumer threads of one ring CTA
 
 enum Dtype : int { kBf16 = 0, kFp16 = 1 };
 enum Pattern : int { kNormOnly = 0, kFp8Static = 1, kFp8Token = 2 };
@@ -39,18 +41,34 @@ struct Params {
 // Geometry of one launch, chosen on the host.
 struct Launch {
   int regime;           // 1 decode (cluster per row), 2 prefill
+  int kernel;           // prefill: 0 direct loads, 1 TMA bulk-copy ring
   int cluster;          // CTAs per row (decode)
   int vpt;              // 16-byte packs per thread
   int tpr;              // threads per row (prefill) / per CTA (decode)
   int rows_per_cta;     // prefill
   int threads;          // threads per CTA
   int64_t grid;         // CTAs
+  int nslot;            // ring: shared-memory slots of one row segment each
+  int smem_bytes;       // ring: dynamic shared memory per CTA
 };
 
 // Enqueue one kernel on `stream`.  Returns the launch error (cudaSuccess if
 // the launch was accepted).
 cudaError_t launch_prefill(const Params& p, int dtype, const Launch& l, cudaStream_t stream);
 cudaError_t launch_decode(const Params& p, int dtype, const Launch& l, cudaStream_t stream);
+cudaError_t launch_ring(const Params& p, int dtype, const Launch& l, cudaStream_t stream);
+
+// Bytes of the ring kernel's shared memory before its first slot.
+int ring_header_bytes(int nslot);
+
+// Resident ring CTAs per SM for this configuration on the current device
+// (0 if it cannot run).
+int ring_occupancy(int dtype, int vpt, int threads, int smem_bytes);
+
+// The device error word of the current device (see far_check): read it
+// after the work on `stream`, or clear it.  Both synchronise `stream`.
+cudaError_t read_error_word(unsigned* out, cudaStream_t stream);
+cudaError_t clear_error_word(cudaStream_t stream);
 
 // One-time per-device set-up of kernel attributes (non-portable cluster
 // sizes).  Call with the device current.

@@ -34,6 +34,20 @@ namespace cg = cooperative_groups;
 namespace far {
 namespace {
 
+// Shared-memory layout of the ring kernel: nslot "full" and nslot "empty"
+// mbarriers (8 bytes each), a RingHeader, then from a 128-byte boundary
+// gamma (H*2 bytes, loaded once per CTA) and the nslot slots.
+struct RingHeader {
+  float red[2][2][32];   // [row parity][0 = sum of squares, 1 = amax][warp]
+  int abort;             // set when any wait of the CTA gave up
+  int producer_done;     // set by the producer when it stops issuing
+  long long issued;      // bulk copies the producer issued
+};
+
+__host__ __device__ constexpr int ring_offset(int nslot) {
+  return (16 * nslot + static_cast<int>(sizeof(RingHeader)) + 127) / 128 * 128;
+}
+
 // ---------------------------------------------------------------------------
 // 16-byte packs of eight 2-byte elements
 // ---------------------------------------------------------------------------
@@ -87,6 +101,17 @@ __device__ __forceinline__ uint32_t e4m3x4(float a, float b, float c, float d) {
   return lo | (hi << 16);
 }
 
+// a / b given inv_b = RN(1/b): q0 = RN(a * inv_b), the exact remainder
+// r = a - b*q0 by one FMA, then q0 + r*inv_b rounded once (Markstein's
+// FMA-based correction; P. Markstein, "IA-64 and Elementary Functions",
+// 2000).  Within one ulp of a/b for normal operands and the correctly
+// rounded quotient in all but rare cases, in three instructions and no branch.
+__device__ __forceinline__ float div_by(float a, float b, float inv_b) {
+  const float q0 = a * inv_b;
+  const float r = fmaf(-q0, b, a);
+  return fmaf(r, inv_b, q0);
+}
+
 // ---------------------------------------------------------------------------
 // memory access
 // ---------------------------------------------------------------------------
@@ -109,6 +134,81 @@ __device__ __forceinline__ uint4 ld_once_coherent(const uint4* p) {
       : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
       : "l"(p));
   return r;
+}
+
+// ---------------------------------------------------------------------------
+// TMA bulk copies and mbarriers (PTX ISA: cp.async.bulk, mbarrier)
+// ---------------------------------------------------------------------------
+
+// Device-side error word of this library, one per device: bit 0 = a consumer
+// gave up waiting for a bulk copy, bit 1 = the producer gave up waiting for
+// a free slot.  Read and cleared by far_check().
+__device__ unsigned int g_far_error = 0u;
+
+constexpr unsigned kErrWaitFull = 1u;
+constexpr unsigned kErrWaitEmpty = 2u;
+constexpr uint64_t kWaitLimitNs = 2000000000ull;  // one wait gives up after 2 s
+
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ uint64_t global_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)), "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t done;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(done)
+      : "r"(smem_addr(bar)), "r"(parity)
+      : "memory");
+  return done != 0u;
+}
+
+// Wait for the phase of parity `parity` to complete.  Gives up after
+// kWaitLimitNs, or as soon as *abort is set (when abort is non-null);
+// returns false then.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const volatile int* abort) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_ns();
+  for (;;) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (abort != nullptr && *abort) return false;
+    if (global_ns() - t0 > kWaitLimitNs) return false;
+  }
+}
+
+// One 1-D bulk copy global -> this CTA's shared memory, completing `bytes`
+// transactions on `bar`.  Both addresses 16-byte aligned, bytes % 16 == 0.
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+      ::"r"(smem_addr(dst)), "l"(src), "r"(bytes), "r"(smem_addr(bar))
+      : "memory");
+}
+
+// Barrier over the first `nthreads` threads of the CTA (the consumer warps).
+__device__ __forceinline__ void consumer_bar(int nthreads) {
+  asm volatile("bar.sync 1, %0;" ::"r"(nthreads) : "memory");
 }
 
 // ---------------------------------------------------------------------------
@@ -178,8 +278,130 @@ struct ClusterRed {
   }
 };
 
+// A row over the consumer warps of the ring kernel (a named barrier that
+// the producer warp does not join).  `buf` alternates between two halves by
+// row parity: a warp can only rewrite a half after every consumer passed the
+// next row's barrier, i.e. after everyone finished reading it.
+struct RingRed {
+  float* buf;     // [2][32]: 0 = sum of squares, 1 = amax
+  int nthreads;   // consumer threads
+  __device__ float reduce(float v, int which, bool is_max) const {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = nthreads >> 5;
+    v = is_max ? group_max(v, 32) : group_sum(v, 32);
+    if (lane == 0) buf[which * 32 + warp] = v;
+    consumer_bar(nthreads);
+    float t = lane < nw ? buf[which * 32 + lane] : 0.f;
+    return is_max ? group_max(t, 32) : group_sum(t, 32);
+  }
+  __device__ float sum(float v) const { return reduce(v, 0, false); }
+  __device__ float max(float v) const { return reduce(v, 1, true); }
+  __device__ bool leader() const { return threadIdx.x == 0; }
+};
+
 // ---------------------------------------------------------------------------
-// one row (or one slice of it): packs j = j0 + k*jstride, k < VPT, j < jend
+// the second half of a row: y (the fp32 sum of partials and residual) is in
+// registers; write the new residual, reduce, normalise, quantise.
+// This thread owns packs j = j0 + k*jstride (k < VPT) where ok[k].
+// ---------------------------------------------------------------------------
+
+template <class DT, int VPT, class Red>
+__device__ __forceinline__ void finish_row(const Params& p, int64_t row, bool row_ok, int j0,
+                                           int jstride, const bool (&ok)[VPT],
+                                           float (&y)[VPT][8], const Red& red,
+                                           const uint4* gamma_smem = nullptr) {
+  const int64_t rbase = row * static_cast<int64_t>(p.packs);  // first pack of the row
+  if (p.residual_out != nullptr) {
+#pragma unroll
+    for (int k = 0; k < VPT; ++k)
+      if (ok[k]) static_cast<uint4*>(p.residual_out)[rbase + j0 + k * jstride] = pack8<DT>(y[k]);
+  }
+
+  // a3: mean of squares; pairwise inside the thread, butterflies above it.
+  float sq[VPT];
+#pragma unroll
+  for (int k = 0; k < VPT; ++k) {
+    const float a = y[k][0] * y[k][0] + y[k][1] * y[k][1];
+    const float b = y[k][2] * y[k][2] + y[k][3] * y[k][3];
+    const float c = y[k][4] * y[k][4] + y[k][5] * y[k][5];
+    const float d = y[k][6] * y[k][6] + y[k][7] * y[k][7];
+    sq[k] = (a + b) + (c + d);
+  }
+#pragma unroll
+  for (int w = 1; w < VPT; w <<= 1)
+#pragma unroll
+    for (int k = 0; k + w < VPT; k += 2 * w) sq[k] += sq[k + w];
+  const float ss = red.sum(sq[0]);
+  const float ms = __fdiv_rn(ss, static_cast<float>(p.H));
+  const float rinv = __frsqrt_rn(ms + p.eps);
+
+  // a4: o = y * rinv * (gamma + weight_bias); a5: FP8 codes.
+  const bool fp8_static = p.pattern == kFp8Static;
+  const bool fp8_token = p.pattern == kFp8Token;
+  const float s_static = fp8_static ? __ldg(p.scale_in) : 1.f;
+  const float inv_static = __frcp_rn(s_static);
+  // outside the normal range of the reciprocal, divide exactly instead
+  const bool exact_static = !(fabsf(inv_static) < 3.0e38f && fabsf(s_static) > 1.0e-37f);
+  float amax = 0.f;
+#pragma unroll
+  for (int k = 0; k < VPT; ++k) {
+    if (!ok[k]) continue;
+    const int64_t pk = rbase + j0 + k * jstride;
+    float g[8];
+    if (gamma_smem != nullptr)
+      DT::unpack(gamma_smem[j0 + k * jstride], g);
+    else
+      DT::unpack(__ldg(static_cast<const uint4*>(p.gamma) + j0 + k * jstride), g);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) y[k][i] = (y[k][i] * rinv) * (g[i] + p.weight_bias);
+    if (p.norm_out != nullptr) static_cast<uint4*>(p.norm_out)[pk] = pack8<DT>(y[k]);
+    if (fp8_static) {
+      float q[8];
+      if (exact_static) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) q[i] = __fdiv_rn(y[k][i], s_static);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) q[i] = div_by(y[k][i], s_static, inv_static);
+      }
+      reinterpret_cast<uint2*>(p.quant_out)[pk] =
+          make_uint2(e4m3x4(q[0], q[1], q[2], q[3]), e4m3x4(q[4], q[5], q[6], q[7]));
+    }
+    if (fp8_token) {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(y[k][i]));
+    }
+  }
+
+  if (fp8_token) {
+    const float rowmax = red.max(amax);
+    const float scale = __fdiv_rn(rowmax, 448.f);
+    if (row_ok && red.leader()) p.scale_out[row] = scale;
+    const float inv = __frcp_rn(scale);
+    const bool exact = !(inv < 3.0e38f && scale > 1.0e-37f);  // row-uniform
+#pragma unroll
+    for (int k = 0; k < VPT; ++k) {
+      if (!ok[k]) continue;
+      const int64_t pk = rbase + j0 + k * jstride;
+      uint2 codes = make_uint2(0u, 0u);
+      if (scale != 0.f) {
+        float q[8];
+        if (exact) {
+#pragma unroll
+          for (int i = 0; i < 8; ++i) q[i] = __fdiv_rn(y[k][i], scale);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 8; ++i) q[i] = div_by(y[k][i], scale, inv);
+        }
+        codes = make_uint2(e4m3x4(q[0], q[1], q[2], q[3]), e4m3x4(q[4], q[5], q[6], q[7]));
+      }
+      reinterpret_cast<uint2*>(p.quant_out)[pk] = codes;
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// one row (or one slice of it) straight from global memory into registers:
+// packs j = j0 + k*jstride, k < VPT, j < jend
 // ---------------------------------------------------------------------------
 
 template <class DT, int VPT, class Red>
@@ -219,7 +441,7 @@ __device__ __forceinline__ void fused_row(const Params& p, int64_t row, bool row
     }
   }
 
-  // a2: add the residual and write the new residual.
+  // a2: add the residual.
   if (p.residual != nullptr) {
     uint4 v[VPT];
 #pragma unroll
@@ -235,75 +457,7 @@ __device__ __forceinline__ void fused_row(const Params& p, int64_t row, bool row
       for (int i = 0; i < 8; ++i) y[k][i] += f[i];
     }
   }
-  if (p.residual_out != nullptr) {
-#pragma unroll
-    for (int k = 0; k < VPT; ++k)
-      if (ok[k]) static_cast<uint4*>(p.residual_out)[rbase + j0 + k * jstride] = pack8<DT>(y[k]);
-  }
-
-  // a3: mean of squares; pairwise inside the thread, butterflies above it.
-  float sq[VPT];
-#pragma unroll
-  for (int k = 0; k < VPT; ++k) {
-    const float a = y[k][0] * y[k][0] + y[k][1] * y[k][1];
-    const float b = y[k][2] * y[k][2] + y[k][3] * y[k][3];
-    const float c = y[k][4] * y[k][4] + y[k][5] * y[k][5];
-    const float d = y[k][6] * y[k][6] + y[k][7] * y[k][7];
-    sq[k] = (a + b) + (c + d);
-  }
-#pragma unroll
-  for (int w = 1; w < VPT; w <<= 1)
-#pragma unroll
-    for (int k = 0; k + w < VPT; k += 2 * w) sq[k] += sq[k + w];
-  const float ss = red.sum(sq[0]);
-  const float ms = __fdiv_rn(ss, static_cast<float>(p.H));
-  const float rinv = __frsqrt_rn(ms + p.eps);
-
-  // a4: o = y * rinv * (gamma + weight_bias); a5: FP8 codes.
-  const bool fp8_static = p.pattern == kFp8Static;
-  const bool fp8_token = p.pattern == kFp8Token;
-  const float s_static = fp8_static ? __ldg(p.scale_in) : 1.f;
-  float amax = 0.f;
-#pragma unroll
-  for (int k = 0; k < VPT; ++k) {
-    if (!ok[k]) continue;
-    const int64_t pk = rbase + j0 + k * jstride;
-    float g[8];
-    DT::unpack(__ldg(static_cast<const uint4*>(p.gamma) + j0 + k * jstride), g);
-#pragma unroll
-    for (int i = 0; i < 8; ++i) y[k][i] = (y[k][i] * rinv) * (g[i] + p.weight_bias);
-    if (p.norm_out != nullptr) static_cast<uint4*>(p.norm_out)[pk] = pack8<DT>(y[k]);
-    if (fp8_static) {
-      float q[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) q[i] = __fdiv_rn(y[k][i], s_static);
-      reinterpret_cast<uint2*>(p.quant_out)[pk] =
-          make_uint2(e4m3x4(q[0], q[1], q[2], q[3]), e4m3x4(q[4], q[5], q[6], q[7]));
-    }
-    if (fp8_token) {
-#pragma unroll
-      for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(y[k][i]));
-    }
-  }
-
-  if (fp8_token) {
-    const float rowmax = red.max(amax);
-    const float scale = __fdiv_rn(rowmax, 448.f);
-    if (row_ok && red.leader()) p.scale_out[row] = scale;
-#pragma unroll
-    for (int k = 0; k < VPT; ++k) {
-      if (!ok[k]) continue;
-      const int64_t pk = rbase + j0 + k * jstride;
-      uint2 codes = make_uint2(0u, 0u);
-      if (scale != 0.f) {
-        float q[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) q[i] = __fdiv_rn(y[k][i], scale);
-        codes = make_uint2(e4m3x4(q[0], q[1], q[2], q[3]), e4m3x4(q[4], q[5], q[6], q[7]));
-      }
-      reinterpret_cast<uint2*>(p.quant_out)[pk] = codes;
-    }
-  }
+  finish_row<DT, VPT>(p, row, row_ok, j0, jstride, ok, y, red);
 }
 
 // ---------------------------------------------------------------------------
@@ -346,6 +500,134 @@ far_decode_kernel(const Params p) {
   cl.sync();  // keep this CTA's shared memory alive until every peer has read it
 }
 
+// Prefill through the TMA engine: a persistent CTA per SM (or two) walks
+// rows blockIdx.x, blockIdx.x + gridDim.x, ...  Its last warp is the producer:
+// one thread streams each row's W partial segments and its residual segment
+// (H*2 bytes each) with cp.async.bulk into a ring of `nslot` shared-memory
+// slots, running up to nslot segments ahead.  The first `ncons` threads are
+// consumers: they wait for a slot (mbarrier, transaction count), fold its
+// packs into their fp32 row registers in the same order as the direct path
+// (partials 0..W-1, then the residual), release the slot, and finish the row
+// from registers.  The bytes in flight live in shared memory, not in
+// registers, so each SM keeps ~100-200 KB of loads outstanding.
+//
+// Every wait is bounded (kWaitLimitNs); a wait that gives up sets the
+// device error word and the CTA's abort flag, after which no wait blocks,
+// the producer stops, and thread 0 waits (bounded) for the copies already
+// issued before the CTA exits.
+template <class DT, int VPT>
+__global__ void __launch_bounds__(kRingMaxConsumers + 32, 1)
+far_ring_kernel(const Params p, int nslot, int ncons) {
+  extern __shared__ __align__(128) unsigned char smem[];
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem);
+  uint64_t* empty = full + nslot;
+  RingHeader* hdr = reinterpret_cast<RingHeader*>(empty + nslot);
+  volatile int* abort_flag = &hdr->abort;
+  volatile int* producer_done = &hdr->producer_done;
+  volatile long long* issued_count = &hdr->issued;
+  const uint32_t seg_bytes = static_cast<uint32_t>(p.H) * 2u;
+  uint4* gamma_s = reinterpret_cast<uint4*>(smem + ring_offset(nslot));
+  unsigned char* ring = smem + ring_offset(nslot) + seg_bytes;
+  const int S = p.W + (p.residual != nullptr ? 1 : 0);
+  const int64_t nrows = p.row_end - p.row_begin;
+  const int64_t my_rows = (nrows - blockIdx.x + gridDim.x - 1) / gridDim.x;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < nslot; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], static_cast<uint32_t>(ncons / 32));
+    }
+    *abort_flag = 0;
+    *producer_done = 0;
+    *issued_count = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  // gamma: read once per CTA, kept in shared memory for every row
+  for (int j = threadIdx.x; j < p.packs; j += blockDim.x)
+    gamma_s[j] = __ldg(static_cast<const uint4*>(p.gamma) + j);
+  __syncthreads();
+
+  if (threadIdx.x >= ncons) {
+    // producer warp: one thread issues, the rest of the warp is idle
+    if (threadIdx.x == ncons) {
+      const int64_t nseg = my_rows * S;
+      int64_t issued = 0;
+      for (int64_t g = 0; g < nseg; ++g) {
+        if (*abort_flag) break;
+        const int slot = static_cast<int>(g % nslot);
+        const uint32_t round = static_cast<uint32_t>(g / nslot);
+        if (!mbar_wait(&empty[slot], (round & 1u) ^ 1u, abort_flag)) {
+          if (!*abort_flag) atomicOr(&g_far_error, kErrWaitEmpty);
+          *abort_flag = 1;
+          break;
+        }
+        const int64_t row = p.row_begin + blockIdx.x + (g / S) * gridDim.x;
+        const int k = static_cast<int>(g % S);
+        const void* base = (k < p.W) ? p.partials[k] : p.residual;
+        const unsigned char* src = static_cast<const unsigned char*>(base) + row * static_cast<int64_t>(seg_bytes);
+        mbar_arrive_expect_tx(&full[slot], seg_bytes);
+        bulk_load(ring + static_cast<size_t>(slot) * seg_bytes, src, seg_bytes, &full[slot]);
+        issued = g + 1;
+      }
+      *issued_count = issued;  // read by the drain below
+      __threadfence_block();
+      *producer_done = 1;
+    }
+    return;
+  }
+
+  // consumers
+  const RingRed red0{&hdr->red[0][0][0], ncons}, red1{&hdr->red[1][0][0], ncons};
+  const int j0 = threadIdx.x;
+  for (int64_t i = 0; i < my_rows; ++i) {
+    const int64_t row = p.row_begin + blockIdx.x + i * gridDim.x;
+    float y[VPT][8];
+    bool ok[VPT];
+#pragma unroll
+    for (int k = 0; k < VPT; ++k) {
+      ok[k] = (j0 + k * ncons) < p.packs;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) y[k][e] = 0.f;
+    }
+    for (int k = 0; k < S; ++k) {
+      const int64_t g = i * S + k;
+      const int slot = static_cast<int>(g % nslot);
+      const uint32_t round = static_cast<uint32_t>(g / nslot);
+      if (!*abort_flag && !mbar_wait(&full[slot], round & 1u, abort_flag)) {
+        if (!*abort_flag) atomicOr(&g_far_error, kErrWaitFull);
+        *abort_flag = 1;
+      }
+      const uint4* seg = reinterpret_cast<const uint4*>(ring + static_cast<size_t>(slot) * seg_bytes);
+#pragma unroll
+      for (int q = 0; q < VPT; ++q) {
+        if (!ok[q]) continue;
+        float f[8];
+        DT::unpack(seg[j0 + q * ncons], f);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) y[q][e] += f[e];
+      }
+      __syncwarp();
+      if ((threadIdx.x & 31) == 0) mbar_arrive(&empty[slot]);
+    }
+    finish_row<DT, VPT>(p, row, true, j0, ncons, ok, y, (i & 1) ? red1 : red0, gamma_s);
+  }
+
+  // Only after an abort can copies still be in flight: thread 0 waits for
+  // the producer to stop and then for the last phase of every used slot.
+  if (threadIdx.x == 0) {
+    const uint64_t t0 = global_ns();
+    while (!*producer_done && global_ns() - t0 < kWaitLimitNs) {
+    }
+    if (*abort_flag) {
+      const int64_t issued = *issued_count;
+      for (int64_t g = (issued > nslot ? issued - nslot : 0); g < issued; ++g) {
+        const int slot = static_cast<int>(g % nslot);
+        mbar_wait(&full[slot], static_cast<uint32_t>(g / nslot) & 1u, nullptr);
+      }
+    }
+  }
+}
+
 template <class DT, int VPT, bool SUB>
 cudaError_t launch_prefill_t(const Params& p, const Launch& l, cudaStream_t s) {
   cudaLaunchConfig_t cfg = {};
@@ -375,6 +657,29 @@ cudaError_t launch_decode_t(const Params& p, const Launch& l, cudaStream_t s) {
   return cudaLaunchKernelEx(&cfg, far_decode_kernel<DT, VPT>, p);
 }
 
+template <class DT, int VPT>
+cudaError_t launch_ring_t(const Params& p, const Launch& l, cudaStream_t s) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(l.grid), 1, 1);
+  cfg.blockDim = dim3(static_cast<unsigned>(l.threads), 1, 1);
+  cfg.dynamicSmemBytes = static_cast<size_t>(l.smem_bytes);
+  cfg.stream = s;
+  cfg.attrs = nullptr;
+  cfg.numAttrs = 0;
+  return cudaLaunchKernelEx(&cfg, far_ring_kernel<DT, VPT>, p, l.nslot, l.tpr);
+}
+
+template <class DT>
+cudaError_t launch_ring_dt(const Params& p, const Launch& l, cudaStream_t s) {
+  switch (l.vpt) {
+    case 1: return launch_ring_t<DT, 1>(p, l, s);
+    case 2: return launch_ring_t<DT, 2>(p, l, s);
+    case 4: return launch_ring_t<DT, 4>(p, l, s);
+    case 8: return launch_ring_t<DT, 8>(p, l, s);
+    default: return cudaErrorInvalidConfiguration;
+  }
+}
+
 template <class DT>
 cudaError_t launch_prefill_dt(const Params& p, const Launch& l, cudaStream_t s) {
   if (l.tpr <= 32 && l.rows_per_cta > 1) return launch_prefill_t<DT, 1, true>(p, l, s);
@@ -396,6 +701,20 @@ cudaError_t launch_decode_dt(const Params& p, const Launch& l, cudaStream_t s) {
     case 8: return launch_decode_t<DT, 8>(p, l, s);
     default: return cudaErrorInvalidConfiguration;
   }
+}
+
+template <class DT>
+cudaError_t allow_large_smem() {
+  cudaError_t e = cudaSuccess;
+  const auto set = [&](auto kern) {
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kRingSmemMax);
+  };
+  set(far_ring_kernel<DT, 1>);
+  set(far_ring_kernel<DT, 2>);
+  set(far_ring_kernel<DT, 4>);
+  set(far_ring_kernel<DT, 8>);
+  return e;
 }
 
 template <class DT>
@@ -422,9 +741,53 @@ cudaError_t launch_decode(const Params& p, int dtype, const Launch& l, cudaStrea
   return dtype == kBf16 ? launch_decode_dt<Bf16T>(p, l, s) : launch_decode_dt<Fp16T>(p, l, s);
 }
 
+cudaError_t launch_ring(const Params& p, int dtype, const Launch& l, cudaStream_t s) {
+  return dtype == kBf16 ? launch_ring_dt<Bf16T>(p, l, s) : launch_ring_dt<Fp16T>(p, l, s);
+}
+
+int ring_header_bytes(int nslot) { return ring_offset(nslot); }
+
+namespace {
+template <class DT>
+int ring_occupancy_dt(int vpt, int threads, int smem) {
+  int n = 0;
+  cudaError_t e = cudaErrorInvalidValue;
+  switch (vpt) {
+    case 1: e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, far_ring_kernel<DT, 1>, threads, smem); break;
+    case 2: e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, far_ring_kernel<DT, 2>, threads, smem); break;
+    case 4: e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, far_ring_kernel<DT, 4>, threads, smem); break;
+    case 8: e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, far_ring_kernel<DT, 8>, threads, smem); break;
+    default: break;
+  }
+  return e == cudaSuccess ? n : 0;
+}
+}  // namespace
+
+int ring_occupancy(int dtype, int vpt, int threads, int smem_bytes) {
+  return dtype == kBf16 ? ring_occupancy_dt<Bf16T>(vpt, threads, smem_bytes)
+                        : ring_occupancy_dt<Fp16T>(vpt, threads, smem_bytes);
+}
+
 cudaError_t configure_kernels() {
   cudaError_t e = allow_large_clusters<Bf16T>();
   if (e == cudaSuccess) e = allow_large_clusters<Fp16T>();
+  if (e == cudaSuccess) e = allow_large_smem<Bf16T>();
+  if (e == cudaSuccess) e = allow_large_smem<Fp16T>();
+  return e;
+}
+
+cudaError_t read_error_word(unsigned* out, cudaStream_t s) {
+  cudaError_t e = cudaMemcpyFromSymbolAsync(out, g_far_error, sizeof(unsigned), 0,
+                                            cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  return e;
+}
+
+cudaError_t clear_error_word(cudaStream_t s) {
+  static const unsigned zero = 0u;
+  cudaError_t e = cudaMemcpyToSymbolAsync(g_far_error, &zero, sizeof(unsigned), 0,
+                                          cudaMemcpyHostToDevice, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
   return e;
 }
 

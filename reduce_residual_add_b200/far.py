@@ -44,8 +44,8 @@ FAR_MAX_H = 16384
 
 # Every symbol include/far.h declares.
 EXPORTS = ("far_create", "far_destroy", "far_fused", "far_fused_rows", "far_validate",
-           "far_set_regime", "far_describe_launch", "far_status_string", "far_last_error",
-           "far_version")
+           "far_set_regime", "far_describe_launch", "far_check", "far_status_string",
+           "far_last_error", "far_version")
 
 _DTYPES = {torch.bfloat16: FAR_BF16, torch.float16: FAR_FP16}
 
@@ -53,7 +53,8 @@ _DTYPES = {torch.bfloat16: FAR_BF16, torch.float16: FAR_FP16}
 class far_launch_info(ctypes.Structure):
     _fields_ = [("regime", ctypes.c_int), ("ctas_per_row", ctypes.c_int),
                 ("rows_per_cta", ctypes.c_int), ("threads_per_cta", ctypes.c_int),
-                ("packs_per_thread", ctypes.c_int), ("grid_ctas", ctypes.c_int64)]
+                ("packs_per_thread", ctypes.c_int), ("grid_ctas", ctypes.c_int64),
+                ("kernel", ctypes.c_int), ("ring_slots", ctypes.c_int)]
 
 
 class FarError(RuntimeError):
@@ -102,6 +103,8 @@ def lib() -> ctypes.CDLL:
     L.far_set_regime.restype = i32
     L.far_describe_launch.argtypes = [vp, i64, i64, i32, ctypes.POINTER(far_launch_info)]
     L.far_describe_launch.restype = i32
+    L.far_check.argtypes = [vp, vp]
+    L.far_check.restype = i32
     L.far_status_string.argtypes = [i32]
     L.far_status_string.restype = ctypes.c_char_p
     L.far_last_error.argtypes = []
@@ -179,6 +182,14 @@ def far_describe_launch(ctx: FarContext, rows: int, H: int, dtype=torch.bfloat16
     if st != FAR_OK:
         raise FarError(st, "far_describe_launch")
     return {name: getattr(info, name) for name, _ in far_launch_info._fields_}
+
+
+def far_check(ctx: FarContext, stream=None) -> None:
+    """Synchronise `stream` and raise FarError(FAR_ERR_TIMEOUT) if a kernel's
+    bounded wait gave up since the last check (see include/far.h)."""
+    st = lib().far_check(ctx.handle, _stream(stream))
+    if st != FAR_OK:
+        raise FarError(st, "far_check")
 
 
 def _ptr(t: Optional[torch.Tensor]):

@@ -97,6 +97,7 @@ def run_gpu(ctx, g: dict, eps: float, wb: float, pattern: int, scale_in=None, ro
     else:
         far.far_fused_rows(ctx, rows[0], rows[1], ps, res, g["gamma"], eps, wb, pattern, **kw)
     torch.cuda.synchronize()
+    far.far_check(ctx, stream)          # no bounded wait inside the kernel gave up
     for raw, gb, n in canaries:
         head, tail = raw[:gb], raw[gb + n:]
         assert bool((head == 0xA5).all()) and bool((tail == 0xA5).all()), "write outside an output"

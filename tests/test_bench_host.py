@@ -1,0 +1,50 @@
+"""Host-side pieces of bench.py that need no GPU."""
+from __future__ import annotations
+
+import json
+import os
+import time
+
+import bench
+from reduce_residual_add_b200.inputs import WORKLOADS
+
+
+def test_algorithmic_bytes_of_the_workloads():
+    c4 = WORKLOADS["c4_prefill_fp8_static"]
+    assert bench.algorithmic_bytes(c4, c4.T, False) == 872_431_616
+    assert bench.algorithmic_bytes(c4, c4.T, True) == 1_006_649_344
+    c5 = WORKLOADS["c5_gemma_fp8_token_bf16"]
+    assert bench.algorithmic_bytes(c5, c5.T, False) == 616_593_408
+    assert bench.algorithmic_bytes(c5, c5.T, True) == 675_313_664
+    c3 = WORKLOADS["c3_3d"]
+    assert bench.algorithmic_bytes(c3, c3.T, True) == 20_975_616
+    c1 = WORKLOADS["c1_small"]
+    assert bench.algorithmic_bytes(c1, c1.T, True) == 5_248
+    for T, b in ((1, 98_304), (8, 729_088), (32, 2_891_776), (80, 7_217_152)):
+        wl = WORKLOADS["c2_decode_T%d" % T]
+        assert bench.algorithmic_bytes(wl, T, True) == b
+
+
+def test_clock_sampler_starts_and_stops_without_a_gpu():
+    s = bench.ClockSampler(0, period_s=0.001)
+    s.start()
+    time.sleep(0.01)
+    out = s.stop()
+    assert set(out) >= {"sm_mhz", "sm_max_mhz", "reasons"}
+
+
+def test_peak_and_traffic_lookup():
+    peak, kind = bench.hbm_peak()
+    assert peak > 1000 and kind in ("measured", "fallback")
+    # the traffic figure is only used while the kernel source is unchanged
+    t = bench.profiled_traffic("c4_prefill_fp8_static")
+    path = os.path.join(bench.ROOT, "profiles", "traffic.json")
+    if os.path.exists(path):
+        d = json.load(open(path))
+        e = d.get("c4_prefill_fp8_static")
+        if e and e.get("source_sha256") == bench.kernel_source_hash():
+            assert t == e["traffic_bytes_per_launch"]
+        else:
+            assert t is None
+    else:
+        assert t is None

@@ -37,6 +37,36 @@ def ctx():
     c.close()
 
 
+def _ctx_with_env(env):
+    old = {k: os.environ.get(k) for k in env}
+    os.environ.update(env)
+    try:
+        return far.FarContext(0)
+    finally:
+        for k, v in old.items():
+            if v is None:
+                os.environ.pop(k, None)
+            else:
+                os.environ[k] = v
+
+
+@pytest.fixture(scope="module")
+def kctx():
+    """Contexts for each prefill kernel: the TMA ring (1 and 2 CTAs per SM)
+    and the direct-load kernel."""
+    out = {"ring": _ctx_with_env({}),
+           "ring256": _ctx_with_env({"FAR_RING_THREADS": "256", "FAR_RING_CTAS_PER_SM": "1"}),
+           "ring512": _ctx_with_env({"FAR_RING_THREADS": "512", "FAR_RING_CTAS_PER_SM": "1"}),
+           "ring2": _ctx_with_env({"FAR_RING_CTAS_PER_SM": "2", "FAR_RING_THREADS": "256"}),
+           "ring4": _ctx_with_env({"FAR_RING_CTAS_PER_SM": "4", "FAR_RING_THREADS": "128"}),
+           "direct": _ctx_with_env({"FAR_PREFILL_KERNEL": "0"})}
+    for c in out.values():
+        far.far_set_regime(c, far.FAR_REGIME_PREFILL)
+    yield out
+    for c in out.values():
+        c.close()
+
+
 @pytest.fixture
 def regime(ctx):
     """Set a regime for one test and restore automatic choice afterwards."""
@@ -74,6 +104,41 @@ def test_small_shapes(ctx, regime, case, reg):
     got = run_gpu(ctx, to_gpu(inp), eps, wb, pattern, scale_in=scale, guard=4096)
     ref = run_oracle(inp, dt, eps, wb, pattern, scale_in=scale)
     log("small %s reg%d" % (case, reg), compare(got, ref, dt))
+
+
+@pytest.mark.parametrize("kern", ["ring", "ring256", "ring512", "ring2", "ring4", "direct"])
+@pytest.mark.parametrize("case", [
+    (2, 3000, 264, "bf16", 2, True, 0.0),    # 33 packs, 32 slots, ~20 rows per CTA
+    (16, 300, 16384, "bf16", 1, True, 1.0),  # 17 segments per row, 6 slots
+    (4, 1000, 8192, "fp16", 0, False, 0.0),  # no residual: W segments per row
+    (8, 149, 7168, "bf16", 2, True, 1.0),    # one more row than CTAs
+    (3, 7, 2048, "bf16", 1, True, 0.0),      # fewer rows than CTAs
+], ids=lambda c: "W%d_T%d_H%d_%s_p%d_res%d_wb%g" % c)
+def test_prefill_kernels(kctx, case, kern):
+    W, T, H, dt, pattern, has_res, wb = case
+    c = kctx[kern]
+    info = far.far_describe_launch(c, T, H, torch.bfloat16)
+    per_sm = {"ring4": 4, "ring2": 2}.get(kern, 1)
+    fits = 228 * 1024 // per_sm - 1024 >= 3 * H * 2 + 1024   # gamma, two slots, header
+    assert info["kernel"] == (1 if (kern != "direct" and fits) else 0)
+    inp = random_inputs(W, T, H, dtype=dt, seed=7 * W + T + H, has_residual=has_res)
+    got = run_gpu(c, to_gpu(inp), 1e-6, wb, pattern, scale_in=0.05, guard=1024)
+    ref = run_oracle(inp, dt, 1e-6, wb, pattern, scale_in=0.05)
+    log("prefill %s %s" % (kern, case), compare(got, ref, dt))
+
+
+@pytest.mark.parametrize("pattern", [1, 2])
+def test_ring_and_direct_agree_bitwise(kctx, pattern):
+    """With the same threads per row, both prefill kernels sum in the same
+    order and reduce in the same tree: identical bits."""
+    inp = random_inputs(4, 600, 8192, seed=21)
+    g = to_gpu(inp)
+    a = run_gpu(kctx["ring256"], g, 1e-5, 0.0, pattern, scale_in=0.05)
+    b = run_gpu(kctx["direct"], g, 1e-5, 0.0, pattern, scale_in=0.05)
+    c = run_gpu(kctx["ring2"], g, 1e-5, 0.0, pattern, scale_in=0.05)
+    for k in ("residual_out", "norm_out", "quant_out", "scale_out"):
+        if a[k] is not None:
+            assert np.array_equal(a[k], b[k]) and np.array_equal(a[k], c[k]), k
 
 
 def test_small_workload_matches_golden_fixture(ctx):
@@ -274,6 +339,7 @@ def test_launch_plan(ctx):
     p = far.far_describe_launch(ctx, 81, 4096)
     assert p["regime"] == far.FAR_REGIME_PREFILL
     c4 = far.far_describe_launch(ctx, 8192, 8192)
-    assert c4["threads_per_cta"] * c4["packs_per_thread"] * 8 >= 8192
+    assert c4["kernel"] == 1 and c4["ring_slots"] >= 2
+    assert (c4["threads_per_cta"] - 32) * c4["packs_per_thread"] * 8 >= 8192
     tiny = far.far_describe_launch(ctx, 8, 64)
     assert tiny["regime"] == far.FAR_REGIME_PREFILL and tiny["rows_per_cta"] > 1
