@@ -53,6 +53,7 @@ __host__ __device__ constexpr int ring_offset(int nslot) {
 // ---------------------------------------------------------------------------
 
 struct Bf16T {
+  static constexpr bool kIsBf16 = true;
   // bf16 is the upper half of an fp32: widening is a shift
   static __device__ __forceinline__ void unpack(const uint4& v, float (&f)[8]) {
     f[0] = __uint_as_float(v.x << 16);
@@ -71,6 +72,7 @@ struct Bf16T {
 };
 
 struct Fp16T {
+  static constexpr bool kIsBf16 = false;
   static __device__ __forceinline__ void unpack(const uint4& v, float (&f)[8]) {
     const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
@@ -86,6 +88,40 @@ struct Fp16T {
     return *reinterpret_cast<uint32_t*>(&h);
   }
 };
+
+// acc[i] += element i of the pack, and out[i] = element i + s: each element
+// is widened exactly and added with one fp32 rounding, the same result as
+// unpack-then-add, in one mixed-precision add (add.rn.f32.bf16 / .f16,
+// sm_100) per element.
+#define FAR_MIXED_ADD_2(TYPE, ACC0, ACC1, WORD, S0, S1)                                   \
+  asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %2;\n\t"                           \
+      "add.rn.f32." TYPE " %0, lo, %3;\n\tadd.rn.f32." TYPE " %1, hi, %4;\n\t}"           \
+      : "=f"(ACC0), "=f"(ACC1)                                                            \
+      : "r"(WORD), "f"(S0), "f"(S1))
+
+template <class DT>
+__device__ __forceinline__ void add_pack(const uint4& v, float (&acc)[8]) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    if constexpr (DT::kIsBf16)
+      FAR_MIXED_ADD_2("bf16", acc[2 * i], acc[2 * i + 1], w[i], acc[2 * i], acc[2 * i + 1]);
+    else
+      FAR_MIXED_ADD_2("f16", acc[2 * i], acc[2 * i + 1], w[i], acc[2 * i], acc[2 * i + 1]);
+  }
+}
+
+template <class DT>
+__device__ __forceinline__ void pack_plus(const uint4& v, float s, float (&out)[8]) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    if constexpr (DT::kIsBf16)
+      FAR_MIXED_ADD_2("bf16", out[2 * i], out[2 * i + 1], w[i], s, s);
+    else
+      FAR_MIXED_ADD_2("f16", out[2 * i], out[2 * i + 1], w[i], s, s);
+  }
+}
 
 template <class DT>
 __device__ __forceinline__ uint4 pack8(const float (&f)[8]) {
@@ -346,13 +382,12 @@ __device__ __forceinline__ void finish_row(const Params& p, int64_t row, bool ro
   for (int k = 0; k < VPT; ++k) {
     if (!ok[k]) continue;
     const int64_t pk = rbase + j0 + k * jstride;
-    float g[8];
-    if (gamma_smem != nullptr)
-      DT::unpack(gamma_smem[j0 + k * jstride], g);
-    else
-      DT::unpack(__ldg(static_cast<const uint4*>(p.gamma) + j0 + k * jstride), g);
+    float g[8];  // gamma + weight_bias in fp32
+    pack_plus<DT>(gamma_smem != nullptr ? gamma_smem[j0 + k * jstride]
+                                        : __ldg(static_cast<const uint4*>(p.gamma) + j0 + k * jstride),
+                  p.weight_bias, g);
 #pragma unroll
-    for (int i = 0; i < 8; ++i) y[k][i] = (y[k][i] * rinv) * (g[i] + p.weight_bias);
+    for (int i = 0; i < 8; ++i) y[k][i] = (y[k][i] * rinv) * g[i];
     if (p.norm_out != nullptr) static_cast<uint4*>(p.norm_out)[pk] = pack8<DT>(y[k]);
     if (fp8_static) {
       float q[8];
@@ -432,12 +467,7 @@ __device__ __forceinline__ void fused_row(const Params& p, int64_t row, bool row
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
 #pragma unroll
-      for (int k = 0; k < VPT; ++k) {
-        float f[8];
-        DT::unpack(v[c][k], f);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) y[k][i] += f[i];
-      }
+      for (int k = 0; k < VPT; ++k) add_pack<DT>(v[c][k], y[k]);
     }
   }
 
@@ -450,12 +480,7 @@ __device__ __forceinline__ void fused_row(const Params& p, int64_t row, bool row
       if (ok[k]) v[k] = ld_once_coherent(static_cast<const uint4*>(p.residual) + rbase + j0 + k * jstride);
     }
 #pragma unroll
-    for (int k = 0; k < VPT; ++k) {
-      float f[8];
-      DT::unpack(v[k], f);
-#pragma unroll
-      for (int i = 0; i < 8; ++i) y[k][i] += f[i];
-    }
+    for (int k = 0; k < VPT; ++k) add_pack<DT>(v[k], y[k]);
   }
   finish_row<DT, VPT>(p, row, row_ok, j0, jstride, ok, y, red);
 }
@@ -599,13 +624,8 @@ far_ring_kernel(const Params p, int nslot, int ncons) {
       }
       const uint4* seg = reinterpret_cast<const uint4*>(ring + static_cast<size_t>(slot) * seg_bytes);
 #pragma unroll
-      for (int q = 0; q < VPT; ++q) {
-        if (!ok[q]) continue;
-        float f[8];
-        DT::unpack(seg[j0 + q * ncons], f);
-#pragma unroll
-        for (int e = 0; e < 8; ++e) y[q][e] += f[e];
-      }
+      for (int q = 0; q < VPT; ++q)
+        if (ok[q]) add_pack<DT>(seg[j0 + q * ncons], y[q]);
       __syncwarp();
       if ((threadIdx.x & 31) == 0) mbar_arrive(&empty[slot]);
     }
