@@ -54,17 +54,6 @@ __host__ __device__ constexpr int ring_offset(int nslot) {
 
 struct Bf16T {
   static constexpr bool kIsBf16 = true;
-  // bf16 is the upper half of an fp32: widening is a shift
-  static __device__ __forceinline__ void unpack(const uint4& v, float (&f)[8]) {
-    f[0] = __uint_as_float(v.x << 16);
-    f[1] = __uint_as_float(v.x & 0xffff0000u);
-    f[2] = __uint_as_float(v.y << 16);
-    f[3] = __uint_as_float(v.y & 0xffff0000u);
-    f[4] = __uint_as_float(v.z << 16);
-    f[5] = __uint_as_float(v.z & 0xffff0000u);
-    f[6] = __uint_as_float(v.w << 16);
-    f[7] = __uint_as_float(v.w & 0xffff0000u);
-  }
   static __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
     __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);  // round to nearest even
     return *reinterpret_cast<uint32_t*>(&h);
@@ -73,16 +62,6 @@ struct Bf16T {
 
 struct Fp16T {
   static constexpr bool kIsBf16 = false;
-  static __device__ __forceinline__ void unpack(const uint4& v, float (&f)[8]) {
-    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      __half2 h = *reinterpret_cast<const __half2*>(&w[i]);
-      float2 x = __half22float2(h);
-      f[2 * i] = x.x;
-      f[2 * i + 1] = x.y;
-    }
-  }
   static __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
     __half2 h = __floats2half2_rn(lo, hi);  // round to nearest even
     return *reinterpret_cast<uint32_t*>(&h);
@@ -266,7 +245,9 @@ __device__ __forceinline__ float group_max(float v, int width) {
 struct SubwarpRed {
   int width;
   __device__ float sum(float v) const { return group_sum(v, width); }
-  __device__ float max(float v) const { return group_max(v, width); }
+  __device__ float2 sum_max(float s, float m) const {
+    return make_float2(group_sum(s, width), group_max(m, width));
+  }
   __device__ bool leader() const { return threadIdx.x == 0; }
 };
 
@@ -276,16 +257,26 @@ struct SubwarpRed {
 struct BlockRed {
   float* s_sum;  // [32]
   float* s_max;  // [32]
-  __device__ float reduce(float v, float* slot, bool is_max) const {
+  __device__ float sum(float v) const {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
-    v = is_max ? group_max(v, 32) : group_sum(v, 32);
-    if (lane == 0) slot[warp] = v;
+    v = group_sum(v, 32);
+    if (lane == 0) s_sum[warp] = v;
     __syncthreads();
-    float t = lane < nw ? slot[lane] : 0.f;
-    return is_max ? group_max(t, 32) : group_sum(t, 32);
+    return group_sum(lane < nw ? s_sum[lane] : 0.f, 32);
   }
-  __device__ float sum(float v) const { return reduce(v, s_sum, false); }
-  __device__ float max(float v) const { return reduce(v, s_max, true); }
+  // both totals in one barrier round
+  __device__ float2 sum_max(float s, float m) const {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    s = group_sum(s, 32);
+    m = group_max(m, 32);
+    if (lane == 0) {
+      s_sum[warp] = s;
+      s_max[warp] = m;
+    }
+    __syncthreads();
+    return make_float2(group_sum(lane < nw ? s_sum[lane] : 0.f, 32),
+                       group_max(lane < nw ? s_max[lane] : 0.f, 32));
+  }
   __device__ bool leader() const { return threadIdx.x == 0; }
 };
 
@@ -296,19 +287,25 @@ struct BlockRed {
 // cluster barrier before any CTA (and its shared memory) goes away.
 struct ClusterRed {
   BlockRed blk;
-  float* s_cta;  // [2]: 0 = sum of squares, 1 = amax
-  __device__ float across(float t, int slot, bool is_max) const {
+  float* s_cta;  // [2]: 0 = sum of squares, 1 = max
+  __device__ float2 across(float2 t) const {
     cg::cluster_group cl = cg::this_cluster();
-    if (threadIdx.x == 0) s_cta[slot] = t;
+    if (threadIdx.x == 0) {
+      s_cta[0] = t.x;
+      s_cta[1] = t.y;
+    }
     cl.sync();
     const int lane = threadIdx.x & 31;
     const int n = static_cast<int>(cl.num_blocks());
-    float u = 0.f;
-    if (lane < n) u = *cl.map_shared_rank(s_cta + slot, lane);
-    return is_max ? group_max(u, 32) : group_sum(u, 32);
+    float u = 0.f, w = 0.f;
+    if (lane < n) {
+      u = *cl.map_shared_rank(s_cta, lane);
+      w = *cl.map_shared_rank(s_cta + 1, lane);
+    }
+    return make_float2(group_sum(u, 32), group_max(w, 32));
   }
-  __device__ float sum(float v) const { return across(blk.sum(v), 0, false); }
-  __device__ float max(float v) const { return across(blk.max(v), 1, true); }
+  __device__ float sum(float v) const { return across(make_float2(blk.sum(v), 0.f)).x; }
+  __device__ float2 sum_max(float s, float m) const { return across(blk.sum_max(s, m)); }
   __device__ bool leader() const {
     return threadIdx.x == 0 && cg::this_cluster().block_rank() == 0;
   }
@@ -319,18 +316,27 @@ struct ClusterRed {
 // row parity: a warp can only rewrite a half after every consumer passed the
 // next row's barrier, i.e. after everyone finished reading it.
 struct RingRed {
-  float* buf;     // [2][32]: 0 = sum of squares, 1 = amax
+  float* buf;     // [2][32]: 0 = sum of squares, 1 = max
   int nthreads;   // consumer threads
-  __device__ float reduce(float v, int which, bool is_max) const {
+  __device__ float sum(float v) const {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = nthreads >> 5;
-    v = is_max ? group_max(v, 32) : group_sum(v, 32);
-    if (lane == 0) buf[which * 32 + warp] = v;
+    v = group_sum(v, 32);
+    if (lane == 0) buf[warp] = v;
     consumer_bar(nthreads);
-    float t = lane < nw ? buf[which * 32 + lane] : 0.f;
-    return is_max ? group_max(t, 32) : group_sum(t, 32);
+    return group_sum(lane < nw ? buf[lane] : 0.f, 32);
   }
-  __device__ float sum(float v) const { return reduce(v, 0, false); }
-  __device__ float max(float v) const { return reduce(v, 1, true); }
+  __device__ float2 sum_max(float s, float m) const {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = nthreads >> 5;
+    s = group_sum(s, 32);
+    m = group_max(m, 32);
+    if (lane == 0) {
+      buf[warp] = s;
+      buf[32 + warp] = m;
+    }
+    consumer_bar(nthreads);
+    return make_float2(group_sum(lane < nw ? buf[lane] : 0.f, 32),
+                       group_max(lane < nw ? buf[32 + lane] : 0.f, 32));
+  }
   __device__ bool leader() const { return threadIdx.x == 0; }
 };
 
@@ -366,59 +372,60 @@ __device__ __forceinline__ void finish_row(const Params& p, int64_t row, bool ro
   for (int w = 1; w < VPT; w <<= 1)
 #pragma unroll
     for (int k = 0; k + w < VPT; k += 2 * w) sq[k] += sq[k + w];
-  const float ss = red.sum(sq[0]);
+
+  const bool fp8_static = p.pattern == kFp8Static;
+  const bool fp8_token = p.pattern == kFp8Token;
+  const uint4* gam = gamma_smem != nullptr ? gamma_smem : static_cast<const uint4*>(p.gamma);
+
+  // a5b needs max|o| = rinv * max|y * (gamma + wb)| (rinv > 0): its local
+  // part goes into the same reduction round as the sum of squares.
+  float ss, gmax = 0.f;
+  if (fp8_token) {
+    float m = 0.f;
+#pragma unroll
+    for (int k = 0; k < VPT; ++k) {
+      if (!ok[k]) continue;
+      float g[8];
+      pack_plus<DT>(gam[j0 + k * jstride], p.weight_bias, g);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) m = fmaxf(m, fabsf(y[k][i] * g[i]));
+    }
+    const float2 r = red.sum_max(sq[0], m);
+    ss = r.x;
+    gmax = r.y;
+  } else {
+    ss = red.sum(sq[0]);
+  }
   const float ms = __fdiv_rn(ss, static_cast<float>(p.H));
   const float rinv = __frsqrt_rn(ms + p.eps);
 
+  // the divisor of the FP8 codes: the static scale, or max|o| / 448
+  float scale = 1.f;
+  if (fp8_static) scale = __ldg(p.scale_in);
+  if (fp8_token) {
+    scale = __fdiv_rn(rinv * gmax, 448.f);
+    // a row with an inf or NaN input has rinv 0 or NaN; its finite o are 0
+    // and the rest NaN, which take no part in the amax: scale 0
+    if (scale != scale) scale = 0.f;
+    if (row_ok && red.leader()) p.scale_out[row] = scale;
+  }
+  const float inv = __frcp_rn(scale);
+  // outside the reciprocal's normal range, divide exactly (uniform per row)
+  const bool exact = !(fabsf(inv) < 3.0e38f && fabsf(scale) > 1.0e-37f);
+
   // a4: o = y * rinv * (gamma + weight_bias); a5: FP8 codes.
-  const bool fp8_static = p.pattern == kFp8Static;
-  const bool fp8_token = p.pattern == kFp8Token;
-  const float s_static = fp8_static ? __ldg(p.scale_in) : 1.f;
-  const float inv_static = __frcp_rn(s_static);
-  // outside the normal range of the reciprocal, divide exactly instead
-  const bool exact_static = !(fabsf(inv_static) < 3.0e38f && fabsf(s_static) > 1.0e-37f);
-  float amax = 0.f;
 #pragma unroll
   for (int k = 0; k < VPT; ++k) {
     if (!ok[k]) continue;
     const int64_t pk = rbase + j0 + k * jstride;
     float g[8];  // gamma + weight_bias in fp32
-    pack_plus<DT>(gamma_smem != nullptr ? gamma_smem[j0 + k * jstride]
-                                        : __ldg(static_cast<const uint4*>(p.gamma) + j0 + k * jstride),
-                  p.weight_bias, g);
+    pack_plus<DT>(gam[j0 + k * jstride], p.weight_bias, g);
 #pragma unroll
     for (int i = 0; i < 8; ++i) y[k][i] = (y[k][i] * rinv) * g[i];
     if (p.norm_out != nullptr) static_cast<uint4*>(p.norm_out)[pk] = pack8<DT>(y[k]);
-    if (fp8_static) {
-      float q[8];
-      if (exact_static) {
-#pragma unroll
-        for (int i = 0; i < 8; ++i) q[i] = __fdiv_rn(y[k][i], s_static);
-      } else {
-#pragma unroll
-        for (int i = 0; i < 8; ++i) q[i] = div_by(y[k][i], s_static, inv_static);
-      }
-      reinterpret_cast<uint2*>(p.quant_out)[pk] =
-          make_uint2(e4m3x4(q[0], q[1], q[2], q[3]), e4m3x4(q[4], q[5], q[6], q[7]));
-    }
-    if (fp8_token) {
-#pragma unroll
-      for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(y[k][i]));
-    }
-  }
-
-  if (fp8_token) {
-    const float rowmax = red.max(amax);
-    const float scale = __fdiv_rn(rowmax, 448.f);
-    if (row_ok && red.leader()) p.scale_out[row] = scale;
-    const float inv = __frcp_rn(scale);
-    const bool exact = !(inv < 3.0e38f && scale > 1.0e-37f);  // row-uniform
-#pragma unroll
-    for (int k = 0; k < VPT; ++k) {
-      if (!ok[k]) continue;
-      const int64_t pk = rbase + j0 + k * jstride;
+    if (fp8_static || fp8_token) {
       uint2 codes = make_uint2(0u, 0u);
-      if (scale != 0.f) {
+      if (scale != 0.f) {  // a per-token row of zeros keeps scale 0 and codes 0
         float q[8];
         if (exact) {
 #pragma unroll
