@@ -101,7 +101,16 @@ typedef enum {
  * FAR_PREFILL_THREADS, FAR_PREFILL_KERNEL=1 ring | 0 direct,
  * FAR_RING_CTAS_PER_SM=1..4 (default 2), FAR_RING_THREADS: consumer threads
  * per ring CTA, at most 512 (default 256), FAR_RING_SLOTS: row-segment slots
- * per ring CTA (2..32; default: about 72 KiB of segments, as many as fit)). */
+ * per ring CTA (2..32; default: about 72 KiB of segments, as many as fit),
+ * FAR_PDL=1|0: launch with programmatic dependent launch, default 1,
+ * FAR_RING_MIN_ROWS: fewest rows for the ring kernel, default by rule). */
+/*
+ * Programmatic dependent launch: every kernel of this library first waits
+ * (griddepcontrol.wait) until the grid it depends on has completed, then
+ * lets its own dependents be scheduled.  The next kernel in the stream may
+ * therefore start its launch while this one runs, but reads nothing before
+ * this one has finished; a preceding kernel that triggers early likewise
+ * overlaps its tail with this call's launch. */
 typedef struct far_ctx far_ctx;
 
 /* How one call would be launched (see far_describe_launch). */

@@ -27,6 +27,8 @@ struct far_ctx {
   int ring_ctas_per_sm; // persistent ring CTAs per SM wanted (1..4)
   int ring_threads;     // target consumer threads of a ring CTA
   int ring_slots_max;   // at most this many ring slots
+  int pdl;              // programmatic dependent launch on every call
+  int ring_min_rows;    // fewer rows than this take the direct kernel
   // ring CTAs per SM the occupancy calculator allows, per (dtype, packs):
   // 0 = not asked yet, -1 = cannot run
   std::mutex occ_mu;
@@ -179,8 +181,17 @@ far::Launch plan(const far_ctx* ctx, int64_t rows, int64_t H, int dtype) {
   } else {
     plan_prefill(packs, ctx->prefill_threads, &l);
     l.grid = (rows + l.rows_per_cta - 1) / l.rows_per_cta;
-    if (ctx->prefill_kernel == 1) plan_ring(ctx, packs, rows, dtype, &l);
+    // The ring pays off once each persistent CTA gets enough rows to keep
+    // its pipeline full: measured crossover about 8 rows per CTA at
+    // H >= 7168 and 16 at H = 2048, i.e. max(8, 4096 / packs) per CTA.
+    int64_t min_rows = ctx->ring_min_rows;
+    if (min_rows <= 0) {
+      const int per_cta = (4096 / packs > 8) ? 4096 / packs : 8;
+      min_rows = static_cast<int64_t>(per_cta) * ctx->sm_count * ctx->ring_ctas_per_sm;
+    }
+    if (ctx->prefill_kernel == 1 && rows >= min_rows) plan_ring(ctx, packs, rows, dtype, &l);
   }
+  l.pdl = ctx->pdl;
   return l;
 }
 
@@ -228,7 +239,7 @@ far_status far_create(far_ctx** ctx, int device) {
     return FAR_ERR_UNSUPPORTED;
   }
   c.decode_max_rows = env_int("FAR_DECODE_MAX_ROWS", 80);
-  c.decode_cluster = env_int("FAR_DECODE_CLUSTER", 8);
+  c.decode_cluster = env_int("FAR_DECODE_CLUSTER", 4);
   c.prefill_threads = env_int("FAR_PREFILL_THREADS", 256);
   if (c.prefill_threads < 32) c.prefill_threads = 32;
   if (c.prefill_threads > far::kMaxThreads) c.prefill_threads = far::kMaxThreads;
@@ -242,6 +253,8 @@ far_status far_create(far_ctx** ctx, int device) {
   if (c.ring_slots_max > 32) c.ring_slots_max = 32;
   if (c.ring_threads < 32) c.ring_threads = 32;
   if (c.ring_threads > far::kRingMaxConsumers) c.ring_threads = far::kRingMaxConsumers;
+  c.pdl = env_int("FAR_PDL", 1) != 0 ? 1 : 0;
+  c.ring_min_rows = env_int("FAR_RING_MIN_ROWS", 0);  // 0: the measured rule
   c.force_regime = FAR_REGIME_AUTO;
   if (const char* f = std::getenv("FAR_FORCE_REGIME")) {
     if (std::strcmp(f, "decode") == 0) c.force_regime = FAR_REGIME_DECODE;

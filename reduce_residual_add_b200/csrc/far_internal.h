@@ -50,6 +50,7 @@ struct Launch {
   int64_t grid;         // CTAs
   int nslot;            // ring: shared-memory slots of one row segment each
   int smem_bytes;       // ring: dynamic shared memory per CTA
+  int pdl;              // launch with programmatic stream serialization
 };
 
 // Enqueue one kernel on `stream`.  Returns the launch error (cudaSuccess if

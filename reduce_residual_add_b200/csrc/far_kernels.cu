@@ -221,6 +221,16 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
       : "memory");
 }
 
+// Programmatic dependent launch (PTX griddepcontrol): wait until the grid
+// this launch depends on has completed and its writes are visible (a no-op
+// without that dependency), then let the next dependent grid be scheduled.
+// Called first thing in every kernel, so no input is read and no output is
+// written before the preceding work in the stream is done.
+__device__ __forceinline__ void pdl_enter() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // Barrier over the first `nthreads` threads of the CTA (the consumer warps).
 __device__ __forceinline__ void consumer_bar(int nthreads) {
   asm volatile("bar.sync 1, %0;" ::"r"(nthreads) : "memory");
@@ -501,6 +511,7 @@ __device__ __forceinline__ void fused_row(const Params& p, int64_t row, bool row
 template <class DT, int VPT, bool SUB>
 __global__ void __launch_bounds__(kMaxThreads, (VPT >= 8 ? 1 : 2))
 far_prefill_kernel(const Params p) {
+  pdl_enter();
   const int64_t row = p.row_begin + static_cast<int64_t>(blockIdx.x) * blockDim.y + threadIdx.y;
   const bool row_ok = row < p.row_end;
   if constexpr (SUB) {
@@ -518,6 +529,7 @@ far_prefill_kernel(const Params p) {
 template <class DT, int VPT>
 __global__ void __launch_bounds__(kMaxThreads, (VPT >= 8 ? 1 : 2))
 far_decode_kernel(const Params p) {
+  pdl_enter();
   __shared__ float s_sum[32], s_max[32], s_cta[2];
   cg::cluster_group cl = cg::this_cluster();
   const int rank = static_cast<int>(cl.block_rank());
@@ -550,6 +562,7 @@ far_decode_kernel(const Params p) {
 template <class DT, int VPT>
 __global__ void __launch_bounds__(kRingMaxConsumers + 32, 1)
 far_ring_kernel(const Params p, int nslot, int ncons) {
+  pdl_enter();
   extern __shared__ __align__(128) unsigned char smem[];
   uint64_t* full = reinterpret_cast<uint64_t*>(smem);
   uint64_t* empty = full + nslot;
@@ -655,44 +668,63 @@ far_ring_kernel(const Params p, int nslot, int ncons) {
   }
 }
 
+// Launch attributes: optional programmatic stream serialization (PDL) and
+// an optional cluster shape.
+struct Attrs {
+  cudaLaunchAttribute a[2];
+  unsigned n = 0;
+  Attrs(const Launch& l, int cluster) {
+    if (l.pdl) {
+      a[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+      a[n].val.programmaticStreamSerializationAllowed = 1;
+      ++n;
+    }
+    if (cluster > 0) {
+      a[n].id = cudaLaunchAttributeClusterDimension;
+      a[n].val.clusterDim.x = static_cast<unsigned>(cluster);
+      a[n].val.clusterDim.y = 1;
+      a[n].val.clusterDim.z = 1;
+      ++n;
+    }
+  }
+};
+
 template <class DT, int VPT, bool SUB>
 cudaError_t launch_prefill_t(const Params& p, const Launch& l, cudaStream_t s) {
+  Attrs at(l, 0);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(l.grid), 1, 1);
   cfg.blockDim = dim3(static_cast<unsigned>(l.tpr), static_cast<unsigned>(l.rows_per_cta), 1);
   cfg.dynamicSmemBytes = 0;
   cfg.stream = s;
-  cfg.attrs = nullptr;
-  cfg.numAttrs = 0;
+  cfg.attrs = at.a;
+  cfg.numAttrs = at.n;
   return cudaLaunchKernelEx(&cfg, far_prefill_kernel<DT, VPT, SUB>, p);
 }
 
 template <class DT, int VPT>
 cudaError_t launch_decode_t(const Params& p, const Launch& l, cudaStream_t s) {
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = static_cast<unsigned>(l.cluster);
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
+  Attrs at(l, l.cluster);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(l.cluster), static_cast<unsigned>(l.grid / l.cluster), 1);
   cfg.blockDim = dim3(static_cast<unsigned>(l.threads), 1, 1);
   cfg.dynamicSmemBytes = 0;
   cfg.stream = s;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.attrs = at.a;
+  cfg.numAttrs = at.n;
   return cudaLaunchKernelEx(&cfg, far_decode_kernel<DT, VPT>, p);
 }
 
 template <class DT, int VPT>
 cudaError_t launch_ring_t(const Params& p, const Launch& l, cudaStream_t s) {
+  Attrs at(l, 0);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(l.grid), 1, 1);
   cfg.blockDim = dim3(static_cast<unsigned>(l.threads), 1, 1);
   cfg.dynamicSmemBytes = static_cast<size_t>(l.smem_bytes);
   cfg.stream = s;
-  cfg.attrs = nullptr;
-  cfg.numAttrs = 0;
+  cfg.attrs = at.a;
+  cfg.numAttrs = at.n;
   return cudaLaunchKernelEx(&cfg, far_ring_kernel<DT, VPT>, p, l.nslot, l.tpr);
 }
 

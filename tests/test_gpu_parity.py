@@ -54,11 +54,12 @@ def _ctx_with_env(env):
 def kctx():
     """Contexts for each prefill kernel: the TMA ring (1 and 2 CTAs per SM)
     and the direct-load kernel."""
-    out = {"ring": _ctx_with_env({}),
-           "ring256": _ctx_with_env({"FAR_RING_THREADS": "256", "FAR_RING_CTAS_PER_SM": "1"}),
-           "ring512": _ctx_with_env({"FAR_RING_THREADS": "512", "FAR_RING_CTAS_PER_SM": "1"}),
-           "ring2": _ctx_with_env({"FAR_RING_CTAS_PER_SM": "2", "FAR_RING_THREADS": "256"}),
-           "ring4": _ctx_with_env({"FAR_RING_CTAS_PER_SM": "4", "FAR_RING_THREADS": "128"}),
+    any_rows = {"FAR_RING_MIN_ROWS": "1"}
+    out = {"ring": _ctx_with_env(dict(any_rows)),
+           "ring256": _ctx_with_env(dict(any_rows, FAR_RING_THREADS="256", FAR_RING_CTAS_PER_SM="1")),
+           "ring512": _ctx_with_env(dict(any_rows, FAR_RING_THREADS="512", FAR_RING_CTAS_PER_SM="1")),
+           "ring2": _ctx_with_env(dict(any_rows, FAR_RING_CTAS_PER_SM="2", FAR_RING_THREADS="256")),
+           "ring4": _ctx_with_env(dict(any_rows, FAR_RING_CTAS_PER_SM="4", FAR_RING_THREADS="128")),
            "direct": _ctx_with_env({"FAR_PREFILL_KERNEL": "0"})}
     for c in out.values():
         far.far_set_regime(c, far.FAR_REGIME_PREFILL)
@@ -344,3 +345,55 @@ def test_launch_plan(ctx):
     assert (c4["threads_per_cta"] - 32) * c4["packs_per_thread"] * 8 >= 8192
     tiny = far.far_describe_launch(ctx, 8, 64)
     assert tiny["regime"] == far.FAR_REGIME_PREFILL and tiny["rows_per_cta"] > 1
+
+
+@pytest.mark.parametrize("kern", ["decode", "ring", "direct"])
+def test_chained_calls_read_completed_outputs(kctx, ctx, kern):
+    """With programmatic dependent launch each call must still read what the
+    previous call wrote: call k+1 takes call k's new residual as its
+    residual, four times in a stream and four times inside a CUDA graph."""
+    H, W = 4096, 4
+    T = 4 if kern == "decode" else 600
+    c = ctx if kern == "decode" else kctx[kern]
+    inps = [random_inputs(W, T, H, seed=300 + k) for k in range(4)]
+    g = [to_gpu(i) for i in inps]
+    gam = g[0]["gamma"]
+    res0 = g[0]["residual"]
+
+    def chain(stream):
+        outs = []
+        res = res0
+        for k in range(4):
+            rout = torch.empty_like(res0)
+            nout = torch.empty_like(res0)
+            far.far_fused(c, g[k]["partials"], res, gam, 1e-6, 0.0, 0,
+                          residual_out=rout, norm_out=nout, stream=stream)
+            outs.append((rout, nout))
+            res = rout
+        return outs
+
+    s = torch.cuda.Stream()
+    outs = chain(s)
+    torch.cuda.synchronize()
+    gr = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(gr, stream=s):
+        gouts = chain(s)
+    with torch.cuda.stream(s):
+        gr.replay()
+    torch.cuda.synchronize()
+    far.far_check(c)
+    info = far.far_describe_launch(c, T, H)
+    assert (info["regime"], info["kernel"]) == {"decode": (1, 0), "ring": (2, 1), "direct": (2, 0)}[kern]
+    from reduce_residual_add_b200.inputs import as_u16
+    import oracle
+    gam16 = as_u16(inps[0]["gamma"].contiguous())
+    for run in (outs, gouts):
+        prev = as_u16(inps[0]["residual"])
+        for k in range(4):
+            ref = oracle.fused([as_u16(p) for p in inps[k]["partials"]], prev, gam16, "bf16",
+                               1e-6, 0.0, 0)
+            got_r = as_u16(run[k][0].cpu())
+            got_n = as_u16(run[k][1].cpu())
+            assert compare({"residual_out": got_r, "norm_out": got_n}, ref, "bf16") is not None
+            prev = got_r          # the next call reads exactly what this one wrote
+    del gr
