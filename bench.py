@@ -360,7 +360,7 @@ def run_far(args, world, rank, local):
     stream = torch.cuda.Stream(device=device)
     ctx = far.FarContext(local)
     case = Case(ctx, wl, inp, device, args.with_norm, stream)
-    launch = far.far_describe_launch(ctx, wl.T, wl.H, wl.torch_dtype)
+    launch = far.far_describe_launch(ctx, wl.T, wl.H, wl.torch_dtype, wl.W, wl.has_residual)
 
     case.time_steps(0, args.warmup, per_launch=False)
     barrier(world)
@@ -401,7 +401,8 @@ def run_far(args, world, rank, local):
                      "peak_source": "%s (MEASURED_PEAKS.json hbm_gbs)" % peak_kind
                                     if peak_kind == "measured" else "fallback 6.65 TB/s",
                      "traffic": profiled_traffic(wl.name),
-                     "kernel": "far_prefill_kernel" if launch["regime"] == 2 else "far_decode_kernel",
+                     "kernel": ("far_decode_kernel" if launch["regime"] == 1 else
+                                "far_ring_kernel" if launch["kernel"] == 1 else "far_prefill_kernel"),
                      "mean_launch_us": round(mean_launch * 1e6, 3)},
         "e2e": {"value": round(case.bytes / e2e_s / 1e9, 3), "unit": "GB/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,

@@ -90,14 +90,15 @@ typedef enum {
 } far_pattern;
 
 typedef enum {
-    FAR_REGIME_AUTO = 0,    /* decode when rows <= decode_max_rows, else prefill */
+    FAR_REGIME_AUTO = 0,    /* decode for rows <= decode_max_rows of large rows, else prefill */
     FAR_REGIME_DECODE = 1,  /* one thread-block cluster per row            */
     FAR_REGIME_PREFILL = 2  /* one CTA per row (or several rows per CTA)  */
 } far_regime;
 
 /* Opaque per-device context: caches the SM count, the compute capability
  * and the tuning knobs (read once from the environment in far_create:
- * FAR_DECODE_MAX_ROWS, FAR_FORCE_REGIME=decode|prefill, FAR_DECODE_CLUSTER,
+ * FAR_DECODE_MAX_ROWS, FAR_FORCE_REGIME=decode|prefill, FAR_DECODE_CLUSTER
+ * (CTAs per row; default by rule),
  * FAR_PREFILL_THREADS, FAR_PREFILL_KERNEL=1 ring | 0 direct,
  * FAR_RING_CTAS_PER_SM=1..4 (default 2), FAR_RING_THREADS: consumer threads
  * per ring CTA, at most 512 (default 256), FAR_RING_SLOTS: row-segment slots
@@ -197,9 +198,11 @@ far_status far_validate(int64_t row_begin, int64_t row_end,
  * (decode_max_rows < 0 keeps the current threshold). */
 far_status far_set_regime(far_ctx *ctx, far_regime regime, int decode_max_rows);
 
-/* Fill `info` with the launch geometry a call on `rows` rows would use. */
+/* Fill `info` with the launch geometry a call on `rows` rows of W partials
+ * (and a residual when has_residual != 0) would use. */
 far_status far_describe_launch(const far_ctx *ctx, int64_t rows, int64_t H,
-                               far_dtype dtype, far_launch_info *info);
+                               far_dtype dtype, int W, int has_residual,
+                               far_launch_info *info);
 
 /* Wait for `stream`, then read and clear the device-side error word of
  * ctx's device.  FAR_ERR_TIMEOUT: a bounded wait inside a kernel launched

@@ -165,18 +165,35 @@ bool plan_ring(const far_ctx* ctx, int packs, int64_t rows, int dtype, far::Laun
   return true;
 }
 
-far::Launch plan(const far_ctx* ctx, int64_t rows, int64_t H, int dtype) {
+// segs = row segments read per row: W partials, plus the residual if any.
+far::Launch plan(const far_ctx* ctx, int64_t rows, int64_t H, int dtype, int segs) {
   const int packs = static_cast<int>(H / far::kPackElems);
   far::Launch l{};
   bool decode;
-  if (ctx->force_regime == FAR_REGIME_DECODE)
+  if (ctx->force_regime == FAR_REGIME_DECODE) {
     decode = true;
-  else if (ctx->force_regime == FAR_REGIME_PREFILL)
+  } else if (ctx->force_regime == FAR_REGIME_PREFILL) {
     decode = false;
-  else
-    decode = rows <= ctx->decode_max_rows && packs >= 64;
+  } else {
+    // Measured on B200: with few rows a cluster per row beats one CTA per
+    // row once the CTA would hold >= 32 16-byte loads per thread (large
+    // rows); below that the single CTA's shorter path wins.
+    far::Launch d{};
+    plan_prefill(packs, ctx->prefill_threads, &d);
+    decode = rows <= ctx->decode_max_rows && packs >= 64 && segs * d.vpt >= 32;
+  }
   if (decode) {
-    plan_decode(packs, ctx->decode_cluster, &l);
+    int cl = ctx->decode_cluster;
+    if (cl <= 0) {
+      // measured: 4 CTAs per row from 32 rows up; below, at most 32 KiB of
+      // a row per CTA (8 at W=8 H=8192, 16 at H=16384)
+      cl = 4;
+      if (rows <= 16) {
+        const int64_t row_bytes = static_cast<int64_t>(segs) * H * 2;
+        while (cl < 16 && row_bytes > static_cast<int64_t>(cl) * 32 * 1024) cl *= 2;
+      }
+    }
+    plan_decode(packs, cl, &l);
     l.grid = rows * l.cluster;
   } else {
     plan_prefill(packs, ctx->prefill_threads, &l);
@@ -239,7 +256,7 @@ far_status far_create(far_ctx** ctx, int device) {
     return FAR_ERR_UNSUPPORTED;
   }
   c.decode_max_rows = env_int("FAR_DECODE_MAX_ROWS", 80);
-  c.decode_cluster = env_int("FAR_DECODE_CLUSTER", 4);
+  c.decode_cluster = env_int("FAR_DECODE_CLUSTER", 0);  // 0: the measured rule
   c.prefill_threads = env_int("FAR_PREFILL_THREADS", 256);
   if (c.prefill_threads < 32) c.prefill_threads = 32;
   if (c.prefill_threads > far::kMaxThreads) c.prefill_threads = far::kMaxThreads;
@@ -289,8 +306,9 @@ far_status far_set_regime(far_ctx* ctx, far_regime regime, int decode_max_rows) 
 }
 
 far_status far_describe_launch(const far_ctx* ctx, int64_t rows, int64_t H, far_dtype dtype,
-                               far_launch_info* info) {
+                               int W, int has_residual, far_launch_info* info) {
   if (ctx == nullptr || info == nullptr || rows < 0) return FAR_ERR_INVALID_ARG;
+  if (W < 1 || W > FAR_MAX_W) return FAR_ERR_INVALID_ARG;
   if (dtype != FAR_BF16 && dtype != FAR_FP16) return FAR_ERR_INVALID_ARG;
   if (H <= 0 || H % far::kPackElems != 0 || H > far::kMaxH) return FAR_ERR_UNSUPPORTED;
   int prev = -1;
@@ -298,7 +316,7 @@ far_status far_describe_launch(const far_ctx* ctx, int64_t rows, int64_t H, far_
   if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
   if (prev != ctx->device && (e = cudaSetDevice(ctx->device)) != cudaSuccess)
     return cuda_fail(e, "cudaSetDevice");
-  const far::Launch l = plan(ctx, rows, H, dtype);
+  const far::Launch l = plan(ctx, rows, H, dtype, W + (has_residual ? 1 : 0));
   if (prev != ctx->device) cudaSetDevice(prev);
   info->regime = l.regime;
   info->ctas_per_row = l.cluster;
@@ -435,7 +453,7 @@ far_status far_fused_rows(far_ctx* ctx, int64_t row_begin, int64_t row_end,
 
   // grid.y (decode) and grid.x (prefill) bound the rows of one launch
   const int64_t rows = row_end - row_begin;
-  const far::Launch whole = plan(ctx, rows, H, dtype);
+  const far::Launch whole = plan(ctx, rows, H, dtype, W + (residual != nullptr ? 1 : 0));
   const int64_t max_rows = whole.regime == FAR_REGIME_DECODE
                                ? 65535
                                : static_cast<int64_t>(0x7fffffff) * whole.rows_per_cta;

@@ -157,11 +157,13 @@ __device__ __forceinline__ uint4 ld_once_coherent(const uint4* p) {
 
 // Device-side error word of this library, one per device: bit 0 = a consumer
 // gave up waiting for a bulk copy, bit 1 = the producer gave up waiting for
-// a free slot.  Read and cleared by far_check().
+// a free slot, bit 2 = a cluster CTA gave up waiting for its peers' totals.
+// Read and cleared by far_check().
 __device__ unsigned int g_far_error = 0u;
 
 constexpr unsigned kErrWaitFull = 1u;
 constexpr unsigned kErrWaitEmpty = 2u;
+constexpr unsigned kErrWaitPeer = 4u;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // one wait gives up after 2 s
 
 __device__ __forceinline__ uint32_t smem_addr(const void* p) {
@@ -208,6 +210,24 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const 
   for (;;) {
     if (mbar_try_wait(bar, parity)) return true;
     if (abort != nullptr && *abort) return false;
+    if (global_ns() - t0 > kWaitLimitNs) return false;
+  }
+}
+
+// As mbar_wait, with cluster-scope acquire (peers arrive on this barrier
+// from other CTAs of the cluster); gives up after kWaitLimitNs.
+__device__ __forceinline__ bool mbar_wait_acquire_cluster(uint64_t* bar, uint32_t parity) {
+  const uint64_t t0 = global_ns();
+  for (;;) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(smem_addr(bar)), "r"(parity)
+        : "memory");
+    if (done) return true;
     if (global_ns() - t0 > kWaitLimitNs) return false;
   }
 }
@@ -290,35 +310,42 @@ struct BlockRed {
   __device__ bool leader() const { return threadIdx.x == 0; }
 };
 
-// A row over a thread-block cluster: CTA totals meet in distributed shared
-// memory.  Every CTA reads all ranks' totals in rank order, so every CTA
-// holds the same bits.  Each quantity has its own slot, so no slot is
-// rewritten while a peer may still read it; the kernel ends with one more
-// cluster barrier before any CTA (and its shared memory) goes away.
+// A row over a thread-block cluster.  Each CTA reduces its slice, then
+// pushes its totals into slot [rank] of every CTA's shared memory
+// (st.shared::cluster) and arrives on that CTA's mbarrier with release
+// semantics; each CTA waits (bounded) for all `ncta` arrivals on its own
+// mbarrier and reduces the slots in rank order, so every CTA holds the same
+// bits.  No CTA touches a peer's shared memory after that peer's arrival
+// count is complete, so none can read or write a CTA that has exited.  The
+// mbarriers are initialised before the cluster arrive that opens the
+// kernel, and the matching cluster wait comes before the first push.
 struct ClusterRed {
   BlockRed blk;
-  float* s_cta;  // [2]: 0 = sum of squares, 1 = max
-  __device__ float2 across(float2 t) const {
-    cg::cluster_group cl = cg::this_cluster();
-    if (threadIdx.x == 0) {
-      s_cta[0] = t.x;
-      s_cta[1] = t.y;
+  float* s_in;    // [2][16]: pushed sums and maxima, by source rank
+  uint64_t* bar;  // counts the ncta pushes
+  int ncta;
+  int rank;
+  __device__ float2 exchange(float2 t) const {
+    asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
+    if (threadIdx.x < static_cast<unsigned>(ncta)) {
+      const uint32_t dst = static_cast<uint32_t>(threadIdx.x);
+      uint32_t rs, rm, rb;
+      asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(rs) : "r"(smem_addr(s_in + rank)), "r"(dst));
+      asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(rm) : "r"(smem_addr(s_in + 16 + rank)), "r"(dst));
+      asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(rb) : "r"(smem_addr(bar)), "r"(dst));
+      asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(rs), "f"(t.x) : "memory");
+      asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(rm), "f"(t.y) : "memory");
+      asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(rb) : "memory");
     }
-    cl.sync();
+    if (!mbar_wait_acquire_cluster(bar, 0u)) atomicOr(&g_far_error, kErrWaitPeer);
     const int lane = threadIdx.x & 31;
-    const int n = static_cast<int>(cl.num_blocks());
-    float u = 0.f, w = 0.f;
-    if (lane < n) {
-      u = *cl.map_shared_rank(s_cta, lane);
-      w = *cl.map_shared_rank(s_cta + 1, lane);
-    }
+    const float u = lane < ncta ? s_in[lane] : 0.f;
+    const float w = lane < ncta ? s_in[16 + lane] : 0.f;
     return make_float2(group_sum(u, 32), group_max(w, 32));
   }
-  __device__ float sum(float v) const { return across(make_float2(blk.sum(v), 0.f)).x; }
-  __device__ float2 sum_max(float s, float m) const { return across(blk.sum_max(s, m)); }
-  __device__ bool leader() const {
-    return threadIdx.x == 0 && cg::this_cluster().block_rank() == 0;
-  }
+  __device__ float sum(float v) const { return exchange(make_float2(blk.sum(v), 0.f)).x; }
+  __device__ float2 sum_max(float s, float m) const { return exchange(blk.sum_max(s, m)); }
+  __device__ bool leader() const { return threadIdx.x == 0 && rank == 0; }
 };
 
 // A row over the consumer warps of the ring kernel (a named barrier that
@@ -530,18 +557,24 @@ template <class DT, int VPT>
 __global__ void __launch_bounds__(kMaxThreads, (VPT >= 8 ? 1 : 2))
 far_decode_kernel(const Params p) {
   pdl_enter();
-  __shared__ float s_sum[32], s_max[32], s_cta[2];
+  __shared__ float s_sum[32], s_max[32], s_in[32];
+  __shared__ uint64_t s_bar;
   cg::cluster_group cl = cg::this_cluster();
   const int rank = static_cast<int>(cl.block_rank());
   const int ncta = static_cast<int>(cl.num_blocks());
+  if (threadIdx.x == 0) {
+    mbar_init(&s_bar, static_cast<uint32_t>(ncta));
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
+  asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
   const int64_t row = p.row_begin + blockIdx.y;
   const int chunk = (p.packs + ncta - 1) / ncta;
   const int jbeg = rank * chunk;
   const int jend = min(p.packs, jbeg + chunk);
-  const ClusterRed red{BlockRed{s_sum, s_max}, s_cta};
+  const ClusterRed red{BlockRed{s_sum, s_max}, s_in, &s_bar, ncta, rank};
   fused_row<DT, VPT>(p, row, row < p.row_end, jbeg + static_cast<int>(threadIdx.x),
                      blockDim.x, jend, red);
-  cl.sync();  // keep this CTA's shared memory alive until every peer has read it
 }
 
 // Prefill through the TMA engine: a persistent CTA per SM (or two) walks

@@ -101,7 +101,7 @@ def lib() -> ctypes.CDLL:
     L.far_validate.restype = i32
     L.far_set_regime.argtypes = [vp, i32, i32]
     L.far_set_regime.restype = i32
-    L.far_describe_launch.argtypes = [vp, i64, i64, i32, ctypes.POINTER(far_launch_info)]
+    L.far_describe_launch.argtypes = [vp, i64, i64, i32, i32, i32, ctypes.POINTER(far_launch_info)]
     L.far_describe_launch.restype = i32
     L.far_check.argtypes = [vp, vp]
     L.far_check.restype = i32
@@ -175,10 +175,11 @@ def far_set_regime(ctx: FarContext, regime: int, decode_max_rows: int = -1) -> N
         raise FarError(st, "far_set_regime")
 
 
-def far_describe_launch(ctx: FarContext, rows: int, H: int, dtype=torch.bfloat16) -> dict:
+def far_describe_launch(ctx: FarContext, rows: int, H: int, dtype=torch.bfloat16, W: int = 8,
+                        has_residual: bool = True) -> dict:
     info = far_launch_info()
     st = lib().far_describe_launch(ctx.handle, int(rows), int(H), _DTYPES.get(dtype, dtype),
-                                   ctypes.byref(info))
+                                   int(W), int(bool(has_residual)), ctypes.byref(info))
     if st != FAR_OK:
         raise FarError(st, "far_describe_launch")
     return {name: getattr(info, name) for name, _ in far_launch_info._fields_}

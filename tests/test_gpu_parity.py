@@ -63,6 +63,8 @@ def kctx():
            "direct": _ctx_with_env({"FAR_PREFILL_KERNEL": "0"})}
     for c in out.values():
         far.far_set_regime(c, far.FAR_REGIME_PREFILL)
+    out["decode"] = _ctx_with_env({})
+    far.far_set_regime(out["decode"], far.FAR_REGIME_DECODE)
     yield out
     for c in out.values():
         c.close()
@@ -118,7 +120,7 @@ def test_small_shapes(ctx, regime, case, reg):
 def test_prefill_kernels(kctx, case, kern):
     W, T, H, dt, pattern, has_res, wb = case
     c = kctx[kern]
-    info = far.far_describe_launch(c, T, H, torch.bfloat16)
+    info = far.far_describe_launch(c, T, H, torch.bfloat16, W, has_res)
     per_sm = {"ring4": 4, "ring2": 2}.get(kern, 1)
     fits = 228 * 1024 // per_sm - 1024 >= 3 * H * 2 + 1024   # gamma, two slots, header
     assert info["kernel"] == (1 if (kern != "direct" and fits) else 0)
@@ -156,12 +158,13 @@ def test_small_workload_matches_golden_fixture(ctx):
 
 
 @pytest.mark.parametrize("T", [1, 8, 32, 80])
-@pytest.mark.parametrize("reg", [far.FAR_REGIME_AUTO, far.FAR_REGIME_PREFILL])
+@pytest.mark.parametrize("reg", [far.FAR_REGIME_AUTO, far.FAR_REGIME_DECODE, far.FAR_REGIME_PREFILL])
 def test_decode_workload(ctx, regime, T, reg):
     wl = WORKLOADS["c2_decode_T%d" % T]
     regime(reg)
-    if reg == far.FAR_REGIME_AUTO:
-        assert far.far_describe_launch(ctx, T, wl.H)["regime"] == far.FAR_REGIME_DECODE
+    info = far.far_describe_launch(ctx, T, wl.H, torch.bfloat16, wl.W, True)
+    if reg == far.FAR_REGIME_DECODE:
+        assert info["regime"] == far.FAR_REGIME_DECODE and info["ctas_per_row"] >= 2
     inp = make_inputs(wl)
     got = run_gpu(ctx, to_gpu(inp), wl.eps, wl.weight_bias, wl.pattern, guard=256)
     ref = run_oracle(inp, wl.dtype, wl.eps, wl.weight_bias, wl.pattern)
@@ -336,14 +339,22 @@ def test_errors_are_reported_not_skipped(ctx):
 
 
 def test_launch_plan(ctx):
-    d = far.far_describe_launch(ctx, 80, 4096)
-    assert d["regime"] == far.FAR_REGIME_DECODE and d["ctas_per_row"] >= 2
-    p = far.far_describe_launch(ctx, 81, 4096)
-    assert p["regime"] == far.FAR_REGIME_PREFILL
-    c4 = far.far_describe_launch(ctx, 8192, 8192)
+    """The measured dispatch rules (see far_abi.cu plan())."""
+    d = lambda rows, H, W, res=True: far.far_describe_launch(ctx, rows, H, torch.bfloat16, W, res)  # noqa: E731
+    # decode-sized rows: a cluster per row once rows are large ...
+    assert (d(4, 16384, 8)["regime"], d(4, 16384, 8)["ctas_per_row"]) == (far.FAR_REGIME_DECODE, 16)
+    assert (d(1, 8192, 8)["regime"], d(1, 8192, 8)["ctas_per_row"]) == (far.FAR_REGIME_DECODE, 8)
+    assert (d(64, 8192, 8)["regime"], d(64, 8192, 8)["ctas_per_row"]) == (far.FAR_REGIME_DECODE, 4)
+    # ... one CTA per row for smaller ones (W=8, H=4096: 18 loads per thread)
+    assert d(80, 4096, 8)["regime"] == far.FAR_REGIME_PREFILL
+    assert d(1, 4096, 2)["regime"] == far.FAR_REGIME_PREFILL
+    assert d(81, 16384, 8)["regime"] == far.FAR_REGIME_PREFILL
+    # prefill: the ring from ~8 rows per persistent CTA, the direct kernel below
+    c4 = d(8192, 8192, 4)
     assert c4["kernel"] == 1 and c4["ring_slots"] >= 2
     assert (c4["threads_per_cta"] - 32) * c4["packs_per_thread"] * 8 >= 8192
-    tiny = far.far_describe_launch(ctx, 8, 64)
+    assert d(1200, 8192, 4)["kernel"] == 0
+    tiny = d(8, 64, 2)
     assert tiny["regime"] == far.FAR_REGIME_PREFILL and tiny["rows_per_cta"] > 1
 
 
@@ -354,7 +365,7 @@ def test_chained_calls_read_completed_outputs(kctx, ctx, kern):
     residual, four times in a stream and four times inside a CUDA graph."""
     H, W = 4096, 4
     T = 4 if kern == "decode" else 600
-    c = ctx if kern == "decode" else kctx[kern]
+    c = kctx[kern]
     inps = [random_inputs(W, T, H, seed=300 + k) for k in range(4)]
     g = [to_gpu(i) for i in inps]
     gam = g[0]["gamma"]
@@ -382,7 +393,7 @@ def test_chained_calls_read_completed_outputs(kctx, ctx, kern):
         gr.replay()
     torch.cuda.synchronize()
     far.far_check(c)
-    info = far.far_describe_launch(c, T, H)
+    info = far.far_describe_launch(c, T, H, torch.bfloat16, W, True)
     assert (info["regime"], info["kernel"]) == {"decode": (1, 0), "ring": (2, 1), "direct": (2, 0)}[kern]
     from reduce_residual_add_b200.inputs import as_u16
     import oracle
