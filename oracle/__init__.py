@@ -15,6 +15,7 @@ sources and for the readings taken where the pages are silent):
     o    = y * rinv * (gamma + weight_bias)        (normed output)
     static FP8:  q = e4m3(fp32(fp32(o) / scale))
     per-token:   scale_t = fp32(max|fp32(o)| / 448); q = e4m3(fp32(fp32(o) / scale_t))
+    per-tensor:  one scale = fp32(max over the rows of |fp32(o)| / 448), in scale_out[0]
 """
 from __future__ import annotations
 
@@ -27,7 +28,7 @@ import numpy as np
 from . import build as _build
 
 BF16, FP16 = 0, 1
-AR_RESIDUAL_RMSNORM, FP8_STATIC, FP8_TOKEN = 0, 1, 2
+AR_RESIDUAL_RMSNORM, FP8_STATIC, FP8_TOKEN, FP8_TENSOR = 0, 1, 2, 3
 
 _lib = None
 
@@ -114,7 +115,7 @@ def fused(partials: Sequence[np.ndarray], residual: Optional[np.ndarray],
 
     Returns a dict with ``residual_out`` (uint16, T x H), ``norm_out``
     (uint16 or None), ``quant_out`` (uint8 or None), ``scale_out`` (float32
-    (T,) or None) and, with ``debug``, fp64 ``y``, ``o`` (T x H) and ``rinv`` (T,).
+    (T,) per token, (1,) per tensor, or None) and, with ``debug``, fp64 ``y``, ``o`` (T x H) and ``rinv`` (T,).
     """
     dt = dtype_code(dtype)
     gamma = np.ascontiguousarray(gamma, dtype=np.uint16).reshape(-1)
@@ -139,12 +140,14 @@ def fused(partials: Sequence[np.ndarray], residual: Optional[np.ndarray],
         o.setdefault("norm_out", np.zeros((T, H), np.uint16))
     else:
         o["norm_out"] = None
-    if pattern in (FP8_STATIC, FP8_TOKEN):
+    if pattern in (FP8_STATIC, FP8_TOKEN, FP8_TENSOR):
         o.setdefault("quant_out", np.zeros((T, H), np.uint8))
     else:
         o["quant_out"] = None
     if pattern == FP8_TOKEN:
         o.setdefault("scale_out", np.zeros((T,), np.float32))
+    elif pattern == FP8_TENSOR:
+        o.setdefault("scale_out", np.zeros((1,), np.float32))
     else:
         o["scale_out"] = None
     sin = None
@@ -169,6 +172,6 @@ def fused(partials: Sequence[np.ndarray], residual: Optional[np.ndarray],
     return o
 
 
-__all__ = ["BF16", "FP16", "AR_RESIDUAL_RMSNORM", "FP8_STATIC", "FP8_TOKEN",
+__all__ = ["BF16", "FP16", "AR_RESIDUAL_RMSNORM", "FP8_STATIC", "FP8_TOKEN", "FP8_TENSOR",
            "load", "lib", "dtype_code", "decode16", "round16", "e4m3_decode",
            "e4m3_encode", "fused"]

@@ -27,6 +27,9 @@
  *       FusedAddRMSNormDynamicQuantPattern (dynamic per-token FP8, returns
  *       result, residual and one scale per token; scale_ub=None); the QuantKey
  *       constants kFp8StaticTensorSym / kFp8DynamicTokenSym (symmetric).
+ *       The same page lists kFp8DynamicTensorSym (dynamic, per-tensor,
+ *       symmetric) among the quantisation keys, with no fused op: one scale
+ *       for the whole tensor, amax / 448 over every element.
  *  [P5] PR #45307 report -- signature of call_trtllm_fused_allreduce_norm:
  *       norm_out, quant_out, scale_out and scale_factor are all optional.
  *
@@ -50,7 +53,9 @@
  *    by the fp32 scale with one correct rounding to fp32, then encoded;
  *  - FP8 encoding saturates to +-448 (e4m3fn has no infinity);
  *  - a dynamic row whose fp32 scale is 0 gets scale 0 and all codes 0x00;
- *    NaN elements take no part in a row's amax.
+ *    NaN elements take no part in a row's amax;
+ *  - dynamic per-tensor FP8 takes its amax over the rows of the call
+ *    ([row_begin, row_end)) and writes the one scale to scale_out[0].
  */
 #include <math.h>
 #include <stddef.h>
@@ -60,7 +65,7 @@
 /* Own copies of the enumerations; numbering follows the library's public
  * interface so that callers can pass the same integers to both. */
 enum { OR_BF16 = 0, OR_FP16 = 1 };
-enum { OR_AR_RESIDUAL_RMSNORM = 0, OR_FP8_STATIC = 1, OR_FP8_TOKEN = 2 };
+enum { OR_AR_RESIDUAL_RMSNORM = 0, OR_FP8_STATIC = 1, OR_FP8_TOKEN = 2, OR_FP8_TENSOR = 3 };
 
 /* ---------------------------------------------------------------------- */
 /* 16-bit floating formats                                                 */
@@ -206,6 +211,36 @@ static double to_f32(double x) { return (double)(float)x; }
 /* The fused epilogue                                                      */
 /* ---------------------------------------------------------------------- */
 
+/* Row t: y = sum of the partials (+ residual) and o = y * rinv * (gamma +
+ * weight_bias), both in fp64 into y[H] and o[H]; returns rinv. */
+static double row_y_o(const uint16_t *const *partials, int W, const uint16_t *residual,
+                      const uint16_t *gamma, int64_t t, int64_t H, int dtype,
+                      float eps, float weight_bias, double *y, double *o)
+{
+    const int64_t base = t * H;
+    /* 1. all-reduce of the partials, then 2. the residual add [P1] */
+    for (int64_t h = 0; h < H; ++h) {
+        double s = 0.0;
+        for (int r = 0; r < W; ++r)
+            s += far_oracle_decode16(partials[r][base + h], dtype);
+        if (residual != NULL)
+            s += far_oracle_decode16(residual[base + h], dtype);
+        y[h] = s;
+    }
+    /* 3. mean of squares over the hidden size, eps inside the root */
+    double ss = 0.0;
+    for (int64_t h = 0; h < H; ++h)
+        ss += y[h] * y[h];
+    double ms = ss / (double)H;
+    double rinv = 1.0 / sqrt(ms + (double)eps); /* fp32 eps, promoted */
+    /* 4. scale by rinv and by (gamma + weight_bias) [P1] */
+    for (int64_t h = 0; h < H; ++h) {
+        double g = far_oracle_decode16(gamma[h], dtype) + (double)weight_bias;
+        o[h] = y[h] * rinv * g;
+    }
+    return rinv;
+}
+
 /*
  * Rows [row_begin, row_end) of a (T, H) problem; all arrays are row-major
  * with row stride H and are indexed by the absolute row.
@@ -217,7 +252,8 @@ static double to_f32(double x) { return (double)(float)x; }
  *   norm_out      receives round(o); may be NULL
  *   quant_out     receives e4m3 codes (patterns 1, 2); may be NULL
  *   scale_in      static per-tensor scale (pattern 1)
- *   scale_out     per-row fp32 scale (pattern 2), indexed by absolute row
+ *   scale_out     per-row fp32 scale (pattern 2), indexed by absolute row,
+ *                 or the one per-tensor scale in scale_out[0] (pattern 3)
  *   y_dbg, o_dbg  optional fp64 copies of y and o (T*H each)
  *   rinv_dbg      optional fp64 1/sqrt(ms+eps) per row (T)
  *
@@ -240,7 +276,8 @@ int far_oracle_fused(const uint16_t *const *partials, int W,
         return -1;
     if (pattern == OR_FP8_STATIC && (quant_out == NULL || scale_in == NULL))
         return -1;
-    if (pattern == OR_FP8_TOKEN && (quant_out == NULL || scale_out == NULL))
+    if ((pattern == OR_FP8_TOKEN || pattern == OR_FP8_TENSOR) &&
+        (quant_out == NULL || scale_out == NULL))
         return -1;
 
     /* one row of y and o at a time, in fp64 */
@@ -252,34 +289,26 @@ int far_oracle_fused(const uint16_t *const *partials, int W,
         return -1;
     }
 
-    const double e = (double)eps;          /* fp32 eps, promoted */
-    const double wb = (double)weight_bias; /* fp32 weight_bias, promoted */
+    /* dynamic per-tensor FP8: a first pass over the rows for the amax */
+    double tensor_scale = 0.0;
+    if (pattern == OR_FP8_TENSOR) {
+        double amax = 0.0;
+        for (int64_t t = row_begin; t < row_end; ++t) {
+            row_y_o(partials, W, residual, gamma, t, H, dtype, eps, weight_bias, y, o);
+            for (int64_t h = 0; h < H; ++h) {
+                double a = fabs(to_f32(o[h]));
+                if (a > amax) /* a NaN element does not take part */
+                    amax = a;
+            }
+        }
+        tensor_scale = to_f32(amax / 448.0);
+        scale_out[0] = (float)tensor_scale;
+    }
 
     for (int64_t t = row_begin; t < row_end; ++t) {
         const int64_t base = t * H;
-
-        /* 1. all-reduce of the partials, then 2. the residual add [P1] */
-        for (int64_t h = 0; h < H; ++h) {
-            double s = 0.0;
-            for (int r = 0; r < W; ++r)
-                s += far_oracle_decode16(partials[r][base + h], dtype);
-            if (residual != NULL)
-                s += far_oracle_decode16(residual[base + h], dtype);
-            y[h] = s;
-        }
-
-        /* 3. mean of squares over the hidden size, eps inside the root */
-        double ss = 0.0;
-        for (int64_t h = 0; h < H; ++h)
-            ss += y[h] * y[h];
-        double ms = ss / (double)H;
-        double rinv = 1.0 / sqrt(ms + e);
-
-        /* 4. scale by rinv and by (gamma + weight_bias) [P1] */
-        for (int64_t h = 0; h < H; ++h) {
-            double g = far_oracle_decode16(gamma[h], dtype) + wb;
-            o[h] = y[h] * rinv * g;
-        }
+        const double rinv = row_y_o(partials, W, residual, gamma, t, H, dtype, eps,
+                                    weight_bias, y, o);
 
         if (residual_out != NULL)
             for (int64_t h = 0; h < H; ++h)
@@ -311,6 +340,17 @@ int far_oracle_fused(const uint16_t *const *partials, int W,
                     quant_out[base + h] = 0x00;
                 else
                     quant_out[base + h] = far_oracle_e4m3_encode(to_f32(to_f32(o[h]) / scale));
+            }
+        }
+
+        /* 5c. dynamic per-tensor FP8 [P4 kFp8DynamicTensorSym]: the one
+         * scale of the first pass */
+        if (pattern == OR_FP8_TENSOR) {
+            for (int64_t h = 0; h < H; ++h) {
+                if (tensor_scale == 0.0)
+                    quant_out[base + h] = 0x00;
+                else
+                    quant_out[base + h] = far_oracle_e4m3_encode(to_f32(to_f32(o[h]) / tensor_scale));
             }
         }
 

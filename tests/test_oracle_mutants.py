@@ -25,14 +25,15 @@ MUTANTS = {
     "last partial dropped": ("for (int r = 0; r < W; ++r)", "for (int r = 0; r < W - 1; ++r)"),
     "partial column shifted": ("partials[r][base + h]", "partials[r][base + (h + r) % H]"),
     "mean over H-1": ("ss / (double)H", "ss / (double)(H - 1)"),
-    "eps outside the root": ("1.0 / sqrt(ms + e)", "1.0 / (sqrt(ms) + e)"),
-    "eps dropped": ("1.0 / sqrt(ms + e)", "1.0 / sqrt(ms)"),
-    "rms instead of 1/rms": ("1.0 / sqrt(ms + e)", "sqrt(ms + e)"),
-    "eps in double, not its fp32 value": ("const double e = (double)eps;", "const double e = eps == 1e-6f ? 1e-6 : (double)eps;"),
-    "weight_bias ignored": ("const double wb = (double)weight_bias;", "const double wb = 0.0;"),
-    "weight_bias subtracted": ("far_oracle_decode16(gamma[h], dtype) + wb", "far_oracle_decode16(gamma[h], dtype) - wb"),
+    "eps outside the root": ("1.0 / sqrt(ms + (double)eps)", "1.0 / (sqrt(ms) + (double)eps)"),
+    "eps dropped": ("1.0 / sqrt(ms + (double)eps)", "1.0 / sqrt(ms)"),
+    "rms instead of 1/rms": ("1.0 / sqrt(ms + (double)eps)", "sqrt(ms + (double)eps)"),
+    "eps in double, not its fp32 value": ("1.0 / sqrt(ms + (double)eps)", "1.0 / sqrt(ms + (eps == 1e-6f ? 1e-6 : (double)eps))"),
+    "weight_bias ignored": ("far_oracle_decode16(gamma[h], dtype) + (double)weight_bias", "far_oracle_decode16(gamma[h], dtype) + 0.0"),
+    "weight_bias subtracted": ("far_oracle_decode16(gamma[h], dtype) + (double)weight_bias", "far_oracle_decode16(gamma[h], dtype) - (double)weight_bias"),
     "gamma reversed": ("gamma[h]", "gamma[H - 1 - h]"),
-    "row offset relative to the slice": ("const int64_t base = t * H;", "const int64_t base = (t - row_begin) * H;"),
+    "row offset relative to the slice": ("        const int64_t base = t * H;\n        const double rinv = row_y_o(",
+                                         "        const int64_t base = (t - row_begin) * H;\n        const double rinv = row_y_o("),
     "16-bit rounding truncates": ("double v = nearbyint(a / quantum) * quantum; /* a/quantum is exact */",
                                   "double v = floor(a / quantum) * quantum;"),
     "16-bit subnormals flushed": ("    if (be < f.emin)\n        be = f.emin;       /* below the normal range the spacing is fixed */\n",
@@ -48,6 +49,10 @@ MUTANTS = {
     "amax without abs": ("double a = fabs(to_f32(o[h]));", "double a = to_f32(o[h]);"),
     "static code decided in fp64": ("far_oracle_e4m3_encode(to_f32(to_f32(o[h]) / s32))", "far_oracle_e4m3_encode(o[h] / s32)"),
     "dynamic code decided in fp64": ("far_oracle_e4m3_encode(to_f32(to_f32(o[h]) / scale))", "far_oracle_e4m3_encode(o[h] / scale)"),
+    "per-tensor code decided in fp64": ("far_oracle_e4m3_encode(to_f32(to_f32(o[h]) / tensor_scale))", "far_oracle_e4m3_encode(o[h] / tensor_scale)"),
+    "per-tensor amax of the first row only": ("            row_y_o(partials, W, residual, gamma, t, H, dtype, eps, weight_bias, y, o);\n            for (int64_t h = 0; h < H; ++h) {",
+                                              "            row_y_o(partials, W, residual, gamma, t, H, dtype, eps, weight_bias, y, o);\n            if (t > row_begin) break;\n            for (int64_t h = 0; h < H; ++h) {"),
+    "per-tensor scale over 240": ("tensor_scale = to_f32(amax / 448.0);", "tensor_scale = to_f32(amax / 240.0);"),
     "y squared without the residual": ("ss += y[h] * y[h];", "ss += (y[h] - (residual ? far_oracle_decode16(residual[base + h], dtype) : 0.0)) * (y[h] - (residual ? far_oracle_decode16(residual[base + h], dtype) : 0.0));"),
 }
 
@@ -55,16 +60,19 @@ MUTANTS = {
 def quick_pins():
     """A subset of the pins that runs in a second or two."""
     for dt in ("bf16", "fp16"):
-        for pattern in (0, 1, 2):
+        for pattern in (0, 1, 2, 3):
             for shape in ((2, 8, 4), (3, 5, 4), (1, 4, 32)):
                 yield "brute force %s %s %s" % (shape, pattern, dt), lambda s=shape, p=pattern, d=dt: pins.test_brute_force_exact_tiny(s, p, d)
-    for pattern in (0, 1, 2):
+    for pattern in (0, 1, 2, 3):
         yield "brute force gemma / no residual %d" % pattern, lambda p=pattern: pins.test_brute_force_exact_gemma_and_no_residual(p)
     yield "worked standard + static", pins.test_worked_example_standard_and_static_fp8
     yield "worked gemma + dynamic", pins.test_worked_example_gemma_and_dynamic_fp8
     yield "worked tie to even", pins.test_worked_example_fp8_tie_to_even
     yield "worked fp32 decision", pins.test_worked_example_fp8_code_decided_in_fp32
     yield "worked fp32 decision dynamic", pins.test_worked_example_dynamic_fp8_code_decided_in_fp32
+    yield "worked per-tensor", pins.test_worked_example_per_tensor_fp8
+    for dt in ("bf16", "fp16"):
+        yield "per-tensor vs per-token %s" % dt, lambda d=dt: pins.test_per_tensor_scale_is_the_largest_per_token_scale(d)
     yield "worked zeros", pins.test_worked_example_zero_input_scale_one
     yield "worked saturation", pins.test_worked_example_saturation_and_zero_row_dynamic
     for dt in ("bf16", "fp16"):

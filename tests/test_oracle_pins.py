@@ -191,6 +191,7 @@ def exact_fused(ps, res, gam, dt, eps, wb, pattern, scale_in=None):
     epsq, wbq = f32(eps), f32(wb)
     g = [decode(int(b), dt) + wbq for b in gam]
     out = {"residual_out": [], "norm_out": [], "quant_out": [], "scale_out": []}
+    rows = []
     for t in range(T):
         y = []
         for h in range(H):
@@ -225,6 +226,16 @@ def exact_fused(ps, res, gam, dt, eps, wb, pattern, scale_in=None):
                 out["quant_out"].append([0] * H)
             else:
                 out["quant_out"].append([encode(e4m3_sat(rne(v / sc, "fp32")), "e4m3") for v in o32])
+        rows.append(o32)
+    if pattern == oracle.FP8_TENSOR:
+        # one scale: amax over every row of the call
+        assert all(v is not None for r in rows for v in r)
+        amax = max(abs(v) for r in rows for v in r)
+        sc = rne(amax / 448, "fp32")
+        out["scale_out"] = [sc]
+        for r in rows:
+            out["quant_out"].append([0] * H if sc == 0 else
+                                    [encode(e4m3_sat(rne(v / sc, "fp32")), "e4m3") for v in r])
     return out
 
 
@@ -253,14 +264,14 @@ def _compare_exact(inp, dt, eps, wb, pattern, scale_in=None):
                     continue
                 a = int(got["quant_out"][t, h])
                 assert (a if a & 0x7F else 0) == (v if v & 0x7F else 0), (t, h, hex(a), hex(v))
-    if pattern == oracle.FP8_TOKEN:
+    if pattern in (oracle.FP8_TOKEN, oracle.FP8_TENSOR):
         for t, sc in enumerate(ex["scale_out"]):
             assert Fraction(float(got["scale_out"][t])) == sc
     assert n_amb == 0
 
 
 @pytest.mark.parametrize("dt", ["bf16", "fp16"])
-@pytest.mark.parametrize("pattern", [0, 1, 2])
+@pytest.mark.parametrize("pattern", [0, 1, 2, 3])
 @pytest.mark.parametrize("shape", [(2, 8, 4), (1, 5, 4), (3, 5, 4), (2, 8, 64)])
 def test_brute_force_exact_tiny(shape, pattern, dt):
     """Tracing shapes [1, 8, 4] (sequence_parallelism patterns), (5, 4)
@@ -270,7 +281,7 @@ def test_brute_force_exact_tiny(shape, pattern, dt):
     _compare_exact(inp, dt, eps=1e-6, wb=0.0, pattern=pattern, scale_in=0.05)
 
 
-@pytest.mark.parametrize("pattern", [0, 1, 2])
+@pytest.mark.parametrize("pattern", [0, 1, 2, 3])
 def test_brute_force_exact_gemma_and_no_residual(pattern):
     inp = random_inputs(2, 6, 16, dtype="bf16", seed=77)
     _compare_exact(inp, "bf16", eps=1e-5, wb=1.0, pattern=pattern, scale_in=0.02)
@@ -373,6 +384,47 @@ def test_worked_example_dynamic_fp8_code_decided_in_fp32():
     assert r["scale_out"][0] == np.float32(2.0 ** -8)
     assert r["o"][0, 1] * 256 > 17
     assert r["quant_out"][0].tolist() == [0x7E, 0x58, 0x74, 0x70]
+
+
+def test_worked_example_per_tensor_fp8():
+    # two rows with the eps of the dynamic example (mean + eps = 4 - 2^-27,
+    # rinv = 1/2 (1 + 2^-30 + ...)): row 0 = [3.5, 17/128, 1.5, 1], row 1 =
+    # [-1, 1.5, 3.5, -17/128].  fp32(o): [1.75, 17/256, 0.75, 0.5] and
+    # [-0.5, 0.75, 1.75, -17/256]; the tensor amax is 1.75 and the one scale
+    # 1.75/448 = 2^-8.  o/scale: [448, 17, 192, 128] -> 0x7E, 0x58 (the tie
+    # 17 goes to the even 16 in fp32; fp64 would give 18), 0x74, 0x70; and
+    # [-128, 192, 448, -17] -> 0xF0, 0x74, 0x7E, 0xD8.
+    eps = 7903 / 65536 - 2.0 ** -27
+    rows = np.concatenate([_bits([3.5, 17 / 128, 1.5, 1.0]), _bits([-1.0, 1.5, 3.5, -17 / 128])])
+    r = oracle.fused([rows], None, _bits([1, 1, 1, 1])[0], "bf16", eps=eps,
+                     pattern=oracle.FP8_TENSOR)
+    assert r["scale_out"].tolist() == [2.0 ** -8]
+    assert r["quant_out"][0].tolist() == [0x7E, 0x58, 0x74, 0x70]
+    assert r["quant_out"][1].tolist() == [0xF0, 0x74, 0x7E, 0xD8]
+
+
+@pytest.mark.parametrize("dt", ["bf16", "fp16"])
+def test_per_tensor_scale_is_the_largest_per_token_scale(dt):
+    """max_t fp32(amax_t / 448) = fp32(max_t amax_t / 448) (rounding is
+    monotonic): the per-tensor scale equals the largest per-token scale bit
+    for bit, the row attaining it gets the same codes under both patterns,
+    and the tensor holds a +-448 code."""
+    wl = WORKLOADS["c5_gemma_fp8_token_%s" % dt].with_(T=40)   # same distributions, 40 rows
+    inp = make_inputs(wl)
+    args = ([as_u16(p) for p in inp["partials"]], as_u16(inp["residual"]), as_u16(inp["gamma"]),
+            dt, wl.eps, wl.weight_bias)
+    tok = oracle.fused(*args, oracle.FP8_TOKEN)
+    ten = oracle.fused(*args, oracle.FP8_TENSOR)
+    assert ten["scale_out"][0] == tok["scale_out"].max()
+    t = int(np.argmax(tok["scale_out"]))
+    np.testing.assert_array_equal(ten["quant_out"][t], tok["quant_out"][t])
+    assert np.any((ten["quant_out"] & 0x7F) == 0x7E)
+    # every other row is quantised more coarsely than alone: |codes| never above its own
+    assert np.all((ten["quant_out"] & 0x7F) <= (tok["quant_out"] & 0x7F))
+    np.testing.assert_array_equal(ten["residual_out"], tok["residual_out"])
+    # the row range sets the tensor: rows [10, 20) only
+    part = oracle.fused(*args, oracle.FP8_TENSOR, rows=(10, 20))
+    assert part["scale_out"][0] == tok["scale_out"][10:20].max()
 
 
 def test_worked_example_zero_input_scale_one():
