@@ -52,10 +52,12 @@ def algorithmic_bytes(wl: Workload, rows: int, with_norm: bool) -> int:
     b += T * H * 2              # new residual out
     if with_norm:
         b += T * H * 2
-    if wl.pattern in (1, 2):
+    if wl.pattern in (1, 2, 3):
         b += T * H             # e4m3 codes
     if wl.pattern == 2:
         b += 4 * T             # per-token scales
+    if wl.pattern == 3:
+        b += 4                 # the one per-tensor scale
     return b
 
 
@@ -221,12 +223,22 @@ class Case:
         self.rout = torch.empty(T, H, dtype=dt, device=device)
         self.nout = torch.empty(T, H, dtype=dt, device=device) if (with_norm or wl.pattern == 0) else None
         self.qout = torch.empty(T, H, dtype=torch.uint8, device=device) if wl.pattern else None
-        self.sout = torch.empty(T, dtype=torch.float32, device=device) if wl.pattern == 2 else None
+        self.sout = (torch.empty(T if wl.pattern == 2 else 1, dtype=torch.float32, device=device)
+                     if wl.pattern in (2, 3) else None)
+        self.ws = (torch.empty(far.far_fp8_tensor_workspace_bytes(T), dtype=torch.uint8, device=device)
+                   if wl.pattern == 3 else None)
         self.sin = (torch.tensor([wl.static_scale], dtype=torch.float32, device=device)
                     if wl.pattern == 1 else None)
         self.bytes = algorithmic_bytes(wl, T, self.nout is not None)
 
     def step(self):
+        if self.wl.pattern == 3:
+            self.far.far_fused_fp8_tensor(self.ctx, self.ps, self.res, self.gam, self.wl.eps,
+                                          self.wl.weight_bias, quant_out=self.qout,
+                                          scale_out=self.sout, workspace=self.ws,
+                                          residual_out=self.rout, norm_out=self.nout,
+                                          stream=self.stream)
+            return
         self.far.far_fused(self.ctx, self.ps, self.res, self.gam, self.wl.eps,
                            self.wl.weight_bias, self.wl.pattern, residual_out=self.rout,
                            norm_out=self.nout, quant_out=self.qout, scale_in=self.sin,
@@ -425,12 +437,14 @@ def extras(ctx, device, stream) -> dict:
     from reduce_residual_add_b200 import far
     out = {}
     peak, _ = hbm_peak()
-    for name in ("c5_gemma_fp8_token_bf16", "c5_gemma_fp8_token_fp16", "c3_3d"):
+    for name in ("c5_gemma_fp8_token_bf16", "c5_gemma_fp8_token_fp16", "c4_prefill_fp8_tensor",
+                 "c3_3d"):
         wl = WORKLOADS[name]
         inp = make_inputs(wl)
         case = Case(ctx, wl, inp, device, False, stream)
         total, mean = case.time_steps(200, 20, per_launch=True)
         out[name] = {"GB/s": round(case.bytes / mean / 1e9, 1),
+                     "launches_per_call": 2 if wl.pattern == 3 else 1,
                      "frac": round(case.bytes / mean / 1e9 / peak, 4),
                      "us_per_call": round(mean * 1e6, 2), "tokens_per_s": round(wl.T / mean, 1),
                      "bytes": case.bytes}

@@ -86,7 +86,10 @@ typedef enum {
     /* + quant_out, reading the fp32 scalar scale_in[0]; norm_out optional */
     FAR_AR_RESIDUAL_RMSNORM_FP8_STATIC = 1,
     /* + quant_out and scale_out[T] (one fp32 scale per row); norm_out optional */
-    FAR_AR_RESIDUAL_RMSNORM_FP8_TOKEN = 2
+    FAR_AR_RESIDUAL_RMSNORM_FP8_TOKEN = 2,
+    /* + quant_out and scale_out[0] (one fp32 scale for all rows of the call);
+     * only through far_fused_fp8_tensor, which takes a workspace */
+    FAR_AR_RESIDUAL_RMSNORM_FP8_TENSOR = 3
 } far_pattern;
 
 typedef enum {
@@ -156,6 +159,8 @@ far_status far_destroy(far_ctx *ctx);
  *  quant_out     (T, H) uint8 e4m3fn codes; required by the FP8 patterns.
  *  scale_in      device pointer to one fp32 (static FP8 only).
  *  scale_out     device array of T fp32 (per-token FP8 only).
+ *  pattern       FAR_AR_RESIDUAL_RMSNORM_FP8_TENSOR is refused here
+ *                (FAR_ERR_INVALID_ARG): use far_fused_fp8_tensor.
  *  stream        a cudaStream_t (NULL: the legacy default stream).
  *
  * Tensor pointers must be 16-byte aligned, scale pointers 4-byte aligned.
@@ -184,8 +189,39 @@ far_status far_fused_rows(far_ctx *ctx, int64_t row_begin, int64_t row_end,
                           void *norm_out, void *quant_out,
                           const float *scale_in, float *scale_out, void *stream);
 
+/* Bytes of workspace far_fused_fp8_tensor needs for `rows` rows:
+ * 256 + 4*rows, rounded up to 256. */
+size_t far_fp8_tensor_workspace_bytes(int64_t rows);
+
+/*
+ * Dynamic per-tensor FP8 (vllm.compilation.fusion, the kFp8DynamicTensorSym
+ * quantisation key: symmetric, dynamic, one scale per tensor; the page has
+ * no fused op for it): the epilogue on rows [row_begin, row_end) of a T-row
+ * problem, with ONE fp32 scale = max |o| over all those rows / 448, written
+ * to scale_out[0], and quant_out = e4m3_satfinite(o / scale).  Other
+ * arguments as far_fused_rows; residual_out, norm_out as there.
+ *
+ * The scale needs every row before any code, so the call enqueues a memset
+ * of the workspace's first word and two kernels: the first reads the inputs
+ * and keeps each row's 1/rms and the running amax in `workspace`, the second
+ * reads the inputs again and writes every output.  Inputs are therefore read
+ * twice.  `workspace`: device memory of at least
+ * far_fp8_tensor_workspace_bytes(row_end - row_begin) bytes, 256-byte
+ * aligned, overlapping no argument; its contents are scratch, and two calls
+ * that share a workspace must not overlap on the GPU.
+ */
+far_status far_fused_fp8_tensor(far_ctx *ctx, int64_t row_begin, int64_t row_end,
+                                const void *const *partials, int W,
+                                const void *residual, void *residual_out,
+                                const void *gamma, int64_t T, int64_t H, far_dtype dtype,
+                                float eps, float weight_bias,
+                                void *norm_out, void *quant_out, float *scale_out,
+                                void *workspace, size_t workspace_bytes, void *stream);
+
 /* Host-only: the status far_fused_rows would return for these arguments
- * before launching (it touches no GPU and needs no context). */
+ * before launching (it touches no GPU and needs no context).  With pattern
+ * FAR_AR_RESIDUAL_RMSNORM_FP8_TENSOR it checks far_fused_fp8_tensor's
+ * arguments other than the workspace. */
 far_status far_validate(int64_t row_begin, int64_t row_end,
                         const void *const *partials, int W,
                         const void *residual, const void *residual_out,

@@ -360,7 +360,7 @@ far_status far_validate(int64_t row_begin, int64_t row_end, const void* const* p
   if (T < 0 || H <= 0) return FAR_ERR_INVALID_ARG;
   if (dtype != FAR_BF16 && dtype != FAR_FP16) return FAR_ERR_INVALID_ARG;
   if (pattern != FAR_AR_RESIDUAL_RMSNORM && pattern != FAR_AR_RESIDUAL_RMSNORM_FP8_STATIC &&
-      pattern != FAR_AR_RESIDUAL_RMSNORM_FP8_TOKEN)
+      pattern != FAR_AR_RESIDUAL_RMSNORM_FP8_TOKEN && pattern != FAR_AR_RESIDUAL_RMSNORM_FP8_TENSOR)
     return FAR_ERR_INVALID_ARG;
   if (H % far::kPackElems != 0 || H > FAR_MAX_H) return FAR_ERR_UNSUPPORTED;
   if (row_begin < 0 || row_end < row_begin || row_end > T) return FAR_ERR_INVALID_ARG;
@@ -373,7 +373,8 @@ far_status far_validate(int64_t row_begin, int64_t row_end, const void* const* p
   if (pattern == FAR_AR_RESIDUAL_RMSNORM && norm_out == nullptr) return FAR_ERR_INVALID_ARG;
   if (pattern == FAR_AR_RESIDUAL_RMSNORM_FP8_STATIC && (quant_out == nullptr || scale_in == nullptr))
     return FAR_ERR_INVALID_ARG;
-  if (pattern == FAR_AR_RESIDUAL_RMSNORM_FP8_TOKEN && (quant_out == nullptr || scale_out == nullptr))
+  if ((pattern == FAR_AR_RESIDUAL_RMSNORM_FP8_TOKEN || pattern == FAR_AR_RESIDUAL_RMSNORM_FP8_TENSOR) &&
+      (quant_out == nullptr || scale_out == nullptr))
     return FAR_ERR_INVALID_ARG;
 
   // 16-byte packs everywhere; fp32 scales need 4 bytes.
@@ -396,6 +397,7 @@ far_status far_validate(int64_t row_begin, int64_t row_end, const void* const* p
     if (norm_out != nullptr) outs[no++] = span(norm_out, tb);
     if (pattern != FAR_AR_RESIDUAL_RMSNORM) outs[no++] = span(quant_out, T * H);
     if (pattern == FAR_AR_RESIDUAL_RMSNORM_FP8_TOKEN) outs[no++] = span(scale_out, T * 4);
+    if (pattern == FAR_AR_RESIDUAL_RMSNORM_FP8_TENSOR) outs[no++] = span(scale_out, 4);
     Range ins[FAR_MAX_W + 3];
     int ni = 0;
     for (int r = 0; r < W; ++r) ins[ni++] = span(partials[r], tb);
@@ -416,19 +418,14 @@ far_status far_validate(int64_t row_begin, int64_t row_end, const void* const* p
   return FAR_OK;
 }
 
-far_status far_fused_rows(far_ctx* ctx, int64_t row_begin, int64_t row_end,
-                          const void* const* partials, int W, const void* residual,
-                          void* residual_out, const void* gamma, int64_t T, int64_t H,
-                          far_dtype dtype, float eps, float weight_bias, far_pattern pattern,
-                          void* norm_out, void* quant_out, const float* scale_in, float* scale_out,
-                          void* stream) {
-  if (ctx == nullptr) return FAR_ERR_INVALID_ARG;
-  far_status st = far_validate(row_begin, row_end, partials, W, residual, residual_out, gamma, T, H,
-                               dtype, eps, weight_bias, pattern, norm_out, quant_out, scale_in,
-                               scale_out);
-  if (st != FAR_OK) return st;
-  if (row_end == row_begin) return FAR_OK;
+}  // extern "C"
 
+namespace {
+
+far::Params make_params(const void* const* partials, int W, const void* residual,
+                        void* residual_out, const void* gamma, int64_t H, far_pattern pattern,
+                        float eps, float weight_bias, void* norm_out, void* quant_out,
+                        const float* scale_in, float* scale_out) {
   far::Params p{};
   for (int r = 0; r < W; ++r) p.partials[r] = partials[r];
   p.residual = residual;
@@ -444,20 +441,17 @@ far_status far_fused_rows(far_ctx* ctx, int64_t row_begin, int64_t row_end,
   p.pattern = static_cast<int>(pattern);
   p.eps = eps;
   p.weight_bias = weight_bias;
+  return p;
+}
 
-  int prev = -1;
-  cudaError_t e = cudaGetDevice(&prev);
-  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
-  if (prev != ctx->device && (e = cudaSetDevice(ctx->device)) != cudaSuccess)
-    return cuda_fail(e, "cudaSetDevice");
-
-  // grid.y (decode) and grid.x (prefill) bound the rows of one launch
-  const int64_t rows = row_end - row_begin;
-  const far::Launch whole = plan(ctx, rows, H, dtype, W + (residual != nullptr ? 1 : 0));
+// Enqueue the kernels of rows [row_begin, row_end) with plan `whole`, in as
+// many launches as the grid limits need (grid.y for decode clusters).
+cudaError_t launch_rows(far::Params p, int dtype, const far::Launch& whole, int64_t row_begin,
+                        int64_t row_end, cudaStream_t s) {
   const int64_t max_rows = whole.regime == FAR_REGIME_DECODE
                                ? 65535
                                : static_cast<int64_t>(0x7fffffff) * whole.rows_per_cta;
-  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaSuccess;
   for (int64_t b = row_begin; b < row_end && e == cudaSuccess; b += max_rows) {
     const int64_t n = (row_end - b < max_rows) ? (row_end - b) : max_rows;
     far::Launch l = whole;
@@ -476,9 +470,127 @@ far_status far_fused_rows(far_ctx* ctx, int64_t row_begin, int64_t row_end,
     else
       e = far::launch_prefill(p, dtype, l, s);
   }
-  if (prev != ctx->device) cudaSetDevice(prev);
+  return e;
+}
+
+// Makes ctx's device current for the lifetime of the object.
+struct DeviceGuard {
+  int prev = -1;
+  int dev;
+  cudaError_t err = cudaSuccess;
+  explicit DeviceGuard(int device) : dev(device) {
+    err = cudaGetDevice(&prev);
+    if (err == cudaSuccess && prev != dev) err = cudaSetDevice(dev);
+  }
+  ~DeviceGuard() {
+    if (prev >= 0 && prev != dev) cudaSetDevice(prev);
+  }
+};
+
+// The per-tensor path once its arguments are checked: zero the amax word,
+// pass 1 (rinv of every row, the call's amax), pass 2 (every output).  The
+// workspace holds the amax word at byte 0 and rinv[rows] from byte 256.
+far_status far_fused_fp8_tensor_launch(far_ctx* ctx, int64_t row_begin, int64_t row_end,
+                                       const void* const* partials, int W, const void* residual,
+                                       void* residual_out, const void* gamma, int64_t H,
+                                       far_dtype dtype, float eps, float weight_bias,
+                                       void* norm_out, void* quant_out, float* scale_out,
+                                       void* workspace, void* stream) {
+  far::Params p = make_params(partials, W, residual, residual_out, gamma, H,
+                              FAR_AR_RESIDUAL_RMSNORM_FP8_TENSOR, eps, weight_bias, norm_out,
+                              quant_out, nullptr, scale_out);
+  p.ws_amax = static_cast<unsigned*>(workspace);
+  p.ws_rinv = reinterpret_cast<float*>(static_cast<unsigned char*>(workspace) + 256);
+  p.ws_row0 = row_begin;
+  DeviceGuard guard(ctx->device);
+  if (guard.err != cudaSuccess) return cuda_fail(guard.err, "cudaSetDevice");
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  // per-tensor: never the cluster kernel (no reduction in the second pass)
+  far::Launch whole = plan(ctx, row_end - row_begin, H, dtype, W + (residual != nullptr ? 1 : 0));
+  if (whole.regime == FAR_REGIME_DECODE) {
+    plan_prefill(static_cast<int>(H / far::kPackElems), ctx->prefill_threads, &whole);
+    whole.grid = (row_end - row_begin + whole.rows_per_cta - 1) / whole.rows_per_cta;
+    whole.pdl = ctx->pdl;
+  }
+  cudaError_t e = cudaMemsetAsync(workspace, 0, sizeof(unsigned), s);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync");
+  far::Launch first = whole;
+  first.pdl = 0;  // it must see the memset above
+  p.pattern = far::kTensorAmax;
+  e = launch_rows(p, dtype, first, row_begin, row_end, s);
+  if (e != cudaSuccess) return cuda_fail(e, "kernel launch (per-tensor pass 1)");
+  p.pattern = far::kTensorQuant;
+  e = launch_rows(p, dtype, whole, row_begin, row_end, s);
+  if (e != cudaSuccess) return cuda_fail(e, "kernel launch (per-tensor pass 2)");
+  return FAR_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+far_status far_fused_rows(far_ctx* ctx, int64_t row_begin, int64_t row_end,
+                          const void* const* partials, int W, const void* residual,
+                          void* residual_out, const void* gamma, int64_t T, int64_t H,
+                          far_dtype dtype, float eps, float weight_bias, far_pattern pattern,
+                          void* norm_out, void* quant_out, const float* scale_in, float* scale_out,
+                          void* stream) {
+  if (ctx == nullptr) return FAR_ERR_INVALID_ARG;
+  // the per-tensor pattern needs a workspace: far_fused_fp8_tensor
+  if (pattern == FAR_AR_RESIDUAL_RMSNORM_FP8_TENSOR) return FAR_ERR_INVALID_ARG;
+  far_status st = far_validate(row_begin, row_end, partials, W, residual, residual_out, gamma, T, H,
+                               dtype, eps, weight_bias, pattern, norm_out, quant_out, scale_in,
+                               scale_out);
+  if (st != FAR_OK) return st;
+  if (row_end == row_begin) return FAR_OK;
+
+  const far::Params p = make_params(partials, W, residual, residual_out, gamma, H, pattern, eps,
+                                    weight_bias, norm_out, quant_out, scale_in, scale_out);
+  DeviceGuard guard(ctx->device);
+  if (guard.err != cudaSuccess) return cuda_fail(guard.err, "cudaSetDevice");
+  const far::Launch whole = plan(ctx, row_end - row_begin, H, dtype, W + (residual != nullptr ? 1 : 0));
+  const cudaError_t e = launch_rows(p, dtype, whole, row_begin, row_end, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "kernel launch");
   return FAR_OK;
+}
+
+size_t far_fp8_tensor_workspace_bytes(int64_t rows) {
+  if (rows < 0) rows = 0;
+  return static_cast<size_t>((256 + 4 * rows + 255) / 256 * 256);
+}
+
+far_status far_fused_fp8_tensor(far_ctx* ctx, int64_t row_begin, int64_t row_end,
+                                const void* const* partials, int W, const void* residual,
+                                void* residual_out, const void* gamma, int64_t T, int64_t H,
+                                far_dtype dtype, float eps, float weight_bias, void* norm_out,
+                                void* quant_out, float* scale_out, void* workspace,
+                                size_t workspace_bytes, void* stream) {
+  if (ctx == nullptr) return FAR_ERR_INVALID_ARG;
+  far_status st = far_validate(row_begin, row_end, partials, W, residual, residual_out, gamma, T, H,
+                               dtype, eps, weight_bias, FAR_AR_RESIDUAL_RMSNORM_FP8_TENSOR, norm_out,
+                               quant_out, nullptr, scale_out);
+  if (st != FAR_OK) return st;
+  if (row_end == row_begin) return FAR_OK;
+  const int64_t rows = row_end - row_begin;
+  if (workspace == nullptr || workspace_bytes < far_fp8_tensor_workspace_bytes(rows))
+    return FAR_ERR_INVALID_ARG;
+  if (!aligned(workspace, 256)) return FAR_ERR_ALIGNMENT;
+  // the workspace is written: it may overlap no argument buffer
+  {
+    const Range ws = span(workspace, static_cast<int64_t>(far_fp8_tensor_workspace_bytes(rows)));
+    const int64_t tb = T * H * 2;
+    for (int r = 0; r < W; ++r)
+      if (overlap(ws, span(partials[r], tb))) return FAR_ERR_INVALID_ARG;
+    const void* bufs16[] = {residual, residual_out, norm_out};
+    for (const void* b : bufs16)
+      if (b != nullptr && overlap(ws, span(b, tb))) return FAR_ERR_INVALID_ARG;
+    if (overlap(ws, span(gamma, H * 2)) || overlap(ws, span(quant_out, T * H)) ||
+        overlap(ws, span(scale_out, 4)))
+      return FAR_ERR_INVALID_ARG;
+  }
+  return far_fused_fp8_tensor_launch(ctx, row_begin, row_end, partials, W, residual, residual_out,
+                                     gamma, H, dtype, eps, weight_bias, norm_out, quant_out,
+                                     scale_out, workspace, stream);
 }
 
 far_status far_fused(far_ctx* ctx, const void* const* partials, int W, const void* residual,

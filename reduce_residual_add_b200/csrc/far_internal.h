@@ -15,7 +15,14 @@ constexpr int kRingSmemMax = 227 * 1024;  // dynamic shared memory of one ring C
 constexpr int kRingMaxConsumers = 512;    // consumer threads of one ring CTA
 
 enum Dtype : int { kBf16 = 0, kFp16 = 1 };
-enum Pattern : int { kNormOnly = 0, kFp8Static = 1, kFp8Token = 2 };
+enum Pattern : int {
+  kNormOnly = 0,
+  kFp8Static = 1,
+  kFp8Token = 2,
+  kFp8Tensor = 3,       // public value of dynamic per-tensor FP8
+  kTensorAmax = 16,     // its first pass: rinv of each row + the call's amax
+  kTensorQuant = 17     // its second pass: every output, from the stored rinv and amax
+};
 
 // Everything one launch needs, passed by value in the kernel's parameter
 // space (about 200 bytes).
@@ -36,6 +43,9 @@ struct Params {
   int pattern;
   float eps;
   float weight_bias;
+  float* ws_rinv;               // per-tensor FP8: rinv of row t at ws_rinv[t - ws_row0]
+  unsigned* ws_amax;            // per-tensor FP8: the call's amax as fp32 bits
+  int64_t ws_row0;              // per-tensor FP8: first row of the call
 };
 
 // Geometry of one launch, chosen on the host.

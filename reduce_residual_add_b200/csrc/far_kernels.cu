@@ -389,7 +389,11 @@ __device__ __forceinline__ void finish_row(const Params& p, int64_t row, bool ro
                                            float (&y)[VPT][8], const Red& red,
                                            const uint4* gamma_smem = nullptr) {
   const int64_t rbase = row * static_cast<int64_t>(p.packs);  // first pack of the row
-  if (p.residual_out != nullptr) {
+  // dynamic per-tensor FP8 runs in two passes: the first only records rinv
+  // and the call's amax; the second writes every output
+  const bool tensor_amax = p.pattern == kTensorAmax;
+  const bool tensor_quant = p.pattern == kTensorQuant;
+  if (p.residual_out != nullptr && !tensor_amax) {
 #pragma unroll
     for (int k = 0; k < VPT; ++k)
       if (ok[k]) static_cast<uint4*>(p.residual_out)[rbase + j0 + k * jstride] = pack8<DT>(y[k]);
@@ -415,9 +419,10 @@ __device__ __forceinline__ void finish_row(const Params& p, int64_t row, bool ro
   const uint4* gam = gamma_smem != nullptr ? gamma_smem : static_cast<const uint4*>(p.gamma);
 
   // a5b needs max|o| = rinv * max|y * (gamma + wb)| (rinv > 0): its local
-  // part goes into the same reduction round as the sum of squares.
-  float ss, gmax = 0.f;
-  if (fp8_token) {
+  // part goes into the same reduction round as the sum of squares.  The
+  // second per-tensor pass reuses the first pass's rinv: no reduction.
+  float ss = 0.f, gmax = 0.f;
+  if (fp8_token || tensor_amax) {
     float m = 0.f;
 #pragma unroll
     for (int k = 0; k < VPT; ++k) {
@@ -430,21 +435,34 @@ __device__ __forceinline__ void finish_row(const Params& p, int64_t row, bool ro
     const float2 r = red.sum_max(sq[0], m);
     ss = r.x;
     gmax = r.y;
-  } else {
+  } else if (!tensor_quant) {
     ss = red.sum(sq[0]);
   }
-  const float ms = __fdiv_rn(ss, static_cast<float>(p.H));
-  const float rinv = __frsqrt_rn(ms + p.eps);
+  const float rinv = tensor_quant ? p.ws_rinv[row - p.ws_row0]
+                                  : __frsqrt_rn(__fdiv_rn(ss, static_cast<float>(p.H)) + p.eps);
 
-  // the divisor of the FP8 codes: the static scale, or max|o| / 448
+  if (tensor_amax) {
+    if (row_ok && red.leader()) {
+      p.ws_rinv[row - p.ws_row0] = rinv;
+      // non-negative floats order like their bit patterns; a row whose rinv
+      // is 0 or NaN (inf / NaN input) has no finite nonzero o: it adds nothing
+      const float a = rinv * gmax;
+      if (a == a) atomicMax(p.ws_amax, __float_as_uint(a));
+    }
+    return;
+  }
+
+  // the divisor of the FP8 codes: the static scale, or max|o| / 448 of the
+  // row or of the call
   float scale = 1.f;
   if (fp8_static) scale = __ldg(p.scale_in);
-  if (fp8_token) {
-    scale = __fdiv_rn(rinv * gmax, 448.f);
+  if (fp8_token || tensor_quant) {
+    scale = __fdiv_rn(fp8_token ? rinv * gmax : __uint_as_float(*p.ws_amax), 448.f);
     // a row with an inf or NaN input has rinv 0 or NaN; its finite o are 0
     // and the rest NaN, which take no part in the amax: scale 0
     if (scale != scale) scale = 0.f;
-    if (row_ok && red.leader()) p.scale_out[row] = scale;
+    if (row_ok && red.leader() && (fp8_token || row == p.ws_row0))
+      p.scale_out[fp8_token ? row : 0] = scale;
   }
   const float inv = __frcp_rn(scale);
   // outside the reciprocal's normal range, divide exactly (uniform per row)
@@ -460,7 +478,7 @@ __device__ __forceinline__ void finish_row(const Params& p, int64_t row, bool ro
 #pragma unroll
     for (int i = 0; i < 8; ++i) y[k][i] = (y[k][i] * rinv) * g[i];
     if (p.norm_out != nullptr) static_cast<uint4*>(p.norm_out)[pk] = pack8<DT>(y[k]);
-    if (fp8_static || fp8_token) {
+    if (fp8_static || fp8_token || tensor_quant) {
       uint2 codes = make_uint2(0u, 0u);
       if (scale != 0.f) {  // a per-token row of zeros keeps scale 0 and codes 0
         float q[8];

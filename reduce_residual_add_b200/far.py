@@ -34,6 +34,7 @@ FAR_FP16 = 1
 FAR_AR_RESIDUAL_RMSNORM = 0
 FAR_AR_RESIDUAL_RMSNORM_FP8_STATIC = 1
 FAR_AR_RESIDUAL_RMSNORM_FP8_TOKEN = 2
+FAR_AR_RESIDUAL_RMSNORM_FP8_TENSOR = 3
 
 FAR_REGIME_AUTO = 0
 FAR_REGIME_DECODE = 1
@@ -43,7 +44,8 @@ FAR_MAX_W = 16
 FAR_MAX_H = 16384
 
 # Every symbol include/far.h declares.
-EXPORTS = ("far_create", "far_destroy", "far_fused", "far_fused_rows", "far_validate",
+EXPORTS = ("far_create", "far_destroy", "far_fused", "far_fused_rows",
+           "far_fp8_tensor_workspace_bytes", "far_fused_fp8_tensor", "far_validate",
            "far_set_regime", "far_describe_launch", "far_check", "far_status_string",
            "far_last_error", "far_version")
 
@@ -99,6 +101,11 @@ def lib() -> ctypes.CDLL:
     L.far_fused_rows.restype = i32
     L.far_validate.argtypes = [i64, i64] + common
     L.far_validate.restype = i32
+    L.far_fp8_tensor_workspace_bytes.argtypes = [i64]
+    L.far_fp8_tensor_workspace_bytes.restype = ctypes.c_size_t
+    L.far_fused_fp8_tensor.argtypes = [vp, i64, i64, pp, i32, vp, vp, vp, i64, i64, i32, f32, f32,
+                                       vp, vp, vp, vp, ctypes.c_size_t, vp]
+    L.far_fused_fp8_tensor.restype = i32
     L.far_set_regime.argtypes = [vp, i32, i32]
     L.far_set_regime.restype = i32
     L.far_describe_launch.argtypes = [vp, i64, i64, i32, i32, i32, ctypes.POINTER(far_launch_info)]
@@ -207,7 +214,8 @@ def _flat(t: Optional[torch.Tensor], H: int, name: str) -> Optional[torch.Tensor
     return t.view(-1, H) if t.dim() != 2 else t
 
 
-def _args(partials, residual, gamma, residual_out, norm_out, quant_out, scale_in, scale_out):
+def _args(partials, residual, gamma, residual_out, norm_out, quant_out, scale_in, scale_out,
+          scale_out_elems=None):
     if isinstance(partials, torch.Tensor):
         partials = [partials]
     if len(partials) == 0:
@@ -236,7 +244,8 @@ def _args(partials, residual, gamma, residual_out, norm_out, quant_out, scale_in
         raise ValueError("quant_out must be (%d, %d) of 1-byte elements" % (T, H))
     if gamma.dtype != ps[0].dtype:
         raise ValueError("gamma must be %s" % ps[0].dtype)
-    for name, t, n in (("scale_in", scale_in, 1), ("scale_out", scale_out, T)):
+    for name, t, n in (("scale_in", scale_in, 1),
+                       ("scale_out", scale_out, T if scale_out_elems is None else scale_out_elems)):
         if t is not None and (not t.is_cuda or t.dtype != torch.float32 or t.numel() < n
                               or not t.is_contiguous()):
             raise ValueError("%s must be a contiguous CUDA float32 tensor of >= %d elements" % (name, n))
@@ -304,3 +313,30 @@ def far_validate(row_begin: int, row_end: int, partial_ptrs: Sequence[int], resi
                                   vp(residual), vp(residual_out), vp(gamma), int(T), int(H),
                                   int(dtype), float(eps), float(weight_bias), int(pattern),
                                   vp(norm_out), vp(quant_out), vp(scale_in), vp(scale_out)))
+
+
+def far_fp8_tensor_workspace_bytes(rows: int) -> int:
+    return int(lib().far_fp8_tensor_workspace_bytes(int(rows)))
+
+
+def far_fused_fp8_tensor(ctx: FarContext, partials: Sequence[torch.Tensor],
+                         residual: Optional[torch.Tensor], gamma: torch.Tensor, eps: float,
+                         weight_bias: float = 0.0, *, quant_out: torch.Tensor,
+                         scale_out: torch.Tensor, workspace: torch.Tensor,
+                         residual_out: Optional[torch.Tensor] = None,
+                         norm_out: Optional[torch.Tensor] = None, rows=None, stream=None) -> None:
+    """Dynamic per-tensor FP8 over rows [b, e) (all rows by default): one
+    scale in scale_out[0].  ``workspace`` is a CUDA tensor of at least
+    far_fp8_tensor_workspace_bytes(e - b) bytes (see include/far.h)."""
+    (arr, W, res, rout, gam, T, H, dt, nout, qout, sin, sout) = _args(
+        partials, residual, gamma, residual_out, norm_out, quant_out, None, scale_out,
+        scale_out_elems=1)
+    if not workspace.is_cuda or not workspace.is_contiguous():
+        raise ValueError("workspace must be a contiguous CUDA tensor")
+    b, e = (0, T) if rows is None else (int(rows[0]), int(rows[1]))
+    st = lib().far_fused_fp8_tensor(ctx.handle, b, e, arr, W, res, rout, gam, T, H, dt,
+                                    float(eps), float(weight_bias), nout, qout, sout,
+                                    _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                    _stream(stream))
+    if st != FAR_OK:
+        raise FarError(st, "far_fused_fp8_tensor")

@@ -31,6 +31,7 @@ import torch
 PATTERN_AR_RESIDUAL_RMSNORM = 0
 PATTERN_FP8_STATIC = 1
 PATTERN_FP8_TOKEN = 2
+PATTERN_FP8_TENSOR = 3
 
 _TORCH_DTYPES = {"bf16": torch.bfloat16, "fp16": torch.float16}
 
@@ -87,6 +88,10 @@ WORKLOADS = {
         "c4_prefill_fp8_static", W=4, T=8192, H=8192, residual_sigma=2.0,
         eps=1e-5, pattern=PATTERN_FP8_STATIC, static_scale=0.05,
         outlier_frac=0.01, outlier_mult=50.0, seed=3),
+    # the prefill workload with dynamic per-tensor FP8 (one scale per call)
+    "c4_prefill_fp8_tensor": Workload(
+        "c4_prefill_fp8_tensor", W=4, T=8192, H=8192, residual_sigma=2.0,
+        eps=1e-5, pattern=PATTERN_FP8_TENSOR, outlier_frac=0.01, outlier_mult=50.0, seed=3),
     # W=8, T=4096, H=7168, Gemma-style weight_bias=1.0 with gamma N(0,0.1),
     # dynamic per-token FP8; in bf16 and in fp16
     **{

@@ -88,14 +88,22 @@ def run_gpu(ctx, g: dict, eps: float, wb: float, pattern: int, scale_in=None, ro
         rout = alloc(T * H, dt).view(T, H)
     nout = alloc(T * H, dt).view(T, H) if want_norm else None
     qout = alloc(T * H, torch.uint8).view(T, H) if pattern != 0 else None
-    sout = alloc(T, torch.float32) if pattern == 2 else None
+    sout = alloc(T if pattern == 2 else 1, torch.float32) if pattern in (2, 3) else None
     sin = torch.tensor([scale_in], dtype=torch.float32, device=dev) if pattern == 1 else None
-    kw = dict(residual_out=rout, norm_out=nout, quant_out=qout, scale_in=sin, scale_out=sout,
-              stream=stream)
-    if rows is None:
-        far.far_fused(ctx, ps, res, g["gamma"], eps, wb, pattern, **kw)
+    if pattern == 3:
+        nrows = T if rows is None else rows[1] - rows[0]
+        ws = torch.empty(far.far_fp8_tensor_workspace_bytes(nrows), dtype=torch.uint8, device=dev)
+        assert ws.data_ptr() % 256 == 0
+        far.far_fused_fp8_tensor(ctx, ps, res, g["gamma"], eps, wb, quant_out=qout, scale_out=sout,
+                                 workspace=ws, residual_out=rout, norm_out=nout, rows=rows,
+                                 stream=stream)
     else:
-        far.far_fused_rows(ctx, rows[0], rows[1], ps, res, g["gamma"], eps, wb, pattern, **kw)
+        kw = dict(residual_out=rout, norm_out=nout, quant_out=qout, scale_in=sin, scale_out=sout,
+                  stream=stream)
+        if rows is None:
+            far.far_fused(ctx, ps, res, g["gamma"], eps, wb, pattern, **kw)
+        else:
+            far.far_fused_rows(ctx, rows[0], rows[1], ps, res, g["gamma"], eps, wb, pattern, **kw)
     torch.cuda.synchronize()
     far.far_check(ctx, stream)          # no bounded wait inside the kernel gave up
     for raw, gb, n in canaries:
@@ -119,6 +127,8 @@ def run_oracle(inp: dict, dtype: str, eps, wb, pattern, scale_in=None, rows=None
     ps = [as_u16(p) for p in inp["partials"]]
     res = None if inp["residual"] is None else as_u16(inp["residual"])
     gam = as_u16(inp["gamma"])
+    if row_list is not None and pattern == 3:
+        raise ValueError("the per-tensor scale needs every row of the call")
     if row_list is None:
         return oracle.fused(ps, res, gam, dtype, eps, wb, pattern, scale_in=scale_in, rows=rows,
                             want_norm=want_norm, want_residual_out=want_residual_out)

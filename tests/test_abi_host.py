@@ -29,7 +29,7 @@ def built():
 
 def declared_functions():
     body = re.sub(r"/\*.*?\*/", "", HEADER, flags=re.S)
-    return sorted(set(re.findall(r"\b(far_[a-z_]+)\s*\(", body)))
+    return sorted(set(re.findall(r"\b(far_[a-z0-9_]+)\s*\(", body)))
 
 
 def test_library_exports_every_declared_function():
@@ -52,16 +52,17 @@ def test_header_constants_match_binding_and_oracle():
     for n in ("FAR_OK", "FAR_ERR_INVALID_ARG", "FAR_ERR_UNSUPPORTED", "FAR_ERR_ALIGNMENT",
               "FAR_ERR_CUDA", "FAR_ERR_TIMEOUT", "FAR_ERR_INTERNAL", "FAR_BF16", "FAR_FP16",
               "FAR_AR_RESIDUAL_RMSNORM", "FAR_AR_RESIDUAL_RMSNORM_FP8_STATIC",
-              "FAR_AR_RESIDUAL_RMSNORM_FP8_TOKEN", "FAR_REGIME_AUTO", "FAR_REGIME_DECODE",
+              "FAR_AR_RESIDUAL_RMSNORM_FP8_TOKEN", "FAR_AR_RESIDUAL_RMSNORM_FP8_TENSOR",
+              "FAR_REGIME_AUTO", "FAR_REGIME_DECODE",
               "FAR_REGIME_PREFILL"):
         assert getattr(far, n) == _enum(n), n
     assert int(re.search(r"#define FAR_MAX_W (\d+)", HEADER).group(1)) == far.FAR_MAX_W
     assert int(re.search(r"#define FAR_MAX_H (\d+)", HEADER).group(1)) == far.FAR_MAX_H
     # the oracle keeps its own copies of the numbering
     assert (oracle.BF16, oracle.FP16) == (far.FAR_BF16, far.FAR_FP16)
-    assert (oracle.AR_RESIDUAL_RMSNORM, oracle.FP8_STATIC, oracle.FP8_TOKEN) == (
+    assert (oracle.AR_RESIDUAL_RMSNORM, oracle.FP8_STATIC, oracle.FP8_TOKEN, oracle.FP8_TENSOR) == (
         far.FAR_AR_RESIDUAL_RMSNORM, far.FAR_AR_RESIDUAL_RMSNORM_FP8_STATIC,
-        far.FAR_AR_RESIDUAL_RMSNORM_FP8_TOKEN)
+        far.FAR_AR_RESIDUAL_RMSNORM_FP8_TOKEN, far.FAR_AR_RESIDUAL_RMSNORM_FP8_TENSOR)
     assert far.far_version() == int(re.search(r"#define FAR_VERSION (\d+)", HEADER).group(1))
 
 
@@ -105,7 +106,7 @@ def v(**over):
 
 def test_validate_accepts_good_arguments():
     assert v() == far.FAR_OK
-    for p in (0, 1, 2):
+    for p in (0, 1, 2, 3):
         assert v(pattern=p) == far.FAR_OK
     assert v(residual_out=0) == far.FAR_OK                      # in place
     assert v(residual_out=good()["residual"]) == far.FAR_OK     # explicitly in place
@@ -136,7 +137,9 @@ def test_validate_accepts_good_arguments():
     (dict(H=12), far.FAR_ERR_UNSUPPORTED),
     (dict(H=16392), far.FAR_ERR_UNSUPPORTED),
     (dict(dtype=2), far.FAR_ERR_INVALID_ARG),
-    (dict(pattern=3), far.FAR_ERR_INVALID_ARG),
+    (dict(pattern=4), far.FAR_ERR_INVALID_ARG),
+    (dict(pattern=3, quant_out=0), far.FAR_ERR_INVALID_ARG),
+    (dict(pattern=3, scale_out=0), far.FAR_ERR_INVALID_ARG),
     (dict(row_begin=-1), far.FAR_ERR_INVALID_ARG),
     (dict(row_begin=10, row_end=9), far.FAR_ERR_INVALID_ARG),
     (dict(row_end=T + 1), far.FAR_ERR_INVALID_ARG),
@@ -185,3 +188,11 @@ def test_validate_rejects_partial_overlaps():
     assert v(pattern=1, scale_in=g["norm_out"] + 64) == far.FAR_ERR_INVALID_ARG
     # ... but a partial read twice is fine (two ranks cannot alias, but reads are harmless)
     assert v(partial_ptrs=[g["partial_ptrs"][0]] * W) == far.FAR_OK
+
+
+def test_per_tensor_workspace_size():
+    assert far.far_fp8_tensor_workspace_bytes(0) == 256
+    assert far.far_fp8_tensor_workspace_bytes(1) == 512
+    assert far.far_fp8_tensor_workspace_bytes(64) == 512
+    assert far.far_fp8_tensor_workspace_bytes(65) == 768
+    assert far.far_fp8_tensor_workspace_bytes(8192) == 256 + 4 * 8192

@@ -408,3 +408,98 @@ def test_chained_calls_read_completed_outputs(kctx, ctx, kern):
             assert compare({"residual_out": got_r, "norm_out": got_n}, ref, "bf16") is not None
             prev = got_r          # the next call reads exactly what this one wrote
     del gr
+
+
+
+# ---------------------------------------------------------------------------
+# dynamic per-tensor FP8 (two passes, workspace)
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("kern", ["ring", "direct", "auto"])
+@pytest.mark.parametrize("case", [
+    (2, 8, 64, "bf16", True, 0.0),
+    (8, 5, 4096, "bf16", True, 0.0),        # decode-sized: never the cluster kernel
+    (4, 300, 8192, "fp16", True, 1.0),
+    (3, 1000, 1000, "bf16", False, 0.0),
+    (16, 40, 16384, "bf16", True, 0.0),
+], ids=lambda c: "W%d_T%d_H%d_%s_res%d_wb%g" % c)
+def test_per_tensor_fp8(kctx, ctx, case, kern):
+    W, T, H, dt, has_res, wb = case
+    c = ctx if kern == "auto" else kctx[kern]
+    inp = random_inputs(W, T, H, dtype=dt, seed=500 + W + T + H, has_residual=has_res)
+    got = run_gpu(c, to_gpu(inp), 1e-6, wb, 3, guard=512)
+    ref = run_oracle(inp, dt, 1e-6, wb, 3)
+    log("tensor %s %s" % (kern, case), compare(got, ref, dt))
+    assert np.any((got["quant_out"] & 0x7F) == 0x7E)
+
+
+def test_per_tensor_fp8_row_range_and_full_size(ctx):
+    # rows [100, 3000) of the Gemma workload: the scale covers those rows only
+    wl = WORKLOADS["c5_gemma_fp8_token_bf16"]
+    inp = make_inputs(wl)
+    g = to_gpu(inp)
+    got = run_gpu(ctx, g, wl.eps, wl.weight_bias, 3, rows=(100, 3000))
+    ref = run_oracle(inp, "bf16", wl.eps, wl.weight_bias, 3, rows=(100, 3000))
+    log("tensor c5 rows", compare(got, ref, "bf16", rows=slice(100, 3000)))
+    assert not got["quant_out"][:100].any() and not got["quant_out"][3000:].any()
+    # all rows, in the launch configuration of a full-size call
+    got = run_gpu(ctx, g, wl.eps, wl.weight_bias, 3)
+    ref = run_oracle(inp, "bf16", wl.eps, wl.weight_bias, 3)
+    log("tensor c5 full", compare(got, ref, "bf16"))
+
+
+def test_per_tensor_fp8_errors(ctx):
+    inp = random_inputs(2, 16, 256, seed=77)
+    g = to_gpu(inp)
+    q = torch.empty(16, 256, dtype=torch.uint8, device="cuda")
+    sc = torch.empty(1, dtype=torch.float32, device="cuda")
+    small = torch.empty(far.far_fp8_tensor_workspace_bytes(16) - 256, dtype=torch.uint8, device="cuda")
+    with pytest.raises(far.FarError) as e:
+        far.far_fused_fp8_tensor(ctx, g["partials"], g["residual"], g["gamma"], 1e-6,
+                                 quant_out=q, scale_out=sc, workspace=small)
+    assert e.value.status == far.FAR_ERR_INVALID_ARG
+    ws = torch.empty(far.far_fp8_tensor_workspace_bytes(16) + 512, dtype=torch.uint8, device="cuda")
+    with pytest.raises(far.FarError) as e:
+        far.far_fused_fp8_tensor(ctx, g["partials"], g["residual"], g["gamma"], 1e-6,
+                                 quant_out=q, scale_out=sc, workspace=ws[16:])
+    assert e.value.status == far.FAR_ERR_ALIGNMENT
+    # the workspace may not overlap an output
+    big = torch.empty(16 * 256 + far.far_fp8_tensor_workspace_bytes(16), dtype=torch.uint8, device="cuda")
+    with pytest.raises(far.FarError) as e:
+        far.far_fused_fp8_tensor(ctx, g["partials"], g["residual"], g["gamma"], 1e-6,
+                                 quant_out=big[:16 * 256].view(16, 256), scale_out=sc,
+                                 workspace=big)
+    assert e.value.status == far.FAR_ERR_INVALID_ARG
+    # far_fused refuses the per-tensor pattern (it has no workspace)
+    with pytest.raises(far.FarError) as e:
+        far.far_fused(ctx, g["partials"], g["residual"], g["gamma"], 1e-6, 0.0, 3,
+                      quant_out=q, scale_out=torch.empty(16, dtype=torch.float32, device="cuda"))
+    assert e.value.status == far.FAR_ERR_INVALID_ARG
+
+
+def test_per_tensor_fp8_repeated_in_a_graph(ctx):
+    """The memset and both passes are captured; replaying reuses the
+    workspace and gives the same bits."""
+    inp = random_inputs(4, 700, 4096, seed=88)
+    g = to_gpu(inp)
+    T, H = 700, 4096
+    q = torch.empty(T, H, dtype=torch.uint8, device="cuda")
+    sc = torch.empty(1, dtype=torch.float32, device="cuda")
+    rout = torch.empty(T, H, dtype=torch.bfloat16, device="cuda")
+    ws = torch.empty(far.far_fp8_tensor_workspace_bytes(T), dtype=torch.uint8, device="cuda")
+    s = torch.cuda.Stream()
+    kw = dict(quant_out=q, scale_out=sc, workspace=ws, residual_out=rout, stream=s)
+    far.far_fused_fp8_tensor(ctx, g["partials"], g["residual"], g["gamma"], 1e-6, **kw)
+    torch.cuda.synchronize()
+    q0, s0 = q.clone(), sc.clone()
+    gr = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(gr, stream=s):
+        far.far_fused_fp8_tensor(ctx, g["partials"], g["residual"], g["gamma"], 1e-6, **kw)
+    q.zero_()
+    for _ in range(3):
+        with torch.cuda.stream(s):
+            gr.replay()
+    torch.cuda.synchronize()
+    far.far_check(ctx)
+    assert torch.equal(q, q0) and torch.equal(sc, s0)
+    del gr
