@@ -218,6 +218,39 @@ far_status far_fused_fp8_tensor(far_ctx *ctx, int64_t row_begin, int64_t row_end
                                 void *norm_out, void *quant_out, float *scale_out,
                                 void *workspace, size_t workspace_bytes, void *stream);
 
+/* Rows one far_fused_fp8_tensor_noalloc call can take. */
+#define FAR_FP8_TENSOR_NOALLOC_MAX_ROWS 65536
+
+/*
+ * far_fused_fp8_tensor for callers that cannot allocate device memory: the
+ * same operation and arguments, minus the workspace.  The paper has no
+ * counterpart; it exists for callers that must not or cannot call
+ * cudaMalloc -- servers that hand all free device memory to a fixed pool
+ * (a KV cache) at start-up, plain-C callers with no device allocator of
+ * their own, and loops that cannot take the device-wide synchronisation
+ * cudaMalloc / cudaFree imply.
+ *
+ * Its scratch (256 KiB + 256 bytes) is a fixed array inside the library:
+ * every GPU that loads the library holds it until the process exits, and
+ * the call allocates nothing (no cudaMalloc, cudaFree or allocating
+ * library routine).  At most FAR_FP8_TENSOR_NOALLOC_MAX_ROWS rows
+ * (row_end - row_begin) per call; more returns FAR_ERR_UNSUPPORTED with
+ * the limit in far_last_error().  Every call on a GPU shares the one
+ * scratch array, which keeps the last call's contents (the call clears the
+ * word that must start at zero itself): calls that overlap on the GPU --
+ * on different streams without ordering between them -- race and give
+ * wrong results.  The first call on each device looks up the array's
+ * device address (cudaGetSymbolAddress) with that device current; make that
+ * first call before any stream capture.
+ */
+far_status far_fused_fp8_tensor_noalloc(far_ctx *ctx, int64_t row_begin, int64_t row_end,
+                                        const void *const *partials, int W,
+                                        const void *residual, void *residual_out,
+                                        const void *gamma, int64_t T, int64_t H,
+                                        far_dtype dtype, float eps, float weight_bias,
+                                        void *norm_out, void *quant_out, float *scale_out,
+                                        void *stream);
+
 /* Host-only: the status far_fused_rows would return for these arguments
  * before launching (it touches no GPU and needs no context).  With pattern
  * FAR_AR_RESIDUAL_RMSNORM_FP8_TENSOR it checks far_fused_fp8_tensor's

@@ -593,6 +593,71 @@ far_status far_fused_fp8_tensor(far_ctx* ctx, int64_t row_begin, int64_t row_end
                                      scale_out, workspace, stream);
 }
 
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Per-tensor FP8 with the library's own scratch instead of a workspace
+// ---------------------------------------------------------------------------
+
+namespace {
+
+// The scratch of far_fused_fp8_tensor_noalloc: the amax word at byte 0 and
+// one rinv per row from byte 256, for at most FAR_FP8_TENSOR_NOALLOC_MAX_ROWS
+// rows (256 KiB + 256 bytes).  It is part of the library image: every GPU
+// that loads the library holds it until the process exits, and every call
+// on that GPU shares it.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[256 + 4 * FAR_FP8_TENSOR_NOALLOC_MAX_ROWS];
+
+// Device address of g_noalloc_scratch for each device ordinal, looked up
+// on the first call on that device.  In host code the array's name only
+// stands for the symbol, so the kernels get this address instead.
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[256] = {};
+
+}  // namespace
+
+extern "C" {
+
+far_status far_fused_fp8_tensor_noalloc(far_ctx* ctx, int64_t row_begin, int64_t row_end,
+                                        const void* const* partials, int W, const void* residual,
+                                        void* residual_out, const void* gamma, int64_t T,
+                                        int64_t H, far_dtype dtype, float eps, float weight_bias,
+                                        void* norm_out, void* quant_out, float* scale_out,
+                                        void* stream) {
+  if (ctx == nullptr) return FAR_ERR_INVALID_ARG;
+  far_status st = far_validate(row_begin, row_end, partials, W, residual, residual_out, gamma, T, H,
+                               dtype, eps, weight_bias, FAR_AR_RESIDUAL_RMSNORM_FP8_TENSOR, norm_out,
+                               quant_out, nullptr, scale_out);
+  if (st != FAR_OK) return st;
+  if (row_end - row_begin > FAR_FP8_TENSOR_NOALLOC_MAX_ROWS) {
+    std::snprintf(g_last_error, sizeof(g_last_error),
+                  "far_fused_fp8_tensor_noalloc handles at most %d rows per call (got %lld); "
+                  "use far_fused_fp8_tensor with a workspace",
+                  FAR_FP8_TENSOR_NOALLOC_MAX_ROWS, static_cast<long long>(row_end - row_begin));
+    return FAR_ERR_UNSUPPORTED;
+  }
+  if (row_end == row_begin) return FAR_OK;
+  if (ctx->device < 0 || ctx->device >= 256) return FAR_ERR_UNSUPPORTED;
+
+  void* scratch = nullptr;
+  {
+    DeviceGuard guard(ctx->device);  // the lookup needs the device current
+    if (guard.err != cudaSuccess) return cuda_fail(guard.err, "cudaSetDevice");
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (g_noalloc_ptr[ctx->device] == nullptr) {
+      void* ptr = nullptr;
+      const cudaError_t e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
+      if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress");
+      g_noalloc_ptr[ctx->device] = ptr;
+    }
+    scratch = g_noalloc_ptr[ctx->device];
+  }
+  // the same two passes as far_fused_fp8_tensor, which zero the amax word first
+  return far_fused_fp8_tensor_launch(ctx, row_begin, row_end, partials, W, residual, residual_out,
+                                     gamma, H, dtype, eps, weight_bias, norm_out, quant_out,
+                                     scale_out, scratch, stream);
+}
+
 far_status far_fused(far_ctx* ctx, const void* const* partials, int W, const void* residual,
                      void* residual_out, const void* gamma, int64_t T, int64_t H, far_dtype dtype,
                      float eps, float weight_bias, far_pattern pattern, void* norm_out,

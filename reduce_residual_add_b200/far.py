@@ -42,10 +42,12 @@ FAR_REGIME_PREFILL = 2
 
 FAR_MAX_W = 16
 FAR_MAX_H = 16384
+FAR_FP8_TENSOR_NOALLOC_MAX_ROWS = 65536
 
 # Every symbol include/far.h declares.
 EXPORTS = ("far_create", "far_destroy", "far_fused", "far_fused_rows",
-           "far_fp8_tensor_workspace_bytes", "far_fused_fp8_tensor", "far_validate",
+           "far_fp8_tensor_workspace_bytes", "far_fused_fp8_tensor",
+           "far_fused_fp8_tensor_noalloc", "far_validate",
            "far_set_regime", "far_describe_launch", "far_check", "far_status_string",
            "far_last_error", "far_version")
 
@@ -106,6 +108,9 @@ def lib() -> ctypes.CDLL:
     L.far_fused_fp8_tensor.argtypes = [vp, i64, i64, pp, i32, vp, vp, vp, i64, i64, i32, f32, f32,
                                        vp, vp, vp, vp, ctypes.c_size_t, vp]
     L.far_fused_fp8_tensor.restype = i32
+    L.far_fused_fp8_tensor_noalloc.argtypes = [vp, i64, i64, pp, i32, vp, vp, vp, i64, i64, i32,
+                                               f32, f32, vp, vp, vp, vp]
+    L.far_fused_fp8_tensor_noalloc.restype = i32
     L.far_set_regime.argtypes = [vp, i32, i32]
     L.far_set_regime.restype = i32
     L.far_describe_launch.argtypes = [vp, i64, i64, i32, i32, i32, ctypes.POINTER(far_launch_info)]
@@ -340,3 +345,24 @@ def far_fused_fp8_tensor(ctx: FarContext, partials: Sequence[torch.Tensor],
                                     _stream(stream))
     if st != FAR_OK:
         raise FarError(st, "far_fused_fp8_tensor")
+
+
+def far_fused_fp8_tensor_noalloc(ctx: FarContext, partials: Sequence[torch.Tensor],
+                                 residual: Optional[torch.Tensor], gamma: torch.Tensor,
+                                 eps: float, weight_bias: float = 0.0, *,
+                                 quant_out: torch.Tensor, scale_out: torch.Tensor,
+                                 residual_out: Optional[torch.Tensor] = None,
+                                 norm_out: Optional[torch.Tensor] = None, rows=None,
+                                 stream=None) -> None:
+    """far_fused_fp8_tensor without a workspace: the library's own scratch,
+    at most FAR_FP8_TENSOR_NOALLOC_MAX_ROWS rows per call; calls that overlap
+    on the GPU race (see include/far.h)."""
+    (arr, W, res, rout, gam, T, H, dt, nout, qout, sin, sout) = _args(
+        partials, residual, gamma, residual_out, norm_out, quant_out, None, scale_out,
+        scale_out_elems=1)
+    b, e = (0, T) if rows is None else (int(rows[0]), int(rows[1]))
+    st = lib().far_fused_fp8_tensor_noalloc(ctx.handle, b, e, arr, W, res, rout, gam, T, H, dt,
+                                            float(eps), float(weight_bias), nout, qout, sout,
+                                            _stream(stream))
+    if st != FAR_OK:
+        raise FarError(st, "far_fused_fp8_tensor_noalloc")

@@ -58,6 +58,8 @@ def test_header_constants_match_binding_and_oracle():
         assert getattr(far, n) == _enum(n), n
     assert int(re.search(r"#define FAR_MAX_W (\d+)", HEADER).group(1)) == far.FAR_MAX_W
     assert int(re.search(r"#define FAR_MAX_H (\d+)", HEADER).group(1)) == far.FAR_MAX_H
+    assert (int(re.search(r"#define FAR_FP8_TENSOR_NOALLOC_MAX_ROWS (\d+)", HEADER).group(1))
+            == far.FAR_FP8_TENSOR_NOALLOC_MAX_ROWS)
     # the oracle keeps its own copies of the numbering
     assert (oracle.BF16, oracle.FP16) == (far.FAR_BF16, far.FAR_FP16)
     assert (oracle.AR_RESIDUAL_RMSNORM, oracle.FP8_STATIC, oracle.FP8_TOKEN, oracle.FP8_TENSOR) == (
