@@ -231,6 +231,13 @@ class Case:
                     if wl.pattern == 1 else None)
         self.bytes = algorithmic_bytes(wl, T, self.nout is not None)
 
+    def prepared(self):
+        """The same step as a far.FarCall (arguments marshalled once)."""
+        return self.far.FarCall(self.ctx, self.ps, self.res, self.gam, self.wl.eps,
+                                self.wl.weight_bias, self.wl.pattern, residual_out=self.rout,
+                                norm_out=self.nout, quant_out=self.qout, scale_in=self.sin,
+                                scale_out=self.sout, stream=self.stream)
+
     def step(self):
         if self.wl.pattern == 3:
             self.far.far_fused_fp8_tensor(self.ctx, self.ps, self.res, self.gam, self.wl.eps,
@@ -456,11 +463,23 @@ def extras(ctx, device, stream) -> dict:
         inp = make_inputs(wl)
         case = Case(ctx, wl, inp, device, False, stream)
         row = {}
-        for reg, nm in ((far.FAR_REGIME_AUTO, "auto"), (far.FAR_REGIME_PREFILL, "prefill_kernel")):
+        for reg, nm in ((far.FAR_REGIME_AUTO, "auto"), (far.FAR_REGIME_DECODE, "cluster_kernel")):
             far.far_set_regime(ctx, reg)
             total, mean = case.time_steps(500, 50, per_launch=False)
             row[nm] = {"stream_us_per_call": round(mean * 1e6, 3),
                        "graph_us_per_call": round(graph_time(case, 100) * 1e6, 3)}
+        far.far_set_regime(ctx, far.FAR_REGIME_AUTO)
+        call = case.prepared()
+        for _ in range(50):
+            call()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(case.stream)
+        for _ in range(500):
+            call()
+        b.record(case.stream)
+        torch.cuda.synchronize()
+        row["auto"]["prepared_stream_us_per_call"] = round(a.elapsed_time(b) / 500 * 1e3, 3)
         far.far_set_regime(ctx, far.FAR_REGIME_AUTO)
         row["tokens_per_s_graph"] = round(T / (row["auto"]["graph_us_per_call"] * 1e-6), 1)
         row["bytes"] = case.bytes

@@ -103,11 +103,14 @@ typedef enum {
  * FAR_DECODE_MAX_ROWS, FAR_FORCE_REGIME=decode|prefill, FAR_DECODE_CLUSTER
  * (CTAs per row; default by rule),
  * FAR_PREFILL_THREADS, FAR_PREFILL_KERNEL=1 ring | 0 direct,
- * FAR_RING_CTAS_PER_SM=1..4 (default 2), FAR_RING_THREADS: consumer threads
- * per ring CTA, at most 512 (default 256), FAR_RING_SLOTS: row-segment slots
+ * FAR_RING_CTAS_PER_SM=1..4 (default: 3 for rows of at most 6 segments,
+ * else 2), FAR_RING_THREADS: consumer threads
+ * per ring CTA, at most 256 (default 256), FAR_RING_SLOTS: row-segment slots
  * per ring CTA (2..32; default: about 72 KiB of segments, as many as fit),
  * FAR_PDL=1|0: launch with programmatic dependent launch, default 1,
- * FAR_RING_MIN_ROWS: fewest rows for the ring kernel, default by rule). */
+ * FAR_RING_MIN_ROWS: fewest rows for the ring kernel, default by rule,
+ * FAR_L2_EVICT_FIRST=0|1: ring loads marked evict-first in L2, default 0,
+ * FAR_STREAM_STORES=0|1: outputs stored with st.global.cs, default 0). */
 /*
  * Programmatic dependent launch: every kernel of this library first waits
  * (griddepcontrol.wait) until the grid it depends on has completed, then
@@ -266,6 +269,15 @@ far_status far_validate(int64_t row_begin, int64_t row_end,
 /* Override the regime choice and the decode row threshold of a context
  * (decode_max_rows < 0 keeps the current threshold). */
 far_status far_set_regime(far_ctx *ctx, far_regime regime, int decode_max_rows);
+
+/* Test hook for the bounded waits.  The TMA ring kernel's producer skips
+ * the bulk copy of row segment `segment` (counted from 0 in each CTA's
+ * order) in every later launch on this context, so the consumers' wait for
+ * it has nothing to end it; every bounded wait then gives up after
+ * wait_limit_us microseconds instead of 2 s (0: back to 2 s), the kernel
+ * ends, and far_check returns FAR_ERR_TIMEOUT.  segment < 0 switches the
+ * hook off.  Outputs of a stalled call are not valid. */
+far_status far_test_stall(far_ctx *ctx, int64_t segment, uint32_t wait_limit_us);
 
 /* Fill `info` with the launch geometry a call on `rows` rows of W partials
  * (and a residual when has_residual != 0) would use. */

@@ -24,15 +24,19 @@ struct far_ctx {
   int decode_cluster;   // preferred CTAs per row in decode
   int prefill_threads;  // target threads per row in prefill
   int prefill_kernel;   // 1 = TMA bulk-copy ring (default), 0 = direct loads
-  int ring_ctas_per_sm; // persistent ring CTAs per SM wanted (1..4)
+  int ring_ctas_per_sm; // persistent ring CTAs per SM wanted (1..4; 0 = by rule)
   int ring_threads;     // target consumer threads of a ring CTA
   int ring_slots_max;   // at most this many ring slots
   int pdl;              // programmatic dependent launch on every call
   int ring_min_rows;    // fewer rows than this take the direct kernel
+  int l2_evict_first;   // ring bulk loads with an L2 evict-first policy
+  int stream_stores;    // outputs stored with st.global.cs
+  uint64_t wait_limit_ns;  // bounded waits in the kernels give up after this
+  int64_t stall_segment;   // test hook (far_test_stall), -1 when off
   // ring CTAs per SM the occupancy calculator allows, per (dtype, packs):
   // 0 = not asked yet, -1 = cannot run
   std::mutex occ_mu;
-  int ring_occ[2][far::kMaxH / far::kPackElems + 1];
+  int ring_occ[2][far::kMaxH / far::kPackElems + 1][2];  // [dtype][packs][2 or 3 CTAs/SM wanted]
 };
 
 namespace {
@@ -124,14 +128,17 @@ void plan_decode(int packs, int cluster_pref, far::Launch* l) {
 // confirms, at most ring_ctas_per_sm), fewer for fewer rows.  Returns false
 // (the direct kernel runs) when fewer than two slots fit or the
 // configuration cannot be resident.
-bool plan_ring(const far_ctx* ctx, int packs, int64_t rows, int dtype, far::Launch* l) {
+bool plan_ring(const far_ctx* ctx, int packs, int64_t rows, int dtype, int segs, far::Launch* l) {
   if (packs <= 32) return false;
   int vpt = 1;
   while (vpt < 8 && (packs + vpt - 1) / vpt > ctx->ring_threads) vpt *= 2;
   const int tpr = (((packs + vpt - 1) / vpt) + 31) / 32 * 32;
   if (tpr > far::kRingMaxConsumers) return false;
   const int seg = packs * 16;
-  const int n_req = ctx->ring_ctas_per_sm;
+  // CTAs per SM: measured on B200, 3 (registers capped at 72) when a row has
+  // few segments (W=4 + residual: 95.5 % vs 93.3 % with 2), 2 (86 registers)
+  // when it has many (W=8 + residual: 89.1 % vs 87.9 % with 3)
+  const int n_req = ctx->ring_ctas_per_sm > 0 ? ctx->ring_ctas_per_sm : (segs <= 6 ? 3 : 2);
   int per_cta = 228 * 1024 / n_req - 1024;
   if (per_cta > far::kRingSmemMax) per_cta = far::kRingSmemMax;
   // header, gamma (one segment's worth of bytes), slots: about 72 KiB of
@@ -144,9 +151,9 @@ bool plan_ring(const far_ctx* ctx, int packs, int64_t rows, int dtype, far::Laun
   int occ;
   {
     std::lock_guard<std::mutex> lock(const_cast<far_ctx*>(ctx)->occ_mu);
-    int& cached = const_cast<far_ctx*>(ctx)->ring_occ[dtype][packs];
+    int& cached = const_cast<far_ctx*>(ctx)->ring_occ[dtype][packs][n_req >= 3 ? 1 : 0];
     if (cached == 0) {
-      const int n = far::ring_occupancy(dtype, vpt, tpr + 32, smem);
+      const int n = far::ring_occupancy(dtype, vpt, n_req >= 3 ? 3 : 2, tpr + 32, smem);
       cached = n > 0 ? n : -1;
     }
     occ = cached;
@@ -154,6 +161,7 @@ bool plan_ring(const far_ctx* ctx, int packs, int64_t rows, int dtype, far::Laun
   if (occ < 1) return false;
   if (occ > n_req) occ = n_req;
   l->kernel = 1;
+  l->ring_minb = n_req >= 3 ? 3 : 2;
   l->vpt = vpt;
   l->tpr = tpr;
   l->rows_per_cta = 1;
@@ -204,9 +212,9 @@ far::Launch plan(const far_ctx* ctx, int64_t rows, int64_t H, int dtype, int seg
     int64_t min_rows = ctx->ring_min_rows;
     if (min_rows <= 0) {
       const int per_cta = (4096 / packs > 8) ? 4096 / packs : 8;
-      min_rows = static_cast<int64_t>(per_cta) * ctx->sm_count * ctx->ring_ctas_per_sm;
+      min_rows = static_cast<int64_t>(per_cta) * ctx->sm_count * 2;
     }
-    if (ctx->prefill_kernel == 1 && rows >= min_rows) plan_ring(ctx, packs, rows, dtype, &l);
+    if (ctx->prefill_kernel == 1 && rows >= min_rows) plan_ring(ctx, packs, rows, dtype, segs, &l);
   }
   l.pdl = ctx->pdl;
   return l;
@@ -261,10 +269,10 @@ far_status far_create(far_ctx** ctx, int device) {
   if (c.prefill_threads < 32) c.prefill_threads = 32;
   if (c.prefill_threads > far::kMaxThreads) c.prefill_threads = far::kMaxThreads;
   c.prefill_kernel = env_int("FAR_PREFILL_KERNEL", 1) != 0 ? 1 : 0;
-  c.ring_ctas_per_sm = env_int("FAR_RING_CTAS_PER_SM", 2);
-  if (c.ring_ctas_per_sm < 1) c.ring_ctas_per_sm = 1;
+  c.ring_ctas_per_sm = env_int("FAR_RING_CTAS_PER_SM", 0);  // 0: by segments per row
+  if (c.ring_ctas_per_sm < 0) c.ring_ctas_per_sm = 0;
   if (c.ring_ctas_per_sm > 4) c.ring_ctas_per_sm = 4;
-  c.ring_threads = env_int("FAR_RING_THREADS", 256);
+  c.ring_threads = env_int("FAR_RING_THREADS", 256);  // at most kRingMaxConsumers
   c.ring_slots_max = env_int("FAR_RING_SLOTS", 0);  // 0: by the 72 KiB rule
   if (c.ring_slots_max < 0) c.ring_slots_max = 0;
   if (c.ring_slots_max > 32) c.ring_slots_max = 32;
@@ -272,6 +280,10 @@ far_status far_create(far_ctx** ctx, int device) {
   if (c.ring_threads > far::kRingMaxConsumers) c.ring_threads = far::kRingMaxConsumers;
   c.pdl = env_int("FAR_PDL", 1) != 0 ? 1 : 0;
   c.ring_min_rows = env_int("FAR_RING_MIN_ROWS", 0);  // 0: the measured rule
+  c.l2_evict_first = env_int("FAR_L2_EVICT_FIRST", 0) != 0 ? 1 : 0;
+  c.stream_stores = env_int("FAR_STREAM_STORES", 0) != 0 ? 1 : 0;
+  c.wait_limit_ns = 2000000000ull;
+  c.stall_segment = -1;
   c.force_regime = FAR_REGIME_AUTO;
   if (const char* f = std::getenv("FAR_FORCE_REGIME")) {
     if (std::strcmp(f, "decode") == 0) c.force_regime = FAR_REGIME_DECODE;
@@ -293,6 +305,13 @@ far_status far_create(far_ctx** ctx, int device) {
 
 far_status far_destroy(far_ctx* ctx) {
   delete ctx;
+  return FAR_OK;
+}
+
+far_status far_test_stall(far_ctx* ctx, int64_t segment, uint32_t wait_limit_us) {
+  if (ctx == nullptr) return FAR_ERR_INVALID_ARG;
+  ctx->stall_segment = segment < 0 ? -1 : segment;
+  ctx->wait_limit_ns = wait_limit_us == 0 ? 2000000000ull : static_cast<uint64_t>(wait_limit_us) * 1000ull;
   return FAR_OK;
 }
 
@@ -499,6 +518,10 @@ far_status far_fused_fp8_tensor_launch(far_ctx* ctx, int64_t row_begin, int64_t 
   far::Params p = make_params(partials, W, residual, residual_out, gamma, H,
                               FAR_AR_RESIDUAL_RMSNORM_FP8_TENSOR, eps, weight_bias, norm_out,
                               quant_out, nullptr, scale_out);
+  p.l2_evict_first = ctx->l2_evict_first;
+  p.stream_stores = ctx->stream_stores;
+  p.wait_limit_ns = ctx->wait_limit_ns;
+  p.stall_segment = ctx->stall_segment;
   p.ws_amax = static_cast<unsigned*>(workspace);
   p.ws_rinv = reinterpret_cast<float*>(static_cast<unsigned char*>(workspace) + 256);
   p.ws_row0 = row_begin;
@@ -544,8 +567,12 @@ far_status far_fused_rows(far_ctx* ctx, int64_t row_begin, int64_t row_end,
   if (st != FAR_OK) return st;
   if (row_end == row_begin) return FAR_OK;
 
-  const far::Params p = make_params(partials, W, residual, residual_out, gamma, H, pattern, eps,
-                                    weight_bias, norm_out, quant_out, scale_in, scale_out);
+  far::Params p = make_params(partials, W, residual, residual_out, gamma, H, pattern, eps,
+                              weight_bias, norm_out, quant_out, scale_in, scale_out);
+  p.l2_evict_first = ctx->l2_evict_first;
+  p.stream_stores = ctx->stream_stores;
+  p.wait_limit_ns = ctx->wait_limit_ns;
+  p.stall_segment = ctx->stall_segment;
   DeviceGuard guard(ctx->device);
   if (guard.err != cudaSuccess) return cuda_fail(guard.err, "cudaSetDevice");
   const far::Launch whole = plan(ctx, row_end - row_begin, H, dtype, W + (residual != nullptr ? 1 : 0));

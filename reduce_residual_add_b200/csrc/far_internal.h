@@ -12,7 +12,7 @@ constexpr int kMaxH = 16384;     // longest row held in registers
 constexpr int kPackElems = 8;    // 2-byte elements per 16-byte pack
 constexpr int kMaxThreads = 256; // threads per row (CTA) in every kernel
 constexpr int kRingSmemMax = 227 * 1024;  // dynamic shared memory of one ring CTA
-constexpr int kRingMaxConsumers = 512;    // consumer threads of one ring CTA
+constexpr int kRingMaxConsumers = 256;    // consumer threads of one ring CTA
 
 enum Dtype : int { kBf16 = 0, kFp16 = 1 };
 enum Pattern : int {
@@ -46,6 +46,10 @@ struct Params {
   float* ws_rinv;               // per-tensor FP8: rinv of row t at ws_rinv[t - ws_row0]
   unsigned* ws_amax;            // per-tensor FP8: the call's amax as fp32 bits
   int64_t ws_row0;              // per-tensor FP8: first row of the call
+  int l2_evict_first;           // ring: bulk loads carry an L2 evict-first policy
+  int stream_stores;            // outputs stored with st.global.cs
+  uint64_t wait_limit_ns;       // every bounded wait gives up after this long
+  int64_t stall_segment;        // test hook: the ring producer skips this copy (-1: none)
 };
 
 // Geometry of one launch, chosen on the host.
@@ -61,6 +65,7 @@ struct Launch {
   int nslot;            // ring: shared-memory slots of one row segment each
   int smem_bytes;       // ring: dynamic shared memory per CTA
   int pdl;              // launch with programmatic stream serialization
+  int ring_minb;        // ring: CTAs per SM its registers are sized for (2 or 3)
 };
 
 // Enqueue one kernel on `stream`.  Returns the launch error (cudaSuccess if
@@ -74,7 +79,7 @@ int ring_header_bytes(int nslot);
 
 // Resident ring CTAs per SM for this configuration on the current device
 // (0 if it cannot run).
-int ring_occupancy(int dtype, int vpt, int threads, int smem_bytes);
+int ring_occupancy(int dtype, int vpt, int minb, int threads, int smem_bytes);
 
 // The device error word of the current device (see far_check): read it
 // after the work on `stream`, or clear it.  Both synchronise `stream`.

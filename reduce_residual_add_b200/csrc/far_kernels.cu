@@ -102,6 +102,23 @@ __device__ __forceinline__ void pack_plus(const uint4& v, float s, float (&out)[
   }
 }
 
+// Output stores: plain, or streaming (st.global.cs: evict-first) when the
+// outputs should not displace other lines from L2.
+__device__ __forceinline__ void store16(void* base, int64_t idx, uint4 v, bool streaming) {
+  uint4* p = static_cast<uint4*>(base) + idx;
+  if (streaming)
+    __stcs(p, v);
+  else
+    *p = v;
+}
+__device__ __forceinline__ void store8(void* base, int64_t idx, uint2 v, bool streaming) {
+  uint2* p = static_cast<uint2*>(base) + idx;
+  if (streaming)
+    __stcs(p, v);
+  else
+    *p = v;
+}
+
 template <class DT>
 __device__ __forceinline__ uint4 pack8(const float (&f)[8]) {
   return make_uint4(DT::pack2(f[0], f[1]), DT::pack2(f[2], f[3]),
@@ -164,7 +181,6 @@ __device__ unsigned int g_far_error = 0u;
 constexpr unsigned kErrWaitFull = 1u;
 constexpr unsigned kErrWaitEmpty = 2u;
 constexpr unsigned kErrWaitPeer = 4u;
-constexpr uint64_t kWaitLimitNs = 2000000000ull;  // one wait gives up after 2 s
 
 __device__ __forceinline__ uint32_t smem_addr(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -202,21 +218,23 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Wait for the phase of parity `parity` to complete.  Gives up after
-// kWaitLimitNs, or as soon as *abort is set (when abort is non-null);
-// returns false then.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const volatile int* abort) {
+// limit_ns, or as soon as *abort is set (when abort is non-null); returns
+// false then.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const volatile int* abort,
+                                          uint64_t limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_ns();
   for (;;) {
     if (mbar_try_wait(bar, parity)) return true;
     if (abort != nullptr && *abort) return false;
-    if (global_ns() - t0 > kWaitLimitNs) return false;
+    if (global_ns() - t0 > limit_ns) return false;
   }
 }
 
 // As mbar_wait, with cluster-scope acquire (peers arrive on this barrier
-// from other CTAs of the cluster); gives up after kWaitLimitNs.
-__device__ __forceinline__ bool mbar_wait_acquire_cluster(uint64_t* bar, uint32_t parity) {
+// from other CTAs of the cluster); gives up after limit_ns.
+__device__ __forceinline__ bool mbar_wait_acquire_cluster(uint64_t* bar, uint32_t parity,
+                                                          uint64_t limit_ns) {
   const uint64_t t0 = global_ns();
   for (;;) {
     uint32_t done;
@@ -228,7 +246,7 @@ __device__ __forceinline__ bool mbar_wait_acquire_cluster(uint64_t* bar, uint32_
         : "r"(smem_addr(bar)), "r"(parity)
         : "memory");
     if (done) return true;
-    if (global_ns() - t0 > kWaitLimitNs) return false;
+    if (global_ns() - t0 > limit_ns) return false;
   }
 }
 
@@ -239,6 +257,22 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
       "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
       ::"r"(smem_addr(dst)), "l"(src), "r"(bytes), "r"(smem_addr(bar))
       : "memory");
+}
+
+// The same with an L2 cache policy (createpolicy): data read once is marked
+// evict-first so it does not displace lines that are still to be used.
+__device__ __forceinline__ void bulk_load_hint(void* dst, const void* src, uint32_t bytes,
+                                               uint64_t* bar, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;"
+      ::"r"(smem_addr(dst)), "l"(src), "r"(bytes), "r"(smem_addr(bar)), "l"(policy)
+      : "memory");
+}
+
+__device__ __forceinline__ uint64_t policy_evict_first() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
 }
 
 // Programmatic dependent launch (PTX griddepcontrol): wait until the grid
@@ -325,6 +359,7 @@ struct ClusterRed {
   uint64_t* bar;  // counts the ncta pushes
   int ncta;
   int rank;
+  uint64_t limit_ns;
   __device__ float2 exchange(float2 t) const {
     asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
     if (threadIdx.x < static_cast<unsigned>(ncta)) {
@@ -337,7 +372,7 @@ struct ClusterRed {
       asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(rm), "f"(t.y) : "memory");
       asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(rb) : "memory");
     }
-    if (!mbar_wait_acquire_cluster(bar, 0u)) atomicOr(&g_far_error, kErrWaitPeer);
+    if (!mbar_wait_acquire_cluster(bar, 0u, limit_ns)) atomicOr(&g_far_error, kErrWaitPeer);
     const int lane = threadIdx.x & 31;
     const float u = lane < ncta ? s_in[lane] : 0.f;
     const float w = lane < ncta ? s_in[16 + lane] : 0.f;
@@ -396,7 +431,7 @@ __device__ __forceinline__ void finish_row(const Params& p, int64_t row, bool ro
   if (p.residual_out != nullptr && !tensor_amax) {
 #pragma unroll
     for (int k = 0; k < VPT; ++k)
-      if (ok[k]) static_cast<uint4*>(p.residual_out)[rbase + j0 + k * jstride] = pack8<DT>(y[k]);
+      if (ok[k]) store16(p.residual_out, rbase + j0 + k * jstride, pack8<DT>(y[k]), p.stream_stores);
   }
 
   // a3: mean of squares; pairwise inside the thread, butterflies above it.
@@ -477,7 +512,7 @@ __device__ __forceinline__ void finish_row(const Params& p, int64_t row, bool ro
     pack_plus<DT>(gam[j0 + k * jstride], p.weight_bias, g);
 #pragma unroll
     for (int i = 0; i < 8; ++i) y[k][i] = (y[k][i] * rinv) * g[i];
-    if (p.norm_out != nullptr) static_cast<uint4*>(p.norm_out)[pk] = pack8<DT>(y[k]);
+    if (p.norm_out != nullptr) store16(p.norm_out, pk, pack8<DT>(y[k]), p.stream_stores);
     if (fp8_static || fp8_token || tensor_quant) {
       uint2 codes = make_uint2(0u, 0u);
       if (scale != 0.f) {  // a per-token row of zeros keeps scale 0 and codes 0
@@ -491,7 +526,7 @@ __device__ __forceinline__ void finish_row(const Params& p, int64_t row, bool ro
         }
         codes = make_uint2(e4m3x4(q[0], q[1], q[2], q[3]), e4m3x4(q[4], q[5], q[6], q[7]));
       }
-      reinterpret_cast<uint2*>(p.quant_out)[pk] = codes;
+      store8(p.quant_out, pk, codes, p.stream_stores);
     }
   }
 }
@@ -590,7 +625,7 @@ far_decode_kernel(const Params p) {
   const int chunk = (p.packs + ncta - 1) / ncta;
   const int jbeg = rank * chunk;
   const int jend = min(p.packs, jbeg + chunk);
-  const ClusterRed red{BlockRed{s_sum, s_max}, s_in, &s_bar, ncta, rank};
+  const ClusterRed red{BlockRed{s_sum, s_max}, s_in, &s_bar, ncta, rank, p.wait_limit_ns};
   fused_row<DT, VPT>(p, row, row < p.row_end, jbeg + static_cast<int>(threadIdx.x),
                      blockDim.x, jend, red);
 }
@@ -606,12 +641,13 @@ far_decode_kernel(const Params p) {
 // from registers.  The bytes in flight live in shared memory, not in
 // registers, so each SM keeps ~100-200 KB of loads outstanding.
 //
-// Every wait is bounded (kWaitLimitNs); a wait that gives up sets the
+// Every wait is bounded (p.wait_limit_ns, 2 s); a wait that gives up sets the
 // device error word and the CTA's abort flag, after which no wait blocks,
 // the producer stops, and thread 0 waits (bounded) for the copies already
 // issued before the CTA exits.
-template <class DT, int VPT>
-__global__ void __launch_bounds__(kRingMaxConsumers + 32, 1)
+// MINB: CTAs per SM the register budget is sized for (2 or 3; 1 at VPT 8).
+template <class DT, int VPT, int MINB>
+__global__ void __launch_bounds__(kRingMaxConsumers + 32, MINB)
 far_ring_kernel(const Params p, int nslot, int ncons) {
   pdl_enter();
   extern __shared__ __align__(128) unsigned char smem[];
@@ -647,22 +683,30 @@ far_ring_kernel(const Params p, int nslot, int ncons) {
     // producer warp: one thread issues, the rest of the warp is idle
     if (threadIdx.x == ncons) {
       const int64_t nseg = my_rows * S;
+      const uint64_t policy = policy_evict_first();
       int64_t issued = 0;
       for (int64_t g = 0; g < nseg; ++g) {
         if (*abort_flag) break;
         const int slot = static_cast<int>(g % nslot);
         const uint32_t round = static_cast<uint32_t>(g / nslot);
-        if (!mbar_wait(&empty[slot], (round & 1u) ^ 1u, abort_flag)) {
+        if (!mbar_wait(&empty[slot], (round & 1u) ^ 1u, abort_flag, p.wait_limit_ns)) {
           if (!*abort_flag) atomicOr(&g_far_error, kErrWaitEmpty);
           *abort_flag = 1;
           break;
+        }
+        if (g == p.stall_segment) {  // test hook: this copy is never issued
+          issued = g + 1;
+          continue;
         }
         const int64_t row = p.row_begin + blockIdx.x + (g / S) * gridDim.x;
         const int k = static_cast<int>(g % S);
         const void* base = (k < p.W) ? p.partials[k] : p.residual;
         const unsigned char* src = static_cast<const unsigned char*>(base) + row * static_cast<int64_t>(seg_bytes);
         mbar_arrive_expect_tx(&full[slot], seg_bytes);
-        bulk_load(ring + static_cast<size_t>(slot) * seg_bytes, src, seg_bytes, &full[slot]);
+        if (p.l2_evict_first)
+          bulk_load_hint(ring + static_cast<size_t>(slot) * seg_bytes, src, seg_bytes, &full[slot], policy);
+        else
+          bulk_load(ring + static_cast<size_t>(slot) * seg_bytes, src, seg_bytes, &full[slot]);
         issued = g + 1;
       }
       *issued_count = issued;  // read by the drain below
@@ -689,7 +733,7 @@ far_ring_kernel(const Params p, int nslot, int ncons) {
       const int64_t g = i * S + k;
       const int slot = static_cast<int>(g % nslot);
       const uint32_t round = static_cast<uint32_t>(g / nslot);
-      if (!*abort_flag && !mbar_wait(&full[slot], round & 1u, abort_flag)) {
+      if (!*abort_flag && !mbar_wait(&full[slot], round & 1u, abort_flag, p.wait_limit_ns)) {
         if (!*abort_flag) atomicOr(&g_far_error, kErrWaitFull);
         *abort_flag = 1;
       }
@@ -707,13 +751,13 @@ far_ring_kernel(const Params p, int nslot, int ncons) {
   // the producer to stop and then for the last phase of every used slot.
   if (threadIdx.x == 0) {
     const uint64_t t0 = global_ns();
-    while (!*producer_done && global_ns() - t0 < kWaitLimitNs) {
+    while (!*producer_done && global_ns() - t0 < p.wait_limit_ns) {
     }
     if (*abort_flag) {
       const int64_t issued = *issued_count;
       for (int64_t g = (issued > nslot ? issued - nslot : 0); g < issued; ++g) {
         const int slot = static_cast<int>(g % nslot);
-        mbar_wait(&full[slot], static_cast<uint32_t>(g / nslot) & 1u, nullptr);
+        mbar_wait(&full[slot], static_cast<uint32_t>(g / nslot) & 1u, nullptr, p.wait_limit_ns);
       }
     }
   }
@@ -766,7 +810,7 @@ cudaError_t launch_decode_t(const Params& p, const Launch& l, cudaStream_t s) {
   return cudaLaunchKernelEx(&cfg, far_decode_kernel<DT, VPT>, p);
 }
 
-template <class DT, int VPT>
+template <class DT, int VPT, int MINB>
 cudaError_t launch_ring_t(const Params& p, const Launch& l, cudaStream_t s) {
   Attrs at(l, 0);
   cudaLaunchConfig_t cfg = {};
@@ -776,16 +820,17 @@ cudaError_t launch_ring_t(const Params& p, const Launch& l, cudaStream_t s) {
   cfg.stream = s;
   cfg.attrs = at.a;
   cfg.numAttrs = at.n;
-  return cudaLaunchKernelEx(&cfg, far_ring_kernel<DT, VPT>, p, l.nslot, l.tpr);
+  return cudaLaunchKernelEx(&cfg, far_ring_kernel<DT, VPT, MINB>, p, l.nslot, l.tpr);
 }
 
 template <class DT>
 cudaError_t launch_ring_dt(const Params& p, const Launch& l, cudaStream_t s) {
+  const bool three = l.ring_minb >= 3;
   switch (l.vpt) {
-    case 1: return launch_ring_t<DT, 1>(p, l, s);
-    case 2: return launch_ring_t<DT, 2>(p, l, s);
-    case 4: return launch_ring_t<DT, 4>(p, l, s);
-    case 8: return launch_ring_t<DT, 8>(p, l, s);
+    case 1: return three ? launch_ring_t<DT, 1, 3>(p, l, s) : launch_ring_t<DT, 1, 2>(p, l, s);
+    case 2: return three ? launch_ring_t<DT, 2, 3>(p, l, s) : launch_ring_t<DT, 2, 2>(p, l, s);
+    case 4: return three ? launch_ring_t<DT, 4, 3>(p, l, s) : launch_ring_t<DT, 4, 2>(p, l, s);
+    case 8: return launch_ring_t<DT, 8, 1>(p, l, s);
     default: return cudaErrorInvalidConfiguration;
   }
 }
@@ -820,10 +865,13 @@ cudaError_t allow_large_smem() {
     if (e == cudaSuccess)
       e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kRingSmemMax);
   };
-  set(far_ring_kernel<DT, 1>);
-  set(far_ring_kernel<DT, 2>);
-  set(far_ring_kernel<DT, 4>);
-  set(far_ring_kernel<DT, 8>);
+  set(far_ring_kernel<DT, 1, 2>);
+  set(far_ring_kernel<DT, 2, 2>);
+  set(far_ring_kernel<DT, 4, 2>);
+  set(far_ring_kernel<DT, 1, 3>);
+  set(far_ring_kernel<DT, 2, 3>);
+  set(far_ring_kernel<DT, 4, 3>);
+  set(far_ring_kernel<DT, 8, 1>);
   return e;
 }
 
@@ -858,24 +906,30 @@ cudaError_t launch_ring(const Params& p, int dtype, const Launch& l, cudaStream_
 int ring_header_bytes(int nslot) { return ring_offset(nslot); }
 
 namespace {
-template <class DT>
-int ring_occupancy_dt(int vpt, int threads, int smem) {
+template <class DT, int VPT, int MINB>
+int occ_of(int threads, int smem) {
   int n = 0;
-  cudaError_t e = cudaErrorInvalidValue;
-  switch (vpt) {
-    case 1: e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, far_ring_kernel<DT, 1>, threads, smem); break;
-    case 2: e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, far_ring_kernel<DT, 2>, threads, smem); break;
-    case 4: e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, far_ring_kernel<DT, 4>, threads, smem); break;
-    case 8: e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, far_ring_kernel<DT, 8>, threads, smem); break;
-    default: break;
-  }
+  const cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(
+      &n, far_ring_kernel<DT, VPT, MINB>, threads, smem);
   return e == cudaSuccess ? n : 0;
+}
+
+template <class DT>
+int ring_occupancy_dt(int vpt, int minb, int threads, int smem) {
+  const bool three = minb >= 3;
+  switch (vpt) {
+    case 1: return three ? occ_of<DT, 1, 3>(threads, smem) : occ_of<DT, 1, 2>(threads, smem);
+    case 2: return three ? occ_of<DT, 2, 3>(threads, smem) : occ_of<DT, 2, 2>(threads, smem);
+    case 4: return three ? occ_of<DT, 4, 3>(threads, smem) : occ_of<DT, 4, 2>(threads, smem);
+    case 8: return occ_of<DT, 8, 1>(threads, smem);
+    default: return 0;
+  }
 }
 }  // namespace
 
-int ring_occupancy(int dtype, int vpt, int threads, int smem_bytes) {
-  return dtype == kBf16 ? ring_occupancy_dt<Bf16T>(vpt, threads, smem_bytes)
-                        : ring_occupancy_dt<Fp16T>(vpt, threads, smem_bytes);
+int ring_occupancy(int dtype, int vpt, int minb, int threads, int smem_bytes) {
+  return dtype == kBf16 ? ring_occupancy_dt<Bf16T>(vpt, minb, threads, smem_bytes)
+                        : ring_occupancy_dt<Fp16T>(vpt, minb, threads, smem_bytes);
 }
 
 cudaError_t configure_kernels() {

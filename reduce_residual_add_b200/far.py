@@ -48,7 +48,8 @@ FAR_FP8_TENSOR_NOALLOC_MAX_ROWS = 65536
 EXPORTS = ("far_create", "far_destroy", "far_fused", "far_fused_rows",
            "far_fp8_tensor_workspace_bytes", "far_fused_fp8_tensor",
            "far_fused_fp8_tensor_noalloc", "far_validate",
-           "far_set_regime", "far_describe_launch", "far_check", "far_status_string",
+           "far_set_regime", "far_describe_launch", "far_check", "far_test_stall",
+           "far_status_string",
            "far_last_error", "far_version")
 
 _DTYPES = {torch.bfloat16: FAR_BF16, torch.float16: FAR_FP16}
@@ -115,6 +116,8 @@ def lib() -> ctypes.CDLL:
     L.far_set_regime.restype = i32
     L.far_describe_launch.argtypes = [vp, i64, i64, i32, i32, i32, ctypes.POINTER(far_launch_info)]
     L.far_describe_launch.restype = i32
+    L.far_test_stall.argtypes = [vp, i64, ctypes.c_uint32]
+    L.far_test_stall.restype = i32
     L.far_check.argtypes = [vp, vp]
     L.far_check.restype = i32
     L.far_status_string.argtypes = [i32]
@@ -195,6 +198,14 @@ def far_describe_launch(ctx: FarContext, rows: int, H: int, dtype=torch.bfloat16
     if st != FAR_OK:
         raise FarError(st, "far_describe_launch")
     return {name: getattr(info, name) for name, _ in far_launch_info._fields_}
+
+
+def far_test_stall(ctx: FarContext, segment: int, wait_limit_us: int = 0) -> None:
+    """Test hook: make the ring kernel's wait for one segment run out
+    (see include/far.h); segment < 0 switches it off."""
+    st = lib().far_test_stall(ctx.handle, int(segment), int(wait_limit_us))
+    if st != FAR_OK:
+        raise FarError(st, "far_test_stall")
 
 
 def far_check(ctx: FarContext, stream=None) -> None:
@@ -366,3 +377,41 @@ def far_fused_fp8_tensor_noalloc(ctx: FarContext, partials: Sequence[torch.Tenso
                                             _stream(stream))
     if st != FAR_OK:
         raise FarError(st, "far_fused_fp8_tensor_noalloc")
+
+
+class FarCall:
+    """One far_fused_rows call with its arguments marshalled once.
+
+    Calling the object enqueues the kernel again on the same buffers (whose
+    contents may change between calls) with no per-call argument checks in
+    Python; the library still checks every argument on its side.  Meant for
+    loops of small calls (decode) where the binding's own marshalling would
+    dominate the launch.  Keyword arguments as far_fused; ``rows=(b, e)``
+    restricts the call to a row range.
+    """
+
+    def __init__(self, ctx: FarContext, partials: Sequence[torch.Tensor],
+                 residual: Optional[torch.Tensor], gamma: torch.Tensor, eps: float,
+                 weight_bias: float = 0.0, pattern: int = FAR_AR_RESIDUAL_RMSNORM, *,
+                 residual_out: Optional[torch.Tensor] = None,
+                 norm_out: Optional[torch.Tensor] = None,
+                 quant_out: Optional[torch.Tensor] = None,
+                 scale_in: Optional[torch.Tensor] = None,
+                 scale_out: Optional[torch.Tensor] = None, rows=None, stream=None):
+        (arr, W, res, rout, gam, T, H, dt, nout, qout, sin, sout) = _args(
+            partials, residual, gamma, residual_out, norm_out, quant_out, scale_in, scale_out)
+        b, e = (0, T) if rows is None else (int(rows[0]), int(rows[1]))
+        # keep every tensor alive for as long as the call may be replayed
+        self._keep = (list(partials) if not isinstance(partials, torch.Tensor) else [partials],
+                      residual, gamma, residual_out, norm_out, quant_out, scale_in, scale_out)
+        self._ctx = ctx
+        self._fn = lib().far_fused_rows
+        self._args = (ctx.handle, ctypes.c_int64(b), ctypes.c_int64(e), arr, ctypes.c_int(W), res,
+                      rout, gam, ctypes.c_int64(T), ctypes.c_int64(H), ctypes.c_int(dt),
+                      ctypes.c_float(eps), ctypes.c_float(weight_bias), ctypes.c_int(pattern),
+                      nout, qout, sin, sout, _stream(stream))
+
+    def __call__(self) -> None:
+        st = self._fn(*self._args)
+        if st != FAR_OK:
+            raise FarError(st, "far_fused_rows")

@@ -57,7 +57,8 @@ def kctx():
     any_rows = {"FAR_RING_MIN_ROWS": "1"}
     out = {"ring": _ctx_with_env(dict(any_rows)),
            "ring256": _ctx_with_env(dict(any_rows, FAR_RING_THREADS="256", FAR_RING_CTAS_PER_SM="1")),
-           "ring512": _ctx_with_env(dict(any_rows, FAR_RING_THREADS="512", FAR_RING_CTAS_PER_SM="1")),
+           "ring3": _ctx_with_env(dict(any_rows, FAR_RING_CTAS_PER_SM="3", FAR_L2_EVICT_FIRST="1",
+                                       FAR_STREAM_STORES="1")),
            "ring2": _ctx_with_env(dict(any_rows, FAR_RING_CTAS_PER_SM="2", FAR_RING_THREADS="256")),
            "ring4": _ctx_with_env(dict(any_rows, FAR_RING_CTAS_PER_SM="4", FAR_RING_THREADS="128")),
            "direct": _ctx_with_env({"FAR_PREFILL_KERNEL": "0"})}
@@ -109,7 +110,7 @@ def test_small_shapes(ctx, regime, case, reg):
     log("small %s reg%d" % (case, reg), compare(got, ref, dt))
 
 
-@pytest.mark.parametrize("kern", ["ring", "ring256", "ring512", "ring2", "ring4", "direct"])
+@pytest.mark.parametrize("kern", ["ring", "ring256", "ring3", "ring2", "ring4", "direct"])
 @pytest.mark.parametrize("case", [
     (2, 3000, 264, "bf16", 2, True, 0.0),    # 33 packs, 32 slots, ~20 rows per CTA
     (16, 300, 16384, "bf16", 1, True, 1.0),  # 17 segments per row, 6 slots
@@ -121,7 +122,7 @@ def test_prefill_kernels(kctx, case, kern):
     W, T, H, dt, pattern, has_res, wb = case
     c = kctx[kern]
     info = far.far_describe_launch(c, T, H, torch.bfloat16, W, has_res)
-    per_sm = {"ring4": 4, "ring2": 2}.get(kern, 1)
+    per_sm = {"ring4": 4, "ring3": 3, "ring2": 2}.get(kern, 1)
     fits = 228 * 1024 // per_sm - 1024 >= 3 * H * 2 + 1024   # gamma, two slots, header
     assert info["kernel"] == (1 if (kern != "direct" and fits) else 0)
     inp = random_inputs(W, T, H, dtype=dt, seed=7 * W + T + H, has_residual=has_res)
@@ -503,3 +504,54 @@ def test_per_tensor_fp8_repeated_in_a_graph(ctx):
     far.far_check(ctx)
     assert torch.equal(q, q0) and torch.equal(sc, s0)
     del gr
+
+
+def test_prepared_call_replays_on_new_contents(ctx):
+    """far.FarCall marshals once; each call uses the buffers' current contents."""
+    inp = random_inputs(8, 16, 4096, seed=61)
+    g = to_gpu(inp)
+    T, H = 16, 4096
+    rout = torch.empty(T, H, dtype=torch.bfloat16, device="cuda")
+    q = torch.empty(T, H, dtype=torch.uint8, device="cuda")
+    sc = torch.empty(T, dtype=torch.float32, device="cuda")
+    call = far.FarCall(ctx, g["partials"], g["residual"], g["gamma"], 1e-6, 1.0, 2,
+                       residual_out=rout, quant_out=q, scale_out=sc)
+    for k in range(3):
+        fresh = random_inputs(8, 16, 4096, seed=62 + k)
+        for dst, src in zip(g["partials"], fresh["partials"]):
+            dst.copy_(src)
+        call()
+        torch.cuda.synchronize()
+        from reduce_residual_add_b200.inputs import as_u16
+        got = {"residual_out": as_u16(rout.cpu()), "norm_out": None,
+               "quant_out": q.cpu().numpy(), "scale_out": sc.cpu().numpy()}
+        ref = run_oracle({"partials": fresh["partials"], "residual": inp["residual"],
+                          "gamma": inp["gamma"]}, "bf16", 1e-6, 1.0, 2, want_norm=False)
+        compare(got, ref, "bf16")
+
+
+def test_bounded_wait_gives_up_reports_timeout_and_context_stays_usable(kctx):
+    """Make a wait run out: the ring producer skips one bulk copy (a barrier
+    that nothing completes).  The consumers' wait gives up after 20 ms, the
+    kernel still ends, far_check reports FAR_ERR_TIMEOUT, and the next call
+    on the same context is correct."""
+    c = kctx["ring"]
+    inp = random_inputs(4, 600, 4096, seed=71)
+    g = to_gpu(inp)
+    assert far.far_describe_launch(c, 600, 4096, torch.bfloat16, 4, True)["kernel"] == 1
+    far.far_test_stall(c, 7, 20000)        # segment 7 of each CTA with two rows or more
+    try:
+        rout = torch.empty(600, 4096, dtype=torch.bfloat16, device="cuda")
+        nout = torch.empty_like(rout)
+        far.far_fused(c, g["partials"], g["residual"], g["gamma"], 1e-6, 0.0, 0,
+                      residual_out=rout, norm_out=nout)
+        torch.cuda.synchronize()
+        with pytest.raises(far.FarError) as e:
+            far.far_check(c)
+        assert e.value.status == far.FAR_ERR_TIMEOUT
+    finally:
+        far.far_test_stall(c, -1, 0)
+    far.far_check(c)                       # the word was cleared
+    got = run_gpu(c, g, 1e-6, 0.0, 0)
+    ref = run_oracle(inp, "bf16", 1e-6, 0.0, 0)
+    compare(got, ref, "bf16")
