@@ -555,3 +555,31 @@ def test_bounded_wait_gives_up_reports_timeout_and_context_stays_usable(kctx):
     got = run_gpu(c, g, 1e-6, 0.0, 0)
     ref = run_oracle(inp, "bf16", 1e-6, 0.0, 0)
     compare(got, ref, "bf16")
+
+
+@pytest.mark.parametrize("kern", ["ring", "direct", "decode"])
+def test_format_edges_overflow_and_subnormals(kctx, kern):
+    """fp16: partials of 30000 sum past 65504; y, held in fp32, stays finite,
+    so the new residual rounds to +inf in fp16 while the normalised output is
+    finite, on both sides.  bf16 / fp16: gamma in the subnormal range gives
+    subnormal normalised outputs, which must be kept, not flushed."""
+    c = kctx[kern]
+    T, H = 300 if kern != "decode" else 8, 4096
+    # overflow rows: fp16 partials of 30000 in the first columns of some rows
+    inp = random_inputs(4, T, H, dtype="fp16", seed=91)
+    for p in inp["partials"]:
+        p[::7, :16] = 30000.0
+    got = run_gpu(c, to_gpu(inp), 1e-6, 0.0, 0)
+    ref = run_oracle(inp, "fp16", 1e-6, 0.0, 0)
+    compare(got, ref, "fp16")
+    assert np.all(got["residual_out"][::7, :16] == 0x7C00)          # +inf
+    # subnormal outputs: gamma around 2^-130 (bf16) / 2^-20 (fp16)
+    for dt, tiny in (("bf16", 2.0 ** -130), ("fp16", 2.0 ** -20)):
+        inp = random_inputs(3, T, H, dtype=dt, seed=92)
+        tdt = torch.bfloat16 if dt == "bf16" else torch.float16
+        inp["gamma"] = (torch.rand(H, generator=torch.Generator().manual_seed(5)) * tiny).to(tdt)
+        got = run_gpu(c, to_gpu(inp), 1e-6, 0.0, 0)
+        ref = run_oracle(inp, dt, 1e-6, 0.0, 0)
+        compare(got, ref, dt)
+        exp = (got["norm_out"].astype(np.int64) >> (7 if dt == "bf16" else 10)) & (0xFF if dt == "bf16" else 0x1F)
+        assert np.mean(exp == 0) > 0.5                               # mostly subnormal, kept
