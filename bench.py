@@ -403,9 +403,10 @@ def run_far(args, world, rank, local):
         "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(total_max / args.steps * 1e3, 5),
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": wl.dtype,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
         "data": "synthetic",
         "config": {"workload": wl.name, "W": wl.W, "T": wl.T, "H": wl.H, "dtype": wl.dtype,
+                   "arithmetic": "fp32 accumulation; bf16/fp16 in and out; e4m3 codes",
                    "pattern": ["ar_residual_rmsnorm", "fp8_static", "fp8_per_token"][wl.pattern],
                    "norm_out": case.nout is not None, "eps": wl.eps,
                    "weight_bias": wl.weight_bias, "static_scale": wl.static_scale,
