@@ -16,6 +16,7 @@ sources and for the readings taken where the pages are silent):
     static FP8:  q = e4m3(fp32(fp32(o) / scale))
     per-token:   scale_t = fp32(max|fp32(o)| / 448); q = e4m3(fp32(fp32(o) / scale_t))
     per-tensor:  one scale = fp32(max over the rows of |fp32(o)| / 448), in scale_out[0]
+    per-group:   one scale per (row, group of `group` elements), amax / 448
 """
 from __future__ import annotations
 
@@ -28,7 +29,7 @@ import numpy as np
 from . import build as _build
 
 BF16, FP16 = 0, 1
-AR_RESIDUAL_RMSNORM, FP8_STATIC, FP8_TOKEN, FP8_TENSOR = 0, 1, 2, 3
+AR_RESIDUAL_RMSNORM, FP8_STATIC, FP8_TOKEN, FP8_TENSOR, FP8_GROUP = 0, 1, 2, 3, 4
 
 _lib = None
 
@@ -49,7 +50,7 @@ def load(path: str) -> ctypes.CDLL:
     L.far_oracle_fused.argtypes = [
         ctypes.POINTER(vp), ctypes.c_int, vp, vp,
         ctypes.c_int64, ctypes.c_int64, ctypes.c_int,
-        ctypes.c_float, ctypes.c_float, ctypes.c_int,
+        ctypes.c_float, ctypes.c_float, ctypes.c_int, ctypes.c_int64,
         ctypes.c_int64, ctypes.c_int64,
         vp, vp, vp, vp, vp, vp, vp, vp]
     return L
@@ -104,7 +105,7 @@ def fused(partials: Sequence[np.ndarray], residual: Optional[np.ndarray],
           pattern: int = AR_RESIDUAL_RMSNORM, scale_in: Optional[float] = None,
           rows: Optional[tuple] = None, want_norm: bool = True,
           want_residual_out: bool = True, debug: bool = False,
-          out: Optional[dict] = None) -> dict:
+          out: Optional[dict] = None, group: int = 0) -> dict:
     """Run the oracle on raw bit patterns.
 
     ``partials`` are W arrays of uint16 patterns of shape (..., H) (any
@@ -140,7 +141,7 @@ def fused(partials: Sequence[np.ndarray], residual: Optional[np.ndarray],
         o.setdefault("norm_out", np.zeros((T, H), np.uint16))
     else:
         o["norm_out"] = None
-    if pattern in (FP8_STATIC, FP8_TOKEN, FP8_TENSOR):
+    if pattern in (FP8_STATIC, FP8_TOKEN, FP8_TENSOR, FP8_GROUP):
         o.setdefault("quant_out", np.zeros((T, H), np.uint8))
     else:
         o["quant_out"] = None
@@ -148,6 +149,10 @@ def fused(partials: Sequence[np.ndarray], residual: Optional[np.ndarray],
         o.setdefault("scale_out", np.zeros((T,), np.float32))
     elif pattern == FP8_TENSOR:
         o.setdefault("scale_out", np.zeros((1,), np.float32))
+    elif pattern == FP8_GROUP:
+        if group < 1 or H % group:
+            raise ValueError("group must divide H")
+        o.setdefault("scale_out", np.zeros((T, H // group), np.float32))
     else:
         o["scale_out"] = None
     sin = None
@@ -163,7 +168,7 @@ def fused(partials: Sequence[np.ndarray], residual: Optional[np.ndarray],
     arr = (ctypes.c_void_p * W)(*[p.ctypes.data for p in ps])
     rc = lib().far_oracle_fused(
         arr, W, _ptr(res), _ptr(gamma), T, H, dt,
-        float(eps), float(weight_bias), int(pattern), b, e,
+        float(eps), float(weight_bias), int(pattern), int(group), b, e,
         _ptr(o["residual_out"]), _ptr(o["norm_out"]), _ptr(o["quant_out"]),
         _ptr(sin), _ptr(o["scale_out"]),
         _ptr(o.get("y")), _ptr(o.get("o")), _ptr(o.get("rinv")))
@@ -173,5 +178,6 @@ def fused(partials: Sequence[np.ndarray], residual: Optional[np.ndarray],
 
 
 __all__ = ["BF16", "FP16", "AR_RESIDUAL_RMSNORM", "FP8_STATIC", "FP8_TOKEN", "FP8_TENSOR",
+           "FP8_GROUP",
            "load", "lib", "dtype_code", "decode16", "round16", "e4m3_decode",
            "e4m3_encode", "fused"]

@@ -30,6 +30,9 @@
  *       The same page lists kFp8DynamicTensorSym (dynamic, per-tensor,
  *       symmetric) among the quantisation keys, with no fused op: one scale
  *       for the whole tensor, amax / 448 over every element.
+ *  [P3] vllm.distributed.device_communicators.aiter_custom_all_reduce --
+ *       build_supports_per_group_quant: a fused all-reduce + RMSNorm +
+ *       per-group quantisation exists; the page gives no group shape.
  *  [P5] PR #45307 report -- signature of call_trtllm_fused_allreduce_norm:
  *       norm_out, quant_out, scale_out and scale_factor are all optional.
  *
@@ -55,7 +58,10 @@
  *  - a dynamic row whose fp32 scale is 0 gets scale 0 and all codes 0x00;
  *    NaN elements take no part in a row's amax;
  *  - dynamic per-tensor FP8 takes its amax over the rows of the call
- *    ([row_begin, row_end)) and writes the one scale to scale_out[0].
+ *    ([row_begin, row_end)) and writes the one scale to scale_out[0];
+ *  - per-group FP8: groups of `group` consecutive hidden elements of a row
+ *    (group divides H), one scale per (row, group) = amax / 448 at
+ *    scale_out[t * (H / group) + h / group].
  */
 #include <math.h>
 #include <stddef.h>
@@ -65,7 +71,8 @@
 /* Own copies of the enumerations; numbering follows the library's public
  * interface so that callers can pass the same integers to both. */
 enum { OR_BF16 = 0, OR_FP16 = 1 };
-enum { OR_AR_RESIDUAL_RMSNORM = 0, OR_FP8_STATIC = 1, OR_FP8_TOKEN = 2, OR_FP8_TENSOR = 3 };
+enum { OR_AR_RESIDUAL_RMSNORM = 0, OR_FP8_STATIC = 1, OR_FP8_TOKEN = 2, OR_FP8_TENSOR = 3,
+       OR_FP8_GROUP = 4 };
 
 /* ---------------------------------------------------------------------- */
 /* 16-bit floating formats                                                 */
@@ -253,7 +260,9 @@ static double row_y_o(const uint16_t *const *partials, int W, const uint16_t *re
  *   quant_out     receives e4m3 codes (patterns 1, 2); may be NULL
  *   scale_in      static per-tensor scale (pattern 1)
  *   scale_out     per-row fp32 scale (pattern 2), indexed by absolute row,
- *                 or the one per-tensor scale in scale_out[0] (pattern 3)
+ *                 or the one per-tensor scale in scale_out[0] (pattern 3),
+ *                 or T x (H / group) per-group scales, row-major (pattern 4)
+ *   group         elements per quantisation group (pattern 4)
  *   y_dbg, o_dbg  optional fp64 copies of y and o (T*H each)
  *   rinv_dbg      optional fp64 1/sqrt(ms+eps) per row (T)
  *
@@ -262,7 +271,7 @@ static double row_y_o(const uint16_t *const *partials, int W, const uint16_t *re
 int far_oracle_fused(const uint16_t *const *partials, int W,
                      const uint16_t *residual, const uint16_t *gamma,
                      int64_t T, int64_t H, int dtype,
-                     float eps, float weight_bias, int pattern,
+                     float eps, float weight_bias, int pattern, int64_t group,
                      int64_t row_begin, int64_t row_end,
                      uint16_t *residual_out, uint16_t *norm_out,
                      uint8_t *quant_out, const float *scale_in,
@@ -276,8 +285,10 @@ int far_oracle_fused(const uint16_t *const *partials, int W,
         return -1;
     if (pattern == OR_FP8_STATIC && (quant_out == NULL || scale_in == NULL))
         return -1;
-    if ((pattern == OR_FP8_TOKEN || pattern == OR_FP8_TENSOR) &&
+    if ((pattern == OR_FP8_TOKEN || pattern == OR_FP8_TENSOR || pattern == OR_FP8_GROUP) &&
         (quant_out == NULL || scale_out == NULL))
+        return -1;
+    if (pattern == OR_FP8_GROUP && (group < 1 || H % group != 0))
         return -1;
 
     /* one row of y and o at a time, in fp64 */
@@ -340,6 +351,28 @@ int far_oracle_fused(const uint16_t *const *partials, int W,
                     quant_out[base + h] = 0x00;
                 else
                     quant_out[base + h] = far_oracle_e4m3_encode(to_f32(to_f32(o[h]) / scale));
+            }
+        }
+
+        /* 5d. per-group FP8 [P3 per-group quant]: each group of `group`
+         * consecutive elements has its own scale, amax / 448 */
+        if (pattern == OR_FP8_GROUP) {
+            const int64_t ngroups = H / group;
+            for (int64_t q = 0; q < ngroups; ++q) {
+                double amax = 0.0;
+                for (int64_t h = q * group; h < (q + 1) * group; ++h) {
+                    double a = fabs(to_f32(o[h]));
+                    if (a > amax) /* a NaN element does not take part */
+                        amax = a;
+                }
+                double scale = to_f32(amax / 448.0);
+                scale_out[t * ngroups + q] = (float)scale;
+                for (int64_t h = q * group; h < (q + 1) * group; ++h) {
+                    if (scale == 0.0)
+                        quant_out[base + h] = 0x00;
+                    else
+                        quant_out[base + h] = far_oracle_e4m3_encode(to_f32(to_f32(o[h]) / scale));
+                }
             }
         }
 

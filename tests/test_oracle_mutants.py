@@ -53,6 +53,8 @@ MUTANTS = {
     "per-tensor amax of the first row only": ("            row_y_o(partials, W, residual, gamma, t, H, dtype, eps, weight_bias, y, o);\n            for (int64_t h = 0; h < H; ++h) {",
                                               "            row_y_o(partials, W, residual, gamma, t, H, dtype, eps, weight_bias, y, o);\n            if (t > row_begin) break;\n            for (int64_t h = 0; h < H; ++h) {"),
     "per-tensor scale over 240": ("tensor_scale = to_f32(amax / 448.0);", "tensor_scale = to_f32(amax / 240.0);"),
+    "per-group amax over the first group only": ("for (int64_t h = q * group; h < (q + 1) * group; ++h) {\n                    double a", "for (int64_t h = 0; h < group; ++h) {\n                    double a"),
+    "per-group scales indexed by group only": ("scale_out[t * ngroups + q] = (float)scale;", "scale_out[q] = (float)scale;"),
     "y squared without the residual": ("ss += y[h] * y[h];", "ss += (y[h] - (residual ? far_oracle_decode16(residual[base + h], dtype) : 0.0)) * (y[h] - (residual ? far_oracle_decode16(residual[base + h], dtype) : 0.0));"),
 }
 
@@ -71,6 +73,10 @@ def quick_pins():
     yield "worked fp32 decision", pins.test_worked_example_fp8_code_decided_in_fp32
     yield "worked fp32 decision dynamic", pins.test_worked_example_dynamic_fp8_code_decided_in_fp32
     yield "worked per-tensor", pins.test_worked_example_per_tensor_fp8
+    yield "worked per-group", pins.test_worked_example_per_group_fp8
+    for dt in ("bf16", "fp16"):
+        yield "per-group invariants %s" % dt, lambda d=dt: pins.test_per_group_invariants(d)
+    yield "brute force per-group", lambda: pins.test_brute_force_exact_per_group((2, 8, 64), 16, "bf16")
     for dt in ("bf16", "fp16"):
         yield "per-tensor vs per-token %s" % dt, lambda d=dt: pins.test_per_tensor_scale_is_the_largest_per_token_scale(d)
     yield "worked zeros", pins.test_worked_example_zero_input_scale_one

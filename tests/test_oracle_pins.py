@@ -185,7 +185,7 @@ def test_e4m3_matches_torch_cast_in_range():
 # exact-rational brute force of the whole epilogue
 # ---------------------------------------------------------------------------
 
-def exact_fused(ps, res, gam, dt, eps, wb, pattern, scale_in=None):
+def exact_fused(ps, res, gam, dt, eps, wb, pattern, scale_in=None, group=0):
     """Fraction-exact epilogue on bit patterns (lists of rows of ints)."""
     T, H = len(ps[0]), len(gam)
     epsq, wbq = f32(eps), f32(wb)
@@ -226,6 +226,15 @@ def exact_fused(ps, res, gam, dt, eps, wb, pattern, scale_in=None):
                 out["quant_out"].append([0] * H)
             else:
                 out["quant_out"].append([encode(e4m3_sat(rne(v / sc, "fp32")), "e4m3") for v in o32])
+        elif pattern == oracle.FP8_GROUP:
+            assert all(v is not None for v in o32)
+            codes = []
+            for q in range(H // group):
+                chunk = o32[q * group:(q + 1) * group]
+                sc = rne(max(abs(v) for v in chunk) / 448, "fp32")
+                out["scale_out"].append(sc)
+                codes += [0] * group if sc == 0 else [encode(e4m3_sat(rne(v / sc, "fp32")), "e4m3") for v in chunk]
+            out["quant_out"].append(codes)
         rows.append(o32)
     if pattern == oracle.FP8_TENSOR:
         # one scale: amax over every row of the call
@@ -239,13 +248,13 @@ def exact_fused(ps, res, gam, dt, eps, wb, pattern, scale_in=None):
     return out
 
 
-def _compare_exact(inp, dt, eps, wb, pattern, scale_in=None):
+def _compare_exact(inp, dt, eps, wb, pattern, scale_in=None, group=0):
     ps = [as_u16(p) for p in inp["partials"]]
     res = None if inp["residual"] is None else as_u16(inp["residual"])
     gam = as_u16(inp["gamma"])
-    got = oracle.fused(ps, res, gam, dt, eps, wb, pattern, scale_in=scale_in)
+    got = oracle.fused(ps, res, gam, dt, eps, wb, pattern, scale_in=scale_in, group=group)
     ex = exact_fused([p.tolist() for p in ps], None if res is None else res.tolist(),
-                     gam.tolist(), dt, eps, wb, pattern, scale_in)
+                     gam.tolist(), dt, eps, wb, pattern, scale_in, group)
     np.testing.assert_array_equal(zero_sign_free(got["residual_out"]),
                                   zero_sign_free(np.array(ex["residual_out"], np.uint16)))
     n_amb = 0
@@ -264,9 +273,10 @@ def _compare_exact(inp, dt, eps, wb, pattern, scale_in=None):
                     continue
                 a = int(got["quant_out"][t, h])
                 assert (a if a & 0x7F else 0) == (v if v & 0x7F else 0), (t, h, hex(a), hex(v))
-    if pattern in (oracle.FP8_TOKEN, oracle.FP8_TENSOR):
+    if pattern in (oracle.FP8_TOKEN, oracle.FP8_TENSOR, oracle.FP8_GROUP):
+        flat = got["scale_out"].reshape(-1)
         for t, sc in enumerate(ex["scale_out"]):
-            assert Fraction(float(got["scale_out"][t])) == sc
+            assert Fraction(float(flat[t])) == sc
     assert n_amb == 0
 
 
@@ -279,6 +289,14 @@ def test_brute_force_exact_tiny(shape, pattern, dt):
     W, T, H = shape
     inp = random_inputs(W, T, H, dtype=dt, seed=100 + W * 7 + T + H + pattern)
     _compare_exact(inp, dt, eps=1e-6, wb=0.0, pattern=pattern, scale_in=0.05)
+
+
+@pytest.mark.parametrize("dt", ["bf16", "fp16"])
+@pytest.mark.parametrize("shape,group", [((2, 8, 4), 2), ((3, 5, 16), 8), ((2, 8, 64), 16), ((1, 4, 32), 32)])
+def test_brute_force_exact_per_group(shape, group, dt):
+    W, T, H = shape
+    inp = random_inputs(W, T, H, dtype=dt, seed=300 + W + T + H + group)
+    _compare_exact(inp, dt, eps=1e-6, wb=0.0, pattern=oracle.FP8_GROUP, group=group)
 
 
 @pytest.mark.parametrize("pattern", [0, 1, 2, 3])
@@ -425,6 +443,40 @@ def test_per_tensor_scale_is_the_largest_per_token_scale(dt):
     # the row range sets the tensor: rows [10, 20) only
     part = oracle.fused(*args, oracle.FP8_TENSOR, rows=(10, 20))
     assert part["scale_out"][0] == tok["scale_out"][10:20].max()
+
+
+def test_worked_example_per_group_fp8():
+    # the dynamic example's row, groups of 2: fp32(o) = [1.75, 17/256 | 0.75, 0.5].
+    # group 0: amax 1.75, scale 2^-8, o/s = [448, 17] -> 0x7E, 0x58 (tie to even
+    # in fp32); group 1: amax 0.75, scale fp32(0.75/448), o/s ~ [448, 298.7]
+    # -> 0x7E, 0x79 (288 = 1.125*2^8)
+    eps = 7903 / 65536 - 2.0 ** -27
+    r = oracle.fused([_bits([3.5, 17 / 128, 1.5, 1.0])], None, _bits([1, 1, 1, 1])[0], "bf16",
+                     eps=eps, pattern=oracle.FP8_GROUP, group=2)
+    s1 = struct.unpack("<f", struct.pack("<f", 0.75 / 448))[0]
+    assert r["scale_out"].tolist() == [[2.0 ** -8, s1]]
+    assert r["quant_out"][0].tolist() == [0x7E, 0x58, 0x7E, 0x79]
+
+
+@pytest.mark.parametrize("dt", ["bf16", "fp16"])
+def test_per_group_invariants(dt):
+    """One group spanning the row is per-token FP8, bit for bit; with smaller
+    groups each row's largest group scale is its per-token scale, and every
+    group holds a +-448 code."""
+    wl = WORKLOADS["c5_gemma_fp8_token_%s" % dt].with_(T=24)
+    inp = make_inputs(wl)
+    args = ([as_u16(p) for p in inp["partials"]], as_u16(inp["residual"]), as_u16(inp["gamma"]),
+            dt, wl.eps, wl.weight_bias)
+    tok = oracle.fused(*args, oracle.FP8_TOKEN)
+    whole = oracle.fused(*args, oracle.FP8_GROUP, group=wl.H)
+    np.testing.assert_array_equal(whole["quant_out"], tok["quant_out"])
+    np.testing.assert_array_equal(whole["scale_out"][:, 0], tok["scale_out"])
+    g128 = oracle.fused(*args, oracle.FP8_GROUP, group=128)
+    assert g128["scale_out"].shape == (24, wl.H // 128)
+    np.testing.assert_array_equal(g128["scale_out"].max(axis=1), tok["scale_out"])
+    q = (g128["quant_out"] & 0x7F).reshape(24, wl.H // 128, 128)
+    assert np.all(np.any(q == 0x7E, axis=2))
+    np.testing.assert_array_equal(g128["residual_out"], tok["residual_out"])
 
 
 def test_worked_example_zero_input_scale_one():
