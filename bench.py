@@ -52,12 +52,14 @@ def algorithmic_bytes(wl: Workload, rows: int, with_norm: bool) -> int:
     b += T * H * 2              # new residual out
     if with_norm:
         b += T * H * 2
-    if wl.pattern in (1, 2, 3):
+    if wl.pattern in (1, 2, 3, 4):
         b += T * H             # e4m3 codes
     if wl.pattern == 2:
         b += 4 * T             # per-token scales
     if wl.pattern == 3:
         b += 4                 # the one per-tensor scale
+    if wl.pattern == 4:
+        b += 4 * T * (H // wl.group_size)   # per-group scales
     return b
 
 
@@ -223,8 +225,9 @@ class Case:
         self.rout = torch.empty(T, H, dtype=dt, device=device)
         self.nout = torch.empty(T, H, dtype=dt, device=device) if (with_norm or wl.pattern == 0) else None
         self.qout = torch.empty(T, H, dtype=torch.uint8, device=device) if wl.pattern else None
-        self.sout = (torch.empty(T if wl.pattern == 2 else 1, dtype=torch.float32, device=device)
-                     if wl.pattern in (2, 3) else None)
+        n_scales = {2: T, 3: 1, 4: T * (H // wl.group_size if wl.group_size else 1)}.get(wl.pattern, 0)
+        self.sout = (torch.empty(n_scales, dtype=torch.float32, device=device)
+                     if wl.pattern in (2, 3, 4) else None)
         self.ws = (torch.empty(far.far_fp8_tensor_workspace_bytes(T), dtype=torch.uint8, device=device)
                    if wl.pattern == 3 else None)
         self.sin = (torch.tensor([wl.static_scale], dtype=torch.float32, device=device)
@@ -239,6 +242,13 @@ class Case:
                                 scale_out=self.sout, stream=self.stream)
 
     def step(self):
+        if self.wl.pattern == 4:
+            self.far.far_fused_fp8_group(self.ctx, self.ps, self.res, self.gam, self.wl.eps,
+                                         self.wl.weight_bias, group_size=self.wl.group_size,
+                                         quant_out=self.qout, scale_out=self.sout,
+                                         residual_out=self.rout, norm_out=self.nout,
+                                         stream=self.stream)
+            return
         if self.wl.pattern == 3:
             self.far.far_fused_fp8_tensor(self.ctx, self.ps, self.res, self.gam, self.wl.eps,
                                           self.wl.weight_bias, quant_out=self.qout,
@@ -446,7 +456,7 @@ def extras(ctx, device, stream) -> dict:
     out = {}
     peak, _ = hbm_peak()
     for name in ("c5_gemma_fp8_token_bf16", "c5_gemma_fp8_token_fp16", "c4_prefill_fp8_tensor",
-                 "c3_3d"):
+                 "c4_prefill_fp8_group128", "c3_3d"):
         wl = WORKLOADS[name]
         inp = make_inputs(wl)
         case = Case(ctx, wl, inp, device, False, stream)

@@ -89,7 +89,10 @@ typedef enum {
     FAR_AR_RESIDUAL_RMSNORM_FP8_TOKEN = 2,
     /* + quant_out and scale_out[0] (one fp32 scale for all rows of the call);
      * only through far_fused_fp8_tensor, which takes a workspace */
-    FAR_AR_RESIDUAL_RMSNORM_FP8_TENSOR = 3
+    FAR_AR_RESIDUAL_RMSNORM_FP8_TENSOR = 3,
+    /* + quant_out and scale_out[T][H / group] (one fp32 scale per row and
+     * group of consecutive elements); only through far_fused_fp8_group */
+    FAR_AR_RESIDUAL_RMSNORM_FP8_GROUP = 4
 } far_pattern;
 
 typedef enum {
@@ -108,9 +111,7 @@ typedef enum {
  * per ring CTA, at most 256 (default 256), FAR_RING_SLOTS: row-segment slots
  * per ring CTA (2..32; default: about 72 KiB of segments, as many as fit),
  * FAR_PDL=1|0: launch with programmatic dependent launch, default 1,
- * FAR_RING_MIN_ROWS: fewest rows for the ring kernel, default by rule,
- * FAR_L2_EVICT_FIRST=0|1: ring loads marked evict-first in L2, default 0,
- * FAR_STREAM_STORES=0|1: outputs stored with st.global.cs, default 0). */
+ * FAR_RING_MIN_ROWS: fewest rows for the ring kernel, default by rule). */
 /*
  * Programmatic dependent launch: every kernel of this library first waits
  * (griddepcontrol.wait) until the grid it depends on has completed, then
@@ -162,8 +163,9 @@ far_status far_destroy(far_ctx *ctx);
  *  quant_out     (T, H) uint8 e4m3fn codes; required by the FP8 patterns.
  *  scale_in      device pointer to one fp32 (static FP8 only).
  *  scale_out     device array of T fp32 (per-token FP8 only).
- *  pattern       FAR_AR_RESIDUAL_RMSNORM_FP8_TENSOR is refused here
- *                (FAR_ERR_INVALID_ARG): use far_fused_fp8_tensor.
+ *  pattern       FAR_AR_RESIDUAL_RMSNORM_FP8_TENSOR and _FP8_GROUP are
+ *                refused here (FAR_ERR_INVALID_ARG): use far_fused_fp8_tensor
+ *                and far_fused_fp8_group.
  *  stream        a cudaStream_t (NULL: the legacy default stream).
  *
  * Tensor pointers must be 16-byte aligned, scale pointers 4-byte aligned.
@@ -221,6 +223,26 @@ far_status far_fused_fp8_tensor(far_ctx *ctx, int64_t row_begin, int64_t row_end
                                 void *norm_out, void *quant_out, float *scale_out,
                                 void *workspace, size_t workspace_bytes, void *stream);
 
+/*
+ * Per-group FP8 (vllm.distributed.device_communicators.aiter_custom_all_reduce,
+ * build_supports_per_group_quant: a fused all-reduce + RMSNorm + per-group
+ * quantisation, whose group shape the page does not give): the epilogue on
+ * rows [row_begin, row_end) with one fp32 scale per row and per group of
+ * `group_size` consecutive hidden elements, scale = max |o| over the group
+ * / 448, written to scale_out[t * (H / group_size) + h / group_size], and
+ * quant_out = e4m3_satfinite(o / that scale).  group_size: a power of two
+ * from 8 to 256 dividing H (else FAR_ERR_UNSUPPORTED).  scale_out holds
+ * T * (H / group_size) floats and overlaps no other buffer.  Other
+ * arguments as far_fused_rows.
+ */
+far_status far_fused_fp8_group(far_ctx *ctx, int64_t row_begin, int64_t row_end,
+                               const void *const *partials, int W,
+                               const void *residual, void *residual_out,
+                               const void *gamma, int64_t T, int64_t H, far_dtype dtype,
+                               float eps, float weight_bias, int group_size,
+                               void *norm_out, void *quant_out, float *scale_out,
+                               void *stream);
+
 /* Rows one far_fused_fp8_tensor_noalloc call can take. */
 #define FAR_FP8_TENSOR_NOALLOC_MAX_ROWS 65536
 
@@ -257,7 +279,9 @@ far_status far_fused_fp8_tensor_noalloc(far_ctx *ctx, int64_t row_begin, int64_t
 /* Host-only: the status far_fused_rows would return for these arguments
  * before launching (it touches no GPU and needs no context).  With pattern
  * FAR_AR_RESIDUAL_RMSNORM_FP8_TENSOR it checks far_fused_fp8_tensor's
- * arguments other than the workspace. */
+ * arguments other than the workspace; with FAR_AR_RESIDUAL_RMSNORM_FP8_GROUP
+ * those of far_fused_fp8_group other than the group size and the extent of
+ * scale_out (a scale_out of T floats is assumed for the overlap checks). */
 far_status far_validate(int64_t row_begin, int64_t row_end,
                         const void *const *partials, int W,
                         const void *residual, const void *residual_out,

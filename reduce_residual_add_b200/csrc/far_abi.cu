@@ -29,8 +29,6 @@ struct far_ctx {
   int ring_slots_max;   // at most this many ring slots
   int pdl;              // programmatic dependent launch on every call
   int ring_min_rows;    // fewer rows than this take the direct kernel
-  int l2_evict_first;   // ring bulk loads with an L2 evict-first policy
-  int stream_stores;    // outputs stored with st.global.cs
   uint64_t wait_limit_ns;  // bounded waits in the kernels give up after this
   int64_t stall_segment;   // test hook (far_test_stall), -1 when off
   // ring CTAs per SM the occupancy calculator allows, per (dtype, packs):
@@ -280,8 +278,6 @@ far_status far_create(far_ctx** ctx, int device) {
   if (c.ring_threads > far::kRingMaxConsumers) c.ring_threads = far::kRingMaxConsumers;
   c.pdl = env_int("FAR_PDL", 1) != 0 ? 1 : 0;
   c.ring_min_rows = env_int("FAR_RING_MIN_ROWS", 0);  // 0: the measured rule
-  c.l2_evict_first = env_int("FAR_L2_EVICT_FIRST", 0) != 0 ? 1 : 0;
-  c.stream_stores = env_int("FAR_STREAM_STORES", 0) != 0 ? 1 : 0;
   c.wait_limit_ns = 2000000000ull;
   c.stall_segment = -1;
   c.force_regime = FAR_REGIME_AUTO;
@@ -379,7 +375,8 @@ far_status far_validate(int64_t row_begin, int64_t row_end, const void* const* p
   if (T < 0 || H <= 0) return FAR_ERR_INVALID_ARG;
   if (dtype != FAR_BF16 && dtype != FAR_FP16) return FAR_ERR_INVALID_ARG;
   if (pattern != FAR_AR_RESIDUAL_RMSNORM && pattern != FAR_AR_RESIDUAL_RMSNORM_FP8_STATIC &&
-      pattern != FAR_AR_RESIDUAL_RMSNORM_FP8_TOKEN && pattern != FAR_AR_RESIDUAL_RMSNORM_FP8_TENSOR)
+      pattern != FAR_AR_RESIDUAL_RMSNORM_FP8_TOKEN && pattern != FAR_AR_RESIDUAL_RMSNORM_FP8_TENSOR &&
+      pattern != FAR_AR_RESIDUAL_RMSNORM_FP8_GROUP)
     return FAR_ERR_INVALID_ARG;
   if (H % far::kPackElems != 0 || H > FAR_MAX_H) return FAR_ERR_UNSUPPORTED;
   if (row_begin < 0 || row_end < row_begin || row_end > T) return FAR_ERR_INVALID_ARG;
@@ -392,7 +389,8 @@ far_status far_validate(int64_t row_begin, int64_t row_end, const void* const* p
   if (pattern == FAR_AR_RESIDUAL_RMSNORM && norm_out == nullptr) return FAR_ERR_INVALID_ARG;
   if (pattern == FAR_AR_RESIDUAL_RMSNORM_FP8_STATIC && (quant_out == nullptr || scale_in == nullptr))
     return FAR_ERR_INVALID_ARG;
-  if ((pattern == FAR_AR_RESIDUAL_RMSNORM_FP8_TOKEN || pattern == FAR_AR_RESIDUAL_RMSNORM_FP8_TENSOR) &&
+  if ((pattern == FAR_AR_RESIDUAL_RMSNORM_FP8_TOKEN || pattern == FAR_AR_RESIDUAL_RMSNORM_FP8_TENSOR ||
+       pattern == FAR_AR_RESIDUAL_RMSNORM_FP8_GROUP) &&
       (quant_out == nullptr || scale_out == nullptr))
     return FAR_ERR_INVALID_ARG;
 
@@ -415,7 +413,8 @@ far_status far_validate(int64_t row_begin, int64_t row_end, const void* const* p
     if (res_w != nullptr) outs[no++] = span(res_w, tb);  // outs[0] when present
     if (norm_out != nullptr) outs[no++] = span(norm_out, tb);
     if (pattern != FAR_AR_RESIDUAL_RMSNORM) outs[no++] = span(quant_out, T * H);
-    if (pattern == FAR_AR_RESIDUAL_RMSNORM_FP8_TOKEN) outs[no++] = span(scale_out, T * 4);
+    if (pattern == FAR_AR_RESIDUAL_RMSNORM_FP8_TOKEN || pattern == FAR_AR_RESIDUAL_RMSNORM_FP8_GROUP)
+      outs[no++] = span(scale_out, T * 4);  // per group: the full extent is checked by far_fused_fp8_group
     if (pattern == FAR_AR_RESIDUAL_RMSNORM_FP8_TENSOR) outs[no++] = span(scale_out, 4);
     Range ins[FAR_MAX_W + 3];
     int ni = 0;
@@ -518,8 +517,6 @@ far_status far_fused_fp8_tensor_launch(far_ctx* ctx, int64_t row_begin, int64_t 
   far::Params p = make_params(partials, W, residual, residual_out, gamma, H,
                               FAR_AR_RESIDUAL_RMSNORM_FP8_TENSOR, eps, weight_bias, norm_out,
                               quant_out, nullptr, scale_out);
-  p.l2_evict_first = ctx->l2_evict_first;
-  p.stream_stores = ctx->stream_stores;
   p.wait_limit_ns = ctx->wait_limit_ns;
   p.stall_segment = ctx->stall_segment;
   p.ws_amax = static_cast<unsigned*>(workspace);
@@ -559,8 +556,10 @@ far_status far_fused_rows(far_ctx* ctx, int64_t row_begin, int64_t row_end,
                           void* norm_out, void* quant_out, const float* scale_in, float* scale_out,
                           void* stream) {
   if (ctx == nullptr) return FAR_ERR_INVALID_ARG;
-  // the per-tensor pattern needs a workspace: far_fused_fp8_tensor
-  if (pattern == FAR_AR_RESIDUAL_RMSNORM_FP8_TENSOR) return FAR_ERR_INVALID_ARG;
+  // the per-tensor pattern needs a workspace (far_fused_fp8_tensor), the
+  // per-group one a group size (far_fused_fp8_group)
+  if (pattern == FAR_AR_RESIDUAL_RMSNORM_FP8_TENSOR || pattern == FAR_AR_RESIDUAL_RMSNORM_FP8_GROUP)
+    return FAR_ERR_INVALID_ARG;
   far_status st = far_validate(row_begin, row_end, partials, W, residual, residual_out, gamma, T, H,
                                dtype, eps, weight_bias, pattern, norm_out, quant_out, scale_in,
                                scale_out);
@@ -569,8 +568,6 @@ far_status far_fused_rows(far_ctx* ctx, int64_t row_begin, int64_t row_end,
 
   far::Params p = make_params(partials, W, residual, residual_out, gamma, H, pattern, eps,
                               weight_bias, norm_out, quant_out, scale_in, scale_out);
-  p.l2_evict_first = ctx->l2_evict_first;
-  p.stream_stores = ctx->stream_stores;
   p.wait_limit_ns = ctx->wait_limit_ns;
   p.stall_segment = ctx->stall_segment;
   DeviceGuard guard(ctx->device);
@@ -683,6 +680,55 @@ far_status far_fused_fp8_tensor_noalloc(far_ctx* ctx, int64_t row_begin, int64_t
   return far_fused_fp8_tensor_launch(ctx, row_begin, row_end, partials, W, residual, residual_out,
                                      gamma, H, dtype, eps, weight_bias, norm_out, quant_out,
                                      scale_out, scratch, stream);
+}
+
+far_status far_fused_fp8_group(far_ctx* ctx, int64_t row_begin, int64_t row_end,
+                               const void* const* partials, int W, const void* residual,
+                               void* residual_out, const void* gamma, int64_t T, int64_t H,
+                               far_dtype dtype, float eps, float weight_bias, int group_size,
+                               void* norm_out, void* quant_out, float* scale_out, void* stream) {
+  if (ctx == nullptr) return FAR_ERR_INVALID_ARG;
+  if (group_size < 8 || group_size > 256 || (group_size & (group_size - 1)) != 0)
+    return FAR_ERR_UNSUPPORTED;
+  far_status st = far_validate(row_begin, row_end, partials, W, residual, residual_out, gamma, T, H,
+                               dtype, eps, weight_bias, FAR_AR_RESIDUAL_RMSNORM_FP8_GROUP, norm_out,
+                               quant_out, nullptr, scale_out);
+  if (st != FAR_OK) return st;
+  if (H % group_size != 0) return FAR_ERR_UNSUPPORTED;
+  if (T > 0) {
+    // scale_out holds T x (H / group_size) floats: it may overlap no other buffer
+    const Range sc = span(scale_out, T * (H / group_size) * 4);
+    const int64_t tb = T * H * 2;
+    for (int r = 0; r < W; ++r)
+      if (overlap(sc, span(partials[r], tb))) return FAR_ERR_INVALID_ARG;
+    const void* bufs16[] = {residual, residual_out, norm_out};
+    for (const void* b : bufs16)
+      if (b != nullptr && overlap(sc, span(b, tb))) return FAR_ERR_INVALID_ARG;
+    if (overlap(sc, span(gamma, H * 2)) || overlap(sc, span(quant_out, T * H)))
+      return FAR_ERR_INVALID_ARG;
+  }
+  if (row_end == row_begin) return FAR_OK;
+
+  far::Params p = make_params(partials, W, residual, residual_out, gamma, H,
+                              FAR_AR_RESIDUAL_RMSNORM_FP8_GROUP, eps, weight_bias, norm_out,
+                              quant_out, nullptr, scale_out);
+  p.wait_limit_ns = ctx->wait_limit_ns;
+  p.stall_segment = ctx->stall_segment;
+  p.group_lanes = group_size / far::kPackElems;
+  p.groups_per_row = static_cast<int>(H / group_size);
+  DeviceGuard guard(ctx->device);
+  if (guard.err != cudaSuccess) return cuda_fail(guard.err, "cudaSetDevice");
+  // a group must sit on consecutive lanes of one warp: not the cluster kernel,
+  // whose per-CTA slices need not start on a group boundary
+  far::Launch whole = plan(ctx, row_end - row_begin, H, dtype, W + (residual != nullptr ? 1 : 0));
+  if (whole.regime == FAR_REGIME_DECODE) {
+    plan_prefill(static_cast<int>(H / far::kPackElems), ctx->prefill_threads, &whole);
+    whole.grid = (row_end - row_begin + whole.rows_per_cta - 1) / whole.rows_per_cta;
+    whole.pdl = ctx->pdl;
+  }
+  const cudaError_t e = launch_rows(p, dtype, whole, row_begin, row_end, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "kernel launch");
+  return FAR_OK;
 }
 
 far_status far_fused(far_ctx* ctx, const void* const* partials, int W, const void* residual,

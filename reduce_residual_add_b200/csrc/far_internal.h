@@ -20,6 +20,7 @@ enum Pattern : int {
   kFp8Static = 1,
   kFp8Token = 2,
   kFp8Tensor = 3,       // public value of dynamic per-tensor FP8
+  kFp8Group = 4,        // per-group FP8: one scale per group of consecutive elements
   kTensorAmax = 16,     // its first pass: rinv of each row + the call's amax
   kTensorQuant = 17     // its second pass: every output, from the stored rinv and amax
 };
@@ -46,8 +47,8 @@ struct Params {
   float* ws_rinv;               // per-tensor FP8: rinv of row t at ws_rinv[t - ws_row0]
   unsigned* ws_amax;            // per-tensor FP8: the call's amax as fp32 bits
   int64_t ws_row0;              // per-tensor FP8: first row of the call
-  int l2_evict_first;           // ring: bulk loads carry an L2 evict-first policy
-  int stream_stores;            // outputs stored with st.global.cs
+  int group_lanes;              // per-group FP8: 16-byte packs per group (power of two <= 32)
+  int groups_per_row;           // per-group FP8: H / group size
   uint64_t wait_limit_ns;       // every bounded wait gives up after this long
   int64_t stall_segment;        // test hook: the ring producer skips this copy (-1: none)
 };

@@ -102,23 +102,6 @@ __device__ __forceinline__ void pack_plus(const uint4& v, float s, float (&out)[
   }
 }
 
-// Output stores: plain, or streaming (st.global.cs: evict-first) when the
-// outputs should not displace other lines from L2.
-__device__ __forceinline__ void store16(void* base, int64_t idx, uint4 v, bool streaming) {
-  uint4* p = static_cast<uint4*>(base) + idx;
-  if (streaming)
-    __stcs(p, v);
-  else
-    *p = v;
-}
-__device__ __forceinline__ void store8(void* base, int64_t idx, uint2 v, bool streaming) {
-  uint2* p = static_cast<uint2*>(base) + idx;
-  if (streaming)
-    __stcs(p, v);
-  else
-    *p = v;
-}
-
 template <class DT>
 __device__ __forceinline__ uint4 pack8(const float (&f)[8]) {
   return make_uint4(DT::pack2(f[0], f[1]), DT::pack2(f[2], f[3]),
@@ -259,21 +242,6 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
       : "memory");
 }
 
-// The same with an L2 cache policy (createpolicy): data read once is marked
-// evict-first so it does not displace lines that are still to be used.
-__device__ __forceinline__ void bulk_load_hint(void* dst, const void* src, uint32_t bytes,
-                                               uint64_t* bar, uint64_t policy) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;"
-      ::"r"(smem_addr(dst)), "l"(src), "r"(bytes), "r"(smem_addr(bar)), "l"(policy)
-      : "memory");
-}
-
-__device__ __forceinline__ uint64_t policy_evict_first() {
-  uint64_t pol;
-  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
-  return pol;
-}
 
 // Programmatic dependent launch (PTX griddepcontrol): wait until the grid
 // this launch depends on has completed and its writes are visible (a no-op
@@ -431,7 +399,7 @@ __device__ __forceinline__ void finish_row(const Params& p, int64_t row, bool ro
   if (p.residual_out != nullptr && !tensor_amax) {
 #pragma unroll
     for (int k = 0; k < VPT; ++k)
-      if (ok[k]) store16(p.residual_out, rbase + j0 + k * jstride, pack8<DT>(y[k]), p.stream_stores);
+      if (ok[k]) static_cast<uint4*>(p.residual_out)[rbase + j0 + k * jstride] = pack8<DT>(y[k]);
   }
 
   // a3: mean of squares; pairwise inside the thread, butterflies above it.
@@ -451,6 +419,7 @@ __device__ __forceinline__ void finish_row(const Params& p, int64_t row, bool ro
 
   const bool fp8_static = p.pattern == kFp8Static;
   const bool fp8_token = p.pattern == kFp8Token;
+  const bool fp8_group = p.pattern == kFp8Group;
   const uint4* gam = gamma_smem != nullptr ? gamma_smem : static_cast<const uint4*>(p.gamma);
 
   // a5b needs max|o| = rinv * max|y * (gamma + wb)| (rinv > 0): its local
@@ -512,8 +481,8 @@ __device__ __forceinline__ void finish_row(const Params& p, int64_t row, bool ro
     pack_plus<DT>(gam[j0 + k * jstride], p.weight_bias, g);
 #pragma unroll
     for (int i = 0; i < 8; ++i) y[k][i] = (y[k][i] * rinv) * g[i];
-    if (p.norm_out != nullptr) store16(p.norm_out, pk, pack8<DT>(y[k]), p.stream_stores);
-    if (fp8_static || fp8_token || tensor_quant) {
+    if (p.norm_out != nullptr) static_cast<uint4*>(p.norm_out)[pk] = pack8<DT>(y[k]);
+    if (fp8_static || fp8_token || tensor_quant) {  // (per-group codes: below)
       uint2 codes = make_uint2(0u, 0u);
       if (scale != 0.f) {  // a per-token row of zeros keeps scale 0 and codes 0
         float q[8];
@@ -526,7 +495,44 @@ __device__ __forceinline__ void finish_row(const Params& p, int64_t row, bool ro
         }
         codes = make_uint2(e4m3x4(q[0], q[1], q[2], q[3]), e4m3x4(q[4], q[5], q[6], q[7]));
       }
-      store8(p.quant_out, pk, codes, p.stream_stores);
+      reinterpret_cast<uint2*>(p.quant_out)[pk] = codes;
+    }
+  }
+
+  // a5d: per-group FP8.  A group is p.group_lanes consecutive packs of the
+  // row, held by as many consecutive lanes of one warp (the pack index is
+  // lane-contiguous and warp-aligned in every kernel that takes this
+  // pattern), so its amax is a shuffle butterfly over those lanes; every
+  // lane takes part before any lane skips its store.
+  if (fp8_group) {
+#pragma unroll
+    for (int k = 0; k < VPT; ++k) {
+      float m = 0.f;
+      if (ok[k]) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) m = fmaxf(m, fabsf(y[k][i]));
+      }
+      m = group_max(m, p.group_lanes);
+      if (!ok[k]) continue;
+      const int jpk = j0 + k * jstride;  // pack index in the row
+      const float sc = __fdiv_rn(m, 448.f);
+      if (row_ok && jpk % p.group_lanes == 0)
+        p.scale_out[row * p.groups_per_row + jpk / p.group_lanes] = sc;
+      uint2 codes = make_uint2(0u, 0u);
+      if (sc != 0.f) {
+        const float inv = __frcp_rn(sc);
+        const bool exact_g = !(inv < 3.0e38f && sc > 1.0e-37f);
+        float q[8];
+        if (exact_g) {
+#pragma unroll
+          for (int i = 0; i < 8; ++i) q[i] = __fdiv_rn(y[k][i], sc);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 8; ++i) q[i] = div_by(y[k][i], sc, inv);
+        }
+        codes = make_uint2(e4m3x4(q[0], q[1], q[2], q[3]), e4m3x4(q[4], q[5], q[6], q[7]));
+      }
+      reinterpret_cast<uint2*>(p.quant_out)[rbase + jpk] = codes;
     }
   }
 }
@@ -683,7 +689,6 @@ far_ring_kernel(const Params p, int nslot, int ncons) {
     // producer warp: one thread issues, the rest of the warp is idle
     if (threadIdx.x == ncons) {
       const int64_t nseg = my_rows * S;
-      const uint64_t policy = policy_evict_first();
       int64_t issued = 0;
       for (int64_t g = 0; g < nseg; ++g) {
         if (*abort_flag) break;
@@ -703,10 +708,7 @@ far_ring_kernel(const Params p, int nslot, int ncons) {
         const void* base = (k < p.W) ? p.partials[k] : p.residual;
         const unsigned char* src = static_cast<const unsigned char*>(base) + row * static_cast<int64_t>(seg_bytes);
         mbar_arrive_expect_tx(&full[slot], seg_bytes);
-        if (p.l2_evict_first)
-          bulk_load_hint(ring + static_cast<size_t>(slot) * seg_bytes, src, seg_bytes, &full[slot], policy);
-        else
-          bulk_load(ring + static_cast<size_t>(slot) * seg_bytes, src, seg_bytes, &full[slot]);
+        bulk_load(ring + static_cast<size_t>(slot) * seg_bytes, src, seg_bytes, &full[slot]);
         issued = g + 1;
       }
       *issued_count = issued;  // read by the drain below

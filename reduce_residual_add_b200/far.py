@@ -35,6 +35,7 @@ FAR_AR_RESIDUAL_RMSNORM = 0
 FAR_AR_RESIDUAL_RMSNORM_FP8_STATIC = 1
 FAR_AR_RESIDUAL_RMSNORM_FP8_TOKEN = 2
 FAR_AR_RESIDUAL_RMSNORM_FP8_TENSOR = 3
+FAR_AR_RESIDUAL_RMSNORM_FP8_GROUP = 4
 
 FAR_REGIME_AUTO = 0
 FAR_REGIME_DECODE = 1
@@ -47,7 +48,7 @@ FAR_FP8_TENSOR_NOALLOC_MAX_ROWS = 65536
 # Every symbol include/far.h declares.
 EXPORTS = ("far_create", "far_destroy", "far_fused", "far_fused_rows",
            "far_fp8_tensor_workspace_bytes", "far_fused_fp8_tensor",
-           "far_fused_fp8_tensor_noalloc", "far_validate",
+           "far_fused_fp8_tensor_noalloc", "far_fused_fp8_group", "far_validate",
            "far_set_regime", "far_describe_launch", "far_check", "far_test_stall",
            "far_status_string",
            "far_last_error", "far_version")
@@ -112,6 +113,9 @@ def lib() -> ctypes.CDLL:
     L.far_fused_fp8_tensor_noalloc.argtypes = [vp, i64, i64, pp, i32, vp, vp, vp, i64, i64, i32,
                                                f32, f32, vp, vp, vp, vp]
     L.far_fused_fp8_tensor_noalloc.restype = i32
+    L.far_fused_fp8_group.argtypes = [vp, i64, i64, pp, i32, vp, vp, vp, i64, i64, i32, f32, f32,
+                                      i32, vp, vp, vp, vp]
+    L.far_fused_fp8_group.restype = i32
     L.far_set_regime.argtypes = [vp, i32, i32]
     L.far_set_regime.restype = i32
     L.far_describe_launch.argtypes = [vp, i64, i64, i32, i32, i32, ctypes.POINTER(far_launch_info)]
@@ -415,3 +419,25 @@ class FarCall:
         st = self._fn(*self._args)
         if st != FAR_OK:
             raise FarError(st, "far_fused_rows")
+
+
+def far_fused_fp8_group(ctx: FarContext, partials: Sequence[torch.Tensor],
+                        residual: Optional[torch.Tensor], gamma: torch.Tensor, eps: float,
+                        weight_bias: float = 0.0, *, group_size: int, quant_out: torch.Tensor,
+                        scale_out: torch.Tensor, residual_out: Optional[torch.Tensor] = None,
+                        norm_out: Optional[torch.Tensor] = None, rows=None, stream=None) -> None:
+    """Per-group FP8: one scale per row and group of ``group_size``
+    consecutive elements, scale_out of T x (H / group_size) floats."""
+    H = gamma.numel()
+    T = partials[0].numel() // H if len(partials) else 0
+    if group_size < 1 or H % group_size:
+        raise ValueError("group_size must divide H")
+    (arr, W, res, rout, gam, T, H, dt, nout, qout, sin, sout) = _args(
+        partials, residual, gamma, residual_out, norm_out, quant_out, None, scale_out,
+        scale_out_elems=T * (H // group_size))
+    b, e = (0, T) if rows is None else (int(rows[0]), int(rows[1]))
+    st = lib().far_fused_fp8_group(ctx.handle, b, e, arr, W, res, rout, gam, T, H, dt, float(eps),
+                                   float(weight_bias), int(group_size), nout, qout, sout,
+                                   _stream(stream))
+    if st != FAR_OK:
+        raise FarError(st, "far_fused_fp8_group")

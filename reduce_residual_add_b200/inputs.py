@@ -32,6 +32,7 @@ PATTERN_AR_RESIDUAL_RMSNORM = 0
 PATTERN_FP8_STATIC = 1
 PATTERN_FP8_TOKEN = 2
 PATTERN_FP8_TENSOR = 3
+PATTERN_FP8_GROUP = 4
 
 _TORCH_DTYPES = {"bf16": torch.bfloat16, "fp16": torch.float16}
 
@@ -59,6 +60,7 @@ class Workload:
     seed: int = 0
     batch_shape: Optional[Tuple[int, ...]] = None   # e.g. (4, 256) for a 3-D view
     has_residual: bool = True
+    group_size: int = 0                               # per-group FP8: elements per group
 
     @property
     def torch_dtype(self) -> torch.dtype:
@@ -92,6 +94,11 @@ WORKLOADS = {
     "c4_prefill_fp8_tensor": Workload(
         "c4_prefill_fp8_tensor", W=4, T=8192, H=8192, residual_sigma=2.0,
         eps=1e-5, pattern=PATTERN_FP8_TENSOR, outlier_frac=0.01, outlier_mult=50.0, seed=3),
+    # the prefill workload with per-group FP8, groups of 128 elements
+    "c4_prefill_fp8_group128": Workload(
+        "c4_prefill_fp8_group128", W=4, T=8192, H=8192, residual_sigma=2.0,
+        eps=1e-5, pattern=PATTERN_FP8_GROUP, outlier_frac=0.01, outlier_mult=50.0, seed=3,
+        group_size=128),
     # W=8, T=4096, H=7168, Gemma-style weight_bias=1.0 with gamma N(0,0.1),
     # dynamic per-token FP8; in bf16 and in fp16
     **{

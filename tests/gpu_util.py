@@ -58,7 +58,7 @@ def to_gpu(inp: dict, device="cuda") -> dict:
 
 def run_gpu(ctx, g: dict, eps: float, wb: float, pattern: int, scale_in=None, rows=None,
             want_norm: bool = True, want_residual_out: bool = True, in_place: bool = False,
-            stream=None, guard: int = 0) -> dict:
+            stream=None, guard: int = 0, group: int = 0) -> dict:
     """One call of the CUDA path; returns numpy arrays of the outputs (full T).
 
     ``guard`` > 0 surrounds every output with that many canary bytes (0xA5)
@@ -88,9 +88,14 @@ def run_gpu(ctx, g: dict, eps: float, wb: float, pattern: int, scale_in=None, ro
         rout = alloc(T * H, dt).view(T, H)
     nout = alloc(T * H, dt).view(T, H) if want_norm else None
     qout = alloc(T * H, torch.uint8).view(T, H) if pattern != 0 else None
-    sout = alloc(T if pattern == 2 else 1, torch.float32) if pattern in (2, 3) else None
+    sout = (alloc({2: T, 3: 1, 4: T * (H // group if group else 1)}[pattern], torch.float32)
+            if pattern in (2, 3, 4) else None)
     sin = torch.tensor([scale_in], dtype=torch.float32, device=dev) if pattern == 1 else None
-    if pattern == 3:
+    if pattern == 4:
+        far.far_fused_fp8_group(ctx, ps, res, g["gamma"], eps, wb, group_size=group, quant_out=qout,
+                                scale_out=sout, residual_out=rout, norm_out=nout, rows=rows,
+                                stream=stream)
+    elif pattern == 3:
         nrows = T if rows is None else rows[1] - rows[0]
         ws = torch.empty(far.far_fp8_tensor_workspace_bytes(nrows), dtype=torch.uint8, device=dev)
         assert ws.data_ptr() % 256 == 0
@@ -119,11 +124,13 @@ def run_gpu(ctx, g: dict, eps: float, wb: float, pattern: int, scale_in=None, ro
     out["norm_out"] = None if nout is None else as_u16(nout.cpu())
     out["quant_out"] = None if qout is None else qout.cpu().numpy()
     out["scale_out"] = None if sout is None else sout.cpu().numpy()
+    if pattern == 4:
+        out["scale_out"] = out["scale_out"].reshape(T, H // group)
     return out
 
 
 def run_oracle(inp: dict, dtype: str, eps, wb, pattern, scale_in=None, rows=None, want_norm=True,
-               want_residual_out=True, row_list=None) -> dict:
+               want_residual_out=True, row_list=None, group=0) -> dict:
     ps = [as_u16(p) for p in inp["partials"]]
     res = None if inp["residual"] is None else as_u16(inp["residual"])
     gam = as_u16(inp["gamma"])
@@ -131,12 +138,12 @@ def run_oracle(inp: dict, dtype: str, eps, wb, pattern, scale_in=None, rows=None
         raise ValueError("the per-tensor scale needs every row of the call")
     if row_list is None:
         return oracle.fused(ps, res, gam, dtype, eps, wb, pattern, scale_in=scale_in, rows=rows,
-                            want_norm=want_norm, want_residual_out=want_residual_out)
+                            want_norm=want_norm, want_residual_out=want_residual_out, group=group)
     out = None
     for t in row_list:
         out = oracle.fused(ps, res, gam, dtype, eps, wb, pattern, scale_in=scale_in,
                            rows=(int(t), int(t) + 1), want_norm=want_norm,
-                           want_residual_out=want_residual_out, out=out)
+                           want_residual_out=want_residual_out, out=out, group=group)
     return out
 
 

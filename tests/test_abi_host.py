@@ -53,6 +53,7 @@ def test_header_constants_match_binding_and_oracle():
               "FAR_ERR_CUDA", "FAR_ERR_TIMEOUT", "FAR_ERR_INTERNAL", "FAR_BF16", "FAR_FP16",
               "FAR_AR_RESIDUAL_RMSNORM", "FAR_AR_RESIDUAL_RMSNORM_FP8_STATIC",
               "FAR_AR_RESIDUAL_RMSNORM_FP8_TOKEN", "FAR_AR_RESIDUAL_RMSNORM_FP8_TENSOR",
+              "FAR_AR_RESIDUAL_RMSNORM_FP8_GROUP",
               "FAR_REGIME_AUTO", "FAR_REGIME_DECODE",
               "FAR_REGIME_PREFILL"):
         assert getattr(far, n) == _enum(n), n
@@ -62,9 +63,11 @@ def test_header_constants_match_binding_and_oracle():
             == far.FAR_FP8_TENSOR_NOALLOC_MAX_ROWS)
     # the oracle keeps its own copies of the numbering
     assert (oracle.BF16, oracle.FP16) == (far.FAR_BF16, far.FAR_FP16)
-    assert (oracle.AR_RESIDUAL_RMSNORM, oracle.FP8_STATIC, oracle.FP8_TOKEN, oracle.FP8_TENSOR) == (
+    assert (oracle.AR_RESIDUAL_RMSNORM, oracle.FP8_STATIC, oracle.FP8_TOKEN, oracle.FP8_TENSOR,
+            oracle.FP8_GROUP) == (
         far.FAR_AR_RESIDUAL_RMSNORM, far.FAR_AR_RESIDUAL_RMSNORM_FP8_STATIC,
-        far.FAR_AR_RESIDUAL_RMSNORM_FP8_TOKEN, far.FAR_AR_RESIDUAL_RMSNORM_FP8_TENSOR)
+        far.FAR_AR_RESIDUAL_RMSNORM_FP8_TOKEN, far.FAR_AR_RESIDUAL_RMSNORM_FP8_TENSOR,
+        far.FAR_AR_RESIDUAL_RMSNORM_FP8_GROUP)
     assert far.far_version() == int(re.search(r"#define FAR_VERSION (\d+)", HEADER).group(1))
 
 
@@ -108,7 +111,7 @@ def v(**over):
 
 def test_validate_accepts_good_arguments():
     assert v() == far.FAR_OK
-    for p in (0, 1, 2, 3):
+    for p in (0, 1, 2, 3, 4):
         assert v(pattern=p) == far.FAR_OK
     assert v(residual_out=0) == far.FAR_OK                      # in place
     assert v(residual_out=good()["residual"]) == far.FAR_OK     # explicitly in place
@@ -139,7 +142,9 @@ def test_validate_accepts_good_arguments():
     (dict(H=12), far.FAR_ERR_UNSUPPORTED),
     (dict(H=16392), far.FAR_ERR_UNSUPPORTED),
     (dict(dtype=2), far.FAR_ERR_INVALID_ARG),
-    (dict(pattern=4), far.FAR_ERR_INVALID_ARG),
+    (dict(pattern=5), far.FAR_ERR_INVALID_ARG),
+    (dict(pattern=4, quant_out=0), far.FAR_ERR_INVALID_ARG),
+    (dict(pattern=4, scale_out=0), far.FAR_ERR_INVALID_ARG),
     (dict(pattern=3, quant_out=0), far.FAR_ERR_INVALID_ARG),
     (dict(pattern=3, scale_out=0), far.FAR_ERR_INVALID_ARG),
     (dict(row_begin=-1), far.FAR_ERR_INVALID_ARG),

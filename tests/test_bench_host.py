@@ -18,6 +18,8 @@ def test_algorithmic_bytes_of_the_workloads():
     assert bench.algorithmic_bytes(c5, c5.T, True) == 675_313_664
     c4t = WORKLOADS["c4_prefill_fp8_tensor"]
     assert bench.algorithmic_bytes(c4t, c4t.T, False) == 872_431_616 + 4
+    c4g = WORKLOADS["c4_prefill_fp8_group128"]
+    assert bench.algorithmic_bytes(c4g, c4g.T, False) == 872_431_616 + 4 * 8192 * 64
     c3 = WORKLOADS["c3_3d"]
     assert bench.algorithmic_bytes(c3, c3.T, True) == 20_975_616
     c1 = WORKLOADS["c1_small"]

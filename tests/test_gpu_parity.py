@@ -583,3 +583,62 @@ def test_format_edges_overflow_and_subnormals(kctx, kern):
         compare(got, ref, dt)
         exp = (got["norm_out"].astype(np.int64) >> (7 if dt == "bf16" else 10)) & (0xFF if dt == "bf16" else 0x1F)
         assert np.mean(exp == 0) > 0.5                               # mostly subnormal, kept
+
+
+
+# ---------------------------------------------------------------------------
+# per-group FP8
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("kern", ["ring", "direct", "auto"])
+@pytest.mark.parametrize("case", [
+    (2, 8, 64, 8, "bf16"),          # one pack per group; rows inside a warp
+    (2, 8, 64, 64, "fp16"),         # one group per row
+    (3, 40, 256, 16, "bf16"),
+    (4, 300, 8192, 128, "bf16"),
+    (8, 150, 7168, 128, "fp16"),
+    (2, 30, 16384, 256, "bf16"),
+    (5, 70, 1000, 8, "bf16"),       # ragged H: 125 packs
+    (8, 4, 4096, 32, "bf16"),       # decode-sized
+], ids=lambda c: "W%d_T%d_H%d_G%d_%s" % c)
+def test_per_group_fp8(kctx, ctx, case, kern):
+    W, T, H, G, dt = case
+    c = ctx if kern == "auto" else kctx[kern]
+    inp = random_inputs(W, T, H, dtype=dt, seed=700 + W + T + H + G)
+    got = run_gpu(c, to_gpu(inp), 1e-6, 0.0, 4, group=G, guard=512)
+    ref = run_oracle(inp, dt, 1e-6, 0.0, 4, group=G)
+    log("group %s %s" % (kern, case), compare(got, ref, dt))
+
+
+def test_per_group_full_size_sampled(ctx):
+    wl = WORKLOADS["c4_prefill_fp8_static"]
+    inp = make_inputs(wl)
+    got = run_gpu(ctx, to_gpu(inp), wl.eps, 0.0, 4, group=128)
+    rows = _sample_rows(wl.T, inp["outlier_rows"].tolist(), 120, 5)
+    ref = run_oracle(inp, "bf16", wl.eps, 0.0, 4, row_list=rows, group=128)
+    log("group c4 full", compare(got, ref, "bf16", rows=rows))
+    q = (got["quant_out"] & 0x7F).reshape(wl.T, wl.H // 128, 128)
+    assert np.all(np.any(q == 0x7E, axis=2))
+
+
+def test_per_group_errors(ctx):
+    inp = random_inputs(2, 4, 2048, seed=78)
+    g = to_gpu(inp)
+    q = torch.empty(4, 2048, dtype=torch.uint8, device="cuda")
+    for G in (24, 512, 4):
+        sc = torch.empty(4 * 2048 // 4, dtype=torch.float32, device="cuda")
+        with pytest.raises(far.FarError) as e:
+            lib = far.lib()
+            import ctypes
+            arr = (ctypes.c_void_p * 2)(*[p.data_ptr() for p in g["partials"]])
+            st = lib.far_fused_fp8_group(ctx.handle, 0, 4, arr, 2, ctypes.c_void_p(g["residual"].data_ptr()),
+                                         None, ctypes.c_void_p(g["gamma"].data_ptr()), 4, 2048, 0, 1e-6,
+                                         0.0, G, None, ctypes.c_void_p(q.data_ptr()),
+                                         ctypes.c_void_p(sc.data_ptr()), None)
+            if st != far.FAR_OK:
+                raise far.FarError(st)
+        assert e.value.status == far.FAR_ERR_UNSUPPORTED
+    with pytest.raises(far.FarError) as e:
+        far.far_fused(ctx, g["partials"], g["residual"], g["gamma"], 1e-6, 0.0, 4, quant_out=q,
+                      scale_out=torch.empty(4, dtype=torch.float32, device="cuda"))
+    assert e.value.status == far.FAR_ERR_INVALID_ARG
