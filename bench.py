@@ -375,6 +375,26 @@ def profiled_traffic(workload: str):
         return None
 
 
+PATTERN_NAMES = {0: "ar_residual_rmsnorm", 1: "fp8_static", 2: "fp8_per_token",
+                 3: "fp8_per_tensor", 4: "fp8_per_group"}
+
+
+def workload_config(wl: Workload, bytes_per_step: int, with_norm: bool, launch: dict,
+                    world: int) -> dict:
+    """The bench line's `config` object for one workload."""
+    cfg = {"workload": wl.name, "W": wl.W, "T": wl.T, "H": wl.H, "dtype": wl.dtype,
+           "arithmetic": "fp32 accumulation; bf16/fp16 in and out; e4m3 codes",
+           "pattern": PATTERN_NAMES[wl.pattern], "norm_out": with_norm, "eps": wl.eps,
+           "weight_bias": wl.weight_bias, "static_scale": wl.static_scale,
+           "bytes_per_step": bytes_per_step, "rows_per_rank": wl.T,
+           "l2": "inputs larger than L2 (%d MiB read per step vs 126 MB L2); no flush"
+                 % ((wl.W + 1) * wl.T * wl.H * 2 // 2 ** 20),
+           "launch": launch, "parallelism": "rows sharded across %d rank(s), no collective" % world}
+    if wl.pattern == 4:
+        cfg["group_size"] = wl.group_size
+    return cfg
+
+
 def run_far(args, world, rank, local):
     from reduce_residual_add_b200 import build as fbuild
     from reduce_residual_add_b200 import far
@@ -415,15 +435,7 @@ def run_far(args, world, rank, local):
         "ms_per_step": round(total_max / args.steps * 1e3, 5),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
         "data": "synthetic",
-        "config": {"workload": wl.name, "W": wl.W, "T": wl.T, "H": wl.H, "dtype": wl.dtype,
-                   "arithmetic": "fp32 accumulation; bf16/fp16 in and out; e4m3 codes",
-                   "pattern": ["ar_residual_rmsnorm", "fp8_static", "fp8_per_token"][wl.pattern],
-                   "norm_out": case.nout is not None, "eps": wl.eps,
-                   "weight_bias": wl.weight_bias, "static_scale": wl.static_scale,
-                   "bytes_per_step": case.bytes, "rows_per_rank": wl.T,
-                   "l2": "inputs larger than L2 (%d MiB read per step vs 126 MB L2); no flush"
-                         % ((wl.W + 1) * wl.T * wl.H * 2 // 2 ** 20),
-                   "launch": launch, "parallelism": "rows sharded across %d rank(s), no collective" % world},
+        "config": workload_config(wl, case.bytes, case.nout is not None, launch, world),
         "tokens_per_s": round(rows_all / total_max, 1),
         "pct_of_peak": round(100 * value / world / peak, 2),
         "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak,

@@ -386,7 +386,9 @@ struct RingRed {
 // This thread owns packs j = j0 + k*jstride (k < VPT) where ok[k].
 // ---------------------------------------------------------------------------
 
-template <class DT, int VPT, class Red>
+// GROUP: this instantiation serves only the per-group pattern (kept apart
+// so that the other patterns' code carries none of its registers).
+template <class DT, int VPT, bool GROUP, class Red>
 __device__ __forceinline__ void finish_row(const Params& p, int64_t row, bool row_ok, int j0,
                                            int jstride, const bool (&ok)[VPT],
                                            float (&y)[VPT][8], const Red& red,
@@ -419,7 +421,7 @@ __device__ __forceinline__ void finish_row(const Params& p, int64_t row, bool ro
 
   const bool fp8_static = p.pattern == kFp8Static;
   const bool fp8_token = p.pattern == kFp8Token;
-  const bool fp8_group = p.pattern == kFp8Group;
+  constexpr bool fp8_group = GROUP;
   const uint4* gam = gamma_smem != nullptr ? gamma_smem : static_cast<const uint4*>(p.gamma);
 
   // a5b needs max|o| = rinv * max|y * (gamma + wb)| (rinv > 0): its local
@@ -504,7 +506,7 @@ __device__ __forceinline__ void finish_row(const Params& p, int64_t row, bool ro
   // lane-contiguous and warp-aligned in every kernel that takes this
   // pattern), so its amax is a shuffle butterfly over those lanes; every
   // lane takes part before any lane skips its store.
-  if (fp8_group) {
+  if constexpr (fp8_group) {
 #pragma unroll
     for (int k = 0; k < VPT; ++k) {
       float m = 0.f;
@@ -542,7 +544,7 @@ __device__ __forceinline__ void finish_row(const Params& p, int64_t row, bool ro
 // packs j = j0 + k*jstride, k < VPT, j < jend
 // ---------------------------------------------------------------------------
 
-template <class DT, int VPT, class Red>
+template <class DT, int VPT, bool GROUP, class Red>
 __device__ __forceinline__ void fused_row(const Params& p, int64_t row, bool row_ok,
                                           int j0, int jstride, int jend, const Red& red) {
   const int64_t rbase = row * static_cast<int64_t>(p.packs);  // first pack of the row
@@ -585,7 +587,7 @@ __device__ __forceinline__ void fused_row(const Params& p, int64_t row, bool row
 #pragma unroll
     for (int k = 0; k < VPT; ++k) add_pack<DT>(v[k], y[k]);
   }
-  finish_row<DT, VPT>(p, row, row_ok, j0, jstride, ok, y, red);
+  finish_row<DT, VPT, GROUP>(p, row, row_ok, j0, jstride, ok, y, red);
 }
 
 // ---------------------------------------------------------------------------
@@ -594,7 +596,7 @@ __device__ __forceinline__ void fused_row(const Params& p, int64_t row, bool row
 
 // Prefill: blockDim = (tpr, rows_per_cta).  SUB: a row lives inside one warp
 // (tpr <= 32, power of two); otherwise one row per CTA.
-template <class DT, int VPT, bool SUB>
+template <class DT, int VPT, bool SUB, bool GROUP>
 __global__ void __launch_bounds__(kMaxThreads, (VPT >= 8 ? 1 : 2))
 far_prefill_kernel(const Params p) {
   pdl_enter();
@@ -602,11 +604,11 @@ far_prefill_kernel(const Params p) {
   const bool row_ok = row < p.row_end;
   if constexpr (SUB) {
     const SubwarpRed red{static_cast<int>(blockDim.x)};
-    fused_row<DT, VPT>(p, row, row_ok, threadIdx.x, blockDim.x, p.packs, red);
+    fused_row<DT, VPT, GROUP>(p, row, row_ok, threadIdx.x, blockDim.x, p.packs, red);
   } else {
     __shared__ float s_sum[32], s_max[32];
     const BlockRed red{s_sum, s_max};
-    fused_row<DT, VPT>(p, row, row_ok, threadIdx.x, blockDim.x, p.packs, red);
+    fused_row<DT, VPT, GROUP>(p, row, row_ok, threadIdx.x, blockDim.x, p.packs, red);
   }
 }
 
@@ -632,8 +634,8 @@ far_decode_kernel(const Params p) {
   const int jbeg = rank * chunk;
   const int jend = min(p.packs, jbeg + chunk);
   const ClusterRed red{BlockRed{s_sum, s_max}, s_in, &s_bar, ncta, rank, p.wait_limit_ns};
-  fused_row<DT, VPT>(p, row, row < p.row_end, jbeg + static_cast<int>(threadIdx.x),
-                     blockDim.x, jend, red);
+  fused_row<DT, VPT, false>(p, row, row < p.row_end, jbeg + static_cast<int>(threadIdx.x),
+                            blockDim.x, jend, red);
 }
 
 // Prefill through the TMA engine: a persistent CTA per SM (or two) walks
@@ -652,7 +654,7 @@ far_decode_kernel(const Params p) {
 // the producer stops, and thread 0 waits (bounded) for the copies already
 // issued before the CTA exits.
 // MINB: CTAs per SM the register budget is sized for (2 or 3; 1 at VPT 8).
-template <class DT, int VPT, int MINB>
+template <class DT, int VPT, int MINB, bool GROUP>
 __global__ void __launch_bounds__(kRingMaxConsumers + 32, MINB)
 far_ring_kernel(const Params p, int nslot, int ncons) {
   pdl_enter();
@@ -746,7 +748,7 @@ far_ring_kernel(const Params p, int nslot, int ncons) {
       __syncwarp();
       if ((threadIdx.x & 31) == 0) mbar_arrive(&empty[slot]);
     }
-    finish_row<DT, VPT>(p, row, true, j0, ncons, ok, y, (i & 1) ? red1 : red0, gamma_s);
+    finish_row<DT, VPT, GROUP>(p, row, true, j0, ncons, ok, y, (i & 1) ? red1 : red0, gamma_s);
   }
 
   // Only after an abort can copies still be in flight: thread 0 waits for
@@ -786,7 +788,7 @@ struct Attrs {
   }
 };
 
-template <class DT, int VPT, bool SUB>
+template <class DT, int VPT, bool SUB, bool GROUP>
 cudaError_t launch_prefill_t(const Params& p, const Launch& l, cudaStream_t s) {
   Attrs at(l, 0);
   cudaLaunchConfig_t cfg = {};
@@ -796,7 +798,7 @@ cudaError_t launch_prefill_t(const Params& p, const Launch& l, cudaStream_t s) {
   cfg.stream = s;
   cfg.attrs = at.a;
   cfg.numAttrs = at.n;
-  return cudaLaunchKernelEx(&cfg, far_prefill_kernel<DT, VPT, SUB>, p);
+  return cudaLaunchKernelEx(&cfg, far_prefill_kernel<DT, VPT, SUB, GROUP>, p);
 }
 
 template <class DT, int VPT>
@@ -812,7 +814,7 @@ cudaError_t launch_decode_t(const Params& p, const Launch& l, cudaStream_t s) {
   return cudaLaunchKernelEx(&cfg, far_decode_kernel<DT, VPT>, p);
 }
 
-template <class DT, int VPT, int MINB>
+template <class DT, int VPT, int MINB, bool GROUP>
 cudaError_t launch_ring_t(const Params& p, const Launch& l, cudaStream_t s) {
   Attrs at(l, 0);
   cudaLaunchConfig_t cfg = {};
@@ -822,31 +824,41 @@ cudaError_t launch_ring_t(const Params& p, const Launch& l, cudaStream_t s) {
   cfg.stream = s;
   cfg.attrs = at.a;
   cfg.numAttrs = at.n;
-  return cudaLaunchKernelEx(&cfg, far_ring_kernel<DT, VPT, MINB>, p, l.nslot, l.tpr);
+  return cudaLaunchKernelEx(&cfg, far_ring_kernel<DT, VPT, MINB, GROUP>, p, l.nslot, l.tpr);
+}
+
+template <class DT, bool GROUP>
+cudaError_t launch_ring_g(const Params& p, const Launch& l, cudaStream_t s) {
+  const bool three = l.ring_minb >= 3;
+  switch (l.vpt) {
+    case 1: return three ? launch_ring_t<DT, 1, 3, GROUP>(p, l, s) : launch_ring_t<DT, 1, 2, GROUP>(p, l, s);
+    case 2: return three ? launch_ring_t<DT, 2, 3, GROUP>(p, l, s) : launch_ring_t<DT, 2, 2, GROUP>(p, l, s);
+    case 4: return three ? launch_ring_t<DT, 4, 3, GROUP>(p, l, s) : launch_ring_t<DT, 4, 2, GROUP>(p, l, s);
+    case 8: return launch_ring_t<DT, 8, 1, GROUP>(p, l, s);
+    default: return cudaErrorInvalidConfiguration;
+  }
 }
 
 template <class DT>
 cudaError_t launch_ring_dt(const Params& p, const Launch& l, cudaStream_t s) {
-  const bool three = l.ring_minb >= 3;
+  return p.pattern == kFp8Group ? launch_ring_g<DT, true>(p, l, s) : launch_ring_g<DT, false>(p, l, s);
+}
+
+template <class DT, bool GROUP>
+cudaError_t launch_prefill_g(const Params& p, const Launch& l, cudaStream_t s) {
+  if (l.tpr <= 32 && l.rows_per_cta > 1) return launch_prefill_t<DT, 1, true, GROUP>(p, l, s);
   switch (l.vpt) {
-    case 1: return three ? launch_ring_t<DT, 1, 3>(p, l, s) : launch_ring_t<DT, 1, 2>(p, l, s);
-    case 2: return three ? launch_ring_t<DT, 2, 3>(p, l, s) : launch_ring_t<DT, 2, 2>(p, l, s);
-    case 4: return three ? launch_ring_t<DT, 4, 3>(p, l, s) : launch_ring_t<DT, 4, 2>(p, l, s);
-    case 8: return launch_ring_t<DT, 8, 1>(p, l, s);
+    case 1: return launch_prefill_t<DT, 1, false, GROUP>(p, l, s);
+    case 2: return launch_prefill_t<DT, 2, false, GROUP>(p, l, s);
+    case 4: return launch_prefill_t<DT, 4, false, GROUP>(p, l, s);
+    case 8: return launch_prefill_t<DT, 8, false, GROUP>(p, l, s);
     default: return cudaErrorInvalidConfiguration;
   }
 }
 
 template <class DT>
 cudaError_t launch_prefill_dt(const Params& p, const Launch& l, cudaStream_t s) {
-  if (l.tpr <= 32 && l.rows_per_cta > 1) return launch_prefill_t<DT, 1, true>(p, l, s);
-  switch (l.vpt) {
-    case 1: return launch_prefill_t<DT, 1, false>(p, l, s);
-    case 2: return launch_prefill_t<DT, 2, false>(p, l, s);
-    case 4: return launch_prefill_t<DT, 4, false>(p, l, s);
-    case 8: return launch_prefill_t<DT, 8, false>(p, l, s);
-    default: return cudaErrorInvalidConfiguration;
-  }
+  return p.pattern == kFp8Group ? launch_prefill_g<DT, true>(p, l, s) : launch_prefill_g<DT, false>(p, l, s);
 }
 
 template <class DT>
@@ -867,13 +879,20 @@ cudaError_t allow_large_smem() {
     if (e == cudaSuccess)
       e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kRingSmemMax);
   };
-  set(far_ring_kernel<DT, 1, 2>);
-  set(far_ring_kernel<DT, 2, 2>);
-  set(far_ring_kernel<DT, 4, 2>);
-  set(far_ring_kernel<DT, 1, 3>);
-  set(far_ring_kernel<DT, 2, 3>);
-  set(far_ring_kernel<DT, 4, 3>);
-  set(far_ring_kernel<DT, 8, 1>);
+  set(far_ring_kernel<DT, 1, 2, false>);
+  set(far_ring_kernel<DT, 2, 2, false>);
+  set(far_ring_kernel<DT, 4, 2, false>);
+  set(far_ring_kernel<DT, 1, 3, false>);
+  set(far_ring_kernel<DT, 2, 3, false>);
+  set(far_ring_kernel<DT, 4, 3, false>);
+  set(far_ring_kernel<DT, 8, 1, false>);
+  set(far_ring_kernel<DT, 1, 2, true>);
+  set(far_ring_kernel<DT, 2, 2, true>);
+  set(far_ring_kernel<DT, 4, 2, true>);
+  set(far_ring_kernel<DT, 1, 3, true>);
+  set(far_ring_kernel<DT, 2, 3, true>);
+  set(far_ring_kernel<DT, 4, 3, true>);
+  set(far_ring_kernel<DT, 8, 1, true>);
   return e;
 }
 
@@ -910,9 +929,10 @@ int ring_header_bytes(int nslot) { return ring_offset(nslot); }
 namespace {
 template <class DT, int VPT, int MINB>
 int occ_of(int threads, int smem) {
+  // the per-group instantiation is sized the same way; the plain one decides
   int n = 0;
   const cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(
-      &n, far_ring_kernel<DT, VPT, MINB>, threads, smem);
+      &n, far_ring_kernel<DT, VPT, MINB, false>, threads, smem);
   return e == cudaSuccess ? n : 0;
 }
 

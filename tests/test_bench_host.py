@@ -52,3 +52,10 @@ def test_peak_and_traffic_lookup():
             assert t is None
     else:
         assert t is None
+
+
+def test_workload_config_for_every_workload():
+    for name, wl in WORKLOADS.items():
+        cfg = bench.workload_config(wl, bench.algorithmic_bytes(wl, wl.T, False), False, {}, 1)
+        assert cfg["workload"] == name and cfg["pattern"] in bench.PATTERN_NAMES.values()
+        json.dumps(cfg)
