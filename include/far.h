@@ -111,7 +111,9 @@ typedef enum {
  * per ring CTA, at most 256 (default 256), FAR_RING_SLOTS: row-segment slots
  * per ring CTA (2..32; default: about 72 KiB of segments, as many as fit),
  * FAR_PDL=1|0: launch with programmatic dependent launch, default 1,
- * FAR_RING_MIN_ROWS: fewest rows for the ring kernel, default by rule). */
+ * FAR_RING_MIN_ROWS: fewest rows for the ring kernel, default by rule,
+ * FAR_TENSOR_REVERSE=1|0: the second pass of per-tensor FP8 takes the rows
+ * from the last one down, default 1). */
 /*
  * Programmatic dependent launch: every kernel of this library first waits
  * (griddepcontrol.wait) until the grid it depends on has completed, then

@@ -27,6 +27,7 @@ struct far_ctx {
   int ring_ctas_per_sm; // persistent ring CTAs per SM wanted (1..4; 0 = by rule)
   int ring_threads;     // target consumer threads of a ring CTA
   int ring_slots_max;   // at most this many ring slots
+  int tensor_reverse;   // per-tensor FP8: second pass from the last row down
   int pdl;              // programmatic dependent launch on every call
   int ring_min_rows;    // fewer rows than this take the direct kernel
   uint64_t wait_limit_ns;  // bounded waits in the kernels give up after this
@@ -128,15 +129,15 @@ void plan_decode(int packs, int cluster_pref, far::Launch* l) {
 // configuration cannot be resident.
 bool plan_ring(const far_ctx* ctx, int packs, int64_t rows, int dtype, int segs, far::Launch* l) {
   if (packs <= 32) return false;
-  int vpt = 1;
-  while (vpt < 8 && (packs + vpt - 1) / vpt > ctx->ring_threads) vpt *= 2;
-  const int tpr = (((packs + vpt - 1) / vpt) + 31) / 32 * 32;
-  if (tpr > far::kRingMaxConsumers) return false;
   const int seg = packs * 16;
   // CTAs per SM: measured on B200, 3 (registers capped at 72) when a row has
   // few segments (W=4 + residual: 95.5 % vs 93.3 % with 2), 2 (86 registers)
   // when it has many (W=8 + residual: 89.1 % vs 87.9 % with 3)
   const int n_req = ctx->ring_ctas_per_sm > 0 ? ctx->ring_ctas_per_sm : (segs <= 6 ? 3 : 2);
+  int vpt = 1;
+  while (vpt < 8 && (packs + vpt - 1) / vpt > ctx->ring_threads) vpt *= 2;
+  const int tpr = (((packs + vpt - 1) / vpt) + 31) / 32 * 32;
+  if (tpr > far::kRingMaxConsumers) return false;
   int per_cta = 228 * 1024 / n_req - 1024;
   if (per_cta > far::kRingSmemMax) per_cta = far::kRingSmemMax;
   // header, gamma (one segment's worth of bytes), slots: about 72 KiB of
@@ -272,6 +273,7 @@ far_status far_create(far_ctx** ctx, int device) {
   if (c.ring_ctas_per_sm > 4) c.ring_ctas_per_sm = 4;
   c.ring_threads = env_int("FAR_RING_THREADS", 256);  // at most kRingMaxConsumers
   c.ring_slots_max = env_int("FAR_RING_SLOTS", 0);  // 0: by the 72 KiB rule
+  c.tensor_reverse = env_int("FAR_TENSOR_REVERSE", 1) != 0;
   if (c.ring_slots_max < 0) c.ring_slots_max = 0;
   if (c.ring_slots_max > 32) c.ring_slots_max = 32;
   if (c.ring_threads < 32) c.ring_threads = 32;
@@ -539,7 +541,10 @@ far_status far_fused_fp8_tensor_launch(far_ctx* ctx, int64_t row_begin, int64_t 
   p.pattern = far::kTensorAmax;
   e = launch_rows(p, dtype, first, row_begin, row_end, s);
   if (e != cudaSuccess) return cuda_fail(e, "kernel launch (per-tensor pass 1)");
+  // the second pass takes the rows last row first: the rows the first pass
+  // read last are still in L2 when it starts
   p.pattern = far::kTensorQuant;
+  p.reverse = ctx->tensor_reverse;
   e = launch_rows(p, dtype, whole, row_begin, row_end, s);
   if (e != cudaSuccess) return cuda_fail(e, "kernel launch (per-tensor pass 2)");
   return FAR_OK;

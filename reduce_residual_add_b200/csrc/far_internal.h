@@ -51,6 +51,7 @@ struct Params {
   int groups_per_row;           // per-group FP8: H / group size
   uint64_t wait_limit_ns;       // every bounded wait gives up after this long
   int64_t stall_segment;        // test hook: the ring producer skips this copy (-1: none)
+  int reverse;                  // take the rows from row_end - 1 down to row_begin
 };
 
 // Geometry of one launch, chosen on the host.

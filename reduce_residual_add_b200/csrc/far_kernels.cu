@@ -48,6 +48,12 @@ __host__ __device__ constexpr int ring_offset(int nslot) {
   return (16 * nslot + static_cast<int>(sizeof(RingHeader)) + 127) / 128 * 128;
 }
 
+// Row number k (0 <= k < row_end - row_begin) of a call, counted from
+// row_begin up, or with p.reverse from row_end - 1 down.
+__device__ __forceinline__ int64_t call_row(const Params& p, int64_t k) {
+  return p.reverse ? p.row_end - 1 - k : p.row_begin + k;
+}
+
 // ---------------------------------------------------------------------------
 // 16-byte packs of eight 2-byte elements
 // ---------------------------------------------------------------------------
@@ -444,7 +450,8 @@ __device__ __forceinline__ void finish_row(const Params& p, int64_t row, bool ro
   } else if (!tensor_quant) {
     ss = red.sum(sq[0]);
   }
-  const float rinv = tensor_quant ? p.ws_rinv[row - p.ws_row0]
+  // (a row past the end of the call, in a CTA of several rows, reads nothing)
+  const float rinv = tensor_quant ? (row_ok ? p.ws_rinv[row - p.ws_row0] : 0.f)
                                   : __frsqrt_rn(__fdiv_rn(ss, static_cast<float>(p.H)) + p.eps);
 
   if (tensor_amax) {
@@ -518,8 +525,9 @@ __device__ __forceinline__ void finish_row(const Params& p, int64_t row, bool ro
       if (!ok[k]) continue;
       const int jpk = j0 + k * jstride;  // pack index in the row
       const float sc = __fdiv_rn(m, 448.f);
-      if (row_ok && jpk % p.group_lanes == 0)
-        p.scale_out[row * p.groups_per_row + jpk / p.group_lanes] = sc;
+      // group_lanes is a power of two: its group is jpk >> log2(group_lanes)
+      if (row_ok && (jpk & (p.group_lanes - 1)) == 0)
+        p.scale_out[row * p.groups_per_row + (jpk >> (__ffs(p.group_lanes) - 1))] = sc;
       uint2 codes = make_uint2(0u, 0u);
       if (sc != 0.f) {
         const float inv = __frcp_rn(sc);
@@ -600,8 +608,9 @@ template <class DT, int VPT, bool SUB, bool GROUP>
 __global__ void __launch_bounds__(kMaxThreads, (VPT >= 8 ? 1 : 2))
 far_prefill_kernel(const Params p) {
   pdl_enter();
-  const int64_t row = p.row_begin + static_cast<int64_t>(blockIdx.x) * blockDim.y + threadIdx.y;
-  const bool row_ok = row < p.row_end;
+  const int64_t k = static_cast<int64_t>(blockIdx.x) * blockDim.y + threadIdx.y;
+  const bool row_ok = k < p.row_end - p.row_begin;
+  const int64_t row = call_row(p, k);
   if constexpr (SUB) {
     const SubwarpRed red{static_cast<int>(blockDim.x)};
     fused_row<DT, VPT, GROUP>(p, row, row_ok, threadIdx.x, blockDim.x, p.packs, red);
@@ -629,13 +638,14 @@ far_decode_kernel(const Params p) {
   }
   __syncthreads();
   asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
-  const int64_t row = p.row_begin + blockIdx.y;
+  const int64_t row = call_row(p, blockIdx.y);
   const int chunk = (p.packs + ncta - 1) / ncta;
   const int jbeg = rank * chunk;
   const int jend = min(p.packs, jbeg + chunk);
   const ClusterRed red{BlockRed{s_sum, s_max}, s_in, &s_bar, ncta, rank, p.wait_limit_ns};
-  fused_row<DT, VPT, false>(p, row, row < p.row_end, jbeg + static_cast<int>(threadIdx.x),
-                            blockDim.x, jend, red);
+  const bool row_ok = blockIdx.y < p.row_end - p.row_begin;
+  fused_row<DT, VPT, false>(p, row, row_ok, jbeg + static_cast<int>(threadIdx.x), blockDim.x, jend,
+                            red);
 }
 
 // Prefill through the TMA engine: a persistent CTA per SM (or two) walks
@@ -692,26 +702,34 @@ far_ring_kernel(const Params p, int nslot, int ncons) {
     if (threadIdx.x == ncons) {
       const int64_t nseg = my_rows * S;
       int64_t issued = 0;
+      // segment g is segment k of row number ord; it goes to slot g mod nslot,
+      // whose use count parity is `phase` (counters, not 64-bit divisions)
+      int slot = 0, k = 0;
+      uint32_t phase = 0;
+      int64_t ord = blockIdx.x;
       for (int64_t g = 0; g < nseg; ++g) {
         if (*abort_flag) break;
-        const int slot = static_cast<int>(g % nslot);
-        const uint32_t round = static_cast<uint32_t>(g / nslot);
-        if (!mbar_wait(&empty[slot], (round & 1u) ^ 1u, abort_flag, p.wait_limit_ns)) {
+        if (!mbar_wait(&empty[slot], phase ^ 1u, abort_flag, p.wait_limit_ns)) {
           if (!*abort_flag) atomicOr(&g_far_error, kErrWaitEmpty);
           *abort_flag = 1;
           break;
         }
-        if (g == p.stall_segment) {  // test hook: this copy is never issued
-          issued = g + 1;
-          continue;
+        if (g != p.stall_segment) {  // test hook: that copy is never issued
+          const void* base = (k < p.W) ? p.partials[k] : p.residual;
+          const unsigned char* src = static_cast<const unsigned char*>(base) +
+                                     call_row(p, ord) * static_cast<int64_t>(seg_bytes);
+          mbar_arrive_expect_tx(&full[slot], seg_bytes);
+          bulk_load(ring + static_cast<size_t>(slot) * seg_bytes, src, seg_bytes, &full[slot]);
         }
-        const int64_t row = p.row_begin + blockIdx.x + (g / S) * gridDim.x;
-        const int k = static_cast<int>(g % S);
-        const void* base = (k < p.W) ? p.partials[k] : p.residual;
-        const unsigned char* src = static_cast<const unsigned char*>(base) + row * static_cast<int64_t>(seg_bytes);
-        mbar_arrive_expect_tx(&full[slot], seg_bytes);
-        bulk_load(ring + static_cast<size_t>(slot) * seg_bytes, src, seg_bytes, &full[slot]);
         issued = g + 1;
+        if (++slot == nslot) {
+          slot = 0;
+          phase ^= 1u;
+        }
+        if (++k == S) {
+          k = 0;
+          ord += gridDim.x;
+        }
       }
       *issued_count = issued;  // read by the drain below
       __threadfence_block();
@@ -723,8 +741,10 @@ far_ring_kernel(const Params p, int nslot, int ncons) {
   // consumers
   const RingRed red0{&hdr->red[0][0][0], ncons}, red1{&hdr->red[1][0][0], ncons};
   const int j0 = threadIdx.x;
+  int slot = 0;  // the slot of the next segment and its use count parity
+  uint32_t phase = 0;
   for (int64_t i = 0; i < my_rows; ++i) {
-    const int64_t row = p.row_begin + blockIdx.x + i * gridDim.x;
+    const int64_t row = call_row(p, blockIdx.x + i * gridDim.x);
     float y[VPT][8];
     bool ok[VPT];
 #pragma unroll
@@ -734,10 +754,7 @@ far_ring_kernel(const Params p, int nslot, int ncons) {
       for (int e = 0; e < 8; ++e) y[k][e] = 0.f;
     }
     for (int k = 0; k < S; ++k) {
-      const int64_t g = i * S + k;
-      const int slot = static_cast<int>(g % nslot);
-      const uint32_t round = static_cast<uint32_t>(g / nslot);
-      if (!*abort_flag && !mbar_wait(&full[slot], round & 1u, abort_flag, p.wait_limit_ns)) {
+      if (!*abort_flag && !mbar_wait(&full[slot], phase, abort_flag, p.wait_limit_ns)) {
         if (!*abort_flag) atomicOr(&g_far_error, kErrWaitFull);
         *abort_flag = 1;
       }
@@ -747,6 +764,10 @@ far_ring_kernel(const Params p, int nslot, int ncons) {
         if (ok[q]) add_pack<DT>(seg[j0 + q * ncons], y[q]);
       __syncwarp();
       if ((threadIdx.x & 31) == 0) mbar_arrive(&empty[slot]);
+      if (++slot == nslot) {
+        slot = 0;
+        phase ^= 1u;
+      }
     }
     finish_row<DT, VPT, GROUP>(p, row, true, j0, ncons, ok, y, (i & 1) ? red1 : red0, gamma_s);
   }

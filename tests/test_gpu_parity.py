@@ -434,6 +434,36 @@ def test_per_tensor_fp8(kctx, ctx, case, kern):
     assert np.any((got["quant_out"] & 0x7F) == 0x7E)
 
 
+@pytest.mark.parametrize("case", [
+    (2, 77, 64, "direct"),      # several rows per CTA, a partly filled last CTA
+    (4, 600, 8192, "ring"),     # persistent CTAs, more rows than CTAs
+    (8, 9, 4096, "auto"),       # decode-sized
+], ids=lambda c: "W%d_T%d_H%d_%s" % c)
+def test_per_tensor_fp8_row_order(case):
+    """The second pass may take the rows last row first: every output is the
+    same bit for bit (each row's arithmetic is untouched, the scale is a max)."""
+    W, T, H, kern = case
+    env = {"FAR_RING_MIN_ROWS": "1"} if kern == "ring" else {}
+    if kern == "direct":
+        env["FAR_PREFILL_KERNEL"] = "0"
+    fwd = _ctx_with_env(dict(env, FAR_TENSOR_REVERSE="0"))
+    rev = _ctx_with_env(dict(env, FAR_TENSOR_REVERSE="1"))
+    try:
+        if kern != "auto":
+            far.far_set_regime(fwd, far.FAR_REGIME_PREFILL)
+            far.far_set_regime(rev, far.FAR_REGIME_PREFILL)
+        inp = random_inputs(W, T, H, seed=900 + T)
+        g = to_gpu(inp)
+        a = run_gpu(fwd, g, 1e-6, 0.0, 3, guard=256)
+        b = run_gpu(rev, g, 1e-6, 0.0, 3, guard=256)
+        for k in a:
+            assert np.array_equal(a[k], b[k]), k
+        log("tensor order %s" % (case,), compare(b, run_oracle(inp, "bf16", 1e-6, 0.0, 3), "bf16"))
+    finally:
+        fwd.close()
+        rev.close()
+
+
 def test_per_tensor_fp8_row_range_and_full_size(ctx):
     # rows [100, 3000) of the Gemma workload: the scale covers those rows only
     wl = WORKLOADS["c5_gemma_fp8_token_bf16"]
