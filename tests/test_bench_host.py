@@ -6,7 +6,7 @@ import os
 import time
 
 import bench
-from reduce_residual_add_b200.inputs import WORKLOADS
+from reduce_residual_add_b200.inputs import WORKLOADS, make_inputs
 
 
 def test_algorithmic_bytes_of_the_workloads():
@@ -59,3 +59,15 @@ def test_workload_config_for_every_workload():
         cfg = bench.workload_config(wl, bench.algorithmic_bytes(wl, wl.T, False), False, {}, 1)
         assert cfg["workload"] == name and cfg["pattern"] in bench.PATTERN_NAMES.values()
         json.dumps(cfg)
+
+
+def test_cpu_baseline_on_all_cores_and_single_threaded():
+    wl = WORKLOADS["c3_3d"].with_(T=96)
+    inp = make_inputs(wl)
+    out = bench.cpu_baseline(wl, inp, False, budget_s=0.05)
+    assert out["kind"] == "oracle" and out["value"] > 0
+    assert 1 <= out["cores"] <= bench.host_cores()
+    assert out["single_thread"]["cores"] == 1 and out["single_thread"]["value"] > 0
+    # per-tensor FP8: one scale over every row, so one thread
+    assert bench.oracle_threads(WORKLOADS["c4_prefill_fp8_tensor"], 8192, 64) == 1
+    assert bench.oracle_threads(WORKLOADS["c4_prefill_fp8_static"], 5, 64) == 5
