@@ -351,10 +351,13 @@ def graph_time(case: Case, launches: int, reps: int = 5) -> float:
     return t
 
 
-def e2e_time(case: Case, inp: dict, steps: int):
+def e2e_time(case: Case, inp: dict, steps: int, chunk_rows: int = 0):
     """Through the public API from pinned host memory: every step copies the
-    inputs host->device, runs the call, and copies the outputs back."""
-    s = case.stream
+    inputs host->device, runs the epilogue and copies the outputs back.
+    far_fused_host does it in chunks of rows whose copies overlap the
+    kernels; per-tensor FP8 (one scale over every row: no chunks) copies
+    everything in, calls far_fused_fp8_tensor and copies everything out."""
+    far, wl, s = case.far, case.wl, case.stream
     h_ps = [p.pin_memory() for p in inp["partials"]]
     h_res = None if inp["residual"] is None else inp["residual"].pin_memory()
     h_gam = inp["gamma"].pin_memory()
@@ -362,25 +365,40 @@ def e2e_time(case: Case, inp: dict, steps: int):
     h_q = torch.empty(case.qout.shape, dtype=torch.uint8).pin_memory() if case.qout is not None else None
     h_s = torch.empty(case.sout.shape, dtype=torch.float32).pin_memory() if case.sout is not None else None
     h_n = torch.empty(case.nout.shape, dtype=case.nout.dtype).pin_memory() if case.nout is not None else None
-    h2d = sum(p.numel() * 2 for p in h_ps) + (h_res.numel() * 2 if h_res is not None else 0) + h_gam.numel() * 2
+    h_sin = torch.tensor([wl.static_scale], dtype=torch.float32) if wl.pattern == 1 else None
+    h2d = sum(p.numel() * 2 for p in h_ps) + (h_res.numel() * 2 if h_res is not None else 0) + \
+        h_gam.numel() * 2 + (4 if h_sin is not None else 0)
     d2h = h_rout.numel() * 2 + (h_q.numel() if h_q is not None else 0) + \
         (h_s.numel() * 4 if h_s is not None else 0) + (h_n.numel() * 2 if h_n is not None else 0)
+    mode = "far_fused_host, chunks of %s rows" % (chunk_rows or "the default")
 
-    def one():
-        with torch.cuda.stream(s):
-            for d, h in zip(case.ps, h_ps):
-                d.copy_(h, non_blocking=True)
-            if h_res is not None:
-                case.res.copy_(h_res, non_blocking=True)
-            case.gam.copy_(h_gam, non_blocking=True)
-            case.step()
-            h_rout.copy_(case.rout, non_blocking=True)
-            if h_q is not None:
+    if wl.pattern == 3:
+        mode = "copies in, far_fused_fp8_tensor, copies out"
+
+        def one():
+            with torch.cuda.stream(s):
+                for d, h in zip(case.ps, h_ps):
+                    d.copy_(h, non_blocking=True)
+                if h_res is not None:
+                    case.res.copy_(h_res, non_blocking=True)
+                case.gam.copy_(h_gam, non_blocking=True)
+                case.step()
+                h_rout.copy_(case.rout, non_blocking=True)
                 h_q.copy_(case.qout, non_blocking=True)
-            if h_s is not None:
                 h_s.copy_(case.sout, non_blocking=True)
-            if h_n is not None:
-                h_n.copy_(case.nout, non_blocking=True)
+                if h_n is not None:
+                    h_n.copy_(case.nout, non_blocking=True)
+    else:
+        H = wl.H
+        staging = torch.empty(far.far_host_staging_bytes(wl.W, H, chunk_rows), dtype=torch.uint8,
+                              device=case.rout.device)
+        h_flat = None if h_s is None else h_s.view(-1)
+
+        def one():
+            far.far_fused_host(case.ctx, h_ps, h_res, h_gam, wl.eps, wl.weight_bias, wl.pattern,
+                               staging=staging, chunk_rows=chunk_rows, group_size=wl.group_size,
+                               residual_out=h_rout, norm_out=h_n, quant_out=h_q, scale_in=h_sin,
+                               scale_out=h_flat, stream=s)
 
     one()
     torch.cuda.synchronize()
@@ -390,7 +408,7 @@ def e2e_time(case: Case, inp: dict, steps: int):
         one()
     b.record(s)
     torch.cuda.synchronize()
-    return a.elapsed_time(b) / 1e3 / steps, h2d, d2h
+    return a.elapsed_time(b) / 1e3 / steps, h2d, d2h, mode
 
 
 def kernel_source_hash() -> str:
@@ -467,7 +485,7 @@ def run_far(args, world, rank, local):
     value = bytes_all / total_max / 1e9
     peak, peak_kind = hbm_peak()
     achieved = case.bytes / mean_launch / 1e9
-    e2e_s, h2d, d2h = e2e_time(case, inp, args.e2e_steps)
+    e2e_s, h2d, d2h, e2e_mode = e2e_time(case, inp, args.e2e_steps, args.e2e_chunk_rows)
     e2e_s = max_over_ranks(e2e_s, world)
 
     line = {
@@ -489,8 +507,8 @@ def run_far(args, world, rank, local):
                      "mean_launch_us": round(mean_launch * 1e6, 3)},
         "e2e": {"value": round(case.bytes / e2e_s / 1e9, 3), "unit": "GB/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "steps": args.e2e_steps, "ms_per_step": round(e2e_s * 1e3, 3)},
-        "gpu_launches": args.steps,
+                "steps": args.e2e_steps, "ms_per_step": round(e2e_s * 1e3, 3), "path": e2e_mode},
+        "gpu_launches": args.steps * (2 if wl.pattern == 3 else 1),
         "clocks": clocks,
     }
 
@@ -603,6 +621,8 @@ def main():
     ap.add_argument("--rows", type=int, default=0,
                     help="override the workload's row count (smaller cases for profiling)")
     ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--e2e-chunk-rows", type=int, default=0,
+                    help="rows per chunk of far_fused_host in the e2e leg (0: the library default)")
     ap.add_argument("--no-extras", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()

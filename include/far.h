@@ -44,7 +44,8 @@
  *
  * Ownership: the caller owns every buffer.  The library allocates and frees
  * nothing per call and never synchronises the stream; a call only enqueues
- * one kernel on `stream` and returns.  Results are ready when the stream
+ * one kernel on `stream` (two for per-tensor FP8; copies and one kernel per
+ * chunk for far_fused_host) and returns.  Results are ready when the stream
  * reaches that point.  The W partials live in the same GPU's memory (the
  * tensor-parallel ranks' outputs gathered on one device); they are read only.
  *
@@ -140,7 +141,9 @@ typedef struct {
  * with FAR_ERR_CUDA when the device cannot be queried. */
 far_status far_create(far_ctx **ctx, int device);
 
-/* Destroy a context (NULL is accepted).  Waits for nothing. */
+/* Destroy a context (NULL is accepted).  Waits for nothing; the copy
+ * streams and events of far_fused_host are released once their work is
+ * done. */
 far_status far_destroy(far_ctx *ctx);
 
 /*
@@ -277,6 +280,58 @@ far_status far_fused_fp8_tensor_noalloc(far_ctx *ctx, int64_t row_begin, int64_t
                                         far_dtype dtype, float eps, float weight_bias,
                                         void *norm_out, void *quant_out, float *scale_out,
                                         void *stream);
+
+/* Bytes of device staging far_fused_host needs for W partials of rows of H
+ * elements in chunks of `chunk_rows` rows (0: the library's default chunk,
+ * about 64 MiB of inputs); 0 for a W or H out of range.  It does not depend
+ * on T, the dtype, the pattern or which outputs are wanted. */
+size_t far_host_staging_bytes(int W, int64_t H, int64_t chunk_rows);
+
+/*
+ * The fused epilogue on HOST buffers: the operation and the arguments of
+ * far_fused (and of far_fused_fp8_group for FAR_AR_RESIDUAL_RMSNORM_FP8_GROUP,
+ * whose group size is `group_size`; ignored otherwise), except that every
+ * tensor -- partials, residual, residual_out, gamma, norm_out, quant_out,
+ * scale_in, scale_out -- is in host memory.  The library has no counterpart
+ * on the pages, whose inputs are already on the GPU; it serves callers whose
+ * activations live in host memory and measures the path end to end.
+ *
+ * The rows go through `staging` (device memory of at least
+ * far_host_staging_bytes(W, H, chunk_rows) bytes, 256-byte aligned) in
+ * chunks of `chunk_rows` rows (0: the default): chunk c is copied in on one
+ * of the context's two copy streams, reduced and normalised on `stream`,
+ * and copied out on the other copy stream, each step ordered by events, so
+ * the copy in of chunk c+1 and the copy out of chunk c-1 overlap chunk c.
+ * Gamma (and the static scale) are copied once per call.  The results are in
+ * the host buffers once `stream` reaches the end of the call (the call
+ * itself does not wait); each chunk's kernel is the one far_fused would
+ * launch for that many rows, so every row's outputs are those of a device
+ * call on the chunk.
+ *
+ * Host buffers should be page-locked (cudaHostAlloc / cudaHostRegister);
+ * pageable memory works, but the driver then copies synchronously and
+ * nothing overlaps.  Tensor pointers must be 16-byte aligned, as for
+ * far_fused, and the same overlap rules apply.  Per-tensor FP8 is refused
+ * (FAR_ERR_UNSUPPORTED): its scale needs every row before any code.
+ * chunk_rows < 0 or a staging area that is NULL or too small gives
+ * FAR_ERR_INVALID_ARG, a misaligned one FAR_ERR_ALIGNMENT.  The staging
+ * area is scratch; calls that share one must not overlap on the GPU (calls
+ * on one context are ordered through its events; the enqueueing is
+ * serialised by a lock of the context).  A CUDA error part-way through the
+ * enqueueing returns FAR_ERR_CUDA, and the work already enqueued still runs.
+ * The first call on a context creates its two copy streams and seven
+ * events, released by far_destroy; make that first call before any stream
+ * capture.
+ */
+far_status far_fused_host(far_ctx *ctx,
+                          const void *const *partials, int W,
+                          const void *residual, void *residual_out,
+                          const void *gamma, int64_t T, int64_t H, far_dtype dtype,
+                          float eps, float weight_bias, far_pattern pattern, int group_size,
+                          void *norm_out, void *quant_out,
+                          const float *scale_in, float *scale_out,
+                          int64_t chunk_rows, void *staging, size_t staging_bytes,
+                          void *stream);
 
 /* Host-only: the status far_fused_rows would return for these arguments
  * before launching (it touches no GPU and needs no context).  With pattern

@@ -36,6 +36,12 @@ struct far_ctx {
   // 0 = not asked yet, -1 = cannot run
   std::mutex occ_mu;
   int ring_occ[2][far::kMaxH / far::kPackElems + 1][2];  // [dtype][packs][2 or 3 CTAs/SM wanted]
+  // far_fused_host: its two copy streams and the events of its two staging
+  // buffers, created on first use, guarded by host_mu
+  std::mutex host_mu;
+  bool host_ready;
+  cudaStream_t host_h2d, host_d2h;
+  cudaEvent_t host_start, host_in[2], host_comp[2], host_out[2];
 };
 
 namespace {
@@ -57,6 +63,24 @@ int env_int(const char* name, int dflt) {
 }
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+// Free far_fused_host's streams and events (each once its work is done).
+void host_pipe_release(far_ctx* ctx) {
+  if (!ctx->host_ready) return;
+  int prev = -1;
+  const bool switched = cudaGetDevice(&prev) == cudaSuccess && prev != ctx->device &&
+                        cudaSetDevice(ctx->device) == cudaSuccess;
+  cudaStreamDestroy(ctx->host_h2d);
+  cudaStreamDestroy(ctx->host_d2h);
+  cudaEventDestroy(ctx->host_start);
+  for (int b = 0; b < 2; ++b) {
+    cudaEventDestroy(ctx->host_in[b]);
+    cudaEventDestroy(ctx->host_comp[b]);
+    cudaEventDestroy(ctx->host_out[b]);
+  }
+  ctx->host_ready = false;
+  if (switched) cudaSetDevice(prev);
+}
 
 struct Range {
   uintptr_t lo, hi;  // [lo, hi)
@@ -302,6 +326,7 @@ far_status far_create(far_ctx** ctx, int device) {
 }
 
 far_status far_destroy(far_ctx* ctx) {
+  if (ctx != nullptr) host_pipe_release(ctx);
   delete ctx;
   return FAR_OK;
 }
@@ -550,6 +575,99 @@ far_status far_fused_fp8_tensor_launch(far_ctx* ctx, int64_t row_begin, int64_t 
   return FAR_OK;
 }
 
+bool group_size_ok(int g) { return g >= 8 && g <= 256 && (g & (g - 1)) == 0; }
+
+// Per-group FP8, once far_validate passed: H must hold whole groups, and
+// scale_out (T x H / group_size floats) may overlap no other buffer.
+far_status check_group_scales(const void* const* partials, int W, const void* residual,
+                              const void* residual_out, const void* gamma, int64_t T, int64_t H,
+                              int group_size, const void* norm_out, const void* quant_out,
+                              const float* scale_out) {
+  if (H % group_size != 0) return FAR_ERR_UNSUPPORTED;
+  if (T > 0) {
+    const Range sc = span(scale_out, T * (H / group_size) * 4);
+    const int64_t tb = T * H * 2;
+    for (int r = 0; r < W; ++r)
+      if (overlap(sc, span(partials[r], tb))) return FAR_ERR_INVALID_ARG;
+    const void* bufs16[] = {residual, residual_out, norm_out};
+    for (const void* b : bufs16)
+      if (b != nullptr && overlap(sc, span(b, tb))) return FAR_ERR_INVALID_ARG;
+    if (overlap(sc, span(gamma, H * 2)) || overlap(sc, span(quant_out, T * H)))
+      return FAR_ERR_INVALID_ARG;
+  }
+  return FAR_OK;
+}
+
+// ---------------------------------------------------------------------------
+// far_fused_host: host buffers through a device staging area, in chunks of
+// rows.  Chunk c uses staging buffer c % 2; its copy in (stream host_h2d),
+// its kernel (the caller's stream) and its copy out (stream host_d2h) are
+// ordered by events, so chunk c+1 is copied in and chunk c-1 copied out
+// while chunk c runs.
+// ---------------------------------------------------------------------------
+
+size_t round256(int64_t x) { return static_cast<size_t>((x + 255) / 256 * 256); }
+
+// About 64 MiB of inputs per chunk: measured on B200 over PCIe with the
+// W=4 8192 x 8192 workload, 4 / 8 / 16 / 32 / 64 MiB chunks gave 47 / 54 /
+// 60 / 64 / 65 GB/s end to end (fewer, larger copies; the first chunk's
+// copy in and the last one's copy out are the only parts not overlapped).
+int64_t default_chunk_rows(int W, int64_t H) {
+  const int64_t row_in = static_cast<int64_t>(W + 1) * H * 2;  // bytes copied in per row
+  const int64_t r = (int64_t{64} << 20) / row_in;
+  return r > 0 ? r : 1;
+}
+
+// Staging layout: [gamma | scale_in | buffer 0 | buffer 1], every part
+// 256-byte aligned; a buffer is [W partials | residual | residual_out |
+// norm_out | quant_out | scale_out] for `rows` rows, with room for the
+// largest scale_out (one per group of 8 elements).
+struct Staging {
+  size_t seg;      // one (rows, H) block of 2-byte elements
+  size_t codes;    // the (rows, H) block of FP8 codes
+  size_t scales;   // rows * H / 8 floats
+  size_t head;     // gamma, then scale_in
+  size_t per_buf;
+  size_t total;
+};
+
+Staging staging_layout(int W, int64_t H, int64_t rows) {
+  Staging L;
+  L.seg = round256(rows * H * 2);
+  L.codes = round256(rows * H);
+  L.scales = round256(rows * (H / 8) * 4);
+  L.head = round256(H * 2) + 256;
+  L.per_buf = static_cast<size_t>(W + 3) * L.seg + L.codes + L.scales;
+  L.total = L.head + 2 * L.per_buf;
+  return L;
+}
+
+far_status host_pipe_ready(far_ctx* ctx) {
+  if (ctx->host_ready) return FAR_OK;
+  cudaError_t e = cudaSuccess;
+  cudaStream_t s[2] = {nullptr, nullptr};
+  cudaEvent_t ev[7] = {};
+  for (int i = 0; i < 2 && e == cudaSuccess; ++i) e = cudaStreamCreateWithFlags(&s[i], cudaStreamNonBlocking);
+  for (int i = 0; i < 7 && e == cudaSuccess; ++i) e = cudaEventCreateWithFlags(&ev[i], cudaEventDisableTiming);
+  if (e != cudaSuccess) {
+    for (cudaStream_t x : s)
+      if (x != nullptr) cudaStreamDestroy(x);
+    for (cudaEvent_t x : ev)
+      if (x != nullptr) cudaEventDestroy(x);
+    return cuda_fail(e, "far_fused_host: creating its streams and events");
+  }
+  ctx->host_h2d = s[0];
+  ctx->host_d2h = s[1];
+  ctx->host_start = ev[0];
+  for (int b = 0; b < 2; ++b) {
+    ctx->host_in[b] = ev[1 + b];
+    ctx->host_comp[b] = ev[3 + b];
+    ctx->host_out[b] = ev[5 + b];
+  }
+  ctx->host_ready = true;
+  return FAR_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -693,25 +811,14 @@ far_status far_fused_fp8_group(far_ctx* ctx, int64_t row_begin, int64_t row_end,
                                far_dtype dtype, float eps, float weight_bias, int group_size,
                                void* norm_out, void* quant_out, float* scale_out, void* stream) {
   if (ctx == nullptr) return FAR_ERR_INVALID_ARG;
-  if (group_size < 8 || group_size > 256 || (group_size & (group_size - 1)) != 0)
-    return FAR_ERR_UNSUPPORTED;
+  if (!group_size_ok(group_size)) return FAR_ERR_UNSUPPORTED;
   far_status st = far_validate(row_begin, row_end, partials, W, residual, residual_out, gamma, T, H,
                                dtype, eps, weight_bias, FAR_AR_RESIDUAL_RMSNORM_FP8_GROUP, norm_out,
                                quant_out, nullptr, scale_out);
   if (st != FAR_OK) return st;
-  if (H % group_size != 0) return FAR_ERR_UNSUPPORTED;
-  if (T > 0) {
-    // scale_out holds T x (H / group_size) floats: it may overlap no other buffer
-    const Range sc = span(scale_out, T * (H / group_size) * 4);
-    const int64_t tb = T * H * 2;
-    for (int r = 0; r < W; ++r)
-      if (overlap(sc, span(partials[r], tb))) return FAR_ERR_INVALID_ARG;
-    const void* bufs16[] = {residual, residual_out, norm_out};
-    for (const void* b : bufs16)
-      if (b != nullptr && overlap(sc, span(b, tb))) return FAR_ERR_INVALID_ARG;
-    if (overlap(sc, span(gamma, H * 2)) || overlap(sc, span(quant_out, T * H)))
-      return FAR_ERR_INVALID_ARG;
-  }
+  st = check_group_scales(partials, W, residual, residual_out, gamma, T, H, group_size, norm_out,
+                          quant_out, scale_out);
+  if (st != FAR_OK) return st;
   if (row_end == row_begin) return FAR_OK;
 
   far::Params p = make_params(partials, W, residual, residual_out, gamma, H,
@@ -742,6 +849,155 @@ far_status far_fused(far_ctx* ctx, const void* const* partials, int W, const voi
                      void* quant_out, const float* scale_in, float* scale_out, void* stream) {
   return far_fused_rows(ctx, 0, T, partials, W, residual, residual_out, gamma, T, H, dtype, eps,
                         weight_bias, pattern, norm_out, quant_out, scale_in, scale_out, stream);
+}
+
+size_t far_host_staging_bytes(int W, int64_t H, int64_t chunk_rows) {
+  if (W < 1 || W > FAR_MAX_W || H <= 0 || H % far::kPackElems != 0 || H > far::kMaxH) return 0;
+  const int64_t rows = chunk_rows > 0 ? chunk_rows : default_chunk_rows(W, H);
+  return staging_layout(W, H, rows).total;
+}
+
+far_status far_fused_host(far_ctx* ctx, const void* const* partials, int W, const void* residual,
+                          void* residual_out, const void* gamma, int64_t T, int64_t H,
+                          far_dtype dtype, float eps, float weight_bias, far_pattern pattern,
+                          int group_size, void* norm_out, void* quant_out, const float* scale_in,
+                          float* scale_out, int64_t chunk_rows, void* staging,
+                          size_t staging_bytes, void* stream) {
+  if (ctx == nullptr) return FAR_ERR_INVALID_ARG;
+  if (pattern == FAR_AR_RESIDUAL_RMSNORM_FP8_TENSOR) {
+    std::snprintf(g_last_error, sizeof(g_last_error),
+                  "far_fused_host: per-tensor FP8 needs every row before any code; "
+                  "use far_fused_fp8_tensor on device buffers");
+    return FAR_ERR_UNSUPPORTED;
+  }
+  const bool group = pattern == FAR_AR_RESIDUAL_RMSNORM_FP8_GROUP;
+  if (group && !group_size_ok(group_size)) return FAR_ERR_UNSUPPORTED;
+  far_status st = far_validate(0, T, partials, W, residual, residual_out, gamma, T, H, dtype, eps,
+                               weight_bias, pattern, norm_out, quant_out, scale_in, scale_out);
+  if (st != FAR_OK) return st;
+  if (group) {
+    st = check_group_scales(partials, W, residual, residual_out, gamma, T, H, group_size,
+                            norm_out, quant_out, scale_out);
+    if (st != FAR_OK) return st;
+  }
+  if (chunk_rows < 0) return FAR_ERR_INVALID_ARG;
+  if (T == 0) return FAR_OK;
+  int64_t R = chunk_rows > 0 ? chunk_rows : default_chunk_rows(W, H);
+  const Staging L = staging_layout(W, H, R);  // sized for R rows, as the caller's query
+  if (R > T) R = T;
+  if (staging == nullptr || staging_bytes < L.total) return FAR_ERR_INVALID_ARG;
+  if (!aligned(staging, 256)) return FAR_ERR_ALIGNMENT;
+
+  DeviceGuard guard(ctx->device);
+  if (guard.err != cudaSuccess) return cuda_fail(guard.err, "cudaSetDevice");
+  std::lock_guard<std::mutex> lock(ctx->host_mu);
+  st = host_pipe_ready(ctx);
+  if (st != FAR_OK) return st;
+
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const cudaStream_t in = ctx->host_h2d, out = ctx->host_d2h;
+  unsigned char* const base = static_cast<unsigned char*>(staging);
+  const int64_t rb = H * 2;  // bytes of one row of 2-byte elements
+  // where the new residual goes: residual_out, else in place into residual
+  void* const h_rout = residual_out != nullptr ? residual_out : const_cast<void*>(residual);
+  const int64_t nsc = pattern == FAR_AR_RESIDUAL_RMSNORM_FP8_TOKEN ? 1
+                      : group                                      ? H / group_size
+                                                                   : 0;  // scales per row
+  cudaError_t e = cudaSuccess;
+#define FAR_HOST_CK(call, what)                 \
+  do {                                          \
+    if ((e = (call)) != cudaSuccess) return cuda_fail(e, "far_fused_host: " what); \
+  } while (0)
+
+  // copies start after the caller's earlier work on `stream`
+  FAR_HOST_CK(cudaEventRecord(ctx->host_start, s), "cudaEventRecord");
+  FAR_HOST_CK(cudaStreamWaitEvent(in, ctx->host_start, 0), "cudaStreamWaitEvent");
+  // gamma and the static scale, once per call
+  FAR_HOST_CK(cudaMemcpyAsync(base, gamma, static_cast<size_t>(rb), cudaMemcpyHostToDevice, in),
+              "copy of gamma");
+  float* const d_scale_in = reinterpret_cast<float*>(base + round256(rb));
+  if (pattern == FAR_AR_RESIDUAL_RMSNORM_FP8_STATIC)
+    FAR_HOST_CK(cudaMemcpyAsync(d_scale_in, scale_in, 4, cudaMemcpyHostToDevice, in),
+                "copy of scale_in");
+
+  const int64_t nchunks = (T + R - 1) / R;
+  for (int64_t c = 0; c < nchunks; ++c) {
+    const int b = static_cast<int>(c & 1);
+    const int64_t r0 = c * R;
+    const int64_t n = T - r0 < R ? T - r0 : R;
+    unsigned char* const buf = base + L.head + b * L.per_buf;
+    unsigned char* const d_res = buf + W * L.seg;
+    unsigned char* const d_rout = d_res + L.seg;
+    unsigned char* const d_norm = d_rout + L.seg;
+    unsigned char* const d_quant = d_norm + L.seg;
+    float* const d_scale = reinterpret_cast<float*>(d_quant + L.codes);
+
+    // copy in, once buffer b's previous chunk (in this call or an earlier
+    // one on this context) has been copied out; an event never recorded
+    // makes no one wait
+    FAR_HOST_CK(cudaStreamWaitEvent(in, ctx->host_out[b], 0), "cudaStreamWaitEvent");
+    const void* d_parts[far::kMaxW];
+    for (int r = 0; r < W; ++r) {
+      d_parts[r] = buf + r * L.seg;
+      FAR_HOST_CK(cudaMemcpyAsync(buf + r * L.seg, static_cast<const unsigned char*>(partials[r]) + r0 * rb,
+                                  static_cast<size_t>(n * rb), cudaMemcpyHostToDevice, in),
+                  "copy in of a partial");
+    }
+    if (residual != nullptr)
+      FAR_HOST_CK(cudaMemcpyAsync(d_res, static_cast<const unsigned char*>(residual) + r0 * rb,
+                                  static_cast<size_t>(n * rb), cudaMemcpyHostToDevice, in),
+                  "copy in of the residual");
+    FAR_HOST_CK(cudaEventRecord(ctx->host_in[b], in), "cudaEventRecord");
+
+    // the kernel, on the caller's stream (no programmatic launch: it follows
+    // an event wait, not a kernel)
+    FAR_HOST_CK(cudaStreamWaitEvent(s, ctx->host_in[b], 0), "cudaStreamWaitEvent");
+    far::Params p = make_params(d_parts, W, residual != nullptr ? d_res : nullptr,
+                                h_rout != nullptr ? d_rout : nullptr, base, H, pattern, eps,
+                                weight_bias, norm_out != nullptr ? d_norm : nullptr,
+                                quant_out != nullptr ? d_quant : nullptr,
+                                pattern == FAR_AR_RESIDUAL_RMSNORM_FP8_STATIC ? d_scale_in : nullptr,
+                                nsc > 0 ? d_scale : nullptr);
+    p.wait_limit_ns = ctx->wait_limit_ns;
+    p.stall_segment = ctx->stall_segment;
+    far::Launch l = plan(ctx, n, H, dtype, W + (residual != nullptr ? 1 : 0));
+    if (group) {
+      p.group_lanes = group_size / far::kPackElems;
+      p.groups_per_row = static_cast<int>(H / group_size);
+      if (l.regime == FAR_REGIME_DECODE) {  // groups need the one-CTA kernels
+        plan_prefill(static_cast<int>(H / far::kPackElems), ctx->prefill_threads, &l);
+        l.grid = (n + l.rows_per_cta - 1) / l.rows_per_cta;
+      }
+    }
+    l.pdl = 0;
+    FAR_HOST_CK(launch_rows(p, dtype, l, 0, n, s), "kernel launch");
+    FAR_HOST_CK(cudaEventRecord(ctx->host_comp[b], s), "cudaEventRecord");
+
+    // copy out
+    FAR_HOST_CK(cudaStreamWaitEvent(out, ctx->host_comp[b], 0), "cudaStreamWaitEvent");
+    if (h_rout != nullptr)
+      FAR_HOST_CK(cudaMemcpyAsync(static_cast<unsigned char*>(h_rout) + r0 * rb, d_rout,
+                                  static_cast<size_t>(n * rb), cudaMemcpyDeviceToHost, out),
+                  "copy out of residual_out");
+    if (norm_out != nullptr)
+      FAR_HOST_CK(cudaMemcpyAsync(static_cast<unsigned char*>(norm_out) + r0 * rb, d_norm,
+                                  static_cast<size_t>(n * rb), cudaMemcpyDeviceToHost, out),
+                  "copy out of norm_out");
+    if (quant_out != nullptr)
+      FAR_HOST_CK(cudaMemcpyAsync(static_cast<unsigned char*>(quant_out) + r0 * H, d_quant,
+                                  static_cast<size_t>(n * H), cudaMemcpyDeviceToHost, out),
+                  "copy out of quant_out");
+    if (nsc > 0)
+      FAR_HOST_CK(cudaMemcpyAsync(scale_out + r0 * nsc, d_scale, static_cast<size_t>(n * nsc * 4),
+                                  cudaMemcpyDeviceToHost, out),
+                  "copy out of scale_out");
+    FAR_HOST_CK(cudaEventRecord(ctx->host_out[b], out), "cudaEventRecord");
+  }
+  // the caller's stream reaches the end of the call once every copy out is done
+  FAR_HOST_CK(cudaStreamWaitEvent(s, ctx->host_out[0], 0), "cudaStreamWaitEvent");
+  if (nchunks > 1) FAR_HOST_CK(cudaStreamWaitEvent(s, ctx->host_out[1], 0), "cudaStreamWaitEvent");
+#undef FAR_HOST_CK
+  return FAR_OK;
 }
 
 }  // extern "C"

@@ -48,7 +48,8 @@ FAR_FP8_TENSOR_NOALLOC_MAX_ROWS = 65536
 # Every symbol include/far.h declares.
 EXPORTS = ("far_create", "far_destroy", "far_fused", "far_fused_rows",
            "far_fp8_tensor_workspace_bytes", "far_fused_fp8_tensor",
-           "far_fused_fp8_tensor_noalloc", "far_fused_fp8_group", "far_validate",
+           "far_fused_fp8_tensor_noalloc", "far_fused_fp8_group",
+           "far_host_staging_bytes", "far_fused_host", "far_validate",
            "far_set_regime", "far_describe_launch", "far_check", "far_test_stall",
            "far_status_string",
            "far_last_error", "far_version")
@@ -116,6 +117,11 @@ def lib() -> ctypes.CDLL:
     L.far_fused_fp8_group.argtypes = [vp, i64, i64, pp, i32, vp, vp, vp, i64, i64, i32, f32, f32,
                                       i32, vp, vp, vp, vp]
     L.far_fused_fp8_group.restype = i32
+    L.far_host_staging_bytes.argtypes = [i32, i64, i64]
+    L.far_host_staging_bytes.restype = ctypes.c_size_t
+    L.far_fused_host.argtypes = [vp, pp, i32, vp, vp, vp, i64, i64, i32, f32, f32, i32, i32,
+                                 vp, vp, vp, vp, i64, vp, ctypes.c_size_t, vp]
+    L.far_fused_host.restype = i32
     L.far_set_regime.argtypes = [vp, i32, i32]
     L.far_set_regime.restype = i32
     L.far_describe_launch.argtypes = [vp, i64, i64, i32, i32, i32, ctypes.POINTER(far_launch_info)]
@@ -224,26 +230,27 @@ def _ptr(t: Optional[torch.Tensor]):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
 
-def _flat(t: Optional[torch.Tensor], H: int, name: str) -> Optional[torch.Tensor]:
+def _flat(t: Optional[torch.Tensor], H: int, name: str, host: bool = False) -> Optional[torch.Tensor]:
     if t is None:
         return None
-    if not t.is_cuda:
-        raise ValueError("%s must be a CUDA tensor" % name)
+    if t.is_cuda == host:
+        raise ValueError("%s must be a %s tensor" % (name, "host (CPU)" if host else "CUDA"))
     if not t.is_contiguous():
         raise ValueError("%s must be contiguous" % name)
     return t.view(-1, H) if t.dim() != 2 else t
 
 
 def _args(partials, residual, gamma, residual_out, norm_out, quant_out, scale_in, scale_out,
-          scale_out_elems=None):
+          scale_out_elems=None, host=False):
+    where = "host (CPU)" if host else "CUDA"
     if isinstance(partials, torch.Tensor):
         partials = [partials]
     if len(partials) == 0:
         raise ValueError("need at least one partial")
-    if not gamma.is_contiguous() or not gamma.is_cuda:
-        raise ValueError("gamma must be a contiguous CUDA tensor")
+    if not gamma.is_contiguous() or gamma.is_cuda == host:
+        raise ValueError("gamma must be a contiguous %s tensor" % where)
     H = gamma.numel()
-    ps = [_flat(p, H, "partials[%d]" % i) for i, p in enumerate(partials)]
+    ps = [_flat(p, H, "partials[%d]" % i, host) for i, p in enumerate(partials)]
     T = ps[0].shape[0]
     dt = _DTYPES.get(ps[0].dtype)
     if dt is None:
@@ -253,10 +260,10 @@ def _args(partials, residual, gamma, residual_out, norm_out, quant_out, scale_in
             raise ValueError("partials must share shape and dtype")
     arr = (ctypes.c_void_p * len(ps))(*[p.data_ptr() for p in ps])
     # the C side sees plain pointers: make sure each buffer covers (T, H)
-    res = _flat(residual, H, "residual")
-    rout = _flat(residual_out, H, "residual_out")
-    nout = _flat(norm_out, H, "norm_out")
-    qout = _flat(quant_out, H, "quant_out")
+    res = _flat(residual, H, "residual", host)
+    rout = _flat(residual_out, H, "residual_out", host)
+    nout = _flat(norm_out, H, "norm_out", host)
+    qout = _flat(quant_out, H, "quant_out", host)
     for name, t in (("residual", res), ("residual_out", rout), ("norm_out", nout)):
         if t is not None and (t.shape != (T, H) or t.dtype != ps[0].dtype):
             raise ValueError("%s must be (%d, %d) %s" % (name, T, H, ps[0].dtype))
@@ -266,9 +273,10 @@ def _args(partials, residual, gamma, residual_out, norm_out, quant_out, scale_in
         raise ValueError("gamma must be %s" % ps[0].dtype)
     for name, t, n in (("scale_in", scale_in, 1),
                        ("scale_out", scale_out, T if scale_out_elems is None else scale_out_elems)):
-        if t is not None and (not t.is_cuda or t.dtype != torch.float32 or t.numel() < n
+        if t is not None and (t.is_cuda == host or t.dtype != torch.float32 or t.numel() < n
                               or not t.is_contiguous()):
-            raise ValueError("%s must be a contiguous CUDA float32 tensor of >= %d elements" % (name, n))
+            raise ValueError("%s must be a contiguous %s float32 tensor of >= %d elements"
+                             % (name, where, n))
     return (arr, len(ps), _ptr(res), _ptr(rout), _ptr(gamma), T, H, dt,
             _ptr(nout), _ptr(qout), _ptr(scale_in), _ptr(scale_out))
 
@@ -441,3 +449,39 @@ def far_fused_fp8_group(ctx: FarContext, partials: Sequence[torch.Tensor],
                                    _stream(stream))
     if st != FAR_OK:
         raise FarError(st, "far_fused_fp8_group")
+
+
+def far_host_staging_bytes(W: int, H: int, chunk_rows: int = 0) -> int:
+    """Device staging bytes far_fused_host needs (0 for W or H out of range)."""
+    return int(lib().far_host_staging_bytes(int(W), int(H), int(chunk_rows)))
+
+
+def far_fused_host(ctx: FarContext, partials: Sequence[torch.Tensor],
+                   residual: Optional[torch.Tensor], gamma: torch.Tensor, eps: float,
+                   weight_bias: float = 0.0, pattern: int = FAR_AR_RESIDUAL_RMSNORM, *,
+                   staging: torch.Tensor, chunk_rows: int = 0, group_size: int = 0,
+                   residual_out: Optional[torch.Tensor] = None,
+                   norm_out: Optional[torch.Tensor] = None,
+                   quant_out: Optional[torch.Tensor] = None,
+                   scale_in: Optional[torch.Tensor] = None,
+                   scale_out: Optional[torch.Tensor] = None, stream=None) -> None:
+    """The fused epilogue on host (CPU) tensors, through the device buffer
+    ``staging`` (uint8, at least far_host_staging_bytes(W, H, chunk_rows)
+    bytes) in chunks of rows; pin the host tensors for the copies to overlap
+    the kernels.  Every host tensor, scale_in included, is a CPU tensor; the
+    results are there once ``stream`` reaches the end of the call."""
+    H = gamma.numel()
+    T = partials[0].numel() // H if len(partials) else 0
+    n_sc = T * (H // group_size) if pattern == FAR_AR_RESIDUAL_RMSNORM_FP8_GROUP and group_size > 0 else None
+    (arr, W, res, rout, gam, T, H, dt, nout, qout, sin, sout) = _args(
+        partials, residual, gamma, residual_out, norm_out, quant_out, scale_in, scale_out,
+        scale_out_elems=n_sc, host=True)
+    if not staging.is_cuda or not staging.is_contiguous():
+        raise ValueError("staging must be a contiguous CUDA tensor")
+    nbytes = staging.numel() * staging.element_size()
+    st = lib().far_fused_host(ctx.handle, arr, W, res, rout, gam, T, H, dt, float(eps),
+                              float(weight_bias), int(pattern), int(group_size), nout, qout, sin,
+                              sout, int(chunk_rows), ctypes.c_void_p(staging.data_ptr()), nbytes,
+                              _stream(stream))
+    if st != FAR_OK:
+        raise FarError(st, "far_fused_host")

@@ -203,3 +203,23 @@ def test_per_tensor_workspace_size():
     assert far.far_fp8_tensor_workspace_bytes(64) == 512
     assert far.far_fp8_tensor_workspace_bytes(65) == 768
     assert far.far_fp8_tensor_workspace_bytes(8192) == 256 + 4 * 8192
+
+
+def test_host_staging_bytes():
+    """far_host_staging_bytes (host only): gamma + scale header, then two
+    buffers of W partials, residual, residual_out, norm_out (2-byte rows),
+    FP8 codes and the largest scale block, each part 256-byte aligned."""
+    def r256(x):
+        return (x + 255) // 256 * 256
+    W, H, R = 4, 8192, 100
+    seg, codes, scales = r256(R * H * 2), r256(R * H), r256(R * (H // 8) * 4)
+    want = r256(H * 2) + 256 + 2 * ((W + 3) * seg + codes + scales)
+    assert far.far_host_staging_bytes(W, H, R) == want
+    # the default chunk: about 64 MiB of inputs
+    dflt = (64 << 20) // ((W + 1) * H * 2)
+    assert far.far_host_staging_bytes(W, H, 0) == far.far_host_staging_bytes(W, H, dflt)
+    # out of range
+    assert far.far_host_staging_bytes(0, H, R) == 0
+    assert far.far_host_staging_bytes(17, H, R) == 0
+    assert far.far_host_staging_bytes(W, 12, R) == 0
+    assert far.far_host_staging_bytes(W, 16392, R) == 0
