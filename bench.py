@@ -526,12 +526,16 @@ def extras(ctx, device, stream) -> dict:
     from reduce_residual_add_b200 import far
     out = {}
     peak, _ = hbm_peak()
-    for name in ("c5_gemma_fp8_token_bf16", "c5_gemma_fp8_token_fp16", "c4_prefill_fp8_tensor",
-                 "c4_prefill_fp8_group128", "c3_3d"):
+    for name, with_norm in (("c5_gemma_fp8_token_bf16", False), ("c5_gemma_fp8_token_fp16", False),
+                            ("c5_gemma_fp8_token_bf16", True), ("c4_prefill_fp8_static", True),
+                            ("c4_prefill_fp8_tensor", False), ("c4_prefill_fp8_group128", False),
+                            ("c3_3d", False)):
         wl = WORKLOADS[name]
         inp = make_inputs(wl)
-        case = Case(ctx, wl, inp, device, False, stream)
+        case = Case(ctx, wl, inp, device, with_norm, stream)
         total, mean = case.time_steps(200, 20, per_launch=True)
+        if with_norm:
+            name += "+norm_out"
         out[name] = {"GB/s": round(case.bytes / mean / 1e9, 1),
                      "launches_per_call": 2 if wl.pattern == 3 else 1,
                      "frac": round(case.bytes / mean / 1e9 / peak, 4),
