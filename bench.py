@@ -468,7 +468,8 @@ def run_far(args, world, rank, local):
     stream = torch.cuda.Stream(device=device)
     ctx = far.FarContext(local)
     case = Case(ctx, wl, inp, device, args.with_norm, stream)
-    launch = far.far_describe_launch(ctx, wl.T, wl.H, wl.torch_dtype, wl.W, wl.has_residual)
+    launch = far.far_describe_launch(ctx, wl.T, wl.H, wl.torch_dtype, wl.W, wl.has_residual,
+                                     case.nout is not None)
 
     case.time_steps(0, args.warmup, per_launch=False)
     barrier(world)
@@ -544,6 +545,12 @@ def extras(ctx, device, stream) -> dict:
         if name == "c3_3d":
             out[name]["graph_us_per_call"] = round(graph_time(case, 50) * 1e6, 3)
         del case
+    # the latency floor of one call: a single row of 64 elements, one partial
+    wl = WORKLOADS["c1_small"].with_(name="floor_W1_T1_H64", W=1, T=1)
+    case = Case(ctx, wl, make_inputs(wl), device, False, stream)
+    out["floor_W1_T1_H64"] = {"graph_us_per_call": round(graph_time(case, 100) * 1e6, 3),
+                              "note": "latency floor: the smallest call, same kernels and launch path"}
+    del case
     for T in (1, 8, 32, 80):
         wl = WORKLOADS["c2_decode_T%d" % T]
         inp = make_inputs(wl)

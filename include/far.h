@@ -107,10 +107,15 @@ typedef enum {
  * FAR_DECODE_MAX_ROWS, FAR_FORCE_REGIME=decode|prefill, FAR_DECODE_CLUSTER
  * (CTAs per row; default by rule),
  * FAR_PREFILL_THREADS, FAR_PREFILL_KERNEL=1 ring | 0 direct,
- * FAR_RING_CTAS_PER_SM=1..4 (default: 3 for rows of at most 6 segments,
- * else 2), FAR_RING_THREADS: consumer threads
- * per ring CTA, at most 256 (default 256), FAR_RING_SLOTS: row-segment slots
- * per ring CTA (2..32; default: about 72 KiB of segments, as many as fit),
+ * FAR_RING_CTAS_PER_SM=1..4, FAR_RING_THREADS: consumer threads per ring
+ * CTA, at most 256, FAR_RING_SLOTS: row-segment slots per ring CTA (2..32),
+ * FAR_RING_GAMMA_SMEM=1|0: gamma staged in shared memory or read through
+ * L1 (each replaces its part of the measured default rule: 3 CTAs per SM
+ * for rows of at most 6 segments, else 2; 256 consumers, 4 packs each for
+ * rows of 512-1023 packs with at most 6 segments; gamma in shared memory and
+ * about 72 KiB of slots; with norm_out and at most 6 segments of >= 16 KiB,
+ * or when fewer than 3 slots would fit: 2 CTAs per SM, gamma through L1,
+ * about 96 KiB of slots),
  * FAR_PDL=1|0: launch with programmatic dependent launch, default 1,
  * FAR_RING_MIN_ROWS: fewest rows for the ring kernel, default by rule,
  * FAR_TENSOR_REVERSE=1|0: the second pass of per-tensor FP8 takes the rows
@@ -134,6 +139,7 @@ typedef struct {
     int64_t grid_ctas;    /* CTAs of the launch                       */
     int kernel;           /* prefill: 1 = TMA bulk-copy ring, 0 = direct loads */
     int ring_slots;       /* ring: shared-memory slots of one row segment */
+    int ring_gamma_smem;  /* ring: 1 = gamma staged in shared memory, 0 = read through L1 */
 } far_launch_info;
 
 /* Create a context for CUDA device `device` (its ordinal).  Fails with
@@ -361,9 +367,10 @@ far_status far_set_regime(far_ctx *ctx, far_regime regime, int decode_max_rows);
 far_status far_test_stall(far_ctx *ctx, int64_t segment, uint32_t wait_limit_us);
 
 /* Fill `info` with the launch geometry a call on `rows` rows of W partials
- * (and a residual when has_residual != 0) would use. */
+ * (and a residual when has_residual != 0, writing norm_out when
+ * has_norm_out != 0) would use. */
 far_status far_describe_launch(const far_ctx *ctx, int64_t rows, int64_t H,
-                               far_dtype dtype, int W, int has_residual,
+                               far_dtype dtype, int W, int has_residual, int has_norm_out,
                                far_launch_info *info);
 
 /* Wait for `stream`, then read and clear the device-side error word of

@@ -26,16 +26,24 @@ struct far_ctx {
   int prefill_kernel;   // 1 = TMA bulk-copy ring (default), 0 = direct loads
   int ring_ctas_per_sm; // persistent ring CTAs per SM wanted (1..4; 0 = by rule)
   int ring_threads;     // target consumer threads of a ring CTA
+  int ring_threads_set; // ring_threads came from the environment
   int ring_slots_max;   // at most this many ring slots
   int tensor_reverse;   // per-tensor FP8: second pass from the last row down
+  int ring_gamma_mode;  // ring: 1 stage gamma in shared memory, 0 read it through L1, -1 by rule
   int pdl;              // programmatic dependent launch on every call
   int ring_min_rows;    // fewer rows than this take the direct kernel
   uint64_t wait_limit_ns;  // bounded waits in the kernels give up after this
   int64_t stall_segment;   // test hook (far_test_stall), -1 when off
   // ring CTAs per SM the occupancy calculator allows, per (dtype, packs):
   // 0 = not asked yet, -1 = cannot run
+  // resident ring CTAs per SM for the configurations asked so far
+  struct OccEntry {
+    int dtype, vpt, minb, threads, smem, ctas;
+  };
+  static constexpr int kOccEntries = 256;
   std::mutex occ_mu;
-  int ring_occ[2][far::kMaxH / far::kPackElems + 1][2];  // [dtype][packs][2 or 3 CTAs/SM wanted]
+  OccEntry occ[kOccEntries];
+  int occ_n;
   // far_fused_host: its two copy streams and the events of its two staging
   // buffers, created on first use, guarded by host_mu
   std::mutex host_mu;
@@ -143,48 +151,77 @@ void plan_decode(int packs, int cluster_pref, far::Launch* l) {
   l->rows_per_cta = 1;
 }
 
-// Ring geometry: consumers = the fewest packs per thread (1, 2, 4, 8) that
-// keep within ring_threads, plus one producer warp; as many row-segment
-// slots (at most 32) as fit in a 1/ring_ctas_per_sm share of the SM's
-// 228 KiB of shared memory (less the 1 KiB the system keeps per CTA); a
+// Resident ring CTAs per SM for one configuration, cached per context
+// (the occupancy calculator costs microseconds): 0 = cannot run.
+int ring_occ_cached(const far_ctx* ctx, int dtype, int vpt, int minb, int threads, int smem);
+
+// Ring geometry, all measured on B200 (fractions of the measured HBM copy
+// bandwidth; each rule is used only where it was measured to win):
+//  * consumers: the fewest packs per thread (1, 2, 4, 8) that keep within
+//    ring_threads (256), plus one producer warp; except that rows of 512 to
+//    1023 packs with at most 6 segments take 4 packs per thread (H=4096,
+//    W=4: 128-thread CTAs, 97 vs 85 %);
+//  * CTAs per SM: 3 (registers capped at 72) for rows of at most 6
+//    segments (W=4 + residual: 95.5 vs 93.3 % with 2), else 2 (W=8 +
+//    residual: 89.1 vs 87.9 % with 3);
+//  * gamma staged in shared memory, and about 72 KiB of row-segment slots
+//    per CTA (as many as fit a 1/(CTAs per SM) share of the SM's 228 KiB,
+//    less the 1 KiB the system keeps per CTA);
+//  * except when norm_out is written, for rows of at most 6 segments of at
+//    least 16 KiB: 2 CTAs per SM, gamma read through L1 and about 96 KiB of
+//    slots (W=3..5, H=8192: 97-102 vs 87-94 %);
+//  * and when fewer than 3 slots fit: 2 CTAs per SM with gamma through L1
+//    (H=16384, W=1..3: 88-92 %, where the one-CTA-per-row kernel gave 63-73 %).
+// Environment overrides (FAR_RING_CTAS_PER_SM, FAR_RING_THREADS,
+// FAR_RING_SLOTS, FAR_RING_GAMMA_SMEM) replace the rule they name.  A
 // persistent grid of sm_count x (the CTAs per SM the occupancy calculator
-// confirms, at most ring_ctas_per_sm), fewer for fewer rows.  Returns false
-// (the direct kernel runs) when fewer than two slots fit or the
-// configuration cannot be resident.
-bool plan_ring(const far_ctx* ctx, int packs, int64_t rows, int dtype, int segs, far::Launch* l) {
+// confirms), fewer for fewer rows.  Returns false (the direct kernel runs)
+// when fewer than two slots fit or the configuration cannot be resident.
+bool plan_ring(const far_ctx* ctx, int packs, int64_t rows, int dtype, int segs, bool norm,
+               far::Launch* l) {
   if (packs <= 32) return false;
   const int seg = packs * 16;
-  // CTAs per SM: measured on B200, 3 (registers capped at 72) when a row has
-  // few segments (W=4 + residual: 95.5 % vs 93.3 % with 2), 2 (86 registers)
-  // when it has many (W=8 + residual: 89.1 % vs 87.9 % with 3)
-  const int n_req = ctx->ring_ctas_per_sm > 0 ? ctx->ring_ctas_per_sm : (segs <= 6 ? 3 : 2);
   int vpt = 1;
   while (vpt < 8 && (packs + vpt - 1) / vpt > ctx->ring_threads) vpt *= 2;
+  if (!ctx->ring_threads_set && segs <= 6 && packs >= 512 && packs < 1024 && vpt < 4) vpt = 4;
   const int tpr = (((packs + vpt - 1) / vpt) + 31) / 32 * 32;
   if (tpr > far::kRingMaxConsumers) return false;
-  int per_cta = 228 * 1024 / n_req - 1024;
-  if (per_cta > far::kRingSmemMax) per_cta = far::kRingSmemMax;
-  // header, gamma (one segment's worth of bytes), slots: about 72 KiB of
-  // segments in flight per CTA measured best (4 slots at H=8192, 5 at 7168)
-  int nslot = ctx->ring_slots_max > 0 ? ctx->ring_slots_max : 72 * 1024 / seg;
-  if (nslot > 32) nslot = 32;
-  while (nslot >= 2 && far::ring_header_bytes(nslot) + (nslot + 1) * seg > per_cta) --nslot;
-  if (nslot < 2) return false;
-  const int smem = far::ring_header_bytes(nslot) + (nslot + 1) * seg;
-  int occ;
-  {
-    std::lock_guard<std::mutex> lock(const_cast<far_ctx*>(ctx)->occ_mu);
-    int& cached = const_cast<far_ctx*>(ctx)->ring_occ[dtype][packs][n_req >= 3 ? 1 : 0];
-    if (cached == 0) {
-      const int n = far::ring_occupancy(dtype, vpt, n_req >= 3 ? 3 : 2, tpr + 32, smem);
-      cached = n > 0 ? n : -1;
-    }
-    occ = cached;
+
+  int n_req = segs <= 6 ? 3 : 2;
+  bool gamma_smem = true;
+  int target = 72 * 1024;  // slot bytes per CTA
+  if (norm && segs <= 6 && seg >= 16 * 1024) {
+    n_req = 2;
+    gamma_smem = false;
+    target = 96 * 1024;
   }
+  if (ctx->ring_ctas_per_sm > 0) n_req = ctx->ring_ctas_per_sm;
+  if (ctx->ring_gamma_mode >= 0) gamma_smem = ctx->ring_gamma_mode != 0;
+  auto fit = [&](int n, bool gs, int bytes) {
+    int per_cta = 228 * 1024 / n - 1024;
+    if (per_cta > far::kRingSmemMax) per_cta = far::kRingSmemMax;
+    int ns = ctx->ring_slots_max > 0 ? ctx->ring_slots_max : bytes / seg;
+    if (ns > 32) ns = 32;
+    while (ns >= 2 && far::ring_header_bytes(ns) + (ns + (gs ? 1 : 0)) * seg > per_cta) --ns;
+    return ns;
+  };
+  int nslot = fit(n_req, gamma_smem, target);
+  if (nslot < 3 && ctx->ring_ctas_per_sm == 0 && ctx->ring_gamma_mode < 0) {
+    n_req = 2;
+    gamma_smem = false;
+    target = 96 * 1024;
+    nslot = fit(n_req, gamma_smem, target);
+  }
+  if (nslot < 2) return false;
+  const int gsegs = gamma_smem ? 1 : 0;
+  const int smem = far::ring_header_bytes(nslot) + (nslot + gsegs) * seg;
+  const int minb = n_req >= 3 ? 3 : 2;
+  int occ = ring_occ_cached(ctx, dtype, vpt, minb, tpr + 32, smem);
   if (occ < 1) return false;
   if (occ > n_req) occ = n_req;
   l->kernel = 1;
-  l->ring_minb = n_req >= 3 ? 3 : 2;
+  l->ring_minb = minb;
+  l->ring_gamma = gsegs;
   l->vpt = vpt;
   l->tpr = tpr;
   l->rows_per_cta = 1;
@@ -196,8 +233,22 @@ bool plan_ring(const far_ctx* ctx, int packs, int64_t rows, int dtype, int segs,
   return true;
 }
 
-// segs = row segments read per row: W partials, plus the residual if any.
-far::Launch plan(const far_ctx* ctx, int64_t rows, int64_t H, int dtype, int segs) {
+int ring_occ_cached(const far_ctx* ctx, int dtype, int vpt, int minb, int threads, int smem) {
+  far_ctx* c = const_cast<far_ctx*>(ctx);
+  std::lock_guard<std::mutex> lock(c->occ_mu);
+  for (int i = 0; i < c->occ_n; ++i) {
+    const far_ctx::OccEntry& e = c->occ[i];
+    if (e.dtype == dtype && e.vpt == vpt && e.minb == minb && e.threads == threads && e.smem == smem)
+      return e.ctas;
+  }
+  const int n = far::ring_occupancy(dtype, vpt, minb, threads, smem);
+  if (c->occ_n < far_ctx::kOccEntries) c->occ[c->occ_n++] = far_ctx::OccEntry{dtype, vpt, minb, threads, smem, n};
+  return n;
+}
+
+// segs = row segments read per row: W partials, plus the residual if any;
+// norm: the call writes norm_out.
+far::Launch plan(const far_ctx* ctx, int64_t rows, int64_t H, int dtype, int segs, bool norm) {
   const int packs = static_cast<int>(H / far::kPackElems);
   far::Launch l{};
   bool decode;
@@ -237,7 +288,7 @@ far::Launch plan(const far_ctx* ctx, int64_t rows, int64_t H, int dtype, int seg
       const int per_cta = (4096 / packs > 8) ? 4096 / packs : 8;
       min_rows = static_cast<int64_t>(per_cta) * ctx->sm_count * 2;
     }
-    if (ctx->prefill_kernel == 1 && rows >= min_rows) plan_ring(ctx, packs, rows, dtype, segs, &l);
+    if (ctx->prefill_kernel == 1 && rows >= min_rows) plan_ring(ctx, packs, rows, dtype, segs, norm, &l);
   }
   l.pdl = ctx->pdl;
   return l;
@@ -296,8 +347,12 @@ far_status far_create(far_ctx** ctx, int device) {
   if (c.ring_ctas_per_sm < 0) c.ring_ctas_per_sm = 0;
   if (c.ring_ctas_per_sm > 4) c.ring_ctas_per_sm = 4;
   c.ring_threads = env_int("FAR_RING_THREADS", 256);  // at most kRingMaxConsumers
+  c.ring_threads_set = std::getenv("FAR_RING_THREADS") != nullptr;
   c.ring_slots_max = env_int("FAR_RING_SLOTS", 0);  // 0: by the 72 KiB rule
   c.tensor_reverse = env_int("FAR_TENSOR_REVERSE", 1) != 0;
+  c.ring_gamma_mode = env_int("FAR_RING_GAMMA_SMEM", -1);
+  if (c.ring_gamma_mode > 1) c.ring_gamma_mode = 1;
+  if (c.ring_gamma_mode < -1) c.ring_gamma_mode = -1;
   if (c.ring_slots_max < 0) c.ring_slots_max = 0;
   if (c.ring_slots_max > 32) c.ring_slots_max = 32;
   if (c.ring_threads < 32) c.ring_threads = 32;
@@ -348,7 +403,7 @@ far_status far_set_regime(far_ctx* ctx, far_regime regime, int decode_max_rows) 
 }
 
 far_status far_describe_launch(const far_ctx* ctx, int64_t rows, int64_t H, far_dtype dtype,
-                               int W, int has_residual, far_launch_info* info) {
+                               int W, int has_residual, int has_norm_out, far_launch_info* info) {
   if (ctx == nullptr || info == nullptr || rows < 0) return FAR_ERR_INVALID_ARG;
   if (W < 1 || W > FAR_MAX_W) return FAR_ERR_INVALID_ARG;
   if (dtype != FAR_BF16 && dtype != FAR_FP16) return FAR_ERR_INVALID_ARG;
@@ -358,7 +413,7 @@ far_status far_describe_launch(const far_ctx* ctx, int64_t rows, int64_t H, far_
   if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
   if (prev != ctx->device && (e = cudaSetDevice(ctx->device)) != cudaSuccess)
     return cuda_fail(e, "cudaSetDevice");
-  const far::Launch l = plan(ctx, rows, H, dtype, W + (has_residual ? 1 : 0));
+  const far::Launch l = plan(ctx, rows, H, dtype, W + (has_residual ? 1 : 0), has_norm_out != 0);
   if (prev != ctx->device) cudaSetDevice(prev);
   info->regime = l.regime;
   info->ctas_per_row = l.cluster;
@@ -368,6 +423,7 @@ far_status far_describe_launch(const far_ctx* ctx, int64_t rows, int64_t H, far_
   info->grid_ctas = l.grid;
   info->kernel = l.kernel;
   info->ring_slots = l.nslot;
+  info->ring_gamma_smem = l.kernel == 1 ? l.ring_gamma : 0;
   return FAR_OK;
 }
 
@@ -553,7 +609,8 @@ far_status far_fused_fp8_tensor_launch(far_ctx* ctx, int64_t row_begin, int64_t 
   if (guard.err != cudaSuccess) return cuda_fail(guard.err, "cudaSetDevice");
   const cudaStream_t s = static_cast<cudaStream_t>(stream);
   // per-tensor: never the cluster kernel (no reduction in the second pass)
-  far::Launch whole = plan(ctx, row_end - row_begin, H, dtype, W + (residual != nullptr ? 1 : 0));
+  far::Launch whole = plan(ctx, row_end - row_begin, H, dtype, W + (residual != nullptr ? 1 : 0),
+                   norm_out != nullptr);
   if (whole.regime == FAR_REGIME_DECODE) {
     plan_prefill(static_cast<int>(H / far::kPackElems), ctx->prefill_threads, &whole);
     whole.grid = (row_end - row_begin + whole.rows_per_cta - 1) / whole.rows_per_cta;
@@ -695,7 +752,8 @@ far_status far_fused_rows(far_ctx* ctx, int64_t row_begin, int64_t row_end,
   p.stall_segment = ctx->stall_segment;
   DeviceGuard guard(ctx->device);
   if (guard.err != cudaSuccess) return cuda_fail(guard.err, "cudaSetDevice");
-  const far::Launch whole = plan(ctx, row_end - row_begin, H, dtype, W + (residual != nullptr ? 1 : 0));
+  const far::Launch whole = plan(ctx, row_end - row_begin, H, dtype, W + (residual != nullptr ? 1 : 0),
+                   norm_out != nullptr);
   const cudaError_t e = launch_rows(p, dtype, whole, row_begin, row_end, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "kernel launch");
   return FAR_OK;
@@ -832,7 +890,8 @@ far_status far_fused_fp8_group(far_ctx* ctx, int64_t row_begin, int64_t row_end,
   if (guard.err != cudaSuccess) return cuda_fail(guard.err, "cudaSetDevice");
   // a group must sit on consecutive lanes of one warp: not the cluster kernel,
   // whose per-CTA slices need not start on a group boundary
-  far::Launch whole = plan(ctx, row_end - row_begin, H, dtype, W + (residual != nullptr ? 1 : 0));
+  far::Launch whole = plan(ctx, row_end - row_begin, H, dtype, W + (residual != nullptr ? 1 : 0),
+                   norm_out != nullptr);
   if (whole.regime == FAR_REGIME_DECODE) {
     plan_prefill(static_cast<int>(H / far::kPackElems), ctx->prefill_threads, &whole);
     whole.grid = (row_end - row_begin + whole.rows_per_cta - 1) / whole.rows_per_cta;
@@ -960,7 +1019,8 @@ far_status far_fused_host(far_ctx* ctx, const void* const* partials, int W, cons
                                 nsc > 0 ? d_scale : nullptr);
     p.wait_limit_ns = ctx->wait_limit_ns;
     p.stall_segment = ctx->stall_segment;
-    far::Launch l = plan(ctx, n, H, dtype, W + (residual != nullptr ? 1 : 0));
+    far::Launch l = plan(ctx, n, H, dtype, W + (residual != nullptr ? 1 : 0),
+                          norm_out != nullptr);
     if (group) {
       p.group_lanes = group_size / far::kPackElems;
       p.groups_per_row = static_cast<int>(H / group_size);

@@ -68,6 +68,7 @@ struct Launch {
   int smem_bytes;       // ring: dynamic shared memory per CTA
   int pdl;              // launch with programmatic stream serialization
   int ring_minb;        // ring: CTAs per SM its registers are sized for (2 or 3)
+  int ring_gamma;       // ring: 1 = gamma staged in shared memory, 0 = read through L1
 };
 
 // Enqueue one kernel on `stream`.  Returns the launch error (cudaSuccess if

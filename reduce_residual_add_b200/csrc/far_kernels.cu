@@ -392,6 +392,12 @@ struct RingRed {
 // This thread owns packs j = j0 + k*jstride (k < VPT) where ok[k].
 // ---------------------------------------------------------------------------
 
+// Pack j of gamma: from shared memory where the CTA staged it, else
+// through L1 (every row of a CTA reads the same packs).
+__device__ __forceinline__ uint4 gamma_pack(const Params& p, const uint4* gamma_smem, int j) {
+  return gamma_smem != nullptr ? gamma_smem[j] : __ldg(static_cast<const uint4*>(p.gamma) + j);
+}
+
 // GROUP: this instantiation serves only the per-group pattern (kept apart
 // so that the other patterns' code carries none of its registers).
 template <class DT, int VPT, bool GROUP, class Red>
@@ -428,7 +434,6 @@ __device__ __forceinline__ void finish_row(const Params& p, int64_t row, bool ro
   const bool fp8_static = p.pattern == kFp8Static;
   const bool fp8_token = p.pattern == kFp8Token;
   constexpr bool fp8_group = GROUP;
-  const uint4* gam = gamma_smem != nullptr ? gamma_smem : static_cast<const uint4*>(p.gamma);
 
   // a5b needs max|o| = rinv * max|y * (gamma + wb)| (rinv > 0): its local
   // part goes into the same reduction round as the sum of squares.  The
@@ -440,7 +445,7 @@ __device__ __forceinline__ void finish_row(const Params& p, int64_t row, bool ro
     for (int k = 0; k < VPT; ++k) {
       if (!ok[k]) continue;
       float g[8];
-      pack_plus<DT>(gam[j0 + k * jstride], p.weight_bias, g);
+      pack_plus<DT>(gamma_pack(p, gamma_smem, j0 + k * jstride), p.weight_bias, g);
 #pragma unroll
       for (int i = 0; i < 8; ++i) m = fmaxf(m, fabsf(y[k][i] * g[i]));
     }
@@ -487,7 +492,7 @@ __device__ __forceinline__ void finish_row(const Params& p, int64_t row, bool ro
     if (!ok[k]) continue;
     const int64_t pk = rbase + j0 + k * jstride;
     float g[8];  // gamma + weight_bias in fp32
-    pack_plus<DT>(gam[j0 + k * jstride], p.weight_bias, g);
+    pack_plus<DT>(gamma_pack(p, gamma_smem, j0 + k * jstride), p.weight_bias, g);
 #pragma unroll
     for (int i = 0; i < 8; ++i) y[k][i] = (y[k][i] * rinv) * g[i];
     if (p.norm_out != nullptr) static_cast<uint4*>(p.norm_out)[pk] = pack8<DT>(y[k]);
@@ -666,7 +671,7 @@ far_decode_kernel(const Params p) {
 // MINB: CTAs per SM the register budget is sized for (2 or 3; 1 at VPT 8).
 template <class DT, int VPT, int MINB, bool GROUP>
 __global__ void __launch_bounds__(kRingMaxConsumers + 32, MINB)
-far_ring_kernel(const Params p, int nslot, int ncons) {
+far_ring_kernel(const Params p, int nslot, int ncons, int stage_gamma) {
   pdl_enter();
   extern __shared__ __align__(128) unsigned char smem[];
   uint64_t* full = reinterpret_cast<uint64_t*>(smem);
@@ -676,8 +681,9 @@ far_ring_kernel(const Params p, int nslot, int ncons) {
   volatile int* producer_done = &hdr->producer_done;
   volatile long long* issued_count = &hdr->issued;
   const uint32_t seg_bytes = static_cast<uint32_t>(p.H) * 2u;
-  uint4* gamma_s = reinterpret_cast<uint4*>(smem + ring_offset(nslot));
-  unsigned char* ring = smem + ring_offset(nslot) + seg_bytes;
+  // gamma, when staged, sits between the header and the slots
+  uint4* gamma_s = stage_gamma ? reinterpret_cast<uint4*>(smem + ring_offset(nslot)) : nullptr;
+  unsigned char* ring = smem + ring_offset(nslot) + (stage_gamma ? seg_bytes : 0u);
   const int S = p.W + (p.residual != nullptr ? 1 : 0);
   const int64_t nrows = p.row_end - p.row_begin;
   const int64_t my_rows = (nrows - blockIdx.x + gridDim.x - 1) / gridDim.x;
@@ -693,8 +699,9 @@ far_ring_kernel(const Params p, int nslot, int ncons) {
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   // gamma: read once per CTA, kept in shared memory for every row
-  for (int j = threadIdx.x; j < p.packs; j += blockDim.x)
-    gamma_s[j] = __ldg(static_cast<const uint4*>(p.gamma) + j);
+  if (stage_gamma)
+    for (int j = threadIdx.x; j < p.packs; j += blockDim.x)
+      gamma_s[j] = __ldg(static_cast<const uint4*>(p.gamma) + j);
   __syncthreads();
 
   if (threadIdx.x >= ncons) {
@@ -845,7 +852,8 @@ cudaError_t launch_ring_t(const Params& p, const Launch& l, cudaStream_t s) {
   cfg.stream = s;
   cfg.attrs = at.a;
   cfg.numAttrs = at.n;
-  return cudaLaunchKernelEx(&cfg, far_ring_kernel<DT, VPT, MINB, GROUP>, p, l.nslot, l.tpr);
+  return cudaLaunchKernelEx(&cfg, far_ring_kernel<DT, VPT, MINB, GROUP>, p, l.nslot, l.tpr,
+                            l.ring_gamma);
 }
 
 template <class DT, bool GROUP>

@@ -61,7 +61,8 @@ class far_launch_info(ctypes.Structure):
     _fields_ = [("regime", ctypes.c_int), ("ctas_per_row", ctypes.c_int),
                 ("rows_per_cta", ctypes.c_int), ("threads_per_cta", ctypes.c_int),
                 ("packs_per_thread", ctypes.c_int), ("grid_ctas", ctypes.c_int64),
-                ("kernel", ctypes.c_int), ("ring_slots", ctypes.c_int)]
+                ("kernel", ctypes.c_int), ("ring_slots", ctypes.c_int),
+                ("ring_gamma_smem", ctypes.c_int)]
 
 
 class FarError(RuntimeError):
@@ -124,7 +125,8 @@ def lib() -> ctypes.CDLL:
     L.far_fused_host.restype = i32
     L.far_set_regime.argtypes = [vp, i32, i32]
     L.far_set_regime.restype = i32
-    L.far_describe_launch.argtypes = [vp, i64, i64, i32, i32, i32, ctypes.POINTER(far_launch_info)]
+    L.far_describe_launch.argtypes = [vp, i64, i64, i32, i32, i32, i32,
+                                      ctypes.POINTER(far_launch_info)]
     L.far_describe_launch.restype = i32
     L.far_test_stall.argtypes = [vp, i64, ctypes.c_uint32]
     L.far_test_stall.restype = i32
@@ -201,10 +203,11 @@ def far_set_regime(ctx: FarContext, regime: int, decode_max_rows: int = -1) -> N
 
 
 def far_describe_launch(ctx: FarContext, rows: int, H: int, dtype=torch.bfloat16, W: int = 8,
-                        has_residual: bool = True) -> dict:
+                        has_residual: bool = True, has_norm_out: bool = False) -> dict:
     info = far_launch_info()
     st = lib().far_describe_launch(ctx.handle, int(rows), int(H), _DTYPES.get(dtype, dtype),
-                                   int(W), int(bool(has_residual)), ctypes.byref(info))
+                                   int(W), int(bool(has_residual)), int(bool(has_norm_out)),
+                                   ctypes.byref(info))
     if st != FAR_OK:
         raise FarError(st, "far_describe_launch")
     return {name: getattr(info, name) for name, _ in far_launch_info._fields_}

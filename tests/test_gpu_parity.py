@@ -60,6 +60,8 @@ def kctx():
            "ring3": _ctx_with_env(dict(any_rows, FAR_RING_CTAS_PER_SM="3", FAR_L2_EVICT_FIRST="1",
                                        FAR_STREAM_STORES="1")),
            "ring2": _ctx_with_env(dict(any_rows, FAR_RING_CTAS_PER_SM="2", FAR_RING_THREADS="256")),
+           # gamma read through L1 instead of staged in shared memory
+           "ring_l1": _ctx_with_env(dict(any_rows, FAR_RING_GAMMA_SMEM="0")),
            "ring4": _ctx_with_env(dict(any_rows, FAR_RING_CTAS_PER_SM="4", FAR_RING_THREADS="128")),
            "direct": _ctx_with_env({"FAR_PREFILL_KERNEL": "0"})}
     for c in out.values():
@@ -110,7 +112,7 @@ def test_small_shapes(ctx, regime, case, reg):
     log("small %s reg%d" % (case, reg), compare(got, ref, dt))
 
 
-@pytest.mark.parametrize("kern", ["ring", "ring256", "ring3", "ring2", "ring4", "direct"])
+@pytest.mark.parametrize("kern", ["ring", "ring256", "ring3", "ring2", "ring_l1", "ring4", "direct"])
 @pytest.mark.parametrize("case", [
     (2, 3000, 264, "bf16", 2, True, 0.0),    # 33 packs, 32 slots, ~20 rows per CTA
     (16, 300, 16384, "bf16", 1, True, 1.0),  # 17 segments per row, 6 slots
@@ -341,7 +343,8 @@ def test_errors_are_reported_not_skipped(ctx):
 
 def test_launch_plan(ctx):
     """The measured dispatch rules (see far_abi.cu plan())."""
-    d = lambda rows, H, W, res=True: far.far_describe_launch(ctx, rows, H, torch.bfloat16, W, res)  # noqa: E731
+    d = lambda rows, H, W, res=True, norm=False: far.far_describe_launch(  # noqa: E731
+        ctx, rows, H, torch.bfloat16, W, res, norm)
     # decode-sized rows: a cluster per row once rows are large ...
     assert (d(4, 16384, 8)["regime"], d(4, 16384, 8)["ctas_per_row"]) == (far.FAR_REGIME_DECODE, 16)
     assert (d(1, 8192, 8)["regime"], d(1, 8192, 8)["ctas_per_row"]) == (far.FAR_REGIME_DECODE, 8)
@@ -355,6 +358,23 @@ def test_launch_plan(ctx):
     assert c4["kernel"] == 1 and c4["ring_slots"] >= 2
     assert (c4["threads_per_cta"] - 32) * c4["packs_per_thread"] * 8 >= 8192
     assert d(1200, 8192, 4)["kernel"] == 0
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    # few segments: 3 CTAs per SM, gamma in shared memory
+    assert (c4["grid_ctas"], c4["ring_gamma_smem"]) == (3 * sms, 1)
+    # ... but with norm_out, 2 CTAs per SM, gamma through L1, ~96 KiB of slots
+    c4n = d(8192, 8192, 4, norm=True)
+    assert (c4n["grid_ctas"], c4n["ring_gamma_smem"], c4n["ring_slots"]) == (2 * sms, 0, 6)
+    # many segments: 2 CTAs per SM, gamma in shared memory, ~72 KiB of slots
+    c5 = d(4096, 7168, 8)
+    assert (c5["grid_ctas"], c5["ring_gamma_smem"], c5["ring_slots"]) == (2 * sms, 1, 5)
+    # H=4096 with few segments: 4 packs per thread (128 consumers)
+    h4 = d(16384, 4096, 4)
+    assert (h4["packs_per_thread"], h4["threads_per_cta"]) == (4, 160)
+    # fewer than 3 slots would fit: the share of 2 CTAs per SM, gamma through
+    # L1 (at 8 packs per thread the registers then allow one CTA per SM)
+    h16 = d(8192, 16384, 2)
+    assert (h16["kernel"], h16["ring_gamma_smem"], h16["ring_slots"]) == (1, 0, 3)
+    assert h16["grid_ctas"] in (sms, 2 * sms)
     tiny = d(8, 64, 2)
     assert tiny["regime"] == far.FAR_REGIME_PREFILL and tiny["rows_per_cta"] > 1
 
@@ -620,7 +640,7 @@ def test_format_edges_overflow_and_subnormals(kctx, kern):
 # per-group FP8
 # ---------------------------------------------------------------------------
 
-@pytest.mark.parametrize("kern", ["ring", "direct", "auto"])
+@pytest.mark.parametrize("kern", ["ring", "ring_l1", "direct", "auto"])
 @pytest.mark.parametrize("case", [
     (2, 8, 64, 8, "bf16"),          # one pack per group; rows inside a warp
     (2, 8, 64, 64, "fp16"),         # one group per row
