@@ -438,6 +438,8 @@ __device__ __forceinline__ void finish_row(const Params& p, int64_t row, bool ro
   // a5b needs max|o| = rinv * max|y * (gamma + wb)| (rinv > 0): its local
   // part goes into the same reduction round as the sum of squares.  The
   // second per-tensor pass reuses the first pass's rinv: no reduction.
+  // Per-token keeps y * (gamma + wb) in y (one read of gamma per row), so
+  // its o is (y * g) * rinv; the other patterns form (y * rinv) * g below.
   float ss = 0.f, gmax = 0.f;
   if (fp8_token || tensor_amax) {
     float m = 0.f;
@@ -446,8 +448,16 @@ __device__ __forceinline__ void finish_row(const Params& p, int64_t row, bool ro
       if (!ok[k]) continue;
       float g[8];
       pack_plus<DT>(gamma_pack(p, gamma_smem, j0 + k * jstride), p.weight_bias, g);
+      if (fp8_token) {
 #pragma unroll
-      for (int i = 0; i < 8; ++i) m = fmaxf(m, fabsf(y[k][i] * g[i]));
+        for (int i = 0; i < 8; ++i) {
+          y[k][i] *= g[i];
+          m = fmaxf(m, fabsf(y[k][i]));
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) m = fmaxf(m, fabsf(y[k][i] * g[i]));
+      }
     }
     const float2 r = red.sum_max(sq[0], m);
     ss = r.x;
@@ -491,10 +501,15 @@ __device__ __forceinline__ void finish_row(const Params& p, int64_t row, bool ro
   for (int k = 0; k < VPT; ++k) {
     if (!ok[k]) continue;
     const int64_t pk = rbase + j0 + k * jstride;
-    float g[8];  // gamma + weight_bias in fp32
-    pack_plus<DT>(gamma_pack(p, gamma_smem, j0 + k * jstride), p.weight_bias, g);
+    if (fp8_token) {  // y already holds y * (gamma + wb)
 #pragma unroll
-    for (int i = 0; i < 8; ++i) y[k][i] = (y[k][i] * rinv) * g[i];
+      for (int i = 0; i < 8; ++i) y[k][i] *= rinv;
+    } else {
+      float g[8];  // gamma + weight_bias in fp32
+      pack_plus<DT>(gamma_pack(p, gamma_smem, j0 + k * jstride), p.weight_bias, g);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) y[k][i] = (y[k][i] * rinv) * g[i];
+    }
     if (p.norm_out != nullptr) static_cast<uint4*>(p.norm_out)[pk] = pack8<DT>(y[k]);
     if (fp8_static || fp8_token || tensor_quant) {  // (per-group codes: below)
       uint2 codes = make_uint2(0u, 0u);
