@@ -160,18 +160,25 @@ int ring_occ_cached(const far_ctx* ctx, int dtype, int vpt, int minb, int thread
 //  * consumers: the fewest packs per thread (1, 2, 4, 8) that keep within
 //    ring_threads (256), plus one producer warp; except that rows of 512 to
 //    1023 packs with at most 6 segments take 4 packs per thread (H=4096,
-//    W=4: 128-thread CTAs, 97 vs 85 %);
+//    W=4: 128-thread CTAs, 97 vs 85 %), and rows of at most 256 packs at
+//    most 128 consumers;
 //  * CTAs per SM: 3 (registers capped at 72) for rows of at most 6
 //    segments (W=4 + residual: 95.5 vs 93.3 % with 2), else 2 (W=8 +
 //    residual: 89.1 vs 87.9 % with 3);
 //  * gamma staged in shared memory, and about 72 KiB of row-segment slots
 //    per CTA (as many as fit a 1/(CTAs per SM) share of the SM's 228 KiB,
 //    less the 1 KiB the system keeps per CTA);
-//  * except when norm_out is written, for rows of at most 6 segments of at
-//    least 16 KiB: 2 CTAs per SM, gamma read through L1 and about 96 KiB of
-//    slots (W=3..5, H=8192: 97-102 vs 87-94 %);
+//  * except: rows of at most 256 packs (H <= 2048), 4 CTAs per SM (W=2..8:
+//    77-99 vs 63-80 %); 8 packs per thread (H >= 12288), one CTA per SM
+//    (all its registers allow) with 6 slots (H=16384, W=4: 82 / 90 vs 75 /
+//    82 % without / with norm_out); norm_out written and at most 6 segments
+//    of at least 16 KiB, 2 CTAs per SM, gamma read through L1 and about
+//    96 KiB of slots (W=3..5, H=8192: 97-102 vs 87-94 %); norm_out and at
+//    most 6 segments of 10-12 KiB, 2 CTAs per SM (H=5120 / 6144: 95-101 vs
+//    84-87 %);
 //  * and when fewer than 3 slots fit: 2 CTAs per SM with gamma through L1
-//    (H=16384, W=1..3: 88-92 %, where the one-CTA-per-row kernel gave 63-73 %).
+//    (H=16384 W=1..3 before the one-CTA rule: 88-92 %, where the
+//    one-CTA-per-row kernel gave 63-73 %).
 // Environment overrides (FAR_RING_CTAS_PER_SM, FAR_RING_THREADS,
 // FAR_RING_SLOTS, FAR_RING_GAMMA_SMEM) replace the rule they name.  A
 // persistent grid of sm_count x (the CTAs per SM the occupancy calculator
@@ -181,8 +188,10 @@ bool plan_ring(const far_ctx* ctx, int packs, int64_t rows, int dtype, int segs,
                far::Launch* l) {
   if (packs <= 32) return false;
   const int seg = packs * 16;
+  const bool small_rows = packs <= 256;  // H <= 2048
+  const int max_cons = !ctx->ring_threads_set && small_rows ? 128 : ctx->ring_threads;
   int vpt = 1;
-  while (vpt < 8 && (packs + vpt - 1) / vpt > ctx->ring_threads) vpt *= 2;
+  while (vpt < 8 && (packs + vpt - 1) / vpt > max_cons) vpt *= 2;
   if (!ctx->ring_threads_set && segs <= 6 && packs >= 512 && packs < 1024 && vpt < 4) vpt = 4;
   const int tpr = (((packs + vpt - 1) / vpt) + 31) / 32 * 32;
   if (tpr > far::kRingMaxConsumers) return false;
@@ -190,10 +199,18 @@ bool plan_ring(const far_ctx* ctx, int packs, int64_t rows, int dtype, int segs,
   int n_req = segs <= 6 ? 3 : 2;
   bool gamma_smem = true;
   int target = 72 * 1024;  // slot bytes per CTA
-  if (norm && segs <= 6 && seg >= 16 * 1024) {
+  if (vpt >= 8) {
+    // 8 packs per thread: the registers allow one CTA per SM
+    n_req = 1;
+    target = 6 * seg;
+  } else if (small_rows) {
+    n_req = 4;
+  } else if (norm && segs <= 6 && seg >= 16 * 1024) {
     n_req = 2;
     gamma_smem = false;
     target = 96 * 1024;
+  } else if (norm && segs <= 6 && seg >= 10 * 1024 && seg <= 12 * 1024) {
+    n_req = 2;
   }
   if (ctx->ring_ctas_per_sm > 0) n_req = ctx->ring_ctas_per_sm;
   if (ctx->ring_gamma_mode >= 0) gamma_smem = ctx->ring_gamma_mode != 0;

@@ -370,11 +370,15 @@ def test_launch_plan(ctx):
     # H=4096 with few segments: 4 packs per thread (128 consumers)
     h4 = d(16384, 4096, 4)
     assert (h4["packs_per_thread"], h4["threads_per_cta"]) == (4, 160)
-    # fewer than 3 slots would fit: the share of 2 CTAs per SM, gamma through
-    # L1 (at 8 packs per thread the registers then allow one CTA per SM)
+    # 8 packs per thread: one CTA per SM (all its registers allow), 6 slots
     h16 = d(8192, 16384, 2)
-    assert (h16["kernel"], h16["ring_gamma_smem"], h16["ring_slots"]) == (1, 0, 3)
-    assert h16["grid_ctas"] in (sms, 2 * sms)
+    assert (h16["kernel"], h16["grid_ctas"], h16["ring_gamma_smem"], h16["ring_slots"]) == (1, sms, 1, 6)
+    # rows of at most 256 packs: 128 consumers, 4 CTAs per SM
+    h2 = d(32768, 2048, 4)
+    assert (h2["threads_per_cta"], h2["packs_per_thread"], h2["grid_ctas"]) == (160, 2, 4 * sms)
+    # norm_out with 10-12 KiB segments: 2 CTAs per SM, gamma in shared memory
+    h6 = d(8192, 6144, 4, norm=True)
+    assert (h6["grid_ctas"], h6["ring_gamma_smem"]) == (2 * sms, 1)
     tiny = d(8, 64, 2)
     assert tiny["regime"] == far.FAR_REGIME_PREFILL and tiny["rows_per_cta"] > 1
 
