@@ -169,16 +169,17 @@ int ring_occ_cached(const far_ctx* ctx, int dtype, int vpt, int minb, int thread
 //    per CTA (as many as fit a 1/(CTAs per SM) share of the SM's 228 KiB,
 //    less the 1 KiB the system keeps per CTA);
 //  * except: rows of at most 256 packs (H <= 2048), 4 CTAs per SM (W=2..8:
-//    77-99 vs 63-80 %); 8 packs per thread (H >= 12288), one CTA per SM
-//    (all its registers allow) with 6 slots (H=16384, W=4: 82 / 90 vs 75 /
-//    82 % without / with norm_out); norm_out written and at most 6 segments
+//    77-99 vs 63-80 %); 8 packs per thread (H >= 12288), 2 CTAs per SM
+//    with the register budget of two (H=12288, W=2..8: 80-93 vs 58-84 % at
+//    one CTA), but one CTA per SM with 6 slots when the row has more than 6
+//    segments and fewer than 3 slots fit the 2-CTA share (H=16384, W=8:
+//    92 / 95 vs 89 / 90 % without / with norm_out); norm_out written and at most 6 segments
 //    of at least 16 KiB, 2 CTAs per SM, gamma read through L1 and about
 //    96 KiB of slots (W=3..5, H=8192: 97-102 vs 87-94 %); norm_out and at
 //    most 6 segments of 10-12 KiB, 2 CTAs per SM (H=5120 / 6144: 95-101 vs
 //    84-87 %);
-//  * and when fewer than 3 slots fit: 2 CTAs per SM with gamma through L1
-//    (H=16384 W=1..3 before the one-CTA rule: 88-92 %, where the
-//    one-CTA-per-row kernel gave 63-73 %).
+//  * and when fewer than 3 slots fit (below 8 packs per thread): 2 CTAs per
+//    SM with gamma through L1.
 // Environment overrides (FAR_RING_CTAS_PER_SM, FAR_RING_THREADS,
 // FAR_RING_SLOTS, FAR_RING_GAMMA_SMEM) replace the rule they name.  A
 // persistent grid of sm_count x (the CTAs per SM the occupancy calculator
@@ -200,9 +201,15 @@ bool plan_ring(const far_ctx* ctx, int packs, int64_t rows, int dtype, int segs,
   bool gamma_smem = true;
   int target = 72 * 1024;  // slot bytes per CTA
   if (vpt >= 8) {
-    // 8 packs per thread: the registers allow one CTA per SM
-    n_req = 1;
-    target = 6 * seg;
+    // 8 packs per thread: 2 CTAs per SM (a build with a few spilled
+    // registers), unless the row has many segments and fewer than 3 slots
+    // would fit: then one CTA per SM, as all its registers allow, 6 slots
+    n_req = 2;
+    if (segs > 6 && ctx->ring_slots_max == 0 &&
+        (228 * 1024 / 2 - 1024 - 1024) / seg - 1 < 3) {
+      n_req = 1;
+      target = 6 * seg;
+    }
   } else if (small_rows) {
     n_req = 4;
   } else if (norm && segs <= 6 && seg >= 16 * 1024) {
@@ -223,7 +230,7 @@ bool plan_ring(const far_ctx* ctx, int packs, int64_t rows, int dtype, int segs,
     return ns;
   };
   int nslot = fit(n_req, gamma_smem, target);
-  if (nslot < 3 && ctx->ring_ctas_per_sm == 0 && ctx->ring_gamma_mode < 0) {
+  if (nslot < 3 && vpt < 8 && ctx->ring_ctas_per_sm == 0 && ctx->ring_gamma_mode < 0) {
     n_req = 2;
     gamma_smem = false;
     target = 96 * 1024;
@@ -232,7 +239,9 @@ bool plan_ring(const far_ctx* ctx, int packs, int64_t rows, int dtype, int segs,
   if (nslot < 2) return false;
   const int gsegs = gamma_smem ? 1 : 0;
   const int smem = far::ring_header_bytes(nslot) + (nslot + gsegs) * seg;
-  const int minb = n_req >= 3 ? 3 : 2;
+  // the register budget the kernel is built for: 3 or 2 CTAs per SM, and at
+  // 8 packs per thread 1 (no spills) or 2 (a few spilled registers)
+  const int minb = vpt >= 8 ? (n_req >= 2 ? 2 : 1) : (n_req >= 3 ? 3 : 2);
   int occ = ring_occ_cached(ctx, dtype, vpt, minb, tpr + 32, smem);
   if (occ < 1) return false;
   if (occ > n_req) occ = n_req;

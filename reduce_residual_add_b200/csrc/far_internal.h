@@ -67,7 +67,7 @@ struct Launch {
   int nslot;            // ring: shared-memory slots of one row segment each
   int smem_bytes;       // ring: dynamic shared memory per CTA
   int pdl;              // launch with programmatic stream serialization
-  int ring_minb;        // ring: CTAs per SM its registers are sized for (2 or 3)
+  int ring_minb;        // ring: CTAs per SM its registers are sized for (2 or 3; 1 or 2 at 8 packs)
   int ring_gamma;       // ring: 1 = gamma staged in shared memory, 0 = read through L1
 };
 

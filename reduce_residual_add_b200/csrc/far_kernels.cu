@@ -683,7 +683,7 @@ far_decode_kernel(const Params p) {
 // device error word and the CTA's abort flag, after which no wait blocks,
 // the producer stops, and thread 0 waits (bounded) for the copies already
 // issued before the CTA exits.
-// MINB: CTAs per SM the register budget is sized for (2 or 3; 1 at VPT 8).
+// MINB: CTAs per SM the register budget is sized for (2 or 3; 1 or 2 at VPT 8).
 template <class DT, int VPT, int MINB, bool GROUP>
 __global__ void __launch_bounds__(kRingMaxConsumers + 32, MINB)
 far_ring_kernel(const Params p, int nslot, int ncons, int stage_gamma) {
@@ -878,7 +878,8 @@ cudaError_t launch_ring_g(const Params& p, const Launch& l, cudaStream_t s) {
     case 1: return three ? launch_ring_t<DT, 1, 3, GROUP>(p, l, s) : launch_ring_t<DT, 1, 2, GROUP>(p, l, s);
     case 2: return three ? launch_ring_t<DT, 2, 3, GROUP>(p, l, s) : launch_ring_t<DT, 2, 2, GROUP>(p, l, s);
     case 4: return three ? launch_ring_t<DT, 4, 3, GROUP>(p, l, s) : launch_ring_t<DT, 4, 2, GROUP>(p, l, s);
-    case 8: return launch_ring_t<DT, 8, 1, GROUP>(p, l, s);
+    case 8: return l.ring_minb >= 2 ? launch_ring_t<DT, 8, 2, GROUP>(p, l, s)
+                                    : launch_ring_t<DT, 8, 1, GROUP>(p, l, s);
     default: return cudaErrorInvalidConfiguration;
   }
 }
@@ -930,6 +931,7 @@ cudaError_t allow_large_smem() {
   set(far_ring_kernel<DT, 2, 3, false>);
   set(far_ring_kernel<DT, 4, 3, false>);
   set(far_ring_kernel<DT, 8, 1, false>);
+  set(far_ring_kernel<DT, 8, 2, false>);
   set(far_ring_kernel<DT, 1, 2, true>);
   set(far_ring_kernel<DT, 2, 2, true>);
   set(far_ring_kernel<DT, 4, 2, true>);
@@ -937,6 +939,7 @@ cudaError_t allow_large_smem() {
   set(far_ring_kernel<DT, 2, 3, true>);
   set(far_ring_kernel<DT, 4, 3, true>);
   set(far_ring_kernel<DT, 8, 1, true>);
+  set(far_ring_kernel<DT, 8, 2, true>);
   return e;
 }
 
@@ -987,7 +990,7 @@ int ring_occupancy_dt(int vpt, int minb, int threads, int smem) {
     case 1: return three ? occ_of<DT, 1, 3>(threads, smem) : occ_of<DT, 1, 2>(threads, smem);
     case 2: return three ? occ_of<DT, 2, 3>(threads, smem) : occ_of<DT, 2, 2>(threads, smem);
     case 4: return three ? occ_of<DT, 4, 3>(threads, smem) : occ_of<DT, 4, 2>(threads, smem);
-    case 8: return occ_of<DT, 8, 1>(threads, smem);
+    case 8: return minb >= 2 ? occ_of<DT, 8, 2>(threads, smem) : occ_of<DT, 8, 1>(threads, smem);
     default: return 0;
   }
 }

@@ -370,9 +370,12 @@ def test_launch_plan(ctx):
     # H=4096 with few segments: 4 packs per thread (128 consumers)
     h4 = d(16384, 4096, 4)
     assert (h4["packs_per_thread"], h4["threads_per_cta"]) == (4, 160)
-    # 8 packs per thread: one CTA per SM (all its registers allow), 6 slots
+    # 8 packs per thread: 2 CTAs per SM, gamma in shared memory ...
     h16 = d(8192, 16384, 2)
-    assert (h16["kernel"], h16["grid_ctas"], h16["ring_gamma_smem"], h16["ring_slots"]) == (1, sms, 1, 6)
+    assert (h16["kernel"], h16["grid_ctas"], h16["ring_gamma_smem"], h16["ring_slots"]) == (1, 2 * sms, 1, 2)
+    # ... but one CTA per SM with 6 slots for many segments of which only 2 would fit
+    h16w8 = d(8192, 16384, 8)
+    assert (h16w8["grid_ctas"], h16w8["ring_gamma_smem"], h16w8["ring_slots"]) == (sms, 1, 6)
     # rows of at most 256 packs: 128 consumers, 4 CTAs per SM
     h2 = d(32768, 2048, 4)
     assert (h2["threads_per_cta"], h2["packs_per_thread"], h2["grid_ctas"]) == (160, 2, 4 * sms)
