@@ -155,34 +155,39 @@ void plan_decode(int packs, int cluster_pref, far::Launch* l) {
 // (the occupancy calculator costs microseconds): 0 = cannot run.
 int ring_occ_cached(const far_ctx* ctx, int dtype, int vpt, int minb, int threads, int smem);
 
-// Ring geometry, all measured on B200 (fractions of the measured HBM copy
-// bandwidth; each rule is used only where it was measured to win):
-//  * consumers: the fewest packs per thread (1, 2, 4, 8) that keep within
-//    ring_threads (256), plus one producer warp; except that rows of 512 to
-//    1023 packs with at most 6 segments take 4 packs per thread (H=4096,
-//    W=4: 128-thread CTAs, 97 vs 85 %), and rows of at most 256 packs at
-//    most 128 consumers;
-//  * CTAs per SM: 3 (registers capped at 72) for rows of at most 6
-//    segments (W=4 + residual: 95.5 vs 93.3 % with 2), else 2 (W=8 +
-//    residual: 89.1 vs 87.9 % with 3);
-//  * gamma staged in shared memory, and about 72 KiB of row-segment slots
-//    per CTA (as many as fit a 1/(CTAs per SM) share of the SM's 228 KiB,
-//    less the 1 KiB the system keeps per CTA);
-//  * except: rows of at most 256 packs (H <= 2048), 4 CTAs per SM (W=2..8:
-//    77-99 vs 63-80 %); 8 packs per thread (H >= 12288), 2 CTAs per SM
-//    with the register budget of two (H=12288, W=2..8: 80-93 vs 58-84 % at
-//    one CTA), but one CTA per SM with 6 slots when the row has more than 6
+// Ring geometry.  Every rule was measured on B200 against its alternatives
+// (fractions of the measured HBM copy bandwidth) and is used only where it
+// won.
+//
+// Consumers: the fewest packs per thread (1, 2, 4, 8) that keep within
+// ring_threads (256), plus one producer warp.  Two exceptions:
+//  * rows of 512-1023 packs with at most 6 segments take 4 packs per
+//    thread (H=4096, W=4: 128-thread CTAs, 97 vs 85 %);
+//  * rows of at most 256 packs (H <= 2048) take at most 128 consumers.
+//
+// CTAs per SM, gamma and slots: 3 CTAs per SM (registers capped at 72) for
+// rows of at most 6 segments (W=4 + residual: 95.5 vs 93.3 % with 2), else
+// 2 (W=8 + residual: 89.1 vs 87.9 % with 3); gamma staged in shared memory;
+// about 72 KiB of row-segment slots per CTA, as many as fit a 1/(CTAs per
+// SM) share of the SM's 228 KiB, less the 1 KiB the system keeps per CTA.
+// Exceptions:
+//  * H <= 2048: 4 CTAs per SM (W=2..8: 77-99 vs 63-80 %);
+//  * 8 packs per thread (H >= 12288): 2 CTAs per SM, with the build whose
+//    registers are sized for two (H=12288, W=2..8: 80-93 vs 58-84 % at one
+//    CTA); but one CTA per SM with 6 slots when the row has more than 6
 //    segments and fewer than 3 slots fit the 2-CTA share (H=16384, W=8:
-//    92 / 95 vs 89 / 90 % without / with norm_out); norm_out written and at most 6 segments
-//    of at least 16 KiB, 2 CTAs per SM, gamma read through L1 and about
-//    96 KiB of slots (W=3..5, H=8192: 97-102 vs 87-94 %); norm_out and at
-//    most 6 segments of 10-12 KiB, 2 CTAs per SM (H=5120 / 6144: 95-101 vs
-//    84-87 %);
-//  * and when fewer than 3 slots fit (below 8 packs per thread): 2 CTAs per
-//    SM with gamma through L1.
+//    92 / 95 vs 89 / 90 % without / with norm_out);
+//  * norm_out written, at most 6 segments of at least 16 KiB: 2 CTAs per
+//    SM, gamma read through L1, about 96 KiB of slots (W=3..5, H=8192:
+//    97-102 vs 87-94 %);
+//  * norm_out written, at most 6 segments of 10-12 KiB: 2 CTAs per SM
+//    (H=5120 / 6144: 95-101 vs 84-87 %);
+//  * fewer than 3 slots fit (below 8 packs per thread): 2 CTAs per SM with
+//    gamma through L1.
+//
 // Environment overrides (FAR_RING_CTAS_PER_SM, FAR_RING_THREADS,
-// FAR_RING_SLOTS, FAR_RING_GAMMA_SMEM) replace the rule they name.  A
-// persistent grid of sm_count x (the CTAs per SM the occupancy calculator
+// FAR_RING_SLOTS, FAR_RING_GAMMA_SMEM) replace the rule they name.  The grid
+// is persistent: sm_count x (the CTAs per SM the occupancy calculator
 // confirms), fewer for fewer rows.  Returns false (the direct kernel runs)
 // when fewer than two slots fit or the configuration cannot be resident.
 bool plan_ring(const far_ctx* ctx, int packs, int64_t rows, int dtype, int segs, bool norm,
