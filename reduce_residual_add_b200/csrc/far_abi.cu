@@ -171,7 +171,9 @@ int ring_occ_cached(const far_ctx* ctx, int dtype, int vpt, int minb, int thread
 // about 72 KiB of row-segment slots per CTA, as many as fit a 1/(CTAs per
 // SM) share of the SM's 228 KiB, less the 1 KiB the system keeps per CTA.
 // Exceptions:
-//  * H <= 2048: 4 CTAs per SM (W=2..8: 77-99 vs 63-80 %);
+//  * H <= 2048: 4 CTAs per SM (W=2..8: 77-99 vs 63-80 %); likewise
+//    H <= 5120 with at most 6 segments and no norm_out (W=2 / 4, H=3072,
+//    4096, 5120: 92-97 vs 78-91 %; with norm_out it lost);
 //  * 8 packs per thread (H >= 12288): 2 CTAs per SM, with the build whose
 //    registers are sized for two (H=12288, W=2..8: 80-93 vs 58-84 % at one
 //    CTA); but one CTA per SM with 6 slots when the row has more than 6
@@ -215,7 +217,7 @@ bool plan_ring(const far_ctx* ctx, int packs, int64_t rows, int dtype, int segs,
       n_req = 1;
       target = 6 * seg;
     }
-  } else if (small_rows) {
+  } else if (small_rows || (!norm && segs <= 6 && packs <= 640)) {
     n_req = 4;
   } else if (norm && segs <= 6 && seg >= 16 * 1024) {
     n_req = 2;

@@ -367,9 +367,11 @@ def test_launch_plan(ctx):
     # many segments: 2 CTAs per SM, gamma in shared memory, ~72 KiB of slots
     c5 = d(4096, 7168, 8)
     assert (c5["grid_ctas"], c5["ring_gamma_smem"], c5["ring_slots"]) == (2 * sms, 1, 5)
-    # H=4096 with few segments: 4 packs per thread (128 consumers)
+    # H=4096 with few segments: 4 packs per thread (128 consumers), and
+    # without norm_out 4 CTAs per SM (3 with it)
     h4 = d(16384, 4096, 4)
-    assert (h4["packs_per_thread"], h4["threads_per_cta"]) == (4, 160)
+    assert (h4["packs_per_thread"], h4["threads_per_cta"], h4["grid_ctas"]) == (4, 160, 4 * sms)
+    assert d(16384, 4096, 4, norm=True)["grid_ctas"] == 3 * sms
     # 8 packs per thread: 2 CTAs per SM, gamma in shared memory ...
     h16 = d(8192, 16384, 2)
     assert (h16["kernel"], h16["grid_ctas"], h16["ring_gamma_smem"], h16["ring_slots"]) == (1, 2 * sms, 1, 2)
