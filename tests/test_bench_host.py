@@ -71,3 +71,22 @@ def test_cpu_baseline_on_all_cores_and_single_threaded():
     # per-tensor FP8: one scale over every row, so one thread
     assert bench.oracle_threads(WORKLOADS["c4_prefill_fp8_tensor"], 8192, 64) == 1
     assert bench.oracle_threads(WORKLOADS["c4_prefill_fp8_static"], 5, 64) == 5
+
+
+def test_reference_arm_line():
+    """`bench.py --impl reference` times the oracle on this host and prints
+    one JSON line with the CUDA arm's metric, unit and config object."""
+    import subprocess
+    import sys
+    out = subprocess.run([sys.executable, os.path.join(bench.ROOT, "bench.py"), "--impl", "reference",
+                          "--workload", "c1_small", "--steps", "3", "--warmup", "3"],
+                         capture_output=True, text=True, timeout=300, cwd=bench.ROOT)
+    assert out.returncode == 0, out.stderr[-2000:]
+    line = json.loads(out.stdout.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["metric"] == bench.METRIC
+    assert line["unit"] == "GB/s" and line["higher_is_better"] is True and line["value"] > 0
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["value"] == line["value"]
+    assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["d2h_bytes_per_step"] == 0
+    wl = WORKLOADS["c1_small"]
+    want = bench.workload_config(wl, bench.algorithmic_bytes(wl, wl.T, True), True, None, 1)
+    assert line["config"] == json.loads(json.dumps(want))
