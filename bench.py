@@ -275,6 +275,7 @@ class Case:
         self.sin = (torch.tensor([wl.static_scale], dtype=torch.float32, device=device)
                     if wl.pattern == 1 else None)
         self.bytes = algorithmic_bytes(wl, T, self.nout is not None)
+        self.median_launch = 0.0  # of the last time_steps(per_launch=True)
 
     def prepared(self):
         """The same step as a far.FarCall (arguments marshalled once)."""
@@ -324,7 +325,12 @@ class Case:
         last.record(s)
         torch.cuda.synchronize()
         total = first.elapsed_time(last) / 1e3
-        mean = (sum(a.elapsed_time(b) for a, b in ev) / k / 1e3) if per_launch else total / k
+        if per_launch:
+            times = [a.elapsed_time(b) / 1e3 for a, b in ev]
+            mean = sum(times) / k
+            self.median_launch = statistics.median(times)
+        else:
+            mean = total / k
         return total, mean
 
 
@@ -513,7 +519,8 @@ def run_far(args, world, rank, local):
                      "traffic": profiled_traffic(wl.name),
                      "kernel": ("far_decode_kernel" if launch["regime"] == 1 else
                                 "far_ring_kernel" if launch["kernel"] == 1 else "far_prefill_kernel"),
-                     "mean_launch_us": round(mean_launch * 1e6, 3)},
+                     "mean_launch_us": round(mean_launch * 1e6, 3),
+                     "median_launch_us": round(case.median_launch * 1e6, 3)},
         "e2e": {"value": round(case.bytes / e2e_s / 1e9, 3), "unit": "GB/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "steps": args.e2e_steps, "ms_per_step": round(e2e_s * 1e3, 3), "path": e2e_mode},
@@ -566,9 +573,9 @@ def extras(ctx, device, stream) -> dict:
         row = {}
         for reg, nm in ((far.FAR_REGIME_AUTO, "auto"), (far.FAR_REGIME_DECODE, "cluster_kernel")):
             far.far_set_regime(ctx, reg)
-            total, mean = case.time_steps(500, 50, per_launch=False)
+            total, mean = case.time_steps(1000, 50, per_launch=False)
             row[nm] = {"stream_us_per_call": round(mean * 1e6, 3),
-                       "graph_us_per_call": round(graph_time(case, 100) * 1e6, 3)}
+                       "graph_us_per_call": round(graph_time(case, 200) * 1e6, 3)}
         far.far_set_regime(ctx, far.FAR_REGIME_AUTO)
         call = case.prepared()
         for _ in range(50):
