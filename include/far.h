@@ -127,6 +127,13 @@ typedef enum {
  * therefore start its launch while this one runs, but reads nothing before
  * this one has finished; a preceding kernel that triggers early likewise
  * overlaps its tail with this call's launch. */
+/*
+ * Threads: calls on one context may come from several host threads at once
+ * (its cache of launch shapes and far_fused_host's streams are guarded by
+ * locks); far_set_regime and far_test_stall change the context and must not
+ * run while other calls on it do.  The device error word far_check reads
+ * and clears is one per device, shared by every context on that device.
+ */
 typedef struct far_ctx far_ctx;
 
 /* How one call would be launched (see far_describe_launch). */
