@@ -1001,9 +1001,14 @@ far_status far_fused_host(far_ctx* ctx, const void* const* partials, int W, cons
     if ((e = (call)) != cudaSuccess) return cuda_fail(e, "far_fused_host: " what); \
   } while (0)
 
-  // copies start after the caller's earlier work on `stream`
+  // copies start after the caller's earlier work on `stream`, and the head
+  // (gamma, scale_in) is rewritten only after the kernels of the previous
+  // call on this context, which read it, are done (an event never recorded
+  // makes no one wait)
   FAR_HOST_CK(cudaEventRecord(ctx->host_start, s), "cudaEventRecord");
   FAR_HOST_CK(cudaStreamWaitEvent(in, ctx->host_start, 0), "cudaStreamWaitEvent");
+  FAR_HOST_CK(cudaStreamWaitEvent(in, ctx->host_comp[0], 0), "cudaStreamWaitEvent");
+  FAR_HOST_CK(cudaStreamWaitEvent(in, ctx->host_comp[1], 0), "cudaStreamWaitEvent");
   // gamma and the static scale, once per call
   FAR_HOST_CK(cudaMemcpyAsync(base, gamma, static_cast<size_t>(rb), cudaMemcpyHostToDevice, in),
               "copy of gamma");

@@ -128,6 +128,39 @@ def test_host_calls_back_to_back_share_staging(ctx):
     compare(got_b, run_oracle(b, "bf16", 1e-6, 0.0, 1, scale_in=0.05), "bf16")
 
 
+def test_host_calls_overlap_on_two_streams(ctx):
+    """Two calls with one staging area and context, on two streams, enqueued
+    back to back with no wait between them: the second rewrites gamma and
+    the static scale only after the first call's kernels are done, and each
+    staging buffer only after the first call copied it out."""
+    W, H, R = 2, 2048, 16
+    a = random_inputs(W, 100, H, seed=21)
+    b = random_inputs(W, 37, H, seed=22)
+    b["gamma"] = b["gamma"] * 2          # a late overwrite of gamma would show
+    staging = torch.empty(far.far_host_staging_bytes(W, H, R), dtype=torch.uint8, device="cuda")
+    s1, s2 = torch.cuda.Stream(), torch.cuda.Stream()
+    calls = []
+    for inp, s, scale in ((a, s1, 0.05), (b, s2, 0.1)):
+        T = inp["partials"][0].shape[0]
+        keep = {"ps": [p.pin_memory() for p in inp["partials"]],
+                "res": inp["residual"].pin_memory(),
+                "rout": torch.empty(T, H, dtype=torch.bfloat16).pin_memory(),
+                "nout": torch.empty(T, H, dtype=torch.bfloat16).pin_memory(),
+                "q": torch.empty(T, H, dtype=torch.uint8).pin_memory(),
+                "sin": torch.tensor([scale], dtype=torch.float32)}
+        far.far_fused_host(ctx, keep["ps"], keep["res"], inp["gamma"], 1e-6, 0.0, 1,
+                           staging=staging, chunk_rows=R, residual_out=keep["rout"],
+                           norm_out=keep["nout"], quant_out=keep["q"], scale_in=keep["sin"],
+                           stream=s)
+        calls.append((inp, scale, keep))    # the host tensors live until the end
+    torch.cuda.synchronize()
+    far.far_check(ctx)
+    for inp, scale, keep in calls:
+        got = {"residual_out": as_u16(keep["rout"]), "norm_out": as_u16(keep["nout"]),
+               "quant_out": keep["q"].numpy(), "scale_out": None}
+        compare(got, run_oracle(inp, "bf16", 1e-6, 0.0, 1, scale_in=scale), "bf16")
+
+
 def test_host_pageable_memory(ctx):
     inp = random_inputs(2, 60, 1024, seed=13)
     got = run_host(ctx, inp, 1e-6, 0.0, 2, chunk_rows=16, pin=False)
