@@ -110,12 +110,9 @@ typedef enum {
  * FAR_RING_CTAS_PER_SM=1..4, FAR_RING_THREADS: consumer threads per ring
  * CTA, at most 256, FAR_RING_SLOTS: row-segment slots per ring CTA (2..32),
  * FAR_RING_GAMMA_SMEM=1|0: gamma staged in shared memory or read through
- * L1 (each replaces its part of the measured default rule: 3 CTAs per SM
- * for rows of at most 6 segments, else 2; 256 consumers, 4 packs each for
- * rows of 512-1023 packs with at most 6 segments; gamma in shared memory and
- * about 72 KiB of slots; with norm_out and at most 6 segments of >= 16 KiB,
- * or when fewer than 3 slots would fit: 2 CTAs per SM, gamma through L1,
- * about 96 KiB of slots),
+ * L1 (each replaces its part of the default geometry, which follows rules
+ * measured on B200 by row length, segments per row and whether norm_out is
+ * written: plan_ring in reduce_residual_add_b200/csrc/far_abi.cu),
  * FAR_PDL=1|0: launch with programmatic dependent launch, default 1,
  * FAR_RING_MIN_ROWS: fewest rows for the ring kernel, default by rule,
  * FAR_TENSOR_REVERSE=1|0: the second pass of per-tensor FP8 takes the rows
