@@ -223,3 +223,43 @@ def test_host_staging_bytes():
     assert far.far_host_staging_bytes(17, H, R) == 0
     assert far.far_host_staging_bytes(W, 12, R) == 0
     assert far.far_host_staging_bytes(W, 16392, R) == 0
+
+
+def test_binding_marshals_host_tensors_for_far_fused_host():
+    """The binding's checks for far_fused_host's host tensors (no GPU needed:
+    nothing reaches the library before they pass)."""
+    import torch
+    T, H = 6, 64
+    ps = [torch.zeros(T, H, dtype=torch.bfloat16) for _ in range(3)]
+    res = torch.zeros(T, H, dtype=torch.bfloat16)
+    gam = torch.ones(H, dtype=torch.bfloat16)
+    rout = torch.empty(T, H, dtype=torch.bfloat16)
+    q = torch.empty(T, H, dtype=torch.uint8)
+    sc = torch.empty(T, dtype=torch.float32)
+    out = far._args(ps, res, gam, rout, None, q, None, sc, host=True)
+    arr, W, _, _, _, T2, H2, dt = out[:8]
+    assert (W, T2, H2, dt) == (3, T, H, far.FAR_BF16)
+    assert [arr[i] for i in range(3)] == [p.data_ptr() for p in ps]
+    # a 3-D view is flattened to (rows, H)
+    out3 = far._args([p.view(2, 3, H) for p in ps], res.view(2, 3, H), gam, rout, None, q, None, sc,
+                     host=True)
+    assert out3[5:7] == (T, H)
+    bad = [
+        dict(partials=[ps[0], ps[1][:5]]),                               # shapes differ
+        dict(partials=[ps[0], ps[1].to(torch.float16)]),                 # dtypes differ
+        dict(residual=torch.zeros(T, H, dtype=torch.float16)),          # residual dtype
+        dict(residual_out=torch.empty(T, 2 * H, dtype=torch.bfloat16)[:, :H]),   # strided
+        dict(quant_out=torch.empty(T, H, dtype=torch.int16)),            # 2-byte codes
+        dict(scale_out=torch.empty(T - 1, dtype=torch.float32)),         # too few scales
+        dict(gamma=torch.ones(H, dtype=torch.float16)),                  # gamma dtype
+        dict(partials=[p.t().contiguous().t() for p in ps]),             # not contiguous
+    ]
+    base = dict(partials=ps, residual=res, gamma=gam, residual_out=rout, quant_out=q, scale_out=sc)
+    for change in bad:
+        kw = dict(base, **change)
+        with pytest.raises(ValueError):
+            far._args(kw["partials"], kw["residual"], kw["gamma"], kw["residual_out"], None,
+                      kw["quant_out"], None, kw["scale_out"], host=True)
+    # host and device are not mixed: the device marshalling refuses CPU tensors
+    with pytest.raises(ValueError):
+        far._args(ps, res, gam, rout, None, q, None, sc)
