@@ -85,7 +85,7 @@ REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_c
 
 
 class ClockSampler(threading.Thread):
-    def __init__(self, device: int, period_s: float = 0.01):
+    def __init__(self, device: int, period_s: float = 0.001):
         super().__init__(daemon=True)
         self.period = period_s
         self.samples = []
@@ -358,6 +358,76 @@ def graph_time(case: Case, launches: int, reps: int = 5) -> float:
     return t
 
 
+def touched_bytes(wl: Workload, with_norm: bool) -> int:
+    """Bytes one call reads and writes at its own addresses (gamma aside)."""
+    return algorithmic_bytes(wl, wl.T, with_norm) - wl.H * 2
+
+
+class RotatingSets:
+    """`n` copies of one workload's inputs and outputs at distinct addresses,
+    enough that one pass over them touches more than `min_bytes` (2x L2):
+    a loop over the sets finds none of a set's bytes left in L2 from its
+    previous use, as a decode step whose partials come fresh from a GEMM
+    would.  Gamma is shared (one weight vector).  Every set holds the same
+    seeded values, so any set's outputs are the workload's outputs."""
+
+    def __init__(self, ctx, wl: Workload, inp: dict, device, with_norm: bool, stream,
+                 min_bytes: int = 2 * L2_BYTES):
+        from reduce_residual_add_b200 import far
+        T, H, W = wl.T, wl.H, wl.W
+        with_norm = with_norm or wl.pattern == 0
+        self.n = max(2, -(-min_bytes // touched_bytes(wl, with_norm)))
+        n_in = W + (1 if wl.has_residual else 0)
+        dt = wl.torch_dtype
+        self.inputs = torch.empty(self.n, n_in, T, H, dtype=dt, device=device)
+        src = torch.stack(list(inp["partials"]) + ([inp["residual"]] if wl.has_residual else []))
+        self.inputs.copy_(src.to(device).unsqueeze(0).expand_as(self.inputs))
+        self.rout = torch.empty(self.n, T, H, dtype=dt, device=device)
+        self.nout = torch.empty(self.n, T, H, dtype=dt, device=device) if with_norm else None
+        self.qout = torch.empty(self.n, T, H, dtype=torch.uint8, device=device) if wl.pattern else None
+        self.sout = (torch.empty(self.n, T, dtype=torch.float32, device=device)
+                     if wl.pattern == 2 else None)
+        self.gam = inp["gamma"].to(device)
+        self.sin = (torch.tensor([wl.static_scale], dtype=torch.float32, device=device)
+                    if wl.pattern == 1 else None)
+        self.stream = stream
+        self.calls = []
+        for i in range(self.n):
+            ps = [self.inputs[i, r] for r in range(W)]
+            res = self.inputs[i, W] if wl.has_residual else None
+            self.calls.append(far.FarCall(
+                ctx, ps, res, self.gam, wl.eps, wl.weight_bias, wl.pattern,
+                residual_out=self.rout[i], norm_out=None if self.nout is None else self.nout[i],
+                quant_out=None if self.qout is None else self.qout[i], scale_in=self.sin,
+                scale_out=None if self.sout is None else self.sout[i], stream=stream))
+
+    def graph_time(self, min_launches: int = 200, reps: int = 3) -> float:
+        """Mean seconds per call in a CUDA graph that cycles through the sets
+        (at least `min_launches` calls and at least one full cycle)."""
+        launches = max(min_launches, self.n)
+        launches = -(-launches // self.n) * self.n
+        s = self.stream
+        for c in self.calls:
+            c()
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=s):
+            for i in range(launches):
+                self.calls[i % self.n]()
+        with torch.cuda.stream(s):
+            g.replay()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(s):
+            a.record(s)
+            for _ in range(reps):
+                g.replay()
+            b.record(s)
+        torch.cuda.synchronize()
+        del g
+        return a.elapsed_time(b) / 1e3 / (reps * launches)
+
+
 def e2e_time(case: Case, inp: dict, steps: int, chunk_rows: int = 0):
     """Through the public API from pinned host memory: every step copies the
     inputs host->device, runs the epilogue and copies the outputs back.
@@ -453,16 +523,17 @@ def l2_note(wl: Workload) -> str:
             "latency-bound case" % (read // 2 ** 20))
 
 
-def workload_config(wl: Workload, bytes_per_step: int, with_norm: bool, launch: dict,
-                    world: int) -> dict:
-    """The bench line's `config` object for one workload."""
+def workload_config(wl: Workload, bytes_per_step: int, with_norm: bool, world: int) -> dict:
+    """The bench line's `config` object for one workload (the same object in
+    the CUDA arm and the reference arm; the launch geometry is reported
+    under `roofline`)."""
     cfg = {"workload": wl.name, "W": wl.W, "T": wl.T, "H": wl.H, "dtype": wl.dtype,
            "arithmetic": "fp32 accumulation; bf16/fp16 in and out; e4m3 codes",
            "pattern": PATTERN_NAMES[wl.pattern], "norm_out": with_norm, "eps": wl.eps,
            "weight_bias": wl.weight_bias, "static_scale": wl.static_scale,
            "bytes_per_step": bytes_per_step, "rows_per_rank": wl.T,
            "l2": l2_note(wl),
-           "launch": launch, "parallelism": "rows sharded across %d rank(s), no collective" % world}
+           "parallelism": "rows sharded across %d rank(s), no collective" % world}
     if wl.pattern == 4:
         cfg["group_size"] = wl.group_size
     return cfg
@@ -499,7 +570,10 @@ def run_far(args, world, rank, local):
 
     value = bytes_all / total_max / 1e9
     peak, peak_kind = hbm_peak()
-    achieved = case.bytes / mean_launch / 1e9
+    # the roofline takes the median launch (robust to the odd launch that
+    # waits on something else); the mean is reported beside it
+    achieved = case.bytes / case.median_launch / 1e9
+    achieved_mean = case.bytes / mean_launch / 1e9
     e2e_s, h2d, d2h, e2e_mode = e2e_time(case, inp, args.e2e_steps, args.e2e_chunk_rows)
     e2e_s = max_over_ranks(e2e_s, world)
 
@@ -509,7 +583,7 @@ def run_far(args, world, rank, local):
         "ms_per_step": round(total_max / args.steps * 1e3, 5),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
         "data": "synthetic",
-        "config": workload_config(wl, case.bytes, case.nout is not None, launch, world),
+        "config": workload_config(wl, case.bytes, case.nout is not None, world),
         "tokens_per_s": round(rows_all / total_max, 1),
         "pct_of_peak": round(100 * value / world / peak, 2),
         "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak,
@@ -519,8 +593,12 @@ def run_far(args, world, rank, local):
                      "traffic": profiled_traffic(wl.name),
                      "kernel": ("far_decode_kernel" if launch["regime"] == 1 else
                                 "far_ring_kernel" if launch["kernel"] == 1 else "far_prefill_kernel"),
+                     "launch_time": "median of %d per-launch CUDA-event intervals" % args.steps,
+                     "median_launch_us": round(case.median_launch * 1e6, 3),
                      "mean_launch_us": round(mean_launch * 1e6, 3),
-                     "median_launch_us": round(case.median_launch * 1e6, 3)},
+                     "achieved_on_mean": round(achieved_mean, 2),
+                     "frac_on_mean": round(achieved_mean / peak, 4),
+                     "launch": launch},
         "e2e": {"value": round(case.bytes / e2e_s / 1e9, 3), "unit": "GB/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "steps": args.e2e_steps, "ms_per_step": round(e2e_s * 1e3, 3), "path": e2e_mode},
@@ -558,7 +636,20 @@ def extras(ctx, device, stream) -> dict:
                      "us_per_call": round(mean * 1e6, 2), "tokens_per_s": round(wl.T / mean, 1),
                      "bytes": case.bytes}
         if name == "c3_3d":
-            out[name]["graph_us_per_call"] = round(graph_time(case, 50) * 1e6, 3)
+            warm = graph_time(case, 50)
+            rot = RotatingSets(ctx, wl, inp, device, with_norm, stream)
+            cold = rot.graph_time()
+            out[name].update({
+                "graph_us_per_call": round(warm * 1e6, 3),
+                "cold_graph_us_per_call": round(cold * 1e6, 3),
+                "cold_GB/s": round(case.bytes / cold / 1e9, 1),
+                "cold_frac": round(case.bytes / cold / 1e9 / peak, 4),
+                "cold_sets": rot.n,
+                "timing": "graph_us_per_call: one input set replayed (L2-resident); "
+                          "cold_*: a CUDA graph cycling through %d input/output sets "
+                          "(%d MiB per cycle, more than 2x L2)"
+                          % (rot.n, rot.n * touched_bytes(wl, True) // 2 ** 20)})
+            del rot
         del case
     # the latency floor of one call: a single row of 64 elements, one partial
     wl = WORKLOADS["c1_small"].with_(name="floor_W1_T1_H64", W=1, T=1)
@@ -571,12 +662,17 @@ def extras(ctx, device, stream) -> dict:
         inp = make_inputs(wl)
         case = Case(ctx, wl, inp, device, False, stream)
         row = {}
-        for reg, nm in ((far.FAR_REGIME_AUTO, "auto"), (far.FAR_REGIME_DECODE, "cluster_kernel")):
+        rot = RotatingSets(ctx, wl, inp, device, False, stream)
+        for reg, nm in ((far.FAR_REGIME_AUTO, "auto"), (far.FAR_REGIME_DECODE, "cluster_kernel"),
+                        (far.FAR_REGIME_PREFILL, "one_cta_per_row")):
             far.far_set_regime(ctx, reg)
-            total, mean = case.time_steps(1000, 50, per_launch=False)
-            row[nm] = {"stream_us_per_call": round(mean * 1e6, 3),
-                       "graph_us_per_call": round(graph_time(case, 200) * 1e6, 3)}
+            row[nm] = {"graph_us_per_call": round(graph_time(case, 200) * 1e6, 3),
+                       "cold_graph_us_per_call": round(rot.graph_time() * 1e6, 3)}
         far.far_set_regime(ctx, far.FAR_REGIME_AUTO)
+        row["auto"]["launch"] = far.far_describe_launch(ctx, T, wl.H, wl.torch_dtype, wl.W, True,
+                                                        True)
+        row["cold_sets"] = rot.n
+        del rot
         call = case.prepared()
         for _ in range(50):
             call()
@@ -590,6 +686,11 @@ def extras(ctx, device, stream) -> dict:
         row["auto"]["prepared_stream_us_per_call"] = round(a.elapsed_time(b) / 500 * 1e3, 3)
         far.far_set_regime(ctx, far.FAR_REGIME_AUTO)
         row["tokens_per_s_graph"] = round(T / (row["auto"]["graph_us_per_call"] * 1e-6), 1)
+        row["tokens_per_s_cold_graph"] = round(T / (row["auto"]["cold_graph_us_per_call"] * 1e-6), 1)
+        row["timing"] = ("graph_us_per_call: one input set replayed (L2-resident); "
+                         "cold_graph_us_per_call: a CUDA graph cycling through %d sets "
+                         "(more than 2x L2 per cycle); prepared_stream_us_per_call: one "
+                         "far.FarCall per call in a stream (host-bound)" % row["cold_sets"])
         row["bytes"] = case.bytes
         out[wl.name] = row
         del case
@@ -627,8 +728,7 @@ def run_reference(args, world, rank):
             "ms_per_step": round(tot_t / args.steps * 1e3, 4), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             # the same workload object as the CUDA arm's line (no kernel launch here)
-            "config": workload_config(wl, algorithmic_bytes(wl, wl.T, with_norm), with_norm, None,
-                                      world),
+            "config": workload_config(wl, algorithmic_bytes(wl, wl.T, with_norm), with_norm, world),
             "tokens_per_s": round(rows * args.steps / tot_t, 3),
             "cpu_baseline": {"value": round(value, 5), "unit": "GB/s", "cores": used,
                              "kind": "oracle", "sample": sample},

@@ -29,6 +29,16 @@ def test_algorithmic_bytes_of_the_workloads():
         assert bench.algorithmic_bytes(wl, T, True) == b
 
 
+def test_touched_bytes_and_rotation_size():
+    # a rotation cycle must touch more than 2x L2 for the cold timings
+    for name in ("c2_decode_T1", "c2_decode_T80", "c3_3d"):
+        wl = WORKLOADS[name]
+        per = bench.touched_bytes(wl, True)
+        n = max(2, -(-2 * bench.L2_BYTES // per))
+        assert n * per >= 2 * bench.L2_BYTES
+    assert bench.touched_bytes(WORKLOADS["c3_3d"], True) == 20_975_616 - 2048 * 2
+
+
 def test_clock_sampler_starts_and_stops_without_a_gpu():
     s = bench.ClockSampler(0, period_s=0.001)
     s.start()
@@ -56,7 +66,8 @@ def test_peak_and_traffic_lookup():
 
 def test_workload_config_for_every_workload():
     for name, wl in WORKLOADS.items():
-        cfg = bench.workload_config(wl, bench.algorithmic_bytes(wl, wl.T, False), False, {}, 1)
+        cfg = bench.workload_config(wl, bench.algorithmic_bytes(wl, wl.T, False), False, 1)
+        assert "launch" not in cfg
         assert cfg["workload"] == name and cfg["pattern"] in bench.PATTERN_NAMES.values()
         json.dumps(cfg)
 
@@ -88,5 +99,5 @@ def test_reference_arm_line():
     assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["value"] == line["value"]
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["d2h_bytes_per_step"] == 0
     wl = WORKLOADS["c1_small"]
-    want = bench.workload_config(wl, bench.algorithmic_bytes(wl, wl.T, True), True, None, 1)
+    want = bench.workload_config(wl, bench.algorithmic_bytes(wl, wl.T, True), True, 1)
     assert line["config"] == json.loads(json.dumps(want))
