@@ -488,11 +488,39 @@ def e2e_time(case: Case, inp: dict, steps: int, chunk_rows: int = 0):
     return a.elapsed_time(b) / 1e3 / steps, h2d, d2h, mode
 
 
+def code_tokens(src: str) -> str:
+    """C/C++ source without its comments, whitespace runs collapsed: what the
+    compiler sees, so that editing a comment keeps a measurement valid."""
+    import re
+    out, i, n = [], 0, len(src)
+    while i < n:
+        c = src[i]
+        if c in "\"'":                      # string or character literal
+            j = i + 1
+            while j < n and src[j] != c:
+                j += 2 if src[j] == "\\" else 1
+            out.append(src[i:j + 1])
+            i = j + 1
+        elif src.startswith("//", i):
+            j = src.find("\n", i)
+            i = n if j < 0 else j
+        elif src.startswith("/*", i):
+            j = src.find("*/", i + 2)
+            out.append(" ")
+            i = n if j < 0 else j + 2
+        else:
+            out.append(c)
+            i += 1
+    return re.sub(r"\s+", " ", "".join(out)).strip()
+
+
 def kernel_source_hash() -> str:
+    """sha256 of the kernels' code (far_kernels.cu and far_internal.h without
+    comments); the committed DRAM traffic is valid only for this hash."""
     h = hashlib.sha256()
     for f in ("far_kernels.cu", "far_internal.h"):
-        with open(os.path.join(ROOT, "reduce_residual_add_b200", "csrc", f), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(ROOT, "reduce_residual_add_b200", "csrc", f)) as fh:
+            h.update(code_tokens(fh.read()).encode())
     return h.hexdigest()
 
 
@@ -697,6 +725,86 @@ def extras(ctx, device, stream) -> dict:
     return out
 
 
+def run_sp(args, world, rank, local):
+    """Sequence-parallel tensor parallelism across the ranks (one per GPU):
+    the batch's W = world partials are the ranks' own row-parallel outputs,
+    each rank owns T / world rows of the residual; one step is the row
+    exchange, the fused epilogue on the local rows (W = world partials) and
+    the all-gather of the normed outputs (reduce_residual_add_b200.sp)."""
+    from reduce_residual_add_b200 import build as fbuild
+    from reduce_residual_add_b200 import far, sp
+    import torch.distributed as dist
+    fbuild.build()
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    base = WORKLOADS[args.workload]
+    if base.pattern not in (0, 1, 2):
+        raise SystemExit("--sp takes the norm, static FP8 and per-token FP8 workloads")
+    wl = base.with_(W=world, T=args.rows or base.T)
+    if not sp.is_applicable(wl.T, world):
+        raise SystemExit("%d rows do not split over %d ranks" % (wl.T, world))
+    inp = make_inputs(wl)                       # the same draw on every rank
+    b, e = sp.rows_for_rank(wl.T, world, rank)
+    part = inp["partials"][rank].to(device)
+    res_rows = inp["residual"][b:e].to(device) if wl.has_residual else None
+    gam = inp["gamma"].to(device)
+    rout = torch.empty(e - b, wl.H, dtype=wl.torch_dtype, device=device)
+    sin = (torch.tensor([wl.static_scale], dtype=torch.float32, device=device)
+           if wl.pattern == 1 else None)
+    del inp
+    ctx = far.FarContext(local)
+    group = dist.group.WORLD if world > 1 else None
+    if world == 1:
+        import datetime
+        dist.init_process_group("nccl", rank=0, world_size=1, init_method="tcp://127.0.0.1:%d"
+                                % _free_port(), timeout=datetime.timedelta(seconds=120),
+                                device_id=device)
+        group = dist.group.WORLD
+    step = sp.SequenceParallelEpilogue(group, wl.T, wl.H, wl.torch_dtype, wl.pattern, device,
+                                       with_norm=args.with_norm, ctx=ctx)
+    s = torch.cuda.current_stream()
+
+    def one():
+        step(part, res_rows, gam, wl.eps, wl.weight_bias, residual_out=rout, scale_in=sin)
+
+    for _ in range(args.warmup):
+        one()
+    dist.barrier()
+    torch.cuda.synchronize()
+    a, z = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(s)
+    for _ in range(args.steps):
+        one()
+    z.record(s)
+    torch.cuda.synchronize()
+    dist.barrier()
+    t = max_over_ranks(a.elapsed_time(z) / 1e3, world)
+    nbytes = algorithmic_bytes(wl, wl.T, step.with_norm)
+    line = {"metric": METRIC, "value": round(nbytes * args.steps / t / 1e9, 2), "unit": "GB/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(t / args.steps * 1e3, 5), "higher_is_better": True,
+            "scaling": "strong", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": dict(workload_config(wl, nbytes, step.with_norm, world),
+                           parallelism="sequence parallel over %d rank(s): row exchange "
+                                       "(all_to_all_single), fused epilogue on T/%d rows with "
+                                       "W=%d partials, all-gather of the normed outputs"
+                                       % (world, world, world)),
+            "tokens_per_s": round(wl.T * args.steps / t, 1),
+            "gpu_launches": args.steps}
+    ctx.close()
+    del step
+    dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def _free_port() -> int:
+    import socket
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        return sk.getsockname()[1]
+
+
 def run_reference(args, world, rank):
     """The CPU oracle, timed on this host's cores, on the same workload."""
     if rank != 0:
@@ -752,6 +860,9 @@ def main():
     ap.add_argument("--e2e-chunk-rows", type=int, default=0,
                     help="rows per chunk of far_fused_host in the e2e leg (0: the library default)")
     ap.add_argument("--no-extras", action="store_true")
+    ap.add_argument("--sp", action="store_true",
+                    help="sequence-parallel step across the ranks: each rank holds one of "
+                         "W = N partials and T/N rows of the residual")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:
@@ -762,6 +873,9 @@ def main():
         run_reference(args, world, rank)
         return
     world, rank, local = dist_setup(args.gpus)
+    if args.sp:
+        run_sp(args, world, rank, local)
+        return
     try:
         run_far(args, world, rank, local)
     finally:

@@ -101,3 +101,14 @@ def test_reference_arm_line():
     wl = WORKLOADS["c1_small"]
     want = bench.workload_config(wl, bench.algorithmic_bytes(wl, wl.T, True), True, 1)
     assert line["config"] == json.loads(json.dumps(want))
+
+
+def test_kernel_hash_ignores_comments_only():
+    a = "int f(int x) { return x + 1; } // one\n/* block */ const char* s = \"// kept\";\n"
+    b = "int f(int x) {\n  return x + 1;  // another comment\n}\nconst char* s = \"// kept\";"
+    c = "int f(int x) { return x + 2; } const char* s = \"// kept\";"
+    d = "int f(int x) { return x + 1; } const char* s = \"// changed\";"
+    assert bench.code_tokens(a) == bench.code_tokens(b)
+    assert bench.code_tokens(a) != bench.code_tokens(c)
+    assert bench.code_tokens(a) != bench.code_tokens(d)
+    assert len(bench.kernel_source_hash()) == 64
