@@ -304,11 +304,15 @@ class Case:
                            norm_out=self.nout, quant_out=self.qout, scale_in=self.sin,
                            scale_out=self.sout, stream=self.stream)
 
-    def time_steps(self, k: int, warmup: int, per_launch: bool = True):
-        """(total seconds for k back-to-back steps, mean per-launch seconds)."""
+    def time_steps(self, k: int, warmup: int, per_launch: bool = True, prepared: bool = False):
+        """(total seconds for k back-to-back steps, mean per-launch seconds).
+        prepared: launch through a far.FarCall (arguments marshalled once), for
+        calls short enough that the binding's per-call marshalling would leave
+        the GPU idle between the events."""
         s = self.stream
+        step = self.prepared() if prepared else self.step
         for _ in range(warmup):
-            self.step()
+            step()
         torch.cuda.synchronize()
         if k == 0:
             return 0.0, 0.0
@@ -319,7 +323,7 @@ class Case:
         for i in range(k):
             if per_launch:
                 ev[i][0].record(s)
-            self.step()
+            step()
             if per_launch:
                 ev[i][1].record(s)
         last.record(s)
@@ -334,8 +338,27 @@ class Case:
         return total, mean
 
 
-def graph_time(case: Case, launches: int, reps: int = 5) -> float:
-    """Mean seconds per launch inside a CUDA graph of `launches` calls."""
+def replay_time(g, s, launches: int, reps: int) -> float:
+    """Seconds per launch of a captured graph of `launches` calls: two
+    untimed replays, then the median of `reps` replays each timed alone."""
+    with torch.cuda.stream(s):          # replay() launches on the current stream
+        g.replay()
+        g.replay()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(reps)]
+    with torch.cuda.stream(s):
+        for a, b in ev:
+            a.record(s)
+            g.replay()
+            b.record(s)
+    torch.cuda.synchronize()
+    return statistics.median(a.elapsed_time(b) for a, b in ev) / 1e3 / launches
+
+
+def graph_time(case: Case, launches: int, reps: int = 7) -> float:
+    """Seconds per launch inside a CUDA graph of `launches` calls on one
+    input set (median replay)."""
     s = case.stream
     g = torch.cuda.CUDAGraph()
     case.step()
@@ -343,17 +366,7 @@ def graph_time(case: Case, launches: int, reps: int = 5) -> float:
     with torch.cuda.graph(g, stream=s):
         for _ in range(launches):
             case.step()
-    with torch.cuda.stream(s):          # replay() launches on the current stream
-        g.replay()
-    torch.cuda.synchronize()
-    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with torch.cuda.stream(s):
-        a.record(s)
-        for _ in range(reps):
-            g.replay()
-        b.record(s)
-    torch.cuda.synchronize()
-    t = a.elapsed_time(b) / 1e3 / (reps * launches)
+    t = replay_time(g, s, launches, reps)
     del g
     return t
 
@@ -401,9 +414,10 @@ class RotatingSets:
                 quant_out=None if self.qout is None else self.qout[i], scale_in=self.sin,
                 scale_out=None if self.sout is None else self.sout[i], stream=stream))
 
-    def graph_time(self, min_launches: int = 200, reps: int = 3) -> float:
-        """Mean seconds per call in a CUDA graph that cycles through the sets
-        (at least `min_launches` calls and at least one full cycle)."""
+    def graph_time(self, min_launches: int = 200, reps: int = 5) -> float:
+        """Seconds per call in a CUDA graph that cycles through the sets (at
+        least `min_launches` calls and at least one full cycle; median
+        replay)."""
         launches = max(min_launches, self.n)
         launches = -(-launches // self.n) * self.n
         s = self.stream
@@ -414,18 +428,9 @@ class RotatingSets:
         with torch.cuda.graph(g, stream=s):
             for i in range(launches):
                 self.calls[i % self.n]()
-        with torch.cuda.stream(s):
-            g.replay()
-        torch.cuda.synchronize()
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        with torch.cuda.stream(s):
-            a.record(s)
-            for _ in range(reps):
-                g.replay()
-            b.record(s)
-        torch.cuda.synchronize()
+        t = replay_time(g, s, launches, reps)
         del g
-        return a.elapsed_time(b) / 1e3 / (reps * launches)
+        return t
 
 
 def e2e_time(case: Case, inp: dict, steps: int, chunk_rows: int = 0):
@@ -655,14 +660,19 @@ def extras(ctx, device, stream) -> dict:
         wl = WORKLOADS[name]
         inp = make_inputs(wl)
         case = Case(ctx, wl, inp, device, with_norm, stream)
-        total, mean = case.time_steps(200, 20, per_launch=True)
+        # a short call is launched through a prepared call: the binding's
+        # marshalling (about 10 us) would otherwise sit between the events
+        short = wl.pattern in (0, 1, 2) and case.bytes < L2_BYTES
+        total, mean = case.time_steps(200, 20, per_launch=True, prepared=short)
         if with_norm:
             name += "+norm_out"
         out[name] = {"GB/s": round(case.bytes / mean / 1e9, 1),
                      "launches_per_call": 2 if wl.pattern == 3 else 1,
                      "frac": round(case.bytes / mean / 1e9 / peak, 4),
                      "us_per_call": round(mean * 1e6, 2), "tokens_per_s": round(wl.T / mean, 1),
-                     "bytes": case.bytes}
+                     "bytes": case.bytes,
+                     "stream_timing": ("far.FarCall per call, per-launch events" if short
+                                       else "far binding per call, per-launch events")}
         if name == "c3_3d":
             warm = graph_time(case, 50)
             rot = RotatingSets(ctx, wl, inp, device, with_norm, stream)
@@ -760,12 +770,20 @@ def run_sp(args, world, rank, local):
                                 % _free_port(), timeout=datetime.timedelta(seconds=120),
                                 device_id=device)
         group = dist.group.WORLD
-    step = sp.SequenceParallelEpilogue(group, wl.T, wl.H, wl.torch_dtype, wl.pattern, device,
-                                       with_norm=args.with_norm, ctx=ctx)
-    s = torch.cuda.current_stream()
+    if args.peer:
+        step = sp.PeerSequenceParallelEpilogue(group, wl.T, wl.H, wl.torch_dtype, wl.pattern,
+                                               device, with_norm=args.with_norm, ctx=ctx)
+        step.partial.copy_(part)        # the row-parallel GEMM would write it there
 
-    def one():
-        step(part, res_rows, gam, wl.eps, wl.weight_bias, residual_out=rout, scale_in=sin)
+        def one():
+            step(res_rows, gam, wl.eps, wl.weight_bias, residual_out=rout, scale_in=sin)
+    else:
+        step = sp.SequenceParallelEpilogue(group, wl.T, wl.H, wl.torch_dtype, wl.pattern, device,
+                                           with_norm=args.with_norm, ctx=ctx)
+
+        def one():
+            step(part, res_rows, gam, wl.eps, wl.weight_bias, residual_out=rout, scale_in=sin)
+    s = torch.cuda.current_stream()
 
     for _ in range(args.warmup):
         one()
@@ -785,10 +803,12 @@ def run_sp(args, world, rank, local):
             "ms_per_step": round(t / args.steps * 1e3, 5), "higher_is_better": True,
             "scaling": "strong", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
             "config": dict(workload_config(wl, nbytes, step.with_norm, world),
-                           parallelism="sequence parallel over %d rank(s): row exchange "
-                                       "(all_to_all_single), fused epilogue on T/%d rows with "
-                                       "W=%d partials, all-gather of the normed outputs"
-                                       % (world, world, world)),
+                           parallelism=("sequence parallel over %d rank(s): %s, fused epilogue "
+                                        "on T/%d rows with W=%d partials, all-gather of the "
+                                        "normed outputs"
+                                        % (world, "the kernel reads the peers' rows directly "
+                                           "(symmetric memory)" if args.peer else
+                                           "row exchange (all_to_all_single)", world, world))),
             "tokens_per_s": round(wl.T * args.steps / t, 1),
             "gpu_launches": args.steps}
     ctx.close()
@@ -860,6 +880,8 @@ def main():
     ap.add_argument("--e2e-chunk-rows", type=int, default=0,
                     help="rows per chunk of far_fused_host in the e2e leg (0: the library default)")
     ap.add_argument("--no-extras", action="store_true")
+    ap.add_argument("--peer", action="store_true",
+                    help="with --sp: the one-shot variant, partials read from the peers' memory")
     ap.add_argument("--sp", action="store_true",
                     help="sequence-parallel step across the ranks: each rank holds one of "
                          "W = N partials and T/N rows of the residual")

@@ -222,10 +222,19 @@ size_t far_fp8_tensor_workspace_bytes(int64_t rows);
  * arguments as far_fused_rows; residual_out, norm_out as there.
  *
  * The scale needs every row before any code, so the call enqueues a memset
- * of the workspace's first word and two kernels: the first reads the inputs
- * and keeps each row's 1/rms and the running amax in `workspace`, the second
- * reads the inputs again and writes every output.  Inputs are therefore read
- * twice.  `workspace`: device memory of at least
+ * of the workspace's first word and two kernels.  The first reads the inputs
+ * and keeps each row's 1/rms and the running amax in `workspace`.  Without
+ * norm_out and with a new residual to write (a residual_out, or a residual
+ * updated in place), the first kernel also writes the new residual and the
+ * second forms o from it -- o = round(y) * rinv * (gamma + weight_bias),
+ * round(y) being the new residual in the 2-byte format -- and writes only
+ * the codes, so the inputs are read once; each code is then within one
+ * step of the code of o formed from y itself, and the scale is the same.
+ * Rows whose sum of squares could hide an element that overflows the format
+ * (and rows with an inf or NaN input) are rebuilt from the inputs by the
+ * second kernel instead.  With norm_out, or with no new residual to write,
+ * the second kernel reads the inputs again and writes every output.
+ * `workspace`: device memory of at least
  * far_fp8_tensor_workspace_bytes(row_end - row_begin) bytes, 256-byte
  * aligned, overlapping no argument; its contents are scratch, and two calls
  * that share a workspace must not overlap on the GPU.
@@ -281,7 +290,10 @@ far_status far_fused_fp8_group(far_ctx *ctx, int64_t row_begin, int64_t row_end,
  * on different streams without ordering between them -- race and give
  * wrong results.  The first call on each device looks up the array's
  * device address (cudaGetSymbolAddress) with that device current; make that
- * first call before any stream capture.
+ * first call before any stream capture.  The address is kept for the life
+ * of the process: no call may follow a cudaDeviceReset (or any other
+ * teardown of the device's primary context) in the same process.  Device
+ * ordinals from 256 up are refused (FAR_ERR_UNSUPPORTED).
  */
 far_status far_fused_fp8_tensor_noalloc(far_ctx *ctx, int64_t row_begin, int64_t row_end,
                                         const void *const *partials, int W,

@@ -601,6 +601,8 @@ cudaError_t launch_rows(far::Params p, int dtype, const far::Launch& whole, int6
       e = far::launch_decode(p, dtype, l, s);
     else if (l.kernel == 1)
       e = far::launch_ring(p, dtype, l, s);
+    else if (l.kernel == 2)
+      e = far::launch_tensor_quant(p, dtype, l, s);
     else
       e = far::launch_prefill(p, dtype, l, s);
   }
@@ -622,8 +624,16 @@ struct DeviceGuard {
 };
 
 // The per-tensor path once its arguments are checked: zero the amax word,
-// pass 1 (rinv of every row, the call's amax), pass 2 (every output).  The
+// pass 1 (rinv of every row, the call's amax), pass 2 (the outputs).  The
 // workspace holds the amax word at byte 0 and rinv[rows] from byte 256.
+//
+// Without norm_out, and with a new residual to write, pass 1 also stores
+// each row's new residual (except in rows that may overflow the format,
+// which it flags) and pass 2 forms the codes from it: the inputs are read
+// once, and pass 2 moves 3 bytes per element.  With norm_out, whose
+// 2-byte result would feel the rounding of y, or with no residual output,
+// pass 2 reads every input again and writes every output, as pass 1's
+// kernel would.
 far_status far_fused_fp8_tensor_launch(far_ctx* ctx, int64_t row_begin, int64_t row_end,
                                        const void* const* partials, int W, const void* residual,
                                        void* residual_out, const void* gamma, int64_t H,
@@ -638,6 +648,8 @@ far_status far_fused_fp8_tensor_launch(far_ctx* ctx, int64_t row_begin, int64_t 
   p.ws_amax = static_cast<unsigned*>(workspace);
   p.ws_rinv = reinterpret_cast<float*>(static_cast<unsigned char*>(workspace) + 256);
   p.ws_row0 = row_begin;
+  const bool from_residual = norm_out == nullptr && p.residual_out != nullptr;
+  p.tensor_stores_residual = from_residual ? 1 : 0;
   DeviceGuard guard(ctx->device);
   if (guard.err != cudaSuccess) return cuda_fail(guard.err, "cudaSetDevice");
   const cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -657,10 +669,18 @@ far_status far_fused_fp8_tensor_launch(far_ctx* ctx, int64_t row_begin, int64_t 
   e = launch_rows(p, dtype, first, row_begin, row_end, s);
   if (e != cudaSuccess) return cuda_fail(e, "kernel launch (per-tensor pass 1)");
   // the second pass takes the rows last row first: the rows the first pass
-  // read last are still in L2 when it starts
+  // wrote last are still in L2 when it starts
   p.pattern = far::kTensorQuant;
   p.reverse = ctx->tensor_reverse;
-  e = launch_rows(p, dtype, whole, row_begin, row_end, s);
+  far::Launch second = whole;
+  if (from_residual) {
+    // one CTA per row (or several short rows), loads straight into registers
+    plan_prefill(static_cast<int>(H / far::kPackElems), far::kMaxThreads, &second);
+    second.kernel = 2;
+    second.grid = (row_end - row_begin + second.rows_per_cta - 1) / second.rows_per_cta;
+    second.pdl = ctx->pdl;
+  }
+  e = launch_rows(p, dtype, second, row_begin, row_end, s);
   if (e != cudaSuccess) return cuda_fail(e, "kernel launch (per-tensor pass 2)");
   return FAR_OK;
 }
@@ -875,7 +895,12 @@ far_status far_fused_fp8_tensor_noalloc(far_ctx* ctx, int64_t row_begin, int64_t
     return FAR_ERR_UNSUPPORTED;
   }
   if (row_end == row_begin) return FAR_OK;
-  if (ctx->device < 0 || ctx->device >= 256) return FAR_ERR_UNSUPPORTED;
+  if (ctx->device < 0 || ctx->device >= 256) {
+    std::snprintf(g_last_error, sizeof(g_last_error),
+                  "far_fused_fp8_tensor_noalloc keeps its scratch address for device "
+                  "ordinals 0-255 only (device %d)", ctx->device);
+    return FAR_ERR_UNSUPPORTED;
+  }
 
   void* scratch = nullptr;
   {

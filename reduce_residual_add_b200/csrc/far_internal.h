@@ -22,7 +22,7 @@ enum Pattern : int {
   kFp8Tensor = 3,       // public value of dynamic per-tensor FP8
   kFp8Group = 4,        // per-group FP8: one scale per group of consecutive elements
   kTensorAmax = 16,     // its first pass: rinv of each row + the call's amax
-  kTensorQuant = 17     // its second pass: every output, from the stored rinv and amax
+  kTensorQuant = 17     // its second pass: the other outputs, from the stored rinv and amax
 };
 
 // Everything one launch needs, passed by value in the kernel's parameter
@@ -52,12 +52,15 @@ struct Params {
   uint64_t wait_limit_ns;       // every bounded wait gives up after this long
   int64_t stall_segment;        // test hook: the ring producer skips this copy (-1: none)
   int reverse;                  // take the rows from row_end - 1 down to row_begin
+  int tensor_stores_residual;   // per-tensor FP8, first pass: store the new residual
+                                // of every row it does not flag for a rebuild
 };
 
 // Geometry of one launch, chosen on the host.
 struct Launch {
   int regime;           // 1 decode (cluster per row), 2 prefill
-  int kernel;           // prefill: 0 direct loads, 1 TMA bulk-copy ring
+  int kernel;           // prefill: 0 direct loads, 1 TMA bulk-copy ring,
+                        // 2 per-tensor FP8 second pass from the stored new residual
   int cluster;          // CTAs per row (decode)
   int vpt;              // 16-byte packs per thread
   int tpr;              // threads per row (prefill) / per CTA (decode)
@@ -76,6 +79,7 @@ struct Launch {
 cudaError_t launch_prefill(const Params& p, int dtype, const Launch& l, cudaStream_t stream);
 cudaError_t launch_decode(const Params& p, int dtype, const Launch& l, cudaStream_t stream);
 cudaError_t launch_ring(const Params& p, int dtype, const Launch& l, cudaStream_t stream);
+cudaError_t launch_tensor_quant(const Params& p, int dtype, const Launch& l, cudaStream_t stream);
 
 // Bytes of the ring kernel's shared memory before its first slot.
 int ring_header_bytes(int nslot);

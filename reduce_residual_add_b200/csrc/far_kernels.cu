@@ -13,14 +13,19 @@
 //
 // The work is HBM-bound (about 8 flops per (W+3)*2 bytes): no tensor cores.
 // A whole row stays in registers between its reduction and its scaling, so
-// every byte crosses HBM once.  Two launch shapes share one row routine:
-//  - prefill: one CTA per row (or 256/tpr rows per CTA when a row has at
-//    most 32 packs), 16-byte vector loads, warp-shuffle + shared-memory
-//    reductions;
-//  - decode: one thread-block cluster per row, each CTA a slice of the
-//    hidden dimension, the row's sum of squares (and amax) combined through
-//    distributed shared memory, so that a handful of rows still spreads
-//    over many SMs.
+// every byte crosses HBM once.  Four kernels, three of which share one row
+// routine (finish_row):
+//  - far_ring_kernel (prefill, many rows): persistent CTAs; one producer
+//    thread streams each row's segments with TMA bulk copies into a ring of
+//    shared-memory slots, the consumer warps fold them into registers;
+//  - far_prefill_kernel (fewer rows): one CTA per row (or 256/tpr rows per
+//    CTA when a row has at most 32 packs), 16-byte vector loads issued
+//    ahead of their use, warp-shuffle + shared-memory reductions;
+//  - far_decode_kernel (a few long rows): one thread-block cluster per row,
+//    each CTA a slice of the hidden dimension, the row's sum of squares
+//    (and amax) combined through distributed shared memory;
+//  - far_tensor_quant_kernel: the second pass of dynamic per-tensor FP8,
+//    codes from the stored new residual (no reduction).
 #include <cooperative_groups.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -58,8 +63,13 @@ __device__ __forceinline__ int64_t call_row(const Params& p, int64_t k) {
 // 16-byte packs of eight 2-byte elements
 // ---------------------------------------------------------------------------
 
+// kOverflowSq: the square of the smallest magnitude that rounds to infinity
+// in the format (bf16: (2 - 2^-8) * 2^127, whose square overflows fp32;
+// fp16: 65520).  A row whose fp32 sum of squares stays below it holds no
+// element whose rounding to the format overflows.
 struct Bf16T {
   static constexpr bool kIsBf16 = true;
+  static constexpr float kOverflowSq = 3.40282347e38f;  // FLT_MAX: y^2 overflows first
   static __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
     __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);  // round to nearest even
     return *reinterpret_cast<uint32_t*>(&h);
@@ -68,6 +78,7 @@ struct Bf16T {
 
 struct Fp16T {
   static constexpr bool kIsBf16 = false;
+  static constexpr float kOverflowSq = 65520.f * 65520.f;  // exact in fp32
   static __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
     __half2 h = __floats2half2_rn(lo, hi);  // round to nearest even
     return *reinterpret_cast<uint32_t*>(&h);
@@ -131,6 +142,28 @@ __device__ __forceinline__ float div_by(float a, float b, float inv_b) {
   const float q0 = a * inv_b;
   const float r = fmaf(-q0, b, a);
   return fmaf(r, inv_b, q0);
+}
+
+// Eight e4m3 codes of o / scale (inv = RN(1/scale); exact: divide exactly,
+// for a reciprocal outside the normal range).  A scale of 0 (a per-token row
+// of zeros, or one with an inf / NaN input) gives zero codes.
+__device__ __forceinline__ uint2 fp8_codes8(const float (&o)[8], float scale, float inv, bool exact) {
+  if (scale == 0.f) return make_uint2(0u, 0u);
+  float q[8];
+  if (exact) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) q[i] = __fdiv_rn(o[i], scale);
+  } else {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) q[i] = div_by(o[i], scale, inv);
+  }
+  return make_uint2(e4m3x4(q[0], q[1], q[2], q[3]), e4m3x4(q[4], q[5], q[6], q[7]));
+}
+
+// True when 1 / scale falls outside the normal range, where the quotient is
+// taken by an exact division instead.
+__device__ __forceinline__ bool needs_exact_div(float scale, float inv) {
+  return !(fabsf(inv) < 3.0e38f && fabsf(scale) > 1.0e-37f);
 }
 
 // ---------------------------------------------------------------------------
@@ -400,14 +433,21 @@ __device__ __forceinline__ uint4 gamma_pack(const Params& p, const uint4* gamma_
 
 // GROUP: this instantiation serves only the per-group pattern (kept apart
 // so that the other patterns' code carries none of its registers).
-template <class DT, int VPT, bool GROUP, class Red>
+// GPRE: gamma's packs were loaded by the caller into gpre[k] (pack
+// j0 + k * jstride); otherwise they come from gamma_smem or through L1.
+template <class DT, int VPT, bool GROUP, bool GPRE, class Red>
 __device__ __forceinline__ void finish_row(const Params& p, int64_t row, bool row_ok, int j0,
                                            int jstride, const bool (&ok)[VPT],
                                            float (&y)[VPT][8], const Red& red,
-                                           const uint4* gamma_smem = nullptr) {
+                                           const uint4* gamma_smem, const uint4 (&gpre)[VPT]) {
+  const auto gamma_k = [&](int k) -> uint4 {
+    if constexpr (GPRE) return gpre[k];
+    else return gamma_pack(p, gamma_smem, j0 + k * jstride);
+  };
   const int64_t rbase = row * static_cast<int64_t>(p.packs);  // first pack of the row
-  // dynamic per-tensor FP8 runs in two passes: the first only records rinv
-  // and the call's amax; the second writes every output
+  // dynamic per-tensor FP8 runs in two passes: the first records rinv and
+  // the call's amax (and, with p.tensor_stores_residual, the new residual);
+  // the second writes the other outputs
   const bool tensor_amax = p.pattern == kTensorAmax;
   const bool tensor_quant = p.pattern == kTensorQuant;
   if (p.residual_out != nullptr && !tensor_amax) {
@@ -447,7 +487,7 @@ __device__ __forceinline__ void finish_row(const Params& p, int64_t row, bool ro
     for (int k = 0; k < VPT; ++k) {
       if (!ok[k]) continue;
       float g[8];
-      pack_plus<DT>(gamma_pack(p, gamma_smem, j0 + k * jstride), p.weight_bias, g);
+      pack_plus<DT>(gamma_k(k), p.weight_bias, g);
       if (fp8_token) {
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
@@ -465,13 +505,26 @@ __device__ __forceinline__ void finish_row(const Params& p, int64_t row, bool ro
   } else if (!tensor_quant) {
     ss = red.sum(sq[0]);
   }
-  // (a row past the end of the call, in a CTA of several rows, reads nothing)
-  const float rinv = tensor_quant ? (row_ok ? p.ws_rinv[row - p.ws_row0] : 0.f)
+  // (a row past the end of the call, in a CTA of several rows, reads nothing;
+  // the stored rinv carries the first pass's row flag in its sign bit)
+  const float rinv = tensor_quant ? (row_ok ? fabsf(p.ws_rinv[row - p.ws_row0]) : 0.f)
                                   : __frsqrt_rn(__fdiv_rn(ss, static_cast<float>(p.H)) + p.eps);
 
   if (tensor_amax) {
+    // A row whose sum of squares reaches the square of the format's overflow
+    // threshold (or is inf / NaN) may hold an element that rounds to
+    // infinity: the second pass must rebuild its y from the inputs, so its
+    // new residual is not stored here and the row is flagged (sign bit of
+    // the stored rinv, which is otherwise +0, positive or +inf).
+    const bool rebuild = !(ss < DT::kOverflowSq);
+    if (p.tensor_stores_residual && !rebuild) {
+#pragma unroll
+      for (int k = 0; k < VPT; ++k)
+        if (ok[k]) static_cast<uint4*>(p.residual_out)[rbase + j0 + k * jstride] = pack8<DT>(y[k]);
+    }
     if (row_ok && red.leader()) {
-      p.ws_rinv[row - p.ws_row0] = rinv;
+      p.ws_rinv[row - p.ws_row0] =
+          __uint_as_float(__float_as_uint(rinv) | (rebuild ? 0x80000000u : 0u));
       // non-negative floats order like their bit patterns; a row whose rinv
       // is 0 or NaN (inf / NaN input) has no finite nonzero o: it adds nothing
       const float a = rinv * gmax;
@@ -494,7 +547,7 @@ __device__ __forceinline__ void finish_row(const Params& p, int64_t row, bool ro
   }
   const float inv = __frcp_rn(scale);
   // outside the reciprocal's normal range, divide exactly (uniform per row)
-  const bool exact = !(fabsf(inv) < 3.0e38f && fabsf(scale) > 1.0e-37f);
+  const bool exact = needs_exact_div(scale, inv);
 
   // a4: o = y * rinv * (gamma + weight_bias); a5: FP8 codes.
 #pragma unroll
@@ -506,26 +559,13 @@ __device__ __forceinline__ void finish_row(const Params& p, int64_t row, bool ro
       for (int i = 0; i < 8; ++i) y[k][i] *= rinv;
     } else {
       float g[8];  // gamma + weight_bias in fp32
-      pack_plus<DT>(gamma_pack(p, gamma_smem, j0 + k * jstride), p.weight_bias, g);
+      pack_plus<DT>(gamma_k(k), p.weight_bias, g);
 #pragma unroll
       for (int i = 0; i < 8; ++i) y[k][i] = (y[k][i] * rinv) * g[i];
     }
     if (p.norm_out != nullptr) static_cast<uint4*>(p.norm_out)[pk] = pack8<DT>(y[k]);
-    if (fp8_static || fp8_token || tensor_quant) {  // (per-group codes: below)
-      uint2 codes = make_uint2(0u, 0u);
-      if (scale != 0.f) {  // a per-token row of zeros keeps scale 0 and codes 0
-        float q[8];
-        if (exact) {
-#pragma unroll
-          for (int i = 0; i < 8; ++i) q[i] = __fdiv_rn(y[k][i], scale);
-        } else {
-#pragma unroll
-          for (int i = 0; i < 8; ++i) q[i] = div_by(y[k][i], scale, inv);
-        }
-        codes = make_uint2(e4m3x4(q[0], q[1], q[2], q[3]), e4m3x4(q[4], q[5], q[6], q[7]));
-      }
-      reinterpret_cast<uint2*>(p.quant_out)[pk] = codes;
-    }
+    if (fp8_static || fp8_token || tensor_quant)  // (per-group codes: below)
+      reinterpret_cast<uint2*>(p.quant_out)[pk] = fp8_codes8(y[k], scale, inv, exact);
   }
 
   // a5d: per-group FP8.  A group is p.group_lanes consecutive packs of the
@@ -548,21 +588,9 @@ __device__ __forceinline__ void finish_row(const Params& p, int64_t row, bool ro
       // group_lanes is a power of two: its group is jpk >> log2(group_lanes)
       if (row_ok && (jpk & (p.group_lanes - 1)) == 0)
         p.scale_out[row * p.groups_per_row + (jpk >> (__ffs(p.group_lanes) - 1))] = sc;
-      uint2 codes = make_uint2(0u, 0u);
-      if (sc != 0.f) {
-        const float inv = __frcp_rn(sc);
-        const bool exact_g = !(inv < 3.0e38f && sc > 1.0e-37f);
-        float q[8];
-        if (exact_g) {
-#pragma unroll
-          for (int i = 0; i < 8; ++i) q[i] = __fdiv_rn(y[k][i], sc);
-        } else {
-#pragma unroll
-          for (int i = 0; i < 8; ++i) q[i] = div_by(y[k][i], sc, inv);
-        }
-        codes = make_uint2(e4m3x4(q[0], q[1], q[2], q[3]), e4m3x4(q[4], q[5], q[6], q[7]));
-      }
-      reinterpret_cast<uint2*>(p.quant_out)[rbase + jpk] = codes;
+      const float inv_g = __frcp_rn(sc);
+      reinterpret_cast<uint2*>(p.quant_out)[rbase + jpk] =
+          fp8_codes8(y[k], sc, inv_g, needs_exact_div(sc, inv_g));
     }
   }
 }
@@ -572,9 +600,25 @@ __device__ __forceinline__ void finish_row(const Params& p, int64_t row, bool ro
 // packs j = j0 + k*jstride, k < VPT, j < jend
 // ---------------------------------------------------------------------------
 
+// Loads are issued ahead of their use so that a short call waits on about
+// one memory round trip per row, not one per batch of partials plus one for
+// the residual and one for gamma: the residual and gamma (read after the
+// reduction) go out with the first batch of partials, and at up to 4 packs
+// per thread each batch is folded in only after the next batch's loads are
+// issued.  kBatch partials per batch keep the loads in flight within the
+// kernels' register budgets.
+template <int VPT>
+struct RowLoads {
+  static constexpr int kBatch = VPT <= 2 ? 4 : (VPT == 4 ? 1 : 4);
+  static constexpr bool kPipelined = VPT <= 4;
+  static constexpr bool kGammaAhead = VPT <= 4;
+};
+
 template <class DT, int VPT, bool GROUP, class Red>
 __device__ __forceinline__ void fused_row(const Params& p, int64_t row, bool row_ok,
                                           int j0, int jstride, int jend, const Red& red) {
+  using L = RowLoads<VPT>;
+  constexpr int B = L::kBatch;
   const int64_t rbase = row * static_cast<int64_t>(p.packs);  // first pack of the row
   float y[VPT][8];
   bool ok[VPT];
@@ -584,12 +628,9 @@ __device__ __forceinline__ void fused_row(const Params& p, int64_t row, bool row
 #pragma unroll
     for (int i = 0; i < 8; ++i) y[k][i] = 0.f;
   }
-
-  // a1: sum the W partials in fp32, four buffers' loads in flight per step.
-  for (int r0 = 0; r0 < p.W; r0 += 4) {
-    uint4 v[4][VPT];
+  const auto load_batch = [&](uint4 (&v)[B][VPT], int r0) {
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
+    for (int c = 0; c < B; ++c) {
 #pragma unroll
       for (int k = 0; k < VPT; ++k) {
         v[c][k] = make_uint4(0u, 0u, 0u, 0u);
@@ -597,25 +638,55 @@ __device__ __forceinline__ void fused_row(const Params& p, int64_t row, bool row
           v[c][k] = ld_once(static_cast<const uint4*>(p.partials[r0 + c]) + rbase + j0 + k * jstride);
       }
     }
+  };
+
+  // a1 (first batch), a2's residual and gamma, all in flight together
+  uint4 cur[B][VPT], res[VPT], gam[VPT];
+  load_batch(cur, 0);
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
+  for (int k = 0; k < VPT; ++k) {
+    res[k] = make_uint4(0u, 0u, 0u, 0u);
+    if (p.residual != nullptr && ok[k])
+      res[k] = ld_once_coherent(static_cast<const uint4*>(p.residual) + rbase + j0 + k * jstride);
+    if constexpr (L::kGammaAhead)
+      gam[k] = ok[k] ? __ldg(static_cast<const uint4*>(p.gamma) + j0 + k * jstride)
+                     : make_uint4(0u, 0u, 0u, 0u);
+  }
+
+  // a1: sum the W partials in fp32 in order 0..W-1
+  for (int r0 = 0; r0 < p.W; r0 += B) {
+    if constexpr (L::kPipelined) {
+      uint4 nxt[B][VPT];
+      const bool more = r0 + B < p.W;
+      if (more) load_batch(nxt, r0 + B);
 #pragma unroll
-      for (int k = 0; k < VPT; ++k) add_pack<DT>(v[c][k], y[k]);
+      for (int c = 0; c < B; ++c) {
+#pragma unroll
+        for (int k = 0; k < VPT; ++k) add_pack<DT>(cur[c][k], y[k]);
+      }
+      if (more) {
+#pragma unroll
+        for (int c = 0; c < B; ++c) {
+#pragma unroll
+          for (int k = 0; k < VPT; ++k) cur[c][k] = nxt[c][k];
+        }
+      }
+    } else {
+      if (r0 > 0) load_batch(cur, r0);
+#pragma unroll
+      for (int c = 0; c < B; ++c) {
+#pragma unroll
+        for (int k = 0; k < VPT; ++k) add_pack<DT>(cur[c][k], y[k]);
+      }
     }
   }
 
-  // a2: add the residual.
+  // a2: add the residual (a zero pack without one: y + 0 = y, y is never -0)
   if (p.residual != nullptr) {
-    uint4 v[VPT];
 #pragma unroll
-    for (int k = 0; k < VPT; ++k) {
-      v[k] = make_uint4(0u, 0u, 0u, 0u);
-      if (ok[k]) v[k] = ld_once_coherent(static_cast<const uint4*>(p.residual) + rbase + j0 + k * jstride);
-    }
-#pragma unroll
-    for (int k = 0; k < VPT; ++k) add_pack<DT>(v[k], y[k]);
+    for (int k = 0; k < VPT; ++k) add_pack<DT>(res[k], y[k]);
   }
-  finish_row<DT, VPT, GROUP>(p, row, row_ok, j0, jstride, ok, y, red);
+  finish_row<DT, VPT, GROUP, L::kGammaAhead>(p, row, row_ok, j0, jstride, ok, y, red, nullptr, gam);
 }
 
 // ---------------------------------------------------------------------------
@@ -624,8 +695,10 @@ __device__ __forceinline__ void fused_row(const Params& p, int64_t row, bool row
 
 // Prefill: blockDim = (tpr, rows_per_cta).  SUB: a row lives inside one warp
 // (tpr <= 32, power of two); otherwise one row per CTA.
+// Registers: at one pack per thread (rows of at most 256 packs, often short
+// calls of many rows) four 256-thread CTAs per SM; otherwise two, one at 8.
 template <class DT, int VPT, bool SUB, bool GROUP>
-__global__ void __launch_bounds__(kMaxThreads, (VPT >= 8 ? 1 : 2))
+__global__ void __launch_bounds__(kMaxThreads, (VPT >= 8 ? 1 : (VPT == 1 ? 4 : 2)))
 far_prefill_kernel(const Params p) {
   pdl_enter();
   const int64_t k = static_cast<int64_t>(blockIdx.x) * blockDim.y + threadIdx.y;
@@ -713,11 +786,7 @@ far_ring_kernel(const Params p, int nslot, int ncons, int stage_gamma) {
     *issued_count = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  // gamma: read once per CTA, kept in shared memory for every row
-  if (stage_gamma)
-    for (int j = threadIdx.x; j < p.packs; j += blockDim.x)
-      gamma_s[j] = __ldg(static_cast<const uint4*>(p.gamma) + j);
-  __syncthreads();
+  __syncthreads();  // the mbarriers are ready: the producer may start at once
 
   if (threadIdx.x >= ncons) {
     // producer warp: one thread issues, the rest of the warp is idle
@@ -760,8 +829,16 @@ far_ring_kernel(const Params p, int nslot, int ncons, int stage_gamma) {
     return;
   }
 
-  // consumers
+  // consumers.  gamma is read once per CTA into shared memory while the
+  // producer issues its first copies; the consumers' barrier orders the
+  // staging before the first row's use of it.
+  if (stage_gamma) {
+    for (int j = threadIdx.x; j < p.packs; j += ncons)
+      gamma_s[j] = __ldg(static_cast<const uint4*>(p.gamma) + j);
+    consumer_bar(ncons);
+  }
   const RingRed red0{&hdr->red[0][0][0], ncons}, red1{&hdr->red[1][0][0], ncons};
+  const uint4 no_gamma[VPT] = {};  // gamma comes from shared memory or L1 here
   const int j0 = threadIdx.x;
   int slot = 0;  // the slot of the next segment and its use count parity
   uint32_t phase = 0;
@@ -791,7 +868,8 @@ far_ring_kernel(const Params p, int nslot, int ncons, int stage_gamma) {
         phase ^= 1u;
       }
     }
-    finish_row<DT, VPT, GROUP>(p, row, true, j0, ncons, ok, y, (i & 1) ? red1 : red0, gamma_s);
+    finish_row<DT, VPT, GROUP, false>(p, row, true, j0, ncons, ok, y, (i & 1) ? red1 : red0,
+                                      gamma_s, no_gamma);
   }
 
   // Only after an abort can copies still be in flight: thread 0 waits for
@@ -805,6 +883,90 @@ far_ring_kernel(const Params p, int nslot, int ncons, int stage_gamma) {
       for (int64_t g = (issued > nslot ? issued - nslot : 0); g < issued; ++g) {
         const int slot = static_cast<int>(g % nslot);
         mbar_wait(&full[slot], static_cast<uint32_t>(g / nslot) & 1u, nullptr, p.wait_limit_ns);
+      }
+    }
+  }
+}
+
+// Second pass of dynamic per-tensor FP8 after a first pass that stored the
+// new residual (no norm_out is written): each row's o is formed from its
+// new residual round(y), read back from residual_out, as
+// o = (round(y) * rinv) * (gamma + weight_bias) with the first pass's rinv,
+// and only the codes are written: 3 bytes per element instead of a second
+// read of every input.  round(y) is y to within half an ulp of the 2-byte
+// format; below the format's normal range it is exact (every fp32 partial
+// sum of 2-byte inputs is a whole multiple of the format's smallest
+// subnormal), so a code differs by at most one step from the code of o
+// formed from y itself.  A row the first pass flagged (sign bit of its
+// stored rinv: an element may round to infinity) has no stored residual:
+// its y is rebuilt from the partials and the residual in the first pass's
+// order (the same bits), and its new residual is written here.
+// blockDim = (tpr, rows_per_cta); rows in grid-stride order.
+// o = (y * rinv) * (gamma + weight_bias) for one pack and its 8 codes.
+template <class DT>
+__device__ __forceinline__ uint2 tensor_codes(const uint4& gam, float wb, float (&y)[8], float rinv,
+                                              float scale, float inv, bool exact) {
+  float g[8];
+  pack_plus<DT>(gam, wb, g);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) y[i] = (y[i] * rinv) * g[i];
+  return fp8_codes8(y, scale, inv, exact);
+}
+
+template <class DT, int VPT>
+__global__ void __launch_bounds__(kMaxThreads)
+far_tensor_quant_kernel(const Params p) {
+  pdl_enter();
+  const int64_t nrows = p.row_end - p.row_begin;
+  float scale = __fdiv_rn(__uint_as_float(*p.ws_amax), 448.f);
+  if (scale != scale) scale = 0.f;
+  if (blockIdx.x == 0 && threadIdx.x == 0 && threadIdx.y == 0) p.scale_out[0] = scale;
+  const float inv = __frcp_rn(scale);
+  const bool exact = needs_exact_div(scale, inv);
+  const int j0 = threadIdx.x, tpr = blockDim.x;
+  const uint4* gamma = static_cast<const uint4*>(p.gamma);
+  const int64_t step = static_cast<int64_t>(gridDim.x) * blockDim.y;
+  for (int64_t k = static_cast<int64_t>(blockIdx.x) * blockDim.y + threadIdx.y; k < nrows; k += step) {
+    const int64_t row = call_row(p, k);
+    const int64_t rbase = row * static_cast<int64_t>(p.packs);
+    const float w = p.ws_rinv[row - p.ws_row0];
+    const bool rebuild = signbit(w);
+    const float rinv = fabsf(w);
+    bool ok[VPT];
+#pragma unroll
+    for (int q = 0; q < VPT; ++q) ok[q] = j0 + q * tpr < p.packs;
+    if (!rebuild) {
+      // every load of the row first (this row's residual_out is only read here)
+      uint4 v[VPT], gv[VPT];
+#pragma unroll
+      for (int q = 0; q < VPT; ++q) {
+        v[q] = make_uint4(0u, 0u, 0u, 0u);
+        gv[q] = make_uint4(0u, 0u, 0u, 0u);
+        if (ok[q]) {
+          v[q] = ld_once(static_cast<const uint4*>(p.residual_out) + rbase + j0 + q * tpr);
+          gv[q] = __ldg(gamma + j0 + q * tpr);
+        }
+      }
+#pragma unroll
+      for (int q = 0; q < VPT; ++q) {
+        if (!ok[q]) continue;
+        float y[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        add_pack<DT>(v[q], y);  // 0 + x: the 2-byte value widened exactly
+        reinterpret_cast<uint2*>(p.quant_out)[rbase + j0 + q * tpr] =
+            tensor_codes<DT>(gv[q], p.weight_bias, y, rinv, scale, inv, exact);
+      }
+    } else {
+      // the first pass's order: partials 0..W-1, then the residual
+      for (int q = 0; q < VPT; ++q) {
+        if (!ok[q]) continue;
+        const int64_t pk = rbase + j0 + q * tpr;
+        float y[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        for (int r = 0; r < p.W; ++r) add_pack<DT>(ld_once(static_cast<const uint4*>(p.partials[r]) + pk), y);
+        if (p.residual != nullptr)
+          add_pack<DT>(ld_once_coherent(static_cast<const uint4*>(p.residual) + pk), y);
+        static_cast<uint4*>(p.residual_out)[pk] = pack8<DT>(y);
+        reinterpret_cast<uint2*>(p.quant_out)[pk] =
+            tensor_codes<DT>(__ldg(gamma + j0 + q * tpr), p.weight_bias, y, rinv, scale, inv, exact);
       }
     }
   }
@@ -906,6 +1068,30 @@ cudaError_t launch_prefill_dt(const Params& p, const Launch& l, cudaStream_t s) 
   return p.pattern == kFp8Group ? launch_prefill_g<DT, true>(p, l, s) : launch_prefill_g<DT, false>(p, l, s);
 }
 
+template <class DT, int VPT>
+cudaError_t launch_tensor_quant_t(const Params& p, const Launch& l, cudaStream_t s) {
+  Attrs at(l, 0);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(l.grid), 1, 1);
+  cfg.blockDim = dim3(static_cast<unsigned>(l.tpr), static_cast<unsigned>(l.rows_per_cta), 1);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = s;
+  cfg.attrs = at.a;
+  cfg.numAttrs = at.n;
+  return cudaLaunchKernelEx(&cfg, far_tensor_quant_kernel<DT, VPT>, p);
+}
+
+template <class DT>
+cudaError_t launch_tensor_quant_dt(const Params& p, const Launch& l, cudaStream_t s) {
+  switch (l.vpt) {
+    case 1: return launch_tensor_quant_t<DT, 1>(p, l, s);
+    case 2: return launch_tensor_quant_t<DT, 2>(p, l, s);
+    case 4: return launch_tensor_quant_t<DT, 4>(p, l, s);
+    case 8: return launch_tensor_quant_t<DT, 8>(p, l, s);
+    default: return cudaErrorInvalidConfiguration;
+  }
+}
+
 template <class DT>
 cudaError_t launch_decode_dt(const Params& p, const Launch& l, cudaStream_t s) {
   switch (l.vpt) {
@@ -969,6 +1155,11 @@ cudaError_t launch_decode(const Params& p, int dtype, const Launch& l, cudaStrea
 
 cudaError_t launch_ring(const Params& p, int dtype, const Launch& l, cudaStream_t s) {
   return dtype == kBf16 ? launch_ring_dt<Bf16T>(p, l, s) : launch_ring_dt<Fp16T>(p, l, s);
+}
+
+cudaError_t launch_tensor_quant(const Params& p, int dtype, const Launch& l, cudaStream_t s) {
+  return dtype == kBf16 ? launch_tensor_quant_dt<Bf16T>(p, l, s)
+                        : launch_tensor_quant_dt<Fp16T>(p, l, s);
 }
 
 int ring_header_bytes(int nslot) { return ring_offset(nslot); }

@@ -311,6 +311,47 @@ def far_fused_rows(ctx: FarContext, row_begin: int, row_end: int,
         raise FarError(st, "far_fused_rows")
 
 
+def far_fused_addrs(ctx: FarContext, partial_addrs: Sequence[int], T: int,
+                    residual: Optional[torch.Tensor], gamma: torch.Tensor, eps: float,
+                    weight_bias: float = 0.0, pattern: int = FAR_AR_RESIDUAL_RMSNORM, *,
+                    residual_out: Optional[torch.Tensor] = None,
+                    norm_out: Optional[torch.Tensor] = None,
+                    quant_out: Optional[torch.Tensor] = None,
+                    scale_in: Optional[torch.Tensor] = None,
+                    scale_out: Optional[torch.Tensor] = None, stream=None) -> None:
+    """far_fused with the W partials given as raw device addresses, each of a
+    contiguous (T, H) tensor of gamma's dtype -- for partials that are not
+    tensors of this process, such as another GPU's buffers mapped into this
+    one's address space.  The library checks alignment and overlap as for
+    far_fused; the caller vouches that each address holds T x H elements."""
+    if len(partial_addrs) == 0:
+        raise ValueError("need at least one partial")
+    H = gamma.numel()
+    dt = _DTYPES.get(gamma.dtype)
+    if dt is None or not gamma.is_cuda or not gamma.is_contiguous():
+        raise ValueError("gamma must be a contiguous CUDA bf16 / fp16 tensor")
+    arr = (ctypes.c_void_p * len(partial_addrs))(*[int(a) for a in partial_addrs])
+    res = _flat(residual, H, "residual")
+    rout = _flat(residual_out, H, "residual_out")
+    nout = _flat(norm_out, H, "norm_out")
+    qout = _flat(quant_out, H, "quant_out")
+    for name, t in (("residual", res), ("residual_out", rout), ("norm_out", nout)):
+        if t is not None and (t.shape != (T, H) or t.dtype != gamma.dtype):
+            raise ValueError("%s must be (%d, %d) %s" % (name, T, H, gamma.dtype))
+    if qout is not None and (qout.shape != (T, H) or qout.element_size() != 1):
+        raise ValueError("quant_out must be (%d, %d) of 1-byte elements" % (T, H))
+    for name, t, n in (("scale_in", scale_in, 1), ("scale_out", scale_out, T)):
+        if t is not None and (not t.is_cuda or t.dtype != torch.float32 or t.numel() < n
+                              or not t.is_contiguous()):
+            raise ValueError("%s must be a contiguous CUDA float32 tensor of >= %d elements"
+                             % (name, n))
+    st = lib().far_fused(ctx.handle, arr, len(partial_addrs), _ptr(res), _ptr(rout), _ptr(gamma),
+                         int(T), H, dt, float(eps), float(weight_bias), int(pattern), _ptr(nout),
+                         _ptr(qout), _ptr(scale_in), _ptr(scale_out), _stream(stream))
+    if st != FAR_OK:
+        raise FarError(st, "far_fused")
+
+
 def far_fused(ctx: FarContext, partials: Sequence[torch.Tensor],
               residual: Optional[torch.Tensor], gamma: torch.Tensor, eps: float,
               weight_bias: float = 0.0, pattern: int = FAR_AR_RESIDUAL_RMSNORM, *,

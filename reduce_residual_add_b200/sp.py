@@ -30,6 +30,12 @@ view of its storage, so the same code runs over NCCL on GPUs and over gloo
 (``far.far_fused``); a caller may pass another callable with its signature.
 Per-tensor FP8 is not offered here: its one scale would need a reduction
 across ranks between the two passes.
+
+``PeerSequenceParallelEpilogue`` is the one-shot form of the same step: the
+partials live in symmetric memory that every peer maps, and rank r's kernel
+reads rows [r n, (r + 1) n) of every peer's partial itself over NVLink
+(plain loads and bulk copies without cluster multicast), so step 1's copy
+disappears into the kernel.
 """
 from __future__ import annotations
 
@@ -145,6 +151,91 @@ class SequenceParallelEpilogue:
                                  ("residual_all", new_res if self.gather_residual else None,
                                   self.residual_all)):
             if local is None or full is None:
+                continue
+            dist.all_gather_into_tensor(_words(full), _words(local), group=self.group)
+            out[key] = full
+        return out
+
+
+class PeerSequenceParallelEpilogue:
+    """One-shot variant: the kernel pulls its rows straight from the peers.
+
+    Every rank's partial lives in a buffer of symmetric memory
+    (``self.partial``, (T, H)) that every peer has mapped into its address
+    space (torch.distributed._symmetric_memory, its CUDA backend: peer
+    mappings over NVLink).  Rank r's epilogue kernel gets, as its W = G
+    partials, the addresses of rows [r n, (r + 1) n) in each peer's buffer
+    and reads them over NVLink with the same loads it uses on local memory
+    (plain 16-byte loads, or bulk copies without cluster multicast), so the
+    row exchange of SequenceParallelEpilogue -- a staging copy of (G-1)/G of
+    each partial -- disappears into the kernel.  One call, in stream order:
+
+    1. a one-element all-reduce over the group: it completes on a rank only
+       after every rank has reached it, i.e. after every rank's partial (the
+       work before it in that rank's stream) is complete;
+    2. far_fused on this rank's n rows, partials read from the G peers;
+    3. all-gather of the normed outputs (as SequenceParallelEpilogue).  It
+       completes on a rank only after every rank's step 2 has finished, so
+       no peer is still reading this rank's partial once the next write into
+       ``self.partial`` (after the call, in stream order) begins.
+
+    The caller writes its partial into ``self.partial`` before each call.
+    Results equal SequenceParallelEpilogue's bit for bit (the same kernel on
+    the same values).
+    """
+
+    def __init__(self, group, T: int, H: int, dtype: torch.dtype, pattern: int, device, *,
+                 with_norm: bool = False, ctx=None):
+        import torch.distributed as dist
+        import torch.distributed._symmetric_memory as symm_mem
+        self.dist = dist
+        self.group = group
+        self.G = dist.get_world_size(group)
+        self.rank = dist.get_rank(group)
+        if pattern not in (0, 1, 2):
+            raise ValueError("pattern %d: the sequence-parallel path takes the norm, static "
+                             "FP8 and per-token FP8 patterns" % pattern)
+        self.T, self.H, self.dtype, self.pattern = T, H, dtype, pattern
+        self.b, self.e = rows_for_rank(T, self.G, self.rank)
+        n = self.n = self.e - self.b
+        self.with_norm = with_norm or pattern == 0
+        self.ctx = ctx
+        dev = torch.device(device)
+        self.partial = symm_mem.empty((T, H), dtype=dtype, device=dev)
+        self.handle = symm_mem.rendezvous(self.partial, group)
+        row_bytes = H * self.partial.element_size()
+        # this rank's rows in every peer's partial, peer j's first
+        self.addrs = [int(base) + self.b * row_bytes for base in self.handle.buffer_ptrs]
+        self.ready = torch.zeros(1, dtype=torch.int32, device=dev)
+        self.norm_local = torch.empty(n, H, dtype=dtype, device=dev) if self.with_norm else None
+        self.quant_local = torch.empty(n, H, dtype=torch.uint8, device=dev) if pattern else None
+        self.scale_local = torch.empty(n, dtype=torch.float32, device=dev) if pattern == 2 else None
+        self.norm_all = torch.empty(T, H, dtype=dtype, device=dev) if self.with_norm else None
+        self.quant_all = torch.empty(T, H, dtype=torch.uint8, device=dev) if pattern else None
+        self.scale_all = torch.empty(T, dtype=torch.float32, device=dev) if pattern == 2 else None
+
+    def __call__(self, residual: Optional[torch.Tensor], gamma: torch.Tensor, eps: float,
+                 weight_bias: float = 0.0, *, residual_out: Optional[torch.Tensor] = None,
+                 scale_in: Optional[torch.Tensor] = None) -> dict:
+        """One step on the partial the caller wrote into ``self.partial``;
+        arguments and result as SequenceParallelEpilogue.__call__ (on the
+        current stream)."""
+        from . import far
+        dist = self.dist
+        n, H = self.n, self.H
+        if residual is not None and residual.shape != (n, H):
+            raise ValueError("residual must hold this rank's %d rows" % n)
+        dist.all_reduce(self.ready, group=self.group)
+        far.far_fused_addrs(self.ctx, self.addrs, n, residual, gamma, eps, weight_bias,
+                            self.pattern, residual_out=residual_out, norm_out=self.norm_local,
+                            quant_out=self.quant_local, scale_in=scale_in,
+                            scale_out=self.scale_local)
+        out = {"norm_out": None, "quant_out": None, "scale_out": None,
+               "residual_out": residual_out if residual_out is not None else residual}
+        for key, local, full in (("norm_out", self.norm_local, self.norm_all),
+                                 ("quant_out", self.quant_local, self.quant_all),
+                                 ("scale_out", self.scale_local, self.scale_all)):
+            if local is None:
                 continue
             dist.all_gather_into_tensor(_words(full), _words(local), group=self.group)
             out[key] = full

@@ -6,7 +6,8 @@ Tolerances:
   value (distance on the format's ordered grid, subnormals included; the sign
   of a zero is not compared);
 * e4m3 codes: at most 1 step on the ordered code grid; a code the oracle
-  saturates (+-448) must be saturated on the GPU too; NaN codes must agree;
+  saturates (+-448) must be saturated on the GPU too (except where no code
+  can be clamped, see ``compare``); NaN codes must agree;
 * per-token scales: relative error at most 1e-6 (exact when 0).
 """
 from __future__ import annotations
@@ -147,8 +148,14 @@ def run_oracle(inp: dict, dtype: str, eps, wb, pattern, scale_in=None, rows=None
     return out
 
 
-def compare(gpu: dict, ref: dict, dtype: str, rows=None) -> dict:
-    """Assert the tolerances on the selected rows; return match statistics."""
+def compare(gpu: dict, ref: dict, dtype: str, rows=None, exact_saturation: bool = True) -> dict:
+    """Assert the tolerances on the selected rows; return match statistics.
+
+    ``exact_saturation``: where the oracle's code is +-448 the GPU's must be
+    too.  Per-tensor FP8 whose codes come from the stored new residual passes
+    False: its quotient never exceeds 448 (the scale is amax / 448), so no
+    code is clamped, and a code that rounds up to 448 follows the one-step
+    rule like every other code."""
     sel = slice(None) if rows is None else rows
     stats = {}
     for key in ("residual_out", "norm_out"):
@@ -163,8 +170,9 @@ def compare(gpu: dict, ref: dict, dtype: str, rows=None) -> dict:
         d = code_steps(a, b)
         stats["quant_out"] = (int(d.max()) if d.size else 0, float((d == 0).mean()) if d.size else 1.0)
         assert d.size == 0 or d.max() <= 1, ("quant_out", int(d.max()), np.argwhere(d > 1)[:5].tolist())
-        sat = (b & 0x7F) == 0x7E
-        assert np.array_equal(a[sat], b[sat]), "saturated codes differ"
+        if exact_saturation:
+            sat = (b & 0x7F) == 0x7E
+            assert np.array_equal(a[sat], b[sat]), "saturated codes differ"
     if ref.get("scale_out") is not None:
         a = gpu["scale_out"][sel].astype(np.float64)
         b = ref["scale_out"][sel].astype(np.float64)

@@ -16,7 +16,7 @@ import pytest
 import torch
 
 from gpu_util import compare, run_gpu, run_oracle, to_gpu
-from reduce_residual_add_b200 import far
+from reduce_residual_add_b200 import far, sp
 from reduce_residual_add_b200.inputs import WORKLOADS, make_inputs, random_inputs
 
 pytestmark = pytest.mark.gpu
@@ -57,8 +57,7 @@ def kctx():
     any_rows = {"FAR_RING_MIN_ROWS": "1"}
     out = {"ring": _ctx_with_env(dict(any_rows)),
            "ring256": _ctx_with_env(dict(any_rows, FAR_RING_THREADS="256", FAR_RING_CTAS_PER_SM="1")),
-           "ring3": _ctx_with_env(dict(any_rows, FAR_RING_CTAS_PER_SM="3", FAR_L2_EVICT_FIRST="1",
-                                       FAR_STREAM_STORES="1")),
+           "ring3": _ctx_with_env(dict(any_rows, FAR_RING_CTAS_PER_SM="3")),
            "ring2": _ctx_with_env(dict(any_rows, FAR_RING_CTAS_PER_SM="2", FAR_RING_THREADS="256")),
            # gamma read through L1 instead of staged in shared memory
            "ring_l1": _ctx_with_env(dict(any_rows, FAR_RING_GAMMA_SMEM="0")),
@@ -206,6 +205,36 @@ def test_3d_input_and_row_slices(ctx):
             assert np.array_equal(qout.cpu().numpy(), whole["quant_out"])
         if pattern == 2:
             assert np.array_equal(sout.cpu().numpy(), whole["scale_out"])
+
+
+@pytest.mark.parametrize("G,T,H,pattern", [(2, 1024, 2048, 0), (4, 4096, 8192, 1), (8, 640, 4096, 2)])
+def test_sequence_parallel_local_steps_equal_the_full_call(ctx, G, T, H, pattern):
+    """The kernel side of the sequence-parallel path (reduce_residual_add_b200.sp),
+    each rank's step run in turn on this GPU: rank r's local call gets the
+    G partial blocks of its rows as G separate buffers (what the row exchange
+    delivers) and its rows of the residual; stitched together, the outputs
+    equal the one-call result over all T rows bit for bit."""
+    inp = random_inputs(G, T, H, seed=700 + G)
+    g = to_gpu(inp)
+    scale = 0.05
+    whole = run_gpu(ctx, g, 1e-6, 0.0, pattern, scale_in=scale, want_norm=pattern == 0)
+    n = T // G
+    parts = {k: [] for k in ("residual_out", "norm_out", "quant_out", "scale_out")}
+    for r in range(G):
+        b, e = sp.rows_for_rank(T, G, r)
+        recv = [p_[b:e].clone() for p_ in g["partials"]]     # block j from rank j
+        local = {"partials": recv, "residual": g["residual"][b:e].clone(), "gamma": g["gamma"]}
+        got = run_gpu(ctx, local, 1e-6, 0.0, pattern, scale_in=scale, want_norm=pattern == 0)
+        for k in parts:
+            if got[k] is not None:
+                parts[k].append(got[k])
+    for k, v in parts.items():
+        if whole[k] is None:
+            continue
+        assert np.array_equal(np.concatenate(v), whole[k]), k
+    assert n * G == T
+    compare(whole, run_oracle(inp, "bf16", 1e-6, 0.0, pattern, scale_in=scale,
+                              want_norm=pattern == 0), "bf16")
 
 
 def test_row_slices_leave_other_rows_alone(ctx):
@@ -445,6 +474,7 @@ def test_chained_calls_read_completed_outputs(kctx, ctx, kern):
 # dynamic per-tensor FP8 (two passes, workspace)
 # ---------------------------------------------------------------------------
 
+@pytest.mark.parametrize("norm", [True, False], ids=["norm_out", "codes_from_new_residual"])
 @pytest.mark.parametrize("kern", ["ring", "direct", "auto"])
 @pytest.mark.parametrize("case", [
     (2, 8, 64, "bf16", True, 0.0),
@@ -452,15 +482,67 @@ def test_chained_calls_read_completed_outputs(kctx, ctx, kern):
     (4, 300, 8192, "fp16", True, 1.0),
     (3, 1000, 1000, "bf16", False, 0.0),
     (16, 40, 16384, "bf16", True, 0.0),
+    (2, 77, 8200, "bf16", True, 0.0),      # 1025 packs: 8 per thread, ragged
 ], ids=lambda c: "W%d_T%d_H%d_%s_res%d_wb%g" % c)
-def test_per_tensor_fp8(kctx, ctx, case, kern):
+def test_per_tensor_fp8(kctx, ctx, case, kern, norm):
+    """Without norm_out the second pass forms the codes from the stored new
+    residual (rounded y); with it, from the inputs read again."""
     W, T, H, dt, has_res, wb = case
     c = ctx if kern == "auto" else kctx[kern]
     inp = random_inputs(W, T, H, dtype=dt, seed=500 + W + T + H, has_residual=has_res)
-    got = run_gpu(c, to_gpu(inp), 1e-6, wb, 3, guard=512)
-    ref = run_oracle(inp, dt, 1e-6, wb, 3)
-    log("tensor %s %s" % (kern, case), compare(got, ref, dt))
+    got = run_gpu(c, to_gpu(inp), 1e-6, wb, 3, guard=512, want_norm=norm)
+    ref = run_oracle(inp, dt, 1e-6, wb, 3, want_norm=norm)
+    st = compare(got, ref, dt, exact_saturation=norm)
+    log("tensor %s %s norm=%d" % (kern, case, norm), st)
     assert np.any((got["quant_out"] & 0x7F) == 0x7E)
+    assert got["scale_out"][0] == ref["scale_out"][0]          # the scale is bit-exact
+    assert st["quant_out"][1] > 0.99                            # nearly every code exact
+
+
+@pytest.mark.parametrize("in_place", [False, True])
+def test_per_tensor_fp8_rebuilt_rows(ctx, in_place):
+    """Codes from the stored new residual: rows that may overflow the format
+    (fp16 sums past 65504, whose new residual is +inf) and rows with an inf
+    or NaN input are not stored by the first pass; the second pass rebuilds
+    their y from the inputs, in place too (the residual is still intact)."""
+    T, H = 300, 4096
+    inp = random_inputs(4, T, H, dtype="fp16", seed=93)
+    for p_ in inp["partials"]:
+        p_[::7, :16] = 30000.0
+    inp["partials"][0][5, 9] = float("inf")
+    inp["partials"][1][6, 3] = float("nan")
+    got = run_gpu(ctx, to_gpu(inp), 1e-6, 0.0, 3, want_norm=False, in_place=in_place)
+    ref = run_oracle(inp, "fp16", 1e-6, 0.0, 3, want_norm=False)
+    compare(got, ref, "fp16", exact_saturation=False)
+    assert np.all(got["residual_out"][::7, :16] == 0x7C00)          # +inf
+    assert got["scale_out"][0] == ref["scale_out"][0]
+
+
+def test_per_tensor_fp8_without_residual_output(ctx):
+    """No residual in and no new residual out: nothing to read back, so the
+    second pass reads the inputs again; with a residual_out it reads that."""
+    inp = random_inputs(3, 200, 2048, seed=94, has_residual=False)
+    for want_rout in (False, True):
+        got = run_gpu(ctx, to_gpu(inp), 1e-6, 0.0, 3, want_norm=False,
+                      want_residual_out=want_rout)
+        ref = run_oracle(inp, "bf16", 1e-6, 0.0, 3, want_norm=False,
+                         want_residual_out=want_rout)
+        compare(got, ref, "bf16", exact_saturation=False)
+        assert got["scale_out"][0] == ref["scale_out"][0]
+
+
+def test_per_tensor_fp8_full_size_c4_shape(ctx):
+    """The c4 prefill shape (W=4, 8192 x 8192 bf16, 82 outlier rows x50) with
+    dynamic per-tensor FP8 and no norm_out, as the bench times it: every row
+    against the oracle (the scale spans all rows)."""
+    wl = WORKLOADS["c4_prefill_fp8_tensor"]
+    inp = make_inputs(wl)
+    got = run_gpu(ctx, to_gpu(inp), wl.eps, wl.weight_bias, 3, want_norm=False)
+    ref = run_oracle(inp, "bf16", wl.eps, wl.weight_bias, 3, want_norm=False)
+    st = compare(got, ref, "bf16", exact_saturation=False)
+    log("tensor c4 full", st)
+    assert got["scale_out"][0] == ref["scale_out"][0]
+    assert st["quant_out"][1] > 0.995
 
 
 @pytest.mark.parametrize("case", [
@@ -483,11 +565,14 @@ def test_per_tensor_fp8_row_order(case):
             far.far_set_regime(rev, far.FAR_REGIME_PREFILL)
         inp = random_inputs(W, T, H, seed=900 + T)
         g = to_gpu(inp)
-        a = run_gpu(fwd, g, 1e-6, 0.0, 3, guard=256)
-        b = run_gpu(rev, g, 1e-6, 0.0, 3, guard=256)
-        for k in a:
-            assert np.array_equal(a[k], b[k]), k
-        log("tensor order %s" % (case,), compare(b, run_oracle(inp, "bf16", 1e-6, 0.0, 3), "bf16"))
+        for norm in (True, False):
+            a = run_gpu(fwd, g, 1e-6, 0.0, 3, guard=256, want_norm=norm)
+            b = run_gpu(rev, g, 1e-6, 0.0, 3, guard=256, want_norm=norm)
+            for k in a:
+                assert np.array_equal(a[k], b[k]), k
+            ref = run_oracle(inp, "bf16", 1e-6, 0.0, 3, want_norm=norm)
+            log("tensor order %s norm=%d" % (case, norm),
+                compare(b, ref, "bf16", exact_saturation=norm))
     finally:
         fwd.close()
         rev.close()
@@ -498,10 +583,13 @@ def test_per_tensor_fp8_row_range_and_full_size(ctx):
     wl = WORKLOADS["c5_gemma_fp8_token_bf16"]
     inp = make_inputs(wl)
     g = to_gpu(inp)
-    got = run_gpu(ctx, g, wl.eps, wl.weight_bias, 3, rows=(100, 3000))
-    ref = run_oracle(inp, "bf16", wl.eps, wl.weight_bias, 3, rows=(100, 3000))
-    log("tensor c5 rows", compare(got, ref, "bf16", rows=slice(100, 3000)))
-    assert not got["quant_out"][:100].any() and not got["quant_out"][3000:].any()
+    for norm in (True, False):
+        got = run_gpu(ctx, g, wl.eps, wl.weight_bias, 3, rows=(100, 3000), want_norm=norm)
+        ref = run_oracle(inp, "bf16", wl.eps, wl.weight_bias, 3, rows=(100, 3000), want_norm=norm)
+        log("tensor c5 rows norm=%d" % norm,
+            compare(got, ref, "bf16", rows=slice(100, 3000), exact_saturation=norm))
+        assert not got["quant_out"][:100].any() and not got["quant_out"][3000:].any()
+        assert not got["residual_out"][:100].any() and not got["residual_out"][3000:].any()
     # all rows, in the launch configuration of a full-size call
     got = run_gpu(ctx, g, wl.eps, wl.weight_bias, 3)
     ref = run_oracle(inp, "bf16", wl.eps, wl.weight_bias, 3)

@@ -8,33 +8,36 @@ cudaFree.  This entry point runs the same two-pass per-tensor FP8 epilogue
 as far_fused_fp8_tensor, with the library's own fixed scratch in place of a
 caller workspace.  The test calls it through the C ABI twice in a row -- the
 second call on smaller inputs, so a scratch that still held the first call's
-amax would give the wrong scale -- and checks each result against
-far_fused_fp8_tensor (the entry point with a workspace) within the parity
-tolerances used everywhere else.  It runs alone or after the other tests.
+amax would give the wrong scale -- and checks each result bit for bit against
+far_fused_fp8_tensor (the entry point with a workspace) and against the
+oracle within the parity tolerances used everywhere else, on whole calls and
+on row ranges that start past row 0.  It runs alone or after the other tests.
 """
 from __future__ import annotations
 
 import ctypes
 
+import numpy as np
 import pytest
 import torch
 
-from gpu_util import compare, to_gpu
+from gpu_util import compare, run_oracle, to_gpu
 from reduce_residual_add_b200 import far
 from reduce_residual_add_b200.inputs import as_u16, random_inputs
 
 pytestmark = pytest.mark.gpu
 
 
-def _outputs(T, H, dtype):
-    return {"residual_out": torch.empty(T, H, dtype=dtype, device="cuda"),
-            "norm_out": torch.empty(T, H, dtype=dtype, device="cuda"),
-            "quant_out": torch.empty(T, H, dtype=torch.uint8, device="cuda"),
-            "scale_out": torch.empty(1, dtype=torch.float32, device="cuda")}
+def _outputs(T, H, dtype, with_norm=True):
+    return {"residual_out": torch.zeros(T, H, dtype=dtype, device="cuda"),
+            "norm_out": torch.zeros(T, H, dtype=dtype, device="cuda") if with_norm else None,
+            "quant_out": torch.zeros(T, H, dtype=torch.uint8, device="cuda"),
+            "scale_out": torch.zeros(1, dtype=torch.float32, device="cuda")}
 
 
 def _numpy(o):
-    return {"residual_out": as_u16(o["residual_out"].cpu()), "norm_out": as_u16(o["norm_out"].cpu()),
+    return {"residual_out": as_u16(o["residual_out"].cpu()),
+            "norm_out": None if o["norm_out"] is None else as_u16(o["norm_out"].cpu()),
             "quant_out": o["quant_out"].cpu().numpy(), "scale_out": o["scale_out"].cpu().numpy()}
 
 
@@ -52,27 +55,47 @@ def _c_abi_noalloc(ctx, g, out, eps, wb, rows):
         vp(out["scale_out"]), stream)
 
 
-@pytest.mark.parametrize("W,T,H,dtype", [(4, 3000, 8192, torch.bfloat16), (8, 40, 7168, torch.float16)])
-def test_noalloc_matches_workspace_entry_point_on_two_calls(W, T, H, dtype):
+def _check_call(ctx, inp, dt, dtype, rows, with_norm):
+    """One no-alloc call: against the workspace entry point on the same
+    inputs (bit for bit: the same kernels and plan) and against the oracle
+    (the stated tolerances)."""
+    g = to_gpu(inp)
+    T, H = g["partials"][0].shape
+    mine = _outputs(T, H, dtype, with_norm)
+    st = _c_abi_noalloc(ctx, g, mine, 1e-6, 0.5, rows)
+    assert st == far.FAR_OK, far.far_status_string(st) + " " + far.far_last_error()
+    ref = _outputs(T, H, dtype, with_norm)
+    ws = torch.empty(far.far_fp8_tensor_workspace_bytes(rows[1] - rows[0]), dtype=torch.uint8,
+                     device="cuda")
+    far.far_fused_fp8_tensor(ctx, g["partials"], g["residual"], g["gamma"], 1e-6, 0.5,
+                             quant_out=ref["quant_out"], scale_out=ref["scale_out"],
+                             workspace=ws, residual_out=ref["residual_out"],
+                             norm_out=ref["norm_out"], rows=rows)
+    torch.cuda.synchronize()
+    far.far_check(ctx)
+    a, b = _numpy(mine), _numpy(ref)
+    for k in a:
+        if a[k] is not None:
+            assert np.array_equal(a[k], b[k]), k
+    orc = run_oracle(inp, dt, 1e-6, 0.5, 3, rows=rows, want_norm=with_norm)
+    compare(a, orc, dt, rows=slice(rows[0], rows[1]), exact_saturation=with_norm)
+
+
+@pytest.mark.parametrize("W,T,H,dtype,rows,with_norm", [
+    (4, 3000, 8192, torch.bfloat16, None, True),
+    (8, 40, 7168, torch.float16, None, True),
+    (4, 3000, 8192, torch.bfloat16, (1000, 3000), False),   # a row offset into the scratch
+    (3, 700, 2048, torch.float16, (5, 650), True),
+])
+def test_noalloc_matches_workspace_entry_point_and_oracle_on_two_calls(W, T, H, dtype, rows, with_norm):
     ctx = far.FarContext(0)
     try:
         dt = "bf16" if dtype == torch.bfloat16 else "fp16"
+        rr = (0, T) if rows is None else rows
         for call, sigma in enumerate((1.0, 0.25)):     # the second call has the smaller amax
             inp = random_inputs(W, T, H, dtype=dt, seed=900 + call, partial_sigma=sigma,
                                 residual_sigma=sigma)
-            g = to_gpu(inp)
-            mine = _outputs(T, H, dtype)
-            st = _c_abi_noalloc(ctx, g, mine, 1e-6, 0.5, (0, T))
-            assert st == far.FAR_OK, far.far_status_string(st) + " " + far.far_last_error()
-            ref = _outputs(T, H, dtype)
-            ws = torch.empty(far.far_fp8_tensor_workspace_bytes(T), dtype=torch.uint8, device="cuda")
-            far.far_fused_fp8_tensor(ctx, g["partials"], g["residual"], g["gamma"], 1e-6, 0.5,
-                                     quant_out=ref["quant_out"], scale_out=ref["scale_out"],
-                                     workspace=ws, residual_out=ref["residual_out"],
-                                     norm_out=ref["norm_out"])
-            torch.cuda.synchronize()
-            far.far_check(ctx)
-            compare(_numpy(mine), _numpy(ref), dt)
+            _check_call(ctx, inp, dt, dtype, rr, with_norm)
     finally:
         ctx.close()
 
