@@ -338,13 +338,17 @@ class Case:
         return total, mean
 
 
-def replay_time(g, s, launches: int, reps: int) -> float:
-    """Seconds per launch of a captured graph of `launches` calls: two
-    untimed replays, then the median of `reps` replays each timed alone."""
-    with torch.cuda.stream(s):          # replay() launches on the current stream
-        g.replay()
-        g.replay()
-    torch.cuda.synchronize()
+def replay_time(g, s, launches: int, reps: int, warm_s: float = 0.02) -> float:
+    """Seconds per launch of a captured graph of `launches` calls: untimed
+    replays for at least `warm_s` (clocks ramp up after the host-side set-up
+    left the GPU idle), then the median of `reps` replays each timed alone."""
+    t0 = time.perf_counter()
+    n = 0
+    while n < 2 or time.perf_counter() - t0 < warm_s:
+        with torch.cuda.stream(s):      # replay() launches on the current stream
+            g.replay()
+        torch.cuda.synchronize()
+        n += 1
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
           for _ in range(reps)]
     with torch.cuda.stream(s):
@@ -581,6 +585,9 @@ def run_far(args, world, rank, local):
     wl = WORKLOADS[args.workload]
     if args.rows:
         wl = wl.with_(T=args.rows, outlier_frac=wl.outlier_frac)
+    if args.shape:
+        W, H = (int(x) for x in args.shape.split(","))
+        wl = wl.with_(name="%s_W%d_H%d" % (wl.name, W, H), W=W, H=H)
     # each rank owns an independent batch of rows (seed offset by rank)
     inp = make_inputs(wl.with_(seed=wl.seed + 1000 * rank))
     stream = torch.cuda.Stream(device=device)
@@ -876,6 +883,9 @@ def main():
     ap.add_argument("--with-norm", action="store_true", help="also write norm_out")
     ap.add_argument("--rows", type=int, default=0,
                     help="override the workload's row count (smaller cases for profiling)")
+    ap.add_argument("--shape", default="",
+                    help="W,H: override the workload's partial count and hidden size "
+                         "(other shapes for profiling)")
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--e2e-chunk-rows", type=int, default=0,
                     help="rows per chunk of far_fused_host in the e2e leg (0: the library default)")

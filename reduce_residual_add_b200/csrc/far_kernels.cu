@@ -285,8 +285,9 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
 // Programmatic dependent launch (PTX griddepcontrol): wait until the grid
 // this launch depends on has completed and its writes are visible (a no-op
 // without that dependency), then let the next dependent grid be scheduled.
-// Called first thing in every kernel, so no input is read and no output is
-// written before the preceding work in the stream is done.
+// Called in every kernel before its first access to global memory (only
+// shared-memory set-up may come first), so no input is read and no output
+// is written before the preceding work in the stream is done.
 __device__ __forceinline__ void pdl_enter() {
   asm volatile("griddepcontrol.wait;" ::: "memory");
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
@@ -719,7 +720,8 @@ far_prefill_kernel(const Params p) {
 template <class DT, int VPT>
 __global__ void __launch_bounds__(kMaxThreads, (VPT >= 8 ? 1 : 2))
 far_decode_kernel(const Params p) {
-  pdl_enter();
+  // the shared-memory set-up touches no global memory: it runs before the
+  // wait for the preceding grid, overlapping its tail
   __shared__ float s_sum[32], s_max[32], s_in[32];
   __shared__ uint64_t s_bar;
   cg::cluster_group cl = cg::this_cluster();
@@ -731,6 +733,7 @@ far_decode_kernel(const Params p) {
   }
   __syncthreads();
   asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+  pdl_enter();
   const int64_t row = call_row(p, blockIdx.y);
   const int chunk = (p.packs + ncta - 1) / ncta;
   const int jbeg = rank * chunk;
@@ -760,7 +763,6 @@ far_decode_kernel(const Params p) {
 template <class DT, int VPT, int MINB, bool GROUP>
 __global__ void __launch_bounds__(kRingMaxConsumers + 32, MINB)
 far_ring_kernel(const Params p, int nslot, int ncons, int stage_gamma) {
-  pdl_enter();
   extern __shared__ __align__(128) unsigned char smem[];
   uint64_t* full = reinterpret_cast<uint64_t*>(smem);
   uint64_t* empty = full + nslot;
@@ -787,6 +789,9 @@ far_ring_kernel(const Params p, int nslot, int ncons, int stage_gamma) {
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   __syncthreads();  // the mbarriers are ready: the producer may start at once
+  // everything above touches shared memory only: it runs before the wait for
+  // the preceding grid, overlapping its tail
+  pdl_enter();
 
   if (threadIdx.x >= ncons) {
     // producer warp: one thread issues, the rest of the warp is idle
@@ -853,7 +858,9 @@ far_ring_kernel(const Params p, int nslot, int ncons, int stage_gamma) {
       for (int e = 0; e < 8; ++e) y[k][e] = 0.f;
     }
     for (int k = 0; k < S; ++k) {
-      if (!*abort_flag && !mbar_wait(&full[slot], phase, abort_flag, p.wait_limit_ns)) {
+      // the abort flag is read only when the segment is not there yet
+      if (!mbar_try_wait(&full[slot], phase) && !*abort_flag &&
+          !mbar_wait(&full[slot], phase, abort_flag, p.wait_limit_ns)) {
         if (!*abort_flag) atomicOr(&g_far_error, kErrWaitFull);
         *abort_flag = 1;
       }
@@ -902,12 +909,22 @@ far_ring_kernel(const Params p, int nslot, int ncons, int stage_gamma) {
 // its y is rebuilt from the partials and the residual in the first pass's
 // order (the same bits), and its new residual is written here.
 // blockDim = (tpr, rows_per_cta); rows in grid-stride order.
-// o = (y * rinv) * (gamma + weight_bias) for one pack and its 8 codes.
+// The 8 codes of one pack.  In the usual case (a scale whose reciprocal is
+// normal) the quotient is formed as q = (y * (rinv / scale)) * (gamma + wb),
+// two multiplies per element with rs = RN(rinv * RN(1 / scale)) per row: a
+// few fp32 ulps from o / scale, nothing against the half-ulp of the 2-byte
+// format already in y here and far inside one e4m3 step.  Otherwise o is
+// formed and divided as in every other pattern.
 template <class DT>
 __device__ __forceinline__ uint2 tensor_codes(const uint4& gam, float wb, float (&y)[8], float rinv,
-                                              float scale, float inv, bool exact) {
+                                              float rs, float scale, float inv, bool exact) {
   float g[8];
   pack_plus<DT>(gam, wb, g);
+  if (!exact && scale != 0.f) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) y[i] = (y[i] * rs) * g[i];
+    return make_uint2(e4m3x4(y[0], y[1], y[2], y[3]), e4m3x4(y[4], y[5], y[6], y[7]));
+  }
 #pragma unroll
   for (int i = 0; i < 8; ++i) y[i] = (y[i] * rinv) * g[i];
   return fp8_codes8(y, scale, inv, exact);
@@ -932,6 +949,7 @@ far_tensor_quant_kernel(const Params p) {
     const float w = p.ws_rinv[row - p.ws_row0];
     const bool rebuild = signbit(w);
     const float rinv = fabsf(w);
+    const float rs = rinv * inv;
     bool ok[VPT];
 #pragma unroll
     for (int q = 0; q < VPT; ++q) ok[q] = j0 + q * tpr < p.packs;
@@ -953,7 +971,7 @@ far_tensor_quant_kernel(const Params p) {
         float y[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
         add_pack<DT>(v[q], y);  // 0 + x: the 2-byte value widened exactly
         reinterpret_cast<uint2*>(p.quant_out)[rbase + j0 + q * tpr] =
-            tensor_codes<DT>(gv[q], p.weight_bias, y, rinv, scale, inv, exact);
+            tensor_codes<DT>(gv[q], p.weight_bias, y, rinv, rs, scale, inv, exact);
       }
     } else {
       // the first pass's order: partials 0..W-1, then the residual
@@ -966,7 +984,7 @@ far_tensor_quant_kernel(const Params p) {
           add_pack<DT>(ld_once_coherent(static_cast<const uint4*>(p.residual) + pk), y);
         static_cast<uint4*>(p.residual_out)[pk] = pack8<DT>(y);
         reinterpret_cast<uint2*>(p.quant_out)[pk] =
-            tensor_codes<DT>(__ldg(gamma + j0 + q * tpr), p.weight_bias, y, rinv, scale, inv, exact);
+            tensor_codes<DT>(__ldg(gamma + j0 + q * tpr), p.weight_bias, y, rinv, rs, scale, inv, exact);
       }
     }
   }
