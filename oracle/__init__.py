@@ -10,7 +10,8 @@ numpy arrays of raw 16-bit / 8-bit patterns in and out of it.
 What it computes, per row t (see the header of ``far_oracle.c`` for the
 sources and for the readings taken where the pages are silent):
 
-    y    = sum_r partials[r][t] + residual[t]      (new residual)
+    y    = sum_r partials[r][t] + residual[t]      (new residual; exact, or in
+                                                    fp32 with acc32=True)
     rinv = 1 / sqrt(mean(y^2) + eps)
     o    = y * rinv * (gamma + weight_bias)        (normed output)
     static FP8:  q = e4m3(fp32(fp32(o) / scale))
@@ -46,13 +47,14 @@ def load(path: str) -> ctypes.CDLL:
     L.far_oracle_e4m3_encode.restype = ctypes.c_uint8
     L.far_oracle_e4m3_encode.argtypes = [ctypes.c_double]
     vp = ctypes.c_void_p
-    L.far_oracle_fused.restype = ctypes.c_int
-    L.far_oracle_fused.argtypes = [
-        ctypes.POINTER(vp), ctypes.c_int, vp, vp,
-        ctypes.c_int64, ctypes.c_int64, ctypes.c_int,
-        ctypes.c_float, ctypes.c_float, ctypes.c_int, ctypes.c_int64,
-        ctypes.c_int64, ctypes.c_int64,
-        vp, vp, vp, vp, vp, vp, vp, vp]
+    for fn in (L.far_oracle_fused, L.far_oracle_fused_acc32):
+        fn.restype = ctypes.c_int
+        fn.argtypes = [
+            ctypes.POINTER(vp), ctypes.c_int, vp, vp,
+            ctypes.c_int64, ctypes.c_int64, ctypes.c_int,
+            ctypes.c_float, ctypes.c_float, ctypes.c_int, ctypes.c_int64,
+            ctypes.c_int64, ctypes.c_int64,
+            vp, vp, vp, vp, vp, vp, vp, vp]
     return L
 
 
@@ -105,8 +107,13 @@ def fused(partials: Sequence[np.ndarray], residual: Optional[np.ndarray],
           pattern: int = AR_RESIDUAL_RMSNORM, scale_in: Optional[float] = None,
           rows: Optional[tuple] = None, want_norm: bool = True,
           want_residual_out: bool = True, debug: bool = False,
-          out: Optional[dict] = None, group: int = 0) -> dict:
+          out: Optional[dict] = None, group: int = 0, acc32: bool = False) -> dict:
     """Run the oracle on raw bit patterns.
+
+    ``acc32``: accumulate the partials and the residual in fp32 (partial 0,
+    1, ..., W-1, then the residual, each addition rounded to fp32) instead
+    of exactly -- the pages' fp32_acc=True taken literally.  The two agree
+    except where a rounded running sum meets cancellation.
 
     ``partials`` are W arrays of uint16 patterns of shape (..., H) (any
     leading shape is flattened to (T, H), as the PR #45307 report does for
@@ -166,7 +173,8 @@ def fused(partials: Sequence[np.ndarray], residual: Optional[np.ndarray],
         o.setdefault("rinv", np.zeros((T,), np.float64))
 
     arr = (ctypes.c_void_p * W)(*[p.ctypes.data for p in ps])
-    rc = lib().far_oracle_fused(
+    fn = lib().far_oracle_fused_acc32 if acc32 else lib().far_oracle_fused
+    rc = fn(
         arr, W, _ptr(res), _ptr(gamma), T, H, dt,
         float(eps), float(weight_bias), int(pattern), int(group), b, e,
         _ptr(o["residual_out"]), _ptr(o["norm_out"]), _ptr(o["quant_out"]),

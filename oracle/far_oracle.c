@@ -63,6 +63,7 @@
  *    (group divides H), one scale per (row, group) = amax / 448 at
  *    scale_out[t * (H / group) + h / group].
  */
+#include <float.h>
 #include <math.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -218,21 +219,43 @@ static double to_f32(double x) { return (double)(float)x; }
 /* The fused epilogue                                                      */
 /* ---------------------------------------------------------------------- */
 
+/* The fp32 accumulation below needs float arithmetic evaluated in float. */
+#if !defined(FLT_EVAL_METHOD) || FLT_EVAL_METHOD != 0
+#error "the fp32 accumulation mode needs FLT_EVAL_METHOD == 0"
+#endif
+
 /* Row t: y = sum of the partials (+ residual) and o = y * rinv * (gamma +
- * weight_bias), both in fp64 into y[H] and o[H]; returns rinv. */
+ * weight_bias), both in fp64 into y[H] and o[H]; returns rinv.
+ *
+ * acc32 = 0: the sum is exact (fp64 holds the sum of these 2-byte values
+ * exactly while their exponents span less than 45 binades).
+ * acc32 = 1: the pages' fp32_acc=True taken literally [P1]: partial 0, 1,
+ * ..., W-1, then the residual, added one after another to an fp32 sum that
+ * starts at 0, each addition rounded to fp32 (to nearest, ties to even).
+ * The two differ only where a rounded running sum is followed by
+ * cancellation; everything after y is fp64 in both. */
 static double row_y_o(const uint16_t *const *partials, int W, const uint16_t *residual,
                       const uint16_t *gamma, int64_t t, int64_t H, int dtype,
-                      float eps, float weight_bias, double *y, double *o)
+                      float eps, float weight_bias, int acc32, double *y, double *o)
 {
     const int64_t base = t * H;
     /* 1. all-reduce of the partials, then 2. the residual add [P1] */
     for (int64_t h = 0; h < H; ++h) {
-        double s = 0.0;
-        for (int r = 0; r < W; ++r)
-            s += far_oracle_decode16(partials[r][base + h], dtype);
-        if (residual != NULL)
-            s += far_oracle_decode16(residual[base + h], dtype);
-        y[h] = s;
+        if (acc32) {
+            float s = 0.0f; /* 2-byte values convert to float exactly */
+            for (int r = 0; r < W; ++r)
+                s = s + (float)far_oracle_decode16(partials[r][base + h], dtype);
+            if (residual != NULL)
+                s = s + (float)far_oracle_decode16(residual[base + h], dtype);
+            y[h] = (double)s;
+        } else {
+            double s = 0.0;
+            for (int r = 0; r < W; ++r)
+                s += far_oracle_decode16(partials[r][base + h], dtype);
+            if (residual != NULL)
+                s += far_oracle_decode16(residual[base + h], dtype);
+            y[h] = s;
+        }
     }
     /* 3. mean of squares over the hidden size, eps inside the root */
     double ss = 0.0;
@@ -268,15 +291,15 @@ static double row_y_o(const uint16_t *const *partials, int W, const uint16_t *re
  *
  * Returns 0, or -1 for arguments it cannot interpret.
  */
-int far_oracle_fused(const uint16_t *const *partials, int W,
-                     const uint16_t *residual, const uint16_t *gamma,
-                     int64_t T, int64_t H, int dtype,
-                     float eps, float weight_bias, int pattern, int64_t group,
-                     int64_t row_begin, int64_t row_end,
-                     uint16_t *residual_out, uint16_t *norm_out,
-                     uint8_t *quant_out, const float *scale_in,
-                     float *scale_out,
-                     double *y_dbg, double *o_dbg, double *rinv_dbg)
+static int fused_impl(const uint16_t *const *partials, int W,
+                      const uint16_t *residual, const uint16_t *gamma,
+                      int64_t T, int64_t H, int dtype,
+                      float eps, float weight_bias, int pattern, int64_t group,
+                      int64_t row_begin, int64_t row_end, int acc32,
+                      uint16_t *residual_out, uint16_t *norm_out,
+                      uint8_t *quant_out, const float *scale_in,
+                      float *scale_out,
+                      double *y_dbg, double *o_dbg, double *rinv_dbg)
 {
     if (W < 1 || H < 1 || T < 0 || row_begin < 0 || row_end > T ||
         row_begin > row_end)
@@ -305,7 +328,7 @@ int far_oracle_fused(const uint16_t *const *partials, int W,
     if (pattern == OR_FP8_TENSOR) {
         double amax = 0.0;
         for (int64_t t = row_begin; t < row_end; ++t) {
-            row_y_o(partials, W, residual, gamma, t, H, dtype, eps, weight_bias, y, o);
+            row_y_o(partials, W, residual, gamma, t, H, dtype, eps, weight_bias, acc32, y, o);
             for (int64_t h = 0; h < H; ++h) {
                 double a = fabs(to_f32(o[h]));
                 if (a > amax) /* a NaN element does not take part */
@@ -319,7 +342,7 @@ int far_oracle_fused(const uint16_t *const *partials, int W,
     for (int64_t t = row_begin; t < row_end; ++t) {
         const int64_t base = t * H;
         const double rinv = row_y_o(partials, W, residual, gamma, t, H, dtype, eps,
-                                    weight_bias, y, o);
+                                    weight_bias, acc32, y, o);
 
         if (residual_out != NULL)
             for (int64_t h = 0; h < H; ++h)
@@ -400,4 +423,37 @@ int far_oracle_fused(const uint16_t *const *partials, int W,
     free(y);
     free(o);
     return 0;
+}
+
+int far_oracle_fused(const uint16_t *const *partials, int W,
+                     const uint16_t *residual, const uint16_t *gamma,
+                     int64_t T, int64_t H, int dtype,
+                     float eps, float weight_bias, int pattern, int64_t group,
+                     int64_t row_begin, int64_t row_end,
+                     uint16_t *residual_out, uint16_t *norm_out,
+                     uint8_t *quant_out, const float *scale_in,
+                     float *scale_out,
+                     double *y_dbg, double *o_dbg, double *rinv_dbg)
+{
+    return fused_impl(partials, W, residual, gamma, T, H, dtype, eps, weight_bias, pattern,
+                      group, row_begin, row_end, 0, residual_out, norm_out, quant_out,
+                      scale_in, scale_out, y_dbg, o_dbg, rinv_dbg);
+}
+
+/* The same with the partials and the residual accumulated in fp32 (acc32,
+ * see row_y_o): the reference for the elements where fp32 accumulation,
+ * which the pages prescribe, is not exact. */
+int far_oracle_fused_acc32(const uint16_t *const *partials, int W,
+                           const uint16_t *residual, const uint16_t *gamma,
+                           int64_t T, int64_t H, int dtype,
+                           float eps, float weight_bias, int pattern, int64_t group,
+                           int64_t row_begin, int64_t row_end,
+                           uint16_t *residual_out, uint16_t *norm_out,
+                           uint8_t *quant_out, const float *scale_in,
+                           float *scale_out,
+                           double *y_dbg, double *o_dbg, double *rinv_dbg)
+{
+    return fused_impl(partials, W, residual, gamma, T, H, dtype, eps, weight_bias, pattern,
+                      group, row_begin, row_end, 1, residual_out, norm_out, quant_out,
+                      scale_in, scale_out, y_dbg, o_dbg, rinv_dbg);
 }

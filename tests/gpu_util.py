@@ -8,7 +8,11 @@ Tolerances:
 * e4m3 codes: at most 1 step on the ordered code grid; a code the oracle
   saturates (+-448) must be saturated on the GPU too (except where no code
   can be clamped, see ``compare``); NaN codes must agree;
-* per-token scales: relative error at most 1e-6 (exact when 0).
+* per-token scales: relative error at most 1e-6 (exact when 0);
+* all of these against the oracle with exact accumulation, except at the
+  rare elements where the pages' fp32 accumulation is not exact (a rounded
+  running sum followed by cancellation): there against the oracle with fp32
+  accumulation (see ``compare``).
 """
 from __future__ import annotations
 
@@ -131,25 +135,69 @@ def run_gpu(ctx, g: dict, eps: float, wb: float, pattern: int, scale_in=None, ro
 
 
 def run_oracle(inp: dict, dtype: str, eps, wb, pattern, scale_in=None, rows=None, want_norm=True,
-               want_residual_out=True, row_list=None, group=0) -> dict:
+               want_residual_out=True, row_list=None, group=0, acc32=False) -> dict:
+    """The oracle's outputs for the call (exact accumulation of the partials),
+    with ``_redo32``: a function that recomputes them with fp32
+    accumulation (oracle.fused acc32), used by ``compare`` only for elements
+    that miss the tolerances."""
     ps = [as_u16(p) for p in inp["partials"]]
     res = None if inp["residual"] is None else as_u16(inp["residual"])
     gam = as_u16(inp["gamma"])
     if row_list is not None and pattern == 3:
         raise ValueError("the per-tensor scale needs every row of the call")
     if row_list is None:
-        return oracle.fused(ps, res, gam, dtype, eps, wb, pattern, scale_in=scale_in, rows=rows,
-                            want_norm=want_norm, want_residual_out=want_residual_out, group=group)
-    out = None
-    for t in row_list:
-        out = oracle.fused(ps, res, gam, dtype, eps, wb, pattern, scale_in=scale_in,
-                           rows=(int(t), int(t) + 1), want_norm=want_norm,
-                           want_residual_out=want_residual_out, out=out, group=group)
+        out = oracle.fused(ps, res, gam, dtype, eps, wb, pattern, scale_in=scale_in, rows=rows,
+                           want_norm=want_norm, want_residual_out=want_residual_out, group=group,
+                           acc32=acc32)
+    else:
+        out = None
+        for t in row_list:
+            out = oracle.fused(ps, res, gam, dtype, eps, wb, pattern, scale_in=scale_in,
+                               rows=(int(t), int(t) + 1), want_norm=want_norm,
+                               want_residual_out=want_residual_out, out=out, group=group,
+                               acc32=acc32)
+    if not acc32:
+        out["_redo32"] = lambda: run_oracle(inp, dtype, eps, wb, pattern, scale_in=scale_in,
+                                            rows=rows, want_norm=want_norm,
+                                            want_residual_out=want_residual_out,
+                                            row_list=row_list, group=group, acc32=True)
     return out
+
+
+def _ref32(ref: dict):
+    """The fp32-accumulation reference of ``ref`` (computed once), or None."""
+    if "_ref32" not in ref:
+        redo = ref.get("_redo32")
+        ref["_ref32"] = redo() if redo is not None else None
+    return ref["_ref32"]
+
+
+def _cancellation_mask(ref: dict, r32: dict, sel) -> np.ndarray:
+    """Elements (of the selected rows) where fp32 accumulation changes any
+    output: there the pages' fp32 sum is not exact."""
+    m = None
+    for key in ("residual_out", "norm_out", "quant_out"):
+        if ref.get(key) is not None and r32.get(key) is not None:
+            k = ref[key][sel] != r32[key][sel]
+            m = k if m is None else (m | k)
+    return m
+
+
+def _scale_rel(a: np.ndarray, b: np.ndarray) -> np.ndarray:
+    a, b = a.astype(np.float64), b.astype(np.float64)
+    return np.where(b == 0, np.abs(a), np.abs(a - b) / np.where(b == 0, 1, np.abs(b)))
 
 
 def compare(gpu: dict, ref: dict, dtype: str, rows=None, exact_saturation: bool = True) -> dict:
     """Assert the tolerances on the selected rows; return match statistics.
+
+    The reference is the oracle with exact accumulation of the partials.
+    The pages prescribe fp32 accumulation (fp32_acc=True), which is exact
+    unless a rounded running sum meets cancellation; an element that misses
+    a tolerance passes only if it is such an element -- the oracle with fp32
+    accumulation (``run_oracle``'s ``_redo32``) gives a different output
+    there -- and the GPU meets the same tolerance against that reference.
+    ``stats[key][2]`` counts the elements that took this path.
 
     ``exact_saturation``: where the oracle's code is +-448 the GPU's must be
     too.  Per-tensor FP8 whose codes come from the stored new residual passes
@@ -158,25 +206,51 @@ def compare(gpu: dict, ref: dict, dtype: str, rows=None, exact_saturation: bool 
     rule like every other code."""
     sel = slice(None) if rows is None else rows
     stats = {}
+
+    def check(key, dist, tol):
+        d = dist(gpu[key][sel], ref[key][sel])
+        n32 = 0
+        bad = d > tol
+        if bad.any():
+            r32 = _ref32(ref)
+            assert r32 is not None, (key, int(d.max()), np.argwhere(bad)[:5].tolist())
+            cancel = _cancellation_mask(ref, r32, sel)
+            d32 = dist(gpu[key][sel], r32[key][sel])
+            ok = cancel & (d32 <= tol)
+            assert np.all(ok[bad]), (key, int(d.max()), np.argwhere(bad & ~ok)[:5].tolist())
+            n32 = int(bad.sum())
+            d = np.where(bad, d32, d)
+        stats[key] = (int(d.max()) if d.size else 0, float((d == 0).mean()) if d.size else 1.0, n32)
+        return d
+
     for key in ("residual_out", "norm_out"):
         if ref.get(key) is None:
             continue
         assert gpu[key] is not None, key
-        d = ulp16(gpu[key][sel], ref[key][sel], dtype)
-        stats[key] = (int(d.max()) if d.size else 0, float((d == 0).mean()) if d.size else 1.0)
-        assert d.size == 0 or d.max() <= 1, (key, int(d.max()), np.argwhere(d > 1)[:5].tolist())
+        check(key, lambda a, b: ulp16(a, b, dtype), 1)
     if ref.get("quant_out") is not None:
-        a, b = gpu["quant_out"][sel], ref["quant_out"][sel]
-        d = code_steps(a, b)
-        stats["quant_out"] = (int(d.max()) if d.size else 0, float((d == 0).mean()) if d.size else 1.0)
-        assert d.size == 0 or d.max() <= 1, ("quant_out", int(d.max()), np.argwhere(d > 1)[:5].tolist())
+        check("quant_out", code_steps, 1)
         if exact_saturation:
+            a, b = gpu["quant_out"][sel], ref["quant_out"][sel]
             sat = (b & 0x7F) == 0x7E
-            assert np.array_equal(a[sat], b[sat]), "saturated codes differ"
+            if not np.array_equal(a[sat], b[sat]):
+                r32 = _ref32(ref)
+                b32 = r32["quant_out"][sel]
+                sat32 = (b32 & 0x7F) == 0x7E
+                assert np.array_equal(a[sat & sat32], b[sat & sat32]) and np.all(
+                    (a == b) | (a == b32) | ~sat), "saturated codes differ"
     if ref.get("scale_out") is not None:
-        a = gpu["scale_out"][sel].astype(np.float64)
-        b = ref["scale_out"][sel].astype(np.float64)
-        rel = np.where(b == 0, np.abs(a), np.abs(a - b) / np.where(b == 0, 1, np.abs(b)))
-        stats["scale_out"] = (float(rel.max()) if rel.size else 0.0, float((a == b).mean()) if a.size else 1.0)
-        assert rel.size == 0 or rel.max() <= SCALE_RTOL, ("scale_out", float(rel.max()))
+        a, b = gpu["scale_out"][sel], ref["scale_out"][sel]
+        rel = _scale_rel(a, b)
+        n32 = 0
+        if rel.size and rel.max() > SCALE_RTOL:
+            # a scale whose amax element is a cancellation element
+            b32 = _ref32(ref)["scale_out"][sel]
+            rel32 = _scale_rel(a, b32)
+            bad = rel > SCALE_RTOL
+            assert np.all((rel32 <= SCALE_RTOL)[bad] & (b32 != b)[bad]), ("scale_out", float(rel.max()))
+            n32 = int(bad.sum())
+            rel = np.where(bad, rel32, rel)
+        stats["scale_out"] = (float(rel.max()) if rel.size else 0.0,
+                              float((a == b).mean()) if a.size else 1.0, n32)
     return stats

@@ -50,8 +50,12 @@ MUTANTS = {
     "static code decided in fp64": ("far_oracle_e4m3_encode(to_f32(to_f32(o[h]) / s32))", "far_oracle_e4m3_encode(o[h] / s32)"),
     "dynamic code decided in fp64": ("far_oracle_e4m3_encode(to_f32(to_f32(o[h]) / scale))", "far_oracle_e4m3_encode(o[h] / scale)"),
     "per-tensor code decided in fp64": ("far_oracle_e4m3_encode(to_f32(to_f32(o[h]) / tensor_scale))", "far_oracle_e4m3_encode(o[h] / tensor_scale)"),
-    "per-tensor amax of the first row only": ("            row_y_o(partials, W, residual, gamma, t, H, dtype, eps, weight_bias, y, o);\n            for (int64_t h = 0; h < H; ++h) {",
-                                              "            row_y_o(partials, W, residual, gamma, t, H, dtype, eps, weight_bias, y, o);\n            if (t > row_begin) break;\n            for (int64_t h = 0; h < H; ++h) {"),
+    "per-tensor amax of the first row only": ("            row_y_o(partials, W, residual, gamma, t, H, dtype, eps, weight_bias, acc32, y, o);\n            for (int64_t h = 0; h < H; ++h) {",
+                                              "            row_y_o(partials, W, residual, gamma, t, H, dtype, eps, weight_bias, acc32, y, o);\n            if (t > row_begin) break;\n            for (int64_t h = 0; h < H; ++h) {"),
+    "fp32 accumulation kept in fp64": ("            float s = 0.0f; /* 2-byte values convert to float exactly */",
+                                       "            double s = 0.0f; /* 2-byte values convert to float exactly */"),
+    "fp32 accumulation drops the residual": ("                s = s + (float)far_oracle_decode16(residual[base + h], dtype);",
+                                             "                s = s + 0.0f;"),
     "per-tensor scale over 240": ("tensor_scale = to_f32(amax / 448.0);", "tensor_scale = to_f32(amax / 240.0);"),
     "per-group amax over the first group only": ("for (int64_t h = q * group; h < (q + 1) * group; ++h) {\n                    double a", "for (int64_t h = 0; h < group; ++h) {\n                    double a"),
     "per-group scales indexed by group only": ("scale_out[t * ngroups + q] = (float)scale;", "scale_out[q] = (float)scale;"),
@@ -91,6 +95,9 @@ def quick_pins():
     yield "first pattern", pins.test_first_pattern_without_residual
     yield "gamma column", pins.test_gamma_is_indexed_by_column
     yield "order", pins.test_partial_order_does_not_matter
+    yield "fp32 accumulation worked example", pins.test_worked_example_fp32_accumulation
+    for pattern in (0, 2):
+        yield "fp32 accumulation exact when the sum is %d" % pattern, lambda p=pattern: pins.test_fp32_accumulation_equals_exact_without_cancellation(p)
 
 
 def run_quick_pins():

@@ -710,6 +710,58 @@ def test_gamma_is_indexed_by_column():
     np.testing.assert_array_equal(b["o"][:, 5], 2 * a["o"][:, 5])
 
 
+def test_worked_example_fp32_accumulation():
+    """The oracle's fp32-accumulation mode (fp32_acc=True taken literally:
+    partial 0, 1, ..., then the residual, each addition rounded to fp32)
+    against a hand-derived case of rounding followed by cancellation, in
+    units of 2^-32: partials -237*2^21, -236, -9*2^24, 129*2^23, residual
+    -207*2^21 (bf16 values; their exact sum is -236, i.e. -5.49e-8).
+      s1 = -237*2^21                                     (exact)
+      s2 = -(237*2^21 + 236) rounds to a multiple of 32 (ulp 2^-27 in
+           [2^-4, 2^-3)): 236/32 = 7.375 -> -(237*2^21 + 224)
+      s3 = -(309*2^21 + 224) rounds to a multiple of 64 (ulp 2^-26):
+           224/64 = 3.5, a tie, to even -> -(309*2^21 + 256)
+      s4 = 207*2^21 - 256                                 (exact)
+      y  = s4 - 207*2^21 = -256, i.e. -2^-24
+    The exact mode keeps -236 * 2^-32: bf16 0xB36C; fp32 accumulation gives
+    -2^-24: bf16 0xB380.  The other columns (all partials 1.0, residual 1.0,
+    sum 5, exact either way) agree, and so does every output there."""
+    units = [-237 * 2 ** 21, -236, -9 * 2 ** 24, 129 * 2 ** 23, -207 * 2 ** 21]
+    vals = [u * 2.0 ** -32 for u in units]
+    H = 8
+    enc = lambda v: oracle.round16(v, "bf16")  # noqa: E731  exact: every value is a bf16
+    ps = [np.array([[enc(v)] + [enc(1.0)] * (H - 1)], dtype=np.uint16) for v in vals[:4]]
+    res = np.array([[enc(vals[4])] + [enc(1.0)] * (H - 1)], dtype=np.uint16)
+    gam = np.array([enc(1.0)] * H, dtype=np.uint16)
+    assert [oracle.decode16(int(p[0, 0]), "bf16") for p in ps] == vals[:4]
+    ex = oracle.fused(ps, res, gam, "bf16", 1e-6, 0.0, 0)
+    f32 = oracle.fused(ps, res, gam, "bf16", 1e-6, 0.0, 0, acc32=True)
+    assert ex["residual_out"][0, 0] == 0xB36C
+    assert f32["residual_out"][0, 0] == 0xB380
+    assert np.array_equal(ex["residual_out"][0, 1:], f32["residual_out"][0, 1:])
+    assert oracle.decode16(int(ex["residual_out"][0, 1]), "bf16") == 5.0
+
+
+@pytest.mark.parametrize("pattern", [0, 1, 2, 3])
+def test_fp32_accumulation_equals_exact_without_cancellation(pattern):
+    """Where every running fp32 sum is exact the two modes agree bit for bit:
+    partials and residual of magnitude in [1, 2) with at most 8 significant
+    bits sum exactly in fp32 (sums below 2^6 need at most 14 bits)."""
+    rng = np.random.default_rng(11)
+    W, T, H = 4, 6, 64
+    mags = 1.0 + rng.integers(0, 128, size=(W + 1, T, H)) / 128.0
+    signs = np.where(rng.random((W + 1, T, H)) < 0.5, -1.0, 1.0)
+    enc = np.vectorize(lambda v: oracle.round16(v, "bf16"))
+    arr = enc(mags * signs).astype(np.uint16)
+    gam = enc(rng.uniform(0.5, 1.5, H)).astype(np.uint16)
+    kw = dict(scale_in=0.05) if pattern == 1 else {}
+    ex = oracle.fused(list(arr[:W]), arr[W], gam, "bf16", 1e-6, 0.0, pattern, **kw)
+    f32 = oracle.fused(list(arr[:W]), arr[W], gam, "bf16", 1e-6, 0.0, pattern, acc32=True, **kw)
+    for k in ("residual_out", "norm_out", "quant_out", "scale_out"):
+        if ex.get(k) is not None:
+            assert np.array_equal(ex[k], f32[k]), k
+
+
 def test_golden_small_workload_fixture_is_reproduced():
     """The stored oracle outputs for the small workload (tests/golden) still
     come out of the oracle bit for bit."""
