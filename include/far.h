@@ -39,8 +39,10 @@
  *  - vllm.distributed.device_communicators.aiter_custom_all_reduce,
  *    use_1stage_fused_ar_rms: rows made of 16-byte packs and a token cap of
  *    80 for the one-kernel path.  Here: H must be a multiple of 8 (16-byte
- *    packs of 2-byte elements), and rows <= decode_max_rows (default 80) take
- *    the cluster-per-row decode kernel.
+ *    packs of 2-byte elements), and calls of at most decode_max_rows rows
+ *    (default 80) whose rows are long (one CTA would need 4 or more packs
+ *    per thread: H >= 8192 at 256 threads) take the cluster-per-row decode
+ *    kernel; shorter rows run faster with one CTA per row (measured).
  *
  * Ownership: the caller owns every buffer.  The library allocates and frees
  * nothing per call and never synchronises the stream; a call only enqueues
@@ -97,7 +99,7 @@ typedef enum {
 } far_pattern;
 
 typedef enum {
-    FAR_REGIME_AUTO = 0,    /* decode for rows <= decode_max_rows of large rows, else prefill */
+    FAR_REGIME_AUTO = 0,    /* decode for <= decode_max_rows long rows, else prefill */
     FAR_REGIME_DECODE = 1,  /* one thread-block cluster per row            */
     FAR_REGIME_PREFILL = 2  /* one CTA per row (or several rows per CTA)  */
 } far_regime;
@@ -116,7 +118,9 @@ typedef enum {
  * FAR_PDL=1|0: launch with programmatic dependent launch, default 1,
  * FAR_RING_MIN_ROWS: fewest rows for the ring kernel, default by rule,
  * FAR_TENSOR_REVERSE=1|0: the second pass of per-tensor FP8 takes the rows
- * from the last one down, default 1). */
+ * from the last one down, default 1, FAR_TENSOR_FUSED=1|0: per-tensor FP8
+ * without norm_out on the ring kernel runs both passes in one cooperative
+ * launch with a grid barrier between them, default 0). */
 /*
  * Programmatic dependent launch: every kernel of this library first waits
  * (griddepcontrol.wait) until the grid it depends on has completed, then
@@ -199,7 +203,14 @@ far_status far_fused(far_ctx *ctx,
  * full T-row tensors; rows outside the range are neither read nor written
  * (scale_out included).  0 <= row_begin <= row_end <= T, else
  * FAR_ERR_INVALID_ARG; an empty range is a no-op.  Disjoint row ranges
- * together give exactly (bit for bit) the far_fused result.
+ * together give exactly (bit for bit) the far_fused result whenever the
+ * calls run with the same packs per thread and threads per row
+ * (far_describe_launch): the one-CTA and ring kernels reduce a row in the
+ * same order then, and the one-CTA kernel's geometry does not depend on the
+ * number of rows.  Otherwise (a cluster per row against one CTA per row, or
+ * a ring geometry other than the one-CTA kernel's) the fp32 sum of squares
+ * is reduced in another order and the outputs agree within the parity
+ * tolerances (1 ulp, 1 FP8 step).
  */
 far_status far_fused_rows(far_ctx *ctx, int64_t row_begin, int64_t row_end,
                           const void *const *partials, int W,
@@ -339,7 +350,10 @@ size_t far_host_staging_bytes(int W, int64_t H, int64_t chunk_rows);
  * FAR_ERR_INVALID_ARG, a misaligned one FAR_ERR_ALIGNMENT.  The staging
  * area is scratch; calls that share one must not overlap on the GPU (calls
  * on one context are ordered through its events; the enqueueing is
- * serialised by a lock of the context).  A CUDA error part-way through the
+ * serialised by a lock of the context).  That ordering is per context, not
+ * per staging area: each call's copies in wait for the previous call's
+ * kernels even when the two calls use different staging areas, so calls
+ * meant to overlap need contexts of their own.  A CUDA error part-way through the
  * enqueueing returns FAR_ERR_CUDA, and the work already enqueued still runs.
  * The first call on a context creates its two copy streams and seven
  * events, released by far_destroy; make that first call before any stream

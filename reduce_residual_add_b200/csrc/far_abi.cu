@@ -29,6 +29,7 @@ struct far_ctx {
   int ring_threads_set; // ring_threads came from the environment
   int ring_slots_max;   // at most this many ring slots
   int tensor_reverse;   // per-tensor FP8: second pass from the last row down
+  int tensor_fused;     // per-tensor FP8: both passes in one ring launch when possible
   int ring_gamma_mode;  // ring: 1 stage gamma in shared memory, 0 read it through L1, -1 by rule
   int pdl;              // programmatic dependent launch on every call
   int ring_min_rows;    // fewer rows than this take the direct kernel
@@ -274,7 +275,9 @@ int ring_occ_cached(const far_ctx* ctx, int dtype, int vpt, int minb, int thread
     if (e.dtype == dtype && e.vpt == vpt && e.minb == minb && e.threads == threads && e.smem == smem)
       return e.ctas;
   }
-  const int n = far::ring_occupancy(dtype, vpt, minb, threads, smem);
+  // minb < 0 marks the decode kernel's entries
+  const int n = minb < 0 ? far::decode_occupancy(dtype, vpt, threads)
+                         : far::ring_occupancy(dtype, vpt, minb, threads, smem);
   if (c->occ_n < far_ctx::kOccEntries) c->occ[c->occ_n++] = far_ctx::OccEntry{dtype, vpt, minb, threads, smem, n};
   return n;
 }
@@ -290,27 +293,41 @@ far::Launch plan(const far_ctx* ctx, int64_t rows, int64_t H, int dtype, int seg
   } else if (ctx->force_regime == FAR_REGIME_PREFILL) {
     decode = false;
   } else {
-    // Measured on B200: with few rows a cluster per row beats one CTA per
-    // row once the CTA would hold >= 32 16-byte loads per thread (large
-    // rows); below that the single CTA's shorter path wins.
+    // Measured on B200 with inputs cold in L2 (CUDA graphs cycling through
+    // more than 2x L2), rows <= 80: a cluster per row beats one CTA per row
+    // once that CTA would need 4 or more packs per thread (H >= 8192 at 256
+    // threads: 2.8-4.1 vs 3.6-4.2 us at W=2, H=8192; 2.9-5.9 vs 6.2-7.6 us
+    // at H=16384) or 32 or more loads per thread; at H=4096 the single
+    // CTA's shorter path wins (W=2 and W=8: 2.4-3.9 vs 2.8-4.2 us).
     far::Launch d{};
     plan_prefill(packs, ctx->prefill_threads, &d);
-    decode = rows <= ctx->decode_max_rows && packs >= 64 && segs * d.vpt >= 32;
+    decode = rows <= ctx->decode_max_rows && packs >= 64 && (d.vpt >= 4 || segs * d.vpt >= 32);
   }
   if (decode) {
     int cl = ctx->decode_cluster;
     if (cl <= 0) {
-      // measured: 4 CTAs per row from 32 rows up; below, at most 32 KiB of
-      // a row per CTA (8 at W=8 H=8192, 16 at H=16384)
-      cl = 4;
-      if (rows <= 16) {
-        const int64_t row_bytes = static_cast<int64_t>(segs) * H * 2;
-        while (cl < 16 && row_bytes > static_cast<int64_t>(cl) * 32 * 1024) cl *= 2;
-      }
+      // measured (cold, as above): 16 CTAs per row for up to 4 rows, 8 up
+      // to 16 rows, 4 beyond (T = 1 / 8 / 32 / 80 at H = 8192 and 16384)
+      cl = rows <= 4 ? 16 : (rows <= 16 ? 8 : 4);
     }
     plan_decode(packs, cl, &l);
+    // ... and no more CTAs than are resident in one wave: a second wave
+    // costs more than a smaller cluster (H=16384, W=2, 80 rows: 4 CTAs per
+    // row in two waves 7.6 us, 2 per row 5.9 us)
+    if (ctx->decode_cluster <= 0) {
+      while (l.cluster > 1) {
+        const int occ = ring_occ_cached(ctx, dtype, l.vpt, -1, l.threads, 0);
+        if (rows * l.cluster <= static_cast<int64_t>(occ) * ctx->sm_count) break;
+        plan_decode(packs, l.cluster / 2, &l);
+      }
+    }
     l.grid = rows * l.cluster;
   } else {
+    // The threads per row do not depend on the number of rows, so that row
+    // slices of a call reduce each row in the same order as the whole call
+    // (rows of 3 segments ran faster cold at 4 packs per thread from 4 rows
+    // per SM up, W=2: 5.9 vs 6.4 us at 1024 x 2048, but a slice below that
+    // size would then round differently from the whole call).
     plan_prefill(packs, ctx->prefill_threads, &l);
     l.grid = (rows + l.rows_per_cta - 1) / l.rows_per_cta;
     // The ring pays off once each persistent CTA gets enough rows to keep
@@ -383,6 +400,7 @@ far_status far_create(far_ctx** ctx, int device) {
   c.ring_threads_set = std::getenv("FAR_RING_THREADS") != nullptr;
   c.ring_slots_max = env_int("FAR_RING_SLOTS", 0);  // 0: by the 72 KiB rule
   c.tensor_reverse = env_int("FAR_TENSOR_REVERSE", 1) != 0;
+  c.tensor_fused = env_int("FAR_TENSOR_FUSED", 0) != 0;
   c.ring_gamma_mode = env_int("FAR_RING_GAMMA_SMEM", -1);
   if (c.ring_gamma_mode > 1) c.ring_gamma_mode = 1;
   if (c.ring_gamma_mode < -1) c.ring_gamma_mode = -1;
@@ -630,7 +648,8 @@ struct DeviceGuard {
 // Without norm_out, and with a new residual to write, pass 1 also stores
 // each row's new residual (except in rows that may overflow the format,
 // which it flags) and pass 2 forms the codes from it: the inputs are read
-// once, and pass 2 moves 3 bytes per element.  With norm_out, whose
+// once, and pass 2 moves 3 bytes per element.  When pass 1 is the ring
+// kernel, pass 2 runs inside the same launch after a grid barrier.  With norm_out, whose
 // 2-byte result would feel the rounding of y, or with no residual output,
 // pass 2 reads every input again and writes every output, as pass 1's
 // kernel would.
@@ -646,6 +665,7 @@ far_status far_fused_fp8_tensor_launch(far_ctx* ctx, int64_t row_begin, int64_t 
   p.wait_limit_ns = ctx->wait_limit_ns;
   p.stall_segment = ctx->stall_segment;
   p.ws_amax = static_cast<unsigned*>(workspace);
+  p.ws_arrive = p.ws_amax + 1;
   p.ws_rinv = reinterpret_cast<float*>(static_cast<unsigned char*>(workspace) + 256);
   p.ws_row0 = row_begin;
   const bool from_residual = norm_out == nullptr && p.residual_out != nullptr;
@@ -661,13 +681,27 @@ far_status far_fused_fp8_tensor_launch(far_ctx* ctx, int64_t row_begin, int64_t 
     whole.grid = (row_end - row_begin + whole.rows_per_cta - 1) / whole.rows_per_cta;
     whole.pdl = ctx->pdl;
   }
-  cudaError_t e = cudaMemsetAsync(workspace, 0, sizeof(unsigned), s);
+  // the amax word and the grid barrier's arrival count start at zero
+  cudaError_t e = cudaMemsetAsync(workspace, 0, 2 * sizeof(unsigned), s);
   if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync");
   far::Launch first = whole;
   first.pdl = 0;  // it must see the memset above
   p.pattern = far::kTensorAmax;
+  // With the ring kernel (persistent CTAs, all co-resident by construction)
+  // and the codes formed from the stored new residual, both passes run in
+  // one cooperative launch: each CTA meets the others at a grid barrier after
+  // its rows, then writes its own rows' codes, newest first.
+  const bool fused = ctx->tensor_fused && from_residual && first.regime == FAR_REGIME_PREFILL &&
+                     first.kernel == 1 &&
+                     row_end - row_begin <= 0x7fffffff;
+  if (fused) {
+    first.cooperative = 1;
+    p.tensor_fused = 1;
+  }
   e = launch_rows(p, dtype, first, row_begin, row_end, s);
   if (e != cudaSuccess) return cuda_fail(e, "kernel launch (per-tensor pass 1)");
+  if (fused) return FAR_OK;
+  p.tensor_fused = 0;
   // the second pass takes the rows last row first: the rows the first pass
   // wrote last are still in L2 when it starts
   p.pattern = far::kTensorQuant;

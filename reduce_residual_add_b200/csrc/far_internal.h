@@ -54,6 +54,10 @@ struct Params {
   int reverse;                  // take the rows from row_end - 1 down to row_begin
   int tensor_stores_residual;   // per-tensor FP8, first pass: store the new residual
                                 // of every row it does not flag for a rebuild
+  int tensor_fused;             // per-tensor FP8 in one ring launch: after its rows, each
+                                // CTA meets the others at a grid barrier (ws_arrive) and
+                                // writes its rows' codes from the stored new residual
+  unsigned* ws_arrive;          // per-tensor FP8: CTAs past their first pass
 };
 
 // Geometry of one launch, chosen on the host.
@@ -72,6 +76,7 @@ struct Launch {
   int pdl;              // launch with programmatic stream serialization
   int ring_minb;        // ring: CTAs per SM its registers are sized for (2 or 3; 1 or 2 at 8 packs)
   int ring_gamma;       // ring: 1 = gamma staged in shared memory, 0 = read through L1
+  int cooperative;      // launch cooperatively (every CTA co-resident; a grid barrier inside)
 };
 
 // Enqueue one kernel on `stream`.  Returns the launch error (cudaSuccess if
@@ -87,6 +92,10 @@ int ring_header_bytes(int nslot);
 // Resident ring CTAs per SM for this configuration on the current device
 // (0 if it cannot run).
 int ring_occupancy(int dtype, int vpt, int minb, int threads, int smem_bytes);
+
+// Resident decode-kernel CTAs per SM at `threads` threads (its clusters
+// aside; 0 if it cannot run).
+int decode_occupancy(int dtype, int vpt, int threads);
 
 // The device error word of the current device (see far_check): read it
 // after the work on `stream`, or clear it.  Both synchronise `stream`.

@@ -53,6 +53,16 @@ __host__ __device__ constexpr int ring_offset(int nslot) {
   return (16 * nslot + static_cast<int>(sizeof(RingHeader)) + 127) / 128 * 128;
 }
 
+// Which instantiation serves a pattern: the per-group and the per-tensor
+// passes have kernels of their own, so that the other patterns' code carries
+// none of their registers.
+constexpr int kModePlain = 0, kModeGroup = 1, kModeTensor = 2;
+__host__ __device__ constexpr int mode_of(int pattern) {
+  return pattern == kFp8Group ? kModeGroup
+         : (pattern == kTensorAmax || pattern == kTensorQuant) ? kModeTensor
+                                                               : kModePlain;
+}
+
 // Row number k (0 <= k < row_end - row_begin) of a call, counted from
 // row_begin up, or with p.reverse from row_end - 1 down.
 __device__ __forceinline__ int64_t call_row(const Params& p, int64_t k) {
@@ -190,19 +200,57 @@ __device__ __forceinline__ uint4 ld_once_coherent(const uint4* p) {
   return r;
 }
 
+// L2 eviction priorities (PTX createpolicy): per-tensor FP8's first pass
+// stores the new residual with evict_last so that as much of it as L2 holds
+// is still there when the second pass reads it back, which reads it with
+// evict_first (it is not read again).
+__device__ __forceinline__ uint64_t l2_evict_last() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+__device__ __forceinline__ uint64_t l2_evict_first() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+__device__ __forceinline__ void st_l2_hint(uint4* p, const uint4& v, uint64_t pol) {
+  asm volatile("st.global.L2::cache_hint.v4.u32 [%0], {%1,%2,%3,%4}, %5;"
+               ::"l"(p), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w), "l"(pol)
+               : "memory");
+}
+// The same through the coherent path, for data written earlier in the same
+// kernel.
+__device__ __forceinline__ uint4 ld_coherent_l2_hint(const uint4* p, uint64_t pol) {
+  uint4 r;
+  asm volatile("ld.global.L1::no_allocate.L2::cache_hint.L2::256B.v4.u32 {%0,%1,%2,%3}, [%4], %5;"
+      : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+      : "l"(p), "l"(pol));
+  return r;
+}
+__device__ __forceinline__ uint4 ld_once_l2_hint(const uint4* p, uint64_t pol) {
+  uint4 r;
+  asm volatile("ld.global.nc.L1::no_allocate.L2::cache_hint.L2::256B.v4.u32 {%0,%1,%2,%3}, [%4], %5;"
+      : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+      : "l"(p), "l"(pol));
+  return r;
+}
+
 // ---------------------------------------------------------------------------
 // TMA bulk copies and mbarriers (PTX ISA: cp.async.bulk, mbarrier)
 // ---------------------------------------------------------------------------
 
 // Device-side error word of this library, one per device: bit 0 = a consumer
 // gave up waiting for a bulk copy, bit 1 = the producer gave up waiting for
-// a free slot, bit 2 = a cluster CTA gave up waiting for its peers' totals.
+// a free slot, bit 2 = a cluster CTA gave up waiting for its peers' totals,
+// bit 3 = a CTA gave up waiting at the per-tensor grid barrier.
 // Read and cleared by far_check().
 __device__ unsigned int g_far_error = 0u;
 
 constexpr unsigned kErrWaitFull = 1u;
 constexpr unsigned kErrWaitEmpty = 2u;
 constexpr unsigned kErrWaitPeer = 4u;
+constexpr unsigned kErrWaitGrid = 8u;
 
 __device__ __forceinline__ uint32_t smem_addr(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -432,11 +480,12 @@ __device__ __forceinline__ uint4 gamma_pack(const Params& p, const uint4* gamma_
   return gamma_smem != nullptr ? gamma_smem[j] : __ldg(static_cast<const uint4*>(p.gamma) + j);
 }
 
-// GROUP: this instantiation serves only the per-group pattern (kept apart
-// so that the other patterns' code carries none of its registers).
+// MODE (kModePlain / kModeGroup / kModeTensor): the patterns this
+// instantiation serves; per-group and per-tensor code is compiled only into
+// their own instantiations, so the other patterns carry none of its registers.
 // GPRE: gamma's packs were loaded by the caller into gpre[k] (pack
 // j0 + k * jstride); otherwise they come from gamma_smem or through L1.
-template <class DT, int VPT, bool GROUP, bool GPRE, class Red>
+template <class DT, int VPT, int MODE, bool GPRE, class Red>
 __device__ __forceinline__ void finish_row(const Params& p, int64_t row, bool row_ok, int j0,
                                            int jstride, const bool (&ok)[VPT],
                                            float (&y)[VPT][8], const Red& red,
@@ -449,8 +498,8 @@ __device__ __forceinline__ void finish_row(const Params& p, int64_t row, bool ro
   // dynamic per-tensor FP8 runs in two passes: the first records rinv and
   // the call's amax (and, with p.tensor_stores_residual, the new residual);
   // the second writes the other outputs
-  const bool tensor_amax = p.pattern == kTensorAmax;
-  const bool tensor_quant = p.pattern == kTensorQuant;
+  const bool tensor_amax = MODE == kModeTensor && p.pattern == kTensorAmax;
+  const bool tensor_quant = MODE == kModeTensor && p.pattern == kTensorQuant;
   if (p.residual_out != nullptr && !tensor_amax) {
 #pragma unroll
     for (int k = 0; k < VPT; ++k)
@@ -474,7 +523,7 @@ __device__ __forceinline__ void finish_row(const Params& p, int64_t row, bool ro
 
   const bool fp8_static = p.pattern == kFp8Static;
   const bool fp8_token = p.pattern == kFp8Token;
-  constexpr bool fp8_group = GROUP;
+  constexpr bool fp8_group = MODE == kModeGroup;
 
   // a5b needs max|o| = rinv * max|y * (gamma + wb)| (rinv > 0): its local
   // part goes into the same reduction round as the sum of squares.  The
@@ -519,9 +568,10 @@ __device__ __forceinline__ void finish_row(const Params& p, int64_t row, bool ro
     // the stored rinv, which is otherwise +0, positive or +inf).
     const bool rebuild = !(ss < DT::kOverflowSq);
     if (p.tensor_stores_residual && !rebuild) {
+      const uint64_t keep = l2_evict_last();
 #pragma unroll
       for (int k = 0; k < VPT; ++k)
-        if (ok[k]) static_cast<uint4*>(p.residual_out)[rbase + j0 + k * jstride] = pack8<DT>(y[k]);
+        if (ok[k]) st_l2_hint(static_cast<uint4*>(p.residual_out) + rbase + j0 + k * jstride, pack8<DT>(y[k]), keep);
     }
     if (row_ok && red.leader()) {
       p.ws_rinv[row - p.ws_row0] =
@@ -615,7 +665,7 @@ struct RowLoads {
   static constexpr bool kGammaAhead = VPT <= 4;
 };
 
-template <class DT, int VPT, bool GROUP, class Red>
+template <class DT, int VPT, int MODE, class Red>
 __device__ __forceinline__ void fused_row(const Params& p, int64_t row, bool row_ok,
                                           int j0, int jstride, int jend, const Red& red) {
   using L = RowLoads<VPT>;
@@ -687,7 +737,7 @@ __device__ __forceinline__ void fused_row(const Params& p, int64_t row, bool row
 #pragma unroll
     for (int k = 0; k < VPT; ++k) add_pack<DT>(res[k], y[k]);
   }
-  finish_row<DT, VPT, GROUP, L::kGammaAhead>(p, row, row_ok, j0, jstride, ok, y, red, nullptr, gam);
+  finish_row<DT, VPT, MODE, L::kGammaAhead>(p, row, row_ok, j0, jstride, ok, y, red, nullptr, gam);
 }
 
 // ---------------------------------------------------------------------------
@@ -698,7 +748,7 @@ __device__ __forceinline__ void fused_row(const Params& p, int64_t row, bool row
 // (tpr <= 32, power of two); otherwise one row per CTA.
 // Registers: at one pack per thread (rows of at most 256 packs, often short
 // calls of many rows) four 256-thread CTAs per SM; otherwise two, one at 8.
-template <class DT, int VPT, bool SUB, bool GROUP>
+template <class DT, int VPT, bool SUB, int MODE>
 __global__ void __launch_bounds__(kMaxThreads, (VPT >= 8 ? 1 : (VPT == 1 ? 4 : 2)))
 far_prefill_kernel(const Params p) {
   pdl_enter();
@@ -707,11 +757,11 @@ far_prefill_kernel(const Params p) {
   const int64_t row = call_row(p, k);
   if constexpr (SUB) {
     const SubwarpRed red{static_cast<int>(blockDim.x)};
-    fused_row<DT, VPT, GROUP>(p, row, row_ok, threadIdx.x, blockDim.x, p.packs, red);
+    fused_row<DT, VPT, MODE>(p, row, row_ok, threadIdx.x, blockDim.x, p.packs, red);
   } else {
     __shared__ float s_sum[32], s_max[32];
     const BlockRed red{s_sum, s_max};
-    fused_row<DT, VPT, GROUP>(p, row, row_ok, threadIdx.x, blockDim.x, p.packs, red);
+    fused_row<DT, VPT, MODE>(p, row, row_ok, threadIdx.x, blockDim.x, p.packs, red);
   }
 }
 
@@ -740,8 +790,127 @@ far_decode_kernel(const Params p) {
   const int jend = min(p.packs, jbeg + chunk);
   const ClusterRed red{BlockRed{s_sum, s_max}, s_in, &s_bar, ncta, rank, p.wait_limit_ns};
   const bool row_ok = blockIdx.y < p.row_end - p.row_begin;
-  fused_row<DT, VPT, false>(p, row, row_ok, jbeg + static_cast<int>(threadIdx.x), blockDim.x, jend,
+  fused_row<DT, VPT, kModePlain>(p, row, row_ok, jbeg + static_cast<int>(threadIdx.x), blockDim.x, jend,
                             red);
+}
+
+// ---------------------------------------------------------------------------
+// dynamic per-tensor FP8: the codes from the stored new residual
+// ---------------------------------------------------------------------------
+
+// The 8 codes of one pack.  In the usual case (a scale whose reciprocal is
+// normal) the quotient is formed as q = (y * (rinv / scale)) * (gamma + wb),
+// two multiplies per element with rs = RN(rinv * RN(1 / scale)) per row: a
+// few fp32 ulps from o / scale, nothing against the half-ulp of the 2-byte
+// format already in y here and far inside one e4m3 step.  Otherwise o is
+// formed and divided as in every other pattern.
+template <class DT>
+__device__ __forceinline__ uint2 tensor_codes(const uint4& gam, float wb, float (&y)[8], float rinv,
+                                              float rs, float scale, float inv, bool exact) {
+  float g[8];
+  pack_plus<DT>(gam, wb, g);
+  if (!exact && scale != 0.f) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) y[i] = (y[i] * rs) * g[i];
+    return make_uint2(e4m3x4(y[0], y[1], y[2], y[3]), e4m3x4(y[4], y[5], y[6], y[7]));
+  }
+#pragma unroll
+  for (int i = 0; i < 8; ++i) y[i] = (y[i] * rinv) * g[i];
+  return fp8_codes8(y, scale, inv, exact);
+}
+
+// One row of the second pass on its own: from the stored new residual, or
+// (a flagged row) rebuilt from the inputs in the first pass's order --
+// partials 0..W-1, then the residual -- with its new residual written here.
+// COHERENT: the stored new residual was written earlier in the same kernel
+// (the fused form), so it is read through the coherent path; gamma_s: gamma
+// staged in shared memory, or null (read through L1).
+template <class DT, int VPT, bool COHERENT = false>
+__device__ __forceinline__ void tensor_quant_row(const Params& p, int64_t row, float w, int j0,
+                                                 int tpr, const bool (&ok)[VPT], float inv,
+                                                 float scale, bool exact, uint64_t drop,
+                                                 const uint4* gamma_s = nullptr) {
+  const uint4* gamma = gamma_s != nullptr ? gamma_s : static_cast<const uint4*>(p.gamma);
+  const int64_t rbase = row * static_cast<int64_t>(p.packs);
+  const bool rebuild = signbit(w);
+  const float rinv = fabsf(w);
+  const float rs = rinv * inv;
+#pragma unroll
+  for (int q = 0; q < VPT; ++q) {
+    if (!ok[q]) continue;
+    const int64_t pk = rbase + j0 + q * tpr;
+    float y[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    if (!rebuild) {
+      const uint4* src = static_cast<const uint4*>(p.residual_out) + pk;
+      add_pack<DT>(COHERENT ? ld_coherent_l2_hint(src, drop) : ld_once_l2_hint(src, drop), y);
+    } else {
+      for (int r = 0; r < p.W; ++r) add_pack<DT>(ld_once(static_cast<const uint4*>(p.partials[r]) + pk), y);
+      if (p.residual != nullptr)
+        add_pack<DT>(ld_once_coherent(static_cast<const uint4*>(p.residual) + pk), y);
+      static_cast<uint4*>(p.residual_out)[pk] = pack8<DT>(y);
+    }
+    const uint4 g = gamma_s != nullptr ? gamma[j0 + q * tpr] : __ldg(gamma + j0 + q * tpr);
+    reinterpret_cast<uint2*>(p.quant_out)[pk] =
+        tensor_codes<DT>(g, p.weight_bias, y, rinv, rs, scale, inv, exact);
+  }
+}
+
+// The scale of dynamic per-tensor FP8 from the call's amax word, and the
+// derived divisor terms (see tensor_codes).  CTA 0 writes scale_out[0].
+struct TensorScale {
+  float scale, inv;
+  bool exact;
+  __device__ explicit TensorScale(const Params& p, unsigned amax_bits) {
+    scale = __fdiv_rn(__uint_as_float(amax_bits), 448.f);
+    if (scale != scale) scale = 0.f;
+    if (blockIdx.x == 0 && threadIdx.x == 0 && threadIdx.y == 0) p.scale_out[0] = scale;
+    inv = __frcp_rn(scale);
+    exact = needs_exact_div(scale, inv);
+  }
+};
+
+// The fused form's second half, run by the consumer threads of a ring CTA
+// once its own rows are done: a grid barrier (every CTA is co-resident:
+// cooperative launch), then this CTA's rows again, the most recently written
+// first (their new residual is the likeliest to be still in L2), codes from
+// the stored new residual.  The wait is bounded; a CTA that gives up sets
+// the device error word and writes no codes.  Only this CTA's own rows are
+// read back, so the only data another CTA wrote is the amax word.
+template <class DT, int VPT>
+__device__ __forceinline__ void ring_tensor_tail(const Params& p, int64_t my_rows, int ncons,
+                                                 const uint4* gamma_s, volatile int* abort_flag) {
+  consumer_bar(ncons);  // every consumer of this CTA is past its last row
+  if (threadIdx.x == 0) {
+    __threadfence();    // this CTA's amax and stores before its arrival (cumulative)
+    atomicAdd(p.ws_arrive, 1u);
+    const uint64_t t0 = global_ns();
+    for (;;) {
+      unsigned n;
+      asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(n) : "l"(p.ws_arrive) : "memory");
+      if (n >= gridDim.x) break;
+      if (global_ns() - t0 > p.wait_limit_ns) {
+        atomicOr(&g_far_error, kErrWaitGrid);
+        *abort_flag = 1;
+        break;
+      }
+    }
+  }
+  consumer_bar(ncons);
+  if (*abort_flag) return;
+  unsigned amax_bits;
+  asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(amax_bits) : "l"(p.ws_amax) : "memory");
+  const TensorScale ts(p, amax_bits);
+  const uint64_t drop = l2_evict_first();
+  const int j0 = threadIdx.x;
+  bool ok[VPT];
+#pragma unroll
+  for (int q = 0; q < VPT; ++q) ok[q] = j0 + q * ncons < p.packs;
+  for (int64_t i = my_rows - 1; i >= 0; --i) {
+    const int64_t row = call_row(p, blockIdx.x + i * gridDim.x);
+    const float w = *reinterpret_cast<volatile const float*>(p.ws_rinv + (row - p.ws_row0));
+    tensor_quant_row<DT, VPT, true>(p, row, w, j0, ncons, ok, ts.inv, ts.scale, ts.exact, drop,
+                                    gamma_s);
+  }
 }
 
 // Prefill through the TMA engine: a persistent CTA per SM (or two) walks
@@ -760,7 +929,7 @@ far_decode_kernel(const Params p) {
 // the producer stops, and thread 0 waits (bounded) for the copies already
 // issued before the CTA exits.
 // MINB: CTAs per SM the register budget is sized for (2 or 3; 1 or 2 at VPT 8).
-template <class DT, int VPT, int MINB, bool GROUP>
+template <class DT, int VPT, int MINB, int MODE>
 __global__ void __launch_bounds__(kRingMaxConsumers + 32, MINB)
 far_ring_kernel(const Params p, int nslot, int ncons, int stage_gamma) {
   extern __shared__ __align__(128) unsigned char smem[];
@@ -858,9 +1027,7 @@ far_ring_kernel(const Params p, int nslot, int ncons, int stage_gamma) {
       for (int e = 0; e < 8; ++e) y[k][e] = 0.f;
     }
     for (int k = 0; k < S; ++k) {
-      // the abort flag is read only when the segment is not there yet
-      if (!mbar_try_wait(&full[slot], phase) && !*abort_flag &&
-          !mbar_wait(&full[slot], phase, abort_flag, p.wait_limit_ns)) {
+      if (!*abort_flag && !mbar_wait(&full[slot], phase, abort_flag, p.wait_limit_ns)) {
         if (!*abort_flag) atomicOr(&g_far_error, kErrWaitFull);
         *abort_flag = 1;
       }
@@ -875,8 +1042,11 @@ far_ring_kernel(const Params p, int nslot, int ncons, int stage_gamma) {
         phase ^= 1u;
       }
     }
-    finish_row<DT, VPT, GROUP, false>(p, row, true, j0, ncons, ok, y, (i & 1) ? red1 : red0,
+    finish_row<DT, VPT, MODE, false>(p, row, true, j0, ncons, ok, y, (i & 1) ? red1 : red0,
                                       gamma_s, no_gamma);
+  }
+  if constexpr (MODE == kModeTensor) {
+    if (p.tensor_fused) ring_tensor_tail<DT, VPT>(p, my_rows, ncons, gamma_s, abort_flag);
   }
 
   // Only after an abort can copies still be in flight: thread 0 waits for
@@ -909,93 +1079,81 @@ far_ring_kernel(const Params p, int nslot, int ncons, int stage_gamma) {
 // its y is rebuilt from the partials and the residual in the first pass's
 // order (the same bits), and its new residual is written here.
 // blockDim = (tpr, rows_per_cta); rows in grid-stride order.
-// The 8 codes of one pack.  In the usual case (a scale whose reciprocal is
-// normal) the quotient is formed as q = (y * (rinv / scale)) * (gamma + wb),
-// two multiplies per element with rs = RN(rinv * RN(1 / scale)) per row: a
-// few fp32 ulps from o / scale, nothing against the half-ulp of the 2-byte
-// format already in y here and far inside one e4m3 step.  Otherwise o is
-// formed and divided as in every other pattern.
-template <class DT>
-__device__ __forceinline__ uint2 tensor_codes(const uint4& gam, float wb, float (&y)[8], float rinv,
-                                              float rs, float scale, float inv, bool exact) {
-  float g[8];
-  pack_plus<DT>(gam, wb, g);
-  if (!exact && scale != 0.f) {
-#pragma unroll
-    for (int i = 0; i < 8; ++i) y[i] = (y[i] * rs) * g[i];
-    return make_uint2(e4m3x4(y[0], y[1], y[2], y[3]), e4m3x4(y[4], y[5], y[6], y[7]));
-  }
-#pragma unroll
-  for (int i = 0; i < 8; ++i) y[i] = (y[i] * rinv) * g[i];
-  return fp8_codes8(y, scale, inv, exact);
-}
-
+// kRows rows per thread per iteration (both rows' loads in flight before
+// either is converted); measured on the W=4 8192 x 8192 call, two rows gave
+// 179-180 us per call against 178 us with one, so one it is.
 template <class DT, int VPT>
 __global__ void __launch_bounds__(kMaxThreads)
 far_tensor_quant_kernel(const Params p) {
+  constexpr int kRows = 1;
   pdl_enter();
   const int64_t nrows = p.row_end - p.row_begin;
-  float scale = __fdiv_rn(__uint_as_float(*p.ws_amax), 448.f);
-  if (scale != scale) scale = 0.f;
-  if (blockIdx.x == 0 && threadIdx.x == 0 && threadIdx.y == 0) p.scale_out[0] = scale;
-  const float inv = __frcp_rn(scale);
-  const bool exact = needs_exact_div(scale, inv);
+  const TensorScale ts(p, *p.ws_amax);
+  const float scale = ts.scale, inv = ts.inv;
+  const bool exact = ts.exact;
   const int j0 = threadIdx.x, tpr = blockDim.x;
   const uint4* gamma = static_cast<const uint4*>(p.gamma);
+  const uint64_t drop = l2_evict_first();
+  bool ok[VPT];
+#pragma unroll
+  for (int q = 0; q < VPT; ++q) ok[q] = j0 + q * tpr < p.packs;
   const int64_t step = static_cast<int64_t>(gridDim.x) * blockDim.y;
-  for (int64_t k = static_cast<int64_t>(blockIdx.x) * blockDim.y + threadIdx.y; k < nrows; k += step) {
-    const int64_t row = call_row(p, k);
-    const int64_t rbase = row * static_cast<int64_t>(p.packs);
-    const float w = p.ws_rinv[row - p.ws_row0];
-    const bool rebuild = signbit(w);
-    const float rinv = fabsf(w);
-    const float rs = rinv * inv;
-    bool ok[VPT];
+  for (int64_t k = static_cast<int64_t>(blockIdx.x) * blockDim.y + threadIdx.y; k < nrows;
+       k += kRows * step) {
+    const bool two = kRows == 2 && k + step < nrows;
+    const int64_t ra = call_row(p, k);
+    const int64_t rb = two ? call_row(p, k + step) : ra;
+    const float wa = p.ws_rinv[ra - p.ws_row0];
+    const float wb = two ? p.ws_rinv[rb - p.ws_row0] : 0.f;
+    if (signbit(wa) || signbit(wb)) {  // a row to rebuild: each row on its own
+      tensor_quant_row<DT, VPT>(p, ra, wa, j0, tpr, ok, inv, scale, exact, drop);
+      if (two) tensor_quant_row<DT, VPT>(p, rb, wb, j0, tpr, ok, inv, scale, exact, drop);
+      continue;
+    }
+    const int64_t ba = ra * static_cast<int64_t>(p.packs), bb = rb * static_cast<int64_t>(p.packs);
+    uint4 va[VPT], vb[VPT], gv[VPT];
 #pragma unroll
-    for (int q = 0; q < VPT; ++q) ok[q] = j0 + q * tpr < p.packs;
-    if (!rebuild) {
-      // every load of the row first (this row's residual_out is only read here)
-      uint4 v[VPT], gv[VPT];
-#pragma unroll
-      for (int q = 0; q < VPT; ++q) {
-        v[q] = make_uint4(0u, 0u, 0u, 0u);
-        gv[q] = make_uint4(0u, 0u, 0u, 0u);
-        if (ok[q]) {
-          v[q] = ld_once(static_cast<const uint4*>(p.residual_out) + rbase + j0 + q * tpr);
-          gv[q] = __ldg(gamma + j0 + q * tpr);
-        }
+    for (int q = 0; q < VPT; ++q) {
+      va[q] = vb[q] = gv[q] = make_uint4(0u, 0u, 0u, 0u);
+      if (ok[q]) {
+        va[q] = ld_once_l2_hint(static_cast<const uint4*>(p.residual_out) + ba + j0 + q * tpr, drop);
+        if (two) vb[q] = ld_once_l2_hint(static_cast<const uint4*>(p.residual_out) + bb + j0 + q * tpr, drop);
+        gv[q] = __ldg(gamma + j0 + q * tpr);
       }
+    }
+    const float rinv_a = fabsf(wa), rinv_b = fabsf(wb);
+#pragma unroll
+    for (int q = 0; q < VPT; ++q) {
+      if (!ok[q]) continue;
+      float y[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      add_pack<DT>(va[q], y);  // 0 + x: the 2-byte value widened exactly
+      reinterpret_cast<uint2*>(p.quant_out)[ba + j0 + q * tpr] =
+          tensor_codes<DT>(gv[q], p.weight_bias, y, rinv_a, rinv_a * inv, scale, inv, exact);
+    }
+    if (two) {
 #pragma unroll
       for (int q = 0; q < VPT; ++q) {
         if (!ok[q]) continue;
         float y[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-        add_pack<DT>(v[q], y);  // 0 + x: the 2-byte value widened exactly
-        reinterpret_cast<uint2*>(p.quant_out)[rbase + j0 + q * tpr] =
-            tensor_codes<DT>(gv[q], p.weight_bias, y, rinv, rs, scale, inv, exact);
-      }
-    } else {
-      // the first pass's order: partials 0..W-1, then the residual
-      for (int q = 0; q < VPT; ++q) {
-        if (!ok[q]) continue;
-        const int64_t pk = rbase + j0 + q * tpr;
-        float y[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-        for (int r = 0; r < p.W; ++r) add_pack<DT>(ld_once(static_cast<const uint4*>(p.partials[r]) + pk), y);
-        if (p.residual != nullptr)
-          add_pack<DT>(ld_once_coherent(static_cast<const uint4*>(p.residual) + pk), y);
-        static_cast<uint4*>(p.residual_out)[pk] = pack8<DT>(y);
-        reinterpret_cast<uint2*>(p.quant_out)[pk] =
-            tensor_codes<DT>(__ldg(gamma + j0 + q * tpr), p.weight_bias, y, rinv, rs, scale, inv, exact);
+        add_pack<DT>(vb[q], y);
+        reinterpret_cast<uint2*>(p.quant_out)[bb + j0 + q * tpr] =
+            tensor_codes<DT>(gv[q], p.weight_bias, y, rinv_b, rinv_b * inv, scale, inv, exact);
       }
     }
   }
 }
 
-// Launch attributes: optional programmatic stream serialization (PDL) and
-// an optional cluster shape.
+// Launch attributes: optional cooperative launch, programmatic stream
+// serialization (PDL) and a cluster shape.
 struct Attrs {
-  cudaLaunchAttribute a[2];
+  cudaLaunchAttribute a[3];
   unsigned n = 0;
   Attrs(const Launch& l, int cluster) {
+    if (l.cooperative) {
+      a[n].id = cudaLaunchAttributeCooperative;
+      a[n].val.cooperative = 1;
+      ++n;
+    }
     if (l.pdl) {
       a[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
       a[n].val.programmaticStreamSerializationAllowed = 1;
@@ -1011,7 +1169,7 @@ struct Attrs {
   }
 };
 
-template <class DT, int VPT, bool SUB, bool GROUP>
+template <class DT, int VPT, bool SUB, int MODE>
 cudaError_t launch_prefill_t(const Params& p, const Launch& l, cudaStream_t s) {
   Attrs at(l, 0);
   cudaLaunchConfig_t cfg = {};
@@ -1021,7 +1179,7 @@ cudaError_t launch_prefill_t(const Params& p, const Launch& l, cudaStream_t s) {
   cfg.stream = s;
   cfg.attrs = at.a;
   cfg.numAttrs = at.n;
-  return cudaLaunchKernelEx(&cfg, far_prefill_kernel<DT, VPT, SUB, GROUP>, p);
+  return cudaLaunchKernelEx(&cfg, far_prefill_kernel<DT, VPT, SUB, MODE>, p);
 }
 
 template <class DT, int VPT>
@@ -1037,7 +1195,7 @@ cudaError_t launch_decode_t(const Params& p, const Launch& l, cudaStream_t s) {
   return cudaLaunchKernelEx(&cfg, far_decode_kernel<DT, VPT>, p);
 }
 
-template <class DT, int VPT, int MINB, bool GROUP>
+template <class DT, int VPT, int MINB, int MODE>
 cudaError_t launch_ring_t(const Params& p, const Launch& l, cudaStream_t s) {
   Attrs at(l, 0);
   cudaLaunchConfig_t cfg = {};
@@ -1047,43 +1205,51 @@ cudaError_t launch_ring_t(const Params& p, const Launch& l, cudaStream_t s) {
   cfg.stream = s;
   cfg.attrs = at.a;
   cfg.numAttrs = at.n;
-  return cudaLaunchKernelEx(&cfg, far_ring_kernel<DT, VPT, MINB, GROUP>, p, l.nslot, l.tpr,
+  return cudaLaunchKernelEx(&cfg, far_ring_kernel<DT, VPT, MINB, MODE>, p, l.nslot, l.tpr,
                             l.ring_gamma);
 }
 
-template <class DT, bool GROUP>
+template <class DT, int MODE>
 cudaError_t launch_ring_g(const Params& p, const Launch& l, cudaStream_t s) {
   const bool three = l.ring_minb >= 3;
   switch (l.vpt) {
-    case 1: return three ? launch_ring_t<DT, 1, 3, GROUP>(p, l, s) : launch_ring_t<DT, 1, 2, GROUP>(p, l, s);
-    case 2: return three ? launch_ring_t<DT, 2, 3, GROUP>(p, l, s) : launch_ring_t<DT, 2, 2, GROUP>(p, l, s);
-    case 4: return three ? launch_ring_t<DT, 4, 3, GROUP>(p, l, s) : launch_ring_t<DT, 4, 2, GROUP>(p, l, s);
-    case 8: return l.ring_minb >= 2 ? launch_ring_t<DT, 8, 2, GROUP>(p, l, s)
-                                    : launch_ring_t<DT, 8, 1, GROUP>(p, l, s);
+    case 1: return three ? launch_ring_t<DT, 1, 3, MODE>(p, l, s) : launch_ring_t<DT, 1, 2, MODE>(p, l, s);
+    case 2: return three ? launch_ring_t<DT, 2, 3, MODE>(p, l, s) : launch_ring_t<DT, 2, 2, MODE>(p, l, s);
+    case 4: return three ? launch_ring_t<DT, 4, 3, MODE>(p, l, s) : launch_ring_t<DT, 4, 2, MODE>(p, l, s);
+    case 8: return l.ring_minb >= 2 ? launch_ring_t<DT, 8, 2, MODE>(p, l, s)
+                                    : launch_ring_t<DT, 8, 1, MODE>(p, l, s);
     default: return cudaErrorInvalidConfiguration;
   }
 }
 
 template <class DT>
 cudaError_t launch_ring_dt(const Params& p, const Launch& l, cudaStream_t s) {
-  return p.pattern == kFp8Group ? launch_ring_g<DT, true>(p, l, s) : launch_ring_g<DT, false>(p, l, s);
+  switch (mode_of(p.pattern)) {
+    case kModeGroup: return launch_ring_g<DT, kModeGroup>(p, l, s);
+    case kModeTensor: return launch_ring_g<DT, kModeTensor>(p, l, s);
+    default: return launch_ring_g<DT, kModePlain>(p, l, s);
+  }
 }
 
-template <class DT, bool GROUP>
+template <class DT, int MODE>
 cudaError_t launch_prefill_g(const Params& p, const Launch& l, cudaStream_t s) {
-  if (l.tpr <= 32 && l.rows_per_cta > 1) return launch_prefill_t<DT, 1, true, GROUP>(p, l, s);
+  if (l.tpr <= 32 && l.rows_per_cta > 1) return launch_prefill_t<DT, 1, true, MODE>(p, l, s);
   switch (l.vpt) {
-    case 1: return launch_prefill_t<DT, 1, false, GROUP>(p, l, s);
-    case 2: return launch_prefill_t<DT, 2, false, GROUP>(p, l, s);
-    case 4: return launch_prefill_t<DT, 4, false, GROUP>(p, l, s);
-    case 8: return launch_prefill_t<DT, 8, false, GROUP>(p, l, s);
+    case 1: return launch_prefill_t<DT, 1, false, MODE>(p, l, s);
+    case 2: return launch_prefill_t<DT, 2, false, MODE>(p, l, s);
+    case 4: return launch_prefill_t<DT, 4, false, MODE>(p, l, s);
+    case 8: return launch_prefill_t<DT, 8, false, MODE>(p, l, s);
     default: return cudaErrorInvalidConfiguration;
   }
 }
 
 template <class DT>
 cudaError_t launch_prefill_dt(const Params& p, const Launch& l, cudaStream_t s) {
-  return p.pattern == kFp8Group ? launch_prefill_g<DT, true>(p, l, s) : launch_prefill_g<DT, false>(p, l, s);
+  switch (mode_of(p.pattern)) {
+    case kModeGroup: return launch_prefill_g<DT, kModeGroup>(p, l, s);
+    case kModeTensor: return launch_prefill_g<DT, kModeTensor>(p, l, s);
+    default: return launch_prefill_g<DT, kModePlain>(p, l, s);
+  }
 }
 
 template <class DT, int VPT>
@@ -1128,22 +1294,30 @@ cudaError_t allow_large_smem() {
     if (e == cudaSuccess)
       e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kRingSmemMax);
   };
-  set(far_ring_kernel<DT, 1, 2, false>);
-  set(far_ring_kernel<DT, 2, 2, false>);
-  set(far_ring_kernel<DT, 4, 2, false>);
-  set(far_ring_kernel<DT, 1, 3, false>);
-  set(far_ring_kernel<DT, 2, 3, false>);
-  set(far_ring_kernel<DT, 4, 3, false>);
-  set(far_ring_kernel<DT, 8, 1, false>);
-  set(far_ring_kernel<DT, 8, 2, false>);
-  set(far_ring_kernel<DT, 1, 2, true>);
-  set(far_ring_kernel<DT, 2, 2, true>);
-  set(far_ring_kernel<DT, 4, 2, true>);
-  set(far_ring_kernel<DT, 1, 3, true>);
-  set(far_ring_kernel<DT, 2, 3, true>);
-  set(far_ring_kernel<DT, 4, 3, true>);
-  set(far_ring_kernel<DT, 8, 1, true>);
-  set(far_ring_kernel<DT, 8, 2, true>);
+  set(far_ring_kernel<DT, 1, 2, kModePlain>);
+  set(far_ring_kernel<DT, 2, 2, kModePlain>);
+  set(far_ring_kernel<DT, 4, 2, kModePlain>);
+  set(far_ring_kernel<DT, 1, 3, kModePlain>);
+  set(far_ring_kernel<DT, 2, 3, kModePlain>);
+  set(far_ring_kernel<DT, 4, 3, kModePlain>);
+  set(far_ring_kernel<DT, 8, 1, kModePlain>);
+  set(far_ring_kernel<DT, 8, 2, kModePlain>);
+  set(far_ring_kernel<DT, 1, 2, kModeGroup>);
+  set(far_ring_kernel<DT, 2, 2, kModeGroup>);
+  set(far_ring_kernel<DT, 4, 2, kModeGroup>);
+  set(far_ring_kernel<DT, 1, 3, kModeGroup>);
+  set(far_ring_kernel<DT, 2, 3, kModeGroup>);
+  set(far_ring_kernel<DT, 4, 3, kModeGroup>);
+  set(far_ring_kernel<DT, 8, 1, kModeGroup>);
+  set(far_ring_kernel<DT, 8, 2, kModeGroup>);
+  set(far_ring_kernel<DT, 1, 2, kModeTensor>);
+  set(far_ring_kernel<DT, 2, 2, kModeTensor>);
+  set(far_ring_kernel<DT, 4, 2, kModeTensor>);
+  set(far_ring_kernel<DT, 1, 3, kModeTensor>);
+  set(far_ring_kernel<DT, 2, 3, kModeTensor>);
+  set(far_ring_kernel<DT, 4, 3, kModeTensor>);
+  set(far_ring_kernel<DT, 8, 1, kModeTensor>);
+  set(far_ring_kernel<DT, 8, 2, kModeTensor>);
   return e;
 }
 
@@ -1188,7 +1362,7 @@ int occ_of(int threads, int smem) {
   // the per-group instantiation is sized the same way; the plain one decides
   int n = 0;
   const cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(
-      &n, far_ring_kernel<DT, VPT, MINB, false>, threads, smem);
+      &n, far_ring_kernel<DT, VPT, MINB, kModePlain>, threads, smem);
   return e == cudaSuccess ? n : 0;
 }
 
@@ -1204,6 +1378,23 @@ int ring_occupancy_dt(int vpt, int minb, int threads, int smem) {
   }
 }
 }  // namespace
+
+int decode_occupancy(int dtype, int vpt, int threads) {
+  int n = 0;
+  cudaError_t e = cudaErrorInvalidValue;
+  const auto occ = [&](auto kern) {
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, threads, 0);
+  };
+  const bool bf = dtype == kBf16;
+  switch (vpt) {
+    case 1: bf ? occ(far_decode_kernel<Bf16T, 1>) : occ(far_decode_kernel<Fp16T, 1>); break;
+    case 2: bf ? occ(far_decode_kernel<Bf16T, 2>) : occ(far_decode_kernel<Fp16T, 2>); break;
+    case 4: bf ? occ(far_decode_kernel<Bf16T, 4>) : occ(far_decode_kernel<Fp16T, 4>); break;
+    case 8: bf ? occ(far_decode_kernel<Bf16T, 8>) : occ(far_decode_kernel<Fp16T, 8>); break;
+    default: return 0;
+  }
+  return e == cudaSuccess ? n : 0;
+}
 
 int ring_occupancy(int dtype, int vpt, int minb, int threads, int smem_bytes) {
   return dtype == kBf16 ? ring_occupancy_dt<Bf16T>(vpt, minb, threads, smem_bytes)

@@ -15,7 +15,9 @@ rows of the residual it owns (rows [r n, (r + 1) n) on rank r).  One call:
    blocks of its own rows as G separate buffers.  This is the reduce-scatter
    with its reduction moved into the kernel: the G blocks are summed in fp32
    by the epilogue kernel (W = G partials), not in the 2-byte format by the
-   collective, so the result is bit for bit the one-GPU result;
+   collective, so the result is the one-GPU result -- bit for bit when the
+   local call runs with the one-GPU call's packs per thread and threads per
+   row (far_describe_launch), else within the parity tolerances;
 2. local step: the fused epilogue on those n rows (``far_fused``), writing
    the rows' new residual (in place, or into ``residual_out``) and the
    normed outputs;
@@ -180,8 +182,8 @@ class PeerSequenceParallelEpilogue:
        ``self.partial`` (after the call, in stream order) begins.
 
     The caller writes its partial into ``self.partial`` before each call.
-    Results equal SequenceParallelEpilogue's bit for bit (the same kernel on
-    the same values).
+    Results equal SequenceParallelEpilogue's bit for bit (the same kernel
+    and launch geometry on the same values).
     """
 
     def __init__(self, group, T: int, H: int, dtype: torch.dtype, pattern: int, device, *,
