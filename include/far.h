@@ -120,7 +120,7 @@ typedef enum {
  * FAR_TENSOR_REVERSE=1|0: the second pass of per-tensor FP8 takes the rows
  * from the last one down, default 1, FAR_TENSOR_FUSED=1|0: per-tensor FP8
  * without norm_out on the ring kernel runs both passes in one cooperative
- * launch with a grid barrier between them, default 0). */
+ * launch with a grid barrier between them, default 1). */
 /*
  * Programmatic dependent launch: every kernel of this library first waits
  * (griddepcontrol.wait) until the grid it depends on has completed, then
@@ -233,18 +233,22 @@ size_t far_fp8_tensor_workspace_bytes(int64_t rows);
  * arguments as far_fused_rows; residual_out, norm_out as there.
  *
  * The scale needs every row before any code, so the call enqueues a memset
- * of the workspace's first word and two kernels.  The first reads the inputs
- * and keeps each row's 1/rms and the running amax in `workspace`.  Without
- * norm_out and with a new residual to write (a residual_out, or a residual
- * updated in place), the first kernel also writes the new residual and the
- * second forms o from it -- o = round(y) * rinv * (gamma + weight_bias),
- * round(y) being the new residual in the 2-byte format -- and writes only
- * the codes, so the inputs are read once; each code is then within one
- * step of the code of o formed from y itself, and the scale is the same.
- * Rows whose sum of squares could hide an element that overflows the format
- * (and rows with an inf or NaN input) are rebuilt from the inputs by the
- * second kernel instead.  With norm_out, or with no new residual to write,
- * the second kernel reads the inputs again and writes every output.
+ * of the workspace's first two words and two passes.  The first reads the
+ * inputs and keeps each row's 1/rms and the running amax in `workspace`.
+ * Without norm_out and with a new residual to write (a residual_out, or a
+ * residual updated in place), the first pass also writes the new residual
+ * and the second forms o from it -- o = round(y) * rinv * (gamma +
+ * weight_bias), round(y) being the new residual in the 2-byte format -- and
+ * writes only the codes, so the inputs are read once; each code is then
+ * within one step of the code of o formed from y itself, and the scale is
+ * the same.  Rows whose sum of squares could hide an element that overflows
+ * the format (and rows with an inf or NaN input) are rebuilt from the
+ * inputs by the second pass instead.  When the persistent kernel serves
+ * the call, both passes run in ONE cooperative launch whose CTAs meet at a
+ * bounded grid barrier (FAR_TENSOR_FUSED=0 in the environment at
+ * far_create splits them into two kernels); otherwise two kernels run.
+ * With norm_out, or with no new residual to write, the second pass reads
+ * the inputs again and writes every output.
  * `workspace`: device memory of at least
  * far_fp8_tensor_workspace_bytes(row_end - row_begin) bytes, 256-byte
  * aligned, overlapping no argument; its contents are scratch, and two calls

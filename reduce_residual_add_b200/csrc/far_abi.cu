@@ -400,7 +400,7 @@ far_status far_create(far_ctx** ctx, int device) {
   c.ring_threads_set = std::getenv("FAR_RING_THREADS") != nullptr;
   c.ring_slots_max = env_int("FAR_RING_SLOTS", 0);  // 0: by the 72 KiB rule
   c.tensor_reverse = env_int("FAR_TENSOR_REVERSE", 1) != 0;
-  c.tensor_fused = env_int("FAR_TENSOR_FUSED", 0) != 0;
+  c.tensor_fused = env_int("FAR_TENSOR_FUSED", 1) != 0;
   c.ring_gamma_mode = env_int("FAR_RING_GAMMA_SMEM", -1);
   if (c.ring_gamma_mode > 1) c.ring_gamma_mode = 1;
   if (c.ring_gamma_mode < -1) c.ring_gamma_mode = -1;

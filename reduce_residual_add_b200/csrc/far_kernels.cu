@@ -329,6 +329,15 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
       : "memory");
 }
 
+// The same with an L2 eviction policy for the lines it reads.
+__device__ __forceinline__ void bulk_load_hint(void* dst, const void* src, uint32_t bytes,
+                                               uint64_t* bar, uint64_t pol) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;"
+      ::"r"(smem_addr(dst)), "l"(src), "r"(bytes), "r"(smem_addr(bar)), "l"(pol)
+      : "memory");
+}
+
 
 // Programmatic dependent launch (PTX griddepcontrol): wait until the grid
 // this launch depends on has completed and its writes are visible (a no-op
@@ -869,19 +878,16 @@ struct TensorScale {
   }
 };
 
-// The fused form's second half, run by the consumer threads of a ring CTA
-// once its own rows are done: a grid barrier (every CTA is co-resident:
-// cooperative launch), then this CTA's rows again, the most recently written
-// first (their new residual is the likeliest to be still in L2), codes from
-// the stored new residual.  The wait is bounded; a CTA that gives up sets
-// the device error word and writes no codes.  Only this CTA's own rows are
-// read back, so the only data another CTA wrote is the amax word.
-template <class DT, int VPT>
-__device__ __forceinline__ void ring_tensor_tail(const Params& p, int64_t my_rows, int ncons,
-                                                 const uint4* gamma_s, volatile int* abort_flag) {
+// The fused per-tensor form's grid barrier, run by the consumer threads of a
+// ring CTA once its own rows are done: every CTA of the (cooperative, so
+// co-resident) launch arrives, then the call's amax is final.  The wait is
+// bounded; a CTA that gives up sets the device error word and its abort
+// flag (it writes no codes).  Returns false then.
+__device__ __forceinline__ bool tensor_grid_barrier(const Params& p, int ncons,
+                                                    volatile int* abort_flag) {
   consumer_bar(ncons);  // every consumer of this CTA is past its last row
   if (threadIdx.x == 0) {
-    __threadfence();    // this CTA's amax and stores before its arrival (cumulative)
+    __threadfence();    // this CTA's amax before its arrival (cumulative)
     atomicAdd(p.ws_arrive, 1u);
     const uint64_t t0 = global_ns();
     for (;;) {
@@ -896,21 +902,12 @@ __device__ __forceinline__ void ring_tensor_tail(const Params& p, int64_t my_row
     }
   }
   consumer_bar(ncons);
-  if (*abort_flag) return;
-  unsigned amax_bits;
-  asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(amax_bits) : "l"(p.ws_amax) : "memory");
-  const TensorScale ts(p, amax_bits);
-  const uint64_t drop = l2_evict_first();
-  const int j0 = threadIdx.x;
-  bool ok[VPT];
-#pragma unroll
-  for (int q = 0; q < VPT; ++q) ok[q] = j0 + q * ncons < p.packs;
-  for (int64_t i = my_rows - 1; i >= 0; --i) {
-    const int64_t row = call_row(p, blockIdx.x + i * gridDim.x);
-    const float w = *reinterpret_cast<volatile const float*>(p.ws_rinv + (row - p.ws_row0));
-    tensor_quant_row<DT, VPT, true>(p, row, w, j0, ncons, ok, ts.inv, ts.scale, ts.exact, drop,
-                                    gamma_s);
-  }
+  return !*abort_flag;
+}
+
+// Barrier between the consumers and the whole producer warp of a ring CTA.
+__device__ __forceinline__ void tail_bar(int nthreads) {
+  asm volatile("bar.sync 2, %0;" ::"r"(nthreads) : "memory");
 }
 
 // Prefill through the TMA engine: a persistent CTA per SM (or two) walks
@@ -963,15 +960,23 @@ far_ring_kernel(const Params p, int nslot, int ncons, int stage_gamma) {
   pdl_enter();
 
   if (threadIdx.x >= ncons) {
-    // producer warp: one thread issues, the rest of the warp is idle
+    // producer warp: one thread issues, the rest of the warp is idle.
+    // Copy g goes to slot g mod nslot, whose use count parity is `phase`
+    // (counters, not 64-bit divisions).
+    int slot = 0;
+    uint32_t phase = 0;
+    int64_t issued = 0;
     if (threadIdx.x == ncons) {
       const int64_t nseg = my_rows * S;
-      int64_t issued = 0;
-      // segment g is segment k of row number ord; it goes to slot g mod nslot,
-      // whose use count parity is `phase` (counters, not 64-bit divisions)
-      int slot = 0, k = 0;
-      uint32_t phase = 0;
+      // segment g is segment k of row number ord
+      int k = 0;
       int64_t ord = blockIdx.x;
+      // per-tensor FP8 reading back its new residual: the inputs, read
+      // once, leave L2 first, so that the new residual (stored evict-last)
+      // is what L2 keeps for the second pass
+      const bool drop_inputs = MODE == kModeTensor && p.tensor_stores_residual;
+      uint64_t drop = 0;
+      if constexpr (MODE == kModeTensor) drop = l2_evict_first();
       for (int64_t g = 0; g < nseg; ++g) {
         if (*abort_flag) break;
         if (!mbar_wait(&empty[slot], phase ^ 1u, abort_flag, p.wait_limit_ns)) {
@@ -984,7 +989,10 @@ far_ring_kernel(const Params p, int nslot, int ncons, int stage_gamma) {
           const unsigned char* src = static_cast<const unsigned char*>(base) +
                                      call_row(p, ord) * static_cast<int64_t>(seg_bytes);
           mbar_arrive_expect_tx(&full[slot], seg_bytes);
-          bulk_load(ring + static_cast<size_t>(slot) * seg_bytes, src, seg_bytes, &full[slot]);
+          if (drop_inputs)
+            bulk_load_hint(ring + static_cast<size_t>(slot) * seg_bytes, src, seg_bytes, &full[slot], drop);
+          else
+            bulk_load(ring + static_cast<size_t>(slot) * seg_bytes, src, seg_bytes, &full[slot]);
         }
         issued = g + 1;
         if (++slot == nslot) {
@@ -996,6 +1004,43 @@ far_ring_kernel(const Params p, int nslot, int ncons, int stage_gamma) {
           ord += gridDim.x;
         }
       }
+    }
+    if constexpr (MODE == kModeTensor) {
+      // The fused per-tensor form: once the consumers have stored this CTA's
+      // new residuals and row flags (and fenced them for the async proxy),
+      // stream the same rows back through the ring, the most recently
+      // written first: the new residual of a row, or for a flagged row all
+      // its input segments.  The copies run ahead while the consumers wait
+      // at the grid barrier.
+      if (p.tensor_fused) {
+        tail_bar(ncons + 32);
+        if (threadIdx.x == ncons) {
+          for (int64_t i = my_rows - 1; i >= 0 && !*abort_flag; --i) {
+            const int64_t row = call_row(p, blockIdx.x + i * gridDim.x);
+            const bool rebuild = signbit(*reinterpret_cast<volatile const float*>(p.ws_rinv + (row - p.ws_row0)));
+            const int nseg = rebuild ? S : 1;
+            for (int k = 0; k < nseg; ++k) {
+              if (!mbar_wait(&empty[slot], phase ^ 1u, abort_flag, p.wait_limit_ns)) {
+                if (!*abort_flag) atomicOr(&g_far_error, kErrWaitEmpty);
+                *abort_flag = 1;
+                break;
+              }
+              const void* base = !rebuild ? p.residual_out : (k < p.W ? p.partials[k] : p.residual);
+              mbar_arrive_expect_tx(&full[slot], seg_bytes);
+              bulk_load_hint(ring + static_cast<size_t>(slot) * seg_bytes,
+                             static_cast<const unsigned char*>(base) + row * static_cast<int64_t>(seg_bytes),
+                             seg_bytes, &full[slot], l2_evict_first());
+              ++issued;
+              if (++slot == nslot) {
+                slot = 0;
+                phase ^= 1u;
+              }
+            }
+          }
+        }
+      }
+    }
+    if (threadIdx.x == ncons) {
       *issued_count = issued;  // read by the drain below
       __threadfence_block();
       *producer_done = 1;
@@ -1046,7 +1091,57 @@ far_ring_kernel(const Params p, int nslot, int ncons, int stage_gamma) {
                                       gamma_s, no_gamma);
   }
   if constexpr (MODE == kModeTensor) {
-    if (p.tensor_fused) ring_tensor_tail<DT, VPT>(p, my_rows, ncons, gamma_s, abort_flag);
+    if (p.tensor_fused) {
+      // this thread's new-residual stores, before the producer's bulk copies read them
+      asm volatile("fence.proxy.async.global;" ::: "memory");
+      tail_bar(ncons + 32);
+      if (tensor_grid_barrier(p, ncons, abort_flag)) {
+        unsigned amax_bits;
+        asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(amax_bits) : "l"(p.ws_amax) : "memory");
+        const TensorScale ts(p, amax_bits);
+        for (int64_t i = my_rows - 1; i >= 0; --i) {
+          const int64_t row = call_row(p, blockIdx.x + i * gridDim.x);
+          const float w = *reinterpret_cast<volatile const float*>(p.ws_rinv + (row - p.ws_row0));
+          const bool rebuild = signbit(w);
+          const int nseg = rebuild ? S : 1;
+          float y[VPT][8];
+          bool ok[VPT];
+#pragma unroll
+          for (int q = 0; q < VPT; ++q) {
+            ok[q] = (j0 + q * ncons) < p.packs;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) y[q][e] = 0.f;
+          }
+          for (int k = 0; k < nseg; ++k) {
+            if (!*abort_flag && !mbar_wait(&full[slot], phase, abort_flag, p.wait_limit_ns)) {
+              if (!*abort_flag) atomicOr(&g_far_error, kErrWaitFull);
+              *abort_flag = 1;
+            }
+            const uint4* seg = reinterpret_cast<const uint4*>(ring + static_cast<size_t>(slot) * seg_bytes);
+#pragma unroll
+            for (int q = 0; q < VPT; ++q)
+              if (ok[q]) add_pack<DT>(seg[j0 + q * ncons], y[q]);  // 0 + x: exact widening
+            __syncwarp();
+            if ((threadIdx.x & 31) == 0) mbar_arrive(&empty[slot]);
+            if (++slot == nslot) {
+              slot = 0;
+              phase ^= 1u;
+            }
+          }
+          const int64_t rbase = row * static_cast<int64_t>(p.packs);
+          const float rinv = fabsf(w);
+#pragma unroll
+          for (int q = 0; q < VPT; ++q) {
+            if (!ok[q]) continue;
+            const int64_t pk = rbase + j0 + q * ncons;
+            if (rebuild) static_cast<uint4*>(p.residual_out)[pk] = pack8<DT>(y[q]);
+            reinterpret_cast<uint2*>(p.quant_out)[pk] =
+                tensor_codes<DT>(gamma_pack(p, gamma_s, j0 + q * ncons), p.weight_bias, y[q], rinv,
+                                 rinv * ts.inv, ts.scale, ts.inv, ts.exact);
+          }
+        }
+      }
+    }
   }
 
   // Only after an abort can copies still be in flight: thread 0 waits for

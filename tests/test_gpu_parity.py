@@ -56,8 +56,10 @@ def kctx():
     and the direct-load kernel."""
     any_rows = {"FAR_RING_MIN_ROWS": "1"}
     out = {"ring": _ctx_with_env(dict(any_rows)),
-           # per-tensor FP8: both passes in one cooperative launch
+           # per-tensor FP8: both passes in one cooperative launch (the
+           # default), and in two kernels
            "ring_fused": _ctx_with_env(dict(any_rows, FAR_TENSOR_FUSED="1")),
+           "ring_two": _ctx_with_env(dict(any_rows, FAR_TENSOR_FUSED="0")),
            "ring256": _ctx_with_env(dict(any_rows, FAR_RING_THREADS="256", FAR_RING_CTAS_PER_SM="1")),
            "ring3": _ctx_with_env(dict(any_rows, FAR_RING_CTAS_PER_SM="3")),
            "ring2": _ctx_with_env(dict(any_rows, FAR_RING_CTAS_PER_SM="2", FAR_RING_THREADS="256")),
@@ -488,7 +490,7 @@ def test_chained_calls_read_completed_outputs(kctx, ctx, kern):
 # ---------------------------------------------------------------------------
 
 @pytest.mark.parametrize("norm", [True, False], ids=["norm_out", "codes_from_new_residual"])
-@pytest.mark.parametrize("kern", ["ring", "ring_fused", "direct", "auto"])
+@pytest.mark.parametrize("kern", ["ring_fused", "ring_two", "direct", "auto"])
 @pytest.mark.parametrize("case", [
     (2, 8, 64, "bf16", True, 0.0),
     (8, 5, 4096, "bf16", True, 0.0),        # decode-sized: never the cluster kernel
@@ -511,14 +513,15 @@ def test_per_tensor_fp8(kctx, ctx, case, kern, norm):
     assert st["quant_out"][1] > 0.95                            # most codes exact
 
 
-@pytest.mark.parametrize("kern", ["ring_fused", "ring", "auto"])
+@pytest.mark.parametrize("kern", ["ring_fused", "ring_two", "auto"])
 @pytest.mark.parametrize("in_place", [False, True])
 def test_per_tensor_fp8_rebuilt_rows(kctx, ctx, in_place, kern):
     """Codes from the stored new residual: rows that may overflow the format
     (fp16 sums past 65504, whose new residual is +inf) and rows with an inf
     or NaN input are not stored by the first pass; the second pass rebuilds
     their y from the inputs, in place too (the residual is still intact).
-    "ring_fused": both passes in one launch; "ring", "auto": two kernels."""
+    "ring_fused": both passes in one launch; "ring_two", "auto" (300 rows:
+    the one-CTA kernel): two kernels."""
     c = ctx if kern == "auto" else kctx[kern]
     T, H = 300, 4096
     inp = random_inputs(4, T, H, dtype="fp16", seed=93)
