@@ -109,7 +109,7 @@ typedef enum {
  * FAR_DECODE_MAX_ROWS, FAR_FORCE_REGIME=decode|prefill, FAR_DECODE_CLUSTER
  * (CTAs per row; default by rule),
  * FAR_PREFILL_THREADS, FAR_PREFILL_KERNEL=1 ring | 0 direct,
- * FAR_RING_CTAS_PER_SM=1..4, FAR_RING_THREADS: consumer threads per ring
+ * FAR_RING_CTAS_PER_SM=1..8, FAR_RING_THREADS: consumer threads per ring
  * CTA, at most 256, FAR_RING_SLOTS: row-segment slots per ring CTA (2..32),
  * FAR_RING_GAMMA_SMEM=1|0: gamma staged in shared memory or read through
  * L1 (each replaces its part of the default geometry, which follows rules

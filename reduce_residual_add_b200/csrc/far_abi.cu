@@ -157,8 +157,9 @@ void plan_decode(int packs, int cluster_pref, far::Launch* l) {
 int ring_occ_cached(const far_ctx* ctx, int dtype, int vpt, int minb, int threads, int smem);
 
 // Ring geometry.  Every rule was measured on B200 against its alternatives
-// (fractions of the measured HBM copy bandwidth) and is used only where it
-// won.
+// (fractions of the measured HBM copy bandwidth, static FP8, bf16, W = 2, 4
+// and 8 at H = 2048-16384, about 768 MiB of inputs per call) and is used
+// only where it won.
 //
 // Consumers: the fewest packs per thread (1, 2, 4, 8) that keep within
 // ring_threads (256), plus one producer warp.  Two exceptions:
@@ -166,27 +167,41 @@ int ring_occ_cached(const far_ctx* ctx, int dtype, int vpt, int minb, int thread
 //    thread (H=4096, W=4: 128-thread CTAs, 97 vs 85 %);
 //  * rows of at most 256 packs (H <= 2048) take at most 128 consumers.
 //
-// CTAs per SM, gamma and slots: 3 CTAs per SM (registers capped at 72) for
-// rows of at most 6 segments (W=4 + residual: 95.5 vs 93.3 % with 2), else
-// 2 (W=8 + residual: 89.1 vs 87.9 % with 3); gamma staged in shared memory;
-// about 72 KiB of row-segment slots per CTA, as many as fit a 1/(CTAs per
-// SM) share of the SM's 228 KiB, less the 1 KiB the system keeps per CTA.
-// Exceptions:
-//  * H <= 2048: 4 CTAs per SM (W=2..8: 77-99 vs 63-80 %); likewise
-//    H <= 5120 with at most 6 segments and no norm_out (W=2 / 4, H=3072,
-//    4096, 5120: 92-97 vs 78-91 %; with norm_out it lost);
+// CTAs per SM and slots.  What pays is many CTAs (consumer warps to hide
+// the per-row latency) with few row-segment slots each: about 96 KiB of
+// slots per SM in all.  More slots in flight lost everywhere (W=8,
+// H=3072: 4 slots 99.8 %, 6 slots 97.0, 8 slots 92.5, at 4 CTAs per SM).
+// By row length (packs = H / 8), CTAs per SM x slots per CTA:
+//  * <= 256 packs: 6 x 4, with norm_out 4 x 6 (W=2/4/8: 93-100 vs 78-97 %
+//    for the previous 4 x 12);
+//  * <= 384: 4 x 4, with norm_out 3 x 4 (94-100 vs 83-93 %);
+//  * <= 512: 4 x 3, 3 x 4 when norm_out is written or the row has more
+//    than 6 segments (92-101 vs 90-100 %);
+//  * <= 640: 4 x 3 (4 x 4 for at most 3 segments), with norm_out 4 x 2
+//    (90-99 vs 88-97 %);
+//  * <= 768: 4 x 2, with norm_out 2 x 4 (95-97 vs 92-97 %);
+//  * <= 896: 2 x 4, 3 x 3 for 4-6 segments, with norm_out 3 x 2 (92-98 vs
+//    83-97 %);
+//  * <= 1024 (4 packs per thread): 3 x 3 for 5 or 6 segments (W=4 + residual,
+//    the c4 shape: 97.4 %), else 2 x 4 (W=2: 98.8 vs 84.0 %); with norm_out
+//    and at most 6 segments of at least 16 KiB, 2 CTAs per SM with gamma
+//    read through L1 and about 96 KiB of slots (W=3..5: 97-102 vs 87-94 %);
 //  * 8 packs per thread (H >= 12288): 2 CTAs per SM, with the build whose
-//    registers are sized for two (H=12288, W=2..8: 80-93 vs 58-84 % at one
-//    CTA); but one CTA per SM with 6 slots when the row has more than 6
-//    segments and fewer than 3 slots fit the 2-CTA share (H=16384, W=8:
-//    92 / 95 vs 89 / 90 % without / with norm_out);
-//  * norm_out written, at most 6 segments of at least 16 KiB: 2 CTAs per
-//    SM, gamma read through L1, about 96 KiB of slots (W=3..5, H=8192:
-//    97-102 vs 87-94 %);
-//  * norm_out written, at most 6 segments of 10-12 KiB: 2 CTAs per SM
-//    (H=5120 / 6144: 95-101 vs 84-87 %);
-//  * fewer than 3 slots fit (below 8 packs per thread): 2 CTAs per SM with
-//    gamma through L1.
+//    registers are sized for two, about 72 KiB of slots (H=12288, W=2..8:
+//    80-93 vs 58-84 % at one CTA); but one CTA per SM with 6 slots when the
+//    row has more than 6 segments and fewer than 3 slots fit the 2-CTA share
+//    (H=16384, W=8: 87-90 %).
+// Per-group FP8 (more work per row, and more registers) keeps the rule that
+// won for it: about 72 KiB of slots per CTA, 3 CTAs per SM for rows of at
+// most 6 segments, else 2; 4 for rows of at most 256 packs and, without
+// norm_out, up to 640 packs with at most 6 segments; with norm_out and at
+// most 6 segments, 2 CTAs per SM for segments of 10-12 KiB, and for
+// segments of at least 16 KiB 2 with gamma through L1 and about 96 KiB of
+// slots (W=4 / 8 at H=4096 / 7168, with and without norm_out: mean 90.3
+// against 86.5 % with the rule above).
+// Gamma is staged in shared memory unless said otherwise; where the slots
+// asked for do not fit, as many as fit; below 2 (below 3 for the byte
+// targets), the rule falls back to 2 CTAs per SM with gamma through L1.
 //
 // Environment overrides (FAR_RING_CTAS_PER_SM, FAR_RING_THREADS,
 // FAR_RING_SLOTS, FAR_RING_GAMMA_SMEM) replace the rule they name.  The grid
@@ -194,7 +209,7 @@ int ring_occ_cached(const far_ctx* ctx, int dtype, int vpt, int minb, int thread
 // confirms), fewer for fewer rows.  Returns false (the direct kernel runs)
 // when fewer than two slots fit or the configuration cannot be resident.
 bool plan_ring(const far_ctx* ctx, int packs, int64_t rows, int dtype, int segs, bool norm,
-               far::Launch* l) {
+               bool group, far::Launch* l) {
   if (packs <= 32) return false;
   const int seg = packs * 16;
   const bool small_rows = packs <= 256;  // H <= 2048
@@ -205,44 +220,74 @@ bool plan_ring(const far_ctx* ctx, int packs, int64_t rows, int dtype, int segs,
   const int tpr = (((packs + vpt - 1) / vpt) + 31) / 32 * 32;
   if (tpr > far::kRingMaxConsumers) return false;
 
-  int n_req = segs <= 6 ? 3 : 2;
+  int n_req = 2;
   bool gamma_smem = true;
-  int target = 72 * 1024;  // slot bytes per CTA
+  int want = 0;            // slots per CTA (0: by `target` bytes)
+  int target = 72 * 1024;  // slot bytes per CTA when want == 0
   if (vpt >= 8) {
     // 8 packs per thread: 2 CTAs per SM (a build with a few spilled
     // registers), unless the row has many segments and fewer than 3 slots
     // would fit: then one CTA per SM, as all its registers allow, 6 slots
-    n_req = 2;
     if (segs > 6 && ctx->ring_slots_max == 0 &&
         (228 * 1024 / 2 - 1024 - 1024) / seg - 1 < 3) {
       n_req = 1;
       target = 6 * seg;
     }
-  } else if (small_rows || (!norm && segs <= 6 && packs <= 640)) {
+  } else if (group) {
+    // per-group FP8 (more work per row): about 72 KiB of slots per CTA
+    n_req = segs <= 6 ? 3 : 2;
+    if (packs <= 256 || (!norm && segs <= 6 && packs <= 640)) {
+      n_req = 4;
+    } else if (norm && segs <= 6 && seg >= 16 * 1024) {
+      n_req = 2;
+      gamma_smem = false;
+      target = 96 * 1024;
+    } else if (norm && segs <= 6 && seg >= 10 * 1024 && seg <= 12 * 1024) {
+      n_req = 2;
+    }
+  } else if (packs <= 256) {
+    n_req = norm ? 4 : 6;
+    want = norm ? 6 : 4;
+  } else if (packs <= 384) {
+    n_req = norm ? 3 : 4;
+    want = 4;
+  } else if (packs <= 512) {
+    n_req = (norm || segs > 6) ? 3 : 4;
+    want = (norm || segs > 6) ? 4 : 3;
+  } else if (packs <= 640) {
     n_req = 4;
+    want = norm ? 2 : (segs <= 3 ? 4 : 3);
+  } else if (packs <= 768) {
+    n_req = norm ? 2 : 4;
+    want = norm ? 4 : 2;
+  } else if (packs <= 896) {
+    const bool mid = !norm && segs >= 4 && segs <= 6;
+    n_req = norm || mid ? 3 : 2;
+    want = norm ? 2 : (mid ? 3 : 4);
   } else if (norm && segs <= 6 && seg >= 16 * 1024) {
-    n_req = 2;
     gamma_smem = false;
     target = 96 * 1024;
-  } else if (norm && segs <= 6 && seg >= 10 * 1024 && seg <= 12 * 1024) {
-    n_req = 2;
+  } else if (segs == 5 || segs == 6) {
+    n_req = 3;
+    want = 3;
+  } else {
+    want = 4;
   }
   if (ctx->ring_ctas_per_sm > 0) n_req = ctx->ring_ctas_per_sm;
   if (ctx->ring_gamma_mode >= 0) gamma_smem = ctx->ring_gamma_mode != 0;
-  auto fit = [&](int n, bool gs, int bytes) {
+  auto fit = [&](int n, bool gs, int bytes, int slots) {
     int per_cta = 228 * 1024 / n - 1024;
     if (per_cta > far::kRingSmemMax) per_cta = far::kRingSmemMax;
-    int ns = ctx->ring_slots_max > 0 ? ctx->ring_slots_max : bytes / seg;
+    int ns = ctx->ring_slots_max > 0 ? ctx->ring_slots_max : (slots > 0 ? slots : bytes / seg);
     if (ns > 32) ns = 32;
     while (ns >= 2 && far::ring_header_bytes(ns) + (ns + (gs ? 1 : 0)) * seg > per_cta) --ns;
     return ns;
   };
-  int nslot = fit(n_req, gamma_smem, target);
-  if (nslot < 3 && vpt < 8 && ctx->ring_ctas_per_sm == 0 && ctx->ring_gamma_mode < 0) {
+  int nslot = fit(n_req, gamma_smem, target, want);
+  if (nslot < (want > 0 ? 2 : 3) && vpt < 8 && ctx->ring_ctas_per_sm == 0 && ctx->ring_gamma_mode < 0) {
     n_req = 2;
     gamma_smem = false;
-    target = 96 * 1024;
-    nslot = fit(n_req, gamma_smem, target);
+    nslot = fit(n_req, gamma_smem, 96 * 1024, 0);
   }
   if (nslot < 2) return false;
   const int gsegs = gamma_smem ? 1 : 0;
@@ -284,7 +329,8 @@ int ring_occ_cached(const far_ctx* ctx, int dtype, int vpt, int minb, int thread
 
 // segs = row segments read per row: W partials, plus the residual if any;
 // norm: the call writes norm_out.
-far::Launch plan(const far_ctx* ctx, int64_t rows, int64_t H, int dtype, int segs, bool norm) {
+far::Launch plan(const far_ctx* ctx, int64_t rows, int64_t H, int dtype, int segs, bool norm,
+                 bool group = false) {
   const int packs = static_cast<int>(H / far::kPackElems);
   far::Launch l{};
   bool decode;
@@ -338,7 +384,7 @@ far::Launch plan(const far_ctx* ctx, int64_t rows, int64_t H, int dtype, int seg
       const int per_cta = (4096 / packs > 8) ? 4096 / packs : 8;
       min_rows = static_cast<int64_t>(per_cta) * ctx->sm_count * 2;
     }
-    if (ctx->prefill_kernel == 1 && rows >= min_rows) plan_ring(ctx, packs, rows, dtype, segs, norm, &l);
+    if (ctx->prefill_kernel == 1 && rows >= min_rows) plan_ring(ctx, packs, rows, dtype, segs, norm, group, &l);
   }
   l.pdl = ctx->pdl;
   return l;
@@ -395,7 +441,7 @@ far_status far_create(far_ctx** ctx, int device) {
   c.prefill_kernel = env_int("FAR_PREFILL_KERNEL", 1) != 0 ? 1 : 0;
   c.ring_ctas_per_sm = env_int("FAR_RING_CTAS_PER_SM", 0);  // 0: by segments per row
   if (c.ring_ctas_per_sm < 0) c.ring_ctas_per_sm = 0;
-  if (c.ring_ctas_per_sm > 4) c.ring_ctas_per_sm = 4;
+  if (c.ring_ctas_per_sm > 8) c.ring_ctas_per_sm = 8;
   c.ring_threads = env_int("FAR_RING_THREADS", 256);  // at most kRingMaxConsumers
   c.ring_threads_set = std::getenv("FAR_RING_THREADS") != nullptr;
   c.ring_slots_max = env_int("FAR_RING_SLOTS", 0);  // 0: by the 72 KiB rule
@@ -983,7 +1029,7 @@ far_status far_fused_fp8_group(far_ctx* ctx, int64_t row_begin, int64_t row_end,
   // a group must sit on consecutive lanes of one warp: not the cluster kernel,
   // whose per-CTA slices need not start on a group boundary
   far::Launch whole = plan(ctx, row_end - row_begin, H, dtype, W + (residual != nullptr ? 1 : 0),
-                   norm_out != nullptr);
+                   norm_out != nullptr, true);
   if (whole.regime == FAR_REGIME_DECODE) {
     plan_prefill(static_cast<int>(H / far::kPackElems), ctx->prefill_threads, &whole);
     whole.grid = (row_end - row_begin + whole.rows_per_cta - 1) / whole.rows_per_cta;
@@ -1117,7 +1163,7 @@ far_status far_fused_host(far_ctx* ctx, const void* const* partials, int W, cons
     p.wait_limit_ns = ctx->wait_limit_ns;
     p.stall_segment = ctx->stall_segment;
     far::Launch l = plan(ctx, n, H, dtype, W + (residual != nullptr ? 1 : 0),
-                          norm_out != nullptr);
+                          norm_out != nullptr, group);
     if (group) {
       p.group_lanes = group_size / far::kPackElems;
       p.groups_per_row = static_cast<int>(H / group_size);

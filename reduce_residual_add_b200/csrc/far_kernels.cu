@@ -1014,29 +1014,43 @@ far_ring_kernel(const Params p, int nslot, int ncons, int stage_gamma) {
       // at the grid barrier.
       if (p.tensor_fused) {
         tail_bar(ncons + 32);
-        if (threadIdx.x == ncons) {
-          for (int64_t i = my_rows - 1; i >= 0 && !*abort_flag; --i) {
-            const int64_t row = call_row(p, blockIdx.x + i * gridDim.x);
-            const bool rebuild = signbit(*reinterpret_cast<volatile const float*>(p.ws_rinv + (row - p.ws_row0)));
-            const int nseg = rebuild ? S : 1;
-            for (int k = 0; k < nseg; ++k) {
-              if (!mbar_wait(&empty[slot], phase ^ 1u, abort_flag, p.wait_limit_ns)) {
-                if (!*abort_flag) atomicOr(&g_far_error, kErrWaitEmpty);
-                *abort_flag = 1;
-                break;
-              }
-              const void* base = !rebuild ? p.residual_out : (k < p.W ? p.partials[k] : p.residual);
-              mbar_arrive_expect_tx(&full[slot], seg_bytes);
-              bulk_load_hint(ring + static_cast<size_t>(slot) * seg_bytes,
-                             static_cast<const unsigned char*>(base) + row * static_cast<int64_t>(seg_bytes),
-                             seg_bytes, &full[slot], l2_evict_first());
-              ++issued;
-              if (++slot == nslot) {
-                slot = 0;
-                phase ^= 1u;
+        // The whole warp reads the row flags, 32 rows per load (one row per
+        // lane), so that lane 0 does not wait on one load per row.
+        const int lane = threadIdx.x - ncons;
+        const uint64_t drop_tail = l2_evict_first();
+        for (int64_t i0 = my_rows - 1; i0 >= 0; i0 -= 32) {
+          if (__shfl_sync(0xffffffffu, lane == 0 ? *abort_flag : 0, 0)) break;
+          bool flagged = false;
+          if (i0 - lane >= 0) {
+            const int64_t r = call_row(p, blockIdx.x + (i0 - lane) * gridDim.x);
+            flagged = signbit(*reinterpret_cast<volatile const float*>(p.ws_rinv + (r - p.ws_row0)));
+          }
+          const unsigned rebuild_mask = __ballot_sync(0xffffffffu, flagged);
+          if (lane == 0) {
+            for (int j = 0; j < 32 && i0 - j >= 0 && !*abort_flag; ++j) {
+              const int64_t row = call_row(p, blockIdx.x + (i0 - j) * gridDim.x);
+              const bool rebuild = (rebuild_mask >> j) & 1u;
+              const int nseg = rebuild ? S : 1;
+              for (int k = 0; k < nseg; ++k) {
+                if (!mbar_wait(&empty[slot], phase ^ 1u, abort_flag, p.wait_limit_ns)) {
+                  if (!*abort_flag) atomicOr(&g_far_error, kErrWaitEmpty);
+                  *abort_flag = 1;
+                  break;
+                }
+                const void* base = !rebuild ? p.residual_out : (k < p.W ? p.partials[k] : p.residual);
+                mbar_arrive_expect_tx(&full[slot], seg_bytes);
+                bulk_load_hint(ring + static_cast<size_t>(slot) * seg_bytes,
+                               static_cast<const unsigned char*>(base) + row * static_cast<int64_t>(seg_bytes),
+                               seg_bytes, &full[slot], drop_tail);
+                ++issued;
+                if (++slot == nslot) {
+                  slot = 0;
+                  phase ^= 1u;
+                }
               }
             }
           }
+          __syncwarp();
         }
       }
     }
@@ -1099,9 +1113,18 @@ far_ring_kernel(const Params p, int nslot, int ncons, int stage_gamma) {
         unsigned amax_bits;
         asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(amax_bits) : "l"(p.ws_amax) : "memory");
         const TensorScale ts(p, amax_bits);
+        // each warp reads the stored rinv of 32 rows per load (lane l: the
+        // l-th row of the chunk) and hands them out by shuffle
+        const int lane = threadIdx.x & 31;
+        float w_lane = 0.f;
         for (int64_t i = my_rows - 1; i >= 0; --i) {
+          const int j = static_cast<int>((my_rows - 1 - i) & 31);
+          if (j == 0 && i - lane >= 0) {
+            const int64_t r = call_row(p, blockIdx.x + (i - lane) * gridDim.x);
+            w_lane = *reinterpret_cast<volatile const float*>(p.ws_rinv + (r - p.ws_row0));
+          }
           const int64_t row = call_row(p, blockIdx.x + i * gridDim.x);
-          const float w = *reinterpret_cast<volatile const float*>(p.ws_rinv + (row - p.ws_row0));
+          const float w = __shfl_sync(0xffffffffu, w_lane, j);
           const bool rebuild = signbit(w);
           const int nseg = rebuild ? S : 1;
           float y[VPT][8];

@@ -403,18 +403,24 @@ def test_launch_plan(ctx):
     assert (c4["threads_per_cta"] - 32) * c4["packs_per_thread"] * 8 >= 8192
     assert d(1200, 8192, 4)["kernel"] == 0
     sms = torch.cuda.get_device_properties(0).multi_processor_count
-    # few segments: 3 CTAs per SM, gamma in shared memory
-    assert (c4["grid_ctas"], c4["ring_gamma_smem"]) == (3 * sms, 1)
+    # 5-6 segments of 1024 packs: 3 CTAs per SM x 3 slots, gamma in shared memory
+    assert (c4["grid_ctas"], c4["ring_gamma_smem"], c4["ring_slots"]) == (3 * sms, 1, 3)
+    # ... 3 segments: 2 CTAs per SM x 4 slots
+    w2 = d(8192, 8192, 2)
+    assert (w2["grid_ctas"], w2["ring_gamma_smem"], w2["ring_slots"]) == (2 * sms, 1, 4)
     # ... but with norm_out, 2 CTAs per SM, gamma through L1, ~96 KiB of slots
     c4n = d(8192, 8192, 4, norm=True)
     assert (c4n["grid_ctas"], c4n["ring_gamma_smem"], c4n["ring_slots"]) == (2 * sms, 0, 6)
-    # many segments: 2 CTAs per SM, gamma in shared memory, ~72 KiB of slots
+    # many segments of 896 packs: 2 CTAs per SM x 4 slots, gamma in shared memory
     c5 = d(4096, 7168, 8)
-    assert (c5["grid_ctas"], c5["ring_gamma_smem"], c5["ring_slots"]) == (2 * sms, 1, 5)
+    assert (c5["grid_ctas"], c5["ring_gamma_smem"], c5["ring_slots"]) == (2 * sms, 1, 4)
+    # rows of at most 384 packs: 4 CTAs per SM x 4 slots, whatever the segments
+    h3 = d(32768, 3072, 8)
+    assert (h3["grid_ctas"], h3["ring_slots"]) == (4 * sms, 4)
     # H=4096 with few segments: 4 packs per thread (128 consumers), and
-    # without norm_out 4 CTAs per SM (3 with it)
+    # without norm_out 4 CTAs per SM x 3 slots (3 CTAs with it)
     h4 = d(16384, 4096, 4)
-    assert (h4["packs_per_thread"], h4["threads_per_cta"], h4["grid_ctas"]) == (4, 160, 4 * sms)
+    assert (h4["packs_per_thread"], h4["threads_per_cta"], h4["grid_ctas"], h4["ring_slots"]) == (4, 160, 4 * sms, 3)
     assert d(16384, 4096, 4, norm=True)["grid_ctas"] == 3 * sms
     # 8 packs per thread: 2 CTAs per SM, gamma in shared memory ...
     h16 = d(8192, 16384, 2)
@@ -422,12 +428,17 @@ def test_launch_plan(ctx):
     # ... but one CTA per SM with 6 slots for many segments of which only 2 would fit
     h16w8 = d(8192, 16384, 8)
     assert (h16w8["grid_ctas"], h16w8["ring_gamma_smem"], h16w8["ring_slots"]) == (sms, 1, 6)
-    # rows of at most 256 packs: 128 consumers, 4 CTAs per SM
+    # rows of at most 256 packs: 128 consumers, 6 CTAs per SM x 4 slots
+    # (4 x 6 with norm_out)
     h2 = d(32768, 2048, 4)
-    assert (h2["threads_per_cta"], h2["packs_per_thread"], h2["grid_ctas"]) == (160, 2, 4 * sms)
-    # norm_out with 10-12 KiB segments: 2 CTAs per SM, gamma in shared memory
+    assert (h2["threads_per_cta"], h2["packs_per_thread"], h2["grid_ctas"], h2["ring_slots"]) == (160, 2, 6 * sms, 4)
+    h2n = d(32768, 2048, 4, norm=True)
+    assert (h2n["grid_ctas"], h2n["ring_slots"]) == (4 * sms, 6)
+    # 768 packs: 4 CTAs per SM x 2 slots; with norm_out 2 x 4
     h6 = d(8192, 6144, 4, norm=True)
-    assert (h6["grid_ctas"], h6["ring_gamma_smem"]) == (2 * sms, 1)
+    assert (h6["grid_ctas"], h6["ring_gamma_smem"], h6["ring_slots"]) == (2 * sms, 1, 4)
+    h6p = d(8192, 6144, 4)
+    assert (h6p["grid_ctas"], h6p["ring_slots"]) == (4 * sms, 2)
     tiny = d(8, 64, 2)
     assert tiny["regime"] == far.FAR_REGIME_PREFILL and tiny["rows_per_cta"] > 1
 
