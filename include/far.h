@@ -233,7 +233,7 @@ size_t far_fp8_tensor_workspace_bytes(int64_t rows);
  * arguments as far_fused_rows; residual_out, norm_out as there.
  *
  * The scale needs every row before any code, so the call enqueues a memset
- * of the workspace's first two words and two passes.  The first reads the
+ * of the workspace's first four words and two passes.  The first reads the
  * inputs and keeps each row's 1/rms and the running amax in `workspace`.
  * Without norm_out and with a new residual to write (a residual_out, or a
  * residual updated in place), the first pass also writes the new residual
@@ -244,9 +244,11 @@ size_t far_fp8_tensor_workspace_bytes(int64_t rows);
  * the same.  Rows whose sum of squares could hide an element that overflows
  * the format (and rows with an inf or NaN input) are rebuilt from the
  * inputs by the second pass instead.  When the persistent kernel serves
- * the call, both passes run in ONE cooperative launch whose CTAs meet at a
- * bounded grid barrier (FAR_TENSOR_FUSED=0 in the environment at
- * far_create splits them into two kernels); otherwise two kernels run.
+ * the call, both passes run in ONE cooperative launch: its CTAs take the
+ * first pass's rows one at a time from a counter in the workspace, meet at
+ * a bounded grid barrier, then write the codes (FAR_TENSOR_FUSED=0 in the
+ * environment at far_create splits them into two kernels); otherwise two
+ * kernels run.
  * With norm_out, or with no new residual to write, the second pass reads
  * the inputs again and writes every output.
  * `workspace`: device memory of at least

@@ -712,6 +712,7 @@ far_status far_fused_fp8_tensor_launch(far_ctx* ctx, int64_t row_begin, int64_t 
   p.stall_segment = ctx->stall_segment;
   p.ws_amax = static_cast<unsigned*>(workspace);
   p.ws_arrive = p.ws_amax + 1;
+  p.ws_claim = p.ws_amax + 2;
   p.ws_rinv = reinterpret_cast<float*>(static_cast<unsigned char*>(workspace) + 256);
   p.ws_row0 = row_begin;
   const bool from_residual = norm_out == nullptr && p.residual_out != nullptr;
@@ -727,16 +728,17 @@ far_status far_fused_fp8_tensor_launch(far_ctx* ctx, int64_t row_begin, int64_t 
     whole.grid = (row_end - row_begin + whole.rows_per_cta - 1) / whole.rows_per_cta;
     whole.pdl = ctx->pdl;
   }
-  // the amax word and the grid barrier's arrival count start at zero
-  cudaError_t e = cudaMemsetAsync(workspace, 0, 2 * sizeof(unsigned), s);
+  // the amax word, the grid barrier's arrival count and the row counter
+  // start at zero
+  cudaError_t e = cudaMemsetAsync(workspace, 0, 4 * sizeof(unsigned), s);
   if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync");
   far::Launch first = whole;
   first.pdl = 0;  // it must see the memset above
   p.pattern = far::kTensorAmax;
   // With the ring kernel (persistent CTAs, all co-resident by construction)
   // and the codes formed from the stored new residual, both passes run in
-  // one cooperative launch: each CTA meets the others at a grid barrier after
-  // its rows, then writes its own rows' codes, newest first.
+  // one cooperative launch: the CTAs take first-pass rows from a counter,
+  // meet at a grid barrier, then write the codes, the rows taken last first.
   const bool fused = ctx->tensor_fused && from_residual && first.regime == FAR_REGIME_PREFILL &&
                      first.kernel == 1 &&
                      row_end - row_begin <= 0x7fffffff;

@@ -54,10 +54,12 @@ struct Params {
   int reverse;                  // take the rows from row_end - 1 down to row_begin
   int tensor_stores_residual;   // per-tensor FP8, first pass: store the new residual
                                 // of every row it does not flag for a rebuild
-  int tensor_fused;             // per-tensor FP8 in one ring launch: after its rows, each
-                                // CTA meets the others at a grid barrier (ws_arrive) and
-                                // writes its rows' codes from the stored new residual
+  int tensor_fused;             // per-tensor FP8 in one ring launch: the CTAs take rows
+                                // from a shared counter (ws_claim), meet at a grid
+                                // barrier (ws_arrive), then write the codes from the
+                                // stored new residual
   unsigned* ws_arrive;          // per-tensor FP8: CTAs past their first pass
+  unsigned* ws_claim;           // per-tensor FP8, one launch: rows taken so far
 };
 
 // Geometry of one launch, chosen on the host.

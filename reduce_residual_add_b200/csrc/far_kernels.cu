@@ -44,6 +44,8 @@ namespace {
 // gamma (H*2 bytes, loaded once per CTA) and the nslot slots.
 struct RingHeader {
   float red[2][2][32];   // [row parity][0 = sum of squares, 1 = amax][warp]
+  int slot_row[32];      // rows taken from a shared counter: the row (ordinal)
+                         // whose first segment sits in the slot, -1: no more rows
   int abort;             // set when any wait of the CTA gave up
   int producer_done;     // set by the producer when it stops issuing
   long long issued;      // bulk copies the producer issued
@@ -353,6 +355,19 @@ __device__ __forceinline__ void pdl_enter() {
 // Barrier over the first `nthreads` threads of the CTA (the consumer warps).
 __device__ __forceinline__ void consumer_bar(int nthreads) {
   asm volatile("bar.sync 1, %0;" ::"r"(nthreads) : "memory");
+}
+
+// The same barrier, returning whether v held for any of those threads (a
+// decision every consumer then takes alike).
+__device__ __forceinline__ bool consumer_any(int nthreads, bool v) {
+  unsigned r;
+  asm volatile(
+      "{\n\t.reg .pred q, a;\n\tsetp.ne.u32 q, %1, 0;\n\t"
+      "bar.red.or.pred a, 1, %2, q;\n\tselp.u32 %0, 1, 0, a;\n\t}"
+      : "=r"(r)
+      : "r"(static_cast<unsigned>(v)), "r"(nthreads)
+      : "memory");
+  return r != 0;
 }
 
 // ---------------------------------------------------------------------------
@@ -967,51 +982,68 @@ far_ring_kernel(const Params p, int nslot, int ncons, int stage_gamma) {
     uint32_t phase = 0;
     int64_t issued = 0;
     if (threadIdx.x == ncons) {
-      const int64_t nseg = my_rows * S;
-      // segment g is segment k of row number ord
-      int k = 0;
-      int64_t ord = blockIdx.x;
       // per-tensor FP8 reading back its new residual: the inputs, read
       // once, leave L2 first, so that the new residual (stored evict-last)
       // is what L2 keeps for the second pass
       const bool drop_inputs = MODE == kModeTensor && p.tensor_stores_residual;
       uint64_t drop = 0;
       if constexpr (MODE == kModeTensor) drop = l2_evict_first();
-      for (int64_t g = 0; g < nseg; ++g) {
-        if (*abort_flag) break;
-        if (!mbar_wait(&empty[slot], phase ^ 1u, abort_flag, p.wait_limit_ns)) {
-          if (!*abort_flag) atomicOr(&g_far_error, kErrWaitEmpty);
-          *abort_flag = 1;
-          break;
+      // Rows: ordinals blockIdx.x + i * gridDim.x; or, in the fused
+      // per-tensor form, taken one at a time from the call's counter (the
+      // next one claimed while this one's segments are issued), so that the
+      // CTAs reach the grid barrier together.  Then the slot of a row's
+      // first segment names the row, and a slot naming -1, completed
+      // without a copy, ends the consumers' first pass.
+      bool dyn = false;
+      if constexpr (MODE == kModeTensor) dyn = p.tensor_fused != 0;
+      int64_t ord = dyn ? static_cast<int64_t>(atomicAdd(p.ws_claim, 1u)) : blockIdx.x;
+      int64_t g = 0;  // copies issued
+      for (int64_t i = 0; !*abort_flag; ++i) {
+        const bool more = dyn ? ord < nrows : i < my_rows;
+        if (!more && !dyn) break;
+        int64_t next = 0;
+        if (dyn && more) next = atomicAdd(p.ws_claim, 1u);
+        const int nk = more ? S : 1;  // the end marker takes one slot
+        bool stop = false;
+        for (int k = 0; k < nk; ++k) {
+          if (!mbar_wait(&empty[slot], phase ^ 1u, abort_flag, p.wait_limit_ns)) {
+            if (!*abort_flag) atomicOr(&g_far_error, kErrWaitEmpty);
+            *abort_flag = 1;
+            stop = true;
+            break;
+          }
+          if (dyn && k == 0) hdr->slot_row[slot] = more ? static_cast<int>(ord) : -1;
+          if (!more) {
+            mbar_arrive(&full[slot]);
+          } else {
+            if (g != p.stall_segment) {  // test hook: that copy is never issued
+              const void* base = (k < p.W) ? p.partials[k] : p.residual;
+              const unsigned char* src = static_cast<const unsigned char*>(base) +
+                                         call_row(p, ord) * static_cast<int64_t>(seg_bytes);
+              mbar_arrive_expect_tx(&full[slot], seg_bytes);
+              if (drop_inputs)
+                bulk_load_hint(ring + static_cast<size_t>(slot) * seg_bytes, src, seg_bytes, &full[slot], drop);
+              else
+                bulk_load(ring + static_cast<size_t>(slot) * seg_bytes, src, seg_bytes, &full[slot]);
+            }
+            ++g;
+          }
+          ++issued;
+          if (++slot == nslot) {
+            slot = 0;
+            phase ^= 1u;
+          }
         }
-        if (g != p.stall_segment) {  // test hook: that copy is never issued
-          const void* base = (k < p.W) ? p.partials[k] : p.residual;
-          const unsigned char* src = static_cast<const unsigned char*>(base) +
-                                     call_row(p, ord) * static_cast<int64_t>(seg_bytes);
-          mbar_arrive_expect_tx(&full[slot], seg_bytes);
-          if (drop_inputs)
-            bulk_load_hint(ring + static_cast<size_t>(slot) * seg_bytes, src, seg_bytes, &full[slot], drop);
-          else
-            bulk_load(ring + static_cast<size_t>(slot) * seg_bytes, src, seg_bytes, &full[slot]);
-        }
-        issued = g + 1;
-        if (++slot == nslot) {
-          slot = 0;
-          phase ^= 1u;
-        }
-        if (++k == S) {
-          k = 0;
-          ord += gridDim.x;
-        }
+        if (stop || !more) break;
+        ord = dyn ? next : ord + gridDim.x;
       }
     }
     if constexpr (MODE == kModeTensor) {
-      // The fused per-tensor form: once the consumers have stored this CTA's
-      // new residuals and row flags (and fenced them for the async proxy),
-      // stream the same rows back through the ring, the most recently
-      // written first: the new residual of a row, or for a flagged row all
-      // its input segments.  The copies run ahead while the consumers wait
-      // at the grid barrier.
+      // The fused per-tensor form: once every CTA has stored its rows' new
+      // residuals and flags (fenced for the async proxy) and the consumers
+      // are past the grid barrier, stream rows blockIdx.x + i * gridDim.x
+      // back through the ring, the highest ordinals (taken last) first: the
+      // new residual of a row, or for a flagged row all its input segments.
       if (p.tensor_fused) {
         tail_bar(ncons + 32);
         // The whole warp reads the row flags, 32 rows per load (one row per
@@ -1075,8 +1107,33 @@ far_ring_kernel(const Params p, int nslot, int ncons, int stage_gamma) {
   const int j0 = threadIdx.x;
   int slot = 0;  // the slot of the next segment and its use count parity
   uint32_t phase = 0;
-  for (int64_t i = 0; i < my_rows; ++i) {
-    const int64_t row = call_row(p, blockIdx.x + i * gridDim.x);
+  bool dyn = false;  // rows named by the producer (the fused per-tensor form)
+  if constexpr (MODE == kModeTensor) dyn = p.tensor_fused != 0;
+  for (int64_t i = 0;; ++i) {
+    int64_t ord;
+    if (dyn) {
+      // the row is named in the slot of its first segment; every consumer
+      // leaves the loop alike, at the end marker or after a wait gave up
+      if (!*abort_flag && !mbar_wait(&full[slot], phase, abort_flag, p.wait_limit_ns)) {
+        if (!*abort_flag) atomicOr(&g_far_error, kErrWaitFull);
+        *abort_flag = 1;
+      }
+      const int named = hdr->slot_row[slot];
+      if (consumer_any(ncons, named < 0 || *abort_flag)) {
+        __syncwarp();
+        if ((threadIdx.x & 31) == 0) mbar_arrive(&empty[slot]);
+        if (++slot == nslot) {
+          slot = 0;
+          phase ^= 1u;
+        }
+        break;
+      }
+      ord = named;
+    } else {
+      if (i >= my_rows) break;
+      ord = blockIdx.x + i * gridDim.x;
+    }
+    const int64_t row = call_row(p, ord);
     float y[VPT][8];
     bool ok[VPT];
 #pragma unroll
@@ -1086,7 +1143,8 @@ far_ring_kernel(const Params p, int nslot, int ncons, int stage_gamma) {
       for (int e = 0; e < 8; ++e) y[k][e] = 0.f;
     }
     for (int k = 0; k < S; ++k) {
-      if (!*abort_flag && !mbar_wait(&full[slot], phase, abort_flag, p.wait_limit_ns)) {
+      if (!(dyn && k == 0) && !*abort_flag &&
+          !mbar_wait(&full[slot], phase, abort_flag, p.wait_limit_ns)) {
         if (!*abort_flag) atomicOr(&g_far_error, kErrWaitFull);
         *abort_flag = 1;
       }
@@ -1106,10 +1164,11 @@ far_ring_kernel(const Params p, int nslot, int ncons, int stage_gamma) {
   }
   if constexpr (MODE == kModeTensor) {
     if (p.tensor_fused) {
-      // this thread's new-residual stores, before the producer's bulk copies read them
+      // this thread's new-residual stores, before any CTA's bulk copies read them
       asm volatile("fence.proxy.async.global;" ::: "memory");
-      tail_bar(ncons + 32);
-      if (tensor_grid_barrier(p, ncons, abort_flag)) {
+      const bool passed = tensor_grid_barrier(p, ncons, abort_flag);
+      tail_bar(ncons + 32);  // the producer starts the second pass
+      if (passed) {
         unsigned amax_bits;
         asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(amax_bits) : "l"(p.ws_amax) : "memory");
         const TensorScale ts(p, amax_bits);
