@@ -112,7 +112,9 @@ typedef enum {
  * FAR_RING_CTAS_PER_SM=1..8, FAR_RING_THREADS: consumer threads per ring
  * CTA, at most 256, FAR_RING_SLOTS: row-segment slots per ring CTA (2..32),
  * FAR_RING_GAMMA_SMEM=1|0: gamma staged in shared memory or read through
- * L1 (each replaces its part of the default geometry, which follows rules
+ * L1, FAR_RING_WIDE=1|0: the 384-consumer build for rows of 1025-1536
+ * packs where the rules take it (each replaces its part of the default
+ * geometry, which follows rules
  * measured on B200 by row length, segments per row and whether norm_out is
  * written: plan_ring in reduce_residual_add_b200/csrc/far_abi.cu),
  * FAR_PDL=1|0: launch with programmatic dependent launch, default 1,

@@ -30,7 +30,9 @@ struct far_ctx {
   int ring_slots_max;   // at most this many ring slots
   int tensor_reverse;   // per-tensor FP8: second pass from the last row down
   int tensor_fused;     // per-tensor FP8: both passes in one ring launch when possible
-  int ring_gamma_mode;  // ring: 1 stage gamma in shared memory, 0 read it through L1, -1 by rule
+  int ring_gamma_mode;
+  int ring_wide;        // the wide ring build for rows of 1025-1536 packs (1 / 0)
+  int ring_wide2;       // the wide 2-pack build for rows of 513-896 packs (1 / 0)  // ring: 1 stage gamma in shared memory, 0 read it through L1, -1 by rule
   int pdl;              // programmatic dependent launch on every call
   int ring_min_rows;    // fewer rows than this take the direct kernel
   uint64_t wait_limit_ns;  // bounded waits in the kernels give up after this
@@ -186,6 +188,11 @@ int ring_occ_cached(const far_ctx* ctx, int dtype, int vpt, int minb, int thread
 //    the c4 shape: 97.4 %), else 2 x 4 (W=2: 98.8 vs 84.0 %); with norm_out
 //    and at most 6 segments of at least 16 KiB, 2 CTAs per SM with gamma
 //    read through L1 and about 96 KiB of slots (W=3..5: 97-102 vs 87-94 %);
+//  * 1025-1536 packs (H = 8200-12288) without norm_out, or with more than
+//    6 segments: the wide build, 4 packs per thread over up to 384
+//    consumers, 2 CTAs per SM, about 72 KiB of slots (W=2/3/4/8 at
+//    H=10240: 94-97 vs 76-89 %; at H=12288: 86-98 vs 80-91 %; with
+//    norm_out and at most 6 segments it lost, 83-91 vs 86-94 %);
 //  * 8 packs per thread (H >= 12288): 2 CTAs per SM, with the build whose
 //    registers are sized for two, about 72 KiB of slots (H=12288, W=2..8:
 //    80-93 vs 58-84 % at one CTA); but one CTA per SM with 6 slots when the
@@ -217,14 +224,32 @@ bool plan_ring(const far_ctx* ctx, int packs, int64_t rows, int dtype, int segs,
   int vpt = 1;
   while (vpt < 8 && (packs + vpt - 1) / vpt > max_cons) vpt *= 2;
   if (!ctx->ring_threads_set && segs <= 6 && packs >= 512 && packs < 1024 && vpt < 4) vpt = 4;
+  // rows of 1025-1536 packs without norm_out (or with more than 6
+  // segments): the wide build, 4 packs per thread over up to 384 consumers,
+  // instead of 8 packs per thread
+  const bool wide4 = ctx->ring_wide && !ctx->ring_threads_set && !group && packs > 1024 &&
+                     packs <= 4 * far::kRingWideConsumers && (!norm || segs > 6);
+  // rows of 513-896 packs: 2 packs per thread over up to 448 consumers
+  const bool wide2 = ctx->ring_wide2 && !ctx->ring_threads_set && !group && packs > 512 &&
+                     packs <= 2 * far::kRingWide2Consumers;
+  const bool wide = wide4 || wide2;
+  if (wide4) vpt = 4;
+  if (wide2) vpt = 2;
   const int tpr = (((packs + vpt - 1) / vpt) + 31) / 32 * 32;
-  if (tpr > far::kRingMaxConsumers) return false;
+  if (tpr > (wide4 ? far::kRingWideConsumers : wide2 ? far::kRingWide2Consumers : far::kRingMaxConsumers))
+    return false;
 
   int n_req = 2;
   bool gamma_smem = true;
   int want = 0;            // slots per CTA (0: by `target` bytes)
   int target = 72 * 1024;  // slot bytes per CTA when want == 0
-  if (vpt >= 8) {
+  if (wide4) {
+    // 2 CTAs per SM (its registers are sized for two), about 72 KiB of slots
+  } else if (wide2) {
+    // 2 CTAs per SM, about 56 KiB of slots each
+    want = 56 * 1024 / seg;
+    if (want < 2) want = 2;
+  } else if (vpt >= 8) {
     // 8 packs per thread: 2 CTAs per SM (a build with a few spilled
     // registers), unless the row has many segments and fewer than 3 slots
     // would fit: then one CTA per SM, as all its registers allow, 6 slots
@@ -294,13 +319,14 @@ bool plan_ring(const far_ctx* ctx, int packs, int64_t rows, int dtype, int segs,
   const int smem = far::ring_header_bytes(nslot) + (nslot + gsegs) * seg;
   // the register budget the kernel is built for: 3 or 2 CTAs per SM, and at
   // 8 packs per thread 1 (no spills) or 2 (a few spilled registers)
-  const int minb = vpt >= 8 ? (n_req >= 2 ? 2 : 1) : (n_req >= 3 ? 3 : 2);
+  const int minb = wide ? 2 : vpt >= 8 ? (n_req >= 2 ? 2 : 1) : (n_req >= 3 ? 3 : 2);
   int occ = ring_occ_cached(ctx, dtype, vpt, minb, tpr + 32, smem);
   if (occ < 1) return false;
   if (occ > n_req) occ = n_req;
   l->kernel = 1;
   l->ring_minb = minb;
   l->ring_gamma = gsegs;
+  l->ring_wide = wide ? 1 : 0;
   l->vpt = vpt;
   l->tpr = tpr;
   l->rows_per_cta = 1;
@@ -448,6 +474,8 @@ far_status far_create(far_ctx** ctx, int device) {
   c.tensor_reverse = env_int("FAR_TENSOR_REVERSE", 1) != 0;
   c.tensor_fused = env_int("FAR_TENSOR_FUSED", 1) != 0;
   c.ring_gamma_mode = env_int("FAR_RING_GAMMA_SMEM", -1);
+  c.ring_wide = env_int("FAR_RING_WIDE", 1) != 0 ? 1 : 0;
+  c.ring_wide2 = env_int("FAR_RING_WIDE2", 0) != 0 ? 1 : 0;
   if (c.ring_gamma_mode > 1) c.ring_gamma_mode = 1;
   if (c.ring_gamma_mode < -1) c.ring_gamma_mode = -1;
   if (c.ring_slots_max < 0) c.ring_slots_max = 0;

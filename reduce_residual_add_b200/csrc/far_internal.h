@@ -13,6 +13,10 @@ constexpr int kPackElems = 8;    // 2-byte elements per 16-byte pack
 constexpr int kMaxThreads = 256; // threads per row (CTA) in every kernel
 constexpr int kRingSmemMax = 227 * 1024;  // dynamic shared memory of one ring CTA
 constexpr int kRingMaxConsumers = 256;    // consumer threads of one ring CTA
+constexpr int kRingWideConsumers = 384;   // ... of the wide build (4 packs per thread,
+                                          // rows of 1025-1536 packs, 2 CTAs per SM)
+constexpr int kRingWide2Consumers = 448;  // ... of the wide 2-pack build (rows of
+                                          // 513-896 packs, 2 CTAs per SM)
 
 enum Dtype : int { kBf16 = 0, kFp16 = 1 };
 enum Pattern : int {
@@ -78,6 +82,7 @@ struct Launch {
   int pdl;              // launch with programmatic stream serialization
   int ring_minb;        // ring: CTAs per SM its registers are sized for (2 or 3; 1 or 2 at 8 packs)
   int ring_gamma;       // ring: 1 = gamma staged in shared memory, 0 = read through L1
+  int ring_wide;        // ring: the wide build (up to kRingWideConsumers consumers)
   int cooperative;      // launch cooperatively (every CTA co-resident; a grid barrier inside)
 };
 

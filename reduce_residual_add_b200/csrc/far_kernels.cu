@@ -941,8 +941,9 @@ __device__ __forceinline__ void tail_bar(int nthreads) {
 // the producer stops, and thread 0 waits (bounded) for the copies already
 // issued before the CTA exits.
 // MINB: CTAs per SM the register budget is sized for (2 or 3; 1 or 2 at VPT 8).
-template <class DT, int VPT, int MINB, int MODE>
-__global__ void __launch_bounds__(kRingMaxConsumers + 32, MINB)
+// MAXC: most consumer threads (the wide build: kRingWideConsumers).
+template <class DT, int VPT, int MINB, int MODE, int MAXC = kRingMaxConsumers>
+__global__ void __launch_bounds__(MAXC + 32, MINB)
 far_ring_kernel(const Params p, int nslot, int ncons, int stage_gamma) {
   extern __shared__ __align__(128) unsigned char smem[];
   uint64_t* full = reinterpret_cast<uint64_t*>(smem);
@@ -1372,7 +1373,7 @@ cudaError_t launch_decode_t(const Params& p, const Launch& l, cudaStream_t s) {
   return cudaLaunchKernelEx(&cfg, far_decode_kernel<DT, VPT>, p);
 }
 
-template <class DT, int VPT, int MINB, int MODE>
+template <class DT, int VPT, int MINB, int MODE, int MAXC = kRingMaxConsumers>
 cudaError_t launch_ring_t(const Params& p, const Launch& l, cudaStream_t s) {
   Attrs at(l, 0);
   cudaLaunchConfig_t cfg = {};
@@ -1382,7 +1383,7 @@ cudaError_t launch_ring_t(const Params& p, const Launch& l, cudaStream_t s) {
   cfg.stream = s;
   cfg.attrs = at.a;
   cfg.numAttrs = at.n;
-  return cudaLaunchKernelEx(&cfg, far_ring_kernel<DT, VPT, MINB, MODE>, p, l.nslot, l.tpr,
+  return cudaLaunchKernelEx(&cfg, far_ring_kernel<DT, VPT, MINB, MODE, MAXC>, p, l.nslot, l.tpr,
                             l.ring_gamma);
 }
 
@@ -1391,8 +1392,14 @@ cudaError_t launch_ring_g(const Params& p, const Launch& l, cudaStream_t s) {
   const bool three = l.ring_minb >= 3;
   switch (l.vpt) {
     case 1: return three ? launch_ring_t<DT, 1, 3, MODE>(p, l, s) : launch_ring_t<DT, 1, 2, MODE>(p, l, s);
-    case 2: return three ? launch_ring_t<DT, 2, 3, MODE>(p, l, s) : launch_ring_t<DT, 2, 2, MODE>(p, l, s);
-    case 4: return three ? launch_ring_t<DT, 4, 3, MODE>(p, l, s) : launch_ring_t<DT, 4, 2, MODE>(p, l, s);
+    case 2:
+      if constexpr (MODE != kModeGroup)
+        if (l.ring_wide) return launch_ring_t<DT, 2, 2, MODE, kRingWide2Consumers>(p, l, s);
+      return three ? launch_ring_t<DT, 2, 3, MODE>(p, l, s) : launch_ring_t<DT, 2, 2, MODE>(p, l, s);
+    case 4:
+      if constexpr (MODE != kModeGroup)
+        if (l.ring_wide) return launch_ring_t<DT, 4, 2, MODE, kRingWideConsumers>(p, l, s);
+      return three ? launch_ring_t<DT, 4, 3, MODE>(p, l, s) : launch_ring_t<DT, 4, 2, MODE>(p, l, s);
     case 8: return l.ring_minb >= 2 ? launch_ring_t<DT, 8, 2, MODE>(p, l, s)
                                     : launch_ring_t<DT, 8, 1, MODE>(p, l, s);
     default: return cudaErrorInvalidConfiguration;
@@ -1495,6 +1502,10 @@ cudaError_t allow_large_smem() {
   set(far_ring_kernel<DT, 4, 3, kModeTensor>);
   set(far_ring_kernel<DT, 8, 1, kModeTensor>);
   set(far_ring_kernel<DT, 8, 2, kModeTensor>);
+  set(far_ring_kernel<DT, 4, 2, kModePlain, kRingWideConsumers>);
+  set(far_ring_kernel<DT, 4, 2, kModeTensor, kRingWideConsumers>);
+  set(far_ring_kernel<DT, 2, 2, kModePlain, kRingWide2Consumers>);
+  set(far_ring_kernel<DT, 2, 2, kModeTensor, kRingWide2Consumers>);
   return e;
 }
 
@@ -1534,12 +1545,12 @@ cudaError_t launch_tensor_quant(const Params& p, int dtype, const Launch& l, cud
 int ring_header_bytes(int nslot) { return ring_offset(nslot); }
 
 namespace {
-template <class DT, int VPT, int MINB>
+template <class DT, int VPT, int MINB, int MAXC = kRingMaxConsumers>
 int occ_of(int threads, int smem) {
   // the per-group instantiation is sized the same way; the plain one decides
   int n = 0;
   const cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(
-      &n, far_ring_kernel<DT, VPT, MINB, kModePlain>, threads, smem);
+      &n, far_ring_kernel<DT, VPT, MINB, kModePlain, MAXC>, threads, smem);
   return e == cudaSuccess ? n : 0;
 }
 
@@ -1548,8 +1559,12 @@ int ring_occupancy_dt(int vpt, int minb, int threads, int smem) {
   const bool three = minb >= 3;
   switch (vpt) {
     case 1: return three ? occ_of<DT, 1, 3>(threads, smem) : occ_of<DT, 1, 2>(threads, smem);
-    case 2: return three ? occ_of<DT, 2, 3>(threads, smem) : occ_of<DT, 2, 2>(threads, smem);
-    case 4: return three ? occ_of<DT, 4, 3>(threads, smem) : occ_of<DT, 4, 2>(threads, smem);
+    case 2:
+      if (threads > kRingMaxConsumers + 32) return occ_of<DT, 2, 2, kRingWide2Consumers>(threads, smem);
+      return three ? occ_of<DT, 2, 3>(threads, smem) : occ_of<DT, 2, 2>(threads, smem);
+    case 4:
+      if (threads > kRingMaxConsumers + 32) return occ_of<DT, 4, 2, kRingWideConsumers>(threads, smem);
+      return three ? occ_of<DT, 4, 3>(threads, smem) : occ_of<DT, 4, 2>(threads, smem);
     case 8: return minb >= 2 ? occ_of<DT, 8, 2>(threads, smem) : occ_of<DT, 8, 1>(threads, smem);
     default: return 0;
   }

@@ -122,6 +122,8 @@ def test_small_shapes(ctx, regime, case, reg):
     (4, 1000, 8192, "fp16", 0, False, 0.0),  # no residual: W segments per row
     (8, 149, 7168, "bf16", 2, True, 1.0),    # one more row than CTAs
     (3, 7, 2048, "bf16", 1, True, 0.0),      # fewer rows than CTAs
+    (2, 1200, 12288, "bf16", 1, True, 0.0),  # 1536 packs: the wide build (384 consumers)
+    (8, 300, 10248, "fp16", 2, True, 1.0),   # 1281 packs, ragged: wide, 352 consumers
 ], ids=lambda c: "W%d_T%d_H%d_%s_p%d_res%d_wb%g" % c)
 def test_prefill_kernels(kctx, case, kern):
     W, T, H, dt, pattern, has_res, wb = case
@@ -134,6 +136,24 @@ def test_prefill_kernels(kctx, case, kern):
     got = run_gpu(c, to_gpu(inp), 1e-6, wb, pattern, scale_in=0.05, guard=1024)
     ref = run_oracle(inp, dt, 1e-6, wb, pattern, scale_in=0.05)
     log("prefill %s %s" % (kern, case), compare(got, ref, dt))
+
+
+@pytest.mark.parametrize("case", [
+    (2, 1200, 12288, "bf16", 1, 0.0),   # 1536 packs: 384 consumers
+    (3, 700, 10248, "fp16", 2, 1.0),    # 1281 packs, ragged: 352 consumers
+], ids=lambda c: "W%d_T%d_H%d_%s_p%d_wb%g" % c)
+def test_ring_wide_build(kctx, case):
+    """Rows of 1025-1536 packs without norm_out take the wide build (4 packs
+    per thread over up to 384 consumers)."""
+    W, T, H, dt, pattern, wb = case
+    c = kctx["ring"]
+    info = far.far_describe_launch(c, T, H, torch.bfloat16, W, True, False)
+    assert (info["kernel"], info["packs_per_thread"]) == (1, 4)
+    assert info["threads_per_cta"] == ((H // 8 + 3) // 4 + 31) // 32 * 32 + 32
+    inp = random_inputs(W, T, H, dtype=dt, seed=11 * W + T + H, has_residual=True)
+    got = run_gpu(c, to_gpu(inp), 1e-6, wb, pattern, scale_in=0.05, guard=1024, want_norm=False)
+    ref = run_oracle(inp, dt, 1e-6, wb, pattern, scale_in=0.05, want_norm=False)
+    log("ring wide %s" % (case,), compare(got, ref, dt))
 
 
 @pytest.mark.parametrize("pattern", [1, 2])
@@ -422,6 +442,11 @@ def test_launch_plan(ctx):
     h4 = d(16384, 4096, 4)
     assert (h4["packs_per_thread"], h4["threads_per_cta"], h4["grid_ctas"], h4["ring_slots"]) == (4, 160, 4 * sms, 3)
     assert d(16384, 4096, 4, norm=True)["grid_ctas"] == 3 * sms
+    # 1025-1536 packs without norm_out: the wide build, 4 packs per thread
+    h12 = d(8192, 12288, 2)
+    assert (h12["packs_per_thread"], h12["threads_per_cta"], h12["grid_ctas"], h12["ring_slots"]) == (4, 416, 2 * sms, 3)
+    # ... with norm_out and at most 6 segments, 8 packs per thread
+    assert d(8192, 12288, 2, norm=True)["packs_per_thread"] == 8
     # 8 packs per thread: 2 CTAs per SM, gamma in shared memory ...
     h16 = d(8192, 16384, 2)
     assert (h16["kernel"], h16["grid_ctas"], h16["ring_gamma_smem"], h16["ring_slots"]) == (1, 2 * sms, 1, 2)
