@@ -113,7 +113,8 @@ typedef enum {
  * CTA, at most 256, FAR_RING_SLOTS: row-segment slots per ring CTA (2..32),
  * FAR_RING_GAMMA_SMEM=1|0: gamma staged in shared memory or read through
  * L1, FAR_RING_WIDE=1|0: the 384-consumer build for rows of 1025-1536
- * packs where the rules take it (each replaces its part of the default
+ * packs, FAR_RING_WIDE2=1|0: the 448-consumer build for rows of 513-896
+ * packs, where the rules take them (each replaces its part of the default
  * geometry, which follows rules
  * measured on B200 by row length, segments per row and whether norm_out is
  * written: plan_ring in reduce_residual_add_b200/csrc/far_abi.cu),
@@ -121,8 +122,8 @@ typedef enum {
  * FAR_RING_MIN_ROWS: fewest rows for the ring kernel, default by rule,
  * FAR_TENSOR_REVERSE=1|0: the second pass of per-tensor FP8 takes the rows
  * from the last one down, default 1, FAR_TENSOR_FUSED=1|0: per-tensor FP8
- * without norm_out on the ring kernel runs both passes in one cooperative
- * launch with a grid barrier between them, default 1). */
+ * without norm_out on the ring kernel runs both passes in one launch with
+ * a bounded grid-wide wait between them, default 1). */
 /*
  * Programmatic dependent launch: every kernel of this library first waits
  * (griddepcontrol.wait) until the grid it depends on has completed, then
@@ -234,8 +235,9 @@ size_t far_fp8_tensor_workspace_bytes(int64_t rows);
  * to scale_out[0], and quant_out = e4m3_satfinite(o / scale).  Other
  * arguments as far_fused_rows; residual_out, norm_out as there.
  *
- * The scale needs every row before any code, so the call enqueues a memset
- * of the workspace's first four words and two passes.  The first reads the
+ * The scale needs every row before any code, so the call enqueues a
+ * one-CTA kernel that zeroes the workspace's first four words, and two
+ * passes.  The first reads the
  * inputs and keeps each row's 1/rms and the running amax in `workspace`.
  * Without norm_out and with a new residual to write (a residual_out, or a
  * residual updated in place), the first pass also writes the new residual
@@ -246,9 +248,10 @@ size_t far_fp8_tensor_workspace_bytes(int64_t rows);
  * the same.  Rows whose sum of squares could hide an element that overflows
  * the format (and rows with an inf or NaN input) are rebuilt from the
  * inputs by the second pass instead.  When the persistent kernel serves
- * the call, both passes run in ONE cooperative launch: its CTAs take the
- * first pass's rows one at a time from a counter in the workspace, meet at
- * a bounded grid barrier, then write the codes (FAR_TENSOR_FUSED=0 in the
+ * the call, both passes run in ONE launch: its CTAs take the first pass's
+ * rows one at a time from a counter in the workspace, wait (bounded) until
+ * every row is done -- a wait on rows, not on CTAs, so the grid need not be
+ * co-resident -- then write the codes (FAR_TENSOR_FUSED=0 in the
  * environment at far_create splits them into two kernels); otherwise two
  * kernels run.
  * With norm_out, or with no new residual to write, the second pass reads

@@ -188,6 +188,11 @@ int ring_occ_cached(const far_ctx* ctx, int dtype, int vpt, int minb, int thread
 //    the c4 shape: 97.4 %), else 2 x 4 (W=2: 98.8 vs 84.0 %); with norm_out
 //    and at most 6 segments of at least 16 KiB, 2 CTAs per SM with gamma
 //    read through L1 and about 96 KiB of slots (W=3..5: 97-102 vs 87-94 %);
+//  * 513-896 packs (H = 4104-7168) with 8 or more segments (W=8 + the
+//    residual): the wide 2-pack build, 2 packs per thread over up to 448
+//    consumers, 2 CTAs per SM, about 56 KiB of slots each (W=8 at H=4608,
+//    5120, 6144, 7168: 98-101 vs 93-98 %, per-token H=7168: 99.4 vs 97.1 %;
+//    at 3-5 segments it lost as often as it won);
 //  * 1025-1536 packs (H = 8200-12288) without norm_out, or with more than
 //    6 segments: the wide build, 4 packs per thread over up to 384
 //    consumers, 2 CTAs per SM, about 72 KiB of slots (W=2/3/4/8 at
@@ -229,9 +234,10 @@ bool plan_ring(const far_ctx* ctx, int packs, int64_t rows, int dtype, int segs,
   // instead of 8 packs per thread
   const bool wide4 = ctx->ring_wide && !ctx->ring_threads_set && !group && packs > 1024 &&
                      packs <= 4 * far::kRingWideConsumers && (!norm || segs > 6);
-  // rows of 513-896 packs: 2 packs per thread over up to 448 consumers
+  // rows of 513-896 packs with 8 or more segments: 2 packs per thread over
+  // up to 448 consumers
   const bool wide2 = ctx->ring_wide2 && !ctx->ring_threads_set && !group && packs > 512 &&
-                     packs <= 2 * far::kRingWide2Consumers;
+                     packs <= 2 * far::kRingWide2Consumers && segs >= 8;
   const bool wide = wide4 || wide2;
   if (wide4) vpt = 4;
   if (wide2) vpt = 2;
@@ -475,7 +481,7 @@ far_status far_create(far_ctx** ctx, int device) {
   c.tensor_fused = env_int("FAR_TENSOR_FUSED", 1) != 0;
   c.ring_gamma_mode = env_int("FAR_RING_GAMMA_SMEM", -1);
   c.ring_wide = env_int("FAR_RING_WIDE", 1) != 0 ? 1 : 0;
-  c.ring_wide2 = env_int("FAR_RING_WIDE2", 0) != 0 ? 1 : 0;
+  c.ring_wide2 = env_int("FAR_RING_WIDE2", 1) != 0 ? 1 : 0;
   if (c.ring_gamma_mode > 1) c.ring_gamma_mode = 1;
   if (c.ring_gamma_mode < -1) c.ring_gamma_mode = -1;
   if (c.ring_slots_max < 0) c.ring_slots_max = 0;
@@ -739,7 +745,7 @@ far_status far_fused_fp8_tensor_launch(far_ctx* ctx, int64_t row_begin, int64_t 
   p.wait_limit_ns = ctx->wait_limit_ns;
   p.stall_segment = ctx->stall_segment;
   p.ws_amax = static_cast<unsigned*>(workspace);
-  p.ws_arrive = p.ws_amax + 1;
+  p.ws_done = p.ws_amax + 1;
   p.ws_claim = p.ws_amax + 2;
   p.ws_rinv = reinterpret_cast<float*>(static_cast<unsigned char*>(workspace) + 256);
   p.ws_row0 = row_begin;
@@ -756,24 +762,23 @@ far_status far_fused_fp8_tensor_launch(far_ctx* ctx, int64_t row_begin, int64_t 
     whole.grid = (row_end - row_begin + whole.rows_per_cta - 1) / whole.rows_per_cta;
     whole.pdl = ctx->pdl;
   }
-  // the amax word, the grid barrier's arrival count and the row counter
-  // start at zero
-  cudaError_t e = cudaMemsetAsync(workspace, 0, 4 * sizeof(unsigned), s);
-  if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync");
+  // the amax word, the count of rows done and the row counter start at
+  // zero: a one-CTA kernel after the preceding work, so that the first pass
+  // can still be launched with PDL (its set-up overlapping this kernel)
+  cudaError_t e = far::launch_ws_zero(static_cast<unsigned*>(workspace), ctx->pdl, s);
+  if (e != cudaSuccess) return cuda_fail(e, "kernel launch (per-tensor workspace)");
   far::Launch first = whole;
-  first.pdl = 0;  // it must see the memset above
+  first.pdl = ctx->pdl;
   p.pattern = far::kTensorAmax;
-  // With the ring kernel (persistent CTAs, all co-resident by construction)
-  // and the codes formed from the stored new residual, both passes run in
-  // one cooperative launch: the CTAs take first-pass rows from a counter,
-  // meet at a grid barrier, then write the codes, the rows taken last first.
+  // With the ring kernel and the codes formed from the stored new residual,
+  // both passes run in one launch: the CTAs take first-pass rows from a
+  // counter, wait until every row is done (a wait on rows, not on CTAs, so
+  // no co-residency is needed), then write the codes, the rows taken last
+  // first.
   const bool fused = ctx->tensor_fused && from_residual && first.regime == FAR_REGIME_PREFILL &&
                      first.kernel == 1 &&
                      row_end - row_begin <= 0x7fffffff;
-  if (fused) {
-    first.cooperative = 1;
-    p.tensor_fused = 1;
-  }
+  if (fused) p.tensor_fused = 1;
   e = launch_rows(p, dtype, first, row_begin, row_end, s);
   if (e != cudaSuccess) return cuda_fail(e, "kernel launch (per-tensor pass 1)");
   if (fused) return FAR_OK;

@@ -59,10 +59,10 @@ struct Params {
   int tensor_stores_residual;   // per-tensor FP8, first pass: store the new residual
                                 // of every row it does not flag for a rebuild
   int tensor_fused;             // per-tensor FP8 in one ring launch: the CTAs take rows
-                                // from a shared counter (ws_claim), meet at a grid
-                                // barrier (ws_arrive), then write the codes from the
+                                // from a shared counter (ws_claim), wait until every
+                                // row is done (ws_done), then write the codes from the
                                 // stored new residual
-  unsigned* ws_arrive;          // per-tensor FP8: CTAs past their first pass
+  unsigned* ws_done;            // per-tensor FP8, one launch: rows past the first pass
   unsigned* ws_claim;           // per-tensor FP8, one launch: rows taken so far
 };
 
@@ -83,7 +83,6 @@ struct Launch {
   int ring_minb;        // ring: CTAs per SM its registers are sized for (2 or 3; 1 or 2 at 8 packs)
   int ring_gamma;       // ring: 1 = gamma staged in shared memory, 0 = read through L1
   int ring_wide;        // ring: the wide build (up to kRingWideConsumers consumers)
-  int cooperative;      // launch cooperatively (every CTA co-resident; a grid barrier inside)
 };
 
 // Enqueue one kernel on `stream`.  Returns the launch error (cudaSuccess if
@@ -92,6 +91,9 @@ cudaError_t launch_prefill(const Params& p, int dtype, const Launch& l, cudaStre
 cudaError_t launch_decode(const Params& p, int dtype, const Launch& l, cudaStream_t stream);
 cudaError_t launch_ring(const Params& p, int dtype, const Launch& l, cudaStream_t stream);
 cudaError_t launch_tensor_quant(const Params& p, int dtype, const Launch& l, cudaStream_t stream);
+// Zero the per-tensor workspace's first four words, after the preceding
+// kernels in the stream (a kernel, so that the next launch may use PDL).
+cudaError_t launch_ws_zero(unsigned* ws, int pdl, cudaStream_t stream);
 
 // Bytes of the ring kernel's shared memory before its first slot.
 int ring_header_bytes(int nslot);

@@ -894,21 +894,24 @@ struct TensorScale {
 };
 
 // The fused per-tensor form's grid barrier, run by the consumer threads of a
-// ring CTA once its own rows are done: every CTA of the (cooperative, so
-// co-resident) launch arrives, then the call's amax is final.  The wait is
-// bounded; a CTA that gives up sets the device error word and its abort
-// flag (it writes no codes).  Returns false then.
+// ring CTA once it has taken no more rows: the CTA adds the rows it did to
+// the call's count, then waits until every row of the call is done, when
+// the call's amax is final.  It waits for rows, not for CTAs: a CTA that
+// has not started holds no row, so the wait needs no co-residency of the
+// grid.  The wait is bounded; a CTA that gives up sets the device error
+// word and its abort flag (it writes no codes).  Returns false then.
 __device__ __forceinline__ bool tensor_grid_barrier(const Params& p, int ncons,
-                                                    volatile int* abort_flag) {
+                                                    volatile int* abort_flag, int64_t rows_done) {
   consumer_bar(ncons);  // every consumer of this CTA is past its last row
   if (threadIdx.x == 0) {
-    __threadfence();    // this CTA's amax before its arrival (cumulative)
-    atomicAdd(p.ws_arrive, 1u);
+    __threadfence();    // this CTA's amax and rows before its count (cumulative)
+    atomicAdd(p.ws_done, static_cast<unsigned>(rows_done));
+    const unsigned nrows = static_cast<unsigned>(p.row_end - p.row_begin);
     const uint64_t t0 = global_ns();
     for (;;) {
       unsigned n;
-      asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(n) : "l"(p.ws_arrive) : "memory");
-      if (n >= gridDim.x) break;
+      asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(n) : "l"(p.ws_done) : "memory");
+      if (n >= nrows) break;
       if (global_ns() - t0 > p.wait_limit_ns) {
         atomicOr(&g_far_error, kErrWaitGrid);
         *abort_flag = 1;
@@ -1110,7 +1113,8 @@ far_ring_kernel(const Params p, int nslot, int ncons, int stage_gamma) {
   uint32_t phase = 0;
   bool dyn = false;  // rows named by the producer (the fused per-tensor form)
   if constexpr (MODE == kModeTensor) dyn = p.tensor_fused != 0;
-  for (int64_t i = 0;; ++i) {
+  int64_t i = 0;  // rows done
+  for (;; ++i) {
     int64_t ord;
     if (dyn) {
       // the row is named in the slot of its first segment; every consumer
@@ -1167,7 +1171,7 @@ far_ring_kernel(const Params p, int nslot, int ncons, int stage_gamma) {
     if (p.tensor_fused) {
       // this thread's new-residual stores, before any CTA's bulk copies read them
       asm volatile("fence.proxy.async.global;" ::: "memory");
-      const bool passed = tensor_grid_barrier(p, ncons, abort_flag);
+      const bool passed = tensor_grid_barrier(p, ncons, abort_flag, i);
       tail_bar(ncons + 32);  // the producer starts the second pass
       if (passed) {
         unsigned amax_bits;
@@ -1321,17 +1325,12 @@ far_tensor_quant_kernel(const Params p) {
   }
 }
 
-// Launch attributes: optional cooperative launch, programmatic stream
-// serialization (PDL) and a cluster shape.
+// Launch attributes: programmatic stream serialization (PDL) and a cluster
+// shape.
 struct Attrs {
-  cudaLaunchAttribute a[3];
+  cudaLaunchAttribute a[2];
   unsigned n = 0;
   Attrs(const Launch& l, int cluster) {
-    if (l.cooperative) {
-      a[n].id = cudaLaunchAttributeCooperative;
-      a[n].val.cooperative = 1;
-      ++n;
-    }
     if (l.pdl) {
       a[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
       a[n].val.programmaticStreamSerializationAllowed = 1;
@@ -1616,4 +1615,26 @@ cudaError_t clear_error_word(cudaStream_t s) {
   return e;
 }
 
+// The per-tensor workspace header (amax, rows done, rows taken) set to zero
+// by a kernel rather than a memset, so that the ring kernel after it can be
+// launched with programmatic dependent launch: its set-up overlaps this one.
+__global__ void far_ws_zero_kernel(unsigned* ws) {
+  pdl_enter();  // the previous call's kernels have finished with the header
+  if (threadIdx.x < 4) ws[threadIdx.x] = 0u;
+}
+
+cudaError_t launch_ws_zero(unsigned* ws, int pdl, cudaStream_t s) {
+  cudaLaunchAttribute a[1];
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(1, 1, 1);
+  cfg.blockDim = dim3(32, 1, 1);
+  cfg.stream = s;
+  if (pdl) {
+    a[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    a[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = a;
+    cfg.numAttrs = 1;
+  }
+  return cudaLaunchKernelEx(&cfg, far_ws_zero_kernel, ws);
+}
 }  // namespace far

@@ -431,9 +431,12 @@ def test_launch_plan(ctx):
     # ... but with norm_out, 2 CTAs per SM, gamma through L1, ~96 KiB of slots
     c4n = d(8192, 8192, 4, norm=True)
     assert (c4n["grid_ctas"], c4n["ring_gamma_smem"], c4n["ring_slots"]) == (2 * sms, 0, 6)
-    # many segments of 896 packs: 2 CTAs per SM x 4 slots, gamma in shared memory
+    # 8 or more segments of 513-896 packs: the wide 2-pack build (448
+    # consumers), 2 CTAs per SM x 4 slots, gamma in shared memory
     c5 = d(4096, 7168, 8)
     assert (c5["grid_ctas"], c5["ring_gamma_smem"], c5["ring_slots"]) == (2 * sms, 1, 4)
+    assert (c5["packs_per_thread"], c5["threads_per_cta"]) == (2, 480)
+    assert d(4096, 7168, 4)["packs_per_thread"] == 4
     # rows of at most 384 packs: 4 CTAs per SM x 4 slots, whatever the segments
     h3 = d(32768, 3072, 8)
     assert (h3["grid_ctas"], h3["ring_slots"]) == (4 * sms, 4)
@@ -534,6 +537,7 @@ def test_chained_calls_read_completed_outputs(kctx, ctx, kern):
     (3, 1000, 1000, "bf16", False, 0.0),
     (16, 40, 16384, "bf16", True, 0.0),
     (2, 77, 8200, "bf16", True, 0.0),      # 1025 packs: 8 per thread, ragged
+    (8, 300, 5128, "bf16", True, 0.0),     # 641 packs, 9 segments: the 448-consumer build
 ], ids=lambda c: "W%d_T%d_H%d_%s_res%d_wb%g" % c)
 def test_per_tensor_fp8(kctx, ctx, case, kern, norm):
     """Without norm_out the second pass forms the codes from the stored new
