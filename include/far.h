@@ -114,7 +114,9 @@ typedef enum {
  * FAR_RING_GAMMA_SMEM=1|0: gamma staged in shared memory or read through
  * L1, FAR_RING_WIDE=1|0: the 384-consumer build for rows of 1025-1536
  * packs, FAR_RING_WIDE2=1|0: the 448-consumer build for rows of 513-896
- * packs, where the rules take them (each replaces its part of the default
+ * packs, FAR_RING_WIDE1=1|0: the one-CTA 512-consumer build for rows of
+ * 1537-2048 packs, where the rules take them (each replaces its part of
+ * the default
  * geometry, which follows rules
  * measured on B200 by row length, segments per row and whether norm_out is
  * written: plan_ring in reduce_residual_add_b200/csrc/far_abi.cu),

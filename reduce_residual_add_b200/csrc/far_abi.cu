@@ -32,7 +32,8 @@ struct far_ctx {
   int tensor_fused;     // per-tensor FP8: both passes in one ring launch when possible
   int ring_gamma_mode;
   int ring_wide;        // the wide ring build for rows of 1025-1536 packs (1 / 0)
-  int ring_wide2;       // the wide 2-pack build for rows of 513-896 packs (1 / 0)  // ring: 1 stage gamma in shared memory, 0 read it through L1, -1 by rule
+  int ring_wide2;       // the wide 2-pack build for rows of 513-896 packs (1 / 0)
+  int ring_wide1;       // the one-CTA wide build for rows of 1537-2048 packs (1 / 0)  // ring: 1 stage gamma in shared memory, 0 read it through L1, -1 by rule
   int pdl;              // programmatic dependent launch on every call
   int ring_min_rows;    // fewer rows than this take the direct kernel
   uint64_t wait_limit_ns;  // bounded waits in the kernels give up after this
@@ -197,7 +198,15 @@ int ring_occ_cached(const far_ctx* ctx, int dtype, int vpt, int minb, int thread
 //    6 segments: the wide build, 4 packs per thread over up to 384
 //    consumers, 2 CTAs per SM, about 72 KiB of slots (W=2/3/4/8 at
 //    H=10240: 94-97 vs 76-89 %; at H=12288: 86-98 vs 80-91 %; with
-//    norm_out and at most 6 segments it lost, 83-91 vs 86-94 %);
+//    norm_out and at most 6 segments it lost, 83-91 vs 86-94 %); for at
+//    most 4 segments gamma through L1 and a slot per segment (W=2 at
+//    H=10240 / 12288: 97.7 / 96.6 vs 94.6 / 84.1 %; W=3: 98.0 / 99.1 vs
+//    95.8 / 98.1 %);
+//  * 1537-2048 packs (H = 12296-16384) without norm_out, or with more than
+//    6 segments: the one-CTA wide build, 4 packs per thread over up to 512
+//    consumers, one CTA per SM, 6 slots (W=2/3/4/8 at H=16384: 88-96 vs
+//    85-90 %; at H=14336: 85-97 vs 80-89 %; with norm_out and 3-5
+//    segments it lost up to 9 points);
 //  * 8 packs per thread (H >= 12288): 2 CTAs per SM, with the build whose
 //    registers are sized for two, about 72 KiB of slots (H=12288, W=2..8:
 //    80-93 vs 58-84 % at one CTA); but one CTA per SM with 6 slots when the
@@ -238,19 +247,34 @@ bool plan_ring(const far_ctx* ctx, int packs, int64_t rows, int dtype, int segs,
   // up to 448 consumers
   const bool wide2 = ctx->ring_wide2 && !ctx->ring_threads_set && !group && packs > 512 &&
                      packs <= 2 * far::kRingWide2Consumers && segs >= 8;
-  const bool wide = wide4 || wide2;
-  if (wide4) vpt = 4;
+  // rows of 1537-2048 packs without norm_out (or with more than 6
+  // segments): one CTA per SM of up to 512 consumers, 4 packs each
+  const bool wide1 = ctx->ring_wide1 && !ctx->ring_threads_set && !group && packs > 1536 &&
+                     packs <= 4 * far::kRingWide1Consumers && (!norm || segs > 6);
+  const bool wide = wide4 || wide2 || wide1;
+  if (wide4 || wide1) vpt = 4;
   if (wide2) vpt = 2;
   const int tpr = (((packs + vpt - 1) / vpt) + 31) / 32 * 32;
-  if (tpr > (wide4 ? far::kRingWideConsumers : wide2 ? far::kRingWide2Consumers : far::kRingMaxConsumers))
+  if (tpr > (wide1 ? far::kRingWide1Consumers : wide4 ? far::kRingWideConsumers
+                                              : wide2 ? far::kRingWide2Consumers
+                                                      : far::kRingMaxConsumers))
     return false;
 
   int n_req = 2;
   bool gamma_smem = true;
   int want = 0;            // slots per CTA (0: by `target` bytes)
   int target = 72 * 1024;  // slot bytes per CTA when want == 0
-  if (wide4) {
-    // 2 CTAs per SM (its registers are sized for two), about 72 KiB of slots
+  if (wide1) {
+    n_req = 1;
+    want = 6;
+  } else if (wide4) {
+    // 2 CTAs per SM (its registers are sized for two), about 72 KiB of
+    // slots; for rows of at most 4 segments gamma through L1 and one slot
+    // per segment
+    if (segs <= 4) {
+      gamma_smem = false;
+      want = segs < 3 ? 3 : segs;
+    }
   } else if (wide2) {
     // 2 CTAs per SM, about 56 KiB of slots each
     want = 56 * 1024 / seg;
@@ -325,7 +349,7 @@ bool plan_ring(const far_ctx* ctx, int packs, int64_t rows, int dtype, int segs,
   const int smem = far::ring_header_bytes(nslot) + (nslot + gsegs) * seg;
   // the register budget the kernel is built for: 3 or 2 CTAs per SM, and at
   // 8 packs per thread 1 (no spills) or 2 (a few spilled registers)
-  const int minb = wide ? 2 : vpt >= 8 ? (n_req >= 2 ? 2 : 1) : (n_req >= 3 ? 3 : 2);
+  const int minb = wide1 ? 1 : wide ? 2 : vpt >= 8 ? (n_req >= 2 ? 2 : 1) : (n_req >= 3 ? 3 : 2);
   int occ = ring_occ_cached(ctx, dtype, vpt, minb, tpr + 32, smem);
   if (occ < 1) return false;
   if (occ > n_req) occ = n_req;
@@ -482,6 +506,7 @@ far_status far_create(far_ctx** ctx, int device) {
   c.ring_gamma_mode = env_int("FAR_RING_GAMMA_SMEM", -1);
   c.ring_wide = env_int("FAR_RING_WIDE", 1) != 0 ? 1 : 0;
   c.ring_wide2 = env_int("FAR_RING_WIDE2", 1) != 0 ? 1 : 0;
+  c.ring_wide1 = env_int("FAR_RING_WIDE1", 1) != 0 ? 1 : 0;
   if (c.ring_gamma_mode > 1) c.ring_gamma_mode = 1;
   if (c.ring_gamma_mode < -1) c.ring_gamma_mode = -1;
   if (c.ring_slots_max < 0) c.ring_slots_max = 0;

@@ -17,6 +17,8 @@ constexpr int kRingWideConsumers = 384;   // ... of the wide build (4 packs per 
                                           // rows of 1025-1536 packs, 2 CTAs per SM)
 constexpr int kRingWide2Consumers = 448;  // ... of the wide 2-pack build (rows of
                                           // 513-896 packs, 2 CTAs per SM)
+constexpr int kRingWide1Consumers = 512;  // ... of the one-CTA wide build (4 packs
+                                          // per thread, rows of 1537-2048 packs)
 
 enum Dtype : int { kBf16 = 0, kFp16 = 1 };
 enum Pattern : int {

@@ -1397,7 +1397,9 @@ cudaError_t launch_ring_g(const Params& p, const Launch& l, cudaStream_t s) {
       return three ? launch_ring_t<DT, 2, 3, MODE>(p, l, s) : launch_ring_t<DT, 2, 2, MODE>(p, l, s);
     case 4:
       if constexpr (MODE != kModeGroup)
-        if (l.ring_wide) return launch_ring_t<DT, 4, 2, MODE, kRingWideConsumers>(p, l, s);
+        if (l.ring_wide)
+          return l.ring_minb == 1 ? launch_ring_t<DT, 4, 1, MODE, kRingWide1Consumers>(p, l, s)
+                                  : launch_ring_t<DT, 4, 2, MODE, kRingWideConsumers>(p, l, s);
       return three ? launch_ring_t<DT, 4, 3, MODE>(p, l, s) : launch_ring_t<DT, 4, 2, MODE>(p, l, s);
     case 8: return l.ring_minb >= 2 ? launch_ring_t<DT, 8, 2, MODE>(p, l, s)
                                     : launch_ring_t<DT, 8, 1, MODE>(p, l, s);
@@ -1505,6 +1507,8 @@ cudaError_t allow_large_smem() {
   set(far_ring_kernel<DT, 4, 2, kModeTensor, kRingWideConsumers>);
   set(far_ring_kernel<DT, 2, 2, kModePlain, kRingWide2Consumers>);
   set(far_ring_kernel<DT, 2, 2, kModeTensor, kRingWide2Consumers>);
+  set(far_ring_kernel<DT, 4, 1, kModePlain, kRingWide1Consumers>);
+  set(far_ring_kernel<DT, 4, 1, kModeTensor, kRingWide1Consumers>);
   return e;
 }
 
@@ -1562,6 +1566,7 @@ int ring_occupancy_dt(int vpt, int minb, int threads, int smem) {
       if (threads > kRingMaxConsumers + 32) return occ_of<DT, 2, 2, kRingWide2Consumers>(threads, smem);
       return three ? occ_of<DT, 2, 3>(threads, smem) : occ_of<DT, 2, 2>(threads, smem);
     case 4:
+      if (threads > kRingWideConsumers + 32) return occ_of<DT, 4, 1, kRingWide1Consumers>(threads, smem);
       if (threads > kRingMaxConsumers + 32) return occ_of<DT, 4, 2, kRingWideConsumers>(threads, smem);
       return three ? occ_of<DT, 4, 3>(threads, smem) : occ_of<DT, 4, 2>(threads, smem);
     case 8: return minb >= 2 ? occ_of<DT, 8, 2>(threads, smem) : occ_of<DT, 8, 1>(threads, smem);

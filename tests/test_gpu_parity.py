@@ -141,10 +141,12 @@ def test_prefill_kernels(kctx, case, kern):
 @pytest.mark.parametrize("case", [
     (2, 1200, 12288, "bf16", 1, 0.0),   # 1536 packs: 384 consumers
     (3, 700, 10248, "fp16", 2, 1.0),    # 1281 packs, ragged: 352 consumers
+    (2, 600, 16384, "bf16", 1, 0.0),    # 2048 packs: one CTA of 512 consumers
+    (3, 400, 14344, "fp16", 2, 1.0),    # 1793 packs, ragged: 480 consumers
 ], ids=lambda c: "W%d_T%d_H%d_%s_p%d_wb%g" % c)
 def test_ring_wide_build(kctx, case):
-    """Rows of 1025-1536 packs without norm_out take the wide build (4 packs
-    per thread over up to 384 consumers)."""
+    """Rows of 1025-2048 packs without norm_out take a wide build (4 packs
+    per thread over up to 384 or 512 consumers)."""
     W, T, H, dt, pattern, wb = case
     c = kctx["ring"]
     info = far.far_describe_launch(c, T, H, torch.bfloat16, W, True, False)
@@ -450,11 +452,16 @@ def test_launch_plan(ctx):
     assert (h12["packs_per_thread"], h12["threads_per_cta"], h12["grid_ctas"], h12["ring_slots"]) == (4, 416, 2 * sms, 3)
     # ... with norm_out and at most 6 segments, 8 packs per thread
     assert d(8192, 12288, 2, norm=True)["packs_per_thread"] == 8
-    # 8 packs per thread: 2 CTAs per SM, gamma in shared memory ...
+    # 1537-2048 packs without norm_out: one CTA per SM of 512 consumers, 6 slots
     h16 = d(8192, 16384, 2)
-    assert (h16["kernel"], h16["grid_ctas"], h16["ring_gamma_smem"], h16["ring_slots"]) == (1, 2 * sms, 1, 2)
-    # ... but one CTA per SM with 6 slots for many segments of which only 2 would fit
-    h16w8 = d(8192, 16384, 8)
+    assert (h16["kernel"], h16["grid_ctas"], h16["ring_gamma_smem"], h16["ring_slots"]) == (1, sms, 1, 6)
+    assert (h16["packs_per_thread"], h16["threads_per_cta"]) == (4, 544)
+    # ... with norm_out and at most 6 segments: 8 packs per thread, 2 CTAs
+    # per SM, gamma in shared memory
+    h16n = d(8192, 16384, 2, norm=True)
+    assert (h16n["packs_per_thread"], h16n["grid_ctas"], h16n["ring_slots"]) == (8, 2 * sms, 2)
+    # ... with more segments, the one-CTA build with 6 slots
+    h16w8 = d(8192, 16384, 8, norm=True)
     assert (h16w8["grid_ctas"], h16w8["ring_gamma_smem"], h16w8["ring_slots"]) == (sms, 1, 6)
     # rows of at most 256 packs: 128 consumers, 6 CTAs per SM x 4 slots
     # (4 x 6 with norm_out)
