@@ -766,6 +766,29 @@ def test_bounded_wait_gives_up_reports_timeout_and_context_stays_usable(kctx):
     compare(got, ref, "bf16")
 
 
+def test_per_tensor_fused_alongside_other_work(kctx, ctx):
+    """The one-launch per-tensor form waits for rows, not for CTAs: with
+    GEMMs holding SMs on another stream while it runs (so its CTAs start as
+    those free up), it completes, no wait gives up, and its outputs match
+    the oracle."""
+    c = kctx["ring_fused"]
+    W, T, H = 4, 2048, 8192
+    inp = random_inputs(W, T, H, dtype="bf16", seed=4242, has_residual=True)
+    g = to_gpu(inp)
+    a = torch.randn(8192, 8192, device="cuda", dtype=torch.bfloat16)
+    side = torch.cuda.Stream()
+    torch.cuda.synchronize()
+    with torch.cuda.stream(side):
+        for _ in range(24):
+            b = a @ a
+    got = run_gpu(c, g, 1e-6, 0.0, 3, guard=512, want_norm=False)
+    ref = run_oracle(inp, "bf16", 1e-6, 0.0, 3, want_norm=False)
+    st = compare(got, ref, "bf16")
+    log("tensor fused alongside GEMMs", st)
+    assert st["quant_out"][1] > 0.95
+    del b
+
+
 def test_per_tensor_fused_bounded_waits(kctx):
     """Per-tensor FP8 in one ring launch (both passes, a grid barrier between
     them): a skipped bulk copy makes the consumers' wait give up; every CTA
