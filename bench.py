@@ -673,10 +673,14 @@ def extras(ctx, device, stream) -> dict:
         total, mean = case.time_steps(200, 20, per_launch=True, prepared=short)
         if with_norm:
             name += "+norm_out"
+        med = case.median_launch
         out[name] = {"GB/s": round(case.bytes / mean / 1e9, 1),
                      "launches_per_call": 2 if wl.pattern == 3 else 1,
                      "frac": round(case.bytes / mean / 1e9 / peak, 4),
                      "us_per_call": round(mean * 1e6, 2), "tokens_per_s": round(wl.T / mean, 1),
+                     "median_us_per_call": round(med * 1e6, 2),
+                     "frac_on_median": round(case.bytes / med / 1e9 / peak, 4),
+                     "traffic": None if with_norm else profiled_traffic(wl.name),
                      "bytes": case.bytes,
                      "stream_timing": ("far.FarCall per call, per-launch events" if short
                                        else "far binding per call, per-launch events")}

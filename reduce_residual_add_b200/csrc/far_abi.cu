@@ -194,14 +194,14 @@ int ring_occ_cached(const far_ctx* ctx, int dtype, int vpt, int minb, int thread
 //    consumers, 2 CTAs per SM, about 56 KiB of slots each (W=8 at H=4608,
 //    5120, 6144, 7168: 98-101 vs 93-98 %, per-token H=7168: 99.4 vs 97.1 %;
 //    at 3-5 segments it lost as often as it won);
-//  * 1025-1536 packs (H = 8200-12288) without norm_out, or with more than
-//    6 segments: the wide build, 4 packs per thread over up to 384
-//    consumers, 2 CTAs per SM, about 72 KiB of slots (W=2/3/4/8 at
-//    H=10240: 94-97 vs 76-89 %; at H=12288: 86-98 vs 80-91 %; with
-//    norm_out and at most 6 segments it lost, 83-91 vs 86-94 %); for at
-//    most 4 segments gamma through L1 and a slot per segment (W=2 at
-//    H=10240 / 12288: 97.7 / 96.6 vs 94.6 / 84.1 %; W=3: 98.0 / 99.1 vs
-//    95.8 / 98.1 %);
+//  * 1025-1536 packs (H = 8200-12288): the wide build, 4 packs per thread
+//    over up to 384 consumers, 2 CTAs per SM, about 72 KiB of slots (W=2/
+//    3/4/8 at H=10240: 94-97 vs 76-89 %; at H=12288: 86-98 vs 80-91 %);
+//    for at most 4 segments gamma through L1 and a slot per segment (W=2
+//    at H=10240 / 12288: 97.7 / 96.6 vs 94.6 / 84.1 %; W=3: 98.0 / 99.1
+//    vs 95.8 / 98.1 %); with norm_out and at most 6 segments gamma through
+//    L1 and 2 slots (W=2/3/4 at H=10240 / 12288: 92-97 vs 86-94 %, where
+//    the default slots lost);
 //  * 1537-2048 packs (H = 12296-16384) without norm_out, or with more than
 //    6 segments: the one-CTA wide build, 4 packs per thread over up to 512
 //    consumers, one CTA per SM, 6 slots (W=2/3/4/8 at H=16384: 88-96 vs
@@ -238,11 +238,10 @@ bool plan_ring(const far_ctx* ctx, int packs, int64_t rows, int dtype, int segs,
   int vpt = 1;
   while (vpt < 8 && (packs + vpt - 1) / vpt > max_cons) vpt *= 2;
   if (!ctx->ring_threads_set && segs <= 6 && packs >= 512 && packs < 1024 && vpt < 4) vpt = 4;
-  // rows of 1025-1536 packs without norm_out (or with more than 6
-  // segments): the wide build, 4 packs per thread over up to 384 consumers,
-  // instead of 8 packs per thread
+  // rows of 1025-1536 packs: the wide build, 4 packs per thread over up to
+  // 384 consumers, instead of 8 packs per thread
   const bool wide4 = ctx->ring_wide && !ctx->ring_threads_set && !group && packs > 1024 &&
-                     packs <= 4 * far::kRingWideConsumers && (!norm || segs > 6);
+                     packs <= 4 * far::kRingWideConsumers;
   // rows of 513-896 packs with 8 or more segments: 2 packs per thread over
   // up to 448 consumers
   const bool wide2 = ctx->ring_wide2 && !ctx->ring_threads_set && !group && packs > 512 &&
@@ -270,8 +269,12 @@ bool plan_ring(const far_ctx* ctx, int packs, int64_t rows, int dtype, int segs,
   } else if (wide4) {
     // 2 CTAs per SM (its registers are sized for two), about 72 KiB of
     // slots; for rows of at most 4 segments gamma through L1 and one slot
-    // per segment
-    if (segs <= 4) {
+    // per segment; with norm_out and at most 6 segments gamma through L1
+    // and 2 slots
+    if (norm && segs <= 6) {
+      gamma_smem = false;
+      want = 2;
+    } else if (segs <= 4) {
       gamma_smem = false;
       want = segs < 3 ? 3 : segs;
     }

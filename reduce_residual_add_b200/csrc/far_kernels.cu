@@ -14,18 +14,21 @@
 // The work is HBM-bound (about 8 flops per (W+3)*2 bytes): no tensor cores.
 // A whole row stays in registers between its reduction and its scaling, so
 // every byte crosses HBM once.  Four kernels, three of which share one row
-// routine (finish_row):
+// routine (finish_row), and a one-CTA helper:
 //  - far_ring_kernel (prefill, many rows): persistent CTAs; one producer
 //    thread streams each row's segments with TMA bulk copies into a ring of
-//    shared-memory slots, the consumer warps fold them into registers;
+//    shared-memory slots, the consumer warps fold them into registers; for
+//    dynamic per-tensor FP8 it also runs both passes in one launch (rows
+//    taken from a counter, a bounded wait until every row is done);
 //  - far_prefill_kernel (fewer rows): one CTA per row (or 256/tpr rows per
 //    CTA when a row has at most 32 packs), 16-byte vector loads issued
 //    ahead of their use, warp-shuffle + shared-memory reductions;
 //  - far_decode_kernel (a few long rows): one thread-block cluster per row,
 //    each CTA a slice of the hidden dimension, the row's sum of squares
 //    (and amax) combined through distributed shared memory;
-//  - far_tensor_quant_kernel: the second pass of dynamic per-tensor FP8,
-//    codes from the stored new residual (no reduction).
+//  - far_tensor_quant_kernel: the second pass of dynamic per-tensor FP8 in
+//    its two-kernel form, codes from the stored new residual (no reduction);
+//  - far_ws_zero_kernel: zeroes the per-tensor workspace header.
 #include <cooperative_groups.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>

@@ -450,8 +450,9 @@ def test_launch_plan(ctx):
     # 1025-1536 packs without norm_out: the wide build, 4 packs per thread
     h12 = d(8192, 12288, 2)
     assert (h12["packs_per_thread"], h12["threads_per_cta"], h12["grid_ctas"], h12["ring_slots"]) == (4, 416, 2 * sms, 3)
-    # ... with norm_out and at most 6 segments, 8 packs per thread
-    assert d(8192, 12288, 2, norm=True)["packs_per_thread"] == 8
+    # ... with norm_out and at most 6 segments, gamma through L1 and 2 slots
+    h12n = d(8192, 12288, 2, norm=True)
+    assert (h12n["packs_per_thread"], h12n["ring_gamma_smem"], h12n["ring_slots"]) == (4, 0, 2)
     # 1537-2048 packs without norm_out: one CTA per SM of 512 consumers, 6 slots
     h16 = d(8192, 16384, 2)
     assert (h16["kernel"], h16["grid_ctas"], h16["ring_gamma_smem"], h16["ring_slots"]) == (1, sms, 1, 6)
