@@ -33,7 +33,8 @@ struct far_ctx {
   int ring_gamma_mode;
   int ring_wide;        // the wide ring build for rows of 1025-1536 packs (1 / 0)
   int ring_wide2;       // the wide 2-pack build for rows of 513-896 packs (1 / 0)
-  int ring_wide1;       // the one-CTA wide build for rows of 1537-2048 packs (1 / 0)  // ring: 1 stage gamma in shared memory, 0 read it through L1, -1 by rule
+  int ring_wide1;       // the one-CTA wide build for rows of 1537-2048 packs (1 / 0)
+  int ring_wide_group;  // per-group FP8 also takes the 384- and 512-consumer builds (1 / 0)  // ring: 1 stage gamma in shared memory, 0 read it through L1, -1 by rule
   int pdl;              // programmatic dependent launch on every call
   int ring_min_rows;    // fewer rows than this take the direct kernel
   uint64_t wait_limit_ns;  // bounded waits in the kernels give up after this
@@ -212,14 +213,16 @@ int ring_occ_cached(const far_ctx* ctx, int dtype, int vpt, int minb, int thread
 //    80-93 vs 58-84 % at one CTA); but one CTA per SM with 6 slots when the
 //    row has more than 6 segments and fewer than 3 slots fit the 2-CTA share
 //    (H=16384, W=8: 87-90 %).
-// Per-group FP8 (more work per row, and more registers) keeps the rule that
-// won for it: about 72 KiB of slots per CTA, 3 CTAs per SM for rows of at
-// most 6 segments, else 2; 4 for rows of at most 256 packs and, without
-// norm_out, up to 640 packs with at most 6 segments; with norm_out and at
-// most 6 segments, 2 CTAs per SM for segments of 10-12 KiB, and for
-// segments of at least 16 KiB 2 with gamma through L1 and about 96 KiB of
-// slots (W=4 / 8 at H=4096 / 7168, with and without norm_out: mean 90.3
-// against 86.5 % with the rule above).
+// Per-group FP8 (more work per row, and more registers) has a rule of its
+// own, from a sweep of CTAs per SM x slots at H = 2048-12288, W = 2, 4, 8,
+// with and without norm_out: 4 CTAs per SM x 6 slots up to 256 packs,
+// 4 x 4 up to 640 (4 x 6 beyond 6 segments), 3 x 3 up to 1024 (W=8 at
+// H=4096 / 5120: 96-99 vs 79-90 %; with norm_out at H=4096 / 5120 / 8192,
+// W=2-4: 83-95 vs 63-87 %; the rule above lost for it: mean 86.5 against
+// 90.3 % at W=4 / 8, H=4096 / 7168).  Beyond 1024 packs it takes the 384-
+// and 512-consumer builds (the one-CTA build with norm_out too), whose
+// registers do not spill as 8 packs per thread do (H = 10240-16384:
+// 65-97 vs 49-81 %).
 // Gamma is staged in shared memory unless said otherwise; where the slots
 // asked for do not fit, as many as fit; below 2 (below 3 for the byte
 // targets), the rule falls back to 2 CTAs per SM with gamma through L1.
@@ -240,16 +243,17 @@ bool plan_ring(const far_ctx* ctx, int packs, int64_t rows, int dtype, int segs,
   if (!ctx->ring_threads_set && segs <= 6 && packs >= 512 && packs < 1024 && vpt < 4) vpt = 4;
   // rows of 1025-1536 packs: the wide build, 4 packs per thread over up to
   // 384 consumers, instead of 8 packs per thread
-  const bool wide4 = ctx->ring_wide && !ctx->ring_threads_set && !group && packs > 1024 &&
-                     packs <= 4 * far::kRingWideConsumers;
+  const bool wide4 = ctx->ring_wide && !ctx->ring_threads_set && (!group || ctx->ring_wide_group) &&
+                     packs > 1024 && packs <= 4 * far::kRingWideConsumers;
   // rows of 513-896 packs with 8 or more segments: 2 packs per thread over
   // up to 448 consumers
   const bool wide2 = ctx->ring_wide2 && !ctx->ring_threads_set && !group && packs > 512 &&
                      packs <= 2 * far::kRingWide2Consumers && segs >= 8;
   // rows of 1537-2048 packs without norm_out (or with more than 6
   // segments): one CTA per SM of up to 512 consumers, 4 packs each
-  const bool wide1 = ctx->ring_wide1 && !ctx->ring_threads_set && !group && packs > 1536 &&
-                     packs <= 4 * far::kRingWide1Consumers && (!norm || segs > 6);
+  const bool wide1 = ctx->ring_wide1 && !ctx->ring_threads_set && (!group || ctx->ring_wide_group) &&
+                     packs > 1536 && packs <= 4 * far::kRingWide1Consumers &&
+                     (!norm || segs > 6 || group);
   const bool wide = wide4 || wide2 || wide1;
   if (wide4 || wide1) vpt = 4;
   if (wide2) vpt = 2;
@@ -292,16 +296,16 @@ bool plan_ring(const far_ctx* ctx, int packs, int64_t rows, int dtype, int segs,
       target = 6 * seg;
     }
   } else if (group) {
-    // per-group FP8 (more work per row): about 72 KiB of slots per CTA
-    n_req = segs <= 6 ? 3 : 2;
-    if (packs <= 256 || (!norm && segs <= 6 && packs <= 640)) {
+    // per-group FP8 (more work per row), measured on its own
+    if (packs <= 256) {
       n_req = 4;
-    } else if (norm && segs <= 6 && seg >= 16 * 1024) {
-      n_req = 2;
-      gamma_smem = false;
-      target = 96 * 1024;
-    } else if (norm && segs <= 6 && seg >= 10 * 1024 && seg <= 12 * 1024) {
-      n_req = 2;
+      want = 6;
+    } else if (packs <= 640) {
+      n_req = 4;
+      want = segs > 6 ? 6 : 4;
+    } else {
+      n_req = 3;
+      want = 3;
     }
   } else if (packs <= 256) {
     n_req = norm ? 4 : 6;
@@ -510,6 +514,7 @@ far_status far_create(far_ctx** ctx, int device) {
   c.ring_wide = env_int("FAR_RING_WIDE", 1) != 0 ? 1 : 0;
   c.ring_wide2 = env_int("FAR_RING_WIDE2", 1) != 0 ? 1 : 0;
   c.ring_wide1 = env_int("FAR_RING_WIDE1", 1) != 0 ? 1 : 0;
+  c.ring_wide_group = env_int("FAR_RING_WIDE_GROUP", 1) != 0 ? 1 : 0;
   if (c.ring_gamma_mode > 1) c.ring_gamma_mode = 1;
   if (c.ring_gamma_mode < -1) c.ring_gamma_mode = -1;
   if (c.ring_slots_max < 0) c.ring_slots_max = 0;

@@ -1399,10 +1399,9 @@ cudaError_t launch_ring_g(const Params& p, const Launch& l, cudaStream_t s) {
         if (l.ring_wide) return launch_ring_t<DT, 2, 2, MODE, kRingWide2Consumers>(p, l, s);
       return three ? launch_ring_t<DT, 2, 3, MODE>(p, l, s) : launch_ring_t<DT, 2, 2, MODE>(p, l, s);
     case 4:
-      if constexpr (MODE != kModeGroup)
-        if (l.ring_wide)
-          return l.ring_minb == 1 ? launch_ring_t<DT, 4, 1, MODE, kRingWide1Consumers>(p, l, s)
-                                  : launch_ring_t<DT, 4, 2, MODE, kRingWideConsumers>(p, l, s);
+      if (l.ring_wide)
+        return l.ring_minb == 1 ? launch_ring_t<DT, 4, 1, MODE, kRingWide1Consumers>(p, l, s)
+                                : launch_ring_t<DT, 4, 2, MODE, kRingWideConsumers>(p, l, s);
       return three ? launch_ring_t<DT, 4, 3, MODE>(p, l, s) : launch_ring_t<DT, 4, 2, MODE>(p, l, s);
     case 8: return l.ring_minb >= 2 ? launch_ring_t<DT, 8, 2, MODE>(p, l, s)
                                     : launch_ring_t<DT, 8, 1, MODE>(p, l, s);
@@ -1512,6 +1511,8 @@ cudaError_t allow_large_smem() {
   set(far_ring_kernel<DT, 2, 2, kModeTensor, kRingWide2Consumers>);
   set(far_ring_kernel<DT, 4, 1, kModePlain, kRingWide1Consumers>);
   set(far_ring_kernel<DT, 4, 1, kModeTensor, kRingWide1Consumers>);
+  set(far_ring_kernel<DT, 4, 2, kModeGroup, kRingWideConsumers>);
+  set(far_ring_kernel<DT, 4, 1, kModeGroup, kRingWide1Consumers>);
   return e;
 }
 

@@ -859,7 +859,9 @@ def test_format_edges_overflow_and_subnormals(kctx, kern):
     (3, 40, 256, 16, "bf16"),
     (4, 300, 8192, 128, "bf16"),
     (8, 150, 7168, 128, "fp16"),
-    (2, 30, 16384, 256, "bf16"),
+    (2, 30, 16384, 256, "bf16"),    # 2048 packs: one CTA of 512 consumers
+    (3, 200, 12288, 128, "bf16"),   # 1536 packs: 384 consumers
+    (8, 60, 10240, 64, "fp16"),     # 1280 packs: 320 consumers
     (5, 70, 1000, 8, "bf16"),       # ragged H: 125 packs
     (8, 4, 4096, 32, "bf16"),       # decode-sized
 ], ids=lambda c: "W%d_T%d_H%d_G%d_%s" % c)
