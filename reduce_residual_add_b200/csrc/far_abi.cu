@@ -205,9 +205,9 @@ int ring_occ_cached(const far_ctx* ctx, int dtype, int vpt, int minb, int thread
 //    the default slots lost);
 //  * 1537-2048 packs (H = 12296-16384) without norm_out, or with more than
 //    6 segments: the one-CTA wide build, 4 packs per thread over up to 512
-//    consumers, one CTA per SM, 6 slots (W=2/3/4/8 at H=16384: 88-96 vs
-//    85-90 %; at H=14336: 85-97 vs 80-89 %; with norm_out and 3-5
-//    segments it lost up to 9 points);
+//    consumers, one CTA per SM, 6 slots, 4 for rows of at most 4 segments
+//    (W=2/3/4/8 at H=16384: 88-98 vs 85-90 %; at H=14336: 88-97 vs
+//    80-89 %; with norm_out and 3-5 segments it lost up to 9 points);
 //  * 8 packs per thread (H >= 12288): 2 CTAs per SM, with the build whose
 //    registers are sized for two, about 72 KiB of slots (H=12288, W=2..8:
 //    80-93 vs 58-84 % at one CTA); but one CTA per SM with 6 slots when the
@@ -268,8 +268,10 @@ bool plan_ring(const far_ctx* ctx, int packs, int64_t rows, int dtype, int segs,
   int want = 0;            // slots per CTA (0: by `target` bytes)
   int target = 72 * 1024;  // slot bytes per CTA when want == 0
   if (wide1) {
+    // one CTA per SM; 4 slots for rows of at most 4 segments without
+    // norm_out (W=2/3 at H=14336 / 16384: 88-98 vs 85-95 % with 6), else 6
     n_req = 1;
-    want = 6;
+    want = (!norm && segs <= 4) ? 4 : 6;
   } else if (wide4) {
     // 2 CTAs per SM (its registers are sized for two), about 72 KiB of
     // slots; for rows of at most 4 segments gamma through L1 and one slot

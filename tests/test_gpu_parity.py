@@ -453,9 +453,11 @@ def test_launch_plan(ctx):
     # ... with norm_out and at most 6 segments, gamma through L1 and 2 slots
     h12n = d(8192, 12288, 2, norm=True)
     assert (h12n["packs_per_thread"], h12n["ring_gamma_smem"], h12n["ring_slots"]) == (4, 0, 2)
-    # 1537-2048 packs without norm_out: one CTA per SM of 512 consumers, 6 slots
+    # 1537-2048 packs without norm_out: one CTA per SM of 512 consumers, 4
+    # slots for at most 4 segments (6 beyond)
     h16 = d(8192, 16384, 2)
-    assert (h16["kernel"], h16["grid_ctas"], h16["ring_gamma_smem"], h16["ring_slots"]) == (1, sms, 1, 6)
+    assert (h16["kernel"], h16["grid_ctas"], h16["ring_gamma_smem"], h16["ring_slots"]) == (1, sms, 1, 4)
+    assert d(8192, 16384, 4)["ring_slots"] == 6
     assert (h16["packs_per_thread"], h16["threads_per_cta"]) == (4, 544)
     # ... with norm_out and at most 6 segments: 8 packs per thread, 2 CTAs
     # per SM, gamma in shared memory
