@@ -56,7 +56,7 @@ def kctx():
     and the direct-load kernel."""
     any_rows = {"FAR_RING_MIN_ROWS": "1"}
     out = {"ring": _ctx_with_env(dict(any_rows)),
-           # per-tensor FP8: both passes in one cooperative launch (the
+           # per-tensor FP8: both passes in one ring launch (the
            # default), and in two kernels
            "ring_fused": _ctx_with_env(dict(any_rows, FAR_TENSOR_FUSED="1")),
            "ring_two": _ctx_with_env(dict(any_rows, FAR_TENSOR_FUSED="0")),
@@ -793,10 +793,11 @@ def test_per_tensor_fused_alongside_other_work(kctx, ctx):
 
 
 def test_per_tensor_fused_bounded_waits(kctx):
-    """Per-tensor FP8 in one ring launch (both passes, a grid barrier between
-    them): a skipped bulk copy makes the consumers' wait give up; every CTA
-    still reaches the grid barrier, the kernel ends, far_check reports
-    FAR_ERR_TIMEOUT, and the next call on the context is correct."""
+    """Per-tensor FP8 in one ring launch (both passes, a bounded wait for
+    every row between them): a skipped bulk copy makes the consumers' wait
+    give up, so not every row is done and the wait between the passes gives
+    up too; the kernel ends, far_check reports FAR_ERR_TIMEOUT, and the next
+    call on the context is correct."""
     c = kctx["ring_fused"]
     T, H = 600, 4096
     inp = random_inputs(4, T, H, seed=72)
