@@ -85,7 +85,10 @@ REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_c
 
 
 class ClockSampler(threading.Thread):
-    def __init__(self, device: int, period_s: float = 0.001):
+    """NVML SM clock and clock-event reasons, sampled from a thread while the
+    timed region runs (every `period_s`, the reasons every few samples), plus
+    one sample taken as the region ends."""
+    def __init__(self, device: int, period_s: float = 0.0002):
         super().__init__(daemon=True)
         self.period = period_s
         self.samples = []
@@ -113,23 +116,31 @@ class ClockSampler(threading.Thread):
     def run(self):
         if not self.ok:
             return
-        nv = self.nv
+        i = 0
         while not self._halt.is_set():
-            try:
-                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+            self._sample(reasons=(i % 5 == 0))
+            i += 1
+            time.sleep(self.period)
+
+    def _sample(self, reasons: bool = True):
+        nv = self.nv
+        try:
+            self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+            if reasons:
                 try:
                     r = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
                 except AttributeError:
                     r = nv.nvmlDeviceGetCurrentClocksThrottleReasons(self.h)
                 self.reasons |= int(r) & ~0x1
-            except Exception:
-                pass
-            time.sleep(self.period)
+        except Exception:
+            pass
 
     def stop(self) -> dict:
         self._halt.set()
         if self.is_alive():
             self.join(timeout=2)
+        if self.ok:
+            self._sample()  # the state as the timed region ends
         if not self.ok or not self.samples:
             return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
         return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
