@@ -214,12 +214,15 @@ int ring_occ_cached(const far_ctx* ctx, int dtype, int vpt, int minb, int thread
 //    row has more than 6 segments and fewer than 3 slots fit the 2-CTA share
 //    (H=16384, W=8: 87-90 %).
 // Per-group FP8 (more work per row, and more registers) has a rule of its
-// own, from a sweep of CTAs per SM x slots at H = 2048-12288, W = 2, 4, 8,
-// with and without norm_out: 4 CTAs per SM x 6 slots up to 256 packs,
-// 4 x 4 up to 640 (4 x 6 beyond 6 segments), 3 x 3 up to 1024 (W=8 at
-// H=4096 / 5120: 96-99 vs 79-90 %; with norm_out at H=4096 / 5120 / 8192,
-// W=2-4: 83-95 vs 63-87 %; the rule above lost for it: mean 86.5 against
-// 90.3 % at W=4 / 8, H=4096 / 7168).  Beyond 1024 packs it takes the 384-
+// own, from sweeps of CTAs per SM x slots at H = 2048-12288, W = 2-8,
+// with and without norm_out: up to 6 segments, 5 CTAs per SM x 6 slots up
+// to 256 packs and 5 x 4 up to 512 (W=2-4 at H=2048 / 4096: 72-97 vs
+// 65-90 % with 4 CTAs); 4 x 4 up to 640 (4 x 6 beyond 6 segments, and
+// beyond 6 segments from 257 packs); 4 x 4 up to 768 (H=6144, W=2-4:
+// 81-96 vs 69-90 % at 3 x 3); 3 x 3 up to 1024 (W=8 at H=4096 / 5120:
+// 96-99 vs 79-90 %; with norm_out at H=4096 / 5120 / 8192, W=2-4: 83-95
+// vs 63-87 %; the static rule lost for it: mean 86.5 against 90.3 % at
+// W=4 / 8, H=4096 / 7168).  Beyond 1024 packs it takes the 384-
 // and 512-consumer builds (the one-CTA build with norm_out too), whose
 // registers do not spill as 8 packs per thread do (H = 10240-16384:
 // 65-97 vs 49-81 %).
@@ -299,12 +302,15 @@ bool plan_ring(const far_ctx* ctx, int packs, int64_t rows, int dtype, int segs,
     }
   } else if (group) {
     // per-group FP8 (more work per row), measured on its own
-    if (packs <= 256) {
-      n_req = 4;
-      want = 6;
+    if (packs <= 512 && segs <= 6) {
+      n_req = 5;
+      want = packs <= 256 ? 6 : 4;
     } else if (packs <= 640) {
       n_req = 4;
       want = segs > 6 ? 6 : 4;
+    } else if (packs <= 768) {
+      n_req = 4;
+      want = 4;
     } else {
       n_req = 3;
       want = 3;
