@@ -241,23 +241,26 @@ size_t far_fp8_tensor_workspace_bytes(int64_t rows);
  * one-CTA kernel that zeroes the workspace's first four words, and two
  * passes.  The first reads the
  * inputs and keeps each row's 1/rms and the running amax in `workspace`.
- * Without norm_out and with a new residual to write (a residual_out, or a
- * residual updated in place), the first pass also writes the new residual
- * and the second forms o from it -- o = round(y) * rinv * (gamma +
- * weight_bias), round(y) being the new residual in the 2-byte format -- and
- * writes only the codes, so the inputs are read once; each code is then
- * within one step of the code of o formed from y itself, and the scale is
- * the same.  Rows whose sum of squares could hide an element that overflows
- * the format (and rows with an inf or NaN input) are rebuilt from the
- * inputs by the second pass instead.  When the persistent kernel serves
+ * With norm_out, the first pass also writes norm_out and the new residual,
+ * and the second forms the codes from norm_out -- round(o), o in the 2-byte
+ * format -- so the inputs are read once.  Without norm_out and with a new
+ * residual to write (a residual_out, or a residual updated in place), the
+ * first pass also writes the new residual and the second forms o from it
+ * -- o = round(y) * rinv * (gamma + weight_bias), round(y) being the new
+ * residual in the 2-byte format -- and writes only the codes.  Either way
+ * each code is within one step of the code of o itself, and the scale is
+ * the same (it comes from the unrounded o).  Rows whose sum of squares
+ * could hide an element that overflows the format, rows with an inf or NaN
+ * input, and (with norm_out) rows whose amax reaches the format's largest
+ * finite value are rebuilt from the inputs by the second pass instead.  When the persistent kernel serves
  * the call, both passes run in ONE launch: its CTAs take the first pass's
  * rows one at a time from a counter in the workspace, wait (bounded) until
  * every row is done -- a wait on rows, not on CTAs, so the grid need not be
  * co-resident -- then write the codes (FAR_TENSOR_FUSED=0 in the
  * environment at far_create splits them into two kernels); otherwise two
  * kernels run.
- * With norm_out, or with no new residual to write, the second pass reads
- * the inputs again and writes every output.
+ * With neither norm_out nor a new residual to write, the second pass reads
+ * the inputs again.
  * `workspace`: device memory of at least
  * far_fp8_tensor_workspace_bytes(row_end - row_begin) bytes, 256-byte
  * aligned, overlapping no argument; its contents are scratch, and two calls

@@ -790,8 +790,11 @@ far_status far_fused_fp8_tensor_launch(far_ctx* ctx, int64_t row_begin, int64_t 
   p.ws_claim = p.ws_amax + 2;
   p.ws_rinv = reinterpret_cast<float*>(static_cast<unsigned char*>(workspace) + 256);
   p.ws_row0 = row_begin;
-  const bool from_residual = norm_out == nullptr && p.residual_out != nullptr;
-  p.tensor_stores_residual = from_residual ? 1 : 0;
+  // what the second pass forms the codes from: norm_out when the call
+  // writes it (the first pass stores it), else the new residual when there
+  // is one to store, else the inputs read again
+  p.tensor_source = norm_out != nullptr ? 2 : (p.residual_out != nullptr ? 1 : 0);
+  const bool from_stored = p.tensor_source != 0;
   DeviceGuard guard(ctx->device);
   if (guard.err != cudaSuccess) return cuda_fail(guard.err, "cudaSetDevice");
   const cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -816,7 +819,7 @@ far_status far_fused_fp8_tensor_launch(far_ctx* ctx, int64_t row_begin, int64_t 
   // counter, wait until every row is done (a wait on rows, not on CTAs, so
   // no co-residency is needed), then write the codes, the rows taken last
   // first.
-  const bool fused = ctx->tensor_fused && from_residual && first.regime == FAR_REGIME_PREFILL &&
+  const bool fused = ctx->tensor_fused && from_stored && first.regime == FAR_REGIME_PREFILL &&
                      first.kernel == 1 &&
                      row_end - row_begin <= 0x7fffffff;
   if (fused) p.tensor_fused = 1;
@@ -829,7 +832,7 @@ far_status far_fused_fp8_tensor_launch(far_ctx* ctx, int64_t row_begin, int64_t 
   p.pattern = far::kTensorQuant;
   p.reverse = ctx->tensor_reverse;
   far::Launch second = whole;
-  if (from_residual) {
+  if (from_stored) {
     // one CTA per row (or several short rows), loads straight into registers
     plan_prefill(static_cast<int>(H / far::kPackElems), far::kMaxThreads, &second);
     second.kernel = 2;

@@ -58,8 +58,9 @@ struct Params {
   uint64_t wait_limit_ns;       // every bounded wait gives up after this long
   int64_t stall_segment;        // test hook: the ring producer skips this copy (-1: none)
   int reverse;                  // take the rows from row_end - 1 down to row_begin
-  int tensor_stores_residual;   // per-tensor FP8, first pass: store the new residual
-                                // of every row it does not flag for a rebuild
+  int tensor_source;            // per-tensor FP8: what the second pass forms the codes
+                                // from -- 0 the inputs again, 1 the new residual the
+                                // first pass stores, 2 the norm_out it stores
   int tensor_fused;             // per-tensor FP8 in one ring launch: the CTAs take rows
                                 // from a shared counter (ws_claim), wait until every
                                 // row is done (ws_done), then write the codes from the

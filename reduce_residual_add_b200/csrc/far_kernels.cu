@@ -61,7 +61,13 @@ __host__ __device__ constexpr int ring_offset(int nslot) {
 // Which instantiation serves a pattern: the per-group and the per-tensor
 // passes have kernels of their own, so that the other patterns' code carries
 // none of their registers.
-constexpr int kModePlain = 0, kModeGroup = 1, kModeTensor = 2;
+// kModeTensorNorm: per-tensor FP8 whose second pass forms the codes from the
+// norm_out the first pass stores (its own instantiations, so that the other
+// per-tensor forms carry none of that code)
+constexpr int kModePlain = 0, kModeGroup = 1, kModeTensor = 2, kModeTensorNorm = 3;
+__host__ __device__ constexpr bool is_tensor_mode(int mode) {
+  return mode == kModeTensor || mode == kModeTensorNorm;
+}
 __host__ __device__ constexpr int mode_of(int pattern) {
   return pattern == kFp8Group ? kModeGroup
          : (pattern == kTensorAmax || pattern == kTensorQuant) ? kModeTensor
@@ -85,6 +91,7 @@ __device__ __forceinline__ int64_t call_row(const Params& p, int64_t k) {
 struct Bf16T {
   static constexpr bool kIsBf16 = true;
   static constexpr float kOverflowSq = 3.40282347e38f;  // FLT_MAX: y^2 overflows first
+  static constexpr float kMaxFinite = 3.38953139e38f;   // 0x7f7f
   static __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
     __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);  // round to nearest even
     return *reinterpret_cast<uint32_t*>(&h);
@@ -94,6 +101,7 @@ struct Bf16T {
 struct Fp16T {
   static constexpr bool kIsBf16 = false;
   static constexpr float kOverflowSq = 65520.f * 65520.f;  // exact in fp32
+  static constexpr float kMaxFinite = 65504.f;
   static __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
     __half2 h = __floats2half2_rn(lo, hi);  // round to nearest even
     return *reinterpret_cast<uint32_t*>(&h);
@@ -507,7 +515,7 @@ __device__ __forceinline__ uint4 gamma_pack(const Params& p, const uint4* gamma_
   return gamma_smem != nullptr ? gamma_smem[j] : __ldg(static_cast<const uint4*>(p.gamma) + j);
 }
 
-// MODE (kModePlain / kModeGroup / kModeTensor): the patterns this
+// MODE (kModePlain / kModeGroup / kModeTensor / kModeTensorNorm): the patterns this
 // instantiation serves; per-group and per-tensor code is compiled only into
 // their own instantiations, so the other patterns carry none of its registers.
 // GPRE: gamma's packs were loaded by the caller into gpre[k] (pack
@@ -523,10 +531,10 @@ __device__ __forceinline__ void finish_row(const Params& p, int64_t row, bool ro
   };
   const int64_t rbase = row * static_cast<int64_t>(p.packs);  // first pack of the row
   // dynamic per-tensor FP8 runs in two passes: the first records rinv and
-  // the call's amax (and, with p.tensor_stores_residual, the new residual);
+  // the call's amax (and the new residual or norm_out the second pass reads);
   // the second writes the other outputs
-  const bool tensor_amax = MODE == kModeTensor && p.pattern == kTensorAmax;
-  const bool tensor_quant = MODE == kModeTensor && p.pattern == kTensorQuant;
+  const bool tensor_amax = is_tensor_mode(MODE) && p.pattern == kTensorAmax;
+  const bool tensor_quant = is_tensor_mode(MODE) && p.pattern == kTensorQuant;
   if (p.residual_out != nullptr && !tensor_amax) {
 #pragma unroll
     for (int k = 0; k < VPT; ++k)
@@ -593,12 +601,33 @@ __device__ __forceinline__ void finish_row(const Params& p, int64_t row, bool ro
     // infinity: the second pass must rebuild its y from the inputs, so its
     // new residual is not stored here and the row is flagged (sign bit of
     // the stored rinv, which is otherwise +0, positive or +inf).
-    const bool rebuild = !(ss < DT::kOverflowSq);
-    if (p.tensor_stores_residual && !rebuild) {
+    // With norm_out stored for the second pass, a row whose amax reaches
+    // the format's largest finite value (an element of norm_out may be
+    // infinite) is flagged too.  norm_out is written here for every row;
+    // the new residual of a flagged row is left to the second pass (which
+    // rebuilds the row from the inputs, the residual possibly among them).
+    bool rebuild = !(ss < DT::kOverflowSq);
+    if (MODE == kModeTensor && p.tensor_source == 1 && !rebuild) {
       const uint64_t keep = l2_evict_last();
 #pragma unroll
       for (int k = 0; k < VPT; ++k)
         if (ok[k]) st_l2_hint(static_cast<uint4*>(p.residual_out) + rbase + j0 + k * jstride, pack8<DT>(y[k]), keep);
+    }
+    if constexpr (MODE == kModeTensorNorm) {
+      rebuild = rebuild || !(rinv * gmax < DT::kMaxFinite);
+      const uint64_t keep = l2_evict_last();
+#pragma unroll
+      for (int k = 0; k < VPT; ++k) {
+        if (!ok[k]) continue;
+        const int64_t pk = rbase + j0 + k * jstride;
+        if (p.residual_out != nullptr && !rebuild) static_cast<uint4*>(p.residual_out)[pk] = pack8<DT>(y[k]);
+        float g[8];
+        pack_plus<DT>(gamma_k(k), p.weight_bias, g);
+        float o[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) o[i] = (y[k][i] * rinv) * g[i];
+        st_l2_hint(static_cast<uint4*>(p.norm_out) + pk, pack8<DT>(o), keep);
+      }
     }
     if (row_ok && red.leader()) {
       p.ws_rinv[row - p.ws_row0] =
@@ -846,6 +875,30 @@ __device__ __forceinline__ uint2 tensor_codes(const uint4& gam, float wb, float 
   return fp8_codes8(y, scale, inv, exact);
 }
 
+// A pack of eight 1.0 in the 2-byte format: with weight_bias 0 and rinv 1,
+// tensor_codes then forms the codes of the pack it is given as o itself
+// (norm_out read back: o within half an ulp of the 2-byte format), by the
+// same instructions as the codes of round(y).
+template <class DT>
+__device__ __forceinline__ uint4 ones_pack() {
+  const uint32_t one2 = DT::kIsBf16 ? 0x3F803F80u : 0x3C003C00u;
+  return make_uint4(one2, one2, one2, one2);
+}
+
+// The 8 codes of one pack from what the first pass stored: the new residual
+// round(y) (tensor_source 1: o formed as above) or norm_out round(o)
+// (tensor_source 2: o itself).
+template <class DT>
+__device__ __forceinline__ uint2 stored_codes(int source, const uint4& v, const uint4& gam, float wb,
+                                              float rinv, float rs, float scale, float inv,
+                                              bool exact) {
+  float x[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  add_pack<DT>(v, x);  // 0 + x: the 2-byte value widened exactly
+  const bool o = source == 2;
+  return tensor_codes<DT>(o ? ones_pack<DT>() : gam, o ? 0.f : wb, x, o ? 1.f : rinv, o ? inv : rs,
+                          scale, inv, exact);
+}
+
 // One row of the second pass on its own: from the stored new residual, or
 // (a flagged row) rebuilt from the inputs in the first pass's order --
 // partials 0..W-1, then the residual -- with its new residual written here.
@@ -866,17 +919,19 @@ __device__ __forceinline__ void tensor_quant_row(const Params& p, int64_t row, f
   for (int q = 0; q < VPT; ++q) {
     if (!ok[q]) continue;
     const int64_t pk = rbase + j0 + q * tpr;
-    float y[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-    if (!rebuild) {
-      const uint4* src = static_cast<const uint4*>(p.residual_out) + pk;
-      add_pack<DT>(COHERENT ? ld_coherent_l2_hint(src, drop) : ld_once_l2_hint(src, drop), y);
-    } else {
-      for (int r = 0; r < p.W; ++r) add_pack<DT>(ld_once(static_cast<const uint4*>(p.partials[r]) + pk), y);
-      if (p.residual != nullptr)
-        add_pack<DT>(ld_once_coherent(static_cast<const uint4*>(p.residual) + pk), y);
-      static_cast<uint4*>(p.residual_out)[pk] = pack8<DT>(y);
-    }
     const uint4 g = gamma_s != nullptr ? gamma[j0 + q * tpr] : __ldg(gamma + j0 + q * tpr);
+    if (!rebuild) {
+      const uint4* src = static_cast<const uint4*>(p.tensor_source == 2 ? p.norm_out : p.residual_out) + pk;
+      reinterpret_cast<uint2*>(p.quant_out)[pk] = stored_codes<DT>(
+          p.tensor_source, COHERENT ? ld_coherent_l2_hint(src, drop) : ld_once_l2_hint(src, drop), g,
+          p.weight_bias, rinv, rs, scale, inv, exact);
+      continue;
+    }
+    float y[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    for (int r = 0; r < p.W; ++r) add_pack<DT>(ld_once(static_cast<const uint4*>(p.partials[r]) + pk), y);
+    if (p.residual != nullptr)
+      add_pack<DT>(ld_once_coherent(static_cast<const uint4*>(p.residual) + pk), y);
+    if (p.residual_out != nullptr) static_cast<uint4*>(p.residual_out)[pk] = pack8<DT>(y);
     reinterpret_cast<uint2*>(p.quant_out)[pk] =
         tensor_codes<DT>(g, p.weight_bias, y, rinv, rs, scale, inv, exact);
   }
@@ -992,9 +1047,9 @@ far_ring_kernel(const Params p, int nslot, int ncons, int stage_gamma) {
       // per-tensor FP8 reading back its new residual: the inputs, read
       // once, leave L2 first, so that the new residual (stored evict-last)
       // is what L2 keeps for the second pass
-      const bool drop_inputs = MODE == kModeTensor && p.tensor_stores_residual;
+      const bool drop_inputs = is_tensor_mode(MODE) && p.tensor_source != 0;
       uint64_t drop = 0;
-      if constexpr (MODE == kModeTensor) drop = l2_evict_first();
+      if constexpr (is_tensor_mode(MODE)) drop = l2_evict_first();
       // Rows: ordinals blockIdx.x + i * gridDim.x; or, in the fused
       // per-tensor form, taken one at a time from the call's counter (the
       // next one claimed while this one's segments are issued), so that the
@@ -1002,7 +1057,7 @@ far_ring_kernel(const Params p, int nslot, int ncons, int stage_gamma) {
       // first segment names the row, and a slot naming -1, completed
       // without a copy, ends the consumers' first pass.
       bool dyn = false;
-      if constexpr (MODE == kModeTensor) dyn = p.tensor_fused != 0;
+      if constexpr (is_tensor_mode(MODE)) dyn = p.tensor_fused != 0;
       int64_t ord = dyn ? static_cast<int64_t>(atomicAdd(p.ws_claim, 1u)) : blockIdx.x;
       int64_t g = 0;  // copies issued
       for (int64_t i = 0; !*abort_flag; ++i) {
@@ -1045,7 +1100,7 @@ far_ring_kernel(const Params p, int nslot, int ncons, int stage_gamma) {
         ord = dyn ? next : ord + gridDim.x;
       }
     }
-    if constexpr (MODE == kModeTensor) {
+    if constexpr (is_tensor_mode(MODE)) {
       // The fused per-tensor form: once every CTA has stored its rows' new
       // residuals and flags (fenced for the async proxy) and the consumers
       // are past the grid barrier, stream rows blockIdx.x + i * gridDim.x
@@ -1076,7 +1131,8 @@ far_ring_kernel(const Params p, int nslot, int ncons, int stage_gamma) {
                   *abort_flag = 1;
                   break;
                 }
-                const void* base = !rebuild ? p.residual_out : (k < p.W ? p.partials[k] : p.residual);
+                const void* stored = MODE == kModeTensorNorm ? p.norm_out : p.residual_out;
+                const void* base = !rebuild ? stored : (k < p.W ? p.partials[k] : p.residual);
                 mbar_arrive_expect_tx(&full[slot], seg_bytes);
                 bulk_load_hint(ring + static_cast<size_t>(slot) * seg_bytes,
                                static_cast<const unsigned char*>(base) + row * static_cast<int64_t>(seg_bytes),
@@ -1115,7 +1171,7 @@ far_ring_kernel(const Params p, int nslot, int ncons, int stage_gamma) {
   int slot = 0;  // the slot of the next segment and its use count parity
   uint32_t phase = 0;
   bool dyn = false;  // rows named by the producer (the fused per-tensor form)
-  if constexpr (MODE == kModeTensor) dyn = p.tensor_fused != 0;
+  if constexpr (is_tensor_mode(MODE)) dyn = p.tensor_fused != 0;
   int64_t i = 0;  // rows done
   for (;; ++i) {
     int64_t ord;
@@ -1170,7 +1226,7 @@ far_ring_kernel(const Params p, int nslot, int ncons, int stage_gamma) {
     finish_row<DT, VPT, MODE, false>(p, row, true, j0, ncons, ok, y, (i & 1) ? red1 : red0,
                                       gamma_s, no_gamma);
   }
-  if constexpr (MODE == kModeTensor) {
+  if constexpr (is_tensor_mode(MODE)) {
     if (p.tensor_fused) {
       // this thread's new-residual stores, before any CTA's bulk copies read them
       asm volatile("fence.proxy.async.global;" ::: "memory");
@@ -1220,14 +1276,31 @@ far_ring_kernel(const Params p, int nslot, int ncons, int stage_gamma) {
           }
           const int64_t rbase = row * static_cast<int64_t>(p.packs);
           const float rinv = fabsf(w);
+          if constexpr (MODE == kModeTensorNorm) {
+            // the slot held norm_out round(o), or the row was rebuilt (y):
+            // o itself is coded through gamma 1, weight_bias 0, rinv 1
+            const float wb_ = rebuild ? p.weight_bias : 0.f;
+            const float rinv_ = rebuild ? rinv : 1.f;
 #pragma unroll
-          for (int q = 0; q < VPT; ++q) {
-            if (!ok[q]) continue;
-            const int64_t pk = rbase + j0 + q * ncons;
-            if (rebuild) static_cast<uint4*>(p.residual_out)[pk] = pack8<DT>(y[q]);
-            reinterpret_cast<uint2*>(p.quant_out)[pk] =
-                tensor_codes<DT>(gamma_pack(p, gamma_s, j0 + q * ncons), p.weight_bias, y[q], rinv,
-                                 rinv * ts.inv, ts.scale, ts.inv, ts.exact);
+            for (int q = 0; q < VPT; ++q) {
+              if (!ok[q]) continue;
+              const int64_t pk = rbase + j0 + q * ncons;
+              if (rebuild && p.residual_out != nullptr) static_cast<uint4*>(p.residual_out)[pk] = pack8<DT>(y[q]);
+              const uint4 gm = rebuild ? gamma_pack(p, gamma_s, j0 + q * ncons) : ones_pack<DT>();
+              reinterpret_cast<uint2*>(p.quant_out)[pk] =
+                  tensor_codes<DT>(gm, wb_, y[q], rinv_, rinv_ * ts.inv, ts.scale, ts.inv, ts.exact);
+            }
+          } else {
+            // the slot held the new residual round(y), or the row was rebuilt: y
+#pragma unroll
+            for (int q = 0; q < VPT; ++q) {
+              if (!ok[q]) continue;
+              const int64_t pk = rbase + j0 + q * ncons;
+              if (rebuild) static_cast<uint4*>(p.residual_out)[pk] = pack8<DT>(y[q]);
+              reinterpret_cast<uint2*>(p.quant_out)[pk] =
+                  tensor_codes<DT>(gamma_pack(p, gamma_s, j0 + q * ncons), p.weight_bias, y[q], rinv,
+                                   rinv * ts.inv, ts.scale, ts.inv, ts.exact);
+            }
           }
         }
       }
@@ -1296,33 +1369,30 @@ far_tensor_quant_kernel(const Params p) {
       continue;
     }
     const int64_t ba = ra * static_cast<int64_t>(p.packs), bb = rb * static_cast<int64_t>(p.packs);
+    const uint4* src = static_cast<const uint4*>(p.tensor_source == 2 ? p.norm_out : p.residual_out);
     uint4 va[VPT], vb[VPT], gv[VPT];
 #pragma unroll
     for (int q = 0; q < VPT; ++q) {
       va[q] = vb[q] = gv[q] = make_uint4(0u, 0u, 0u, 0u);
       if (ok[q]) {
-        va[q] = ld_once_l2_hint(static_cast<const uint4*>(p.residual_out) + ba + j0 + q * tpr, drop);
-        if (two) vb[q] = ld_once_l2_hint(static_cast<const uint4*>(p.residual_out) + bb + j0 + q * tpr, drop);
-        gv[q] = __ldg(gamma + j0 + q * tpr);
+        va[q] = ld_once_l2_hint(src + ba + j0 + q * tpr, drop);
+        if (two) vb[q] = ld_once_l2_hint(src + bb + j0 + q * tpr, drop);
+        if (p.tensor_source == 1) gv[q] = __ldg(gamma + j0 + q * tpr);
       }
     }
     const float rinv_a = fabsf(wa), rinv_b = fabsf(wb);
 #pragma unroll
     for (int q = 0; q < VPT; ++q) {
       if (!ok[q]) continue;
-      float y[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-      add_pack<DT>(va[q], y);  // 0 + x: the 2-byte value widened exactly
-      reinterpret_cast<uint2*>(p.quant_out)[ba + j0 + q * tpr] =
-          tensor_codes<DT>(gv[q], p.weight_bias, y, rinv_a, rinv_a * inv, scale, inv, exact);
+      reinterpret_cast<uint2*>(p.quant_out)[ba + j0 + q * tpr] = stored_codes<DT>(
+          p.tensor_source, va[q], gv[q], p.weight_bias, rinv_a, rinv_a * inv, scale, inv, exact);
     }
     if (two) {
 #pragma unroll
       for (int q = 0; q < VPT; ++q) {
         if (!ok[q]) continue;
-        float y[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-        add_pack<DT>(vb[q], y);
-        reinterpret_cast<uint2*>(p.quant_out)[bb + j0 + q * tpr] =
-            tensor_codes<DT>(gv[q], p.weight_bias, y, rinv_b, rinv_b * inv, scale, inv, exact);
+        reinterpret_cast<uint2*>(p.quant_out)[bb + j0 + q * tpr] = stored_codes<DT>(
+            p.tensor_source, vb[q], gv[q], p.weight_bias, rinv_b, rinv_b * inv, scale, inv, exact);
       }
     }
   }
@@ -1413,7 +1483,9 @@ template <class DT>
 cudaError_t launch_ring_dt(const Params& p, const Launch& l, cudaStream_t s) {
   switch (mode_of(p.pattern)) {
     case kModeGroup: return launch_ring_g<DT, kModeGroup>(p, l, s);
-    case kModeTensor: return launch_ring_g<DT, kModeTensor>(p, l, s);
+    case kModeTensor:
+      return p.tensor_source == 2 ? launch_ring_g<DT, kModeTensorNorm>(p, l, s)
+                                  : launch_ring_g<DT, kModeTensor>(p, l, s);
     default: return launch_ring_g<DT, kModePlain>(p, l, s);
   }
 }
@@ -1434,7 +1506,9 @@ template <class DT>
 cudaError_t launch_prefill_dt(const Params& p, const Launch& l, cudaStream_t s) {
   switch (mode_of(p.pattern)) {
     case kModeGroup: return launch_prefill_g<DT, kModeGroup>(p, l, s);
-    case kModeTensor: return launch_prefill_g<DT, kModeTensor>(p, l, s);
+    case kModeTensor:
+      return p.tensor_source == 2 ? launch_prefill_g<DT, kModeTensorNorm>(p, l, s)
+                                  : launch_prefill_g<DT, kModeTensor>(p, l, s);
     default: return launch_prefill_g<DT, kModePlain>(p, l, s);
   }
 }
@@ -1511,6 +1585,17 @@ cudaError_t allow_large_smem() {
   set(far_ring_kernel<DT, 2, 2, kModeTensor, kRingWide2Consumers>);
   set(far_ring_kernel<DT, 4, 1, kModePlain, kRingWide1Consumers>);
   set(far_ring_kernel<DT, 4, 1, kModeTensor, kRingWide1Consumers>);
+  set(far_ring_kernel<DT, 1, 2, kModeTensorNorm>);
+  set(far_ring_kernel<DT, 2, 2, kModeTensorNorm>);
+  set(far_ring_kernel<DT, 4, 2, kModeTensorNorm>);
+  set(far_ring_kernel<DT, 1, 3, kModeTensorNorm>);
+  set(far_ring_kernel<DT, 2, 3, kModeTensorNorm>);
+  set(far_ring_kernel<DT, 4, 3, kModeTensorNorm>);
+  set(far_ring_kernel<DT, 8, 1, kModeTensorNorm>);
+  set(far_ring_kernel<DT, 8, 2, kModeTensorNorm>);
+  set(far_ring_kernel<DT, 4, 2, kModeTensorNorm, kRingWideConsumers>);
+  set(far_ring_kernel<DT, 2, 2, kModeTensorNorm, kRingWide2Consumers>);
+  set(far_ring_kernel<DT, 4, 1, kModeTensorNorm, kRingWide1Consumers>);
   set(far_ring_kernel<DT, 4, 2, kModeGroup, kRingWideConsumers>);
   set(far_ring_kernel<DT, 4, 1, kModeGroup, kRingWide1Consumers>);
   return e;

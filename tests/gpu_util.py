@@ -200,10 +200,10 @@ def compare(gpu: dict, ref: dict, dtype: str, rows=None, exact_saturation: bool 
     ``stats[key][2]`` counts the elements that took this path.
 
     ``exact_saturation``: where the oracle's code is +-448 the GPU's must be
-    too.  Per-tensor FP8 whose codes come from the stored new residual passes
-    False: its quotient never exceeds 448 (the scale is amax / 448), so no
-    code is clamped, and a code that rounds up to 448 follows the one-step
-    rule like every other code."""
+    too.  Per-tensor FP8 whose codes come from the stored new residual or
+    norm_out passes False: its quotient never exceeds 448 (the scale is
+    amax / 448), so no code is clamped, and a code that rounds up to 448
+    follows the one-step rule like every other code."""
     sel = slice(None) if rows is None else rows
     stats = {}
 
