@@ -412,9 +412,11 @@ far_status far_set_regime(far_ctx *ctx, far_regime regime, int decode_max_rows);
  * hook off.  Outputs of a stalled call are not valid. */
 far_status far_test_stall(far_ctx *ctx, int64_t segment, uint32_t wait_limit_us);
 
-/* Fill `info` with the launch geometry a call on `rows` rows of W partials
- * (and a residual when has_residual != 0, writing norm_out when
- * has_norm_out != 0) would use. */
+/* Fill `info` with the launch geometry a far_fused / far_fused_rows call on
+ * `rows` rows of W partials (and a residual when has_residual != 0, writing
+ * norm_out when has_norm_out != 0) would use.  far_fused_fp8_tensor and
+ * far_fused_fp8_group plan the ring kernel's CTAs per SM and slots by rules
+ * of their own, so their geometry can differ from this. */
 far_status far_describe_launch(const far_ctx *ctx, int64_t rows, int64_t H,
                                far_dtype dtype, int W, int has_residual, int has_norm_out,
                                far_launch_info *info);

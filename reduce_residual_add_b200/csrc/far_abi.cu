@@ -226,6 +226,10 @@ int ring_occ_cached(const far_ctx* ctx, int dtype, int vpt, int minb, int thread
 // and 512-consumer builds (the one-CTA build with norm_out too), whose
 // registers do not spill as 8 packs per thread do (H = 10240-16384:
 // 65-97 vs 49-81 %).
+// Dynamic per-tensor FP8 (both passes in one launch, the second reading
+// rows back from L2) wants more CTAs per SM below H = 4096 and fewer slots:
+// its own rule from H = 2048 to 4096 and at H = 8192, the static rule
+// elsewhere.
 // Gamma is staged in shared memory unless said otherwise; where the slots
 // asked for do not fit, as many as fit; below 2 (below 3 for the byte
 // targets), the rule falls back to 2 CTAs per SM with gamma through L1.
@@ -236,7 +240,7 @@ int ring_occ_cached(const far_ctx* ctx, int dtype, int vpt, int minb, int thread
 // confirms), fewer for fewer rows.  Returns false (the direct kernel runs)
 // when fewer than two slots fit or the configuration cannot be resident.
 bool plan_ring(const far_ctx* ctx, int packs, int64_t rows, int dtype, int segs, bool norm,
-               bool group, far::Launch* l) {
+               bool group, bool tensor, far::Launch* l) {
   if (packs <= 32) return false;
   const int seg = packs * 16;
   const bool small_rows = packs <= 256;  // H <= 2048
@@ -315,6 +319,23 @@ bool plan_ring(const far_ctx* ctx, int packs, int64_t rows, int dtype, int segs,
       n_req = 3;
       want = 3;
     }
+  } else if (tensor && packs > 256 && packs <= 384 && norm) {
+    // dynamic per-tensor FP8 (two passes in one launch) has a rule of its
+    // own, from sweeps of CTAs per SM x slots at H = 2048-8192, W = 2-8:
+    // H = 2056-3072 with norm_out 4 x 6 (W=2/3/4/8: 75-86 vs 65-79 %)
+    n_req = 4;
+    want = 6;
+  } else if (tensor && (packs <= 256 || (packs <= 512 && segs <= 6))) {
+    // ... H <= 2048 6 x 4, with norm_out too (W=2/3/4/8 with norm_out:
+    // 72-85 vs 62-80 %); H <= 4096 with at most 6 segments 5 x 4 (W=2/3/4
+    // at H=4096: 75-83 vs 65-78 %)
+    n_req = packs <= 256 ? 6 : 5;
+    want = 4;
+  } else if (tensor && packs > 896 && packs <= 1024) {
+    // ... H=8192: 3 x 3 for every W, with norm_out too (W=2/3/4: 78-85 vs
+    // 71-82 %)
+    n_req = 3;
+    want = 3;
   } else if (packs <= 256) {
     n_req = norm ? 4 : 6;
     want = norm ? 6 : 4;
@@ -401,7 +422,7 @@ int ring_occ_cached(const far_ctx* ctx, int dtype, int vpt, int minb, int thread
 // segs = row segments read per row: W partials, plus the residual if any;
 // norm: the call writes norm_out.
 far::Launch plan(const far_ctx* ctx, int64_t rows, int64_t H, int dtype, int segs, bool norm,
-                 bool group = false) {
+                 bool group = false, bool tensor = false) {
   const int packs = static_cast<int>(H / far::kPackElems);
   far::Launch l{};
   bool decode;
@@ -455,7 +476,7 @@ far::Launch plan(const far_ctx* ctx, int64_t rows, int64_t H, int dtype, int seg
       const int per_cta = (4096 / packs > 8) ? 4096 / packs : 8;
       min_rows = static_cast<int64_t>(per_cta) * ctx->sm_count * 2;
     }
-    if (ctx->prefill_kernel == 1 && rows >= min_rows) plan_ring(ctx, packs, rows, dtype, segs, norm, group, &l);
+    if (ctx->prefill_kernel == 1 && rows >= min_rows) plan_ring(ctx, packs, rows, dtype, segs, norm, group, tensor, &l);
   }
   l.pdl = ctx->pdl;
   return l;
@@ -800,7 +821,7 @@ far_status far_fused_fp8_tensor_launch(far_ctx* ctx, int64_t row_begin, int64_t 
   const cudaStream_t s = static_cast<cudaStream_t>(stream);
   // per-tensor: never the cluster kernel (no reduction in the second pass)
   far::Launch whole = plan(ctx, row_end - row_begin, H, dtype, W + (residual != nullptr ? 1 : 0),
-                   norm_out != nullptr);
+                   norm_out != nullptr, false, true);
   if (whole.regime == FAR_REGIME_DECODE) {
     plan_prefill(static_cast<int>(H / far::kPackElems), ctx->prefill_threads, &whole);
     whole.grid = (row_end - row_begin + whole.rows_per_cta - 1) / whole.rows_per_cta;
