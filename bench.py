@@ -605,7 +605,7 @@ def run_far(args, world, rank, local):
     ctx = far.FarContext(local)
     case = Case(ctx, wl, inp, device, args.with_norm, stream)
     launch = far.far_describe_launch(ctx, wl.T, wl.H, wl.torch_dtype, wl.W, wl.has_residual,
-                                     case.nout is not None)
+                                     case.nout is not None, pattern=wl.pattern)
 
     case.time_steps(0, args.warmup, per_launch=False)
     barrier(world)

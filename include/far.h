@@ -46,8 +46,9 @@
  *
  * Ownership: the caller owns every buffer.  The library allocates and frees
  * nothing per call and never synchronises the stream; a call only enqueues
- * one kernel on `stream` (two for per-tensor FP8; copies and one kernel per
- * chunk for far_fused_host) and returns.  Results are ready when the stream
+ * one kernel on `stream` (for per-tensor FP8 a one-CTA kernel that zeroes
+ * the workspace's counters, then one or two passes; copies and one kernel
+ * per chunk for far_fused_host) and returns.  Results are ready when the stream
  * reaches that point.  The W partials live in the same GPU's memory (the
  * tensor-parallel ranks' outputs gathered on one device); they are read only.
  *
@@ -124,8 +125,9 @@ typedef enum {
  * FAR_RING_MIN_ROWS: fewest rows for the ring kernel, default by rule,
  * FAR_TENSOR_REVERSE=1|0: the second pass of per-tensor FP8 takes the rows
  * from the last one down, default 1, FAR_TENSOR_FUSED=1|0: per-tensor FP8
- * without norm_out on the ring kernel runs both passes in one launch with
- * a bounded grid-wide wait between them, default 1). */
+ * on the ring kernel with a residual_out or norm_out to read back runs both
+ * passes in one launch with a bounded wait on rows done between them,
+ * default 1). */
 /*
  * Programmatic dependent launch: every kernel of this library first waits
  * (griddepcontrol.wait) until the grid it depends on has completed, then
@@ -414,12 +416,23 @@ far_status far_test_stall(far_ctx *ctx, int64_t segment, uint32_t wait_limit_us)
 
 /* Fill `info` with the launch geometry a far_fused / far_fused_rows call on
  * `rows` rows of W partials (and a residual when has_residual != 0, writing
- * norm_out when has_norm_out != 0) would use.  far_fused_fp8_tensor and
- * far_fused_fp8_group plan the ring kernel's CTAs per SM and slots by rules
- * of their own, so their geometry can differ from this. */
+ * norm_out when has_norm_out != 0) would use: far_describe_launch_pattern
+ * with FAR_AR_RESIDUAL_RMSNORM (patterns 0-2 share one plan). */
 far_status far_describe_launch(const far_ctx *ctx, int64_t rows, int64_t H,
                                far_dtype dtype, int W, int has_residual, int has_norm_out,
                                far_launch_info *info);
+
+/* The same for a call of `pattern`.  FAR_AR_RESIDUAL_RMSNORM_FP8_GROUP: the
+ * one launch of far_fused_fp8_group (any group size); _FP8_TENSOR: the
+ * first launch of far_fused_fp8_tensor, which on the ring kernel with a
+ * residual_out or norm_out to read back (kernel 1) also runs the second
+ * pass.  Both plan the ring kernel's CTAs per SM and slots by rules of
+ * their own and never take the cluster kernel (regime 1 falls back to the
+ * one-CTA kernel).  A pattern outside 0-4 gives FAR_ERR_INVALID_ARG. */
+far_status far_describe_launch_pattern(const far_ctx *ctx, int64_t rows, int64_t H,
+                                       far_dtype dtype, int W, int has_residual,
+                                       int has_norm_out, far_pattern pattern,
+                                       far_launch_info *info);
 
 /* Wait for `stream`, then read and clear the device-side error word of
  * ctx's device.  FAR_ERR_TIMEOUT: a bounded wait inside a kernel launched

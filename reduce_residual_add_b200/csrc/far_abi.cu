@@ -482,6 +482,24 @@ far::Launch plan(const far_ctx* ctx, int64_t rows, int64_t H, int dtype, int seg
   return l;
 }
 
+// The geometry a call of `pattern` runs with.  Per-group and per-tensor FP8
+// plan the ring kernel by rules of their own and never take the cluster
+// kernel: a group must sit on consecutive lanes of one warp, which a
+// cluster CTA's slice need not start on, and the per-tensor second pass
+// has no reduction for a cluster to share.
+far::Launch plan_call(const far_ctx* ctx, int64_t rows, int64_t H, int dtype, int segs, bool norm,
+                      int pattern) {
+  const bool group = pattern == FAR_AR_RESIDUAL_RMSNORM_FP8_GROUP;
+  const bool tensor = pattern == FAR_AR_RESIDUAL_RMSNORM_FP8_TENSOR;
+  far::Launch l = plan(ctx, rows, H, dtype, segs, norm, group, tensor);
+  if ((group || tensor) && l.regime == FAR_REGIME_DECODE) {
+    plan_prefill(static_cast<int>(H / far::kPackElems), ctx->prefill_threads, &l);
+    l.grid = (rows + l.rows_per_cta - 1) / l.rows_per_cta;
+    l.pdl = ctx->pdl;
+  }
+  return l;
+}
+
 }  // namespace
 
 extern "C" {
@@ -597,7 +615,16 @@ far_status far_set_regime(far_ctx* ctx, far_regime regime, int decode_max_rows) 
 
 far_status far_describe_launch(const far_ctx* ctx, int64_t rows, int64_t H, far_dtype dtype,
                                int W, int has_residual, int has_norm_out, far_launch_info* info) {
+  return far_describe_launch_pattern(ctx, rows, H, dtype, W, has_residual, has_norm_out,
+                                     FAR_AR_RESIDUAL_RMSNORM, info);
+}
+
+far_status far_describe_launch_pattern(const far_ctx* ctx, int64_t rows, int64_t H,
+                                       far_dtype dtype, int W, int has_residual, int has_norm_out,
+                                       far_pattern pattern, far_launch_info* info) {
   if (ctx == nullptr || info == nullptr || rows < 0) return FAR_ERR_INVALID_ARG;
+  if (pattern < FAR_AR_RESIDUAL_RMSNORM || pattern > FAR_AR_RESIDUAL_RMSNORM_FP8_GROUP)
+    return FAR_ERR_INVALID_ARG;
   if (W < 1 || W > FAR_MAX_W) return FAR_ERR_INVALID_ARG;
   if (dtype != FAR_BF16 && dtype != FAR_FP16) return FAR_ERR_INVALID_ARG;
   if (H <= 0 || H % far::kPackElems != 0 || H > far::kMaxH) return FAR_ERR_UNSUPPORTED;
@@ -606,7 +633,8 @@ far_status far_describe_launch(const far_ctx* ctx, int64_t rows, int64_t H, far_
   if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
   if (prev != ctx->device && (e = cudaSetDevice(ctx->device)) != cudaSuccess)
     return cuda_fail(e, "cudaSetDevice");
-  const far::Launch l = plan(ctx, rows, H, dtype, W + (has_residual ? 1 : 0), has_norm_out != 0);
+  const far::Launch l =
+      plan_call(ctx, rows, H, dtype, W + (has_residual ? 1 : 0), has_norm_out != 0, pattern);
   if (prev != ctx->device) cudaSetDevice(prev);
   info->regime = l.regime;
   info->ctas_per_row = l.cluster;
@@ -819,14 +847,9 @@ far_status far_fused_fp8_tensor_launch(far_ctx* ctx, int64_t row_begin, int64_t 
   DeviceGuard guard(ctx->device);
   if (guard.err != cudaSuccess) return cuda_fail(guard.err, "cudaSetDevice");
   const cudaStream_t s = static_cast<cudaStream_t>(stream);
-  // per-tensor: never the cluster kernel (no reduction in the second pass)
-  far::Launch whole = plan(ctx, row_end - row_begin, H, dtype, W + (residual != nullptr ? 1 : 0),
-                   norm_out != nullptr, false, true);
-  if (whole.regime == FAR_REGIME_DECODE) {
-    plan_prefill(static_cast<int>(H / far::kPackElems), ctx->prefill_threads, &whole);
-    whole.grid = (row_end - row_begin + whole.rows_per_cta - 1) / whole.rows_per_cta;
-    whole.pdl = ctx->pdl;
-  }
+  const far::Launch whole = plan_call(ctx, row_end - row_begin, H, dtype,
+                                      W + (residual != nullptr ? 1 : 0), norm_out != nullptr,
+                                      FAR_AR_RESIDUAL_RMSNORM_FP8_TENSOR);
   // the amax word, the count of rows done and the row counter start at
   // zero: a one-CTA kernel after the preceding work, so that the first pass
   // can still be launched with PDL (its set-up overlapping this kernel)
@@ -1126,15 +1149,9 @@ far_status far_fused_fp8_group(far_ctx* ctx, int64_t row_begin, int64_t row_end,
   p.groups_per_row = static_cast<int>(H / group_size);
   DeviceGuard guard(ctx->device);
   if (guard.err != cudaSuccess) return cuda_fail(guard.err, "cudaSetDevice");
-  // a group must sit on consecutive lanes of one warp: not the cluster kernel,
-  // whose per-CTA slices need not start on a group boundary
-  far::Launch whole = plan(ctx, row_end - row_begin, H, dtype, W + (residual != nullptr ? 1 : 0),
-                   norm_out != nullptr, true);
-  if (whole.regime == FAR_REGIME_DECODE) {
-    plan_prefill(static_cast<int>(H / far::kPackElems), ctx->prefill_threads, &whole);
-    whole.grid = (row_end - row_begin + whole.rows_per_cta - 1) / whole.rows_per_cta;
-    whole.pdl = ctx->pdl;
-  }
+  const far::Launch whole = plan_call(ctx, row_end - row_begin, H, dtype,
+                                      W + (residual != nullptr ? 1 : 0), norm_out != nullptr,
+                                      FAR_AR_RESIDUAL_RMSNORM_FP8_GROUP);
   const cudaError_t e = launch_rows(p, dtype, whole, row_begin, row_end, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "kernel launch");
   return FAR_OK;
@@ -1262,15 +1279,11 @@ far_status far_fused_host(far_ctx* ctx, const void* const* partials, int W, cons
                                 nsc > 0 ? d_scale : nullptr);
     p.wait_limit_ns = ctx->wait_limit_ns;
     p.stall_segment = ctx->stall_segment;
-    far::Launch l = plan(ctx, n, H, dtype, W + (residual != nullptr ? 1 : 0),
-                          norm_out != nullptr, group);
+    far::Launch l = plan_call(ctx, n, H, dtype, W + (residual != nullptr ? 1 : 0),
+                              norm_out != nullptr, pattern);
     if (group) {
       p.group_lanes = group_size / far::kPackElems;
       p.groups_per_row = static_cast<int>(H / group_size);
-      if (l.regime == FAR_REGIME_DECODE) {  // groups need the one-CTA kernels
-        plan_prefill(static_cast<int>(H / far::kPackElems), ctx->prefill_threads, &l);
-        l.grid = (n + l.rows_per_cta - 1) / l.rows_per_cta;
-      }
     }
     l.pdl = 0;
     FAR_HOST_CK(launch_rows(p, dtype, l, 0, n, s), "kernel launch");

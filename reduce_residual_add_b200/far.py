@@ -50,9 +50,9 @@ EXPORTS = ("far_create", "far_destroy", "far_fused", "far_fused_rows",
            "far_fp8_tensor_workspace_bytes", "far_fused_fp8_tensor",
            "far_fused_fp8_tensor_noalloc", "far_fused_fp8_group",
            "far_host_staging_bytes", "far_fused_host", "far_validate",
-           "far_set_regime", "far_describe_launch", "far_check", "far_test_stall",
-           "far_status_string",
-           "far_last_error", "far_version")
+           "far_set_regime", "far_describe_launch", "far_describe_launch_pattern",
+           "far_check", "far_test_stall", "far_status_string", "far_last_error",
+           "far_version")
 
 _DTYPES = {torch.bfloat16: FAR_BF16, torch.float16: FAR_FP16}
 
@@ -128,6 +128,9 @@ def lib() -> ctypes.CDLL:
     L.far_describe_launch.argtypes = [vp, i64, i64, i32, i32, i32, i32,
                                       ctypes.POINTER(far_launch_info)]
     L.far_describe_launch.restype = i32
+    L.far_describe_launch_pattern.argtypes = [vp, i64, i64, i32, i32, i32, i32, i32,
+                                              ctypes.POINTER(far_launch_info)]
+    L.far_describe_launch_pattern.restype = i32
     L.far_test_stall.argtypes = [vp, i64, ctypes.c_uint32]
     L.far_test_stall.restype = i32
     L.far_check.argtypes = [vp, vp]
@@ -203,11 +206,20 @@ def far_set_regime(ctx: FarContext, regime: int, decode_max_rows: int = -1) -> N
 
 
 def far_describe_launch(ctx: FarContext, rows: int, H: int, dtype=torch.bfloat16, W: int = 8,
-                        has_residual: bool = True, has_norm_out: bool = False) -> dict:
+                        has_residual: bool = True, has_norm_out: bool = False,
+                        pattern: Optional[int] = None) -> dict:
+    """The launch geometry of a call; `pattern` None: far_fused / far_fused_rows
+    (far_describe_launch), else that pattern's own plan (far_describe_launch_pattern)."""
     info = far_launch_info()
-    st = lib().far_describe_launch(ctx.handle, int(rows), int(H), _DTYPES.get(dtype, dtype),
-                                   int(W), int(bool(has_residual)), int(bool(has_norm_out)),
-                                   ctypes.byref(info))
+    dt = _DTYPES.get(dtype, dtype)
+    if pattern is None:
+        st = lib().far_describe_launch(ctx.handle, int(rows), int(H), dt, int(W),
+                                       int(bool(has_residual)), int(bool(has_norm_out)),
+                                       ctypes.byref(info))
+    else:
+        st = lib().far_describe_launch_pattern(ctx.handle, int(rows), int(H), dt, int(W),
+                                               int(bool(has_residual)), int(bool(has_norm_out)),
+                                               int(pattern), ctypes.byref(info))
     if st != FAR_OK:
         raise FarError(st, "far_describe_launch")
     return {name: getattr(info, name) for name, _ in far_launch_info._fields_}

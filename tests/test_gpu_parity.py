@@ -481,6 +481,48 @@ def test_launch_plan(ctx):
     assert tiny["regime"] == far.FAR_REGIME_PREFILL and tiny["rows_per_cta"] > 1
 
 
+def test_launch_plan_tensor_and_group(ctx):
+    """Per-tensor and per-group FP8 plan the ring kernel by rules of their
+    own (see far_abi.cu plan_ring) and never take the cluster kernel."""
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+
+    def d(rows, H, W, pattern, norm=False):
+        return far.far_describe_launch(ctx, rows, H, torch.bfloat16, W, True, norm, pattern=pattern)
+
+    def geo(i):
+        return (i["kernel"], i["grid_ctas"], i["ring_slots"])
+
+    T3, G4 = far.FAR_AR_RESIDUAL_RMSNORM_FP8_TENSOR, far.FAR_AR_RESIDUAL_RMSNORM_FP8_GROUP
+    # patterns 0-2 share far_describe_launch's plan
+    for pat in (0, 1, 2):
+        assert d(8192, 8192, 4, pat) == far.far_describe_launch(ctx, 8192, 8192, torch.bfloat16, 4, True)
+    # per-tensor, H <= 2048: 6 CTAs per SM x 4 slots, with norm_out too
+    # (the static rule: 4 x 6 with norm_out)
+    assert geo(d(32768, 2048, 2, T3)) == (1, 6 * sms, 4)
+    assert geo(d(32768, 2048, 4, T3, norm=True)) == (1, 6 * sms, 4)
+    # ... H = 3072 with norm_out: 4 x 6 (static: 3 x 4)
+    h3 = d(32768, 3072, 4, T3, norm=True)
+    assert (geo(h3), h3["threads_per_cta"]) == ((1, 4 * sms, 6), 224)
+    assert geo(d(32768, 3072, 4, None, norm=True)) == (1, 3 * sms, 4)
+    # ... H = 4096, at most 6 segments: 5 x 4 (static: 4 x 3)
+    h4 = d(16384, 4096, 4, T3)
+    assert (geo(h4), h4["packs_per_thread"]) == ((1, 5 * sms, 4), 4)
+    # ... H = 8192: 3 x 3 for every W (static at W=2: 2 x 4)
+    assert geo(d(8192, 8192, 2, T3)) == (1, 3 * sms, 3)
+    assert geo(d(8192, 8192, 4, T3)) == (1, 3 * sms, 3)
+    assert geo(d(8192, 8192, 2, None)) == (1, 2 * sms, 4)
+    # per-group, up to 256 packs and 6 segments: 5 x 6
+    assert geo(d(32768, 2048, 2, G4)) == (1, 5 * sms, 6)
+    # decode-sized calls of both stay on one CTA per row
+    assert d(4, 16384, 8, None)["regime"] == far.FAR_REGIME_DECODE
+    for pat in (T3, G4):
+        i = d(4, 16384, 8, pat)
+        assert (i["regime"], i["ctas_per_row"], i["grid_ctas"]) == (far.FAR_REGIME_PREFILL, 1, 4)
+    with pytest.raises(far.FarError) as e:
+        d(8192, 8192, 4, 5)
+    assert e.value.status == far.FAR_ERR_INVALID_ARG
+
+
 @pytest.mark.parametrize("kern", ["decode", "ring", "direct"])
 def test_chained_calls_read_completed_outputs(kctx, ctx, kern):
     """With programmatic dependent launch each call must still read what the
