@@ -837,6 +837,14 @@ far_status far_fused_fp8_tensor_launch(far_ctx* ctx, int64_t row_begin, int64_t 
   p.ws_amax = static_cast<unsigned*>(workspace);
   p.ws_done = p.ws_amax + 1;
   p.ws_claim = p.ws_amax + 2;
+  p.ws_claim2 = p.ws_amax + 3;
+  // second-pass rows per claim: about 1024 packs (16 KiB of each stored
+  // row) per claim, so that a claim's rows outlast the next claim's round
+  // trip, and the rows left over when the counter runs dry stay few
+  {
+    const int64_t packs = H / far::kPackElems;
+    p.tail_chunk = static_cast<int>(packs >= 1024 ? 1 : (1024 / packs > 8 ? 8 : 1024 / packs));
+  }
   p.ws_rinv = reinterpret_cast<float*>(static_cast<unsigned char*>(workspace) + 256);
   p.ws_row0 = row_begin;
   // what the second pass forms the codes from: norm_out when the call
@@ -850,7 +858,7 @@ far_status far_fused_fp8_tensor_launch(far_ctx* ctx, int64_t row_begin, int64_t 
   const far::Launch whole = plan_call(ctx, row_end - row_begin, H, dtype,
                                       W + (residual != nullptr ? 1 : 0), norm_out != nullptr,
                                       FAR_AR_RESIDUAL_RMSNORM_FP8_TENSOR);
-  // the amax word, the count of rows done and the row counter start at
+  // the amax word, the count of rows done and the two row counters start at
   // zero: a one-CTA kernel after the preceding work, so that the first pass
   // can still be launched with PDL (its set-up overlapping this kernel)
   cudaError_t e = far::launch_ws_zero(static_cast<unsigned*>(workspace), ctx->pdl, s);

@@ -49,6 +49,7 @@ struct RingHeader {
   float red[2][2][32];   // [row parity][0 = sum of squares, 1 = amax][warp]
   int slot_row[32];      // rows taken from a shared counter: the row (ordinal)
                          // whose first segment sits in the slot, -1: no more rows
+  float slot_w[32];      // per-tensor second pass: that row's stored rinv (flag)
   int abort;             // set when any wait of the CTA gave up
   int producer_done;     // set by the producer when it stops issuing
   long long issued;      // bulk copies the producer issued
@@ -1103,39 +1104,85 @@ far_ring_kernel(const Params p, int nslot, int ncons, int stage_gamma) {
     if constexpr (is_tensor_mode(MODE)) {
       // The fused per-tensor form: once every CTA has stored its rows' new
       // residuals and flags (fenced for the async proxy) and the consumers
-      // are past the grid barrier, stream rows blockIdx.x + i * gridDim.x
-      // back through the ring, the highest ordinals (taken last) first: the
-      // new residual of a row, or for a flagged row all its input segments.
+      // are past the grid barrier, stream the rows back through the ring:
+      // the stored row, or for a flagged row all its input segments.  Rows
+      // are taken in chunks of p.tail_chunk ordinals, the highest ordinals
+      // (taken last in the first pass, so the likeliest in L2) first: one
+      // chunk per CTA to start, then from a second counter, so that a CTA
+      // whose SM drains its ring faster takes more rows.
+      // The slot of a row's first segment names the row and holds its stored
+      // rinv (sign bit: the flag); a slot naming -1, completed without a
+      // copy, ends the second pass.  The next chunk is claimed while this
+      // one is issued, and its flags are read (one row per lane) once this
+      // one is issued, while the ring still holds nslot segments.
       if (p.tensor_fused) {
         tail_bar(ncons + 32);
-        // The whole warp reads the row flags, 32 rows per load (one row per
-        // lane), so that lane 0 does not wait on one load per row.
         const int lane = threadIdx.x - ncons;
         const uint64_t drop_tail = l2_evict_first();
-        for (int64_t i0 = my_rows - 1; i0 >= 0; i0 -= 32) {
-          if (__shfl_sync(0xffffffffu, lane == 0 ? *abort_flag : 0, 0)) break;
-          bool flagged = false;
-          if (i0 - lane >= 0) {
-            const int64_t r = call_row(p, blockIdx.x + (i0 - lane) * gridDim.x);
-            flagged = signbit(*reinterpret_cast<volatile const float*>(p.ws_rinv + (r - p.ws_row0)));
+        const int64_t C = p.tail_chunk;
+        // the first chunk is CTA b's own (chunk b), so that no CTA starts
+        // the pass by queueing on the counter; the counter deals out the rest
+        const int64_t first_dealt = static_cast<int64_t>(gridDim.x) * C;
+        const auto claim = [&]() -> int64_t {
+          unsigned b = 0;
+          if (lane == 0) b = atomicAdd(p.ws_claim2, static_cast<unsigned>(C));
+          return first_dealt + static_cast<int64_t>(__shfl_sync(0xffffffffu, b, 0));
+        };
+        const auto flags = [&](int64_t b) -> float {
+          float w = 0.f;
+          if (lane < C && b + lane < nrows) {
+            const int64_t r = call_row(p, nrows - 1 - (b + lane));
+            w = *reinterpret_cast<volatile const float*>(p.ws_rinv + (r - p.ws_row0));
           }
-          const unsigned rebuild_mask = __ballot_sync(0xffffffffu, flagged);
-          if (lane == 0) {
-            for (int j = 0; j < 32 && i0 - j >= 0 && !*abort_flag; ++j) {
-              const int64_t row = call_row(p, blockIdx.x + (i0 - j) * gridDim.x);
-              const bool rebuild = (rebuild_mask >> j) & 1u;
+          return w;
+        };
+        int64_t base = static_cast<int64_t>(blockIdx.x) * C;
+        float w = flags(base);
+        int64_t next = claim();
+        bool stop = false;
+        while (!stop) {
+          if (__shfl_sync(0xffffffffu, lane == 0 ? *abort_flag : 0, 0)) break;
+          if (base >= nrows) {
+            // the end marker
+            if (lane == 0) {
+              if (mbar_wait(&empty[slot], phase ^ 1u, abort_flag, p.wait_limit_ns)) {
+                hdr->slot_row[slot] = -1;
+                mbar_arrive(&full[slot]);
+                ++issued;
+                if (++slot == nslot) {
+                  slot = 0;
+                  phase ^= 1u;
+                }
+              } else {
+                if (!*abort_flag) atomicOr(&g_far_error, kErrWaitEmpty);
+                *abort_flag = 1;
+              }
+            }
+            break;
+          }
+          for (int j = 0; j < C; ++j) {
+            const float wj = __shfl_sync(0xffffffffu, w, j);
+            if (lane == 0 && !stop && base + j < nrows) {
+              const int64_t ord = nrows - 1 - (base + j);
+              const int64_t row = call_row(p, ord);
+              const bool rebuild = signbit(wj);
               const int nseg = rebuild ? S : 1;
               for (int k = 0; k < nseg; ++k) {
                 if (!mbar_wait(&empty[slot], phase ^ 1u, abort_flag, p.wait_limit_ns)) {
                   if (!*abort_flag) atomicOr(&g_far_error, kErrWaitEmpty);
                   *abort_flag = 1;
+                  stop = true;
                   break;
                 }
+                if (k == 0) {
+                  hdr->slot_row[slot] = static_cast<int>(ord);
+                  hdr->slot_w[slot] = wj;
+                }
                 const void* stored = MODE == kModeTensorNorm ? p.norm_out : p.residual_out;
-                const void* base = !rebuild ? stored : (k < p.W ? p.partials[k] : p.residual);
+                const void* src = !rebuild ? stored : (k < p.W ? p.partials[k] : p.residual);
                 mbar_arrive_expect_tx(&full[slot], seg_bytes);
                 bulk_load_hint(ring + static_cast<size_t>(slot) * seg_bytes,
-                               static_cast<const unsigned char*>(base) + row * static_cast<int64_t>(seg_bytes),
+                               static_cast<const unsigned char*>(src) + row * static_cast<int64_t>(seg_bytes),
                                seg_bytes, &full[slot], drop_tail);
                 ++issued;
                 if (++slot == nslot) {
@@ -1145,7 +1192,10 @@ far_ring_kernel(const Params p, int nslot, int ncons, int stage_gamma) {
               }
             }
           }
-          __syncwarp();
+          stop = __shfl_sync(0xffffffffu, stop ? 1 : 0, 0) != 0;
+          base = next;
+          w = flags(base);
+          next = claim();
         }
       }
     }
@@ -1236,18 +1286,25 @@ far_ring_kernel(const Params p, int nslot, int ncons, int stage_gamma) {
         unsigned amax_bits;
         asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(amax_bits) : "l"(p.ws_amax) : "memory");
         const TensorScale ts(p, amax_bits);
-        // each warp reads the stored rinv of 32 rows per load (lane l: the
-        // l-th row of the chunk) and hands them out by shuffle
-        const int lane = threadIdx.x & 31;
-        float w_lane = 0.f;
-        for (int64_t i = my_rows - 1; i >= 0; --i) {
-          const int j = static_cast<int>((my_rows - 1 - i) & 31);
-          if (j == 0 && i - lane >= 0) {
-            const int64_t r = call_row(p, blockIdx.x + (i - lane) * gridDim.x);
-            w_lane = *reinterpret_cast<volatile const float*>(p.ws_rinv + (r - p.ws_row0));
+        // rows as the producer names them, each with its stored rinv, until
+        // the end marker (or a wait that gave up: every warp leaves alike)
+        for (;;) {
+          if (!*abort_flag && !mbar_wait(&full[slot], phase, abort_flag, p.wait_limit_ns)) {
+            if (!*abort_flag) atomicOr(&g_far_error, kErrWaitFull);
+            *abort_flag = 1;
           }
-          const int64_t row = call_row(p, blockIdx.x + i * gridDim.x);
-          const float w = __shfl_sync(0xffffffffu, w_lane, j);
+          const int named = hdr->slot_row[slot];
+          const float w = hdr->slot_w[slot];
+          if (__any_sync(0xffffffffu, named < 0 || *abort_flag)) {
+            __syncwarp();
+            if ((threadIdx.x & 31) == 0) mbar_arrive(&empty[slot]);
+            if (++slot == nslot) {
+              slot = 0;
+              phase ^= 1u;
+            }
+            break;
+          }
+          const int64_t row = call_row(p, named);
           const bool rebuild = signbit(w);
           const int nseg = rebuild ? S : 1;
           float y[VPT][8];
@@ -1259,7 +1316,7 @@ far_ring_kernel(const Params p, int nslot, int ncons, int stage_gamma) {
             for (int e = 0; e < 8; ++e) y[q][e] = 0.f;
           }
           for (int k = 0; k < nseg; ++k) {
-            if (!*abort_flag && !mbar_wait(&full[slot], phase, abort_flag, p.wait_limit_ns)) {
+            if (k > 0 && !*abort_flag && !mbar_wait(&full[slot], phase, abort_flag, p.wait_limit_ns)) {
               if (!*abort_flag) atomicOr(&g_far_error, kErrWaitFull);
               *abort_flag = 1;
             }

@@ -861,7 +861,12 @@ def test_per_tensor_fused_bounded_waits(kctx):
     up too; the kernel ends, far_check reports FAR_ERR_TIMEOUT, and the next
     call on the context is correct."""
     c = kctx["ring_fused"]
-    T, H = 600, 4096
+    # more rows than the grid has CTAs (at most 8 per SM): the first pass
+    # deals rows from a counter, so some CTA takes two rows or more, and
+    # its copy 7 (in its second row: 5 segments per row) is skipped
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    T, H = 9 * sms, 4096
+    assert far.far_describe_launch(c, T, H, torch.bfloat16, 4, True, pattern=3)["grid_ctas"] < T
     inp = random_inputs(4, T, H, seed=72)
     g = to_gpu(inp)
     q = torch.empty(T, H, dtype=torch.uint8, device="cuda")
