@@ -258,8 +258,9 @@ size_t far_fp8_tensor_workspace_bytes(int64_t rows);
  * the call, both passes run in ONE launch: its CTAs take the first pass's
  * rows one at a time from a counter in the workspace, wait (bounded) until
  * every row is done -- a wait on rows, not on CTAs, so the grid need not be
- * co-resident -- then write the codes, taking those rows in small chunks
- * from a second counter, the rows done last first (FAR_TENSOR_FUSED=0 in the
+ * co-resident -- then write the codes, the rows done last first, about
+ * three quarters of them in fixed rounds and the rest in small chunks from
+ * a second counter (FAR_TENSOR_FUSED=0 in the
  * environment at far_create splits them into two kernels); otherwise two
  * kernels run.
  * With neither norm_out nor a new residual to write, the second pass reads

@@ -64,8 +64,8 @@ struct Params {
   int tensor_fused;             // per-tensor FP8 in one ring launch: the CTAs take rows
                                 // from a shared counter (ws_claim), wait until every
                                 // row is done (ws_done), then write the codes from the
-                                // stored new residual or norm_out, rows taken in
-                                // chunks from a second counter (ws_claim2)
+                                // stored new residual or norm_out, the last quarter
+                                // of rows in chunks from a second counter (ws_claim2)
   unsigned* ws_done;            // per-tensor FP8, one launch: rows past the first pass
   unsigned* ws_claim;           // per-tensor FP8, one launch: rows taken so far
   unsigned* ws_claim2;          // ... second-pass rows taken so far

@@ -1107,9 +1107,10 @@ far_ring_kernel(const Params p, int nslot, int ncons, int stage_gamma) {
       // are past the grid barrier, stream the rows back through the ring:
       // the stored row, or for a flagged row all its input segments.  Rows
       // are taken in chunks of p.tail_chunk ordinals, the highest ordinals
-      // (taken last in the first pass, so the likeliest in L2) first: one
-      // chunk per CTA to start, then from a second counter, so that a CTA
-      // whose SM drains its ring faster takes more rows.
+      // (taken last in the first pass, so the likeliest in L2) first: about
+      // three quarters in fixed rounds, the rest from a second counter, so
+      // that a CTA whose SM drains its ring faster takes more of the last
+      // rows.
       // The slot of a row's first segment names the row and holds its stored
       // rinv (sign bit: the flag); a slot naming -1, completed without a
       // copy, ends the second pass.  The next chunk is claimed while this
@@ -1120,10 +1121,16 @@ far_ring_kernel(const Params p, int nslot, int ncons, int stage_gamma) {
         const int lane = threadIdx.x - ncons;
         const uint64_t drop_tail = l2_evict_first();
         const int64_t C = p.tail_chunk;
-        // the first chunk is CTA b's own (chunk b), so that no CTA starts
-        // the pass by queueing on the counter; the counter deals out the rest
-        const int64_t first_dealt = static_cast<int64_t>(gridDim.x) * C;
+        // about three quarters of the rows are dealt out in fixed rounds
+        // (CTA b takes chunk b of each round): no claim round trip for
+        // them; the counter deals out the rest, which evens out the ends
+        const int64_t G = gridDim.x;
+        int64_t rounds = (3 * nrows / 4) / (G * C);
+        if (rounds < 1) rounds = 1;
+        const int64_t first_dealt = rounds * G * C;
+        int64_t dealt = 0;  // fixed rounds taken so far
         const auto claim = [&]() -> int64_t {
+          if (dealt < rounds) return (dealt++ * G + blockIdx.x) * C;
           unsigned b = 0;
           if (lane == 0) b = atomicAdd(p.ws_claim2, static_cast<unsigned>(C));
           return first_dealt + static_cast<int64_t>(__shfl_sync(0xffffffffu, b, 0));
@@ -1136,7 +1143,7 @@ far_ring_kernel(const Params p, int nslot, int ncons, int stage_gamma) {
           }
           return w;
         };
-        int64_t base = static_cast<int64_t>(blockIdx.x) * C;
+        int64_t base = claim();
         float w = flags(base);
         int64_t next = claim();
         bool stop = false;
