@@ -7,6 +7,7 @@ runs before it launches anything).
 """
 from __future__ import annotations
 
+import ctypes
 import os
 import re
 import subprocess
@@ -82,6 +83,17 @@ def test_create_without_a_gpu_fails_cleanly():
     with pytest.raises(far.FarError) as e:
         far.FarContext(0)
     assert e.value.status == far.FAR_ERR_CUDA
+
+
+def test_describe_launch_needs_a_context():
+    """Both describe calls refuse a NULL context or info before any CUDA call."""
+    info = far.far_launch_info()
+    L = far.lib()
+    assert L.far_describe_launch(None, 8, 4096, far.FAR_BF16, 4, 1, 0, ctypes.byref(info)) == \
+        far.FAR_ERR_INVALID_ARG
+    for pattern in range(5):
+        assert L.far_describe_launch_pattern(None, 8, 4096, far.FAR_BF16, 4, 1, 0, pattern,
+                                             ctypes.byref(info)) == far.FAR_ERR_INVALID_ARG
 
 
 # --------------------------------------------------------------------------
